@@ -1,0 +1,346 @@
+/*
+ * lattice_oracle.c -- plain fp64 CPU oracle of the Lattice compression-layer
+ * state recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path links, loads or calls
+ * this file; only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg use it. It shares no code, header or constant with the CUDA library.
+ *
+ * Source: "Lattice: Learning to Efficiently Compress the Memory" (Karami,
+ * Pascanu, Mirrokni; arXiv 2504.05646).
+ *   - §3.1.1, eq. (similarity_recurrence) and eq. (OSR): the online gradient
+ *     step of the dot-product objective writes, into slot i, the part of the
+ *     input orthogonal to that slot, P(s_i) x / ||s_i||, scaled by the writing
+ *     intensity c_i (h_t = -v_t for the similarity objective).
+ *   - §3.2, eq. (normalized_recurrence): each slot is projected back onto the
+ *     unit sphere after the write.
+ *   - §3.3, eq. (dacay_recurrence) and the "General Form": the forget gate mu
+ *     scales the previous state; the normaliser applies to mu*s + write.
+ *   - §3.4, Eq. 14 (recurrence_detailed): P(s) h = h - s (s.h)/||s||^2 costs one
+ *     dot product and one axpy per slot.
+ *   - §3.4.1 / Appendix B.1, Eq. 17 (recurrence_linear2) and eq. (beta_chunk):
+ *     within a chunk the projection uses the chunk-start state; the update
+ *     becomes the gated linear recurrence S_t = G_t (.) S_{t-1} - h_t k_t^T.
+ *   - Appendix D (Implementation): argument shapes and the read-out y = q S_t
+ *     with the updated state.
+ *
+ * Readings of points the paper leaves open (each is listed in the design notes):
+ *   - slots are rows of S ([m][d]), as in the Appendix D listing;
+ *   - the normaliser targets the unit sphere (§3.2), with no epsilon;
+ *   - the normaliser of the chunked form is 1/sqrt(mu^2 n^2 + |Delta|^2), the
+ *     Pythagorean norm of mu*s + Delta (the printed eta^2 coefficient reads as
+ *     a typo: only mu^2 makes chunk size 1 equal the exact recurrence);
+ *   - D_S uses "minus" (Pythagoras, §3.2), clipped at zero;
+ *   - a slot whose update has zero norm (mu = 0 and no orthogonal write) is
+ *     left unchanged and counted.
+ *
+ * Layouts (row-major):  x[B][T][H][d]  c,q[B][T][H][m]  mu,eta[B][T][H]
+ *                       S[B][H][m][d]  y[B][T][H][d].   eta == NULL means 1.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define IDX_TOK(b, t, h, T, H) ((((size_t)(b) * (T)) + (t)) * (H) + (h))
+
+/* ------------------------------------------------------------------------ */
+/* One slot, one token (exact recurrence).                                   */
+/* ------------------------------------------------------------------------ */
+
+/* Unnormalised write w = mu*s + eta*(c/||s||) * P(s) x  (§3.1.1 eq. OSR with
+ * h = -x, the forget gate of §3.3, the projection of §3.4 Eq. 14).
+ * Returns ||s||^2 via *n2_out. */
+void oracle_osr_write(int d, const double *s, const double *x, double c, double mu,
+                      double eta, double *w, double *n2_out)
+{
+    double n2 = 0.0, p = 0.0;
+    for (int k = 0; k < d; ++k) {
+        n2 += s[k] * s[k];
+        p += s[k] * x[k];
+    }
+    double n = sqrt(n2);
+    for (int k = 0; k < d; ++k) {
+        double x_perp = x[k] - (p / n2) * s[k]; /* P(s) x */
+        w[k] = mu * s[k] + eta * (c / n) * x_perp;
+    }
+    if (n2_out) *n2_out = n2;
+}
+
+/* One exact step of the whole state (all m slots) followed by the read-out.
+ * Updates S in place; writes y if non-NULL; counts zero-norm updates. */
+static void exact_token(int m, int d, double *S, const double *x, const double *c,
+                        const double *q, double mu, double eta, double *y, double *w,
+                        long long *degenerate)
+{
+    for (int i = 0; i < m; ++i) {
+        double *s = S + (size_t)i * d;
+        double n2;
+        oracle_osr_write(d, s, x, c[i], mu, eta, w, &n2);
+        double nw2 = 0.0;
+        for (int k = 0; k < d; ++k) nw2 += w[k] * w[k];
+        if (n2 == 0.0 || nw2 == 0.0) { /* undefined projection: keep the slot */
+            ++*degenerate;
+            continue;
+        }
+        double nw = sqrt(nw2);
+        for (int k = 0; k < d; ++k) s[k] = w[k] / nw; /* §3.2 unit sphere */
+    }
+    if (y) {
+        for (int k = 0; k < d; ++k) y[k] = 0.0;
+        for (int i = 0; i < m; ++i)
+            for (int k = 0; k < d; ++k) y[k] += q[i] * S[(size_t)i * d + k];
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Chunked recurrence, Eq. 17: per-token gates from the chunk-start state.   */
+/* ------------------------------------------------------------------------ */
+
+/* Gates of one token against the chunk-start state S0 (Eq. 17 and eq.
+ * beta_chunk, Appendix B.1):
+ *   h = -x;  hhat_i = (h.s0_i)/n_i^2;  khat_i = c_i/n_i;
+ *   dsq_i  = eta^2 * max(0, khat_i^2 |h|^2 - n_i^2 hhat_i^2 khat_i^2)
+ *   beta_i = 1/sqrt(mu^2 n_i^2 + dsq_i)
+ *   g_i    = beta_i (mu + eta hhat_i khat_i),   kt_i = -beta_i eta khat_i
+ * so that the token's update is s_i <- g_i s_i + kt_i h. */
+void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
+                              const double *x, const double *c, double mu, double eta,
+                              double *g, double *kt, double *dsq_out, long long *degenerate)
+{
+    double hh = 0.0;
+    for (int k = 0; k < d; ++k) hh += x[k] * x[k]; /* |h|^2, h = -x */
+    for (int i = 0; i < m; ++i) {
+        const double *s0 = S0 + (size_t)i * d;
+        double hdot = 0.0;
+        for (int k = 0; k < d; ++k) hdot += (-x[k]) * s0[k];
+        double hhat = hdot / n2[i];
+        double khat = c[i] / sqrt(n2[i]);
+        double t = khat * khat * hh - n2[i] * hhat * hhat * khat * khat;
+        double dsq = eta * eta * (t > 0.0 ? t : 0.0);
+        double den = mu * mu * n2[i] + dsq;
+        if (dsq_out) dsq_out[i] = dsq;
+        if (den == 0.0) { /* zero-norm update: keep the slot */
+            g[i] = 1.0;
+            kt[i] = 0.0;
+            if (degenerate) ++*degenerate;
+            continue;
+        }
+        double beta = 1.0 / sqrt(den);
+        g[i] = beta * (mu + eta * hhat * khat);
+        kt[i] = -beta * eta * khat;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Whole-sequence drivers, one (b,h) sequence at a time.                     */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int B, T, H, m, d, C, form; /* form: 0 exact, 1 chunked token-wise, 2 chunked matrix form */
+    const double *x, *c, *q, *mu, *eta, *S0;
+    double *S_out, *y;
+    long long degenerate;
+    int next;
+    pthread_mutex_t lock;
+} job_t;
+
+static void run_exact(job_t *J, int b, int h, double *S, double *w, long long *deg)
+{
+    const int T = J->T, H = J->H, m = J->m, d = J->d;
+    for (int t = 0; t < T; ++t) {
+        size_t tok = IDX_TOK(b, t, h, T, H);
+        double eta = J->eta ? J->eta[tok] : 1.0;
+        exact_token(m, d, S, J->x + tok * d, J->c + tok * m, J->q + tok * m, J->mu[tok], eta,
+                    J->y + tok * d, w, deg);
+    }
+}
+
+static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0, double *n2,
+                                  double *g, double *kt, long long *deg)
+{
+    const int T = J->T, H = J->H, m = J->m, d = J->d, C = J->C;
+    for (int t0 = 0; t0 < T; t0 += C) {
+        int t1 = t0 + C < T ? t0 + C : T;
+        memcpy(S0, S, sizeof(double) * (size_t)m * d); /* chunk-start state S_{t'} */
+        for (int i = 0; i < m; ++i) {
+            double a = 0.0;
+            for (int k = 0; k < d; ++k) a += S0[(size_t)i * d + k] * S0[(size_t)i * d + k];
+            n2[i] = a;
+        }
+        for (int t = t0; t < t1; ++t) {
+            size_t tok = IDX_TOK(b, t, h, T, H);
+            const double *x = J->x + tok * d;
+            double eta = J->eta ? J->eta[tok] : 1.0;
+            oracle_chunk_token_gates(m, d, S0, n2, x, J->c + tok * m, J->mu[tok], eta, g, kt,
+                                     NULL, deg);
+            for (int i = 0; i < m; ++i) /* s_i <- g_i s_i + kt_i h,  h = -x */
+                for (int k = 0; k < d; ++k)
+                    S[(size_t)i * d + k] = g[i] * S[(size_t)i * d + k] + kt[i] * (-x[k]);
+            double *y = J->y + tok * d;
+            const double *q = J->q + tok * m;
+            for (int k = 0; k < d; ++k) y[k] = 0.0;
+            for (int i = 0; i < m; ++i)
+                for (int k = 0; k < d; ++k) y[k] += q[i] * S[(size_t)i * d + k];
+        }
+    }
+}
+
+/* Chunk-level closed form of the gated linear recurrence of Eq. 17 (the form
+ * that a chunk-parallel evaluation computes, §3.4.1 / Appendix B.1):
+ *   y_tau = sum_i q_tau,i A_tau,i s0_i + sum_{j<=tau} P_tau,j h_j,
+ *   P_tau,j = sum_i q_tau,i kt_j,i prod_{l=j+1..tau} g_l,i,
+ *   S_C,i   = A_C,i s0_i + sum_j kt_j,i prod_{l=j+1..C} g_l,i h_j,
+ * with A_tau = prod_{l<=tau} g_l. Products are formed directly (no division).
+ * Used to check the token-wise form; both share the per-token gates. */
+static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, double *n2,
+                               double *G, double *KT, long long *deg)
+{
+    const int T = J->T, H = J->H, m = J->m, d = J->d, C = J->C;
+    for (int t0 = 0; t0 < T; t0 += C) {
+        int L = (t0 + C < T ? t0 + C : T) - t0;
+        memcpy(S0, S, sizeof(double) * (size_t)m * d);
+        for (int i = 0; i < m; ++i) {
+            double a = 0.0;
+            for (int k = 0; k < d; ++k) a += S0[(size_t)i * d + k] * S0[(size_t)i * d + k];
+            n2[i] = a;
+        }
+        for (int tau = 0; tau < L; ++tau) {
+            size_t tok = IDX_TOK(b, t0 + tau, h, T, H);
+            double eta = J->eta ? J->eta[tok] : 1.0;
+            oracle_chunk_token_gates(m, d, S0, n2, J->x + tok * d, J->c + tok * m, J->mu[tok],
+                                     eta, G + (size_t)tau * m, KT + (size_t)tau * m, NULL, deg);
+        }
+        for (int tau = 0; tau < L; ++tau) {
+            size_t tok = IDX_TOK(b, t0 + tau, h, T, H);
+            const double *q = J->q + tok * m;
+            double *y = J->y + tok * d;
+            for (int k = 0; k < d; ++k) y[k] = 0.0;
+            for (int i = 0; i < m; ++i) { /* inter-chunk term (Q (.) A) S0 */
+                double A = 1.0;
+                for (int l = 0; l <= tau; ++l) A *= G[(size_t)l * m + i];
+                for (int k = 0; k < d; ++k) y[k] += q[i] * A * S0[(size_t)i * d + k];
+            }
+            for (int j = 0; j <= tau; ++j) { /* intra-chunk term P H */
+                double P = 0.0;
+                for (int i = 0; i < m; ++i) {
+                    double prod = 1.0;
+                    for (int l = j + 1; l <= tau; ++l) prod *= G[(size_t)l * m + i];
+                    P += q[i] * KT[(size_t)j * m + i] * prod;
+                }
+                const double *xj = J->x + IDX_TOK(b, t0 + j, h, T, H) * d;
+                for (int k = 0; k < d; ++k) y[k] += P * (-xj[k]);
+            }
+        }
+        for (int i = 0; i < m; ++i) { /* chunk-end state */
+            double A = 1.0;
+            for (int l = 0; l < L; ++l) A *= G[(size_t)l * m + i];
+            for (int k = 0; k < d; ++k) S[(size_t)i * d + k] = A * S0[(size_t)i * d + k];
+            for (int j = 0; j < L; ++j) {
+                double prod = 1.0;
+                for (int l = j + 1; l < L; ++l) prod *= G[(size_t)l * m + i];
+                double coef = KT[(size_t)j * m + i] * prod;
+                const double *xj = J->x + IDX_TOK(b, t0 + j, h, T, H) * d;
+                for (int k = 0; k < d; ++k) S[(size_t)i * d + k] += coef * (-xj[k]);
+            }
+        }
+    }
+}
+
+static void *worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    const int m = J->m, d = J->d;
+    int C = J->C > 0 ? J->C : 1;
+    double *S = malloc(sizeof(double) * (size_t)m * d);
+    double *S0 = malloc(sizeof(double) * (size_t)m * d);
+    double *n2 = malloc(sizeof(double) * (size_t)m);
+    double *w = malloc(sizeof(double) * (size_t)d);
+    double *G = malloc(sizeof(double) * (size_t)C * m);
+    double *KT = malloc(sizeof(double) * (size_t)C * m);
+    long long deg = 0;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int item = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (item >= J->B * J->H) break;
+        int b = item / J->H, h = item % J->H;
+        size_t so = ((size_t)b * J->H + h) * (size_t)m * d;
+        memcpy(S, J->S0 + so, sizeof(double) * (size_t)m * d);
+        if (J->form == 0)
+            run_exact(J, b, h, S, w, &deg);
+        else if (J->form == 1)
+            run_chunked_tokenwise(J, b, h, S, S0, n2, G, KT, &deg);
+        else
+            run_chunked_matrix(J, b, h, S, S0, n2, G, KT, &deg);
+        if (J->S_out) memcpy(J->S_out + so, S, sizeof(double) * (size_t)m * d);
+    }
+    pthread_mutex_lock(&J->lock);
+    J->degenerate += deg;
+    pthread_mutex_unlock(&J->lock);
+    free(S); free(S0); free(n2); free(w); free(G); free(KT);
+    return NULL;
+}
+
+static long long run(int form, int B, int T, int H, int m, int d, int C, const double *x,
+                     const double *c, const double *q, const double *mu, const double *eta,
+                     const double *S0, double *S_out, double *y, int nthreads)
+{
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C; J.form = form;
+    J.x = x; J.c = c; J.q = q; J.mu = mu; J.eta = eta; J.S0 = S0; J.S_out = S_out; J.y = y;
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > B * H) nthreads = B * H;
+    if (nthreads <= 1) {
+        worker(&J);
+    } else {
+        pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+        for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, &J);
+        for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+        free(th);
+    }
+    pthread_mutex_destroy(&J.lock);
+    return J.degenerate;
+}
+
+/* Exact recurrence (chunk size 1). Returns the number of zero-norm updates. */
+long long oracle_exact_scan(int B, int T, int H, int m, int d, const double *x, const double *c,
+                            const double *q, const double *mu, const double *eta,
+                            const double *S0, double *S_out, double *y, int nthreads)
+{
+    return run(0, B, T, H, m, d, 1, x, c, q, mu, eta, S0, S_out, y, nthreads);
+}
+
+/* Chunked recurrence of Eq. 17, chunk size C, evaluated token by token. */
+long long oracle_chunked_scan(int B, int T, int H, int m, int d, int C, const double *x,
+                              const double *c, const double *q, const double *mu,
+                              const double *eta, const double *S0, double *S_out, double *y,
+                              int nthreads)
+{
+    return run(1, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
+}
+
+/* Same definition evaluated through the chunk-level closed form (self-check). */
+long long oracle_chunked_matrix_scan(int B, int T, int H, int m, int d, int C, const double *x,
+                                     const double *c, const double *q, const double *mu,
+                                     const double *eta, const double *S0, double *S_out,
+                                     double *y, int nthreads)
+{
+    return run(2, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
+}
+
+/* Read-out y = sum_i q_i s_i for every (b,h): S[B][H][m][d], q[B][H][m], y[B][H][d]
+ * (Appendix D listing, y = q @ S_t; §2 eq. LA read-out). */
+void oracle_readout(int B, int H, int m, int d, const double *S, const double *q, double *y)
+{
+    for (int bh = 0; bh < B * H; ++bh) {
+        const double *Sb = S + (size_t)bh * m * d;
+        const double *qb = q + (size_t)bh * m;
+        double *yb = y + (size_t)bh * d;
+        for (int k = 0; k < d; ++k) yb[k] = 0.0;
+        for (int i = 0; i < m; ++i)
+            for (int k = 0; k < d; ++k) yb[k] += qb[i] * Sb[(size_t)i * d + k];
+    }
+}

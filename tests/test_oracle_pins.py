@@ -1,0 +1,329 @@
+"""Pins of the fp64 oracle to facts fixed by the paper and by the mathematics.
+
+Paper: "Lattice: Learning to Efficiently Compress the Memory" (arXiv 2504.05646).
+Each test names the passage or property it checks. None of these tests re-types
+the oracle's formula: they use printed values (Figure 1), independent
+constructions (explicit d x d projection matrices, finite differences of the
+loss, the d = 2 rotation angle) or invariants.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rand_inputs(rng, B, T, H, m, d, unit=True, mu_range=(0.3, 1.0), xs=1.0):
+    x = rng.standard_normal((B, T, H, d)) * xs
+    q = rng.standard_normal((B, T, H, m))
+    c = rng.uniform(0.05, 1.0, (B, T, H, m))
+    mu = rng.uniform(*mu_range, (B, T, H))
+    S0 = rng.standard_normal((B, H, m, d))
+    if unit:
+        S0 /= np.linalg.norm(S0, axis=-1, keepdims=True)
+    else:
+        S0 *= rng.uniform(0.5, 2.0, (B, H, m, 1))
+    return x, c, q, mu, S0
+
+
+def _read_golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, *v = line.split()
+            vals[k] = np.array([float(t) for t in v])
+    return vals
+
+
+# ---------------------------------------------------------------- Figure 1 ---
+
+def test_fig1_worked_example():
+    """Figure 1 (a),(b): P(s)h = (1.2,-0.6); s + alpha P(s)h = (2.2,1.4) at alpha = 1.
+    The oracle's write carries intensity c/|s|, so c = |s| gives alpha = 1."""
+    g = _read_golden("fig1_orthogonal_update.txt")
+    s, h = g["s"], g["h"]
+    n = math.sqrt(float(s @ s))
+    w, n2 = oracle.osr_write(s, h, c=n * g["alpha"][0], mu=1.0, eta=1.0)
+    assert n2 == pytest.approx(5.0, abs=1e-15)
+    np.testing.assert_allclose(w, g["s_next"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(w - s, g["h_perp"], rtol=0, atol=1e-14)
+    # the orthogonal write is not the linear-attention superposition
+    assert np.abs(w - g["s_hat_linear_attention"]).max() > 0.5
+    # other intensities and gates scale the same orthogonal direction
+    w2, _ = oracle.osr_write(s, h, c=0.7, mu=0.3, eta=0.5)
+    np.testing.assert_allclose(w2 - 0.3 * s, 0.5 * (0.7 / n) * g["h_perp"], atol=1e-14)
+
+
+# ------------------------------------------------------ §3.1.1 / §3.2 facts ---
+
+@pytest.mark.parametrize("d", [2, 7, 64])
+def test_write_is_orthogonal_and_pythagorean(d):
+    """§3.1.1: only the part orthogonal to the slot is written; §3.2:
+    |s + Delta|^2 = |s|^2 + |Delta|^2."""
+    rng = _rng(d)
+    for _ in range(20):
+        s = rng.standard_normal(d) * rng.uniform(0.2, 3.0)
+        x = rng.standard_normal(d)
+        mu, c, eta = rng.uniform(0, 1), rng.uniform(0, 2), rng.uniform(0.1, 2)
+        w, _ = oracle.osr_write(s, x, c, mu, eta)
+        delta = w - mu * s
+        assert abs(delta @ s) <= 1e-12 * np.linalg.norm(delta) * np.linalg.norm(s) + 1e-15
+        w1, _ = oracle.osr_write(s, x, c, 1.0, eta)
+        assert (w1 @ w1) == pytest.approx(s @ s + (w1 - s) @ (w1 - s), rel=1e-12)
+
+
+def test_write_is_negative_ogd_gradient_of_similarity_loss():
+    """§3.1.1 eq. (similarity_obj_stateNorm) and eq. (OSR), OGD step of eq. (OGD):
+    with mu = 1 the write equals -eta * dL/ds_i for L(S) = -<phi(S) c, x>,
+    phi normalising each slot. Checked by central finite differences at |s| != 1."""
+    rng = _rng(11)
+    m, d = 3, 5
+    S = rng.standard_normal((m, d)) * rng.uniform(0.5, 2.0, (m, 1))
+    x = rng.standard_normal(d)
+    c = rng.uniform(0.1, 1.0, m)
+    eta = 0.37
+
+    def loss(Sm):
+        phi = Sm / np.linalg.norm(Sm, axis=1, keepdims=True)
+        return -float((phi.T @ c) @ x)
+
+    eps = 1e-6
+    for i in range(m):
+        grad = np.zeros(d)
+        for k in range(d):
+            Sp, Sn = S.copy(), S.copy()
+            Sp[i, k] += eps
+            Sn[i, k] -= eps
+            grad[k] = (loss(Sp) - loss(Sn)) / (2 * eps)
+        w, _ = oracle.osr_write(S[i], x, c[i], 1.0, eta)
+        np.testing.assert_allclose(w - S[i], -eta * grad, rtol=1e-7, atol=1e-9)
+
+
+def test_unit_norm_after_every_exact_step():
+    """§3.2 eq. (normalized_recurrence): every slot is on the unit sphere after
+    each step, also when the initial slots are not."""
+    rng = _rng(3)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 12, 2, 5, 6, unit=False)
+    S = S0
+    for t in range(12):
+        y, S, deg = oracle.step(S, x[:, t], c[:, t], q[:, t], mu[:, t])
+        assert deg == 0
+        np.testing.assert_allclose(np.linalg.norm(S, axis=-1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_identity_when_gate_one_and_no_write():
+    """§3.3 eq. (dacay_recurrence) with mu = 1 and zero intensity: the state is
+    unchanged and the read-out is q . S0 at every step."""
+    rng = _rng(4)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 9, 3, 4, 8)
+    c[:] = 0.0
+    mu[:] = 1.0
+    y, S, deg = oracle.scan(x, c, q, mu, S0)
+    np.testing.assert_allclose(S, S0, atol=1e-15)
+    y_ref = np.einsum("bthm,bhmd->bthd", q, S0)
+    np.testing.assert_allclose(y, y_ref, atol=1e-13)
+    # the same holds for the chunked form
+    y2, S2, _ = oracle.scan(x, c, q, mu, S0, chunk=4)
+    np.testing.assert_allclose(S2, S0, atol=1e-15)
+    np.testing.assert_allclose(y2, y_ref, atol=1e-13)
+
+
+def test_redundant_input_leaves_slot_unchanged():
+    """§3.1.1 (highlight box): an input already aligned with a slot carries no
+    new information for it, so with mu = 1 that slot does not move."""
+    rng = _rng(5)
+    m, d = 4, 6
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 1, 1, m, d)
+    x[0, 0, 0] = -2.5 * S0[0, 0, 1]
+    mu[:] = 1.0
+    _, S, _ = oracle.scan(x, c, q, mu, S0)
+    np.testing.assert_allclose(S[0, 0, 1], S0[0, 0, 1], atol=1e-15)
+    assert np.abs(S[0, 0, 0] - S0[0, 0, 0]).max() > 1e-3
+
+
+def test_zero_norm_update_is_kept_and_counted():
+    """mu = 0 with an input parallel to the slot: the update is the zero vector,
+    whose projection onto the sphere is undefined; the slot is kept."""
+    rng = _rng(6)
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 1, 1, 3, 5)
+    x[0, 0, 0] = 0.8 * S0[0, 0, 2]
+    mu[:] = 0.0
+    _, S, deg = oracle.scan(x, c, q, mu, S0)
+    assert deg == 1
+    np.testing.assert_allclose(S[0, 0, 2], S0[0, 0, 2], atol=0)
+    _, S2, deg2 = oracle.scan(x, c, q, mu, S0, chunk=4)
+    assert deg2 == 1
+    np.testing.assert_allclose(S2[0, 0, 2], S0[0, 0, 2], atol=0)
+
+
+def test_closed_form_rotation_in_the_plane():
+    """d = 2, m = 1: a unit slot is an angle theta; the write adds eta c (x.t)
+    along the tangent t and mu along s, so theta' = theta + atan2(eta c (x.t), mu)."""
+    rng = _rng(7)
+    T = 6
+    for mu0 in (None, 0.0):
+        theta = rng.uniform(-np.pi, np.pi)
+        S0 = np.array([np.cos(theta), np.sin(theta)]).reshape(1, 1, 1, 2)
+        x = rng.standard_normal((1, T, 1, 2))
+        c = rng.uniform(0.1, 2.0, (1, T, 1, 1))
+        mu = rng.uniform(0.0, 1.0, (1, T, 1)) if mu0 is None else np.full((1, T, 1), mu0)
+        eta = rng.uniform(0.2, 1.5, (1, T, 1))
+        _, S, _ = oracle.scan(x, c, np.ones((1, T, 1, 1)), mu, S0, eta=eta)
+        th = theta
+        for t in range(T):
+            tang = np.array([-np.sin(th), np.cos(th)])
+            th = th + math.atan2(eta[0, t, 0] * c[0, t, 0, 0] * float(x[0, t, 0] @ tang),
+                                 mu[0, t, 0])
+        np.testing.assert_allclose(S[0, 0, 0], [np.cos(th), np.sin(th)], atol=1e-12)
+
+
+def test_brute_force_projection_matrices():
+    """eq. (OSR) evaluated literally: stack the Jacobians P(s_i)/|s_i| into a
+    d x d x m tensor, contract h^T with it (einsum 'd1, d1 d m -> d m'), scale
+    by the intensities, add mu S (General Form), project each slot onto the unit
+    sphere (§3.2) and read out with the updated state. Paper layout S is d x m."""
+    rng = _rng(8)
+    B, T, H, m, d = 2, 8, 2, 3, 5
+    x, c, q, mu, S0 = _rand_inputs(rng, B, T, H, m, d, unit=False)
+    eta = rng.uniform(0.2, 1.2, (B, T, H))
+    y_o, S_o, _ = oracle.scan(x, c, q, mu, S0, eta=eta)
+    for b in range(B):
+        for hh in range(H):
+            Sdm = S0[b, hh].T.copy()  # d x m, slots are columns
+            for t in range(T):
+                P = np.zeros((d, d, m))
+                for i in range(m):
+                    s = Sdm[:, i]
+                    P[:, :, i] = (np.eye(d) - np.outer(s, s) / (s @ s)) / np.linalg.norm(s)
+                h = -x[b, t, hh]
+                grad = np.einsum("a,adm->dm", h, P) * c[b, t, hh][None, :]
+                Snew = mu[b, t, hh] * Sdm - eta[b, t, hh] * grad
+                Sdm = Snew / np.linalg.norm(Snew, axis=0, keepdims=True)
+                np.testing.assert_allclose(y_o[b, t, hh], Sdm @ q[b, t, hh], atol=1e-12)
+            np.testing.assert_allclose(S_o[b, hh], Sdm.T, atol=1e-12)
+
+
+# ------------------------------------------------------ chunked form (Eq. 17) ---
+
+def test_chunk_size_one_is_the_exact_recurrence():
+    """Appendix C / Appendix D: chunk size 1 is the exact recurrence. With the
+    mu^2 reading of the chunk normaliser the two forms agree to rounding, also
+    for non-unit initial slots."""
+    rng = _rng(9)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 17, 3, 6, 7, unit=False)
+    eta = rng.uniform(0.2, 1.2, mu.shape)
+    y1, S1, _ = oracle.scan(x, c, q, mu, S0, eta=eta, chunk=1)
+    y2, S2, _ = oracle.scan(x, c, q, mu, S0, eta=eta, chunk=1, form="matrix")
+    # chunk=1 via the chunked code path (token form) too
+    y3, S3, _ = oracle.scan(x, c, q, mu, S0, eta=eta, chunk=1, form="token")
+    from oracle import _load, _f64, _p
+    lib = _load()
+    y4 = np.zeros_like(y1)
+    S4 = np.zeros_like(S1)
+    B, T, H, d = x.shape
+    m = c.shape[-1]
+    lib.oracle_chunked_scan(B, T, H, m, d, 1, _p(_f64(x)), _p(_f64(c)), _p(_f64(q)),
+                            _p(_f64(mu)), _p(_f64(eta)), _p(_f64(S0)), _p(S4), _p(y4), 1)
+    for y, S in ((y2, S2), (y3, S3), (y4, S4)):
+        np.testing.assert_allclose(y, y1, atol=1e-12)
+        np.testing.assert_allclose(S, S1, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [2, 4, 16, 64])
+def test_chunk_closed_form_equals_token_form(C):
+    """§3.4.1 / Appendix B.1: the chunk-level matrix form (cumulative gates,
+    causal score matrix, chunk-end state) equals the token-wise linear
+    recurrence of Eq. 17. Ragged final chunk included."""
+    rng = _rng(100 + C)
+    T = 2 * C + C // 2 + 1
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, T, 2, 5, 4, unit=False, mu_range=(0.6, 1.0))
+    y1, S1, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="token")
+    y2, S2, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="matrix")
+    np.testing.assert_allclose(y2, y1, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(S2, S1, rtol=1e-10, atol=1e-10)
+
+
+def test_chunk_first_token_matches_exact_step_and_later_tokens_differ():
+    """Eq. 17 is exact for the first token of each chunk (the chunk-start state
+    is the current state) and an approximation afterwards."""
+    rng = _rng(12)
+    C = 8
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, C, 1, 4, 6)
+    ye, Se, _ = oracle.scan(x, c, q, mu, S0, chunk=1)
+    yc, Sc, _ = oracle.scan(x, c, q, mu, S0, chunk=C)
+    np.testing.assert_allclose(yc[:, 0], ye[:, 0], atol=1e-13)
+    assert np.abs(yc[:, -1] - ye[:, -1]).max() > 1e-6
+
+
+def test_beta_matrix_form_equals_materialised_update_norm():
+    """Appendix B.1 eq. (beta_chunk): |Delta s_i|^2 from the closed form (with
+    the minus sign and clip at 0) equals the squared norm of the materialised
+    update Delta s_i = -khat_i P(s0_i) h, built here from an explicit projection
+    matrix; the printed '+' would not."""
+    rng = _rng(13)
+    m, d = 6, 9
+    S0 = rng.standard_normal((m, d)) * rng.uniform(0.5, 2.0, (m, 1))
+    for _ in range(10):
+        x = rng.standard_normal(d)
+        c = rng.uniform(0.0, 1.5, m)
+        eta = rng.uniform(0.2, 2.0)
+        g, kt, dsq, _ = oracle.chunk_token_gates(S0, x, c, mu=0.8, eta=eta)
+        h = -x
+        for i in range(m):
+            s = S0[i]
+            P = np.eye(d) - np.outer(s, s) / (s @ s)
+            delta = -(c[i] / np.linalg.norm(s)) * (P @ h)
+            assert dsq[i] == pytest.approx(eta ** 2 * (delta @ delta), rel=1e-10, abs=1e-14)
+            khat = c[i] / np.linalg.norm(s)
+            hhat = (h @ s) / (s @ s)
+            plus = eta ** 2 * (khat ** 2 * (h @ h) + (s @ s) * hhat ** 2 * khat ** 2)
+            if abs(hhat) > 1e-3 and c[i] > 1e-3:
+                assert abs(plus - dsq[i]) > 1e-8
+
+
+# ------------------------------------------------------------ composition ---
+
+def test_resume_composes():
+    """The state is the whole carry: scan(T1) then scan(T2) from S_T1 equals
+    scan(T1+T2) (exact: any split; chunked: T1 a multiple of C)."""
+    rng = _rng(14)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 24, 2, 4, 5)
+    for chunk, T1 in ((1, 7), (8, 16)):
+        y, S, _ = oracle.scan(x, c, q, mu, S0, chunk=chunk)
+        ya, Sa, _ = oracle.scan(x[:, :T1], c[:, :T1], q[:, :T1], mu[:, :T1], S0, chunk=chunk)
+        yb, Sb, _ = oracle.scan(x[:, T1:], c[:, T1:], q[:, T1:], mu[:, T1:], Sa, chunk=chunk)
+        np.testing.assert_array_equal(np.concatenate([ya, yb], 1), y)
+        np.testing.assert_array_equal(Sb, S)
+
+
+def test_readout_definition():
+    """Appendix D listing y = q @ S: y = sum_i q_i s_i, checked entrywise."""
+    rng = _rng(15)
+    S = rng.standard_normal((2, 3, 5, 7))
+    q = rng.standard_normal((2, 3, 5))
+    y = oracle.readout(S, q)
+    for b in range(2):
+        for h in range(3):
+            ref = sum(q[b, h, i] * S[b, h, i] for i in range(5))
+            np.testing.assert_allclose(y[b, h], ref, atol=1e-13)
+
+
+def test_threads_do_not_change_results():
+    rng = _rng(16)
+    x, c, q, mu, S0 = _rand_inputs(rng, 3, 10, 3, 4, 5)
+    for chunk in (1, 4):
+        y1, S1, _ = oracle.scan(x, c, q, mu, S0, chunk=chunk, nthreads=1)
+        y8, S8, _ = oracle.scan(x, c, q, mu, S0, chunk=chunk, nthreads=8)
+        np.testing.assert_array_equal(y1, y8)
+        np.testing.assert_array_equal(S1, S8)
