@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the Lattice compression-layer state recurrence on B200.
+
+A step is one lattice_scan_fwd over one batch of the small training shape
+(B=4, H=8, T=2048, m=d=64, chunk 64, bf16 x/q, fp32 state): the whole hot path
+(projection, orthogonal write, forget gate, unit-sphere projection, read-out,
+chunk state carry). Inputs are resident in HBM before the timed region; the L2
+is flushed (a 256 MiB write) between timed steps because this workload's
+inputs fit in L2. Each step is timed with CUDA events on the launching stream.
+
+The same JSON line also reports, as context, the mid-size and long-context
+scans, the exact recurrence, and the decode step (1000 consecutive steps of
+B=256, H=32, m=d=128), each with its roofline fraction.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no
+data-path collective); the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+
+import lattice_inputs as LI
+
+METRIC = "Lattice layer fwd tokens/s (1 B200) + % of roofline; decode step GB/s"
+HEADLINE = "small_train"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- arithmetic
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def scan_alg_bytes(w: LI.Workload, B=None, T=None, H=None) -> int:
+    """Algorithmic HBM bytes of one scan: every input read once, y and S written once."""
+    B = w.B if B is None else B
+    T = w.T if T is None else T
+    H = w.H if H is None else H
+    xb = 2 if w.x_dtype == "bf16" else 4
+    qb = 2 if w.q_dtype == "bf16" else 4
+    per_tok = w.d * xb + w.m * qb + 4 * w.m + 4 + 4 * w.d
+    return B * T * H * per_tok + 2 * 4 * B * H * w.m * w.d
+
+
+def chunk_mma_flops(w: LI.Workload, C: int, B=None, T=None, H=None) -> int:
+    """Tensor-core flops of the chunked form per token and head: 6md + C(m+d)
+    (projection, inter-chunk read-out and state update: 2md each; causal score
+    and intra-chunk read-out: C*m and C*d with the causal half counted once)."""
+    B = w.B if B is None else B
+    T = w.T if T is None else T
+    H = w.H if H is None else H
+    return B * T * H * (6 * w.m * w.d + C * (w.m + w.d))
+
+
+def step_alg_bytes(w: LI.Workload, B=None, H=None) -> int:
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    xb = 2 if w.x_dtype == "bf16" else 4
+    qb = 2 if w.q_dtype == "bf16" else 4
+    return B * H * (2 * 4 * w.m * w.d + w.d * xb + w.m * qb + 4 * w.m + 4 + 4 * w.d)
+
+
+# -------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        top = max(r[0] for r in rows)
+        loaded = [r[0] for r in rows if r[0] >= 0.5 * top] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": rows[0][1], "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------- GPU timing
+
+def _dev_inputs(torch, inp, device):
+    def vec(n):
+        b = inp.get(n + "_bits")
+        if b is not None:
+            return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(inp[n], np.float32)).to(device)
+    return dict(x=vec("x"), q=vec("q"), c=torch.from_numpy(inp["c"]).to(device),
+                mu=torch.from_numpy(inp["mu"]).to(device), S0=torch.from_numpy(inp["S0"]).to(device))
+
+
+def time_scan(torch, L, t, chunk, steps, warmup, flush=None, impl="auto"):
+    """Per-step device time (ms) of lattice_scan_fwd, CUDA events on its stream."""
+    stream = torch.cuda.current_stream()
+    y = torch.empty(t["x"].shape[:3] + (t["S0"].shape[-1],), dtype=torch.float32, device=t["x"].device)
+    S = torch.empty_like(t["S0"])
+    run = lambda: L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], chunk=chunk, S_out=S, y=y,
+                             impl=impl, stream=stream)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for e0, e1 in ev:
+        if flush is not None:
+            flush.add_(1)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    L.device_status()
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+
+def time_scan_e2e(torch, L, inp, chunk, steps, warmup, device):
+    """End to end through the public call with host buffers: pinned host inputs
+    are copied in, the scan runs, y and the final state are copied back."""
+    host = {}
+    for n in ("x", "q"):
+        b = inp.get(n + "_bits")
+        host[n] = (torch.from_numpy(b.view(np.int16)).view(torch.bfloat16) if b is not None
+                   else torch.from_numpy(inp[n])).pin_memory()
+    for n in ("c", "mu", "S0"):
+        host[n] = torch.from_numpy(inp[n]).pin_memory()
+    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    B, T, H, d = host["x"].shape
+    y = torch.empty((B, T, H, d), dtype=torch.float32, device=device)
+    S = torch.empty_like(dev["S0"])
+    y_h = torch.empty(y.shape, dtype=torch.float32).pin_memory()
+    S_h = torch.empty(S.shape, dtype=torch.float32).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y_h.numel() * 4 + S_h.numel() * 4
+
+    def run():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        L.scan_fwd(dev["x"], dev["c"], dev["q"], dev["mu"], dev["S0"], chunk=chunk, S_out=S, y=y,
+                   stream=stream)
+        y_h.copy_(y, non_blocking=True)
+        S_h.copy_(S, non_blocking=True)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def time_decode(torch, L, w, n_steps, ring, device):
+    """n_steps consecutive decode steps replayed from a CUDA graph over a ring of
+    pre-drawn per-step inputs (the ring and the 512 MiB state exceed L2)."""
+    S = torch.from_numpy(LI.make_decode_state(w)).to(device)
+    st = LI.make_decode_steps(w, ring)
+    xs = torch.from_numpy(st["x_bits"].view(np.int16)).view(torch.bfloat16).to(device)
+    qs = torch.from_numpy(st["q_bits"].view(np.int16)).view(torch.bfloat16).to(device)
+    cs = torch.from_numpy(st["c"]).to(device)
+    mus = torch.from_numpy(st["mu"]).to(device)
+    y = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=device)
+    s = torch.cuda.Stream(device=device)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for k in range(3):  # warm-up
+            L.step(S, xs[k], cs[k], qs[k], mus[k], y=y, stream=s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for k in range(ring):
+                L.step(S, xs[k], cs[k], qs[k], mus[k], y=y, stream=s)
+    torch.cuda.synchronize()
+    reps = max(1, n_steps // ring)
+    with torch.cuda.stream(s):
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(reps):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    L.device_status()
+    del g
+    return e0.elapsed_time(e1) / (reps * ring), reps * ring
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 10.0, max_reps: int = 50):
+    """The fp64 oracle, as it stands, on the host cores: whole workload passes
+    repeated until about min_seconds of CPU work. Returns (tokens/s, cores, sample)."""
+    import oracle
+    inp = LI.make_inputs(w)
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=chunk, nthreads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            break
+    tok = w.B * w.T * reps
+    sample = (f"{reps} full pass(es) of {w.name} (B={w.B},H={w.H},T={w.T},m={w.m},d={w.d}), "
+              f"{'exact' if chunk == 1 else f'chunked C={chunk}'}, fp64 oracle, {el:.1f} s")
+    return tok / el, cores, sample
+
+
+# ---------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the context workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = LI.WORKLOADS[HEADLINE]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        steps = max(1, args.steps)
+        import oracle
+        inp = LI.make_inputs(w)
+        cores = len(os.sched_getaffinity(0))
+        for _ in range(1):  # one untimed pass (the oracle has no warm-up state)
+            oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=w.chunk, nthreads=cores)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=w.chunk, nthreads=cores)
+        el = time.perf_counter() - t0
+        v = w.B * w.T * steps / el
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "m": w.m, "d": w.d,
+                           "chunk": w.chunk},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                 "sample": f"one full pass of {w.name} per step, chunked C={w.chunk}, "
+                                           f"fp64 C oracle on {cores} threads"},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import orthogonal_update_recurrent_b200 as L
+    from orthogonal_update_recurrent_b200 import build as Bld
+    if rank == 0 or not os.path.exists(Bld.LIB):
+        Bld.build()
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    L.lib()
+
+    pk, pk_src = peaks()
+    inp = LI.make_inputs(w)
+    t = _dev_inputs(torch, inp, device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        times = time_scan(torch, L, t, w.chunk, args.steps, args.warmup, flush=flush)
+    torch.cuda.synchronize()
+    total_ms = sum(times)
+    if dist is not None:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+        dist.barrier()
+    ms = total_ms / args.steps
+    value = world * w.B * w.T / (ms * 1e-3)
+
+    # roofline of the (single) kernel of the step
+    tc = L.chunk_impl(w.m, w.d, w.chunk) == "tcgen05"
+    alg_b = scan_alg_bytes(w)
+    kern_ms = statistics.mean(times)
+    achieved = alg_b / (kern_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / pk["hbm_gbs"], "traffic": None,
+            "kernel": "chunk_tc_kernel" if tc else "scan_simt_kernel<chunked>",
+            "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"}
+    if tc:
+        fl = chunk_mma_flops(w, w.chunk)
+        roof["tensor"] = {"achieved_tflops": fl / (kern_ms * 1e-3) / 1e12,
+                          "peak_tflops": pk["bf16_tflops"],
+                          "frac": fl / (kern_ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                          "flops_per_launch": fl}
+    t_roof_ms = 1e3 * max(alg_b / (pk["hbm_gbs"] * 1e9),
+                          (chunk_mma_flops(w, w.chunk) / (pk["bf16_tflops"] * 1e12)) if tc else 0.0)
+    roof["frac_of_binding_roofline"] = t_roof_ms / kern_ms
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if tc else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "m": w.m, "d": w.d,
+                       "chunk": w.chunk, "x_q_dtype": "bf16", "state_dtype": "f32",
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "parallelism": f"independent batches per GPU x{world}"},
+            "roofline": roof, "gpu_launches": args.steps}
+    cs = clk.summary()
+    if cs is not None:
+        line["clocks"] = cs
+
+    if rank == 0:
+        # end to end through the public call with host buffers
+        e2e_ms, h2d, d2h = time_scan_e2e(torch, L, inp, w.chunk, max(3, args.steps // 2), 3, device)
+        line["e2e"] = {"value": world * w.B * w.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        extra = {}
+        if not args.no_extra:
+            # exact recurrence on the headline workload
+            te = time_scan(torch, L, t, 1, 5, 3, flush=flush)
+            extra["small_train_exact"] = {"ms": statistics.mean(te),
+                                          "tokens_per_s": w.B * w.T / (statistics.mean(te) * 1e-3)}
+            del t
+            for name in ("mid_layer", "long_ctx"):
+                wn = LI.WORKLOADS[name]
+                inn = LI.make_inputs(wn)
+                tn = _dev_inputs(torch, inn, device)
+                del inn
+                tch = time_scan(torch, L, tn, wn.chunk, 5, 3)
+                ab = scan_alg_bytes(wn)
+                kms = statistics.mean(tch)
+                ent = {"chunk_ms": kms, "tokens_per_s": wn.B * wn.T / (kms * 1e-3),
+                       "hbm_gbs": ab / (kms * 1e-3) / 1e9, "hbm_frac": ab / (kms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                       "alg_bytes": ab}
+                fl = chunk_mma_flops(wn, wn.chunk)
+                ent["tensor_tflops"] = fl / (kms * 1e-3) / 1e12
+                ent["frac_of_binding_roofline"] = 1e3 * max(ab / (pk["hbm_gbs"] * 1e9),
+                                                            fl / (pk["bf16_tflops"] * 1e12)) / kms
+                tex = time_scan(torch, L, tn, 1, 3, 3)
+                ent["exact_ms"] = statistics.mean(tex)
+                ent["exact_tokens_per_s"] = wn.B * wn.T / (ent["exact_ms"] * 1e-3)
+                extra[name] = ent
+                del tn
+                torch.cuda.empty_cache()
+            wd = LI.WORKLOADS["decode"]
+            us_ms, n = time_decode(torch, L, wd, 1000, 40, device)
+            sb = step_alg_bytes(wd)
+            extra["decode"] = {"us_per_step": us_ms * 1e3, "steps": n, "gbps": sb / (us_ms * 1e-3) / 1e9,
+                               "hbm_frac": sb / (us_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                               "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb}
+        line["extra"] = extra
+        if not args.no_cpu:
+            v, cores, sample = oracle_baseline(w, w.chunk)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": sample}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,138 @@
+/*
+ * lattice.h -- C ABI of the B200 (sm_100a) Lattice compression-layer library.
+ *
+ * The library computes the state recurrence of "Lattice: Learning to
+ * Efficiently Compress the Memory" (Karami, Pascanu, Mirrokni; arXiv
+ * 2504.05646) for the similarity objective (h_t = -x_t):
+ *
+ *   per (batch b, head h), a state of m slots s_i in R^d (rows of S, the
+ *   layout of the paper's Appendix D listing), for every token t:
+ *     n_i = |s_i|,  p_i = s_i . x_t
+ *     w_i = mu_t s_i + eta_t (c_{t,i}/n_i) (x_t - (p_i/n_i^2) s_i)
+ *           [§3.1.1 eq. OSR: write only the part of x orthogonal to the slot,
+ *            scaled by the writing intensity c; §3.3 eq. dacay_recurrence:
+ *            forget gate mu; §3.4 Eq. 14: projection by one dot + one axpy]
+ *     s_i <- w_i / |w_i|        [§3.2 eq. normalized_recurrence: unit sphere]
+ *     y_t = sum_i q_{t,i} s_i   [read-out with the updated state, §3 General
+ *                                Form; Appendix D, y = q @ S_t]
+ *   If w_i = 0 (mu = 0 and no orthogonal write) the slot is left unchanged.
+ *
+ * The chunked form (chunk_size C > 1) is the paper's Eq. 17
+ * (recurrence_linear2, §3.4.1 and Appendix B.1): inside a chunk the projection
+ * uses the chunk-start state S0 (n_i = |s0_i|, p_i = s0_i . x_t) and the token
+ * update is the gated linear recurrence s_i <- g_{t,i} s_i + kappa_{t,i} x_t with
+ *   den = mu_t^2 n_i^2 + (eta_t c_{t,i}/n_i)^2 max(0, |x_t|^2 - p_i^2/n_i^2)
+ *   g   = n_i (mu_t - eta_t c_{t,i} p_i / n_i^3) / sqrt(den)
+ *   kappa = n_i (eta_t c_{t,i} / n_i) / sqrt(den)      [eq. beta_chunk]
+ * (g = 1, kappa = 0 where den = 0). The factor n_i = |s0_i| follows the paper's
+ * Appendix D listing, whose chunk normaliser keeps each slot's chunk-start
+ * norm. Chunks are consecutive blocks of C tokens; the last one may be
+ * partial. For unit-norm states, C = 1 is exactly the recurrence above.
+ *
+ * Layouts (row-major, element strides, no padding):
+ *   x    [B][T][H][d]   fp32 or bf16          input written into the slots
+ *   c    [B][T][H][m]   fp32                  writing intensities (codes)
+ *   q    [B][T][H][m]   fp32 or bf16          read-out queries
+ *   mu   [B][T][H]      fp32                  forget gate
+ *   eta  [B][T][H]      fp32, or NULL for 1   step size
+ *   S    [B][H][m][d]   fp32                  state, one slot per row
+ *   y    [B][T][H][d]   fp32                  read-out
+ * Decode calls drop the T axis.
+ *
+ * Ownership and execution: every pointer is caller-owned DEVICE memory. The
+ * library allocates nothing and keeps no state besides one device status
+ * word. Every call is asynchronous on `stream` (a cudaStream_t passed as
+ * void*, NULL = the legacy default stream) and returns after the launch.
+ *
+ * Errors: arguments are checked on the host before anything is launched; a
+ * failed check launches nothing and returns the code. LATTICE_ERR_CUDA means a
+ * launch or attribute call failed (call cudaGetLastError for the detail).
+ * Device-side waits are bounded: a kernel that gives up sets the status word
+ * and returns; lattice_get_device_status() reports it as LATTICE_ERR_TIMEOUT.
+ *
+ * Supported sizes: d in {16, 32, 64, 128}; 1 <= m <= 256; B, H >= 1; T >= 0.
+ * The tensor-core chunked kernel serves C = 64, m in {64, 128},
+ * d in {64, 128} with bf16 x and q; other chunked shapes run a CUDA-core
+ * kernel of the same definition.
+ */
+#ifndef LATTICE_H_
+#define LATTICE_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LATTICE_OK = 0,
+    LATTICE_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, partial aliasing  */
+    LATTICE_ERR_UNSUPPORTED = 2, /* valid but outside the supported sizes     */
+    LATTICE_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed      */
+    LATTICE_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up        */
+} lattice_status;
+
+typedef enum { LATTICE_F32 = 0, LATTICE_BF16 = 1 } lattice_dtype;
+
+/* Objective (§3.1.1). Only the similarity objective (h_t = -x_t) is built. */
+typedef enum { LATTICE_SIM = 0, LATTICE_DEC = 1 } lattice_mode;
+
+/* Kernel choice for chunked scans. AUTO picks the tensor-core kernel when the
+ * shape allows it. SIMT forces the CUDA-core kernel. TCGEN05 requires the
+ * tensor-core kernel and returns LATTICE_ERR_UNSUPPORTED when it cannot run. */
+typedef enum { LATTICE_IMPL_AUTO = 0, LATTICE_IMPL_SIMT = 1, LATTICE_IMPL_TCGEN05 = 2 } lattice_impl;
+
+/* Which kernel LATTICE_IMPL_AUTO runs for a chunked scan of this shape:
+ * returns LATTICE_IMPL_TCGEN05 or LATTICE_IMPL_SIMT (chunk_size 1 is always
+ * LATTICE_IMPL_SIMT). Pure host function; launches nothing. */
+lattice_impl lattice_chunk_impl(int m, int d, int chunk_size, lattice_dtype x_dtype,
+                                lattice_dtype q_dtype);
+
+/* Whole-sequence forward (the paper's lattice_compress, Appendix D).
+ * Reads S0, writes the final state to S_out (S_out == S0 is allowed: the
+ * update is then in place; any other overlap between outputs and inputs is
+ * LATTICE_ERR_INVALID_ARG) and the read-out of every token to y.
+ * chunk_size = 1: exact recurrence; chunk_size > 1: Eq. 17 chunked form.
+ * T = 0 copies S0 to S_out and writes nothing else. */
+lattice_status lattice_scan_fwd(const void *x, lattice_dtype x_dtype, const float *c,
+                                const void *q, lattice_dtype q_dtype, const float *mu,
+                                const float *eta, const float *S0, float *S_out, float *y,
+                                int B, int T, int H, int m, int d, int chunk_size,
+                                lattice_mode mode, void *stream);
+
+/* As lattice_scan_fwd, with an explicit kernel choice (see lattice_impl). */
+lattice_status lattice_scan_fwd_impl(const void *x, lattice_dtype x_dtype, const float *c,
+                                     const void *q, lattice_dtype q_dtype, const float *mu,
+                                     const float *eta, const float *S0, float *S_out, float *y,
+                                     int B, int T, int H, int m, int d, int chunk_size,
+                                     lattice_mode mode, lattice_impl impl, void *stream);
+
+/* One decode step: the exact recurrence for one new token per (b,h), state
+ * updated in place (constant work per token, §1-§2 of the paper).
+ *   S [B][H][m][d] in/out, x [B][H][d], c [B][H][m], q [B][H][m],
+ *   mu [B][H], eta [B][H] or NULL, y [B][H][d] out. */
+lattice_status lattice_step(float *S, const void *x, lattice_dtype x_dtype, const float *c,
+                            const void *q, lattice_dtype q_dtype, const float *mu,
+                            const float *eta, float *y, int B, int H, int m, int d,
+                            lattice_mode mode, void *stream);
+
+/* Read-out without an update: y[b][h][:] = sum_i q[b][h][i] S[b][h][i][:]
+ * (§2 eq. LA memory read-out; Appendix D y = q @ S). S [B][H][m][d],
+ * q [B][H][m], y [B][H][d]. */
+lattice_status lattice_readout(const float *S, const void *q, lattice_dtype q_dtype, float *y,
+                               int B, int H, int m, int d, void *stream);
+
+/* Synchronises `stream`, returns LATTICE_ERR_TIMEOUT if any kernel since the
+ * last call gave up a bounded wait (and clears the flag), LATTICE_ERR_CUDA if
+ * the stream reports an error, else LATTICE_OK. */
+lattice_status lattice_get_device_status(void *stream);
+
+/* Static English text for a status code. */
+const char *lattice_status_string(lattice_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int lattice_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LATTICE_H_ */

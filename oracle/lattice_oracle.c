@@ -27,9 +27,14 @@
  * Readings of points the paper leaves open (each is listed in the design notes):
  *   - slots are rows of S ([m][d]), as in the Appendix D listing;
  *   - the normaliser targets the unit sphere (§3.2), with no epsilon;
- *   - the normaliser of the chunked form is 1/sqrt(mu^2 n^2 + |Delta|^2), the
- *     Pythagorean norm of mu*s + Delta (the printed eta^2 coefficient reads as
- *     a typo: only mu^2 makes chunk size 1 equal the exact recurrence);
+ *   - the normaliser of the chunked form is n/sqrt(mu^2 n^2 + |Delta|^2) with
+ *     n = |s0| the chunk-start norm: the Appendix D listing (compress_chunk)
+ *     scales its rsqrt by s_norm, so a slot keeps its chunk-start norm; §B.1's
+ *     (1 + D_S)^(-1/2) is the same value for n = 1. Without the n factor the
+ *     chunked recurrence diverges (slot norms leave O(1) within a few chunks
+ *     and the gates of small-norm slots explode). The printed eta^2 in front
+ *     of s_norm^2 reads as a typo for mu^2: only mu^2 makes chunk size 1 equal
+ *     the exact recurrence (for unit-norm states);
  *   - D_S uses "minus" (Pythagoras, §3.2), clipped at zero;
  *   - a slot whose update has zero norm (mu = 0 and no orthogonal write) is
  *     left unchanged and counted.
@@ -98,10 +103,10 @@ static void exact_token(int m, int d, double *S, const double *x, const double *
 /* ------------------------------------------------------------------------ */
 
 /* Gates of one token against the chunk-start state S0 (Eq. 17 and eq.
- * beta_chunk, Appendix B.1):
+ * beta_chunk, Appendix B.1; normaliser as in the Appendix D listing):
  *   h = -x;  hhat_i = (h.s0_i)/n_i^2;  khat_i = c_i/n_i;
  *   dsq_i  = eta^2 * max(0, khat_i^2 |h|^2 - n_i^2 hhat_i^2 khat_i^2)
- *   beta_i = 1/sqrt(mu^2 n_i^2 + dsq_i)
+ *   beta_i = n_i/sqrt(mu^2 n_i^2 + dsq_i)
  *   g_i    = beta_i (mu + eta hhat_i khat_i),   kt_i = -beta_i eta khat_i
  * so that the token's update is s_i <- g_i s_i + kt_i h. */
 void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
@@ -126,7 +131,7 @@ void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
             if (degenerate) ++*degenerate;
             continue;
         }
-        double beta = 1.0 / sqrt(den);
+        double beta = sqrt(n2[i]) / sqrt(den);
         g[i] = beta * (mu + eta * hhat * khat);
         kt[i] = -beta * eta * khat;
     }

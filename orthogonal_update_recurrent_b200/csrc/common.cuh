@@ -1,0 +1,150 @@
+// common.cuh -- device helpers shared by the Lattice kernels (sm_100a).
+//
+// Slot layout on CUDA cores ("octet" layout): a slot s_i in R^D is held by 8
+// consecutive lanes of a warp; a warp therefore holds 4 slots at once (one per
+// octet). Lane j (0..7) of an octet owns EPL = D/8 elements, in VW-wide
+// vectors: element k of the lane lives at position VW*(j + 8*(k/VW)) + k%VW.
+// With this interleave, vector r of the 8 lanes covers one contiguous span of
+// 8*VW elements, so a row load or store is fully coalesced, and a dot product
+// over the slot is a lane-local sum followed by a 3-level octet shuffle.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lattice {
+
+// Device status word: set by kernels that gave up a bounded wait.
+__device__ unsigned int g_device_status = 0;
+constexpr unsigned int kStatusTimeout = 1u;
+
+__device__ __forceinline__ void flag_timeout() { atomicOr(&g_device_status, kStatusTimeout); }
+
+template <int D>
+struct Octet {
+    static_assert(D == 16 || D == 32 || D == 64 || D == 128, "D must be 16, 32, 64 or 128");
+    static constexpr int EPL = D / 8;                 // elements per lane
+    static constexpr int VW = EPL >= 4 ? 4 : EPL;     // vector width
+    static constexpr int NV = EPL / VW;               // vectors per lane
+    __device__ __forceinline__ static int pos(int j, int k) {
+        return VW * (j + 8 * (k / VW)) + (k % VW);
+    }
+};
+
+// Load the lane's EPL elements of a D-vector of fp32.
+template <int D>
+__device__ __forceinline__ void load_row_f32(const float* __restrict__ row, int j, float* v) {
+    using O = Octet<D>;
+#pragma unroll
+    for (int r = 0; r < O::NV; ++r) {
+        const float* p = row + O::VW * (j + 8 * r);
+        if constexpr (O::VW == 4) {
+            float4 t = *reinterpret_cast<const float4*>(p);
+            v[4 * r] = t.x; v[4 * r + 1] = t.y; v[4 * r + 2] = t.z; v[4 * r + 3] = t.w;
+        } else {
+            float2 t = *reinterpret_cast<const float2*>(p);
+            v[2 * r] = t.x; v[2 * r + 1] = t.y;
+        }
+    }
+}
+
+// Streaming (evict-first) variant for state rows read once per call.
+template <int D>
+__device__ __forceinline__ void load_row_f32_stream(const float* row, int j, float* v) {
+    using O = Octet<D>;
+#pragma unroll
+    for (int r = 0; r < O::NV; ++r) {
+        const float* p = row + O::VW * (j + 8 * r);
+        if constexpr (O::VW == 4) {
+            float4 t = __ldcs(reinterpret_cast<const float4*>(p));
+            v[4 * r] = t.x; v[4 * r + 1] = t.y; v[4 * r + 2] = t.z; v[4 * r + 3] = t.w;
+        } else {
+            float2 t = __ldcs(reinterpret_cast<const float2*>(p));
+            v[2 * r] = t.x; v[2 * r + 1] = t.y;
+        }
+    }
+}
+
+template <int D, bool STREAM>
+__device__ __forceinline__ void store_row_f32(float* row, int j, const float* v) {
+    using O = Octet<D>;
+#pragma unroll
+    for (int r = 0; r < O::NV; ++r) {
+        float* p = row + O::VW * (j + 8 * r);
+        if constexpr (O::VW == 4) {
+            float4 t = make_float4(v[4 * r], v[4 * r + 1], v[4 * r + 2], v[4 * r + 3]);
+            if constexpr (STREAM) __stcs(reinterpret_cast<float4*>(p), t);
+            else *reinterpret_cast<float4*>(p) = t;
+        } else {
+            float2 t = make_float2(v[2 * r], v[2 * r + 1]);
+            if constexpr (STREAM) __stcs(reinterpret_cast<float2*>(p), t);
+            else *reinterpret_cast<float2*>(p) = t;
+        }
+    }
+}
+
+// Load the lane's elements of a D-vector stored as bf16 or fp32 (global or shared).
+template <int D>
+__device__ __forceinline__ void load_row_any(const void* row, bool bf16, int j, float* v) {
+    using O = Octet<D>;
+    if (!bf16) {
+        load_row_f32<D>(static_cast<const float*>(row), j, v);
+        return;
+    }
+    const __nv_bfloat16* b = static_cast<const __nv_bfloat16*>(row);
+#pragma unroll
+    for (int r = 0; r < O::NV; ++r) {
+        const __nv_bfloat16* p = b + O::VW * (j + 8 * r);
+        if constexpr (O::VW == 4) {
+            uint2 t = *reinterpret_cast<const uint2*>(p);
+            v[4 * r + 0] = __uint_as_float(t.x << 16);
+            v[4 * r + 1] = __uint_as_float(t.x & 0xffff0000u);
+            v[4 * r + 2] = __uint_as_float(t.y << 16);
+            v[4 * r + 3] = __uint_as_float(t.y & 0xffff0000u);
+        } else {
+            uint32_t t = *reinterpret_cast<const uint32_t*>(p);
+            v[2 * r + 0] = __uint_as_float(t << 16);
+            v[2 * r + 1] = __uint_as_float(t & 0xffff0000u);
+        }
+    }
+}
+
+__device__ __forceinline__ float load_elem(const void* base, bool bf16, size_t i) {
+    if (bf16) {
+        uint16_t u = static_cast<const uint16_t*>(base)[i];
+        return __uint_as_float(static_cast<uint32_t>(u) << 16);
+    }
+    return static_cast<const float*>(base)[i];
+}
+
+__device__ __forceinline__ float octet_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    return v;
+}
+
+// Per-slot update coefficients. The new slot is alpha*s + gamma*x.
+//   n2 = |s_ref|^2, p = s_ref . x, xx = |x|^2 (s_ref = current slot for the exact
+//   recurrence, chunk-start slot for the chunked form).
+//   w = (mu - a p/n2) s + a x with a = eta c / n; |w|^2 = mu^2 n2 + a^2 (xx - p^2/n2)
+//   (Pythagoras: the write is orthogonal to s_ref). The result is scaled to norm
+//   `target` (1 for the exact recurrence's unit sphere, |s0| for the chunked
+//   form's normaliser). Zero-norm updates keep the slot.
+__device__ __forceinline__ void update_coefs(float n2, float p, float xx, float c, float mu,
+                                             float eta, float target, float& alpha,
+                                             float& gamma) {
+    bool ok = n2 > 0.f;
+    float n2s = ok ? n2 : 1.f;
+    float inv_n = rsqrtf(n2s);
+    float r = p / n2s;                      // p / n^2
+    float a = eta * c * inv_n;              // eta c / n
+    float perp2 = fmaxf(fmaf(-p, r, xx), 0.f);  // |x_perp|^2
+    float w2 = fmaf(a * a, perp2, mu * mu * n2s);
+    ok = ok && (w2 > 0.f);
+    float iw = rsqrtf(ok ? w2 : 1.f) * target;
+    alpha = ok ? fmaf(-a, r, mu) * iw : 1.f;
+    gamma = ok ? a * iw : 0.f;
+}
+
+}  // namespace lattice

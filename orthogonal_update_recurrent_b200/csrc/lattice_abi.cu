@@ -1,0 +1,253 @@
+// lattice_abi.cu -- extern "C" entry points of liblattice (declared in
+// include/lattice.h): argument checks, kernel choice and launches.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lattice.h"
+#include "common.cuh"
+#include "scan_simt.cuh"
+#include "step.cuh"
+#include "chunk_tc.cuh"
+
+using namespace lattice;
+
+namespace {
+
+struct Span {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+
+Span span(const void* p, size_t bytes) {
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Span{a, a + bytes};
+}
+bool overlap(Span a, Span b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+bool dtype_ok(lattice_dtype t) { return t == LATTICE_F32 || t == LATTICE_BF16; }
+size_t dsize(lattice_dtype t) { return t == LATTICE_BF16 ? 2 : 4; }
+bool d_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+lattice_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? LATTICE_OK : LATTICE_ERR_CUDA;
+}
+
+// ---- exact / chunked CUDA-core scan
+template <int D, int RQ, bool CH>
+lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
+    size_t smem = scan_smem_bytes<D>(a.m, nw);
+    auto k = scan_simt_kernel<D, RQ, CH>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return LATTICE_ERR_CUDA;
+    k<<<a.B * a.H, nw * 32, smem, st>>>(a);
+    return launch_status();
+}
+
+template <int D, bool CH>
+lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
+    const int quads = (a.m + 3) / 4;
+    if (quads <= 16) return launch_scan_simt_t<D, 1, CH>(a, quads < 4 ? 4 : quads, st);
+    if (quads <= 32) return launch_scan_simt_t<D, 2, CH>(a, 16, st);
+    return launch_scan_simt_t<D, 4, CH>(a, 16, st);
+}
+
+template <bool CH>
+lattice_status launch_scan_simt(const ScanArgs& a, int d, cudaStream_t st) {
+    switch (d) {
+        case 16: return launch_scan_simt_d<16, CH>(a, st);
+        case 32: return launch_scan_simt_d<32, CH>(a, st);
+        case 64: return launch_scan_simt_d<64, CH>(a, st);
+        case 128: return launch_scan_simt_d<128, CH>(a, st);
+    }
+    return LATTICE_ERR_UNSUPPORTED;
+}
+
+// ---- decode step / read-out: NW warps x RQ quads per warp
+void step_shape(int m, int& nw, int& rq) {
+    const int quads = (m + 3) / 4;
+    if (quads <= 8) { nw = quads; rq = 1; }
+    else if (quads <= 16) { nw = 8; rq = 2; }
+    else if (quads <= 32) { nw = 8; rq = 4; }
+    else { nw = 16; rq = 4; }
+}
+
+template <int D>
+lattice_status launch_step_d(const StepArgs& a, cudaStream_t st) {
+    int nw, rq;
+    step_shape(a.m, nw, rq);
+    dim3 grid(a.B * a.H), block(nw * 32);
+    switch (rq) {
+        case 1: step_kernel<D, 1><<<grid, block, 0, st>>>(a); break;
+        case 2: step_kernel<D, 2><<<grid, block, 0, st>>>(a); break;
+        default: step_kernel<D, 4><<<grid, block, 0, st>>>(a); break;
+    }
+    return launch_status();
+}
+
+template <int D>
+lattice_status launch_readout_d(const ReadoutArgs& a, cudaStream_t st) {
+    int nw, rq;
+    step_shape(a.m, nw, rq);
+    dim3 grid(a.B * a.H), block(nw * 32);
+    switch (rq) {
+        case 1: readout_kernel<D, 1><<<grid, block, 0, st>>>(a); break;
+        case 2: readout_kernel<D, 2><<<grid, block, 0, st>>>(a); break;
+        default: readout_kernel<D, 4><<<grid, block, 0, st>>>(a); break;
+    }
+    return launch_status();
+}
+
+lattice_status check_dims(int B, int H, int m, int d) {
+    if (B < 1 || H < 1 || m < 1 || d < 1) return LATTICE_ERR_INVALID_ARG;
+    if ((long long)B * H > 0x7fffffffLL) return LATTICE_ERR_UNSUPPORTED;
+    if (!d_supported(d) || m > kMaxM) return LATTICE_ERR_UNSUPPORTED;
+    return LATTICE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lattice_version(void) { return 100; }
+
+const char* lattice_status_string(lattice_status s) {
+    switch (s) {
+        case LATTICE_OK: return "ok";
+        case LATTICE_ERR_INVALID_ARG: return "invalid argument";
+        case LATTICE_ERR_UNSUPPORTED: return "unsupported size or dtype";
+        case LATTICE_ERR_CUDA: return "CUDA error";
+        case LATTICE_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+lattice_impl lattice_chunk_impl(int m, int d, int chunk_size, lattice_dtype x_dtype,
+                                lattice_dtype q_dtype) {
+    if (chunk_size > 1 && chunk_tc_supported(m, d, chunk_size, x_dtype == LATTICE_BF16,
+                                             q_dtype == LATTICE_BF16))
+        return LATTICE_IMPL_TCGEN05;
+    return LATTICE_IMPL_SIMT;
+}
+
+lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const float* c,
+                                     const void* q, lattice_dtype q_dtype, const float* mu,
+                                     const float* eta, const float* S0, float* S_out, float* y,
+                                     int B, int T, int H, int m, int d, int chunk_size,
+                                     lattice_mode mode, lattice_impl impl, void* stream) {
+    if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return LATTICE_ERR_INVALID_ARG;
+    if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
+    if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05)
+        return LATTICE_ERR_INVALID_ARG;
+    if (mode != LATTICE_SIM) return mode == LATTICE_DEC ? LATTICE_ERR_UNSUPPORTED : LATTICE_ERR_INVALID_ARG;
+    lattice_status ds = check_dims(B, H, m, d);
+    if (ds != LATTICE_OK) return ds;
+    if (!S0 || !S_out) return LATTICE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !c || !q || !mu || !y)) return LATTICE_ERR_INVALID_ARG;
+    if (!aligned(S0, 16) || !aligned(S_out, 16)) return LATTICE_ERR_INVALID_ARG;
+    const size_t nS = (size_t)B * H * m * d * 4;
+    const Span sS0 = span(S0, nS), sSo = span(S_out, nS);
+    if (S0 != S_out && overlap(sS0, sSo)) return LATTICE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (S0 != S_out && cudaMemcpyAsync(S_out, S0, nS, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return LATTICE_ERR_CUDA;
+        return LATTICE_OK;
+    }
+    const size_t ntok = (size_t)B * T * H;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(c, 4) || !aligned(mu, 4) ||
+        !aligned(q, dsize(q_dtype)) || (eta && !aligned(eta, 4)))
+        return LATTICE_ERR_INVALID_ARG;
+    const Span sx = span(x, ntok * d * dsize(x_dtype)), sc = span(c, ntok * m * 4),
+               sq = span(q, ntok * m * dsize(q_dtype)), smu = span(mu, ntok * 4),
+               seta = span(eta, eta ? ntok * 4 : 0), sy = span(y, ntok * d * 4);
+    const Span ins[] = {sx, sc, sq, smu, seta, sS0};
+    for (const Span& s : ins)
+        if (overlap(s, sy) || (s.lo != sS0.lo && overlap(s, sSo))) return LATTICE_ERR_INVALID_ARG;
+    if (overlap(sy, sSo)) return LATTICE_ERR_INVALID_ARG;
+
+    ScanArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, S_out, y,
+               B, T, H, m, chunk_size};
+    if (chunk_size == 1) {
+        if (impl == LATTICE_IMPL_TCGEN05) return LATTICE_ERR_UNSUPPORTED;
+        return launch_scan_simt<false>(a, d, st);
+    }
+    const bool tc_ok = chunk_tc_supported(m, d, chunk_size, a.x_bf16, a.q_bf16);
+    if (impl == LATTICE_IMPL_TCGEN05 && !tc_ok) return LATTICE_ERR_UNSUPPORTED;
+    if (tc_ok && impl != LATTICE_IMPL_SIMT) {
+        cudaError_t e = launch_chunk_tc(a, d, st);
+        return e == cudaSuccess ? LATTICE_OK : LATTICE_ERR_CUDA;
+    }
+    return launch_scan_simt<true>(a, d, st);
+}
+
+lattice_status lattice_scan_fwd(const void* x, lattice_dtype x_dtype, const float* c,
+                                const void* q, lattice_dtype q_dtype, const float* mu,
+                                const float* eta, const float* S0, float* S_out, float* y, int B,
+                                int T, int H, int m, int d, int chunk_size, lattice_mode mode,
+                                void* stream) {
+    return lattice_scan_fwd_impl(x, x_dtype, c, q, q_dtype, mu, eta, S0, S_out, y, B, T, H, m, d,
+                                 chunk_size, mode, LATTICE_IMPL_AUTO, stream);
+}
+
+lattice_status lattice_step(float* S, const void* x, lattice_dtype x_dtype, const float* c,
+                            const void* q, lattice_dtype q_dtype, const float* mu,
+                            const float* eta, float* y, int B, int H, int m, int d,
+                            lattice_mode mode, void* stream) {
+    if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
+    if (mode != LATTICE_SIM) return mode == LATTICE_DEC ? LATTICE_ERR_UNSUPPORTED : LATTICE_ERR_INVALID_ARG;
+    lattice_status ds = check_dims(B, H, m, d);
+    if (ds != LATTICE_OK) return ds;
+    if (!S || !x || !c || !q || !mu || !y) return LATTICE_ERR_INVALID_ARG;
+    if (!aligned(S, 16) || !aligned(x, 16) || !aligned(y, 16) || !aligned(c, 4) ||
+        !aligned(mu, 4) || !aligned(q, dsize(q_dtype)) || (eta && !aligned(eta, 4)))
+        return LATTICE_ERR_INVALID_ARG;
+    const size_t nbh = (size_t)B * H;
+    const Span sS = span(S, nbh * m * d * 4), sy = span(y, nbh * d * 4);
+    const Span ins[] = {span(x, nbh * d * dsize(x_dtype)), span(c, nbh * m * 4),
+                        span(q, nbh * m * dsize(q_dtype)), span(mu, nbh * 4),
+                        span(eta, eta ? nbh * 4 : 0)};
+    for (const Span& s : ins)
+        if (overlap(s, sS) || overlap(s, sy)) return LATTICE_ERR_INVALID_ARG;
+    if (overlap(sS, sy)) return LATTICE_ERR_INVALID_ARG;
+    StepArgs a{S, x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, y, B, H, m};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (d) {
+        case 16: return launch_step_d<16>(a, st);
+        case 32: return launch_step_d<32>(a, st);
+        case 64: return launch_step_d<64>(a, st);
+        default: return launch_step_d<128>(a, st);
+    }
+}
+
+lattice_status lattice_readout(const float* S, const void* q, lattice_dtype q_dtype, float* y,
+                               int B, int H, int m, int d, void* stream) {
+    if (!dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
+    lattice_status ds = check_dims(B, H, m, d);
+    if (ds != LATTICE_OK) return ds;
+    if (!S || !q || !y) return LATTICE_ERR_INVALID_ARG;
+    if (!aligned(S, 16) || !aligned(y, 16) || !aligned(q, dsize(q_dtype))) return LATTICE_ERR_INVALID_ARG;
+    const size_t nbh = (size_t)B * H;
+    const Span sy = span(y, nbh * d * 4);
+    if (overlap(sy, span(S, nbh * m * d * 4)) || overlap(sy, span(q, nbh * m * dsize(q_dtype))))
+        return LATTICE_ERR_INVALID_ARG;
+    ReadoutArgs a{S, q, q_dtype == LATTICE_BF16, y, B, H, m};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (d) {
+        case 16: return launch_readout_d<16>(a, st);
+        case 32: return launch_readout_d<32>(a, st);
+        case 64: return launch_readout_d<64>(a, st);
+        default: return launch_readout_d<128>(a, st);
+    }
+}
+
+lattice_status lattice_get_device_status(void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return LATTICE_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return LATTICE_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+        return LATTICE_ERR_CUDA;
+    return v ? LATTICE_ERR_TIMEOUT : LATTICE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,261 @@
+// scan_simt.cuh -- CUDA-core scan of the Lattice recurrence, exact or chunked.
+//
+// One CTA per (b, h) sequence; the m slots live in registers (octet layout,
+// common.cuh), RQ slot quads per warp. Tokens are processed in order; inputs
+// are staged through shared memory TB tokens at a time (loaded into registers
+// one block ahead, stored after the current block's compute), and the
+// read-out partial sums of the warps are reduced across warps through shared
+// memory once per block, in a fixed order (bit-reproducible).
+//
+// EXACT (CHUNKED = false): §3.1.1 eq. OSR + §3.2 eq. normalized_recurrence +
+// §3.3 forget gate, projection by Eq. 14 against the current slot.
+// CHUNKED: Eq. 17 (§3.4.1, Appendix B.1): the projection and the normaliser use
+// the state at the start of the chunk, kept in a second register set; the
+// normaliser n/sqrt(mu^2 n^2 + |Delta|^2) keeps the chunk-start norm n (the
+// paper's Appendix D listing scales its rsqrt by the slot norm).
+#pragma once
+#include "common.cuh"
+
+namespace lattice {
+
+constexpr int kScanTB = 8;      // tokens per staged block
+constexpr int kMaxM = 256;
+
+struct ScanArgs {
+    const void* x; bool x_bf16;
+    const float* c;
+    const void* q; bool q_bf16;
+    const float* mu;
+    const float* eta;            // may be null (=> 1)
+    const float* S0;
+    float* S_out;
+    float* y;
+    int B, T, H, m, chunk;
+};
+
+// Per-token staged record: x[D] | q[m] | c[m] | mu | eta, padded to a multiple
+// of 4 floats so that every record starts 16-byte aligned.
+__host__ __device__ inline int scan_record_floats(int D, int m) { return (D + 2 * m + 2 + 3) & ~3; }
+
+// Shared memory: in[2][TB][record] floats, ybuf[2][TB][NW][D] floats.
+template <int D>
+__host__ __device__ inline size_t scan_smem_bytes(int m, int nw) {
+    return sizeof(float) * (2ull * kScanTB * scan_record_floats(D, m) + 2ull * kScanTB * nw * D);
+}
+
+template <int D, int RQ, bool CHUNKED>
+__global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
+    using O = Octet<D>;
+    constexpr int EPL = O::EPL;
+    extern __shared__ __align__(16) float smem[];
+    const int NW = blockDim.x >> 5;
+    const int NT = blockDim.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int j = lane & 7, oct = lane >> 3;
+    const int bh = blockIdx.x;
+    const int b = bh / a.H, h = bh % a.H;
+    const int m = a.m, T = a.T, H = a.H;
+    const int per_tok = scan_record_floats(D, m);  // x | q | c | mu | eta | pad
+    float* in_buf = smem;
+    float* ybuf = smem + 2 * kScanTB * per_tok;
+
+    // ---- load the initial state into registers
+    float s[RQ][EPL];
+    float s0[CHUNKED ? RQ : 1][CHUNKED ? EPL : 1];
+    float n0sq[RQ], n0[RQ];
+    int slot[RQ];
+    const float* S0bh = a.S0 + (size_t)bh * m * D;
+#pragma unroll
+    for (int r = 0; r < RQ; ++r) {
+        slot[r] = 4 * (warp + NW * r) + oct;
+        if (slot[r] < m) {
+            load_row_f32<D>(S0bh + (size_t)slot[r] * D, j, s[r]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) s[r][k] = 0.f;
+        }
+        n0sq[r] = 0.f;
+        n0[r] = 1.f;
+    }
+
+    // ---- staging helpers
+    const int n_blocks = (T + kScanTB - 1) / kScanTB;
+    const int stage_total = kScanTB * per_tok;
+    // per-thread staging registers: the host launches NW >= 4 warps when RQ == 1, NW = 16 otherwise
+    constexpr int kMinThreads = RQ == 1 ? 128 : 512;
+    constexpr int kStg = (kScanTB * (D + 2 * kMaxM + 4) + kMinThreads - 1) / kMinThreads;
+    float stg[kStg];
+    auto stage_load = [&](int blk) {
+        const int t0 = blk * kScanTB;
+#pragma unroll
+        for (int u = 0; u < kStg; ++u) {
+            int idx = tid + u * NT;
+            float v = 0.f;
+            if (idx < stage_total) {
+                int tok = idx / per_tok, e = idx - tok * per_tok;
+                int t = t0 + tok;
+                if (t < T) {
+                    size_t bth = ((size_t)b * T + t) * H + h;
+                    if (e < D) v = load_elem(a.x, a.x_bf16, bth * D + e);
+                    else if (e < D + m) v = load_elem(a.q, a.q_bf16, bth * m + (e - D));
+                    else if (e < D + 2 * m) v = a.c[bth * m + (e - D - m)];
+                    else if (e == D + 2 * m) v = a.mu[bth];
+                    else if (e == D + 2 * m + 1) v = a.eta ? a.eta[bth] : 1.f;
+                }
+            }
+            stg[u] = v;
+        }
+    };
+    auto stage_store = [&](int buf) {
+        float* dst = in_buf + buf * stage_total;
+#pragma unroll
+        for (int u = 0; u < kStg; ++u) {
+            int idx = tid + u * NT;
+            if (idx < stage_total) dst[idx] = stg[u];
+        }
+    };
+
+    if (n_blocks > 0) {
+        stage_load(0);
+        stage_store(0);
+    }
+    __syncthreads();
+
+    for (int blk = 0; blk < n_blocks; ++blk) {
+        const int buf = blk & 1;
+        const int t0 = blk * kScanTB;
+        // flush the previous block's read-out (fixed-order sum over warps)
+        if (blk > 0) {
+            const int pt0 = t0 - kScanTB;
+            const float* yb = ybuf + (size_t)(buf ^ 1) * kScanTB * NW * D;
+            for (int idx = tid; idx < kScanTB * D; idx += NT) {
+                int tok = idx / D, k = idx - tok * D;
+                float acc = 0.f;
+                for (int w = 0; w < NW; ++w) acc += yb[((size_t)tok * NW + w) * D + k];
+                a.y[(((size_t)b * T + pt0 + tok) * H + h) * D + k] = acc;
+            }
+        }
+        if (blk + 1 < n_blocks) stage_load(blk + 1);
+
+        const float* inb = in_buf + buf * stage_total;
+        float* yb = ybuf + (size_t)buf * kScanTB * NW * D;
+        const int ntok = min(kScanTB, T - t0);
+        for (int tok = 0; tok < ntok; ++tok) {
+            const int t = t0 + tok;
+            const float* rec = inb + tok * per_tok;
+            float xv[EPL];
+            load_row_f32<D>(rec, j, xv);
+            const float mu = rec[D + 2 * m], eta = rec[D + 2 * m + 1];
+            float xx = 0.f;
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) xx = fmaf(xv[k], xv[k], xx);
+            xx = octet_sum(xx);
+
+            if constexpr (CHUNKED) {
+                if (t % a.chunk == 0) {  // chunk start: snapshot the state and its norms
+#pragma unroll
+                    for (int r = 0; r < RQ; ++r) {
+                        float n2 = 0.f;
+#pragma unroll
+                        for (int k = 0; k < EPL; ++k) { s0[r][k] = s[r][k]; n2 = fmaf(s[r][k], s[r][k], n2); }
+                        n0sq[r] = octet_sum(n2);
+                        n0[r] = sqrtf(n0sq[r]);
+                    }
+                }
+            }
+            float p[RQ], n2[RQ];
+#pragma unroll
+            for (int r = 0; r < RQ; ++r) {
+                float pp = 0.f, nn = 0.f;
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) {
+                    if constexpr (CHUNKED) {
+                        pp = fmaf(s0[r][k], xv[k], pp);
+                    } else {
+                        pp = fmaf(s[r][k], xv[k], pp);
+                        nn = fmaf(s[r][k], s[r][k], nn);
+                    }
+                }
+                p[r] = pp;
+                n2[r] = nn;
+            }
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    p[r] += __shfl_xor_sync(0xffffffffu, p[r], o);
+                    if constexpr (!CHUNKED) n2[r] += __shfl_xor_sync(0xffffffffu, n2[r], o);
+                }
+            }
+            float yp[EPL];
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) yp[k] = 0.f;
+#pragma unroll
+            for (int r = 0; r < RQ; ++r) {
+                const bool valid = slot[r] < m;
+                const float cv = valid ? rec[D + m + slot[r]] : 0.f;
+                const float qv = valid ? rec[D + slot[r]] : 0.f;
+                float alpha, gamma;
+                update_coefs(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
+                             CHUNKED ? n0[r] : 1.f, alpha, gamma);
+                if (!valid) { alpha = 0.f; gamma = 0.f; }
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) {
+                    s[r][k] = fmaf(alpha, s[r][k], gamma * xv[k]);
+                    yp[k] = fmaf(qv, s[r][k], yp[k]);
+                }
+            }
+            // reduce the read-out over the 4 octets of the warp (reduce-scatter)
+            float* ydst = yb + ((size_t)tok * NW + warp) * D;
+            if constexpr (EPL >= 4) {
+                const int hi = (lane >> 4) & 1, mid = (lane >> 3) & 1;
+                float v1[EPL / 2];
+#pragma unroll
+                for (int k = 0; k < EPL / 2; ++k) {
+                    float send = hi ? yp[k] : yp[k + EPL / 2];
+                    float keep = hi ? yp[k + EPL / 2] : yp[k];
+                    v1[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+                float v2[EPL / 4];
+#pragma unroll
+                for (int k = 0; k < EPL / 4; ++k) {
+                    float send = mid ? v1[k] : v1[k + EPL / 4];
+                    float keep = mid ? v1[k + EPL / 4] : v1[k];
+                    v2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+                const int kbase = hi * (EPL / 2) + mid * (EPL / 4);
+#pragma unroll
+                for (int k = 0; k < EPL / 4; ++k) ydst[O::pos(j, kbase + k)] = v2[k];
+            } else {  // EPL == 2
+                const int hi = (lane >> 4) & 1, mid = (lane >> 3) & 1;
+                float send = hi ? yp[0] : yp[1];
+                float keep = hi ? yp[1] : yp[0];
+                float v = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                if (!mid) ydst[O::pos(j, hi)] = v;
+            }
+        }
+        if (blk + 1 < n_blocks) stage_store(buf ^ 1);
+        __syncthreads();
+    }
+    // flush the last block
+    if (n_blocks > 0) {
+        const int lb = n_blocks - 1;
+        const int pt0 = lb * kScanTB;
+        const int ntok = min(kScanTB, T - pt0);
+        const float* yb = ybuf + (size_t)(lb & 1) * kScanTB * NW * D;
+        for (int idx = tid; idx < ntok * D; idx += NT) {
+            int tok = idx / D, k = idx - tok * D;
+            float acc = 0.f;
+            for (int w = 0; w < NW; ++w) acc += yb[((size_t)tok * NW + w) * D + k];
+            a.y[(((size_t)b * T + pt0 + tok) * H + h) * D + k] = acc;
+        }
+    }
+    // final state
+    float* Sbh = a.S_out + (size_t)bh * m * D;
+#pragma unroll
+    for (int r = 0; r < RQ; ++r)
+        if (slot[r] < m) store_row_f32<D, false>(Sbh + (size_t)slot[r] * D, j, s[r]);
+}
+
+}  // namespace lattice

@@ -1,0 +1,86 @@
+"""The C-ABI library loads and exports every entry point include/lattice.h
+declares; host-side argument checks answer before anything reaches a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import orthogonal_update_recurrent_b200 as L
+from orthogonal_update_recurrent_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "lattice.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lattice_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("lattice_scan_fwd", "lattice_step", "lattice_readout", "lattice_get_device_status",
+              "lattice_status_string", "lattice_scan_fwd_impl", "lattice_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert lib.lattice_version() >= 100
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert lib.lattice_status_string(code)
+    assert lib.lattice_status_string(99) == b"unknown status"
+
+
+def _scan(lib, **kw):
+    a = dict(x=1 << 20, xdt=0, c=2 << 20, q=3 << 20, qdt=0, mu=4 << 20, eta=None, S0=5 << 20,
+             So=6 << 20, y=7 << 20, B=1, T=4, H=1, m=4, d=16, chunk=1, mode=0, impl=0)
+    a.update(kw)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return lib.lattice_scan_fwd_impl(v(a["x"]), a["xdt"], v(a["c"]), v(a["q"]), a["qdt"], v(a["mu"]),
+                                     v(a["eta"]), v(a["S0"]), v(a["So"]), v(a["y"]), a["B"], a["T"],
+                                     a["H"], a["m"], a["d"], a["chunk"], a["mode"], a["impl"], None)
+
+
+def test_argument_checks_return_before_launch(lib):
+    # Every case below fails validation, so no CUDA call is made (none could run here).
+    assert _scan(lib, x=None) == L.ERR_INVALID_ARG
+    assert _scan(lib, S0=None) == L.ERR_INVALID_ARG
+    assert _scan(lib, B=0) == L.ERR_INVALID_ARG
+    assert _scan(lib, T=-1) == L.ERR_INVALID_ARG
+    assert _scan(lib, chunk=0) == L.ERR_INVALID_ARG
+    assert _scan(lib, d=48) == L.ERR_UNSUPPORTED
+    assert _scan(lib, m=257) == L.ERR_UNSUPPORTED
+    assert _scan(lib, xdt=7) == L.ERR_INVALID_ARG
+    assert _scan(lib, mode=1) == L.ERR_UNSUPPORTED
+    assert _scan(lib, impl=9) == L.ERR_INVALID_ARG
+    assert _scan(lib, impl=2) == L.ERR_UNSUPPORTED          # tensor cores need chunk > 1
+    assert _scan(lib, chunk=64, impl=2) == L.ERR_UNSUPPORTED  # and bf16 x/q, m,d in {64,128}
+    assert _scan(lib, y=(1 << 20) + 64) == L.ERR_INVALID_ARG  # y overlaps x
+    assert _scan(lib, So=(5 << 20) + 16) == L.ERR_INVALID_ARG  # partial S0/S_out aliasing
+    assert _scan(lib, x=(1 << 20) + 4) == L.ERR_INVALID_ARG   # misaligned x
+    v = ctypes.c_void_p
+    assert lib.lattice_step(None, v(1 << 20), 0, v(2 << 20), v(3 << 20), 0, v(4 << 20), None,
+                            v(5 << 20), 1, 1, 4, 16, 0, None) == L.ERR_INVALID_ARG
+    assert lib.lattice_readout(v(1 << 20), v(2 << 20), 0, v(3 << 20), 1, 1, 4, 24,
+                               None) == L.ERR_UNSUPPORTED
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    x = torch.zeros(1, 2, 1, 16)
+    with pytest.raises(TypeError):
+        L.scan_fwd(x, torch.zeros(1, 2, 1, 4), torch.zeros(1, 2, 1, 4), torch.zeros(1, 2, 1),
+                   torch.zeros(1, 1, 4, 16))

@@ -1,0 +1,227 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Inputs come from lattice_inputs (seeded, shared with the oracle). The error
+metric is per (b,h) slice max|gpu - ref| / max|ref|, then the max over slices.
+Tolerances: 1e-4 for fp32 arithmetic paths (exact recurrence, CUDA-core
+chunked form, decode step, read-out) - the inputs are exactly representable,
+so the error is the kernel's fp32 rounding; 2e-2 for the tensor-core chunked
+path, whose matrix operands are rounded to bf16 while the state stays fp32.
+"""
+import numpy as np
+import pytest
+
+import lattice_inputs as LI
+import oracle
+from helpers import dev_inputs, s_err, y_err
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_TC = 2e-2
+
+
+@pytest.fixture(scope="module")
+def L():
+    import orthogonal_update_recurrent_b200 as L
+    from orthogonal_update_recurrent_b200 import build
+    build.build()
+    return L
+
+
+def run_gpu(L, inp, chunk, impl="auto", eta=None):
+    t = dev_inputs(inp)
+    y, S = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], eta=t["eta"] if eta is None else eta,
+                      chunk=chunk, impl=impl)
+    torch.cuda.synchronize()
+    L.device_status()
+    return y.cpu().numpy(), S.cpu().numpy()
+
+
+def run_oracle(inp, chunk):
+    y, S, _ = oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], eta=inp["eta"],
+                          chunk=chunk)
+    return y, S
+
+
+def small(name, **kw):
+    return LI.WORKLOADS[name].with_(**kw)
+
+
+# ----------------------------------------------------------- exact recurrence
+
+def test_exact_tiny_f32_full(L):
+    """The tiny fp32 workload at full size: B=1,H=1,T=256,m=16,d=32."""
+    w = LI.WORKLOADS["tiny_f32"]
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, 1)
+    yo, So = run_oracle(inp, 1)
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
+    np.testing.assert_allclose(np.linalg.norm(Sg, axis=-1), 1.0, atol=1e-5)
+
+
+@pytest.mark.parametrize("m,d", [(16, 16), (5, 32), (64, 64), (128, 128), (64, 128), (200, 64),
+                                 (256, 128)])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_exact_shapes(L, m, d, dt):
+    w = LI.Workload("t", B=2, T=37, H=3, m=m, d=d, x_dtype=dt, q_dtype=dt, seed=m * 7 + d)
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, 1)
+    yo, So = run_oracle(inp, 1)
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
+
+
+def test_exact_with_eta_and_edge_gates(L):
+    """eta given; mu = 0 and mu = 1 tokens; a zero-intensity token; duplicates."""
+    w = LI.Workload("t", B=2, T=41, H=2, m=32, d=64, x_dtype="f32", q_dtype="bf16",
+                    dup_frac=0.2, seed=5)
+    inp = LI.make_inputs(w)
+    rng = np.random.default_rng(0)
+    inp["eta"] = rng.uniform(0.2, 1.5, inp["mu"].shape).astype(np.float32)
+    inp["mu"][:, 3] = 0.0
+    inp["mu"][:, 4] = 1.0
+    inp["c"][:, 5] = 0.0
+    yg, Sg = run_gpu(L, inp, 1)
+    yo, So = run_oracle(inp, 1)
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
+
+
+def test_exact_identity_and_in_place(L):
+    """mu = 1, c = 0: the state does not move; S_out == S0 updates in place."""
+    w = LI.Workload("t", B=1, T=20, H=2, m=16, d=32, seed=9)
+    inp = LI.make_inputs(w)
+    inp["mu"][:] = 1.0
+    inp["c"][:] = 0.0
+    t = dev_inputs(inp)
+    S = t["S0"].clone()
+    y, S2 = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], S, S_out=S)
+    torch.cuda.synchronize()
+    assert S2.data_ptr() == S.data_ptr()
+    np.testing.assert_allclose(S.cpu().numpy(), inp["S0"], atol=2e-7)
+    yref = np.einsum("bthm,bhmd->bthd", inp["q"].astype(np.float64), inp["S0"].astype(np.float64))
+    assert y_err(y.cpu().numpy(), yref) <= TOL_F32
+
+
+def test_empty_sequence_copies_state(L):
+    w = LI.Workload("t", B=2, T=0, H=2, m=16, d=32, seed=1)
+    inp = LI.make_inputs(w)
+    t = dev_inputs(inp)
+    y, S = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(S.cpu().numpy(), inp["S0"])
+    assert y.numel() == 0
+
+
+@pytest.mark.parametrize("chunk,T1", [(1, 13), (64, 128)])
+def test_resume_is_bitwise(L, chunk, T1):
+    """scan(T1) then scan(T2) from the carried state equals scan(T1 + T2)."""
+    w = LI.Workload("t", B=2, T=200, H=2, m=64, d=64, seed=3)
+    inp = LI.make_inputs(w)
+    t = dev_inputs(inp)
+    y, S = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], chunk=chunk)
+    sl = lambda a, s: a[:, s].contiguous()
+    ya, Sa = L.scan_fwd(sl(t["x"], slice(0, T1)), sl(t["c"], slice(0, T1)), sl(t["q"], slice(0, T1)),
+                        sl(t["mu"], slice(0, T1)), t["S0"], chunk=chunk)
+    yb, Sb = L.scan_fwd(sl(t["x"], slice(T1, None)), sl(t["c"], slice(T1, None)),
+                        sl(t["q"], slice(T1, None)), sl(t["mu"], slice(T1, None)), Sa, chunk=chunk)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([ya, yb], 1), y)
+    assert torch.equal(Sb, S)
+
+
+def test_deterministic(L):
+    w = LI.Workload("t", B=2, T=100, H=4, m=128, d=128, seed=4)
+    t = dev_inputs(LI.make_inputs(w))
+    for chunk in (1, 64):
+        y1, S1 = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], chunk=chunk)
+        y2, S2 = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], chunk=chunk)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2) and torch.equal(S1, S2)
+
+
+# -------------------------------------------------- chunked (Eq. 17) CUDA cores
+
+@pytest.mark.parametrize("m,d,C", [(16, 32, 4), (64, 64, 64), (128, 128, 64), (64, 128, 16),
+                                   (48, 16, 8)])
+def test_chunked_simt(L, m, d, C):
+    w = LI.Workload("t", B=2, T=2 * C + C // 2 + 3, H=2, m=m, d=d, seed=m + d + C)
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, C, impl="simt")
+    yo, So = run_oracle(inp, C)
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
+
+
+# ------------------------------------------------------------- decode step
+
+@pytest.mark.parametrize("m,d", [(128, 128), (64, 64), (16, 32), (7, 16), (200, 128)])
+def test_step_matches_oracle_over_steps(L, m, d):
+    w = LI.WORKLOADS["decode"].with_(m=m, d=d)
+    B, H, n = 3, 5, 6
+    S0 = LI.make_decode_state(w, B=B, H=H)
+    st = LI.make_decode_steps(w, n, B=B, H=H)
+    S = torch.from_numpy(S0.copy()).cuda()
+    So = S0.astype(np.float64)
+    for k in range(n):
+        one = {key: st[key][k] for key in ("x", "q", "c", "mu")}
+        one["x_bits"] = None if st["x_bits"] is None else st["x_bits"][k]
+        one["q_bits"] = None if st["q_bits"] is None else st["q_bits"][k]
+        one["eta"] = None
+        t = dev_inputs(one)
+        y = L.step(S, t["x"], t["c"], t["q"], t["mu"])
+        yo, So, _ = oracle.step(So, one["x"], one["c"], one["q"], one["mu"])
+        torch.cuda.synchronize()
+        assert y_err(y.cpu().numpy()[:, None], yo[:, None]) <= TOL_F32
+    assert s_err(S.cpu().numpy(), So) <= TOL_F32
+
+
+def test_readout(L):
+    rng = np.random.default_rng(2)
+    for m, d in ((128, 128), (5, 16), (64, 32)):
+        S = rng.standard_normal((3, 4, m, d)).astype(np.float32)
+        q = rng.standard_normal((3, 4, m)).astype(np.float32)
+        y = L.readout(torch.from_numpy(S).cuda(), torch.from_numpy(q).cuda())
+        yo = oracle.readout(S, q)
+        torch.cuda.synchronize()
+        assert y_err(y.cpu().numpy()[:, None], yo[:, None]) <= TOL_F32
+
+
+# ------------------------------------- full-size workloads, sampled sequences
+
+FULL = [("small_train", [(0, 0), (3, 7), (2, 4)]),
+        ("mid_layer", [(0, 0), (7, 15), (4, 9)]),
+        ("long_ctx", [(0, 0), (0, 11)])]
+
+
+@pytest.mark.parametrize("name,pairs", FULL)
+def test_full_size_exact_sampled(L, name, pairs):
+    """Full-size workload on the GPU (the launch the benchmark times), sampled
+    (b,h) sequences recomputed by the oracle over the whole sequence."""
+    w = LI.WORKLOADS[name]
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, 1)
+    sub = LI.sample_heads(inp, pairs)
+    yo, So = run_oracle(sub, 1)
+    bs = [p[0] for p in pairs]
+    hs = [p[1] for p in pairs]
+    assert y_err(yg[bs, :, hs][:, :, None], yo) <= TOL_F32
+    assert s_err(Sg[bs, hs][:, None], So) <= TOL_F32
+
+
+@pytest.mark.parametrize("name,pairs", FULL)
+@pytest.mark.parametrize("impl", ["simt"])
+def test_full_size_chunked_sampled(L, name, pairs, impl):
+    """Full-size workload, chunk 64, against the oracle's Eq. 17 chunked form."""
+    w = LI.WORKLOADS[name]
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, w.chunk, impl=impl)
+    sub = LI.sample_heads(inp, pairs)
+    yo, So = run_oracle(sub, w.chunk)
+    bs = [p[0] for p in pairs]
+    hs = [p[1] for p in pairs]
+    tol = TOL_F32 if impl == "simt" else TOL_TC
+    assert y_err(yg[bs, :, hs][:, :, None], yo) <= tol
+    assert s_err(Sg[bs, hs][:, None], So) <= tol

@@ -218,10 +218,10 @@ def test_brute_force_projection_matrices():
 
 def test_chunk_size_one_is_the_exact_recurrence():
     """Appendix C / Appendix D: chunk size 1 is the exact recurrence. With the
-    mu^2 reading of the chunk normaliser the two forms agree to rounding, also
-    for non-unit initial slots."""
+    mu^2 reading of the chunk normaliser the two forms agree to rounding for
+    unit-norm initial slots (every state the exact recurrence produces)."""
     rng = _rng(9)
-    x, c, q, mu, S0 = _rand_inputs(rng, 2, 17, 3, 6, 7, unit=False)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 17, 3, 6, 7, unit=True)
     eta = rng.uniform(0.2, 1.2, mu.shape)
     y1, S1, _ = oracle.scan(x, c, q, mu, S0, eta=eta, chunk=1)
     y2, S2, _ = oracle.scan(x, c, q, mu, S0, eta=eta, chunk=1, form="matrix")
@@ -238,6 +238,34 @@ def test_chunk_size_one_is_the_exact_recurrence():
     for y, S in ((y2, S2), (y3, S3), (y4, S4)):
         np.testing.assert_allclose(y, y1, atol=1e-12)
         np.testing.assert_allclose(S, S1, atol=1e-12)
+
+
+def test_chunk_normaliser_keeps_the_chunk_start_norm():
+    """Appendix D listing (compress_chunk): the normaliser carries the
+    chunk-start norm, so the first token of a chunk - where Eq. 17 is exact -
+    leaves each slot with its chunk-start norm, unit or not; the exact
+    recurrence (§3.2) projects onto the unit sphere instead."""
+    rng = _rng(10)
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 1, 2, 5, 6, unit=False)
+    _, Sc, _ = oracle.scan(x, c, q, mu, S0, chunk=4)
+    np.testing.assert_allclose(np.linalg.norm(Sc, axis=-1), np.linalg.norm(S0, axis=-1), rtol=1e-12)
+    _, Se, _ = oracle.scan(x, c, q, mu, S0, chunk=1)
+    np.testing.assert_allclose(np.linalg.norm(Se, axis=-1), 1.0, rtol=1e-12)
+    # direction after the first token is the same in both forms
+    np.testing.assert_allclose(Sc / np.linalg.norm(Sc, axis=-1, keepdims=True), Se, atol=1e-12)
+
+
+def test_chunked_form_stays_bounded_on_the_training_shape():
+    """The chunk-normaliser reading keeps the chunked recurrence stable over a
+    whole small-training-shape sequence (2048 tokens, 32 chunks of 64): slot
+    norms stay O(1). The unit-sphere reading (1/sqrt(mu^2 n^2 + |Delta|^2))
+    overflows within a few chunks on the same inputs."""
+    import lattice_inputs as LI
+    inp = LI.make_inputs(LI.WORKLOADS["small_train"].with_(B=1, H=2))
+    y, S, deg = oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=64)
+    assert np.isfinite(y).all() and deg == 0
+    n = np.linalg.norm(S, axis=-1)
+    assert 0.1 < n.min() and n.max() < 10.0
 
 
 @pytest.mark.parametrize("C", [2, 4, 16, 64])
