@@ -125,6 +125,11 @@ lattice_status lattice_readout(const float *S, const void *q, lattice_dtype q_dt
  * the stream reports an error, else LATTICE_OK. */
 lattice_status lattice_get_device_status(void *stream);
 
+/* Name and description of the last CUDA error the library saw on this host
+ * thread when a call returned LATTICE_ERR_CUDA ("" if none). The text is
+ * owned by the library and stays valid until the next call on this thread. */
+const char *lattice_last_cuda_error(void);
+
 /* Static English text for a status code. */
 const char *lattice_status_string(lattice_status s);
 

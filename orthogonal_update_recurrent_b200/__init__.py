@@ -37,6 +37,8 @@ class LatticeError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
         msg = _lib.lattice_status_string(code).decode() if _lib is not None else str(code)
+        if code == ERR_CUDA and _lib is not None:
+            msg += " [" + _lib.lattice_last_cuda_error().decode() + "]"
         super().__init__(f"{what}: {msg} (status {code})")
 
 
@@ -60,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.lattice_status_string.restype = ctypes.c_char_p
         L.lattice_version.argtypes = []
         L.lattice_chunk_impl.argtypes = [i, i, i, i, i]
+        L.lattice_last_cuda_error.argtypes = []
+        L.lattice_last_cuda_error.restype = ctypes.c_char_p
         for f in ("lattice_scan_fwd", "lattice_scan_fwd_impl", "lattice_step", "lattice_readout",
                   "lattice_get_device_status", "lattice_version", "lattice_chunk_impl"):
             getattr(L, f).restype = ctypes.c_int

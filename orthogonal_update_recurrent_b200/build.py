@@ -16,7 +16,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
-    "-O3", "-lineinfo", "-std=c++17", "--use_fast_math",
+    "-O3", "-lineinfo", "-std=c++17",
     "-shared", "-Xcompiler", "-fPIC,-O2", "-cudart", "static",
     "-Xptxas", "-warn-spills",
 ]

@@ -1,12 +1,701 @@
-// chunk_tc.cuh -- tensor-core (tcgen05) chunked scan. Not built yet: every
-// chunked call runs the CUDA-core kernel.
+// chunk_tc.cuh -- tensor-core (tcgen05) chunked scan of the Lattice recurrence.
+//
+// Computes the chunked form, Eq. 17 of "Lattice: Learning to Efficiently
+// Compress the Memory" (§3.4.1 and Appendix B.1), chunk size C = 64: inside a
+// chunk every token's per-slot gate g and write coefficient kappa come from the
+// chunk-start state S0 (projection p = x . s0, normaliser of eq. beta_chunk with
+// the chunk-start norm as in the Appendix D listing), and the state follows the
+// diagonal-gated linear recurrence  s_i <- g_i s_i + kappa_i x.
+//
+// Chunk-parallel evaluation. Products of gates over a whole chunk reach 1e-58
+// on the paper-shaped workloads (small-norm slots get small or negative gates),
+// so nothing is ever divided by a product longer than one 16-token sub-chunk:
+//   y_t   = sum_i q_ti A_ti s0_i + sum_{j<=t} P_tj x_j,  A_t = prod_{l<=t} g_l
+//   P_tj  = sum_i QR_b(t)_i KD(j)_i           for j in sub-chunk b (16b..16b+15)
+//   QR_b(t) = q_t prod_{l=16b..t} g_l          (t >= 16b; plain products)
+//   KD(j)   = kappa_j / prod_{l=16b..j} g_l    (division inside one sub-chunk)
+//   S_C   = diag(A_C) S0 + sum_j (kappa_j prod_{l=j+1..C-1} g_l) x_j^T
+// with kappa_j prod_{l=j+1..C-1} g_l = KD(j) F_b, F_b = prod_{l>=16b} g_l.
+//
+// One CTA per (b, h) sequence. The fp32 state lives in tensor memory as
+// S = diag(sigma) T: the chunk decay diag(A_C) is folded into the per-slot scale
+// sigma, so the state-update GEMM accumulates straight onto T; rows whose
+// sigma*A_C drops below 2^-100 (the old state is then below fp32 resolution)
+// are rescaled in TMEM first, and T is renormalised when sigma leaves
+// [2^-32, 2^32]. The GEMMs that carry the state use hi+lo bf16 operand pairs,
+// so the carried state keeps close to fp32 accuracy over thousands of chunks.
+// Per chunk (bf16 operands in 128B-swizzled shared memory, fp32 TMEM accumulators):
+//   G1: D1  [m x C]  = (S0hi + S0lo) . X^T        projections x_t . s0_i
+//   G7: T   [m x d] += (KShi + KSlo)^T . X        state update
+//   G5: P   [C x 16] = QR_b . KD_b^T, b = 0..3     scores, one 16-column block each
+//   G4: Y^T [d x C]  = S0hi^T . QR_0^T            inter-chunk read-out
+//   G6: Y^T [d x C] += X^T . P_causal^T           intra-chunk read-out
+// Warp roles (576 threads): warps 0-15 are workers, warp 4*sb + q owning TMEM
+// lane quadrant q (slots 32q..32q+31) and sub-chunk sb: it computes the gates of
+// tokens 16sb..16sb+15 for its 32 slots (so the 64-token gate recurrence runs as
+// four independent 16-token pieces, tied together by four sub-chunk products per
+// slot exchanged through shared memory), converts state columns
+// sb*d/4..(sb+1)*d/4, masks score columns 16sb..16sb+15 and stores y for tokens
+// 16sb..16sb+15. Warp 16 = TMA producer, MMA issuer and TMEM owner; warp 17 =
+// per-token |x|^2, mu, eta. Every mbarrier wait is bounded by %globaltimer: on
+// timeout the kernel sets the device status word, skips the remaining work and
+// still meets every named barrier.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "scan_simt.cuh"
+#include "tc_ptx.cuh"
 
 namespace lattice {
 
-inline bool chunk_tc_supported(int, int, int, bool, bool) { return false; }
-inline cudaError_t launch_chunk_tc(const ScanArgs&, int, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int kTcC = 64;            // chunk size of the tensor-core path
+constexpr int kTcSub = 16;          // sub-chunk: the longest product ever divided by
+constexpr int kTcWorkWarps = 16;   // 4 lane quadrants x 4 sub-chunks
+constexpr int kTcThreads = 32 * (kTcWorkWarps + 2);  // + control warp + aux warp
+constexpr uint64_t kTcWaitNs = 2000000000ull;  // 2 s bound on any single wait
+
+inline bool chunk_tc_supported(int m, int d, int chunk, bool x_bf16, bool q_bf16) {
+    return chunk == kTcC && x_bf16 && q_bf16 && (m == 64 || m == 128) && (d == 64 || d == 128);
+}
+
+template <int MS, int DS>
+struct TcLayout {
+    static constexpr int NST = 2;                         // X stages
+    static constexpr uint32_t X_STAGE = DS * 128;         // DS/64 blocks x 64 rows x 128 B
+    static constexpr uint32_t S0_TILE = MS * DS * 2;      // DS/64 blocks x m rows x 128 B
+    static constexpr uint32_t ROW_TILE = MS * 128;        // [m][64] bf16, one 128 B row per slot
+    static constexpr uint32_t X_OFF = 0;
+    static constexpr uint32_t S0HI_OFF = X_OFF + NST * X_STAGE;
+    static constexpr uint32_t S0LO_OFF = S0HI_OFF + S0_TILE;
+    static constexpr uint32_t QR_OFF = S0LO_OFF + S0_TILE;        // QR_0..QR_3
+    static constexpr uint32_t KD_OFF = QR_OFF + 4 * ROW_TILE;
+    static constexpr uint32_t KSHI_OFF = KD_OFF + ROW_TILE;
+    static constexpr uint32_t KSLO_OFF = KSHI_OFF + ROW_TILE;
+    static constexpr uint32_t P_OFF = QR_OFF + 3 * ROW_TILE;      // [C][128 B], reuses QR_3
+    static constexpr uint32_t AUX_OFF = KSLO_OFF + ROW_TILE;      // [NST][C] float4
+    static constexpr uint32_t GSUB_OFF = AUX_OFF + NST * kTcC * 16;   // [4][m] float
+    static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * MS * 4;        // [4][m] float
+    static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * MS * 4;
+    static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * 8;
+    static constexpr uint32_t BYTES = MISC_OFF + 64;
+    static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;          // room to align the base
+    static_assert(kTcC * 128 <= ROW_TILE, "P must fit in the QR_3 tile");
+    // TMEM columns (fp32): state T | D1 | P | Y^T
+    static constexpr uint32_t T_COL = 0;
+    static constexpr uint32_t D1_COL = DS;
+    static constexpr uint32_t P_COL = DS + kTcC;
+    static constexpr uint32_t Y_COL = DS + 2 * kTcC;
+    static constexpr uint32_t TMEM_COLS = (DS + 3 * kTcC) <= 256 ? 256 : 512;
+    static constexpr uint32_t TX_BYTES = X_STAGE;
+};
+
+struct TcMaps {
+    CUtensorMap x, q, c;
+};
+
+// Bounded wait: true when the phase completed; false (and the abort flag set)
+// when the bound elapsed or another thread already aborted.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+    if (*abort) return false;
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    for (;;) {
+        if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;  // sleep <= 20 us per try
+        if (*abort) return false;
+        if (ptx::globaltimer() - t0 > kTcWaitNs) {
+            *abort = 1u;
+            flag_timeout();
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag: used at exit so that no TMA write
+// into shared memory is still in flight when the CTA retires.
+__device__ __forceinline__ void tc_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = ptx::globaltimer();
+    for (;;) {
+        if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return;
+        if (ptx::globaltimer() - t0 > kTcWaitNs) {
+            flag_timeout();
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* v) {
+    uint4 u;
+    u.x = ptx::pack_bf16x2(v[0], v[1]);
+    u.y = ptx::pack_bf16x2(v[2], v[3]);
+    u.z = ptx::pack_bf16x2(v[4], v[5]);
+    u.w = ptx::pack_bf16x2(v[6], v[7]);
+    return u;
+}
+
+// hi = bf16(v), lo = bf16(v - hi): two bf16 tiles whose sum carries ~16 mantissa bits.
+__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
+    float h[8], l[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+        l[e] = v[e] - h[e];
+    }
+    hi = pack8(h);
+    lo = pack8(l);
+}
+
+// 18 warps are charged as 20 for registers (warps are allocated in groups of
+// four), so the launch bound caps the kernel at 96 registers per thread.
+template <int MS, int DS>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    chunk_tc_kernel(const __grid_constant__ TcMaps maps, ScanArgs a) {
+    using Lay = TcLayout<MS, DS>;
+    constexpr int NSUB = kTcC / kTcSub;   // 4 sub-chunks, one per worker group
+    constexpr int DCOL = DS / NSUB;       // state columns converted by each group
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+    const int T = a.T, H = a.H;
+    const int nch = (T + kTcC - 1) / kTcC;
+
+    const uint32_t bar_full0 = sbase + Lay::BAR_OFF;          // [2]
+    const uint32_t bar_free0 = sbase + Lay::BAR_OFF + 16;     // [2]
+    const uint32_t bar_mma = sbase + Lay::BAR_OFF + 32;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+    volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 4);
+    float4* aux = reinterpret_cast<float4*>(smem + Lay::AUX_OFF);
+    float* gsub = reinterpret_cast<float*>(smem + Lay::GSUB_OFF);   // [NSUB][MS] sub-chunk products
+    float* tsqp = reinterpret_cast<float*>(smem + Lay::TSQ_OFF);    // [NSUB][MS] partial |s|^2
+
+    // named barriers: ids and participant counts (16 worker warps, control warp, aux warp)
+    constexpr uint32_t BAR_S = 1, BAR_G = 2, BAR_A = 3, BAR_B = 4;
+    constexpr uint32_t N_S = kTcThreads;           // everyone
+    constexpr uint32_t N_G = 32 * kTcWorkWarps;    // workers
+    constexpr uint32_t N_A = N_G + 32;             // workers + control
+    constexpr uint32_t N_B = N_G + 64;             // workers + control + aux
+    constexpr int CTRL = kTcWorkWarps, AUXW = kTcWorkWarps + 1;
+
+    if (warp == CTRL) {
+        if (lane == 0) {
+            ptx::mbar_init(bar_full0, 1);
+            ptx::mbar_init(bar_full0 + 8, 1);
+            ptx::mbar_init(bar_free0, 1);
+            ptx::mbar_init(bar_free0 + 8, 1);
+            ptx::mbar_init(bar_mma, 1);
+            *abort = 0u;
+            ptx::fence_mbar_init();
+            ptx::prefetch_tensormap(&maps.x);
+            ptx::prefetch_tensormap(&maps.q);
+            ptx::prefetch_tensormap(&maps.c);
+        }
+        __syncwarp();
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), Lay::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == CTRL) {
+        // ------------------------------------------------------------ control
+        int last_tma[2] = {-1, -1};  // last chunk loaded into each stage
+        auto issue_tma = [&](int k) {  // X of chunk k -> stage k % 2, q and c of chunk k -> L2
+            const int s = k & 1;
+            last_tma[s] = k;
+            const uint32_t bar = bar_full0 + 8 * s;
+            ptx::mbar_arrive_expect_tx(bar, Lay::TX_BYTES);
+#pragma unroll
+            for (int kb = 0; kb < DS / 64; ++kb)
+                ptx::tma_load_4d(sbase + Lay::X_OFF + s * Lay::X_STAGE + kb * (64 * 128), &maps.x,
+                                 bar, kb * 64, h, k * kTcC, b);
+            ptx::tma_prefetch_l2_4d(&maps.q, 0, h, k * kTcC, b);
+            ptx::tma_prefetch_l2_4d(&maps.c, 0, h, k * kTcC, b);
+        };
+        const uint32_t idesc_g1 = ptx::idesc_bf16(MS, kTcC, 0, 0);
+        const uint32_t idesc_g7 = ptx::idesc_bf16(MS, DS, 0, 1);
+        const uint32_t idesc_g5 = ptx::idesc_bf16(kTcC, kTcSub, 1, 1);
+        const uint32_t idesc_g4 = ptx::idesc_bf16(DS, kTcC, 1, 1);
+        const uint32_t idesc_g6 = ptx::idesc_bf16(DS, kTcC, 1, 0);
+        const uint32_t s0hi = sbase + Lay::S0HI_OFF, s0lo = sbase + Lay::S0LO_OFF,
+                       qr = sbase + Lay::QR_OFF, kd = sbase + Lay::KD_OFF,
+                       kshi = sbase + Lay::KSHI_OFF, kslo = sbase + Lay::KSLO_OFF,
+                       pp = sbase + Lay::P_OFF;
+        auto g1 = [&](int k) {  // D1 = (S0hi + S0lo) . X_k^T   (M = m, N = C, K = d)
+            const uint32_t xs = sbase + Lay::X_OFF + (k & 1) * Lay::X_STAGE;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t s0 = part ? s0lo : s0hi;
+#pragma unroll
+                for (int kk = 0; kk < DS / 16; ++kk) {
+                    const uint32_t kb = kk >> 2, ko = (kk & 3) * 32;
+                    ptx::mma_bf16(tmem + Lay::D1_COL,
+                                  ptx::sdesc_sw128(s0 + kb * MS * 128 + ko, 16, 1024),
+                                  ptx::sdesc_sw128(xs + kb * 64 * 128 + ko, 16, 1024), idesc_g1,
+                                  (part | kk) != 0);
+                }
+            }
+        };
+        if (lane == 0 && nch > 0) {
+            issue_tma(0);
+            if (nch > 1) issue_tma(1);
+        }
+        __syncwarp();
+        ptx::named_bar(BAR_S, N_S);  // S0 operand and aux[0] ready
+        ptx::tc_fence_after();
+        if (lane == 0) {
+            if (tc_wait(bar_full0, 0, abort)) g1(0);
+            ptx::mma_commit(bar_mma);
+        }
+        __syncwarp();
+        for (int k = 0; k < nch; ++k) {
+            const int s = k & 1;
+            const uint32_t xs = sbase + Lay::X_OFF + s * Lay::X_STAGE;
+            ptx::named_bar(BAR_A, N_A);  // QR, KD, KS written; T prescaled; D1 and Y^T drained
+            ptx::tc_fence_after();
+            if (lane == 0) {
+                if (!*abort) {
+                    // G7: T += (KShi + KSlo)^T . X  (M = m, N = d, K = C); A K-major, B MN-major
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int kk = 0; kk < kTcC / 16; ++kk)
+                            ptx::mma_bf16(tmem + Lay::T_COL,
+                                          ptx::sdesc_sw128((part ? kslo : kshi) + kk * 32, 16, 1024),
+                                          ptx::sdesc_sw128(xs + kk * 2048, 64 * 128, 1024), idesc_g7, 1);
+                    // G5: P[:, 16b..16b+15] = QR_b . KD_b^T  (M = C, N = 16, K = m); both MN-major
+#pragma unroll
+                    for (int sb = 0; sb < NSUB; ++sb)
+#pragma unroll
+                        for (int kk = 0; kk < MS / 16; ++kk)
+                            ptx::mma_bf16(tmem + Lay::P_COL + sb * kTcSub,
+                                          ptx::sdesc_sw128(qr + sb * Lay::ROW_TILE + kk * 2048, MS * 128, 1024),
+                                          ptx::sdesc_sw128(kd + sb * (kTcSub * 2) + kk * 2048, MS * 128, 1024),
+                                          idesc_g5, kk > 0);
+                    // G4: Y^T = S0hi^T . QR_0^T  (M = d, N = C, K = m); both MN-major
+#pragma unroll
+                    for (int kk = 0; kk < MS / 16; ++kk)
+                        ptx::mma_bf16(tmem + Lay::Y_COL, ptx::sdesc_sw128(s0hi + kk * 2048, MS * 128, 1024),
+                                      ptx::sdesc_sw128(qr + kk * 2048, MS * 128, 1024), idesc_g4, kk > 0);
+                }
+                ptx::mma_commit(bar_mma);
+            }
+            __syncwarp();
+            ptx::named_bar(BAR_B, N_B);  // next S0 operand, masked P, aux[k+1] ready
+            ptx::tc_fence_after();
+            if (lane == 0) {
+                if (!*abort) {
+                    // G6: Y^T += X^T . P^T  (M = d, N = C, K = C); A MN-major, B K-major
+#pragma unroll
+                    for (int kk = 0; kk < kTcC / 16; ++kk)
+                        ptx::mma_bf16(tmem + Lay::Y_COL, ptx::sdesc_sw128(xs + kk * 2048, 64 * 128, 1024),
+                                      ptx::sdesc_sw128(pp + kk * 32, 16, 1024), idesc_g6, 1);
+                }
+                ptx::mma_commit(bar_free0 + 8 * s);
+                if (k + 1 < nch && tc_wait(bar_full0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1, abort))
+                    g1(k + 1);
+                ptx::mma_commit(bar_mma);
+                // stage s is free once G6 of chunk k has completed
+                if (k + 2 < nch && tc_wait(bar_free0 + 8 * s, (k >> 1) & 1, abort)) issue_tma(k + 2);
+            }
+            __syncwarp();
+        }
+        // drain: the last commit covers every MMA; wait for it before TMEM goes away,
+        // and for every TMA load still in flight before shared memory goes away
+        if (lane == 0) {
+            tc_wait(bar_mma, (2 * nch) & 1, abort);
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+                if (last_tma[s] >= 0) tc_drain(bar_full0 + 8 * s, (last_tma[s] >> 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == AUXW) {
+        // ------------------------------------------------------------ aux:
+        // per-token {mu, eta, |x|^2, mu^2} of chunk k into aux[k % 2]
+        auto aux_chunk = [&](int k) {
+            const int s = k & 1;
+            float mu2[2], eta2[2];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {  // global loads first, X wait second
+                const int t = k * kTcC + lane + 32 * half;
+                mu2[half] = 0.f;
+                eta2[half] = 1.f;
+                if (t < T) {
+                    const size_t bth = ((size_t)b * T + t) * H + h;
+                    mu2[half] = __ldg(a.mu + bth);
+                    if (a.eta) eta2[half] = __ldg(a.eta + bth);
+                }
+            }
+            const bool ok = tc_wait(bar_full0 + 8 * s, (k >> 1) & 1, abort);
+            const uint8_t* xs = smem + Lay::X_OFF + s * Lay::X_STAGE;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int tau = lane + 32 * half;
+                float xx = 0.f;
+                if (ok) {
+#pragma unroll
+                    for (int kb = 0; kb < DS / 64; ++kb)
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) {
+                            // any order sums the row; rotating by the row spreads lanes over banks
+                            const int pc = (ch + tau) & 7;
+                            uint4 v = *reinterpret_cast<const uint4*>(xs + kb * (64 * 128) + tau * 128 + pc * 16);
+                            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+                                xx = fmaf(lo, lo, xx);
+                                xx = fmaf(hi, hi, xx);
+                            }
+                        }
+                }
+                const float mu = mu2[half];
+                aux[s * kTcC + tau] = make_float4(mu, eta2[half], xx, mu * mu);
+            }
+        };
+        if (nch > 0) aux_chunk(0);
+        ptx::named_bar(BAR_S, N_S);
+        for (int k = 0; k < nch; ++k) {
+            if (k + 1 < nch) aux_chunk(k + 1);
+            ptx::named_bar(BAR_B, N_B);
+        }
+    } else {
+        // ------------------------------------------------------------ workers
+        // warp = 4 * sb + q4: TMEM lane quadrant q4, sub-chunk / column block sb
+        const int q4 = warp & 3, sb = warp >> 2;
+        const bool active = (MS == 128) || (lane < 16);
+        const int i = (MS == 128) ? (32 * q4 + lane) : (16 * q4 + (lane & 15));  // slot
+        const uint32_t lane_base = uint32_t(32 * q4) << 16;
+        // y column in the Y^T accumulator (M = d) and P row (M = 64: lanes 0-15 per quadrant)
+        const bool ycol_ok = (DS == 128) || (lane < 16);
+        const int kcol = (DS == 128) ? (32 * q4 + lane) : (16 * q4 + lane);
+        const bool prow_ok = lane < 16;
+        const int tau_row = 16 * q4 + lane;
+        uint8_t* s0hi = smem + Lay::S0HI_OFF;
+        uint8_t* s0lo = smem + Lay::S0LO_OFF;
+        uint8_t* qr = smem + Lay::QR_OFF;
+        uint8_t* kd = smem + Lay::KD_OFF;
+        uint8_t* kshi = smem + Lay::KSHI_OFF;
+        uint8_t* kslo = smem + Lay::KSLO_OFF;
+        uint8_t* ps = smem + Lay::P_OFF;
+
+        // a block of DCOL state columns starting at col0 -> hi/lo bf16 operand rows
+        auto store_s0 = [&](int col0, const float* v) {
+            const int kb = col0 >> 6;
+#pragma unroll
+            for (int ch = 0; ch < DCOL / 8; ++ch) {
+                uint4 hi, lo;
+                split8(v + 8 * ch, hi, lo);
+                const uint32_t off = kb * Lay::ROW_TILE + ptx::sw128_chunk(i, ((col0 & 63) >> 3) + ch);
+                *reinterpret_cast<uint4*>(s0hi + off) = hi;
+                *reinterpret_cast<uint4*>(s0lo + off) = lo;
+            }
+        };
+        // q and c of this group's 16 tokens of chunk k: coalesced over the slots
+        auto load_qc = [&](int k, float* qv, float* cv) {
+            const int t0 = k * kTcC + sb * kTcSub;
+            const size_t e0 = (((size_t)b * T + t0) * H + h) * MS + i;
+            const uint16_t* qp = static_cast<const uint16_t*>(a.q) + e0;
+            const float* cp = a.c + e0;
+            const int stride = H * MS;
+            const int nvalid = active ? min(kTcSub, T - t0) : 0;
+#pragma unroll
+            for (int u = 0; u < kTcSub; ++u) {
+                qv[u] = 0.f;
+                cv[u] = 0.f;
+                if (u < nvalid) {
+                    qv[u] = __uint_as_float(uint32_t(__ldg(qp + u * stride)) << 16);
+                    cv[u] = __ldg(cp + u * stride);
+                }
+            }
+        };
+        auto store_y = [&](int kc) {  // 16 tokens of chunk kc from the Y^T accumulator
+            uint32_t yv[kTcSub];
+            ptx::tmem_ld16(tmem + lane_base + Lay::Y_COL + sb * kTcSub, yv);
+            ptx::tmem_wait_ld();
+            if (!ycol_ok || *abort) return;
+            const int t0 = kc * kTcC + sb * kTcSub;
+            float* yb = a.y + (((size_t)b * T + t0) * H + h) * DS + kcol;
+            const size_t stride = (size_t)H * DS;
+#pragma unroll
+            for (int u = 0; u < kTcSub; ++u)
+                if (t0 + u < T) yb[u * stride] = __uint_as_float(yv[u]);
+        };
+
+        // initial state: T = S0 (sigma = 1), operand, partial norms; this group's DCOL columns
+        float sigma = 1.f;
+        {
+            const float* S0g = a.S0 + ((size_t)bh * MS + i) * DS + sb * DCOL;
+            float v[DCOL];
+            uint32_t r[DCOL];
+            float ns = 0.f;
+#pragma unroll
+            for (int e = 0; e < DCOL; e += 4) {
+                float4 t4 = active ? *reinterpret_cast<const float4*>(S0g + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[e] = t4.x; v[e + 1] = t4.y; v[e + 2] = t4.z; v[e + 3] = t4.w;
+            }
+#pragma unroll
+            for (int e = 0; e < DCOL; ++e) {
+                ns = fmaf(v[e], v[e], ns);
+                r[e] = __float_as_uint(v[e]);
+            }
+            ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+            ptx::tmem_wait_st();
+            if (active) {
+                store_s0(sb * DCOL, v);
+                tsqp[sb * MS + i] = ns;
+            }
+        }
+        float qv[kTcSub], cv[kTcSub];
+        if (nch > 0) load_qc(0, qv, cv);
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::named_bar(BAR_S, N_S);
+        float nsq = 0.f;
+        if (active)
+#pragma unroll
+            for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+
+        for (int k = 0; k < nch; ++k) {
+            const int s = k & 1;
+            // ---- phase A: gates of this group's 16 tokens (needs D1 = S0 . X_k^T)
+            tc_wait(bar_mma, 0, abort);  // completion #2k: G1_k and (k > 0) G6_{k-1}
+            ptx::tc_fence_after();
+            if (k > 0) store_y(k - 1);
+            uint32_t pr[kTcSub];
+            ptx::tmem_ld16(tmem + lane_base + Lay::D1_COL + sb * kTcSub, pr);
+            ptx::tmem_wait_ld();
+            const float n = sqrtf(nsq);
+            const float inv_n = 1.f / n, inv_n2 = 1.f / nsq;
+            const float4* ax = aux + s * kTcC + sb * kTcSub;
+            float gv[kTcSub], kdv[kTcSub], base[kTcSub];
+            float R = 1.f;
+#pragma unroll
+            for (int u = 0; u < kTcSub; ++u) {
+                const float4 z = ax[u];  // mu, eta, |x|^2, mu^2
+                const float p = __uint_as_float(pr[u]);
+                const float av = z.y * cv[u] * inv_n;              // eta c / n
+                const float r = p * inv_n2;                        // p / n^2
+                const float perp2 = fmaxf(fmaf(-p, r, z.z), 0.f);  // |x_perp|^2
+                const float den = fmaf(av * av, perp2, z.w * nsq);
+                const bool ok = den > 0.f;
+                const float bn = ok ? n * ptx::rsqrt_nr(den) : 0.f;  // n / sqrt(den)
+                const float g = ok ? bn * fmaf(-av, r, z.x) : 1.f;
+                gv[u] = g;
+                kdv[u] = bn * av;                                   // kappa for now
+                R *= g;
+                base[u] = qv[u] * R;                                // q_t prod_{16sb..t} g
+            }
+            if (active) gsub[sb * MS + i] = R;
+            // KD(t) = kappa_t / prod_{16sb..t} g: one reciprocal, then a backward product
+            {
+                float inv = ptx::rcp_nr(copysignf(fmaxf(fabsf(R), 1e-37f), R));
+#pragma unroll
+                for (int u = kTcSub - 1; u >= 0; --u) {
+                    kdv[u] *= inv;
+                    inv *= gv[u];
+                }
+            }
+            if (active) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int g8 = 2 * sb + hh;
+                    *reinterpret_cast<uint4*>(qr + sb * Lay::ROW_TILE + ptx::sw128_chunk(i, g8)) =
+                        pack8(base + 8 * hh);
+                    *reinterpret_cast<uint4*>(kd + ptx::sw128_chunk(i, g8)) = pack8(kdv + 8 * hh);
+                }
+            }
+            ptx::named_bar(BAR_G, N_G);  // all four sub-chunk products of every slot known
+            float G[NSUB];
+#pragma unroll
+            for (int g = 0; g < NSUB; ++g) G[g] = active ? gsub[g * MS + i] : 1.f;
+            // query operands of the earlier sub-chunks' key blocks (plain products), zeros
+            // for the later ones; then the state-update coefficients of this group's tokens
+            float F = 1.f, AC = 1.f;   // prod_{c >= sb} G_c, prod_c G_c
+#pragma unroll
+            for (int g = NSUB - 1; g >= 0; --g) {
+                AC *= G[g];
+                if (g >= sb) F *= G[g];
+            }
+            const float sig_c = sigma * AC;  // sigma * A_C
+            const bool pre = !(fabsf(sig_c) >= 7.8886091e-31f);  // 2^-100, or not finite
+            const float inv_sig = pre ? 1.f : 1.f / sig_c;
+            if (active) {
+#pragma unroll
+                for (int bb = 0; bb < NSUB; ++bb) {
+                    if (bb == sb) continue;
+                    float cgb = 1.f;  // prod_{c=bb..sb-1} G_c
+#pragma unroll
+                    for (int g = 0; g < NSUB; ++g)
+                        if (g >= bb && g < sb) cgb *= G[g];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] = bb < sb ? base[8 * hh + e] * cgb : 0.f;
+                        *reinterpret_cast<uint4*>(qr + bb * Lay::ROW_TILE + ptx::sw128_chunk(i, 2 * sb + hh)) =
+                            pack8(v);
+                    }
+                }
+                const float ksc = F * inv_sig;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = kdv[8 * hh + e] * ksc;
+                    uint4 hi, lo;
+                    split8(v, hi, lo);
+                    *reinterpret_cast<uint4*>(kshi + ptx::sw128_chunk(i, 2 * sb + hh)) = hi;
+                    *reinterpret_cast<uint4*>(kslo + ptx::sw128_chunk(i, 2 * sb + hh)) = lo;
+                }
+            }
+            // rows whose old state fell below fp32 resolution: T <- sigma A_C T, sigma = 1
+            if (__any_sync(0xffffffffu, pre && active)) {
+                const float sc = (pre && active) ? (isfinite(sig_c) ? sig_c : 0.f) : 1.f;
+                uint32_t r[DCOL];
+                ptx::tmem_ld<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < DCOL; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * sc);
+                ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+                ptx::tmem_wait_st();
+            }
+            sigma = pre ? 1.f : sig_c;
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::named_bar(BAR_A, N_A);
+
+            // ---- phase B: state after the chunk (S = sigma T'), masked scores
+            tc_wait(bar_mma, 1, abort);  // completion #2k+1 (G7, G5, G4)
+            ptx::tc_fence_after();
+            const bool renorm = !(fabsf(sigma) >= 2.3283064e-10f && fabsf(sigma) <= 4.2949673e9f);
+            const bool any_renorm = __any_sync(0xffffffffu, renorm && active);  // tcgen05.st is warp-collective
+            {
+                uint32_t r[DCOL];
+                float v[DCOL];
+                ptx::tmem_ld<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+                ptx::tmem_wait_ld();
+                float ts = 0.f;
+#pragma unroll
+                for (int e = 0; e < DCOL; ++e) {
+                    v[e] = __uint_as_float(r[e]) * sigma;  // true state
+                    ts = fmaf(v[e], v[e], ts);
+                    if (renorm) r[e] = __float_as_uint(v[e]);
+                }
+                if (any_renorm) {
+                    ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+                    ptx::tmem_wait_st();
+                }
+                if (active) {
+                    tsqp[sb * MS + i] = ts;
+                    if (k + 1 == nch) {
+                        float* So = a.S_out + ((size_t)bh * MS + i) * DS + sb * DCOL;
+#pragma unroll
+                        for (int e = 0; e < DCOL; e += 4)
+                            *reinterpret_cast<float4*>(So + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    } else {
+                        store_s0(sb * DCOL, v);
+                    }
+                }
+            }
+            if (renorm) sigma = 1.f;
+            {   // causal mask of P: this group's 16 score columns of row tau_row
+                uint32_t r[kTcSub];
+                ptx::tmem_ld16(tmem + lane_base + Lay::P_COL + sb * kTcSub, r);
+                ptx::tmem_wait_ld();
+                if (prow_ok) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = sb * kTcSub + 8 * hh + e;
+                            v[e] = (j <= tau_row) ? __uint_as_float(r[8 * hh + e]) : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(ps + ptx::sw128_chunk(tau_row, 2 * sb + hh)) = pack8(v);
+                    }
+                }
+            }
+            if (k + 1 < nch) load_qc(k + 1, qv, cv);
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::named_bar(BAR_B, N_B);
+            nsq = 0.f;
+            if (active)
+#pragma unroll
+                for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+        }
+        if (nch > 0) {  // read-out of the last chunk
+            tc_wait(bar_mma, 0, abort);  // completion #2nch: G6 of the last chunk
+            ptx::tc_fence_after();
+            store_y(nch - 1);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == CTRL) ptx::tmem_dealloc(tmem, Lay::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------- host side
+
+inline PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 4-D map over [B][T][H][inner] (innermost first: inner, H, T, B), box {box0, 1, C, 1}.
+inline bool make_map_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize,
+                        int inner, int H, int T, int B, int box0, bool swizzle) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)inner * esize, (cuuint64_t)inner * esize * H,
+                             (cuuint64_t)inner * esize * H * T};
+    cuuint32_t box[4] = {(cuuint32_t)box0, 1, (cuuint32_t)kTcC, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MS, int DS>
+cudaError_t launch_chunk_tc_t(const ScanArgs& a, cudaStream_t st) {
+    using Lay = TcLayout<MS, DS>;
+    TcMaps maps;
+    if (!make_map_4d(&maps.x, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DS, a.H, a.T, a.B, 64, true) ||
+        !make_map_4d(&maps.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, MS, a.H, a.T, a.B, MS, false) ||
+        !make_map_4d(&maps.c, a.c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, MS, a.H, a.T, a.B, MS, false))
+        return cudaErrorInvalidValue;
+    auto k = chunk_tc_kernel<MS, DS>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Lay::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    k<<<a.B * a.H, kTcThreads, Lay::SMEM_ALLOC, st>>>(maps, a);
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_chunk_tc(const ScanArgs& a, int d, cudaStream_t st) {
+    if (a.m == 128 && d == 128) return launch_chunk_tc_t<128, 128>(a, st);
+    if (a.m == 128 && d == 64) return launch_chunk_tc_t<128, 64>(a, st);
+    if (a.m == 64 && d == 128) return launch_chunk_tc_t<64, 128>(a, st);
+    if (a.m == 64 && d == 64) return launch_chunk_tc_t<64, 64>(a, st);
+    return cudaErrorNotSupported;
+}
 
 }  // namespace lattice

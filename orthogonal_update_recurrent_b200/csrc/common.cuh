@@ -131,18 +131,24 @@ __device__ __forceinline__ float octet_sum(float v) {
 //   (Pythagoras: the write is orthogonal to s_ref). The result is scaled to norm
 //   `target` (1 for the exact recurrence's unit sphere, |s0| for the chunked
 //   form's normaliser). Zero-norm updates keep the slot.
+// PRECISE selects correctly rounded reciprocal square root and division. The
+// chunked form carries each slot's norm from chunk to chunk without restoring
+// it, so a systematic one-ulp bias in the normaliser accumulates linearly over
+// the sequence (about 6e-3 after 65536 tokens); the exact recurrence projects
+// onto the unit sphere every token and can use the fast approximations.
+template <bool PRECISE>
 __device__ __forceinline__ void update_coefs(float n2, float p, float xx, float c, float mu,
                                              float eta, float target, float& alpha,
                                              float& gamma) {
     bool ok = n2 > 0.f;
     float n2s = ok ? n2 : 1.f;
-    float inv_n = rsqrtf(n2s);
-    float r = p / n2s;                      // p / n^2
+    float inv_n = PRECISE ? __frsqrt_rn(n2s) : rsqrtf(n2s);
+    float r = PRECISE ? __fdiv_rn(p, n2s) : __fdividef(p, n2s);  // p / n^2
     float a = eta * c * inv_n;              // eta c / n
     float perp2 = fmaxf(fmaf(-p, r, xx), 0.f);  // |x_perp|^2
     float w2 = fmaf(a * a, perp2, mu * mu * n2s);
     ok = ok && (w2 > 0.f);
-    float iw = rsqrtf(ok ? w2 : 1.f) * target;
+    float iw = (PRECISE ? __frsqrt_rn(ok ? w2 : 1.f) : rsqrtf(ok ? w2 : 1.f)) * target;
     alpha = ok ? fmaf(-a, r, mu) * iw : 1.f;
     gamma = ok ? a * iw : 0.f;
 }

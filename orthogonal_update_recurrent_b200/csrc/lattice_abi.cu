@@ -2,6 +2,7 @@
 // include/lattice.h): argument checks, kernel choice and launches.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 
 #include "../../include/lattice.h"
 #include "common.cuh"
@@ -27,8 +28,16 @@ bool dtype_ok(lattice_dtype t) { return t == LATTICE_F32 || t == LATTICE_BF16; }
 size_t dsize(lattice_dtype t) { return t == LATTICE_BF16 ? 2 : 4; }
 bool d_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
+thread_local char g_last_error[256] = "";
+
+lattice_status cuda_fail(cudaError_t e) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return LATTICE_ERR_CUDA;
+}
+
 lattice_status launch_status() {
-    return cudaGetLastError() == cudaSuccess ? LATTICE_OK : LATTICE_ERR_CUDA;
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
 }
 
 // ---- exact / chunked CUDA-core scan
@@ -36,9 +45,8 @@ template <int D, int RQ, bool CH>
 lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
     size_t smem = scan_smem_bytes<D>(a.m, nw);
     auto k = scan_simt_kernel<D, RQ, CH>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return LATTICE_ERR_CUDA;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e);
     k<<<a.B * a.H, nw * 32, smem, st>>>(a);
     return launch_status();
 }
@@ -149,8 +157,10 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
     if (S0 != S_out && overlap(sS0, sSo)) return LATTICE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (T == 0) {
-        if (S0 != S_out && cudaMemcpyAsync(S_out, S0, nS, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-            return LATTICE_ERR_CUDA;
+        if (S0 != S_out) {
+            cudaError_t e = cudaMemcpyAsync(S_out, S0, nS, cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
         return LATTICE_OK;
     }
     const size_t ntok = (size_t)B * T * H;
@@ -175,7 +185,7 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
     if (impl == LATTICE_IMPL_TCGEN05 && !tc_ok) return LATTICE_ERR_UNSUPPORTED;
     if (tc_ok && impl != LATTICE_IMPL_SIMT) {
         cudaError_t e = launch_chunk_tc(a, d, st);
-        return e == cudaSuccess ? LATTICE_OK : LATTICE_ERR_CUDA;
+        return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
     }
     return launch_scan_simt<true>(a, d, st);
 }
@@ -242,12 +252,16 @@ lattice_status lattice_readout(const float* S, const void* q, lattice_dtype q_dt
 
 lattice_status lattice_get_device_status(void* stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(st) != cudaSuccess) return LATTICE_ERR_CUDA;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
     unsigned int v = 0, zero = 0;
-    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return LATTICE_ERR_CUDA;
-    if (v && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
-        return LATTICE_ERR_CUDA;
+    e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (v && (e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero))) != cudaSuccess)
+        return cuda_fail(e);
     return v ? LATTICE_ERR_TIMEOUT : LATTICE_OK;
 }
+
+const char* lattice_last_cuda_error(void) { return g_last_error; }
 
 }  // extern "C"

@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
 #pragma unroll
                         for (int k = 0; k < EPL; ++k) { s0[r][k] = s[r][k]; n2 = fmaf(s[r][k], s[r][k], n2); }
                         n0sq[r] = octet_sum(n2);
-                        n0[r] = sqrtf(n0sq[r]);
+                        n0[r] = __fsqrt_rn(n0sq[r]);
                     }
                 }
             }
@@ -196,8 +196,8 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
                 const float cv = valid ? rec[D + m + slot[r]] : 0.f;
                 const float qv = valid ? rec[D + slot[r]] : 0.f;
                 float alpha, gamma;
-                update_coefs(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
-                             CHUNKED ? n0[r] : 1.f, alpha, gamma);
+                update_coefs<CHUNKED>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
+                                      CHUNKED ? n0[r] : 1.f, alpha, gamma);
                 if (!valid) { alpha = 0.f; gamma = 0.f; }
 #pragma unroll
                 for (int k = 0; k < EPL; ++k) {

@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(512) step_kernel(StepArgs a) {
 #pragma unroll
     for (int r = 0; r < RQ; ++r) {
         float alpha, gamma;
-        update_coefs(n2[r], p[r], xx, cv[r], mu, eta, 1.f, alpha, gamma);
+        update_coefs<false>(n2[r], p[r], xx, cv[r], mu, eta, 1.f, alpha, gamma);
 #pragma unroll
         for (int k = 0; k < EPL; ++k) {
             s[r][k] = fmaf(alpha, s[r][k], gamma * xv[k]);
