@@ -82,6 +82,27 @@ def step_alg_bytes(w: LI.Workload, B=None, H=None) -> int:
     return B * H * (2 * 4 * w.m * w.d + w.d * xb + w.m * qb + 4 * w.m + 4 + 4 * w.d)
 
 
+# ------------------------------------------------------------ multi-rank host
+
+def rank_workload(w: LI.Workload, rank: int) -> LI.Workload:
+    """Each rank scans its own batch: the same shapes and distributions, its own seed."""
+    return w if rank == 0 else w.with_(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(torch, dist, value: float, device) -> float:
+    """The slowest rank's time (every rank calls this, in the same order)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, w: LI.Workload, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's B*T tokens in the slowest rank's step time."""
+    return world * w.B * w.T / (ms_per_step * 1e-3)
+
+
 # -------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -253,7 +274,7 @@ def time_decode(torch, L, w, n_steps, ring, device):
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 10.0, max_reps: int = 50):
+def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 12.0, max_reps: int = 10000):
     """The fp64 oracle, as it stands, on the host cores: whole workload passes
     repeated until about min_seconds of CPU work. Returns (tokens/s, cores, sample)."""
     import oracle
@@ -289,7 +310,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = LI.WORKLOADS[HEADLINE]
+    w0 = LI.WORKLOADS[HEADLINE]
+    w = rank_workload(w0, rank)
 
     if args.impl == "reference":
         if rank != 0:
@@ -298,7 +320,7 @@ def main():
         import oracle
         inp = LI.make_inputs(w)
         cores = len(os.sched_getaffinity(0))
-        for _ in range(1):  # one untimed pass (the oracle has no warm-up state)
+        for _ in range(args.warmup):  # untimed passes
             oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=w.chunk, nthreads=cores)
         t0 = time.perf_counter()
         for _ in range(steps):
@@ -344,14 +366,11 @@ def main():
     with ClockSampler(local) as clk:
         times = time_scan(torch, L, t, w.chunk, args.steps, args.warmup, flush=flush)
     torch.cuda.synchronize()
-    total_ms = sum(times)
+    total_ms = max_over_ranks(torch, dist, sum(times), device)
     if dist is not None:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
         dist.barrier()
     ms = total_ms / args.steps
-    value = world * w.B * w.T / (ms * 1e-3)
+    value = job_tokens_per_s(world, w, ms)
 
     # roofline of the (single) kernel of the step
     tc = L.chunk_impl(w.m, w.d, w.chunk) == "tcgen05"
@@ -384,10 +403,11 @@ def main():
     if cs is not None:
         line["clocks"] = cs
 
+    # end to end through the public call with host buffers (every rank; the slowest counts)
+    e2e_ms, h2d, d2h = time_scan_e2e(torch, L, inp, w.chunk, max(3, args.steps // 2), 3, device)
+    e2e_ms = max_over_ranks(torch, dist, e2e_ms, device)
     if rank == 0:
-        # end to end through the public call with host buffers
-        e2e_ms, h2d, d2h = time_scan_e2e(torch, L, inp, w.chunk, max(3, args.steps // 2), 3, device)
-        line["e2e"] = {"value": world * w.B * w.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+        line["e2e"] = {"value": job_tokens_per_s(world, w, e2e_ms), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
         extra = {}
         if not args.no_extra:

@@ -22,24 +22,28 @@
 // sigma, so the state-update GEMM accumulates straight onto T; rows whose
 // sigma*A_C drops below 2^-100 (the old state is then below fp32 resolution)
 // are rescaled in TMEM first, and T is renormalised when sigma leaves
-// [2^-32, 2^32]. The GEMMs that carry the state use hi+lo bf16 operand pairs,
-// so the carried state keeps close to fp32 accuracy over thousands of chunks.
-// Per chunk (bf16 operands in 128B-swizzled shared memory, fp32 TMEM accumulators):
-//   G1: D1  [m x C]  = (S0hi + S0lo) . X^T        projections x_t . s0_i
-//   G7: T   [m x d] += (KShi + KSlo)^T . X        state update
-//   G5: P   [C x 16] = QR_b . KD_b^T, b = 0..3     scores, one 16-column block each
-//   G4: Y^T [d x C]  = S0hi^T . QR_0^T            inter-chunk read-out
-//   G6: Y^T [d x C] += X^T . P_causal^T           intra-chunk read-out
-// Warp roles (576 threads): warps 0-15 are workers, warp 4*sb + q owning TMEM
-// lane quadrant q (slots 32q..32q+31) and sub-chunk sb: it computes the gates of
-// tokens 16sb..16sb+15 for its 32 slots (so the 64-token gate recurrence runs as
-// four independent 16-token pieces, tied together by four sub-chunk products per
-// slot exchanged through shared memory), converts state columns
-// sb*d/4..(sb+1)*d/4, masks score columns 16sb..16sb+15 and stores y for tokens
-// 16sb..16sb+15. Warp 16 = TMA producer, MMA issuer and TMEM owner; warp 17 =
-// per-token |x|^2, mu, eta. Every mbarrier wait is bounded by %globaltimer: on
-// timeout the kernel sets the device status word, skips the remaining work and
-// still meets every named barrier.
+// [2^-32, 2^32]. The GEMMs that carry the state use hi+lo bf16 operand pairs
+// (kept in tensor memory), so the carried state keeps close to fp32 accuracy
+// over thousands of chunks. Per chunk (fp32 TMEM accumulators):
+//   G1: D1  [m x C]  = (S0hi + S0lo) . X^T       projections x_t . s0_i (A in TMEM)
+//   G7: T   [m x d] += (KShi + KSlo)^T . X       state update (A in TMEM)
+//   G4: Y^T [d x C]  = S0hi^T . QR_0^T           inter-chunk read-out (smem operands)
+//   G5: P   [C x 16] = QR_b . KD_b^T, b = 0..3    scores, one 16-column block each
+//   G6: Y^T [d x C] += X^T . P_causal^T          intra-chunk read-out
+//
+// Warp roles (640 threads, 5 warpgroups). Warps 0-15 are workers: warp 4*sb + q
+// owns TMEM lane quadrant q (slots 32q..32q+31) and sub-chunk sb. It computes
+// the gates of tokens 16sb..16sb+15 for its 32 slots (the 64-token gate
+// recurrence runs as four independent 16-token pieces, tied together by four
+// sub-chunk products per slot exchanged through shared memory), converts state
+// columns sb*d/4..(sb+1)*d/4, masks score columns 16sb..16sb+15, stores y for
+// tokens 16sb..16sb+15 and prepares |x|^2, mu, eta of four tokens of the next
+// chunk. Warp 16 issues every MMA, warp 17 every TMA copy (an MMA issue blocks
+// its warp while the MMA runs, so neither sits on a worker). The state chain
+// (G1 -> gates -> G7 -> state conversion -> next G1) is signalled separately
+// from the read-out path (G5, P mask, G6), which overlaps the next chunk.
+// Every mbarrier wait is bounded by %globaltimer: on timeout the kernel sets the
+// device status word, skips the remaining work and still meets every named barrier.
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -52,8 +56,8 @@ namespace lattice {
 
 constexpr int kTcC = 64;            // chunk size of the tensor-core path
 constexpr int kTcSub = 16;          // sub-chunk: the longest product ever divided by
-constexpr int kTcWorkWarps = 16;   // 4 lane quadrants x 4 sub-chunks
-constexpr int kTcThreads = 32 * (kTcWorkWarps + 2);  // + control warp + aux warp
+constexpr int kTcWorkers = 512;     // 16 worker warps: 4 lane quadrants x 4 sub-chunks
+constexpr int kTcThreads = kTcWorkers + 128;  // + control warpgroup (MMA warp, TMA warp, 2 idle)
 constexpr uint64_t kTcWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
 inline bool chunk_tc_supported(int m, int d, int chunk, bool x_bf16, bool q_bf16) {
@@ -66,29 +70,36 @@ struct TcLayout {
     static constexpr uint32_t X_STAGE = DS * 128;         // DS/64 blocks x 64 rows x 128 B
     static constexpr uint32_t S0_TILE = MS * DS * 2;      // DS/64 blocks x m rows x 128 B
     static constexpr uint32_t ROW_TILE = MS * 128;        // [m][64] bf16, one 128 B row per slot
+    static constexpr uint32_t Q_TILE = kTcC * MS * 2;     // [C][m] bf16, row-major (TMA)
+    static constexpr uint32_t C_TILE = kTcC * MS * 4;     // [C][m] fp32, row-major (TMA)
     static constexpr uint32_t X_OFF = 0;
-    static constexpr uint32_t S0HI_OFF = X_OFF + NST * X_STAGE;
-    static constexpr uint32_t S0LO_OFF = S0HI_OFF + S0_TILE;
-    static constexpr uint32_t QR_OFF = S0LO_OFF + S0_TILE;        // QR_0..QR_3
+    static constexpr uint32_t Q_OFF = X_OFF + NST * X_STAGE;
+    static constexpr uint32_t CC_OFF = Q_OFF + Q_TILE;
+    static constexpr uint32_t S0HI_OFF = CC_OFF + C_TILE;          // A of the read-out GEMM
+    static constexpr uint32_t QR_OFF = S0HI_OFF + S0_TILE;         // QR_0..QR_3
     static constexpr uint32_t KD_OFF = QR_OFF + 4 * ROW_TILE;
-    static constexpr uint32_t KSHI_OFF = KD_OFF + ROW_TILE;
-    static constexpr uint32_t KSLO_OFF = KSHI_OFF + ROW_TILE;
-    static constexpr uint32_t P_OFF = QR_OFF + 3 * ROW_TILE;      // [C][128 B], reuses QR_3
-    static constexpr uint32_t AUX_OFF = KSLO_OFF + ROW_TILE;      // [NST][C] float4
+    static constexpr uint32_t P_OFF = KD_OFF + ROW_TILE;           // [C][128 B]
+    static constexpr uint32_t AUX_OFF = P_OFF + kTcC * 128;        // [NST][C] float4
     static constexpr uint32_t GSUB_OFF = AUX_OFF + NST * kTcC * 16;   // [4][m] float
     static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * MS * 4;        // [4][m] float
-    static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * MS * 4;
+    static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * MS * 4;         // 8 mbarriers
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * 8;
     static constexpr uint32_t BYTES = MISC_OFF + 64;
     static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;          // room to align the base
-    static_assert(kTcC * 128 <= ROW_TILE, "P must fit in the QR_3 tile");
-    // TMEM columns (fp32): state T | D1 | P | Y^T
+    // TMEM columns: fp32 state T | D1 | P | Y^T, then bf16 pairs (two per column) of
+    // the GEMM A operands kept in tensor memory: S0 hi/lo (d/2 each), KS hi/lo (C/2 each)
     static constexpr uint32_t T_COL = 0;
     static constexpr uint32_t D1_COL = DS;
     static constexpr uint32_t P_COL = DS + kTcC;
     static constexpr uint32_t Y_COL = DS + 2 * kTcC;
-    static constexpr uint32_t TMEM_COLS = (DS + 3 * kTcC) <= 256 ? 256 : 512;
+    static constexpr uint32_t S0HI_TCOL = DS + 3 * kTcC;
+    static constexpr uint32_t S0LO_TCOL = S0HI_TCOL + DS / 2;
+    static constexpr uint32_t KSHI_TCOL = S0LO_TCOL + DS / 2;
+    static constexpr uint32_t KSLO_TCOL = KSHI_TCOL + kTcC / 2;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(KSLO_TCOL + kTcC / 2 <= TMEM_COLS, "TMEM budget");
     static constexpr uint32_t TX_BYTES = X_STAGE;
+    static constexpr uint32_t QC_BYTES = Q_TILE + C_TILE;
 };
 
 struct TcMaps {
@@ -110,6 +121,17 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
             return false;
         }
     }
+}
+
+// Warp-uniform form for the MMA warp: every lane waits, the warp agrees on the
+// outcome (and is converged for the elect.sync issue that follows).
+__device__ __forceinline__ bool tc_wait_warp(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+    const bool ok = tc_wait(bar, parity, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool tc_live(volatile uint32_t* abort) {
+    return __all_sync(0xffffffffu, *abort == 0u);
 }
 
 // Bounded wait that ignores the abort flag: used at exit so that no TMA write
@@ -134,20 +156,22 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
     return u;
 }
 
-// hi = bf16(v), lo = bf16(v - hi): two bf16 tiles whose sum carries ~16 mantissa bits.
+// hi = v truncated to bf16 (the top 16 bits: one byte permute per pair, no
+// conversion unit), lo = bf16_rn(v - hi) (v - hi is exact in fp32). hi + lo
+// carries ~16 mantissa bits and, since lo is rounded to nearest, no bias.
 __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
-    float h[8], l[8];
+    uint32_t hb[4];
+    float l[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-        h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
-        l[e] = v[e] - h[e];
+        const uint32_t bits = __float_as_uint(v[e]);
+        l[e] = v[e] - __uint_as_float(bits & 0xffff0000u);
+        if (e & 1) hb[e >> 1] = __byte_perm(__float_as_uint(v[e - 1]), bits, 0x7632);
     }
-    hi = pack8(h);
+    hi = make_uint4(hb[0], hb[1], hb[2], hb[3]);
     lo = pack8(l);
 }
 
-// 18 warps are charged as 20 for registers (warps are allocated in groups of
-// four), so the launch bound caps the kernel at 96 registers per thread.
 template <int MS, int DS>
 __global__ void __launch_bounds__(kTcThreads, 1)
     chunk_tc_kernel(const __grid_constant__ TcMaps maps, ScanArgs a) {
@@ -162,36 +186,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int T = a.T, H = a.H;
     const int nch = (T + kTcC - 1) / kTcC;
+    constexpr int MMA_WARP = 16, TMA_WARP = 17;
 
-    const uint32_t bar_full0 = sbase + Lay::BAR_OFF;          // [2]
-    const uint32_t bar_free0 = sbase + Lay::BAR_OFF + 16;     // [2]
-    const uint32_t bar_mma = sbase + Lay::BAR_OFF + 32;
+    // mbarriers: X stage landed [2], q/c landed, D1 ready, T updated (and S0 operand
+    // free), scores ready, read-out complete
+    const uint32_t bar_full0 = sbase + Lay::BAR_OFF;
+    const uint32_t bar_qc = sbase + Lay::BAR_OFF + 16;
+    const uint32_t bar_d1 = sbase + Lay::BAR_OFF + 24;
+    const uint32_t bar_t = sbase + Lay::BAR_OFF + 32;
+    const uint32_t bar_p5 = sbase + Lay::BAR_OFF + 40;
+    const uint32_t bar_y = sbase + Lay::BAR_OFF + 48;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
     volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 4);
     float4* aux = reinterpret_cast<float4*>(smem + Lay::AUX_OFF);
     float* gsub = reinterpret_cast<float*>(smem + Lay::GSUB_OFF);   // [NSUB][MS] sub-chunk products
     float* tsqp = reinterpret_cast<float*>(smem + Lay::TSQ_OFF);    // [NSUB][MS] partial |s|^2
 
-    // named barriers: ids and participant counts (16 worker warps, control warp, aux warp)
-    constexpr uint32_t BAR_S = 1, BAR_G = 2, BAR_A = 3, BAR_B = 4;
-    constexpr uint32_t N_S = kTcThreads;           // everyone
-    constexpr uint32_t N_G = 32 * kTcWorkWarps;    // workers
-    constexpr uint32_t N_A = N_G + 32;             // workers + control
-    constexpr uint32_t N_B = N_G + 64;             // workers + control + aux
-    constexpr int CTRL = kTcWorkWarps, AUXW = kTcWorkWarps + 1;
+    // named barriers (ids, participants): workers + MMA warp, or workers + TMA warp
+    constexpr uint32_t BAR_INIT = 1, BAR_G = 2, BAR_A = 3, BAR_S0 = 4, BAR_P = 5;
+    constexpr uint32_t N_WM = kTcWorkers + 32;
 
-    if (warp == CTRL) {
+    if (warp == MMA_WARP) {
         if (lane == 0) {
-            ptx::mbar_init(bar_full0, 1);
-            ptx::mbar_init(bar_full0 + 8, 1);
-            ptx::mbar_init(bar_free0, 1);
-            ptx::mbar_init(bar_free0 + 8, 1);
-            ptx::mbar_init(bar_mma, 1);
+            for (int j = 0; j < 8; ++j) ptx::mbar_init(sbase + Lay::BAR_OFF + 8 * j, 1);
             *abort = 0u;
             ptx::fence_mbar_init();
-            ptx::prefetch_tensormap(&maps.x);
-            ptx::prefetch_tensormap(&maps.q);
-            ptx::prefetch_tensormap(&maps.c);
         }
         __syncwarp();
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), Lay::TMEM_COLS);
@@ -202,171 +221,149 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == CTRL) {
-        // ------------------------------------------------------------ control
-        int last_tma[2] = {-1, -1};  // last chunk loaded into each stage
-        auto issue_tma = [&](int k) {  // X of chunk k -> stage k % 2, q and c of chunk k -> L2
-            const int s = k & 1;
-            last_tma[s] = k;
-            const uint32_t bar = bar_full0 + 8 * s;
-            ptx::mbar_arrive_expect_tx(bar, Lay::TX_BYTES);
+    if (warp >= kTcWorkers / 32) {
+        // ================================================================ control
+        if (warp == MMA_WARP) {
+            // -------------------------------------------------- MMA issue (warp-converged,
+            // one elected lane issues; descriptors get per-MMA start-address offsets)
+            constexpr uint32_t idesc_g1 = ptx::idesc_bf16(MS, kTcC, 0, 0);
+            constexpr uint32_t idesc_g7 = ptx::idesc_bf16(MS, DS, 0, 1);
+            constexpr uint32_t idesc_g5 = ptx::idesc_bf16(kTcC, kTcSub, 1, 1);
+            constexpr uint32_t idesc_g4 = ptx::idesc_bf16(DS, kTcC, 1, 1);
+            constexpr uint32_t idesc_g6 = ptx::idesc_bf16(DS, kTcC, 1, 0);
+            auto off = [](uint32_t bytes) { return uint64_t(bytes >> 4); };
+            auto g1 = [&](int k) {  // D1 = (S0hi + S0lo) . X_k^T  (M = m, N = C, K = d)
+                const uint64_t dK_x = ptx::sdesc_sw128(sbase + Lay::X_OFF, 16, 1024);
+                const uint32_t xo = (k & 1) * Lay::X_STAGE;
 #pragma unroll
-            for (int kb = 0; kb < DS / 64; ++kb)
-                ptx::tma_load_4d(sbase + Lay::X_OFF + s * Lay::X_STAGE + kb * (64 * 128), &maps.x,
-                                 bar, kb * 64, h, k * kTcC, b);
-            ptx::tma_prefetch_l2_4d(&maps.q, 0, h, k * kTcC, b);
-            ptx::tma_prefetch_l2_4d(&maps.c, 0, h, k * kTcC, b);
-        };
-        const uint32_t idesc_g1 = ptx::idesc_bf16(MS, kTcC, 0, 0);
-        const uint32_t idesc_g7 = ptx::idesc_bf16(MS, DS, 0, 1);
-        const uint32_t idesc_g5 = ptx::idesc_bf16(kTcC, kTcSub, 1, 1);
-        const uint32_t idesc_g4 = ptx::idesc_bf16(DS, kTcC, 1, 1);
-        const uint32_t idesc_g6 = ptx::idesc_bf16(DS, kTcC, 1, 0);
-        const uint32_t s0hi = sbase + Lay::S0HI_OFF, s0lo = sbase + Lay::S0LO_OFF,
-                       qr = sbase + Lay::QR_OFF, kd = sbase + Lay::KD_OFF,
-                       kshi = sbase + Lay::KSHI_OFF, kslo = sbase + Lay::KSLO_OFF,
-                       pp = sbase + Lay::P_OFF;
-        auto g1 = [&](int k) {  // D1 = (S0hi + S0lo) . X_k^T   (M = m, N = C, K = d)
-            const uint32_t xs = sbase + Lay::X_OFF + (k & 1) * Lay::X_STAGE;
+                for (int part = 0; part < 2; ++part)
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t s0 = part ? s0lo : s0hi;
-#pragma unroll
-                for (int kk = 0; kk < DS / 16; ++kk) {
-                    const uint32_t kb = kk >> 2, ko = (kk & 3) * 32;
-                    ptx::mma_bf16(tmem + Lay::D1_COL,
-                                  ptx::sdesc_sw128(s0 + kb * MS * 128 + ko, 16, 1024),
-                                  ptx::sdesc_sw128(xs + kb * 64 * 128 + ko, 16, 1024), idesc_g1,
-                                  (part | kk) != 0);
-                }
+                    for (int kk = 0; kk < DS / 16; ++kk) {
+                        const uint32_t kb = kk >> 2, ko = (kk & 3) * 32;
+                        ptx::mma_bf16_tmem_a_elect(tmem + Lay::D1_COL,
+                                                   tmem + (part ? Lay::S0LO_TCOL : Lay::S0HI_TCOL) + kk * 8,
+                                                   dK_x + off(xo + kb * 64 * 128 + ko), idesc_g1,
+                                                   (part | kk) != 0);
+                    }
+            };
+            if (nch > 0) {
+                ptx::named_bar(BAR_INIT, N_WM);  // S0 operand written
+                ptx::tc_fence_after();
+                if (tc_wait_warp(bar_full0, 0, abort)) g1(0);
+                ptx::mma_commit_elect(bar_d1);
             }
-        };
-        if (lane == 0 && nch > 0) {
-            issue_tma(0);
-            if (nch > 1) issue_tma(1);
-        }
-        __syncwarp();
-        ptx::named_bar(BAR_S, N_S);  // S0 operand and aux[0] ready
-        ptx::tc_fence_after();
-        if (lane == 0) {
-            if (tc_wait(bar_full0, 0, abort)) g1(0);
-            ptx::mma_commit(bar_mma);
-        }
-        __syncwarp();
-        for (int k = 0; k < nch; ++k) {
-            const int s = k & 1;
-            const uint32_t xs = sbase + Lay::X_OFF + s * Lay::X_STAGE;
-            ptx::named_bar(BAR_A, N_A);  // QR, KD, KS written; T prescaled; D1 and Y^T drained
-            ptx::tc_fence_after();
-            if (lane == 0) {
-                if (!*abort) {
-                    // G7: T += (KShi + KSlo)^T . X  (M = m, N = d, K = C); A K-major, B MN-major
+            const uint64_t dM_x = ptx::sdesc_sw128(sbase + Lay::X_OFF, 64 * 128, 1024);
+            const uint64_t dM_qr = ptx::sdesc_sw128(sbase + Lay::QR_OFF, MS * 128, 1024);
+            const uint64_t dM_kd = ptx::sdesc_sw128(sbase + Lay::KD_OFF, MS * 128, 1024);
+            const uint64_t dM_s0hi = ptx::sdesc_sw128(sbase + Lay::S0HI_OFF, MS * 128, 1024);
+            const uint64_t dK_p = ptx::sdesc_sw128(sbase + Lay::P_OFF, 16, 1024);
+            for (int k = 0; k < nch; ++k) {
+                const uint32_t xo = (k & 1) * Lay::X_STAGE;
+                ptx::named_bar(BAR_A, N_WM);  // KS in TMEM, QR/KD written, T prescaled, Y drained
+                ptx::tc_fence_after();
+                if (tc_live(abort)) {
+                    // G4: Y^T = S0hi^T . QR_0^T  (M = d, N = C, K = m); both MN-major. Issued
+                    // before G7 so that one commit covers every reader of the S0 operand.
+#pragma unroll
+                    for (int kk = 0; kk < MS / 16; ++kk)
+                        ptx::mma_bf16_elect(tmem + Lay::Y_COL, dM_s0hi + off(kk * 2048), dM_qr + off(kk * 2048),
+                                            idesc_g4, kk > 0);
+                    // G7: T += (KShi + KSlo)^T . X  (M = m, N = d, K = C); A in TMEM, B MN-major
 #pragma unroll
                     for (int part = 0; part < 2; ++part)
 #pragma unroll
                         for (int kk = 0; kk < kTcC / 16; ++kk)
-                            ptx::mma_bf16(tmem + Lay::T_COL,
-                                          ptx::sdesc_sw128((part ? kslo : kshi) + kk * 32, 16, 1024),
-                                          ptx::sdesc_sw128(xs + kk * 2048, 64 * 128, 1024), idesc_g7, 1);
+                            ptx::mma_bf16_tmem_a_elect(tmem + Lay::T_COL,
+                                                       tmem + (part ? Lay::KSLO_TCOL : Lay::KSHI_TCOL) + kk * 8,
+                                                       dM_x + off(xo + kk * 2048), idesc_g7, 1);
+                }
+                ptx::mma_commit_elect(bar_t);
+                if (tc_live(abort)) {
                     // G5: P[:, 16b..16b+15] = QR_b . KD_b^T  (M = C, N = 16, K = m); both MN-major
 #pragma unroll
-                    for (int sb = 0; sb < NSUB; ++sb)
-#pragma unroll
-                        for (int kk = 0; kk < MS / 16; ++kk)
-                            ptx::mma_bf16(tmem + Lay::P_COL + sb * kTcSub,
-                                          ptx::sdesc_sw128(qr + sb * Lay::ROW_TILE + kk * 2048, MS * 128, 1024),
-                                          ptx::sdesc_sw128(kd + sb * (kTcSub * 2) + kk * 2048, MS * 128, 1024),
-                                          idesc_g5, kk > 0);
-                    // G4: Y^T = S0hi^T . QR_0^T  (M = d, N = C, K = m); both MN-major
-#pragma unroll
                     for (int kk = 0; kk < MS / 16; ++kk)
-                        ptx::mma_bf16(tmem + Lay::Y_COL, ptx::sdesc_sw128(s0hi + kk * 2048, MS * 128, 1024),
-                                      ptx::sdesc_sw128(qr + kk * 2048, MS * 128, 1024), idesc_g4, kk > 0);
+#pragma unroll
+                        for (int sb = 0; sb < NSUB; ++sb)
+                            ptx::mma_bf16_elect(tmem + Lay::P_COL + sb * kTcSub,
+                                                dM_qr + off(sb * Lay::ROW_TILE + kk * 2048),
+                                                dM_kd + off(sb * (kTcSub * 2) + kk * 2048), idesc_g5, kk > 0);
                 }
-                ptx::mma_commit(bar_mma);
-            }
-            __syncwarp();
-            ptx::named_bar(BAR_B, N_B);  // next S0 operand, masked P, aux[k+1] ready
-            ptx::tc_fence_after();
-            if (lane == 0) {
-                if (!*abort) {
+                ptx::mma_commit_elect(bar_p5);
+                ptx::named_bar(BAR_S0, N_WM);  // S0 operand of chunk k+1 written
+                ptx::tc_fence_after();
+                if (k + 1 < nch) {
+                    if (tc_wait_warp(bar_full0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1, abort)) g1(k + 1);
+                    ptx::mma_commit_elect(bar_d1);
+                }
+                ptx::named_bar(BAR_P, N_WM);  // masked scores written
+                ptx::tc_fence_after();
+                if (tc_live(abort)) {
                     // G6: Y^T += X^T . P^T  (M = d, N = C, K = C); A MN-major, B K-major
 #pragma unroll
                     for (int kk = 0; kk < kTcC / 16; ++kk)
-                        ptx::mma_bf16(tmem + Lay::Y_COL, ptx::sdesc_sw128(xs + kk * 2048, 64 * 128, 1024),
-                                      ptx::sdesc_sw128(pp + kk * 32, 16, 1024), idesc_g6, 1);
+                        ptx::mma_bf16_elect(tmem + Lay::Y_COL, dM_x + off(xo + kk * 2048), dK_p + off(kk * 32),
+                                            idesc_g6, 1);
                 }
-                ptx::mma_commit(bar_free0 + 8 * s);
-                if (k + 1 < nch && tc_wait(bar_full0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1, abort))
-                    g1(k + 1);
-                ptx::mma_commit(bar_mma);
-                // stage s is free once G6 of chunk k has completed
-                if (k + 2 < nch && tc_wait(bar_free0 + 8 * s, (k >> 1) & 1, abort)) issue_tma(k + 2);
+                ptx::mma_commit_elect(bar_y);
+            }
+            if (nch > 0) tc_drain(bar_y, (nch - 1) & 1);  // every MMA done before TMEM goes away
+        } else if (warp == TMA_WARP) {
+            // -------------------------------------------------- TMA issue (lane 0)
+            int last_x[2] = {-1, -1}, last_qc = -1;
+            auto issue_x = [&](int k) {  // X of chunk k -> stage k % 2
+                const int s = k & 1;
+                last_x[s] = k;
+                const uint32_t bar = bar_full0 + 8 * s;
+                ptx::mbar_arrive_expect_tx(bar, Lay::TX_BYTES);
+#pragma unroll
+                for (int kb = 0; kb < DS / 64; ++kb)
+                    ptx::tma_load_4d(sbase + Lay::X_OFF + s * Lay::X_STAGE + kb * (64 * 128), &maps.x, bar,
+                                     kb * 64, h, k * kTcC, b);
+            };
+            auto issue_qc = [&](int k) {  // q and c of chunk k -> the single q/c stage
+                last_qc = k;
+                ptx::mbar_arrive_expect_tx(bar_qc, Lay::QC_BYTES);
+                ptx::tma_load_4d(sbase + Lay::Q_OFF, &maps.q, bar_qc, 0, h, k * kTcC, b);
+                ptx::tma_load_4d(sbase + Lay::CC_OFF, &maps.c, bar_qc, 0, h, k * kTcC, b);
+            };
+            auto prefetch_l2 = [&](int k) {  // X, q and c of chunk k into L2
+#pragma unroll
+                for (int kb = 0; kb < DS / 64; ++kb) ptx::tma_prefetch_l2_4d(&maps.x, kb * 64, h, k * kTcC, b);
+                ptx::tma_prefetch_l2_4d(&maps.q, 0, h, k * kTcC, b);
+                ptx::tma_prefetch_l2_4d(&maps.c, 0, h, k * kTcC, b);
+            };
+            if (lane == 0 && nch > 0) {
+                ptx::prefetch_tensormap(&maps.x);
+                ptx::prefetch_tensormap(&maps.q);
+                ptx::prefetch_tensormap(&maps.c);
+                issue_x(0);
+                issue_qc(0);
+                if (nch > 1) issue_x(1);
+                for (int j = 1; j < 4 && j < nch; ++j) prefetch_l2(j);
+            }
+            for (int k = 0; k < nch; ++k) {
+                ptx::named_bar(BAR_G, N_WM);  // every worker is done reading q and c of chunk k
+                if (lane == 0) {
+                    if (k + 1 < nch) issue_qc(k + 1);
+                    // X of chunk k is read last by G6_k; then its stage takes chunk k+2
+                    if (k + 2 < nch && tc_wait(bar_y, k & 1, abort)) {
+                        issue_x(k + 2);
+                        if (k + 4 < nch) prefetch_l2(k + 4);
+                    }
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {  // no TMA write may be in flight when the CTA retires
+#pragma unroll
+                for (int s = 0; s < 2; ++s)
+                    if (last_x[s] >= 0) tc_drain(bar_full0 + 8 * s, (last_x[s] >> 1) & 1);
+                if (last_qc >= 0) tc_drain(bar_qc, last_qc & 1);
             }
             __syncwarp();
         }
-        // drain: the last commit covers every MMA; wait for it before TMEM goes away,
-        // and for every TMA load still in flight before shared memory goes away
-        if (lane == 0) {
-            tc_wait(bar_mma, (2 * nch) & 1, abort);
-#pragma unroll
-            for (int s = 0; s < 2; ++s)
-                if (last_tma[s] >= 0) tc_drain(bar_full0 + 8 * s, (last_tma[s] >> 1) & 1);
-        }
-        __syncwarp();
-    } else if (warp == AUXW) {
-        // ------------------------------------------------------------ aux:
-        // per-token {mu, eta, |x|^2, mu^2} of chunk k into aux[k % 2]
-        auto aux_chunk = [&](int k) {
-            const int s = k & 1;
-            float mu2[2], eta2[2];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {  // global loads first, X wait second
-                const int t = k * kTcC + lane + 32 * half;
-                mu2[half] = 0.f;
-                eta2[half] = 1.f;
-                if (t < T) {
-                    const size_t bth = ((size_t)b * T + t) * H + h;
-                    mu2[half] = __ldg(a.mu + bth);
-                    if (a.eta) eta2[half] = __ldg(a.eta + bth);
-                }
-            }
-            const bool ok = tc_wait(bar_full0 + 8 * s, (k >> 1) & 1, abort);
-            const uint8_t* xs = smem + Lay::X_OFF + s * Lay::X_STAGE;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int tau = lane + 32 * half;
-                float xx = 0.f;
-                if (ok) {
-#pragma unroll
-                    for (int kb = 0; kb < DS / 64; ++kb)
-#pragma unroll
-                        for (int ch = 0; ch < 8; ++ch) {
-                            // any order sums the row; rotating by the row spreads lanes over banks
-                            const int pc = (ch + tau) & 7;
-                            uint4 v = *reinterpret_cast<const uint4*>(xs + kb * (64 * 128) + tau * 128 + pc * 16);
-                            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
-                                xx = fmaf(lo, lo, xx);
-                                xx = fmaf(hi, hi, xx);
-                            }
-                        }
-                }
-                const float mu = mu2[half];
-                aux[s * kTcC + tau] = make_float4(mu, eta2[half], xx, mu * mu);
-            }
-        };
-        if (nch > 0) aux_chunk(0);
-        ptx::named_bar(BAR_S, N_S);
-        for (int k = 0; k < nch; ++k) {
-            if (k + 1 < nch) aux_chunk(k + 1);
-            ptx::named_bar(BAR_B, N_B);
-        }
     } else {
-        // ------------------------------------------------------------ workers
-        // warp = 4 * sb + q4: TMEM lane quadrant q4, sub-chunk / column block sb
+        // ================================================================ workers
+        // warp 4*sb + q4 owns TMEM lane quadrant q4 and sub-chunk sb
         const int q4 = warp & 3, sb = warp >> 2;
         const bool active = (MS == 128) || (lane < 16);
         const int i = (MS == 128) ? (32 * q4 + lane) : (16 * q4 + (lane & 15));  // slot
@@ -377,42 +374,65 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool prow_ok = lane < 16;
         const int tau_row = 16 * q4 + lane;
         uint8_t* s0hi = smem + Lay::S0HI_OFF;
-        uint8_t* s0lo = smem + Lay::S0LO_OFF;
         uint8_t* qr = smem + Lay::QR_OFF;
         uint8_t* kd = smem + Lay::KD_OFF;
-        uint8_t* kshi = smem + Lay::KSHI_OFF;
-        uint8_t* kslo = smem + Lay::KSLO_OFF;
         uint8_t* ps = smem + Lay::P_OFF;
+        const uint16_t* qsm = reinterpret_cast<const uint16_t*>(smem + Lay::Q_OFF);
+        const float* csm = reinterpret_cast<const float*>(smem + Lay::CC_OFF);
 
-        // a block of DCOL state columns starting at col0 -> hi/lo bf16 operand rows
+        // a block of DCOL state columns starting at col0 -> hi/lo bf16 operand rows: both
+        // into tensor memory (A of the projection GEMM; warp-collective), hi into shared
+        // memory too (A of the read-out GEMM). Lanes without a slot store zeros.
         auto store_s0 = [&](int col0, const float* v) {
             const int kb = col0 >> 6;
+            uint32_t hw[DCOL / 2], lw[DCOL / 2];
 #pragma unroll
             for (int ch = 0; ch < DCOL / 8; ++ch) {
                 uint4 hi, lo;
                 split8(v + 8 * ch, hi, lo);
-                const uint32_t off = kb * Lay::ROW_TILE + ptx::sw128_chunk(i, ((col0 & 63) >> 3) + ch);
-                *reinterpret_cast<uint4*>(s0hi + off) = hi;
-                *reinterpret_cast<uint4*>(s0lo + off) = lo;
+                hw[4 * ch + 0] = hi.x; hw[4 * ch + 1] = hi.y; hw[4 * ch + 2] = hi.z; hw[4 * ch + 3] = hi.w;
+                lw[4 * ch + 0] = lo.x; lw[4 * ch + 1] = lo.y; lw[4 * ch + 2] = lo.z; lw[4 * ch + 3] = lo.w;
+                if (active)
+                    *reinterpret_cast<uint4*>(s0hi + kb * Lay::ROW_TILE +
+                                              ptx::sw128_chunk(i, ((col0 & 63) >> 3) + ch)) = hi;
+            }
+            ptx::tmem_st<DCOL / 2>(tmem + lane_base + Lay::S0HI_TCOL + col0 / 2, hw);
+            ptx::tmem_st<DCOL / 2>(tmem + lane_base + Lay::S0LO_TCOL + col0 / 2, lw);
+        };
+        auto load_mueta = [&](int k, float& mu, float& eta) {  // this lane's token of aux_part(k)
+            const int t = k * kTcC + 4 * warp + (lane >> 3);
+            mu = 0.f;
+            eta = 1.f;
+            if ((lane & 7) == 0 && t < T) {
+                const size_t bth = ((size_t)b * T + t) * H + h;
+                mu = __ldg(a.mu + bth);
+                if (a.eta) eta = __ldg(a.eta + bth);
             }
         };
-        // q and c of this group's 16 tokens of chunk k: coalesced over the slots
-        auto load_qc = [&](int k, float* qv, float* cv) {
-            const int t0 = k * kTcC + sb * kTcSub;
-            const size_t e0 = (((size_t)b * T + t0) * H + h) * MS + i;
-            const uint16_t* qp = static_cast<const uint16_t*>(a.q) + e0;
-            const float* cp = a.c + e0;
-            const int stride = H * MS;
-            const int nvalid = active ? min(kTcSub, T - t0) : 0;
+        // per-token {mu, eta, |x|^2, mu^2} of 4 tokens of chunk k (this warp's share) into aux[k % 2]
+        auto aux_part = [&](int k, float mu, float eta) {
+            const int s = k & 1;
+            const int u = lane >> 3, part = lane & 7;
+            const int tau = 4 * warp + u;
+            const bool ok = tc_wait(bar_full0 + 8 * s, (k >> 1) & 1, abort);
+            const uint8_t* xs = smem + Lay::X_OFF + s * Lay::X_STAGE;
+            float xx = 0.f;
+            if (ok) {
 #pragma unroll
-            for (int u = 0; u < kTcSub; ++u) {
-                qv[u] = 0.f;
-                cv[u] = 0.f;
-                if (u < nvalid) {
-                    qv[u] = __uint_as_float(uint32_t(__ldg(qp + u * stride)) << 16);
-                    cv[u] = __ldg(cp + u * stride);
+                for (int kb = 0; kb < DS / 64; ++kb) {
+                    // the 8 lanes of a token read its 8 chunks of 16 B (any order sums the row)
+                    uint4 v = *reinterpret_cast<const uint4*>(xs + kb * (64 * 128) + tau * 128 + part * 16);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+                        xx = fmaf(lo, lo, xx);
+                        xx = fmaf(hi, hi, xx);
+                    }
                 }
             }
+            xx = octet_sum(xx);
+            if (part == 0) aux[s * kTcC + tau] = make_float4(mu, eta, xx, mu * mu);
         };
         auto store_y = [&](int kc) {  // 16 tokens of chunk kc from the Y^T accumulator
             uint32_t yv[kTcSub];
@@ -427,7 +447,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (t0 + u < T) yb[u * stride] = __uint_as_float(yv[u]);
         };
 
-        // initial state: T = S0 (sigma = 1), operand, partial norms; this group's DCOL columns
+        // ---- prologue: initial state T = S0 (sigma = 1), operands, norms, aux of chunk 0
         float sigma = 1.f;
         {
             const float* S0g = a.S0 + ((size_t)bh * MS + i) * DS + sb * DCOL;
@@ -445,17 +465,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 r[e] = __float_as_uint(v[e]);
             }
             ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+            store_s0(sb * DCOL, v);
             ptx::tmem_wait_st();
-            if (active) {
-                store_s0(sb * DCOL, v);
-                tsqp[sb * MS + i] = ns;
-            }
+            if (active) tsqp[sb * MS + i] = ns;
         }
-        float qv[kTcSub], cv[kTcSub];
-        if (nch > 0) load_qc(0, qv, cv);
+        if (nch > 0) {
+            float mu0, eta0;
+            load_mueta(0, mu0, eta0);
+            aux_part(0, mu0, eta0);
+        }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        ptx::named_bar(BAR_S, N_S);
+        if (nch > 0) ptx::named_bar(BAR_INIT, N_WM);
         float nsq = 0.f;
         if (active)
 #pragma unroll
@@ -464,12 +485,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int k = 0; k < nch; ++k) {
             const int s = k & 1;
             // ---- phase A: gates of this group's 16 tokens (needs D1 = S0 . X_k^T)
-            tc_wait(bar_mma, 0, abort);  // completion #2k: G1_k and (k > 0) G6_{k-1}
+            float mu1, eta1;  // next chunk's gate inputs, stored at the end of phase B
+            if (k + 1 < nch) load_mueta(k + 1, mu1, eta1);
+            tc_wait(bar_d1, k & 1, abort);
+            __syncwarp();
             ptx::tc_fence_after();
-            if (k > 0) store_y(k - 1);
             uint32_t pr[kTcSub];
             ptx::tmem_ld16(tmem + lane_base + Lay::D1_COL + sb * kTcSub, pr);
             ptx::tmem_wait_ld();
+            tc_wait(bar_qc, k & 1, abort);  // q and c of chunk k in shared memory
+            __syncwarp();
             const float n = sqrtf(nsq);
             const float inv_n = 1.f / n, inv_n2 = 1.f / nsq;
             const float4* ax = aux + s * kTcC + sb * kTcSub;
@@ -478,8 +503,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int u = 0; u < kTcSub; ++u) {
                 const float4 z = ax[u];  // mu, eta, |x|^2, mu^2
+                const int tau = sb * kTcSub + u;
+                const float cvu = csm[tau * MS + i];
+                const float qvu = __uint_as_float(uint32_t(qsm[tau * MS + i]) << 16);
                 const float p = __uint_as_float(pr[u]);
-                const float av = z.y * cv[u] * inv_n;              // eta c / n
+                const float av = z.y * cvu * inv_n;                // eta c / n
                 const float r = p * inv_n2;                        // p / n^2
                 const float perp2 = fmaxf(fmaf(-p, r, z.z), 0.f);  // |x_perp|^2
                 const float den = fmaf(av * av, perp2, z.w * nsq);
@@ -489,11 +517,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 gv[u] = g;
                 kdv[u] = bn * av;                                   // kappa for now
                 R *= g;
-                base[u] = qv[u] * R;                                // q_t prod_{16sb..t} g
+                base[u] = qvu * R;                                  // q_t prod_{16sb..t} g
             }
             if (active) gsub[sb * MS + i] = R;
-            // KD(t) = kappa_t / prod_{16sb..t} g: one reciprocal, then a backward product
-            {
+            {   // KD(t) = kappa_t / prod_{16sb..t} g: one reciprocal, then a backward product
                 float inv = ptx::rcp_nr(copysignf(fmaxf(fabsf(R), 1e-37f), R));
 #pragma unroll
                 for (int u = kTcSub - 1; u >= 0; --u) {
@@ -505,27 +532,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int g8 = 2 * sb + hh;
-                    *reinterpret_cast<uint4*>(qr + sb * Lay::ROW_TILE + ptx::sw128_chunk(i, g8)) =
-                        pack8(base + 8 * hh);
+                    *reinterpret_cast<uint4*>(qr + sb * Lay::ROW_TILE + ptx::sw128_chunk(i, g8)) = pack8(base + 8 * hh);
                     *reinterpret_cast<uint4*>(kd + ptx::sw128_chunk(i, g8)) = pack8(kdv + 8 * hh);
                 }
             }
-            ptx::named_bar(BAR_G, N_G);  // all four sub-chunk products of every slot known
+            ptx::named_bar(BAR_G, N_WM);  // sub-chunk products known; q and c free for chunk k+1
             float G[NSUB];
 #pragma unroll
             for (int g = 0; g < NSUB; ++g) G[g] = active ? gsub[g * MS + i] : 1.f;
-            // query operands of the earlier sub-chunks' key blocks (plain products), zeros
-            // for the later ones; then the state-update coefficients of this group's tokens
-            float F = 1.f, AC = 1.f;   // prod_{c >= sb} G_c, prod_c G_c
+            float F = 1.f, AC = 1.f;  // prod_{c >= sb} G_c, prod_c G_c
 #pragma unroll
             for (int g = NSUB - 1; g >= 0; --g) {
                 AC *= G[g];
                 if (g >= sb) F *= G[g];
             }
-            const float sig_c = sigma * AC;  // sigma * A_C
+            const float sig_c = sigma * AC;                     // sigma * A_C
             const bool pre = !(fabsf(sig_c) >= 7.8886091e-31f);  // 2^-100, or not finite
             const float inv_sig = pre ? 1.f : 1.f / sig_c;
             if (active) {
+                // query operands of the other sub-chunks' key blocks for this group's tokens:
+                // plain products for the earlier blocks, zeros for the later ones
 #pragma unroll
                 for (int bb = 0; bb < NSUB; ++bb) {
                     if (bb == sb) continue;
@@ -535,14 +561,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         if (g >= bb && g < sb) cgb *= G[g];
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        float v[8];
+                        uint4 u4 = make_uint4(0u, 0u, 0u, 0u);
+                        if (bb < sb) {
+                            float v[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] = bb < sb ? base[8 * hh + e] * cgb : 0.f;
-                        *reinterpret_cast<uint4*>(qr + bb * Lay::ROW_TILE + ptx::sw128_chunk(i, 2 * sb + hh)) =
-                            pack8(v);
+                            for (int e = 0; e < 8; ++e) v[e] = base[8 * hh + e] * cgb;
+                            u4 = pack8(v);
+                        }
+                        *reinterpret_cast<uint4*>(qr + bb * Lay::ROW_TILE + ptx::sw128_chunk(i, 2 * sb + hh)) = u4;
                     }
                 }
-                const float ksc = F * inv_sig;
+            }
+            {   // state-update coefficients KS(t) = KD(t) F_sb / (sigma A_C) -> tensor memory
+                const float ksc = active ? F * inv_sig : 0.f;
+                uint32_t hw[8], lw[8];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[8];
@@ -550,9 +582,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int e = 0; e < 8; ++e) v[e] = kdv[8 * hh + e] * ksc;
                     uint4 hi, lo;
                     split8(v, hi, lo);
-                    *reinterpret_cast<uint4*>(kshi + ptx::sw128_chunk(i, 2 * sb + hh)) = hi;
-                    *reinterpret_cast<uint4*>(kslo + ptx::sw128_chunk(i, 2 * sb + hh)) = lo;
+                    hw[4 * hh + 0] = hi.x; hw[4 * hh + 1] = hi.y; hw[4 * hh + 2] = hi.z; hw[4 * hh + 3] = hi.w;
+                    lw[4 * hh + 0] = lo.x; lw[4 * hh + 1] = lo.y; lw[4 * hh + 2] = lo.z; lw[4 * hh + 3] = lo.w;
                 }
+                ptx::tmem_st8(tmem + lane_base + Lay::KSHI_TCOL + 8 * sb, hw);
+                ptx::tmem_st8(tmem + lane_base + Lay::KSLO_TCOL + 8 * sb, lw);
             }
             // rows whose old state fell below fp32 resolution: T <- sigma A_C T, sigma = 1
             if (__any_sync(0xffffffffu, pre && active)) {
@@ -563,15 +597,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int e = 0; e < DCOL; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * sc);
                 ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
-                ptx::tmem_wait_st();
             }
+            ptx::tmem_wait_st();
             sigma = pre ? 1.f : sig_c;
+            if (k > 0) {  // y of chunk k-1 (before this chunk's read-out GEMM reuses Y^T)
+                tc_wait(bar_y, (k - 1) & 1, abort);
+                __syncwarp();
+                ptx::tc_fence_after();
+                store_y(k - 1);
+            }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::named_bar(BAR_A, N_A);
+            ptx::named_bar(BAR_A, N_WM);
 
-            // ---- phase B: state after the chunk (S = sigma T'), masked scores
-            tc_wait(bar_mma, 1, abort);  // completion #2k+1 (G7, G5, G4)
+            // ---- phase B1: state after the chunk (S = sigma T') and the next S0 operand
+            tc_wait(bar_t, k & 1, abort);  // G4 and G7 complete
+            __syncwarp();
             ptx::tc_fence_after();
             const bool renorm = !(fabsf(sigma) >= 2.3283064e-10f && fabsf(sigma) <= 4.2949673e9f);
             const bool any_renorm = __any_sync(0xffffffffu, renorm && active);  // tcgen05.st is warp-collective
@@ -587,23 +628,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ts = fmaf(v[e], v[e], ts);
                     if (renorm) r[e] = __float_as_uint(v[e]);
                 }
-                if (any_renorm) {
-                    ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
-                    ptx::tmem_wait_st();
-                }
-                if (active) {
-                    tsqp[sb * MS + i] = ts;
-                    if (k + 1 == nch) {
+                if (any_renorm) ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+                if (active) tsqp[sb * MS + i] = ts;
+                if (k + 1 == nch) {
+                    if (active) {
                         float* So = a.S_out + ((size_t)bh * MS + i) * DS + sb * DCOL;
 #pragma unroll
                         for (int e = 0; e < DCOL; e += 4)
                             *reinterpret_cast<float4*>(So + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                    } else {
-                        store_s0(sb * DCOL, v);
                     }
+                } else {
+                    store_s0(sb * DCOL, v);
                 }
+                ptx::tmem_wait_st();
             }
             if (renorm) sigma = 1.f;
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::named_bar(BAR_S0, N_WM);
+            nsq = 0.f;
+            if (active)
+#pragma unroll
+                for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+
+            // ---- phase B2: masked scores, next chunk's per-token inputs
+            tc_wait(bar_p5, k & 1, abort);  // G5 complete
+            __syncwarp();
+            ptx::tc_fence_after();
             {   // causal mask of P: this group's 16 score columns of row tau_row
                 uint32_t r[kTcSub];
                 ptx::tmem_ld16(tmem + lane_base + Lay::P_COL + sb * kTcSub, r);
@@ -621,17 +672,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
             }
-            if (k + 1 < nch) load_qc(k + 1, qv, cv);
+            if (k + 1 < nch) aux_part(k + 1, mu1, eta1);
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::named_bar(BAR_B, N_B);
-            nsq = 0.f;
-            if (active)
-#pragma unroll
-                for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+            ptx::named_bar(BAR_P, N_WM);
         }
         if (nch > 0) {  // read-out of the last chunk
-            tc_wait(bar_mma, 0, abort);  // completion #2nch: G6 of the last chunk
+            tc_wait(bar_y, (nch - 1) & 1, abort);
+            __syncwarp();
             ptx::tc_fence_after();
             store_y(nch - 1);
         }
@@ -639,7 +687,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == CTRL) ptx::tmem_dealloc(tmem, Lay::TMEM_COLS);
+    if (warp == MMA_WARP) ptx::tmem_dealloc(tmem, Lay::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- host side
