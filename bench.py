@@ -304,13 +304,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the context workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--workload", default=HEADLINE, choices=["small_train", "mid_layer", "long_ctx"],
+                    help="chunked workload of the timed step (default: the small training shape)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w0 = LI.WORKLOADS[HEADLINE]
+    w0 = LI.WORKLOADS[args.workload]
     w = rank_workload(w0, rank)
 
     if args.impl == "reference":
@@ -404,19 +407,21 @@ def main():
         line["clocks"] = cs
 
     # end to end through the public call with host buffers (every rank; the slowest counts)
-    e2e_ms, h2d, d2h = time_scan_e2e(torch, L, inp, w.chunk, max(3, args.steps // 2), 3, device)
-    e2e_ms = max_over_ranks(torch, dist, e2e_ms, device)
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_scan_e2e(torch, L, inp, w.chunk, max(3, args.steps // 2), 3, device)
+        e2e_ms = max_over_ranks(torch, dist, e2e_ms, device)
     if rank == 0:
-        line["e2e"] = {"value": job_tokens_per_s(world, w, e2e_ms), "unit": "tokens/s",
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        if not args.no_e2e:
+            line["e2e"] = {"value": job_tokens_per_s(world, w, e2e_ms), "unit": "tokens/s",
+                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
         extra = {}
         if not args.no_extra:
-            # exact recurrence on the headline workload
+            # exact recurrence on the timed workload
             te = time_scan(torch, L, t, 1, 5, 3, flush=flush)
-            extra["small_train_exact"] = {"ms": statistics.mean(te),
-                                          "tokens_per_s": w.B * w.T / (statistics.mean(te) * 1e-3)}
+            extra[f"{w.name}_exact"] = {"ms": statistics.mean(te),
+                                        "tokens_per_s": w.B * w.T / (statistics.mean(te) * 1e-3)}
             del t
-            for name in ("mid_layer", "long_ctx"):
+            for name in [n for n in ("mid_layer", "long_ctx") if n != w.name]:
                 wn = LI.WORKLOADS[name]
                 inn = LI.make_inputs(wn)
                 tn = _dev_inputs(torch, inn, device)

@@ -79,25 +79,26 @@ struct TcLayout {
     static constexpr uint32_t QR_OFF = S0HI_OFF + S0_TILE;         // QR_0..QR_3
     static constexpr uint32_t KD_OFF = QR_OFF + 4 * ROW_TILE;
     static constexpr uint32_t P_OFF = KD_OFF + ROW_TILE;           // [C][128 B]
-    static constexpr uint32_t AUX_OFF = P_OFF + kTcC * 128;        // [NST][C] float4
+    static constexpr uint32_t AUX_OFF = P_OFF + kTcC * 128;        // [NST][C/2][2] float4
     static constexpr uint32_t GSUB_OFF = AUX_OFF + NST * kTcC * 16;   // [4][m] float
     static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * MS * 4;        // [4][m] float
     static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * MS * 4;         // 8 mbarriers
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * 8;
     static constexpr uint32_t BYTES = MISC_OFF + 64;
     static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;          // room to align the base
-    // TMEM columns: fp32 state T | D1 | P | Y^T, then bf16 pairs (two per column) of
-    // the GEMM A operands kept in tensor memory: S0 hi/lo (d/2 each), KS hi/lo (C/2 each)
+    // TMEM columns: fp32 state T | D1 (projections; its columns also hold the bf16
+    // hi/lo pairs of the state-update operand KS, whose lifetime never overlaps
+    // D1's) | P | Y^T, double-buffered | S0 hi/lo bf16 pairs (two per column, d/2 each)
     static constexpr uint32_t T_COL = 0;
     static constexpr uint32_t D1_COL = DS;
+    static constexpr uint32_t KSHI_TCOL = D1_COL;
+    static constexpr uint32_t KSLO_TCOL = D1_COL + kTcC / 2;
     static constexpr uint32_t P_COL = DS + kTcC;
-    static constexpr uint32_t Y_COL = DS + 2 * kTcC;
-    static constexpr uint32_t S0HI_TCOL = DS + 3 * kTcC;
+    static constexpr uint32_t Y_COL = DS + 2 * kTcC;               // + (chunk & 1) * C
+    static constexpr uint32_t S0HI_TCOL = DS + 4 * kTcC;
     static constexpr uint32_t S0LO_TCOL = S0HI_TCOL + DS / 2;
-    static constexpr uint32_t KSHI_TCOL = S0LO_TCOL + DS / 2;
-    static constexpr uint32_t KSLO_TCOL = KSHI_TCOL + kTcC / 2;
     static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(KSLO_TCOL + kTcC / 2 <= TMEM_COLS, "TMEM budget");
+    static_assert(S0LO_TCOL + DS / 2 <= TMEM_COLS, "TMEM budget");
     static constexpr uint32_t TX_BYTES = X_STAGE;
     static constexpr uint32_t QC_BYTES = Q_TILE + C_TILE;
 };
@@ -159,17 +160,12 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // hi = v truncated to bf16 (the top 16 bits: one byte permute per pair, no
 // conversion unit), lo = bf16_rn(v - hi) (v - hi is exact in fp32). hi + lo
 // carries ~16 mantissa bits and, since lo is rounded to nearest, no bias.
-__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
-    uint32_t hb[4];
-    float l[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const uint32_t bits = __float_as_uint(v[e]);
-        l[e] = v[e] - __uint_as_float(bits & 0xffff0000u);
-        if (e & 1) hb[e >> 1] = __byte_perm(__float_as_uint(v[e - 1]), bits, 0x7632);
-    }
-    hi = make_uint4(hb[0], hb[1], hb[2], hb[3]);
-    lo = pack8(l);
+__device__ __forceinline__ void split2(float2 v, uint32_t& hi, uint32_t& lo) {
+    const uint32_t bx = __float_as_uint(v.x), by = __float_as_uint(v.y);
+    hi = __byte_perm(bx, by, 0x7632);
+    const float2 h = make_float2(__uint_as_float(bx & 0xffff0000u), __uint_as_float(by & 0xffff0000u));
+    const float2 l = ptx::f2add(v, ptx::f2neg(h));
+    lo = ptx::pack_bf16x2(l.x, l.y);
 }
 
 template <int MS, int DS>
@@ -188,17 +184,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nch = (T + kTcC - 1) / kTcC;
     constexpr int MMA_WARP = 16, TMA_WARP = 17;
 
-    // mbarriers: X stage landed [2], q/c landed, D1 ready, T updated (and S0 operand
-    // free), scores ready, read-out complete
+    // mbarriers: X stage landed [2], q/c landed, D1 ready, T updated (G7), S0 operand
+    // read (G4), scores ready (G5), read-out complete (G6)
     const uint32_t bar_full0 = sbase + Lay::BAR_OFF;
     const uint32_t bar_qc = sbase + Lay::BAR_OFF + 16;
     const uint32_t bar_d1 = sbase + Lay::BAR_OFF + 24;
     const uint32_t bar_t = sbase + Lay::BAR_OFF + 32;
     const uint32_t bar_p5 = sbase + Lay::BAR_OFF + 40;
     const uint32_t bar_y = sbase + Lay::BAR_OFF + 48;
+    const uint32_t bar_g4 = sbase + Lay::BAR_OFF + 56;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
     volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 4);
-    float4* aux = reinterpret_cast<float4*>(smem + Lay::AUX_OFF);
+    // per X stage: set when a token of that chunk has mu^2 below 2^-60, where the normaliser's
+    // argument may be denormal or zero (a zero-norm update keeps the slot)
+    volatile uint32_t* zmu = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 8);
+    float* aux = reinterpret_cast<float*>(smem + Lay::AUX_OFF);
     float* gsub = reinterpret_cast<float*>(smem + Lay::GSUB_OFF);   // [NSUB][MS] sub-chunk products
     float* tsqp = reinterpret_cast<float*>(smem + Lay::TSQ_OFF);    // [NSUB][MS] partial |s|^2
 
@@ -210,6 +210,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             for (int j = 0; j < 8; ++j) ptx::mbar_init(sbase + Lay::BAR_OFF + 8 * j, 1);
             *abort = 0u;
+            zmu[0] = 0u;
+            zmu[1] = 0u;
             ptx::fence_mbar_init();
         }
         __syncwarp();
@@ -259,15 +261,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint64_t dK_p = ptx::sdesc_sw128(sbase + Lay::P_OFF, 16, 1024);
             for (int k = 0; k < nch; ++k) {
                 const uint32_t xo = (k & 1) * Lay::X_STAGE;
-                ptx::named_bar(BAR_A, N_WM);  // KS in TMEM, QR/KD written, T prescaled, Y drained
+                const uint32_t ycol = Lay::Y_COL + (k & 1) * kTcC;
+                ptx::named_bar(BAR_A, N_WM);  // KS in TMEM, QR/KD written, T prescaled
                 ptx::tc_fence_after();
                 if (tc_live(abort)) {
-                    // G4: Y^T = S0hi^T . QR_0^T  (M = d, N = C, K = m); both MN-major. Issued
-                    // before G7 so that one commit covers every reader of the S0 operand.
-#pragma unroll
-                    for (int kk = 0; kk < MS / 16; ++kk)
-                        ptx::mma_bf16_elect(tmem + Lay::Y_COL, dM_s0hi + off(kk * 2048), dM_qr + off(kk * 2048),
-                                            idesc_g4, kk > 0);
                     // G7: T += (KShi + KSlo)^T . X  (M = m, N = d, K = C); A in TMEM, B MN-major
 #pragma unroll
                     for (int part = 0; part < 2; ++part)
@@ -278,6 +275,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                        dM_x + off(xo + kk * 2048), idesc_g7, 1);
                 }
                 ptx::mma_commit_elect(bar_t);
+                if (tc_live(abort)) {
+                    // G4: Y^T = S0hi^T . QR_0^T  (M = d, N = C, K = m); both MN-major
+#pragma unroll
+                    for (int kk = 0; kk < MS / 16; ++kk)
+                        ptx::mma_bf16_elect(tmem + ycol, dM_s0hi + off(kk * 2048), dM_qr + off(kk * 2048),
+                                            idesc_g4, kk > 0);
+                }
+                ptx::mma_commit_elect(bar_g4);
                 if (tc_live(abort)) {
                     // G5: P[:, 16b..16b+15] = QR_b . KD_b^T  (M = C, N = 16, K = m); both MN-major
 #pragma unroll
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     // G6: Y^T += X^T . P^T  (M = d, N = C, K = C); A MN-major, B K-major
 #pragma unroll
                     for (int kk = 0; kk < kTcC / 16; ++kk)
-                        ptx::mma_bf16_elect(tmem + Lay::Y_COL, dM_x + off(xo + kk * 2048), dK_p + off(kk * 32),
+                        ptx::mma_bf16_elect(tmem + ycol, dM_x + off(xo + kk * 2048), dK_p + off(kk * 32),
                                             idesc_g6, 1);
                 }
                 ptx::mma_commit_elect(bar_y);
@@ -387,14 +392,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int kb = col0 >> 6;
             uint32_t hw[DCOL / 2], lw[DCOL / 2];
 #pragma unroll
-            for (int ch = 0; ch < DCOL / 8; ++ch) {
-                uint4 hi, lo;
-                split8(v + 8 * ch, hi, lo);
-                hw[4 * ch + 0] = hi.x; hw[4 * ch + 1] = hi.y; hw[4 * ch + 2] = hi.z; hw[4 * ch + 3] = hi.w;
-                lw[4 * ch + 0] = lo.x; lw[4 * ch + 1] = lo.y; lw[4 * ch + 2] = lo.z; lw[4 * ch + 3] = lo.w;
-                if (active)
+            for (int e = 0; e < DCOL / 2; ++e) split2(make_float2(v[2 * e], v[2 * e + 1]), hw[e], lw[e]);
+            if (active) {
+#pragma unroll
+                for (int ch = 0; ch < DCOL / 8; ++ch)
                     *reinterpret_cast<uint4*>(s0hi + kb * Lay::ROW_TILE +
-                                              ptx::sw128_chunk(i, ((col0 & 63) >> 3) + ch)) = hi;
+                                              ptx::sw128_chunk(i, ((col0 & 63) >> 3) + ch)) =
+                        make_uint4(hw[4 * ch], hw[4 * ch + 1], hw[4 * ch + 2], hw[4 * ch + 3]);
             }
             ptx::tmem_st<DCOL / 2>(tmem + lane_base + Lay::S0HI_TCOL + col0 / 2, hw);
             ptx::tmem_st<DCOL / 2>(tmem + lane_base + Lay::S0LO_TCOL + col0 / 2, lw);
@@ -409,14 +413,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (a.eta) eta = __ldg(a.eta + bth);
             }
         };
-        // per-token {mu, eta, |x|^2, mu^2} of 4 tokens of chunk k (this warp's share) into aux[k % 2]
+        // per-token mu, eta, |x|^2, mu^2 of 4 tokens of chunk k (this warp's share) into
+        // aux[k % 2], laid out per token pair {mu0 mu1 eta0 eta1 | xx0 xx1 mu2_0 mu2_1}
         auto aux_part = [&](int k, float mu, float eta) {
             const int s = k & 1;
             const int u = lane >> 3, part = lane & 7;
             const int tau = 4 * warp + u;
             const bool ok = tc_wait(bar_full0 + 8 * s, (k >> 1) & 1, abort);
             const uint8_t* xs = smem + Lay::X_OFF + s * Lay::X_STAGE;
-            float xx = 0.f;
+            float2 acc = ptx::f2(0.f);
             if (ok) {
 #pragma unroll
                 for (int kb = 0; kb < DS / 64; ++kb) {
@@ -425,25 +430,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
-                        xx = fmaf(lo, lo, xx);
-                        xx = fmaf(hi, hi, xx);
+                        const float2 xv = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+                        acc = ptx::f2fma(xv, xv, acc);
                     }
                 }
             }
-            xx = octet_sum(xx);
-            if (part == 0) aux[s * kTcC + tau] = make_float4(mu, eta, xx, mu * mu);
+            const float xx = octet_sum(acc.x + acc.y);
+            if (part == 0) {
+                float* A = aux + (s * (kTcC / 2) + (tau >> 1)) * 8 + (tau & 1);
+                const float mu2 = mu * mu;
+                A[0] = mu;
+                A[2] = eta;
+                A[4] = xx;
+                A[6] = mu2;
+                if (!(mu2 >= 8.6736174e-19f)) zmu[s] = 1u;  // mu^2 < 2^-60 (or zero)
+            }
         };
-        auto store_y = [&](int kc) {  // 16 tokens of chunk kc from the Y^T accumulator
-            uint32_t yv[kTcSub];
-            ptx::tmem_ld16(tmem + lane_base + Lay::Y_COL + sb * kTcSub, yv);
+        // 8 tokens (half hf of this group's 16) of chunk kc from the Y^T accumulator
+        auto store_y = [&](int kc, int hf) {
+            uint32_t yv[8];
+            ptx::tmem_ld8(tmem + lane_base + Lay::Y_COL + (kc & 1) * kTcC + sb * kTcSub + 8 * hf, yv);
             ptx::tmem_wait_ld();
             if (!ycol_ok || *abort) return;
-            const int t0 = kc * kTcC + sb * kTcSub;
+            const int t0 = kc * kTcC + sb * kTcSub + 8 * hf;
             float* yb = a.y + (((size_t)b * T + t0) * H + h) * DS + kcol;
             const size_t stride = (size_t)H * DS;
 #pragma unroll
-            for (int u = 0; u < kTcSub; ++u)
+            for (int u = 0; u < 8; ++u)
                 if (t0 + u < T) yb[u * stride] = __uint_as_float(yv[u]);
         };
 
@@ -495,33 +508,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ptx::tmem_wait_ld();
             tc_wait(bar_qc, k & 1, abort);  // q and c of chunk k in shared memory
             __syncwarp();
+            const bool zero_mu = zmu[s] != 0u;
+            // per slot: n = |s0|; the gate of token t is g = mu - (eta c/n^2)(p/n) scaled by
+            // n / sqrt(den), den = mu^2 n^2 + (eta c/n)^2 |x_perp|^2, i.e. by
+            // 1/sqrt(mu^2 + (eta c/n^2)^2 |x_perp|^2); kappa/n = (eta c/n^2) by the same factor
             const float n = sqrtf(nsq);
             const float inv_n = 1.f / n, inv_n2 = 1.f / nsq;
-            const float4* ax = aux + s * kTcC + sb * kTcSub;
+            const float4* ax = reinterpret_cast<const float4*>(aux) + (s * (kTcC / 2) + sb * (kTcSub / 2)) * 2;
             float gv[kTcSub], kdv[kTcSub], base[kTcSub];
             float R = 1.f;
 #pragma unroll
-            for (int u = 0; u < kTcSub; ++u) {
-                const float4 z = ax[u];  // mu, eta, |x|^2, mu^2
+            for (int u = 0; u < kTcSub; u += 2) {
+                const float4 z0 = ax[u], z1 = ax[u + 1];  // {mu eta} x2, {|x|^2 mu^2} x2
                 const int tau = sb * kTcSub + u;
-                const float cvu = csm[tau * MS + i];
-                const float qvu = __uint_as_float(uint32_t(qsm[tau * MS + i]) << 16);
-                const float p = __uint_as_float(pr[u]);
-                const float av = z.y * cvu * inv_n;                // eta c / n
-                const float r = p * inv_n2;                        // p / n^2
-                const float perp2 = fmaxf(fmaf(-p, r, z.z), 0.f);  // |x_perp|^2
-                const float den = fmaf(av * av, perp2, z.w * nsq);
-                const bool ok = den > 0.f;
-                const float bn = ok ? n * ptx::rsqrt_nr(den) : 0.f;  // n / sqrt(den)
-                const float g = ok ? bn * fmaf(-av, r, z.x) : 1.f;
-                gv[u] = g;
-                kdv[u] = bn * av;                                   // kappa for now
-                R *= g;
-                base[u] = qvu * R;                                  // q_t prod_{16sb..t} g
+                const float2 cc = make_float2(csm[tau * MS + i], csm[(tau + 1) * MS + i]);
+                const float2 qq = make_float2(__uint_as_float(uint32_t(qsm[tau * MS + i]) << 16),
+                                              __uint_as_float(uint32_t(qsm[(tau + 1) * MS + i]) << 16));
+                const float2 pp = make_float2(__uint_as_float(pr[u]), __uint_as_float(pr[u + 1]));
+                const float2 mu = make_float2(z0.x, z0.y), eta = make_float2(z0.z, z0.w);
+                const float2 xx = make_float2(z1.x, z1.y), mu2 = make_float2(z1.z, z1.w);
+                const float2 e2 = ptx::f2mul(cc, ptx::f2mul(eta, ptx::f2(inv_n2)));  // eta c / n^2
+                const float2 pn = ptx::f2mul(pp, ptx::f2(inv_n));                    // p / n
+                float2 perp = ptx::f2fma(ptx::f2neg(pn), pn, xx);                     // |x_perp|^2
+                perp.x = fmaxf(perp.x, 0.f);
+                perp.y = fmaxf(perp.y, 0.f);
+                const float2 den = ptx::f2fma(ptx::f2mul(e2, e2), perp, mu2);
+                const float2 bn = ptx::rsqrt2_nr(den);
+                float2 g = ptx::f2mul(bn, ptx::f2fma(ptx::f2neg(e2), pn, mu));
+                float2 kn = ptx::f2mul(bn, e2);                                       // kappa / n
+                if (zero_mu) {  // denormal-safe normaliser; a zero-norm update keeps the slot
+                    const float2 bs = make_float2(den.x > 0.f ? ptx::rsqrt_nr(den.x) : 0.f,
+                                                  den.y > 0.f ? ptx::rsqrt_nr(den.y) : 0.f);
+                    g = ptx::f2mul(bs, ptx::f2fma(ptx::f2neg(e2), pn, mu));
+                    kn = ptx::f2mul(bs, e2);
+                    if (!(den.x > 0.f)) { g.x = 1.f; kn.x = 0.f; }
+                    if (!(den.y > 0.f)) { g.y = 1.f; kn.y = 0.f; }
+                }
+                gv[u] = g.x;
+                gv[u + 1] = g.y;
+                kdv[u] = kn.x;
+                kdv[u + 1] = kn.y;
+                R *= g.x;
+                const float R0 = R;
+                R *= g.y;
+                const float2 qb = ptx::f2mul(qq, make_float2(R0, R));              // q_t prod_{16sb..t} g
+                base[u] = qb.x;
+                base[u + 1] = qb.y;
             }
             if (active) gsub[sb * MS + i] = R;
             {   // KD(t) = kappa_t / prod_{16sb..t} g: one reciprocal, then a backward product
-                float inv = ptx::rcp_nr(copysignf(fmaxf(fabsf(R), 1e-37f), R));
+                float inv = n * ptx::rcp_nr(copysignf(fmaxf(fabsf(R), 1e-37f), R));
 #pragma unroll
                 for (int u = kTcSub - 1; u >= 0; --u) {
                     kdv[u] *= inv;
@@ -536,7 +572,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     *reinterpret_cast<uint4*>(kd + ptx::sw128_chunk(i, g8)) = pack8(kdv + 8 * hh);
                 }
             }
-            ptx::named_bar(BAR_G, N_WM);  // sub-chunk products known; q and c free for chunk k+1
+            ptx::tc_fence_before();
+            ptx::named_bar(BAR_G, N_WM);  // sub-chunk products known; q, c and D1 read
+            ptx::tc_fence_after();
+            if (tid == 0) zmu[s] = 0u;  // every worker read it before the barrier
             float G[NSUB];
 #pragma unroll
             for (int g = 0; g < NSUB; ++g) G[g] = active ? gsub[g * MS + i] : 1.f;
@@ -563,10 +602,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int hh = 0; hh < 2; ++hh) {
                         uint4 u4 = make_uint4(0u, 0u, 0u, 0u);
                         if (bb < sb) {
-                            float v[8];
+                            uint32_t w[4];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) v[e] = base[8 * hh + e] * cgb;
-                            u4 = pack8(v);
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 v = ptx::f2mul(make_float2(base[8 * hh + 2 * e], base[8 * hh + 2 * e + 1]),
+                                                            ptx::f2(cgb));
+                                w[e] = ptx::pack_bf16x2(v.x, v.y);
+                            }
+                            u4 = make_uint4(w[0], w[1], w[2], w[3]);
                         }
                         *reinterpret_cast<uint4*>(qr + bb * Lay::ROW_TILE + ptx::sw128_chunk(i, 2 * sb + hh)) = u4;
                     }
@@ -576,15 +619,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const float ksc = active ? F * inv_sig : 0.f;
                 uint32_t hw[8], lw[8];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float v[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = kdv[8 * hh + e] * ksc;
-                    uint4 hi, lo;
-                    split8(v, hi, lo);
-                    hw[4 * hh + 0] = hi.x; hw[4 * hh + 1] = hi.y; hw[4 * hh + 2] = hi.z; hw[4 * hh + 3] = hi.w;
-                    lw[4 * hh + 0] = lo.x; lw[4 * hh + 1] = lo.y; lw[4 * hh + 2] = lo.z; lw[4 * hh + 3] = lo.w;
-                }
+                for (int e = 0; e < 8; ++e)
+                    split2(ptx::f2mul(make_float2(kdv[2 * e], kdv[2 * e + 1]), ptx::f2(ksc)), hw[e], lw[e]);
                 ptx::tmem_st8(tmem + lane_base + Lay::KSHI_TCOL + 8 * sb, hw);
                 ptx::tmem_st8(tmem + lane_base + Lay::KSLO_TCOL + 8 * sb, lw);
             }
@@ -600,18 +636,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             ptx::tmem_wait_st();
             sigma = pre ? 1.f : sig_c;
-            if (k > 0) {  // y of chunk k-1 (before this chunk's read-out GEMM reuses Y^T)
-                tc_wait(bar_y, (k - 1) & 1, abort);
-                __syncwarp();
-                ptx::tc_fence_after();
-                store_y(k - 1);
-            }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::named_bar(BAR_A, N_WM);
 
-            // ---- phase B1: state after the chunk (S = sigma T') and the next S0 operand
-            tc_wait(bar_t, k & 1, abort);  // G4 and G7 complete
+            // ---- phase B: y of the previous chunk (first half), while G7 and G4 run
+            if (k > 0) {
+                tc_wait(bar_y, (k - 1) & 1, abort);
+                __syncwarp();
+                ptx::tc_fence_after();
+                store_y(k - 1, 0);
+            }
+            // state after the chunk (S = sigma T') and the next chunk's S0 operands
+            tc_wait(bar_t, k & 1, abort);  // G7 complete
             __syncwarp();
             ptx::tc_fence_after();
             const bool renorm = !(fabsf(sigma) >= 2.3283064e-10f && fabsf(sigma) <= 4.2949673e9f);
@@ -621,15 +658,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 float v[DCOL];
                 ptx::tmem_ld<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
                 ptx::tmem_wait_ld();
-                float ts = 0.f;
+                float2 ts = ptx::f2(0.f);
 #pragma unroll
-                for (int e = 0; e < DCOL; ++e) {
-                    v[e] = __uint_as_float(r[e]) * sigma;  // true state
-                    ts = fmaf(v[e], v[e], ts);
-                    if (renorm) r[e] = __float_as_uint(v[e]);
+                for (int e = 0; e < DCOL; e += 2) {
+                    const float2 vv = ptx::f2mul(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])),
+                                                 ptx::f2(sigma));  // true state
+                    ts = ptx::f2fma(vv, vv, ts);
+                    v[e] = vv.x;
+                    v[e + 1] = vv.y;
                 }
-                if (any_renorm) ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
-                if (active) tsqp[sb * MS + i] = ts;
+                if (any_renorm) {
+#pragma unroll
+                    for (int e = 0; e < DCOL; ++e)
+                        if (renorm) r[e] = __float_as_uint(v[e]);
+                    ptx::tmem_st<DCOL>(tmem + lane_base + Lay::T_COL + sb * DCOL, r);
+                }
+                if (active) tsqp[sb * MS + i] = ts.x + ts.y;
                 if (k + 1 == nch) {
                     if (active) {
                         float* So = a.S_out + ((size_t)bh * MS + i) * DS + sb * DCOL;
@@ -638,6 +682,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             *reinterpret_cast<float4*>(So + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                     }
                 } else {
+                    tc_wait(bar_g4, k & 1, abort);  // the read-out GEMM is done with S0hi
+                    __syncwarp();
                     store_s0(sb * DCOL, v);
                 }
                 ptx::tmem_wait_st();
@@ -650,8 +696,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (active)
 #pragma unroll
                 for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+            if (k > 0) store_y(k - 1, 1);  // second half of the previous chunk's y
 
-            // ---- phase B2: masked scores, next chunk's per-token inputs
+            // ---- masked scores, next chunk's per-token inputs
             tc_wait(bar_p5, k & 1, abort);  // G5 complete
             __syncwarp();
             ptx::tc_fence_after();
@@ -681,7 +728,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_wait(bar_y, (nch - 1) & 1, abort);
             __syncwarp();
             ptx::tc_fence_after();
-            store_y(nch - 1);
+            store_y(nch - 1, 0);
+            store_y(nch - 1, 1);
         }
     }
     ptx::tc_fence_before();

@@ -3,6 +3,7 @@
 // and the shared-memory matrix descriptors of 128-byte-swizzled bf16 tiles.
 #pragma once
 #include <cuda.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace lattice {
@@ -121,6 +122,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
         : "r"(taddr));
 }
 // 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -255,6 +262,21 @@ __device__ __forceinline__ float rsqrt_nr(float x) {
     const float y = rsqrtf(x);
     const float e = fmaf(-x * y, y, 1.f);
     return fmaf(0.5f * y, e, y);
+}
+// Paired fp32 arithmetic (sm_100: one instruction for two lanes of fp32 work,
+// each lane rounded to nearest like its scalar counterpart).
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 f2neg(float2 a) { return make_float2(-a.x, -a.y); }
+// Two reciprocal square roots, each refined by one Newton step (see rsqrt_nr).
+__device__ __forceinline__ float2 rsqrt2_nr(float2 x) {
+    float2 y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y.x) : "f"(x.x));
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y.y) : "f"(x.y));
+    const float2 e = f2fma(f2neg(f2mul(x, y)), y, f2(1.f));
+    return f2fma(f2mul(y, f2(0.5f)), e, y);
 }
 __device__ __forceinline__ float rcp_nr(float x) {
     float y;
