@@ -376,13 +376,14 @@ def main():
     value = job_tokens_per_s(world, w, ms)
 
     # roofline of the (single) kernel of the step
-    tc = L.chunk_impl(w.m, w.d, w.chunk) == "tcgen05"
+    kimpl = L.chunk_impl(w.B, w.H, w.m, w.d, w.chunk)
+    tc = kimpl.startswith("tcgen05")
     alg_b = scan_alg_bytes(w)
     kern_ms = statistics.mean(times)
     achieved = alg_b / (kern_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / pk["hbm_gbs"], "traffic": None,
-            "kernel": "chunk_tc_kernel" if tc else "scan_simt_kernel<chunked>",
+            "kernel": {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(kimpl, "scan_simt_kernel<chunked>"),
             "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"}
     if tc:
         fl = chunk_mma_flops(w, w.chunk)

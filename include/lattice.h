@@ -75,15 +75,31 @@ typedef enum { LATTICE_F32 = 0, LATTICE_BF16 = 1 } lattice_dtype;
 /* Objective (§3.1.1). Only the similarity objective (h_t = -x_t) is built. */
 typedef enum { LATTICE_SIM = 0, LATTICE_DEC = 1 } lattice_mode;
 
-/* Kernel choice for chunked scans. AUTO picks the tensor-core kernel when the
- * shape allows it. SIMT forces the CUDA-core kernel. TCGEN05 requires the
- * tensor-core kernel and returns LATTICE_ERR_UNSUPPORTED when it cannot run. */
-typedef enum { LATTICE_IMPL_AUTO = 0, LATTICE_IMPL_SIMT = 1, LATTICE_IMPL_TCGEN05 = 2 } lattice_impl;
+/* Kernel choice for chunked scans.
+ *   AUTO            picks the fastest kernel that can run the shape (see
+ *                   lattice_chunk_impl).
+ *   SIMT            the CUDA-core kernel (any chunk size, fp32 or bf16 x/q).
+ *   TCGEN05         the tensor-core kernel with one CTA per sequence
+ *                   (chunk 64, bf16 x and q, m and d in {64, 128}).
+ *   TCGEN05_SPLIT   the tensor-core kernel with each sequence's 64 slots split
+ *                   over a cluster of 4 CTAs (chunk 64, bf16 x and q, m = 64,
+ *                   d in {64, 128}); for batches with fewer sequences than SMs.
+ * An explicit choice that cannot run the shape returns LATTICE_ERR_UNSUPPORTED.
+ * All tensor-core choices compute the same chunked form; they differ only in
+ * fp32 summation order. */
+typedef enum {
+    LATTICE_IMPL_AUTO = 0,
+    LATTICE_IMPL_SIMT = 1,
+    LATTICE_IMPL_TCGEN05 = 2,
+    LATTICE_IMPL_TCGEN05_SPLIT = 3
+} lattice_impl;
 
-/* Which kernel LATTICE_IMPL_AUTO runs for a chunked scan of this shape:
- * returns LATTICE_IMPL_TCGEN05 or LATTICE_IMPL_SIMT (chunk_size 1 is always
- * LATTICE_IMPL_SIMT). Pure host function; launches nothing. */
-lattice_impl lattice_chunk_impl(int m, int d, int chunk_size, lattice_dtype x_dtype,
+/* Which kernel LATTICE_IMPL_AUTO runs for a chunked scan of B x H sequences of
+ * this shape: TCGEN05_SPLIT when it applies and B*H*4 CTAs fit on the current
+ * device's SMs at once, else TCGEN05 when it applies, else SIMT (chunk_size 1
+ * is always SIMT). Host function; launches nothing (without a device it
+ * assumes 148 SMs). */
+lattice_impl lattice_chunk_impl(int B, int H, int m, int d, int chunk_size, lattice_dtype x_dtype,
                                 lattice_dtype q_dtype);
 
 /* Whole-sequence forward (the paper's lattice_compress, Appendix D).

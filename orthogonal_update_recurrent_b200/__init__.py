@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblattice.
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
 _F32, _BF16 = 0, 1
-_IMPL = {"auto": 0, "simt": 1, "tcgen05": 2}
+_IMPL = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3}
 _lib = None
 
 
@@ -61,7 +61,7 @@ def lib() -> ctypes.CDLL:
         L.lattice_status_string.argtypes = [i]
         L.lattice_status_string.restype = ctypes.c_char_p
         L.lattice_version.argtypes = []
-        L.lattice_chunk_impl.argtypes = [i, i, i, i, i]
+        L.lattice_chunk_impl.argtypes = [i, i, i, i, i, i, i]
         L.lattice_last_cuda_error.argtypes = []
         L.lattice_last_cuda_error.restype = ctypes.c_char_p
         for f in ("lattice_scan_fwd", "lattice_scan_fwd_impl", "lattice_step", "lattice_readout",
@@ -173,11 +173,13 @@ def readout(S: torch.Tensor, q: torch.Tensor, y: Optional[torch.Tensor] = None,
     return y
 
 
-def chunk_impl(m: int, d: int, chunk: int, x_dtype=torch.bfloat16, q_dtype=torch.bfloat16) -> str:
-    """Name of the kernel the automatic choice runs for a chunked scan: "tcgen05" or "simt"."""
+def chunk_impl(B: int, H: int, m: int, d: int, chunk: int, x_dtype=torch.bfloat16,
+               q_dtype=torch.bfloat16) -> str:
+    """Name of the kernel the automatic choice runs for a chunked scan of B x H sequences:
+    "tcgen05_split", "tcgen05" or "simt"."""
     dt = lambda t: _BF16 if t == torch.bfloat16 else _F32
-    code = lib().lattice_chunk_impl(m, d, chunk, dt(x_dtype), dt(q_dtype))
-    return {1: "simt", 2: "tcgen05"}[code]
+    code = lib().lattice_chunk_impl(B, H, m, d, chunk, dt(x_dtype), dt(q_dtype))
+    return {1: "simt", 2: "tcgen05", 3: "tcgen05_split"}[code]
 
 
 def device_status(stream=None) -> int:

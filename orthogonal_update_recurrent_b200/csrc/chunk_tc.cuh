@@ -490,10 +490,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         if (nch > 0) ptx::named_bar(BAR_INIT, N_WM);
-        float nsq = 0.f;
-        if (active)
+        // n = |s0|, 1/n and 1/n^2 of this lane's slot for the next chunk's gates
+        float n, inv_n, inv_n2;
+        auto load_norm = [&]() {
+            float nsq = 0.f;
+            if (active)
 #pragma unroll
-            for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+                for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+            if (!active) nsq = 1.f;
+            inv_n = ptx::rsqrt_nr(nsq);
+            n = nsq * inv_n;
+            inv_n2 = inv_n * inv_n;
+        };
+        load_norm();
 
         for (int k = 0; k < nch; ++k) {
             const int s = k & 1;
@@ -512,8 +521,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // per slot: n = |s0|; the gate of token t is g = mu - (eta c/n^2)(p/n) scaled by
             // n / sqrt(den), den = mu^2 n^2 + (eta c/n)^2 |x_perp|^2, i.e. by
             // 1/sqrt(mu^2 + (eta c/n^2)^2 |x_perp|^2); kappa/n = (eta c/n^2) by the same factor
-            const float n = sqrtf(nsq);
-            const float inv_n = 1.f / n, inv_n2 = 1.f / nsq;
             const float4* ax = reinterpret_cast<const float4*>(aux) + (s * (kTcC / 2) + sb * (kTcSub / 2)) * 2;
             float gv[kTcSub], kdv[kTcSub], base[kTcSub];
             float R = 1.f;
@@ -587,7 +594,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             const float sig_c = sigma * AC;                     // sigma * A_C
             const bool pre = !(fabsf(sig_c) >= 7.8886091e-31f);  // 2^-100, or not finite
-            const float inv_sig = pre ? 1.f : 1.f / sig_c;
+            const float inv_sig = pre ? 1.f : ptx::rcp_nr(sig_c);  // |sig_c| >= 2^-100: a normal float
             if (active) {
                 // query operands of the other sub-chunks' key blocks for this group's tokens:
                 // plain products for the earlier blocks, zeros for the later ones
@@ -692,10 +699,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::named_bar(BAR_S0, N_WM);
-            nsq = 0.f;
-            if (active)
-#pragma unroll
-                for (int g = 0; g < NSUB; ++g) nsq += tsqp[g * MS + i];
+            load_norm();
             if (k > 0) store_y(k - 1, 1);  // second half of the previous chunk's y
 
             // ---- masked scores, next chunk's per-token inputs

@@ -9,6 +9,7 @@
 #include "scan_simt.cuh"
 #include "step.cuh"
 #include "chunk_tc.cuh"
+#include "chunk_split.cuh"
 
 using namespace lattice;
 
@@ -29,6 +30,16 @@ size_t dsize(lattice_dtype t) { return t == LATTICE_BF16 ? 2 : 4; }
 bool d_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
 thread_local char g_last_error[256] = "";
+
+// SMs of the current device (148 on B200; also the answer without a device).
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        return n;
+    cudaGetLastError();  // clear the error of a host without a device
+    return 148;
+}
 
 lattice_status cuda_fail(cudaError_t e) {
     snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
@@ -129,11 +140,14 @@ const char* lattice_status_string(lattice_status s) {
     return "unknown status";
 }
 
-lattice_impl lattice_chunk_impl(int m, int d, int chunk_size, lattice_dtype x_dtype,
+lattice_impl lattice_chunk_impl(int B, int H, int m, int d, int chunk_size, lattice_dtype x_dtype,
                                 lattice_dtype q_dtype) {
-    if (chunk_size > 1 && chunk_tc_supported(m, d, chunk_size, x_dtype == LATTICE_BF16,
-                                             q_dtype == LATTICE_BF16))
-        return LATTICE_IMPL_TCGEN05;
+    if (chunk_size <= 1) return LATTICE_IMPL_SIMT;
+    const bool xb = x_dtype == LATTICE_BF16, qb = q_dtype == LATTICE_BF16;
+    if (chunk_split_supported(m, d, chunk_size, xb, qb) && B >= 1 && H >= 1 &&
+        (long long)B * H * kSpNC <= sm_count())
+        return LATTICE_IMPL_TCGEN05_SPLIT;
+    if (chunk_tc_supported(m, d, chunk_size, xb, qb)) return LATTICE_IMPL_TCGEN05;
     return LATTICE_IMPL_SIMT;
 }
 
@@ -144,7 +158,8 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
                                      lattice_mode mode, lattice_impl impl, void* stream) {
     if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return LATTICE_ERR_INVALID_ARG;
     if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
-    if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05)
+    if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05 &&
+        impl != LATTICE_IMPL_TCGEN05_SPLIT)
         return LATTICE_ERR_INVALID_ARG;
     if (mode != LATTICE_SIM) return mode == LATTICE_DEC ? LATTICE_ERR_UNSUPPORTED : LATTICE_ERR_INVALID_ARG;
     lattice_status ds = check_dims(B, H, m, d);
@@ -178,12 +193,17 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
     ScanArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, S_out, y,
                B, T, H, m, chunk_size};
     if (chunk_size == 1) {
-        if (impl == LATTICE_IMPL_TCGEN05) return LATTICE_ERR_UNSUPPORTED;
+        if (impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT) return LATTICE_ERR_UNSUPPORTED;
         return launch_scan_simt<false>(a, d, st);
     }
-    const bool tc_ok = chunk_tc_supported(m, d, chunk_size, a.x_bf16, a.q_bf16);
-    if (impl == LATTICE_IMPL_TCGEN05 && !tc_ok) return LATTICE_ERR_UNSUPPORTED;
-    if (tc_ok && impl != LATTICE_IMPL_SIMT) {
+    if (impl == LATTICE_IMPL_AUTO) impl = lattice_chunk_impl(B, H, m, d, chunk_size, x_dtype, q_dtype);
+    if (impl == LATTICE_IMPL_TCGEN05_SPLIT) {
+        if (!chunk_split_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
+        cudaError_t e = launch_chunk_split(a, d, st);
+        return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
+    }
+    if (impl == LATTICE_IMPL_TCGEN05) {
+        if (!chunk_tc_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
         cudaError_t e = launch_chunk_tc(a, d, st);
         return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
     }
