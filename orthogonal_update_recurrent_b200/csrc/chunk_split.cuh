@@ -72,7 +72,8 @@ struct SpLayout {
     static constexpr uint32_t GSUB_OFF = AUX_OFF + 2 * kTcC * 16;    // [4][16] float
     static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * kSpSlots * 4;  // [4][16] float
     static constexpr uint32_t SIG_OFF = TSQ_OFF + 4 * kSpSlots * 4;   // [2][16] float
-    static constexpr uint32_t BAR_OFF = SIG_OFF + 2 * kSpSlots * 4;   // 14 mbarriers
+    static constexpr uint32_t PSC_OFF = SIG_OFF + 2 * kSpSlots * 4;   // [16] float: rescale factors
+    static constexpr uint32_t BAR_OFF = PSC_OFF + kSpSlots * 4;       // 14 mbarriers
     static constexpr uint32_t MISC_OFF = BAR_OFF + 14 * 8;
     static constexpr uint32_t BYTES = MISC_OFF + 64;
     static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;
@@ -148,14 +149,18 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
     volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 4);
     volatile uint32_t* zmu = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 8);
+    // per chunk parity: set when some slot's old state must be rescaled before the state-update GEMM
+    volatile uint32_t* pflag = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 16);
+    float* psc = reinterpret_cast<float*>(smem + Lay::PSC_OFF);
     float4* aux = reinterpret_cast<float4*>(smem + Lay::AUX_OFF);
     float* gsub = reinterpret_cast<float*>(smem + Lay::GSUB_OFF);
     float* tsqp = reinterpret_cast<float*>(smem + Lay::TSQ_OFF);
     float* sig = reinterpret_cast<float*>(smem + Lay::SIG_OFF);
 
     // named barriers: workers + MMA warp (INIT, A, S0), workers + TMA warp (G),
-    // read-out warps (arrive) + MMA warp (P), workers alone (N)
-    constexpr uint32_t BAR_INIT = 1, BAR_G = 2, BAR_A = 3, BAR_S0 = 4, BAR_P = 5, BAR_N = 6;
+    // read-out warps (arrive) + MMA warp (P), workers alone (N), workers + MMA warp
+    // only in chunks with a rescale (T)
+    constexpr uint32_t BAR_INIT = 1, BAR_G = 2, BAR_A = 3, BAR_S0 = 4, BAR_P = 5, BAR_N = 6, BAR_T = 7;
     constexpr uint32_t N_WM = kSpWorkers + 32, N_RM = kSpReadout + 32;
 
     if (warp == MMA_WARP) {
@@ -170,6 +175,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             *abort = 0u;
             zmu[0] = 0u;
             zmu[1] = 0u;
+            pflag[0] = 0u;
+            pflag[1] = 0u;
             ptx::fence_mbar_init();
         }
         __syncwarp();
@@ -220,7 +227,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         for (int k = 0; k < nch; ++k) {
             const uint32_t xo = (k & 1) * Lay::X_STAGE;
             const uint32_t ycol = Lay::Y_COL + (k & 1) * DS;
-            ptx::named_bar(BAR_A, N_WM);  // KS, QR, KD written; T^T rescaled
+            ptx::named_bar(BAR_A, N_WM);  // KS, QR, KD written
+            if (pflag[k & 1]) ptx::named_bar(BAR_T, N_WM);  // T^T rescaled (rare)
             ptx::tc_fence_after();
             if (tc_live(abort)) {
                 // G7: T^T += X^T . KS  (M = d, N = 16, K = C); both MN-major
@@ -676,44 +684,43 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 const uint32_t o = ptx::sw128_off(tau, s0);
                 *reinterpret_cast<uint2*>(smem + Lay::KSHI_OFF + o) = make_uint2(hw[0], hw[1]);
                 *reinterpret_cast<uint2*>(smem + Lay::KSLO_OFF + o) = make_uint2(lw[0], lw[1]);
-                if (tau == 0)
+                if (tau == 0) {
                     *reinterpret_cast<float4*>(sig + (s ^ 1) * kSpSlots + s0) =
                         make_float4(sig_new[0], sig_new[1], sig_new[2], sig_new[3]);
-            }
-            {   // state side: columns whose decayed old state fell below fp32 resolution
-                float sc[8];
-                bool any = false;
-#pragma unroll
-                for (int h4 = 0; h4 < 2; ++h4) {
-                    float4 gq[4];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) gq[c] = *reinterpret_cast<const float4*>(gsub + c * kSpSlots + 8 * j + 4 * h4);
-                    const float4 sg = *reinterpret_cast<const float4*>(sig + s * kSpSlots + 8 * j + 4 * h4);
-                    const float G4s[4][4] = {{gq[0].x, gq[1].x, gq[2].x, gq[3].x}, {gq[0].y, gq[1].y, gq[2].y, gq[3].y},
-                                             {gq[0].z, gq[1].z, gq[2].z, gq[3].z}, {gq[0].w, gq[1].w, gq[2].w, gq[3].w}};
-                    const float sgv[4] = {sg.x, sg.y, sg.z, sg.w};
+                    float sc[4];
+                    bool any = false;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
+                        const float G4[4] = {G[0][c], G[1][c], G[2][c], G[3][c]};
                         float F, AC, sig_c;
                         bool pre;
-                        sp_decay(G4s[c], 0, sgv[c], F, AC, sig_c, pre);
-                        sc[4 * h4 + c] = pre ? (isfinite(sig_c) ? sig_c : 0.f) : 1.f;
+                        sp_decay(G4, q, sgv[c], F, AC, sig_c, pre);
+                        sc[c] = pre ? (isfinite(sig_c) ? sig_c : 0.f) : 1.f;
                         any = any || pre;
                     }
-                }
-                if (any) {  // the same for every lane of the warp
-                    uint32_t r[8];
-                    ptx::tmem_ld8(tmem + lane_base + Lay::T_COL + 8 * j, r);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * sc[c]);
-                    ptx::tmem_st8(tmem + lane_base + Lay::T_COL + 8 * j, r);
-                    ptx::tmem_wait_st();
+                    *reinterpret_cast<float4*>(psc + s0) = make_float4(sc[0], sc[1], sc[2], sc[3]);
+                    if (any) pflag[s] = 1u;
                 }
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::named_bar(BAR_A, N_WM);
+            if (pflag[s]) {  // the same decision as the MMA warp's
+                // columns whose decayed old state fell below fp32 resolution: T <- sigma A_C T
+                const float4 sa = *reinterpret_cast<const float4*>(psc + 8 * j);
+                const float4 sb4 = *reinterpret_cast<const float4*>(psc + 8 * j + 4);
+                const float sc[8] = {sa.x, sa.y, sa.z, sa.w, sb4.x, sb4.y, sb4.z, sb4.w};
+                ptx::tc_fence_after();
+                uint32_t r[8];
+                ptx::tmem_ld8(tmem + lane_base + Lay::T_COL + 8 * j, r);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 8; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * sc[c]);
+                ptx::tmem_st8(tmem + lane_base + Lay::T_COL + 8 * j, r);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::named_bar(BAR_T, N_WM);
+            }
 
             // ---- phase B: state after the chunk, next S0 operands
             tc_wait(bar_t, k & 1, abort);
@@ -754,6 +761,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 // the next chunk's slot norms, while the projection GEMM runs
                 if (k + 1 < nch) col_norms(v);
             }
+            if (tid == 0) pflag[s] = 0u;  // read by every worker and the MMA warp before BAR_S0
             if (tau == 0) {  // renormalised slots restart at sigma = 1
                 float* sp = sig + (s ^ 1) * kSpSlots + s0;
 #pragma unroll
