@@ -103,6 +103,15 @@ def job_tokens_per_s(world: int, w: LI.Workload, ms_per_step: float) -> float:
     return world * w.B * w.T / (ms_per_step * 1e-3)
 
 
+# DRAM bytes (read + write) per launch, from one `ncu --set full` capture of each kernel on
+# each workload (the profile summaries keep the commands). None where no capture exists.
+CAPTURED_TRAFFIC = {
+    ("chunk_split_kernel", "small_train"): 34.41e6 + 0.19e6,
+    ("chunk_split_kernel", "long_ctx"): 676.22e6 + 500.96e6,
+    ("chunk_tc_kernel", "mid_layer"): 550.62e6 + 240.43e6,
+}
+
+
 # -------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -381,9 +390,10 @@ def main():
     alg_b = scan_alg_bytes(w)
     kern_ms = statistics.mean(times)
     achieved = alg_b / (kern_ms * 1e-3) / 1e9
+    kname = {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(kimpl, "scan_simt_kernel<chunked>")
     roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / pk["hbm_gbs"], "traffic": None,
-            "kernel": {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(kimpl, "scan_simt_kernel<chunked>"),
+            "frac": achieved / pk["hbm_gbs"], "traffic": CAPTURED_TRAFFIC.get((kname, w0.name)),
+            "kernel": kname,
             "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"}
     if tc:
         fl = chunk_mma_flops(w, w.chunk)
@@ -434,6 +444,10 @@ def main():
                        "hbm_gbs": ab / (kms * 1e-3) / 1e9, "hbm_frac": ab / (kms * 1e-3) / 1e9 / pk["hbm_gbs"],
                        "alg_bytes": ab}
                 fl = chunk_mma_flops(wn, wn.chunk)
+                kn = {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(
+                    L.chunk_impl(wn.B, wn.H, wn.m, wn.d, wn.chunk), "scan_simt_kernel<chunked>")
+                ent["kernel"] = kn
+                ent["traffic"] = CAPTURED_TRAFFIC.get((kn, name))
                 ent["tensor_tflops"] = fl / (kms * 1e-3) / 1e12
                 ent["frac_of_binding_roofline"] = 1e3 * max(ab / (pk["hbm_gbs"] * 1e9),
                                                             fl / (pk["bf16_tflops"] * 1e12)) / kms
