@@ -48,6 +48,14 @@ def _load():
             f = getattr(lib, name)
             f.argtypes = [i, i, i, i, i, i, _D, _D, _D, _D, _D, _D, _D, _D, i]
             f.restype = ll
+        lib.oracle_exact_scan_mode.argtypes = [i] + scan_args
+        lib.oracle_exact_scan_mode.restype = ll
+        for name in ("oracle_chunked_scan_mode", "oracle_chunked_matrix_scan_mode"):
+            f = getattr(lib, name)
+            f.argtypes = [i, i, i, i, i, i, i, _D, _D, _D, _D, _D, _D, _D, _D, i]
+            f.restype = ll
+        lib.oracle_write_input.argtypes = [i, i, i, _D, _D, _D, _D]
+        lib.oracle_write_input.restype = None
         lib.oracle_readout.argtypes = [i, i, i, i, _D, _D, _D]
         lib.oracle_readout.restype = None
         lib.oracle_osr_write.argtypes = [i, _D, _D, ctypes.c_double, ctypes.c_double,
@@ -78,12 +86,18 @@ def _threads(n: Optional[int]) -> int:
         return os.cpu_count() or 1
 
 
+_MODES = {"sim": 0, "dec": 1}
+
+
 def scan(x, c, q, mu, S0, eta=None, chunk: int = 1, form: str = "token",
-         nthreads: Optional[int] = None):
+         nthreads: Optional[int] = None, mode: str = "sim"):
     """Whole-sequence forward. x[B][T][H][d], c/q[B][T][H][m], mu/eta[B][T][H],
     S0[B][H][m][d]. chunk == 1: exact recurrence; chunk > 1: Eq. 17 chunked
     recurrence, evaluated token by token (form="token") or through the
-    chunk-level closed form (form="matrix"). Returns (y, S_T, n_degenerate)."""
+    chunk-level closed form (form="matrix"). mode "sim": similarity objective
+    (h = -x); "dec": reconstruction objective (h = phi(S) c - x).
+    Returns (y, S_T, n_degenerate)."""
+    md = _MODES[mode]
     x, c, q, mu, S0 = map(_f64, (x, c, q, mu, S0))
     eta = None if eta is None else _f64(eta)
     B, T, H, d = x.shape
@@ -96,17 +110,17 @@ def scan(x, c, q, mu, S0, eta=None, chunk: int = 1, form: str = "token",
     nt = _threads(nthreads)
     args = (_p(x), _p(c), _p(q), _p(mu), _p(eta), _p(S0), _p(S), _p(y), nt)
     if chunk == 1 and form == "token":
-        deg = lib.oracle_exact_scan(B, T, H, m, d, *args)
+        deg = lib.oracle_exact_scan_mode(md, B, T, H, m, d, *args)
     elif form == "token":
-        deg = lib.oracle_chunked_scan(B, T, H, m, d, chunk, *args)
+        deg = lib.oracle_chunked_scan_mode(md, B, T, H, m, d, chunk, *args)
     elif form == "matrix":
-        deg = lib.oracle_chunked_matrix_scan(B, T, H, m, d, chunk, *args)
+        deg = lib.oracle_chunked_matrix_scan_mode(md, B, T, H, m, d, chunk, *args)
     else:
         raise ValueError(form)
     return y, S, int(deg)
 
 
-def step(S, x, c, q, mu, eta=None, nthreads: Optional[int] = None):
+def step(S, x, c, q, mu, eta=None, nthreads: Optional[int] = None, mode: str = "sim"):
     """One decode step (the exact recurrence with T = 1). S[B][H][m][d],
     x[B][H][d], c/q[B][H][m], mu/eta[B][H]. Returns (y[B][H][d], S_new, n_degenerate)."""
     x = _f64(x)[:, None]
@@ -114,8 +128,17 @@ def step(S, x, c, q, mu, eta=None, nthreads: Optional[int] = None):
     q = _f64(q)[:, None]
     mu = _f64(mu)[:, None]
     eta = None if eta is None else _f64(eta)[:, None]
-    y, S_new, deg = scan(x, c, q, mu, S, eta=eta, chunk=1, nthreads=nthreads)
+    y, S_new, deg = scan(x, c, q, mu, S, eta=eta, chunk=1, nthreads=nthreads, mode=mode)
     return y[:, 0], S_new, deg
+
+
+def write_input(S, c, x, mode: str = "dec"):
+    """-h of one token against the slots S[m][d] (x for "sim"; x - sum_i c_i s_i/|s_i| for "dec")."""
+    S, c, x = _f64(S), _f64(c), _f64(x)
+    m, d = S.shape
+    out = np.zeros(d)
+    _load().oracle_write_input(_MODES[mode], m, d, _p(S), _p(c), _p(x), _p(out))
+    return out
 
 
 def readout(S, q):

@@ -24,6 +24,10 @@
  *   - Appendix D (Implementation): argument shapes and the read-out y = q S_t
  *     with the updated state.
  *
+ *   - §3.1.1 eq. (decoding_stateNorm_loss) and eq. (decoding_recurrence): the
+ *     reconstruction objective writes the part of the reconstruction error
+ *     e = phi(S) c - x orthogonal to each slot (h_t = e_t in eq. OSR).
+ *
  * Readings of points the paper leaves open (each is listed in the design notes):
  *   - slots are rows of S ([m][d]), as in the Appendix D listing;
  *   - the normaliser targets the unit sphere (§3.2), with no epsilon;
@@ -37,7 +41,12 @@
  *     the exact recurrence (for unit-norm states);
  *   - D_S uses "minus" (Pythagoras, §3.2), clipped at zero;
  *   - a slot whose update has zero norm (mu = 0 and no orthogonal write) is
- *     left unchanged and counted.
+ *     left unchanged and counted;
+ *   - the reconstruction objective's step is -eta (c_i/|s_i|) P(s_i) e, the
+ *     gradient of eq. (decoding_recurrence) as printed (that of |phi(S) c - x|^2 / 2);
+ *     its error e is taken from the state the token's projection uses: the
+ *     current state (exact recurrence) or the chunk-start state (Eq. 17), as in
+ *     the Appendix D listing.
  *
  * Layouts (row-major):  x[B][T][H][d]  c,q[B][T][H][m]  mu,eta[B][T][H]
  *                       S[B][H][m][d]  y[B][T][H][d].   eta == NULL means 1.
@@ -70,6 +79,30 @@ void oracle_osr_write(int d, const double *s, const double *x, double c, double 
         w[k] = mu * s[k] + eta * (c / n) * x_perp;
     }
     if (n2_out) *n2_out = n2;
+}
+
+/* The negated write direction of one token, x_eff = -h_t (§3.1.1 eq. OSR).
+ *   similarity objective (mode 0): h = -x, so x_eff = x;
+ *   reconstruction objective (mode 1, §3.1.1 eq. decoding_stateNorm_loss and
+ *   eq. decoding_recurrence): h = e = phi(S) c - x, the reconstruction error of
+ *   the token with the normalised slots phi(s_i) = s_i/|s_i| (the listing's
+ *   h = k @ Phi - v), so x_eff = x - sum_i c_i s_i/|s_i|.
+ * S is the state the token's projection uses (the current state for the exact
+ * recurrence, the chunk-start state for Eq. 17). A zero slot has no direction
+ * and contributes nothing. */
+void oracle_write_input(int mode, int m, int d, const double *S, const double *c,
+                        const double *x, double *x_eff)
+{
+    for (int k = 0; k < d; ++k) x_eff[k] = x[k];
+    if (mode != 1) return;
+    for (int i = 0; i < m; ++i) {
+        const double *s = S + (size_t)i * d;
+        double n2 = 0.0;
+        for (int k = 0; k < d; ++k) n2 += s[k] * s[k];
+        if (n2 == 0.0) continue;
+        double f = c[i] / sqrt(n2);
+        for (int k = 0; k < d; ++k) x_eff[k] -= f * s[k];
+    }
 }
 
 /* One exact step of the whole state (all m slots) followed by the read-out.
@@ -143,6 +176,7 @@ void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
 
 typedef struct {
     int B, T, H, m, d, C, form; /* form: 0 exact, 1 chunked token-wise, 2 chunked matrix form */
+    int mode;                   /* 0 similarity objective, 1 reconstruction objective */
     const double *x, *c, *q, *mu, *eta, *S0;
     double *S_out, *y;
     long long degenerate;
@@ -150,19 +184,20 @@ typedef struct {
     pthread_mutex_t lock;
 } job_t;
 
-static void run_exact(job_t *J, int b, int h, double *S, double *w, long long *deg)
+static void run_exact(job_t *J, int b, int h, double *S, double *w, double *xe, long long *deg)
 {
     const int T = J->T, H = J->H, m = J->m, d = J->d;
     for (int t = 0; t < T; ++t) {
         size_t tok = IDX_TOK(b, t, h, T, H);
         double eta = J->eta ? J->eta[tok] : 1.0;
-        exact_token(m, d, S, J->x + tok * d, J->c + tok * m, J->q + tok * m, J->mu[tok], eta,
-                    J->y + tok * d, w, deg);
+        oracle_write_input(J->mode, m, d, S, J->c + tok * m, J->x + tok * d, xe); /* before the update */
+        exact_token(m, d, S, xe, J->c + tok * m, J->q + tok * m, J->mu[tok], eta, J->y + tok * d, w,
+                    deg);
     }
 }
 
 static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0, double *n2,
-                                  double *g, double *kt, long long *deg)
+                                  double *g, double *kt, double *xe, long long *deg)
 {
     const int T = J->T, H = J->H, m = J->m, d = J->d, C = J->C;
     for (int t0 = 0; t0 < T; t0 += C) {
@@ -175,7 +210,8 @@ static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0,
         }
         for (int t = t0; t < t1; ++t) {
             size_t tok = IDX_TOK(b, t, h, T, H);
-            const double *x = J->x + tok * d;
+            oracle_write_input(J->mode, m, d, S0, J->c + tok * m, J->x + tok * d, xe); /* chunk start */
+            const double *x = xe;
             double eta = J->eta ? J->eta[tok] : 1.0;
             oracle_chunk_token_gates(m, d, S0, n2, x, J->c + tok * m, J->mu[tok], eta, g, kt,
                                      NULL, deg);
@@ -199,7 +235,7 @@ static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0,
  * with A_tau = prod_{l<=tau} g_l. Products are formed directly (no division).
  * Used to check the token-wise form; both share the per-token gates. */
 static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, double *n2,
-                               double *G, double *KT, long long *deg)
+                               double *G, double *KT, double *XE, long long *deg)
 {
     const int T = J->T, H = J->H, m = J->m, d = J->d, C = J->C;
     for (int t0 = 0; t0 < T; t0 += C) {
@@ -213,7 +249,8 @@ static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, do
         for (int tau = 0; tau < L; ++tau) {
             size_t tok = IDX_TOK(b, t0 + tau, h, T, H);
             double eta = J->eta ? J->eta[tok] : 1.0;
-            oracle_chunk_token_gates(m, d, S0, n2, J->x + tok * d, J->c + tok * m, J->mu[tok],
+            oracle_write_input(J->mode, m, d, S0, J->c + tok * m, J->x + tok * d, XE + (size_t)tau * d);
+            oracle_chunk_token_gates(m, d, S0, n2, XE + (size_t)tau * d, J->c + tok * m, J->mu[tok],
                                      eta, G + (size_t)tau * m, KT + (size_t)tau * m, NULL, deg);
         }
         for (int tau = 0; tau < L; ++tau) {
@@ -233,7 +270,7 @@ static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, do
                     for (int l = j + 1; l <= tau; ++l) prod *= G[(size_t)l * m + i];
                     P += q[i] * KT[(size_t)j * m + i] * prod;
                 }
-                const double *xj = J->x + IDX_TOK(b, t0 + j, h, T, H) * d;
+                const double *xj = XE + (size_t)j * d;
                 for (int k = 0; k < d; ++k) y[k] += P * (-xj[k]);
             }
         }
@@ -245,7 +282,7 @@ static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, do
                 double prod = 1.0;
                 for (int l = j + 1; l < L; ++l) prod *= G[(size_t)l * m + i];
                 double coef = KT[(size_t)j * m + i] * prod;
-                const double *xj = J->x + IDX_TOK(b, t0 + j, h, T, H) * d;
+                const double *xj = XE + (size_t)j * d;
                 for (int k = 0; k < d; ++k) S[(size_t)i * d + k] += coef * (-xj[k]);
             }
         }
@@ -263,6 +300,7 @@ static void *worker(void *arg)
     double *w = malloc(sizeof(double) * (size_t)d);
     double *G = malloc(sizeof(double) * (size_t)C * m);
     double *KT = malloc(sizeof(double) * (size_t)C * m);
+    double *XE = malloc(sizeof(double) * (size_t)C * d);
     long long deg = 0;
     for (;;) {
         pthread_mutex_lock(&J->lock);
@@ -273,27 +311,27 @@ static void *worker(void *arg)
         size_t so = ((size_t)b * J->H + h) * (size_t)m * d;
         memcpy(S, J->S0 + so, sizeof(double) * (size_t)m * d);
         if (J->form == 0)
-            run_exact(J, b, h, S, w, &deg);
+            run_exact(J, b, h, S, w, XE, &deg);
         else if (J->form == 1)
-            run_chunked_tokenwise(J, b, h, S, S0, n2, G, KT, &deg);
+            run_chunked_tokenwise(J, b, h, S, S0, n2, G, KT, XE, &deg);
         else
-            run_chunked_matrix(J, b, h, S, S0, n2, G, KT, &deg);
+            run_chunked_matrix(J, b, h, S, S0, n2, G, KT, XE, &deg);
         if (J->S_out) memcpy(J->S_out + so, S, sizeof(double) * (size_t)m * d);
     }
     pthread_mutex_lock(&J->lock);
     J->degenerate += deg;
     pthread_mutex_unlock(&J->lock);
-    free(S); free(S0); free(n2); free(w); free(G); free(KT);
+    free(S); free(S0); free(n2); free(w); free(G); free(KT); free(XE);
     return NULL;
 }
 
-static long long run(int form, int B, int T, int H, int m, int d, int C, const double *x,
+static long long run(int form, int mode, int B, int T, int H, int m, int d, int C, const double *x,
                      const double *c, const double *q, const double *mu, const double *eta,
                      const double *S0, double *S_out, double *y, int nthreads)
 {
     job_t J;
     memset(&J, 0, sizeof(J));
-    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C; J.form = form;
+    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C; J.form = form; J.mode = mode;
     J.x = x; J.c = c; J.q = q; J.mu = mu; J.eta = eta; J.S0 = S0; J.S_out = S_out; J.y = y;
     pthread_mutex_init(&J.lock, NULL);
     if (nthreads < 1) nthreads = 1;
@@ -310,30 +348,59 @@ static long long run(int form, int B, int T, int H, int m, int d, int C, const d
     return J.degenerate;
 }
 
-/* Exact recurrence (chunk size 1). Returns the number of zero-norm updates. */
+/* Whole-sequence drivers. mode 0: similarity objective (h = -x); mode 1:
+ * reconstruction objective (h = phi(S) c - x, see oracle_write_input).
+ * Each returns the number of zero-norm updates. */
+
+/* Exact recurrence (chunk size 1). */
+long long oracle_exact_scan_mode(int mode, int B, int T, int H, int m, int d, const double *x,
+                                 const double *c, const double *q, const double *mu,
+                                 const double *eta, const double *S0, double *S_out, double *y,
+                                 int nthreads)
+{
+    return run(0, mode, B, T, H, m, d, 1, x, c, q, mu, eta, S0, S_out, y, nthreads);
+}
+
+/* Chunked recurrence of Eq. 17, chunk size C, evaluated token by token. */
+long long oracle_chunked_scan_mode(int mode, int B, int T, int H, int m, int d, int C,
+                                   const double *x, const double *c, const double *q,
+                                   const double *mu, const double *eta, const double *S0,
+                                   double *S_out, double *y, int nthreads)
+{
+    return run(1, mode, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
+}
+
+/* Same definition evaluated through the chunk-level closed form (self-check). */
+long long oracle_chunked_matrix_scan_mode(int mode, int B, int T, int H, int m, int d, int C,
+                                          const double *x, const double *c, const double *q,
+                                          const double *mu, const double *eta, const double *S0,
+                                          double *S_out, double *y, int nthreads)
+{
+    return run(2, mode, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
+}
+
+/* The similarity-objective drivers. */
 long long oracle_exact_scan(int B, int T, int H, int m, int d, const double *x, const double *c,
                             const double *q, const double *mu, const double *eta,
                             const double *S0, double *S_out, double *y, int nthreads)
 {
-    return run(0, B, T, H, m, d, 1, x, c, q, mu, eta, S0, S_out, y, nthreads);
+    return run(0, 0, B, T, H, m, d, 1, x, c, q, mu, eta, S0, S_out, y, nthreads);
 }
 
-/* Chunked recurrence of Eq. 17, chunk size C, evaluated token by token. */
 long long oracle_chunked_scan(int B, int T, int H, int m, int d, int C, const double *x,
                               const double *c, const double *q, const double *mu,
                               const double *eta, const double *S0, double *S_out, double *y,
                               int nthreads)
 {
-    return run(1, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
+    return run(1, 0, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
 }
 
-/* Same definition evaluated through the chunk-level closed form (self-check). */
 long long oracle_chunked_matrix_scan(int B, int T, int H, int m, int d, int C, const double *x,
                                      const double *c, const double *q, const double *mu,
                                      const double *eta, const double *S0, double *S_out,
                                      double *y, int nthreads)
 {
-    return run(2, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
+    return run(2, 0, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
 }
 
 /* Read-out y = sum_i q_i s_i for every (b,h): S[B][H][m][d], q[B][H][m], y[B][H][d]

@@ -355,3 +355,121 @@ def test_threads_do_not_change_results():
         y8, S8, _ = oracle.scan(x, c, q, mu, S0, chunk=chunk, nthreads=8)
         np.testing.assert_array_equal(y1, y8)
         np.testing.assert_array_equal(S1, S8)
+
+
+# --------------------------------------------- reconstruction objective (DEC) ---
+
+def test_dec_write_is_negative_half_gradient_of_reconstruction_loss():
+    """§3.1.1 eq. (decoding_stateNorm_loss), eq. (decoding_recurrence) and eq. (OSR)
+    with h = e: with mu = 1 the write is -eta (c_i/|s_i|) P(s_i) e, the gradient
+    as printed, which is half the gradient of L(S) = |phi(S) c - x|^2 (phi
+    normalises each slot). Checked by central finite differences at |s| != 1."""
+    rng = _rng(21)
+    m, d = 4, 6
+    S = rng.standard_normal((m, d)) * rng.uniform(0.5, 2.0, (m, 1))
+    x = rng.standard_normal(d)
+    c = rng.uniform(0.1, 1.0, m)
+    eta = 0.41
+
+    def loss(Sm):
+        phi = Sm / np.linalg.norm(Sm, axis=1, keepdims=True)
+        e = phi.T @ c - x
+        return float(e @ e)
+
+    x_eff = oracle.write_input(S, c, x, mode="dec")
+    eps = 1e-6
+    for i in range(m):
+        grad = np.zeros(d)
+        for k in range(d):
+            Sp, Sn = S.copy(), S.copy()
+            Sp[i, k] += eps
+            Sn[i, k] -= eps
+            grad[k] = (loss(Sp) - loss(Sn)) / (2 * eps)
+        w, _ = oracle.osr_write(S[i], x_eff, c[i], 1.0, eta)
+        np.testing.assert_allclose(w - S[i], -eta * grad / 2, rtol=1e-7, atol=1e-9)
+
+
+@pytest.mark.parametrize("chunk", [1, 4])
+def test_dec_perfect_reconstruction_leaves_the_state(chunk):
+    """With x_t = phi(S0)^T c_t the reconstruction error is zero, so eq. (OSR)
+    writes nothing; the forget gate and the normaliser then leave every slot
+    unchanged (§3.2, §3.3), and y_t = q_t S0 at every step, in both forms."""
+    rng = _rng(22)
+    B, T, H, m, d = 1, 9, 2, 5, 6
+    x, c, q, mu, S0 = _rand_inputs(rng, B, T, H, m, d, unit=True)
+    for b in range(B):
+        for h in range(H):
+            phi = S0[b, h] / np.linalg.norm(S0[b, h], axis=1, keepdims=True)
+            for t in range(T):
+                x[b, t, h] = phi.T @ c[b, t, h]
+    y, S, deg = oracle.scan(x, c, q, mu, S0, chunk=chunk, mode="dec")
+    assert deg == 0
+    np.testing.assert_allclose(S, S0, atol=1e-12)
+    np.testing.assert_allclose(y, np.einsum("bthm,bhmd->bthd", q, S0), atol=1e-12)
+
+
+def test_dec_brute_force_projection_matrices():
+    """eq. (OSR) with h = e evaluated literally in the paper's d x m layout: the
+    error e = Phi c - x from the current state, the stacked Jacobians
+    P(s_i)/|s_i|, the General Form mu S - eta grad, the unit-sphere projection
+    (§3.2) and the read-out with the updated state."""
+    rng = _rng(23)
+    B, T, H, m, d = 2, 8, 2, 3, 5
+    x, c, q, mu, S0 = _rand_inputs(rng, B, T, H, m, d, unit=False)
+    eta = rng.uniform(0.2, 1.2, (B, T, H))
+    y_o, S_o, _ = oracle.scan(x, c, q, mu, S0, eta=eta, mode="dec")
+    for b in range(B):
+        for hh in range(H):
+            Sdm = S0[b, hh].T.copy()  # d x m, slots are columns
+            for t in range(T):
+                Phi = Sdm / np.linalg.norm(Sdm, axis=0, keepdims=True)
+                e = Phi @ c[b, t, hh] - x[b, t, hh]
+                P = np.zeros((d, d, m))
+                for i in range(m):
+                    s = Sdm[:, i]
+                    P[:, :, i] = (np.eye(d) - np.outer(s, s) / (s @ s)) / np.linalg.norm(s)
+                grad = np.einsum("a,adm->dm", e, P) * c[b, t, hh][None, :]
+                Snew = mu[b, t, hh] * Sdm - eta[b, t, hh] * grad
+                Sdm = Snew / np.linalg.norm(Snew, axis=0, keepdims=True)
+                np.testing.assert_allclose(y_o[b, t, hh], Sdm @ q[b, t, hh], atol=1e-12)
+            np.testing.assert_allclose(S_o[b, hh], Sdm.T, atol=1e-12)
+
+
+def test_dec_chunk_size_one_is_the_exact_recurrence():
+    """Appendix D: chunk size 1 is the exact recurrence under the reconstruction
+    objective too (the chunk-start state is the current state)."""
+    rng = _rng(24)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 13, 2, 6, 7, unit=True)
+    y1, S1, _ = oracle.scan(x, c, q, mu, S0, chunk=1, mode="dec")
+    from oracle import _load, _f64, _p
+    lib = _load()
+    B, T, H, d = x.shape
+    m = c.shape[-1]
+    y2, S2 = np.zeros_like(y1), np.zeros_like(S1)
+    lib.oracle_chunked_scan_mode(1, B, T, H, m, d, 1, _p(_f64(x)), _p(_f64(c)), _p(_f64(q)),
+                                 _p(_f64(mu)), None, _p(_f64(S0)), _p(S2), _p(y2), 1)
+    np.testing.assert_allclose(y2, y1, atol=1e-12)
+    np.testing.assert_allclose(S2, S1, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [4, 16])
+def test_dec_chunk_closed_form_equals_token_form(C):
+    """§3.4.1 / Appendix B.1 with H = K Phi - V (Appendix D, compress_chunk): the
+    chunk-level matrix form equals the token-wise Eq. 17 recurrence."""
+    rng = _rng(200 + C)
+    T = 2 * C + 3
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, T, 2, 5, 4, unit=False, mu_range=(0.6, 1.0))
+    y1, S1, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="token", mode="dec")
+    y2, S2, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="matrix", mode="dec")
+    np.testing.assert_allclose(y2, y1, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(S2, S1, rtol=1e-10, atol=1e-10)
+
+
+def test_dec_differs_from_sim():
+    """The two objectives write different things (guards against a mode flag
+    that is ignored)."""
+    rng = _rng(25)
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 4, 1, 3, 5)
+    ys, _, _ = oracle.scan(x, c, q, mu, S0, mode="sim")
+    yd, _, _ = oracle.scan(x, c, q, mu, S0, mode="dec")
+    assert np.abs(ys - yd).max() > 1e-3
