@@ -183,13 +183,13 @@ def _dev_inputs(torch, inp, device):
                 mu=torch.from_numpy(inp["mu"]).to(device), S0=torch.from_numpy(inp["S0"]).to(device))
 
 
-def time_scan(torch, L, t, chunk, steps, warmup, flush=None, impl="auto"):
+def time_scan(torch, L, t, chunk, steps, warmup, flush=None, impl="auto", mode="sim"):
     """Per-step device time (ms) of lattice_scan_fwd, CUDA events on its stream."""
     stream = torch.cuda.current_stream()
     y = torch.empty(t["x"].shape[:3] + (t["S0"].shape[-1],), dtype=torch.float32, device=t["x"].device)
     S = torch.empty_like(t["S0"])
     run = lambda: L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], chunk=chunk, S_out=S, y=y,
-                             impl=impl, stream=stream)
+                             impl=impl, stream=stream, mode=mode)
     for _ in range(warmup):
         run()
     torch.cuda.synchronize()
@@ -246,7 +246,7 @@ def time_scan_e2e(torch, L, inp, chunk, steps, warmup, device):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
-def time_decode(torch, L, w, n_steps, ring, device):
+def time_decode(torch, L, w, n_steps, ring, device, mode="sim"):
     """n_steps consecutive decode steps replayed from a CUDA graph over a ring of
     pre-drawn per-step inputs (the ring and the 512 MiB state exceed L2)."""
     S = torch.from_numpy(LI.make_decode_state(w)).to(device)
@@ -260,11 +260,11 @@ def time_decode(torch, L, w, n_steps, ring, device):
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         for k in range(3):  # warm-up
-            L.step(S, xs[k], cs[k], qs[k], mus[k], y=y, stream=s)
+            L.step(S, xs[k], cs[k], qs[k], mus[k], y=y, stream=s, mode=mode)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             for k in range(ring):
-                L.step(S, xs[k], cs[k], qs[k], mus[k], y=y, stream=s)
+                L.step(S, xs[k], cs[k], qs[k], mus[k], y=y, stream=s, mode=mode)
     torch.cuda.synchronize()
     reps = max(1, n_steps // ring)
     with torch.cuda.stream(s):
@@ -431,6 +431,20 @@ def main():
             te = time_scan(torch, L, t, 1, 5, 3, flush=flush)
             extra[f"{w.name}_exact"] = {"ms": statistics.mean(te),
                                         "tokens_per_s": w.B * w.T / (statistics.mean(te) * 1e-3)}
+            # the reconstruction objective (CUDA-core kernels), exact and chunked; the
+            # chunked form takes intensities sigmoid(N(-4,1)), with which it stays bounded
+            td = time_scan(torch, L, t, 1, 5, 3, flush=flush, mode="dec")
+            extra[f"{w.name}_dec_exact"] = {"ms": statistics.mean(td),
+                                            "tokens_per_s": w.B * w.T / (statistics.mean(td) * 1e-3),
+                                            "kernel": "scan_simt_kernel<exact, dec>"}
+            wdc = w.with_(c_loc=-4.0)
+            tdc = _dev_inputs(torch, LI.make_inputs(wdc), device)
+            td = time_scan(torch, L, tdc, w.chunk, 5, 3, flush=flush, mode="dec")
+            extra[f"{w.name}_dec_chunked"] = {"ms": statistics.mean(td),
+                                              "tokens_per_s": w.B * w.T / (statistics.mean(td) * 1e-3),
+                                              "kernel": "scan_simt_kernel<chunked, dec>",
+                                              "inputs": "c = sigmoid(N(-4,1))"}
+            del tdc
             del t
             for name in [n for n in ("mid_layer", "long_ctx") if n != w.name]:
                 wn = LI.WORKLOADS[name]
@@ -463,6 +477,10 @@ def main():
             extra["decode"] = {"us_per_step": us_ms * 1e3, "steps": n, "gbps": sb / (us_ms * 1e-3) / 1e9,
                                "hbm_frac": sb / (us_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                                "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb}
+            us_ms, n = time_decode(torch, L, wd, 1000, 40, device, mode="dec")
+            extra["decode_dec"] = {"us_per_step": us_ms * 1e3, "steps": n, "gbps": sb / (us_ms * 1e-3) / 1e9,
+                                   "hbm_frac": sb / (us_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                   "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb}
         line["extra"] = extra
         if not args.no_cpu:
             v, cores, sample = oracle_baseline(w, w.chunk)

@@ -72,7 +72,19 @@ typedef enum {
 
 typedef enum { LATTICE_F32 = 0, LATTICE_BF16 = 1 } lattice_dtype;
 
-/* Objective (§3.1.1). Only the similarity objective (h_t = -x_t) is built. */
+/* Objective (§3.1.1, eq. OSR): what each token writes into the slots.
+ *   LATTICE_SIM  dot-product similarity objective, h_t = -x_t: slot i takes
+ *                the part of x_t orthogonal to it (eq. similarity_recurrence).
+ *   LATTICE_DEC  l2 reconstruction objective, h_t = e_t = phi(S) c_t - x_t with
+ *                phi(s_i) = s_i/|s_i| (eq. decoding_stateNorm_loss and
+ *                eq. decoding_recurrence): slot i takes the part of the
+ *                reconstruction residual x_t - sum_j c_tj s_j/|s_j| orthogonal
+ *                to it. e is formed from the state the token's projection uses:
+ *                the current state (exact recurrence, decode step) or the
+ *                chunk-start state (chunked form, as in the Appendix D listing).
+ * DEC runs on the CUDA-core kernels only. The tensor-core choices return
+ * LATTICE_ERR_UNSUPPORTED for it, and LATTICE_IMPL_AUTO takes the CUDA-core
+ * kernel. */
 typedef enum { LATTICE_SIM = 0, LATTICE_DEC = 1 } lattice_mode;
 
 /* Kernel choice for chunked scans.

@@ -30,6 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblattice.
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
 _F32, _BF16 = 0, 1
 _IMPL = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3}
+_MODE = {"sim": 0, "dec": 1}
 _lib = None
 
 
@@ -110,9 +111,10 @@ _XQ = (torch.float32, torch.bfloat16)
 def scan_fwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor,
              S0: torch.Tensor, eta: Optional[torch.Tensor] = None, chunk: int = 1,
              S_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
-             impl: str = "auto", stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+             impl: str = "auto", stream=None, mode: str = "sim") -> Tuple[torch.Tensor, torch.Tensor]:
     """Whole-sequence forward (the paper's lattice_compress, Appendix D).
     chunk == 1: exact recurrence; chunk > 1: the Eq. 17 chunked form.
+    mode "sim": similarity objective; "dec": reconstruction objective.
     Returns (y [B,T,H,d] float32, S_T [B,H,m,d] float32). S_out may be S0."""
     B, T, H, d = x.shape
     m = c.shape[-1]
@@ -131,15 +133,15 @@ def scan_fwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor
     _chk(y, "y", (B, T, H, d))
     L = lib()
     code = L.lattice_scan_fwd_impl(_ptr(x), _dt(x), _ptr(c), _ptr(q), _dt(q), _ptr(mu), _ptr(eta),
-                                   _ptr(S0), _ptr(S_out), _ptr(y), B, T, H, m, d, int(chunk), 0,
-                                   _IMPL[impl], _stream(stream))
+                                   _ptr(S0), _ptr(S_out), _ptr(y), B, T, H, m, d, int(chunk),
+                                   _MODE[mode], _IMPL[impl], _stream(stream))
     _raise(code, "lattice_scan_fwd")
     return y, S_out
 
 
 def step(S: torch.Tensor, x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor,
          eta: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
-         stream=None) -> torch.Tensor:
+         stream=None, mode: str = "sim") -> torch.Tensor:
     """One decode step, state updated in place. S [B,H,m,d], x [B,H,d], c/q [B,H,m],
     mu/eta [B,H]. Returns y [B,H,d]."""
     B, H, m, d = S.shape
@@ -154,7 +156,7 @@ def step(S: torch.Tensor, x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu:
         y = torch.empty((B, H, d), dtype=torch.float32, device=S.device)
     _chk(y, "y", (B, H, d))
     code = lib().lattice_step(_ptr(S), _ptr(x), _dt(x), _ptr(c), _ptr(q), _dt(q), _ptr(mu),
-                              _ptr(eta), _ptr(y), B, H, m, d, 0, _stream(stream))
+                              _ptr(eta), _ptr(y), B, H, m, d, _MODE[mode], _stream(stream))
     _raise(code, "lattice_step")
     return y
 

@@ -124,6 +124,28 @@ __device__ __forceinline__ float octet_sum(float v) {
     return v;
 }
 
+// Reconstruction objective ("Lattice: Learning to Efficiently Compress the
+// Memory", §3.1.1 eq. decoding_recurrence): the write direction is -e with
+// e = sum_i c_i s_i/|s_i| - x. This is the warp's share of sum_i f_i s_i
+// (f_i = c_i/|s_i|) over the slots it holds, summed over its four octets, so
+// every octet ends with the warp's partial for its lane's element positions.
+template <int D, int RQ>
+__device__ __forceinline__ void recon_warp_partial(const float (*s)[Octet<D>::EPL], const float* f,
+                                                   float* rp) {
+    constexpr int EPL = Octet<D>::EPL;
+#pragma unroll
+    for (int k = 0; k < EPL; ++k) rp[k] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RQ; ++r)
+#pragma unroll
+        for (int k = 0; k < EPL; ++k) rp[k] = fmaf(f[r], s[r][k], rp[k]);
+#pragma unroll
+    for (int k = 0; k < EPL; ++k) {
+        rp[k] += __shfl_xor_sync(0xffffffffu, rp[k], 8);
+        rp[k] += __shfl_xor_sync(0xffffffffu, rp[k], 16);
+    }
+}
+
 // Per-slot update coefficients. The new slot is alpha*s + gamma*x.
 //   n2 = |s_ref|^2, p = s_ref . x, xx = |x|^2 (s_ref = current slot for the exact
 //   recurrence, chunk-start slot for the chunked form).

@@ -52,33 +52,38 @@ lattice_status launch_status() {
 }
 
 // ---- exact / chunked CUDA-core scan
-template <int D, int RQ, bool CH>
+template <int D, int RQ, bool CH, bool DEC>
 lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
-    size_t smem = scan_smem_bytes<D>(a.m, nw);
-    auto k = scan_simt_kernel<D, RQ, CH>;
+    size_t smem = scan_smem_bytes<D>(a.m, nw, DEC);
+    auto k = scan_simt_kernel<D, RQ, CH, DEC>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e);
     k<<<a.B * a.H, nw * 32, smem, st>>>(a);
     return launch_status();
 }
 
-template <int D, bool CH>
+template <int D, bool CH, bool DEC>
 lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
     const int quads = (a.m + 3) / 4;
-    if (quads <= 16) return launch_scan_simt_t<D, 1, CH>(a, quads < 4 ? 4 : quads, st);
-    if (quads <= 32) return launch_scan_simt_t<D, 2, CH>(a, 16, st);
-    return launch_scan_simt_t<D, 4, CH>(a, 16, st);
+    if (quads <= 16) return launch_scan_simt_t<D, 1, CH, DEC>(a, quads < 4 ? 4 : quads, st);
+    if (quads <= 32) return launch_scan_simt_t<D, 2, CH, DEC>(a, 16, st);
+    return launch_scan_simt_t<D, 4, CH, DEC>(a, 16, st);
+}
+
+template <bool CH, bool DEC>
+lattice_status launch_scan_simt_m(const ScanArgs& a, int d, cudaStream_t st) {
+    switch (d) {
+        case 16: return launch_scan_simt_d<16, CH, DEC>(a, st);
+        case 32: return launch_scan_simt_d<32, CH, DEC>(a, st);
+        case 64: return launch_scan_simt_d<64, CH, DEC>(a, st);
+        case 128: return launch_scan_simt_d<128, CH, DEC>(a, st);
+    }
+    return LATTICE_ERR_UNSUPPORTED;
 }
 
 template <bool CH>
-lattice_status launch_scan_simt(const ScanArgs& a, int d, cudaStream_t st) {
-    switch (d) {
-        case 16: return launch_scan_simt_d<16, CH>(a, st);
-        case 32: return launch_scan_simt_d<32, CH>(a, st);
-        case 64: return launch_scan_simt_d<64, CH>(a, st);
-        case 128: return launch_scan_simt_d<128, CH>(a, st);
-    }
-    return LATTICE_ERR_UNSUPPORTED;
+lattice_status launch_scan_simt(const ScanArgs& a, int d, bool dec, cudaStream_t st) {
+    return dec ? launch_scan_simt_m<CH, true>(a, d, st) : launch_scan_simt_m<CH, false>(a, d, st);
 }
 
 // ---- decode step / read-out: NW warps x RQ quads per warp
@@ -90,17 +95,22 @@ void step_shape(int m, int& nw, int& rq) {
     else { nw = 16; rq = 4; }
 }
 
-template <int D>
-lattice_status launch_step_d(const StepArgs& a, cudaStream_t st) {
+template <int D, bool DEC>
+lattice_status launch_step_dm(const StepArgs& a, cudaStream_t st) {
     int nw, rq;
     step_shape(a.m, nw, rq);
     dim3 grid(a.B * a.H), block(nw * 32);
     switch (rq) {
-        case 1: step_kernel<D, 1><<<grid, block, 0, st>>>(a); break;
-        case 2: step_kernel<D, 2><<<grid, block, 0, st>>>(a); break;
-        default: step_kernel<D, 4><<<grid, block, 0, st>>>(a); break;
+        case 1: step_kernel<D, 1, DEC><<<grid, block, 0, st>>>(a); break;
+        case 2: step_kernel<D, 2, DEC><<<grid, block, 0, st>>>(a); break;
+        default: step_kernel<D, 4, DEC><<<grid, block, 0, st>>>(a); break;
     }
     return launch_status();
+}
+
+template <int D>
+lattice_status launch_step_d(const StepArgs& a, bool dec, cudaStream_t st) {
+    return dec ? launch_step_dm<D, true>(a, st) : launch_step_dm<D, false>(a, st);
 }
 
 template <int D>
@@ -161,7 +171,8 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
     if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05 &&
         impl != LATTICE_IMPL_TCGEN05_SPLIT)
         return LATTICE_ERR_INVALID_ARG;
-    if (mode != LATTICE_SIM) return mode == LATTICE_DEC ? LATTICE_ERR_UNSUPPORTED : LATTICE_ERR_INVALID_ARG;
+    if (mode != LATTICE_SIM && mode != LATTICE_DEC) return LATTICE_ERR_INVALID_ARG;
+    const bool dec = mode == LATTICE_DEC;
     lattice_status ds = check_dims(B, H, m, d);
     if (ds != LATTICE_OK) return ds;
     if (!S0 || !S_out) return LATTICE_ERR_INVALID_ARG;
@@ -192,9 +203,10 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
 
     ScanArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, S_out, y,
                B, T, H, m, chunk_size};
-    if (chunk_size == 1) {
-        if (impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT) return LATTICE_ERR_UNSUPPORTED;
-        return launch_scan_simt<false>(a, d, st);
+    const bool tc_choice = impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT;
+    if (chunk_size == 1 || dec) {  // the tensor-core kernels run the similarity objective
+        if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
+        return chunk_size == 1 ? launch_scan_simt<false>(a, d, dec, st) : launch_scan_simt<true>(a, d, dec, st);
     }
     if (impl == LATTICE_IMPL_AUTO) impl = lattice_chunk_impl(B, H, m, d, chunk_size, x_dtype, q_dtype);
     if (impl == LATTICE_IMPL_TCGEN05_SPLIT) {
@@ -207,7 +219,7 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
         cudaError_t e = launch_chunk_tc(a, d, st);
         return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
     }
-    return launch_scan_simt<true>(a, d, st);
+    return launch_scan_simt<true>(a, d, false, st);
 }
 
 lattice_status lattice_scan_fwd(const void* x, lattice_dtype x_dtype, const float* c,
@@ -224,7 +236,8 @@ lattice_status lattice_step(float* S, const void* x, lattice_dtype x_dtype, cons
                             const float* eta, float* y, int B, int H, int m, int d,
                             lattice_mode mode, void* stream) {
     if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
-    if (mode != LATTICE_SIM) return mode == LATTICE_DEC ? LATTICE_ERR_UNSUPPORTED : LATTICE_ERR_INVALID_ARG;
+    if (mode != LATTICE_SIM && mode != LATTICE_DEC) return LATTICE_ERR_INVALID_ARG;
+    const bool dec = mode == LATTICE_DEC;
     lattice_status ds = check_dims(B, H, m, d);
     if (ds != LATTICE_OK) return ds;
     if (!S || !x || !c || !q || !mu || !y) return LATTICE_ERR_INVALID_ARG;
@@ -242,10 +255,10 @@ lattice_status lattice_step(float* S, const void* x, lattice_dtype x_dtype, cons
     StepArgs a{S, x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, y, B, H, m};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     switch (d) {
-        case 16: return launch_step_d<16>(a, st);
-        case 32: return launch_step_d<32>(a, st);
-        case 64: return launch_step_d<64>(a, st);
-        default: return launch_step_d<128>(a, st);
+        case 16: return launch_step_d<16>(a, dec, st);
+        case 32: return launch_step_d<32>(a, dec, st);
+        case 64: return launch_step_d<64>(a, dec, st);
+        default: return launch_step_d<128>(a, dec, st);
     }
 }
 

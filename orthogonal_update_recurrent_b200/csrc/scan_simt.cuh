@@ -37,13 +37,19 @@ struct ScanArgs {
 // of 4 floats so that every record starts 16-byte aligned.
 __host__ __device__ inline int scan_record_floats(int D, int m) { return (D + 2 * m + 2 + 3) & ~3; }
 
-// Shared memory: in[2][TB][record] floats, ybuf[2][TB][NW][D] floats.
+// Shared memory: in[2][TB][record] floats, ybuf[2][TB][NW][D] floats and, for the
+// reconstruction objective, rbuf[2][NW][D] floats (per-warp partial reconstructions).
 template <int D>
-__host__ __device__ inline size_t scan_smem_bytes(int m, int nw) {
-    return sizeof(float) * (2ull * kScanTB * scan_record_floats(D, m) + 2ull * kScanTB * nw * D);
+__host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec) {
+    return sizeof(float) * (2ull * kScanTB * scan_record_floats(D, m) + 2ull * kScanTB * nw * D +
+                            (dec ? 2ull * nw * D : 0ull));
 }
 
-template <int D, int RQ, bool CHUNKED>
+// DEC selects the reconstruction objective (§3.1.1 eq. decoding_recurrence): each
+// token's write direction is x - sum_i (c_i/|s_i|) s_i, with the slots of the state
+// the token's projection uses (the current state; the chunk-start state when
+// CHUNKED). It costs one cross-warp reduction and one barrier per token.
+template <int D, int RQ, bool CHUNKED, bool DEC>
 __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
@@ -58,6 +64,7 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
     const int per_tok = scan_record_floats(D, m);  // x | q | c | mu | eta | pad
     float* in_buf = smem;
     float* ybuf = smem + 2 * kScanTB * per_tok;
+    float* rbuf = ybuf + 2 * kScanTB * NW * D;  // DEC only
 
     // ---- load the initial state into registers
     float s[RQ][EPL];
@@ -146,10 +153,6 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
             float xv[EPL];
             load_row_f32<D>(rec, j, xv);
             const float mu = rec[D + 2 * m], eta = rec[D + 2 * m + 1];
-            float xx = 0.f;
-#pragma unroll
-            for (int k = 0; k < EPL; ++k) xx = fmaf(xv[k], xv[k], xx);
-            xx = octet_sum(xx);
 
             if constexpr (CHUNKED) {
                 if (t % a.chunk == 0) {  // chunk start: snapshot the state and its norms
@@ -163,6 +166,41 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
                     }
                 }
             }
+            if constexpr (DEC) {  // x <- x - sum_i (c_i/|s_i|) s_i over every slot of the CTA
+                float f[RQ], rp[EPL];
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    const float cv = slot[r] < m ? rec[D + m + slot[r]] : 0.f;
+                    float nsq;
+                    if constexpr (CHUNKED) {
+                        nsq = n0sq[r];
+                    } else {
+                        float nn = 0.f;
+#pragma unroll
+                        for (int k = 0; k < EPL; ++k) nn = fmaf(s[r][k], s[r][k], nn);
+                        nsq = octet_sum(nn);
+                    }
+                    f[r] = nsq > 0.f ? __fdiv_rn(cv, __fsqrt_rn(nsq)) : 0.f;
+                }
+                if constexpr (CHUNKED) recon_warp_partial<D, RQ>(s0, f, rp);
+                else recon_warp_partial<D, RQ>(s, f, rp);
+                float* rb = rbuf + (size_t)(t & 1) * NW * D;
+                if (oct == 0) {
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) rb[warp * D + O::pos(j, k)] = rp[k];
+                }
+                __syncthreads();
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) {
+                    float acc = 0.f;
+                    for (int w = 0; w < NW; ++w) acc += rb[w * D + O::pos(j, k)];
+                    xv[k] -= acc;
+                }
+            }
+            float xx = 0.f;
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) xx = fmaf(xv[k], xv[k], xx);
+            xx = octet_sum(xx);
             float p[RQ], n2[RQ];
 #pragma unroll
             for (int r = 0; r < RQ; ++r) {
@@ -196,8 +234,8 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
                 const float cv = valid ? rec[D + m + slot[r]] : 0.f;
                 const float qv = valid ? rec[D + slot[r]] : 0.f;
                 float alpha, gamma;
-                update_coefs<CHUNKED>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
-                                      CHUNKED ? n0[r] : 1.f, alpha, gamma);
+                update_coefs<CHUNKED || DEC>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
+                                             CHUNKED ? n0[r] : 1.f, alpha, gamma);
                 if (!valid) { alpha = 0.f; gamma = 0.f; }
 #pragma unroll
                 for (int k = 0; k < EPL; ++k) {

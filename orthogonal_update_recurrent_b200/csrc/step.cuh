@@ -22,8 +22,10 @@ struct StepArgs {
     int B, H, m;
 };
 
-// One CTA per (b, h); NW warps, RQ slot quads per warp (4*NW*RQ >= m).
-template <int D, int RQ>
+// One CTA per (b, h); NW warps, RQ slot quads per warp (4*NW*RQ >= m). DEC selects
+// the reconstruction objective (§3.1.1 eq. decoding_recurrence): the write direction
+// is x - sum_i (c_i/|s_i|) s_i, from the state before the step.
+template <int D, int RQ, bool DEC>
 __global__ void __launch_bounds__(512) step_kernel(StepArgs a) {
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
@@ -58,6 +60,30 @@ __global__ void __launch_bounds__(512) step_kernel(StepArgs a) {
         cv[r] = valid ? a.c[bh * m + slot[r]] : 0.f;
         qv[r] = valid ? load_elem(a.q, a.q_bf16, bh * m + slot[r]) : 0.f;
     }
+    if constexpr (DEC) {  // x <- x - sum_i (c_i/|s_i|) s_i over every slot of the CTA
+        float f[RQ], rp[EPL];
+#pragma unroll
+        for (int r = 0; r < RQ; ++r) {
+            float nn = 0.f;
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) nn = fmaf(s[r][k], s[r][k], nn);
+            nn = octet_sum(nn);
+            f[r] = nn > 0.f ? __fdiv_rn(cv[r], __fsqrt_rn(nn)) : 0.f;
+        }
+        recon_warp_partial<D, RQ>(s, f, rp);
+        if (oct == 0) {
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) ysm[warp][O::pos(j, k)] = rp[k];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < EPL; ++k) {
+            float acc = 0.f;
+            for (int w = 0; w < NW; ++w) acc += ysm[w][O::pos(j, k)];
+            xv[k] -= acc;
+        }
+        __syncthreads();  // ysm is reused for the read-out
+    }
     float xx = 0.f;
 #pragma unroll
     for (int k = 0; k < EPL; ++k) xx = fmaf(xv[k], xv[k], xx);
@@ -89,7 +115,7 @@ __global__ void __launch_bounds__(512) step_kernel(StepArgs a) {
 #pragma unroll
     for (int r = 0; r < RQ; ++r) {
         float alpha, gamma;
-        update_coefs<false>(n2[r], p[r], xx, cv[r], mu, eta, 1.f, alpha, gamma);
+        update_coefs<DEC>(n2[r], p[r], xx, cv[r], mu, eta, 1.f, alpha, gamma);
 #pragma unroll
         for (int k = 0; k < EPL; ++k) {
             s[r][k] = fmaf(alpha, s[r][k], gamma * xv[k]);

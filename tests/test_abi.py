@@ -64,7 +64,9 @@ def test_argument_checks_return_before_launch(lib):
     assert _scan(lib, d=48) == L.ERR_UNSUPPORTED
     assert _scan(lib, m=257) == L.ERR_UNSUPPORTED
     assert _scan(lib, xdt=7) == L.ERR_INVALID_ARG
-    assert _scan(lib, mode=1) == L.ERR_UNSUPPORTED
+    assert _scan(lib, mode=2) == L.ERR_INVALID_ARG
+    assert _scan(lib, mode=1, impl=2) == L.ERR_UNSUPPORTED  # DEC runs on the CUDA-core kernels
+    assert _scan(lib, mode=1, chunk=64, impl=3) == L.ERR_UNSUPPORTED
     assert _scan(lib, impl=9) == L.ERR_INVALID_ARG
     assert _scan(lib, impl=2) == L.ERR_UNSUPPORTED          # tensor cores need chunk > 1
     assert _scan(lib, chunk=64, impl=2) == L.ERR_UNSUPPORTED  # and bf16 x/q, m,d in {64,128}
