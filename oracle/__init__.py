@@ -54,6 +54,8 @@ def _load():
             f = getattr(lib, name)
             f.argtypes = [i, i, i, i, i, i, i, _D, _D, _D, _D, _D, _D, _D, _D, i]
             f.restype = ll
+        lib.oracle_chunked_scan_lin.argtypes = [i, i, i, i, i, i, i, i, i, _D, _D, _D, _D, _D, _D, _D, _D, i]
+        lib.oracle_chunked_scan_lin.restype = ll
         lib.oracle_write_input.argtypes = [i, i, i, _D, _D, _D, _D]
         lib.oracle_write_input.restype = None
         lib.oracle_readout.argtypes = [i, i, i, i, _D, _D, _D]
@@ -90,13 +92,14 @@ _MODES = {"sim": 0, "dec": 1}
 
 
 def scan(x, c, q, mu, S0, eta=None, chunk: int = 1, form: str = "token",
-         nthreads: Optional[int] = None, mode: str = "sim"):
+         nthreads: Optional[int] = None, mode: str = "sim", lin: int = 2):
     """Whole-sequence forward. x[B][T][H][d], c/q[B][T][H][m], mu/eta[B][T][H],
     S0[B][H][m][d]. chunk == 1: exact recurrence; chunk > 1: Eq. 17 chunked
     recurrence, evaluated token by token (form="token") or through the
     chunk-level closed form (form="matrix"). mode "sim": similarity objective
-    (h = -x); "dec": reconstruction objective (h = phi(S) c - x).
-    Returns (y, S_T, n_degenerate)."""
+    (h = -x); "dec": reconstruction objective (h = phi(S) c - x). lin selects the
+    chunk linearisation of §3.4.1: 2 = Eq. 17 (recurrence_linear2), 1 =
+    recurrence_linear1. Returns (y, S_T, n_degenerate)."""
     md = _MODES[mode]
     x, c, q, mu, S0 = map(_f64, (x, c, q, mu, S0))
     eta = None if eta is None else _f64(eta)
@@ -109,8 +112,12 @@ def scan(x, c, q, mu, S0, eta=None, chunk: int = 1, form: str = "token",
     lib = _load()
     nt = _threads(nthreads)
     args = (_p(x), _p(c), _p(q), _p(mu), _p(eta), _p(S0), _p(S), _p(y), nt)
+    if lin not in (1, 2):
+        raise ValueError(lin)
     if chunk == 1 and form == "token":
         deg = lib.oracle_exact_scan_mode(md, B, T, H, m, d, *args)
+    elif lin == 1 and form in ("token", "matrix"):
+        deg = lib.oracle_chunked_scan_lin(1 if form == "token" else 2, md, 1, B, T, H, m, d, chunk, *args)
     elif form == "token":
         deg = lib.oracle_chunked_scan_mode(md, B, T, H, m, d, chunk, *args)
     elif form == "matrix":

@@ -18,6 +18,9 @@
  *     scales the previous state; the normaliser applies to mu*s + write.
  *   - §3.4, Eq. 14 (recurrence_detailed): P(s) h = h - s (s.h)/||s||^2 costs one
  *     dot product and one axpy per slot.
+ *   - §3.4.1 eq. (recurrence_linear1) and eq. (chunkwise_OSR): the other
+ *     linearisation keeps the h~ k^ term on the chunk-start state:
+ *     S_t = G_t (.) S_{t-1} + 1 (h~_t (.) k^_t)^T (.) S_{t'} - h_t k^_t^T, G_t = mu_t 1 beta_t^T.
  *   - §3.4.1 / Appendix B.1, Eq. 17 (recurrence_linear2) and eq. (beta_chunk):
  *     within a chunk the projection uses the chunk-start state; the update
  *     becomes the gated linear recurrence S_t = G_t (.) S_{t-1} - h_t k_t^T.
@@ -142,9 +145,24 @@ static void exact_token(int m, int d, double *S, const double *x, const double *
  *   beta_i = n_i/sqrt(mu^2 n_i^2 + dsq_i)
  *   g_i    = beta_i (mu + eta hhat_i khat_i),   kt_i = -beta_i eta khat_i
  * so that the token's update is s_i <- g_i s_i + kt_i h. */
+void oracle_chunk_token_gates2(int m, int d, const double *S0, const double *n2,
+                               const double *x, const double *c, double mu, double eta,
+                               double *g, double *kt, double *dsq_out, long long *degenerate,
+                               double *gs, double *g0);
 void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
                               const double *x, const double *c, double mu, double eta,
                               double *g, double *kt, double *dsq_out, long long *degenerate)
+{
+    oracle_chunk_token_gates2(m, d, S0, n2, x, c, mu, eta, g, kt, dsq_out, degenerate, NULL, NULL);
+}
+
+/* As above, and the two parts of g: gs_i = beta_i mu (what scales the running slot
+ * in eq. recurrence_linear1, the G_t of §3.4.1) and g0_i = beta_i eta hhat_i khat_i
+ * (what scales the chunk-start slot there); g = gs + g0. */
+void oracle_chunk_token_gates2(int m, int d, const double *S0, const double *n2,
+                               const double *x, const double *c, double mu, double eta,
+                               double *g, double *kt, double *dsq_out, long long *degenerate,
+                               double *gs, double *g0)
 {
     double hh = 0.0;
     for (int k = 0; k < d; ++k) hh += x[k] * x[k]; /* |h|^2, h = -x */
@@ -161,12 +179,14 @@ void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
         if (den == 0.0) { /* zero-norm update: keep the slot */
             g[i] = 1.0;
             kt[i] = 0.0;
+            if (gs) { gs[i] = 1.0; g0[i] = 0.0; }
             if (degenerate) ++*degenerate;
             continue;
         }
         double beta = sqrt(n2[i]) / sqrt(den);
         g[i] = beta * (mu + eta * hhat * khat);
         kt[i] = -beta * eta * khat;
+        if (gs) { gs[i] = beta * mu; g0[i] = beta * eta * hhat * khat; }
     }
 }
 
@@ -177,6 +197,7 @@ void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
 typedef struct {
     int B, T, H, m, d, C, form; /* form: 0 exact, 1 chunked token-wise, 2 chunked matrix form */
     int mode;                   /* 0 similarity objective, 1 reconstruction objective */
+    int lin;                    /* chunked forms: 2 Eq. 17 (recurrence_linear2), 1 recurrence_linear1 */
     const double *x, *c, *q, *mu, *eta, *S0;
     double *S_out, *y;
     long long degenerate;
@@ -197,7 +218,8 @@ static void run_exact(job_t *J, int b, int h, double *S, double *w, double *xe, 
 }
 
 static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0, double *n2,
-                                  double *g, double *kt, double *xe, long long *deg)
+                                  double *g, double *kt, double *xe, double *gs, double *g0,
+                                  long long *deg)
 {
     const int T = J->T, H = J->H, m = J->m, d = J->d, C = J->C;
     for (int t0 = 0; t0 < T; t0 += C) {
@@ -213,11 +235,18 @@ static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0,
             oracle_write_input(J->mode, m, d, S0, J->c + tok * m, J->x + tok * d, xe); /* chunk start */
             const double *x = xe;
             double eta = J->eta ? J->eta[tok] : 1.0;
-            oracle_chunk_token_gates(m, d, S0, n2, x, J->c + tok * m, J->mu[tok], eta, g, kt,
-                                     NULL, deg);
-            for (int i = 0; i < m; ++i) /* s_i <- g_i s_i + kt_i h,  h = -x */
-                for (int k = 0; k < d; ++k)
-                    S[(size_t)i * d + k] = g[i] * S[(size_t)i * d + k] + kt[i] * (-x[k]);
+            oracle_chunk_token_gates2(m, d, S0, n2, x, J->c + tok * m, J->mu[tok], eta, g, kt,
+                                      NULL, deg, gs, g0);
+            if (J->lin == 1) { /* eq. recurrence_linear1: s_i <- gs_i s_i + g0_i s0_i + kt_i h */
+                for (int i = 0; i < m; ++i)
+                    for (int k = 0; k < d; ++k)
+                        S[(size_t)i * d + k] = gs[i] * S[(size_t)i * d + k] +
+                                               g0[i] * S0[(size_t)i * d + k] + kt[i] * (-x[k]);
+            } else { /* Eq. 17: s_i <- g_i s_i + kt_i h,  h = -x */
+                for (int i = 0; i < m; ++i)
+                    for (int k = 0; k < d; ++k)
+                        S[(size_t)i * d + k] = g[i] * S[(size_t)i * d + k] + kt[i] * (-x[k]);
+            }
             double *y = J->y + tok * d;
             const double *q = J->q + tok * m;
             for (int k = 0; k < d; ++k) y[k] = 0.0;
@@ -235,8 +264,12 @@ static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0,
  * with A_tau = prod_{l<=tau} g_l. Products are formed directly (no division).
  * Used to check the token-wise form; both share the per-token gates. */
 static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, double *n2,
-                               double *G, double *KT, double *XE, long long *deg)
+                               double *G, double *KT, double *XE, double *GS, double *G0,
+                               long long *deg)
 {
+    /* eq. recurrence_linear1's chunk form (eq. chunkwise_OSR) multiplies by the running
+     * gates gs and adds f / F terms for g0 s0; Eq. 17's multiplies by g = gs + g0. */
+    const int lin1 = J->lin == 1;
     const int T = J->T, H = J->H, m = J->m, d = J->d, C = J->C;
     for (int t0 = 0; t0 < T; t0 += C) {
         int L = (t0 + C < T ? t0 + C : T) - t0;
@@ -250,17 +283,27 @@ static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, do
             size_t tok = IDX_TOK(b, t0 + tau, h, T, H);
             double eta = J->eta ? J->eta[tok] : 1.0;
             oracle_write_input(J->mode, m, d, S0, J->c + tok * m, J->x + tok * d, XE + (size_t)tau * d);
-            oracle_chunk_token_gates(m, d, S0, n2, XE + (size_t)tau * d, J->c + tok * m, J->mu[tok],
-                                     eta, G + (size_t)tau * m, KT + (size_t)tau * m, NULL, deg);
+            oracle_chunk_token_gates2(m, d, S0, n2, XE + (size_t)tau * d, J->c + tok * m, J->mu[tok],
+                                      eta, G + (size_t)tau * m, KT + (size_t)tau * m, NULL, deg,
+                                      GS + (size_t)tau * m, G0 + (size_t)tau * m);
+            if (lin1) /* the products run over the running gates */
+                memcpy(G + (size_t)tau * m, GS + (size_t)tau * m, sizeof(double) * (size_t)m);
         }
         for (int tau = 0; tau < L; ++tau) {
             size_t tok = IDX_TOK(b, t0 + tau, h, T, H);
             const double *q = J->q + tok * m;
             double *y = J->y + tok * d;
             for (int k = 0; k < d; ++k) y[k] = 0.0;
-            for (int i = 0; i < m; ++i) { /* inter-chunk term (Q (.) A) S0 */
+            for (int i = 0; i < m; ++i) { /* inter-chunk term (Q (.) (A + F)) S0 */
                 double A = 1.0;
                 for (int l = 0; l <= tau; ++l) A *= G[(size_t)l * m + i];
+                if (lin1) { /* F_tau,i = sum_{j<=tau} g0_j,i prod_{l=j+1..tau} gs_l,i */
+                    for (int j = 0; j <= tau; ++j) {
+                        double prod = 1.0;
+                        for (int l = j + 1; l <= tau; ++l) prod *= G[(size_t)l * m + i];
+                        A += G0[(size_t)j * m + i] * prod;
+                    }
+                }
                 for (int k = 0; k < d; ++k) y[k] += q[i] * A * S0[(size_t)i * d + k];
             }
             for (int j = 0; j <= tau; ++j) { /* intra-chunk term P H */
@@ -277,6 +320,13 @@ static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, do
         for (int i = 0; i < m; ++i) { /* chunk-end state */
             double A = 1.0;
             for (int l = 0; l < L; ++l) A *= G[(size_t)l * m + i];
+            if (lin1) { /* + f_i = sum_j g0_j,i prod_{l=j+1..C} gs_l,i */
+                for (int j = 0; j < L; ++j) {
+                    double prod = 1.0;
+                    for (int l = j + 1; l < L; ++l) prod *= G[(size_t)l * m + i];
+                    A += G0[(size_t)j * m + i] * prod;
+                }
+            }
             for (int k = 0; k < d; ++k) S[(size_t)i * d + k] = A * S0[(size_t)i * d + k];
             for (int j = 0; j < L; ++j) {
                 double prod = 1.0;
@@ -301,6 +351,8 @@ static void *worker(void *arg)
     double *G = malloc(sizeof(double) * (size_t)C * m);
     double *KT = malloc(sizeof(double) * (size_t)C * m);
     double *XE = malloc(sizeof(double) * (size_t)C * d);
+    double *GS = malloc(sizeof(double) * (size_t)C * m);
+    double *G0 = malloc(sizeof(double) * (size_t)C * m);
     long long deg = 0;
     for (;;) {
         pthread_mutex_lock(&J->lock);
@@ -313,25 +365,26 @@ static void *worker(void *arg)
         if (J->form == 0)
             run_exact(J, b, h, S, w, XE, &deg);
         else if (J->form == 1)
-            run_chunked_tokenwise(J, b, h, S, S0, n2, G, KT, XE, &deg);
+            run_chunked_tokenwise(J, b, h, S, S0, n2, G, KT, XE, GS, G0, &deg);
         else
-            run_chunked_matrix(J, b, h, S, S0, n2, G, KT, XE, &deg);
+            run_chunked_matrix(J, b, h, S, S0, n2, G, KT, XE, GS, G0, &deg);
         if (J->S_out) memcpy(J->S_out + so, S, sizeof(double) * (size_t)m * d);
     }
     pthread_mutex_lock(&J->lock);
     J->degenerate += deg;
     pthread_mutex_unlock(&J->lock);
-    free(S); free(S0); free(n2); free(w); free(G); free(KT); free(XE);
+    free(S); free(S0); free(n2); free(w); free(G); free(KT); free(XE); free(GS); free(G0);
     return NULL;
 }
 
-static long long run(int form, int mode, int B, int T, int H, int m, int d, int C, const double *x,
-                     const double *c, const double *q, const double *mu, const double *eta,
-                     const double *S0, double *S_out, double *y, int nthreads)
+static long long run_lin(int form, int mode, int lin, int B, int T, int H, int m, int d, int C,
+                         const double *x, const double *c, const double *q, const double *mu,
+                         const double *eta, const double *S0, double *S_out, double *y,
+                         int nthreads)
 {
     job_t J;
     memset(&J, 0, sizeof(J));
-    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C; J.form = form; J.mode = mode;
+    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C; J.form = form; J.mode = mode; J.lin = lin;
     J.x = x; J.c = c; J.q = q; J.mu = mu; J.eta = eta; J.S0 = S0; J.S_out = S_out; J.y = y;
     pthread_mutex_init(&J.lock, NULL);
     if (nthreads < 1) nthreads = 1;
@@ -346,6 +399,24 @@ static long long run(int form, int mode, int B, int T, int H, int m, int d, int 
     }
     pthread_mutex_destroy(&J.lock);
     return J.degenerate;
+}
+
+static long long run(int form, int mode, int B, int T, int H, int m, int d, int C, const double *x,
+                     const double *c, const double *q, const double *mu, const double *eta,
+                     const double *S0, double *S_out, double *y, int nthreads)
+{
+    return run_lin(form, mode, 2, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
+}
+
+/* Chunked recurrence in either linearisation of §3.4.1 (lin 2: Eq. 17,
+ * recurrence_linear2; lin 1: recurrence_linear1), token by token (form 1) or through
+ * the chunk closed form (form 2). */
+long long oracle_chunked_scan_lin(int form, int mode, int lin, int B, int T, int H, int m, int d,
+                                  int C, const double *x, const double *c, const double *q,
+                                  const double *mu, const double *eta, const double *S0,
+                                  double *S_out, double *y, int nthreads)
+{
+    return run_lin(form, mode, lin, B, T, H, m, d, C, x, c, q, mu, eta, S0, S_out, y, nthreads);
 }
 
 /* Whole-sequence drivers. mode 0: similarity objective (h = -x); mode 1:

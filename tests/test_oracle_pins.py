@@ -473,3 +473,62 @@ def test_dec_differs_from_sim():
     ys, _, _ = oracle.scan(x, c, q, mu, S0, mode="sim")
     yd, _, _ = oracle.scan(x, c, q, mu, S0, mode="dec")
     assert np.abs(ys - yd).max() > 1e-3
+
+
+# ------------------------------------------- linearisation 1 (recurrence_linear1) ---
+
+def test_lin1_chunk_size_one_is_the_exact_recurrence():
+    """§3.4.1: with chunk size 1 the chunk-start state is the current state, so
+    eq. (recurrence_linear1) is the exact recurrence."""
+    rng = _rng(31)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 11, 2, 5, 6, unit=True)
+    y1, S1, _ = oracle.scan(x, c, q, mu, S0, chunk=1)
+    from oracle import _load, _f64, _p
+    lib = _load()
+    B, T, H, d = x.shape
+    m = c.shape[-1]
+    y2, S2 = np.zeros_like(y1), np.zeros_like(S1)
+    lib.oracle_chunked_scan_lin(1, 0, 1, B, T, H, m, d, 1, _p(_f64(x)), _p(_f64(c)), _p(_f64(q)),
+                                _p(_f64(mu)), None, _p(_f64(S0)), _p(S2), _p(y2), 1)
+    np.testing.assert_allclose(y2, y1, atol=1e-12)
+    np.testing.assert_allclose(S2, S1, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [4, 16])
+@pytest.mark.parametrize("mode", ["sim", "dec"])
+def test_lin1_chunk_closed_form_equals_token_form(C, mode):
+    """eq. (chunkwise_OSR): the chunk-level form of recurrence_linear1 - gates
+    a_tau = prod beta mu, the f / F terms carrying h~ k^ on the chunk-start state,
+    the causal score matrix - equals the token-wise recurrence."""
+    rng = _rng(300 + C)
+    T = 2 * C + 5
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, T, 2, 5, 4, unit=False, mu_range=(0.6, 1.0))
+    if mode == "dec":
+        c *= 0.1
+    y1, S1, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="token", lin=1, mode=mode)
+    y2, S2, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="matrix", lin=1, mode=mode)
+    np.testing.assert_allclose(y2, y1, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(S2, S1, rtol=1e-10, atol=1e-10)
+
+
+def test_lin1_first_token_is_exact_and_differs_from_eq17_later():
+    """Both linearisations are exact on the first token of a chunk; afterwards
+    recurrence_linear1 (h~ k^ on the chunk-start slot) and Eq. 17 (on the running
+    slot) differ."""
+    rng = _rng(32)
+    C = 8
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, C, 1, 4, 6)
+    ye, _, _ = oracle.scan(x, c, q, mu, S0, chunk=1)
+    y1, _, _ = oracle.scan(x, c, q, mu, S0, chunk=C, lin=1)
+    y2, _, _ = oracle.scan(x, c, q, mu, S0, chunk=C, lin=2)
+    np.testing.assert_allclose(y1[:, 0], ye[:, 0], atol=1e-13)
+    assert np.abs(y1[:, -1] - y2[:, -1]).max() > 1e-6
+
+
+def test_lin1_on_the_training_shape_stays_bounded():
+    import lattice_inputs as LI
+    inp = LI.make_inputs(LI.WORKLOADS["small_train"].with_(B=1, H=2))
+    y, S, deg = oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=64, lin=1)
+    assert np.isfinite(y).all() and deg == 0
+    n = np.linalg.norm(S, axis=-1)
+    assert 0.05 < n.min() and n.max() < 20.0
