@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.lattice_scan_fwd.argtypes = [vp, i, fp, vp, i, fp, fp, fp, fp, fp, i, i, i, i, i, i, i, vp]
         L.lattice_scan_fwd_impl.argtypes = [vp, i, fp, vp, i, fp, fp, fp, fp, fp, i, i, i, i, i,
                                             i, i, i, vp]
+        L.lattice_scan_fwd_ex.argtypes = [vp, i, fp, vp, i, fp, fp, fp, fp, fp, i, i, i, i, i,
+                                          i, i, i, i, vp]
         L.lattice_step.argtypes = [fp, vp, i, fp, vp, i, fp, fp, fp, i, i, i, i, i, vp]
         L.lattice_readout.argtypes = [fp, vp, i, fp, i, i, i, i, vp]
         L.lattice_get_device_status.argtypes = [vp]
@@ -65,7 +67,7 @@ def lib() -> ctypes.CDLL:
         L.lattice_chunk_impl.argtypes = [i, i, i, i, i, i, i]
         L.lattice_last_cuda_error.argtypes = []
         L.lattice_last_cuda_error.restype = ctypes.c_char_p
-        for f in ("lattice_scan_fwd", "lattice_scan_fwd_impl", "lattice_step", "lattice_readout",
+        for f in ("lattice_scan_fwd", "lattice_scan_fwd_impl", "lattice_scan_fwd_ex", "lattice_step", "lattice_readout",
                   "lattice_get_device_status", "lattice_version", "lattice_chunk_impl"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -111,10 +113,12 @@ _XQ = (torch.float32, torch.bfloat16)
 def scan_fwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor,
              S0: torch.Tensor, eta: Optional[torch.Tensor] = None, chunk: int = 1,
              S_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
-             impl: str = "auto", stream=None, mode: str = "sim") -> Tuple[torch.Tensor, torch.Tensor]:
+             impl: str = "auto", stream=None, mode: str = "sim",
+             lin: int = 2) -> Tuple[torch.Tensor, torch.Tensor]:
     """Whole-sequence forward (the paper's lattice_compress, Appendix D).
-    chunk == 1: exact recurrence; chunk > 1: the Eq. 17 chunked form.
-    mode "sim": similarity objective; "dec": reconstruction objective.
+    chunk == 1: exact recurrence; chunk > 1: the chunked form, Eq. 17 (lin=2) or
+    eq. recurrence_linear1 (lin=1). mode "sim": similarity objective; "dec":
+    reconstruction objective.
     Returns (y [B,T,H,d] float32, S_T [B,H,m,d] float32). S_out may be S0."""
     B, T, H, d = x.shape
     m = c.shape[-1]
@@ -132,9 +136,9 @@ def scan_fwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor
         y = torch.empty((B, T, H, d), dtype=torch.float32, device=x.device)
     _chk(y, "y", (B, T, H, d))
     L = lib()
-    code = L.lattice_scan_fwd_impl(_ptr(x), _dt(x), _ptr(c), _ptr(q), _dt(q), _ptr(mu), _ptr(eta),
-                                   _ptr(S0), _ptr(S_out), _ptr(y), B, T, H, m, d, int(chunk),
-                                   _MODE[mode], _IMPL[impl], _stream(stream))
+    code = L.lattice_scan_fwd_ex(_ptr(x), _dt(x), _ptr(c), _ptr(q), _dt(q), _ptr(mu), _ptr(eta),
+                                 _ptr(S0), _ptr(S_out), _ptr(y), B, T, H, m, d, int(chunk),
+                                 _MODE[mode], {2: 0, 1: 1}[lin], _IMPL[impl], _stream(stream))
     _raise(code, "lattice_scan_fwd")
     return y, S_out
 

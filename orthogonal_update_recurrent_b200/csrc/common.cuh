@@ -175,4 +175,26 @@ __device__ __forceinline__ void update_coefs(float n2, float p, float xx, float 
     gamma = ok ? a * iw : 0.f;
 }
 
+// As update_coefs, split for the chunk linearisation of eq. recurrence_linear1
+// (§3.4.1): the new slot is alpha_s*s + alpha_0*s0 + gamma*x, where the forget part
+// mu scales the running slot s and the projection part (-a p/n^2) the chunk-start
+// slot s0 (alpha_s + alpha_0 is update_coefs' alpha).
+template <bool PRECISE>
+__device__ __forceinline__ void update_coefs_lin1(float n2, float p, float xx, float c, float mu,
+                                                  float eta, float target, float& alpha_s,
+                                                  float& alpha_0, float& gamma) {
+    bool ok = n2 > 0.f;
+    float n2s = ok ? n2 : 1.f;
+    float inv_n = PRECISE ? __frsqrt_rn(n2s) : rsqrtf(n2s);
+    float r = PRECISE ? __fdiv_rn(p, n2s) : __fdividef(p, n2s);
+    float a = eta * c * inv_n;
+    float perp2 = fmaxf(fmaf(-p, r, xx), 0.f);
+    float w2 = fmaf(a * a, perp2, mu * mu * n2s);
+    ok = ok && (w2 > 0.f);
+    float iw = (PRECISE ? __frsqrt_rn(ok ? w2 : 1.f) : rsqrtf(ok ? w2 : 1.f)) * target;
+    alpha_s = ok ? mu * iw : 1.f;
+    alpha_0 = ok ? -a * r * iw : 0.f;
+    gamma = ok ? a * iw : 0.f;
+}
+
 }  // namespace lattice

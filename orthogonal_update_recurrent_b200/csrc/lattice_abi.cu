@@ -52,38 +52,45 @@ lattice_status launch_status() {
 }
 
 // ---- exact / chunked CUDA-core scan
-template <int D, int RQ, bool CH, bool DEC>
+template <int D, int RQ, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
     size_t smem = scan_smem_bytes<D>(a.m, nw, DEC);
-    auto k = scan_simt_kernel<D, RQ, CH, DEC>;
+    auto k = scan_simt_kernel<D, RQ, CH, DEC, LIN1>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e);
     k<<<a.B * a.H, nw * 32, smem, st>>>(a);
     return launch_status();
 }
 
-template <int D, bool CH, bool DEC>
+template <int D, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
     const int quads = (a.m + 3) / 4;
-    if (quads <= 16) return launch_scan_simt_t<D, 1, CH, DEC>(a, quads < 4 ? 4 : quads, st);
-    if (quads <= 32) return launch_scan_simt_t<D, 2, CH, DEC>(a, 16, st);
-    return launch_scan_simt_t<D, 4, CH, DEC>(a, 16, st);
+    if (quads <= 16) return launch_scan_simt_t<D, 1, CH, DEC, LIN1>(a, quads < 4 ? 4 : quads, st);
+    if (quads <= 32) return launch_scan_simt_t<D, 2, CH, DEC, LIN1>(a, 16, st);
+    return launch_scan_simt_t<D, 4, CH, DEC, LIN1>(a, 16, st);
 }
 
-template <bool CH, bool DEC>
+template <bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_m(const ScanArgs& a, int d, cudaStream_t st) {
     switch (d) {
-        case 16: return launch_scan_simt_d<16, CH, DEC>(a, st);
-        case 32: return launch_scan_simt_d<32, CH, DEC>(a, st);
-        case 64: return launch_scan_simt_d<64, CH, DEC>(a, st);
-        case 128: return launch_scan_simt_d<128, CH, DEC>(a, st);
+        case 16: return launch_scan_simt_d<16, CH, DEC, LIN1>(a, st);
+        case 32: return launch_scan_simt_d<32, CH, DEC, LIN1>(a, st);
+        case 64: return launch_scan_simt_d<64, CH, DEC, LIN1>(a, st);
+        case 128: return launch_scan_simt_d<128, CH, DEC, LIN1>(a, st);
     }
     return LATTICE_ERR_UNSUPPORTED;
 }
 
+// exact: CH = false (LIN1 does not apply); chunked: either linearisation
 template <bool CH>
-lattice_status launch_scan_simt(const ScanArgs& a, int d, bool dec, cudaStream_t st) {
-    return dec ? launch_scan_simt_m<CH, true>(a, d, st) : launch_scan_simt_m<CH, false>(a, d, st);
+lattice_status launch_scan_simt(const ScanArgs& a, int d, bool dec, bool lin1, cudaStream_t st) {
+    if constexpr (!CH) {
+        return dec ? launch_scan_simt_m<false, true, false>(a, d, st) : launch_scan_simt_m<false, false, false>(a, d, st);
+    } else {
+        if (lin1)
+            return dec ? launch_scan_simt_m<true, true, true>(a, d, st) : launch_scan_simt_m<true, false, true>(a, d, st);
+        return dec ? launch_scan_simt_m<true, true, false>(a, d, st) : launch_scan_simt_m<true, false, false>(a, d, st);
+    }
 }
 
 // ---- decode step / read-out: NW warps x RQ quads per warp
@@ -161,11 +168,14 @@ lattice_impl lattice_chunk_impl(int B, int H, int m, int d, int chunk_size, latt
     return LATTICE_IMPL_SIMT;
 }
 
-lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const float* c,
-                                     const void* q, lattice_dtype q_dtype, const float* mu,
-                                     const float* eta, const float* S0, float* S_out, float* y,
-                                     int B, int T, int H, int m, int d, int chunk_size,
-                                     lattice_mode mode, lattice_impl impl, void* stream) {
+lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const float* c,
+                                   const void* q, lattice_dtype q_dtype, const float* mu,
+                                   const float* eta, const float* S0, float* S_out, float* y,
+                                   int B, int T, int H, int m, int d, int chunk_size,
+                                   lattice_mode mode, lattice_chunk_form form, lattice_impl impl,
+                                   void* stream) {
+    if (form != LATTICE_CHUNK_LIN2 && form != LATTICE_CHUNK_LIN1) return LATTICE_ERR_INVALID_ARG;
+    const bool lin1 = form == LATTICE_CHUNK_LIN1;
     if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return LATTICE_ERR_INVALID_ARG;
     if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
     if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05 &&
@@ -204,9 +214,10 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
     ScanArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, S_out, y,
                B, T, H, m, chunk_size};
     const bool tc_choice = impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT;
-    if (chunk_size == 1 || dec) {  // the tensor-core kernels run the similarity objective
+    if (chunk_size == 1 || dec || lin1) {  // the tensor-core kernels run Eq. 17, similarity objective
         if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
-        return chunk_size == 1 ? launch_scan_simt<false>(a, d, dec, st) : launch_scan_simt<true>(a, d, dec, st);
+        return chunk_size == 1 ? launch_scan_simt<false>(a, d, dec, false, st)
+                               : launch_scan_simt<true>(a, d, dec, lin1, st);
     }
     if (impl == LATTICE_IMPL_AUTO) impl = lattice_chunk_impl(B, H, m, d, chunk_size, x_dtype, q_dtype);
     if (impl == LATTICE_IMPL_TCGEN05_SPLIT) {
@@ -219,7 +230,16 @@ lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const
         cudaError_t e = launch_chunk_tc(a, d, st);
         return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
     }
-    return launch_scan_simt<true>(a, d, false, st);
+    return launch_scan_simt<true>(a, d, false, false, st);
+}
+
+lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const float* c,
+                                     const void* q, lattice_dtype q_dtype, const float* mu,
+                                     const float* eta, const float* S0, float* S_out, float* y,
+                                     int B, int T, int H, int m, int d, int chunk_size,
+                                     lattice_mode mode, lattice_impl impl, void* stream) {
+    return lattice_scan_fwd_ex(x, x_dtype, c, q, q_dtype, mu, eta, S0, S_out, y, B, T, H, m, d,
+                               chunk_size, mode, LATTICE_CHUNK_LIN2, impl, stream);
 }
 
 lattice_status lattice_scan_fwd(const void* x, lattice_dtype x_dtype, const float* c,

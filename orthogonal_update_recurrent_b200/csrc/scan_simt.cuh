@@ -49,7 +49,10 @@ __host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec) {
 // token's write direction is x - sum_i (c_i/|s_i|) s_i, with the slots of the state
 // the token's projection uses (the current state; the chunk-start state when
 // CHUNKED). It costs one cross-warp reduction and one barrier per token.
-template <int D, int RQ, bool CHUNKED, bool DEC>
+// LIN1 (chunked only) selects the chunk linearisation of eq. recurrence_linear1
+// (§3.4.1): the projection part of each token's update scales the chunk-start slot
+// instead of the running one.
+template <int D, int RQ, bool CHUNKED, bool DEC, bool LIN1 = false>
 __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
@@ -233,14 +236,25 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
                 const bool valid = slot[r] < m;
                 const float cv = valid ? rec[D + m + slot[r]] : 0.f;
                 const float qv = valid ? rec[D + slot[r]] : 0.f;
-                float alpha, gamma;
-                update_coefs<CHUNKED || DEC>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
-                                             CHUNKED ? n0[r] : 1.f, alpha, gamma);
-                if (!valid) { alpha = 0.f; gamma = 0.f; }
+                if constexpr (CHUNKED && LIN1) {
+                    float alpha_s, alpha_0, gamma;
+                    update_coefs_lin1<true>(n0sq[r], p[r], xx, cv, mu, eta, n0[r], alpha_s, alpha_0, gamma);
+                    if (!valid) { alpha_s = 0.f; alpha_0 = 0.f; gamma = 0.f; }
 #pragma unroll
-                for (int k = 0; k < EPL; ++k) {
-                    s[r][k] = fmaf(alpha, s[r][k], gamma * xv[k]);
-                    yp[k] = fmaf(qv, s[r][k], yp[k]);
+                    for (int k = 0; k < EPL; ++k) {
+                        s[r][k] = fmaf(alpha_s, s[r][k], fmaf(alpha_0, s0[r][k], gamma * xv[k]));
+                        yp[k] = fmaf(qv, s[r][k], yp[k]);
+                    }
+                } else {
+                    float alpha, gamma;
+                    update_coefs<CHUNKED || DEC>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
+                                                 CHUNKED ? n0[r] : 1.f, alpha, gamma);
+                    if (!valid) { alpha = 0.f; gamma = 0.f; }
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) {
+                        s[r][k] = fmaf(alpha, s[r][k], gamma * xv[k]);
+                        yp[k] = fmaf(qv, s[r][k], yp[k]);
+                    }
                 }
             }
             // reduce the read-out over the 4 octets of the warp (reduce-scatter)

@@ -65,6 +65,12 @@ def test_argument_checks_return_before_launch(lib):
     assert _scan(lib, m=257) == L.ERR_UNSUPPORTED
     assert _scan(lib, xdt=7) == L.ERR_INVALID_ARG
     assert _scan(lib, mode=2) == L.ERR_INVALID_ARG
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    ex = lambda form, impl: lib.lattice_scan_fwd_ex(v(1 << 20), 0, v(2 << 20), v(3 << 20), 0, v(4 << 20), None,
+                                                    v(5 << 20), v(6 << 20), v(7 << 20), 1, 4, 1, 64, 64, 64,
+                                                    0, form, impl, None)
+    assert ex(5, 0) == L.ERR_INVALID_ARG        # unknown chunk form
+    assert ex(1, 2) == L.ERR_UNSUPPORTED        # linearisation 1 runs on the CUDA-core kernel
     assert _scan(lib, mode=1, impl=2) == L.ERR_UNSUPPORTED  # DEC runs on the CUDA-core kernels
     assert _scan(lib, mode=1, chunk=64, impl=3) == L.ERR_UNSUPPORTED
     assert _scan(lib, impl=9) == L.ERR_INVALID_ARG

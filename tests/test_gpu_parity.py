@@ -33,18 +33,18 @@ def L():
     return L
 
 
-def run_gpu(L, inp, chunk, impl="auto", eta=None, mode="sim"):
+def run_gpu(L, inp, chunk, impl="auto", eta=None, mode="sim", lin=2):
     t = dev_inputs(inp)
     y, S = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], eta=t["eta"] if eta is None else eta,
-                      chunk=chunk, impl=impl, mode=mode)
+                      chunk=chunk, impl=impl, mode=mode, lin=lin)
     torch.cuda.synchronize()
     L.device_status()
     return y.cpu().numpy(), S.cpu().numpy()
 
 
-def run_oracle(inp, chunk, mode="sim"):
+def run_oracle(inp, chunk, mode="sim", lin=2):
     y, S, _ = oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], eta=inp["eta"],
-                          chunk=chunk, mode=mode)
+                          chunk=chunk, mode=mode, lin=lin)
     return y, S
 
 
@@ -465,3 +465,53 @@ def test_dec_full_size(L, name, pairs, chunk):
     bs = [p[0] for p in pairs]
     hs = [p[1] for p in pairs]
     assert y_err(yg[bs, :4, hs][:, :, None], yo) <= TOL_F32
+
+
+# ------------------------------------- chunk linearisation 1 (recurrence_linear1)
+
+@pytest.mark.parametrize("m,d,C", [(16, 32, 4), (64, 64, 64), (128, 128, 64), (64, 128, 16), (48, 16, 8)])
+def test_lin1_chunked(L, m, d, C):
+    """eq. recurrence_linear1 on the CUDA-core kernel vs the oracle: several chunks
+    and a ragged tail."""
+    w = LI.Workload("t", B=2, T=2 * C + C // 2 + 3, H=2, m=m, d=d, seed=600 + m + d + C)
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, C, lin=1)
+    yo, So = run_oracle(inp, C, lin=1)
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
+
+
+def test_lin1_dec_resynchronised(L):
+    w = LI.Workload("t", B=2, T=3 * 16 + 5, H=2, m=32, d=64, seed=610, c_loc=DEC_CHUNK_C_LOC)
+    inp = LI.make_inputs(w)
+    T = inp["x"].shape[1]
+    S = inp["S0"].astype(np.float32)
+    for t0 in range(0, T, 16):
+        sub = {k: (v[:, t0:t0 + 16] if isinstance(v, np.ndarray) and v.ndim >= 3 and k != "S0" else v)
+               for k, v in inp.items()}
+        sub["S0"] = S
+        yg, Sg = run_gpu(L, sub, 16, mode="dec", lin=1)
+        yo, So = run_oracle(sub, 16, mode="dec", lin=1)
+        assert y_err(yg, yo) <= TOL_F32 and s_err(Sg, So) <= TOL_F32
+        S = So.astype(np.float32)
+
+
+def test_lin1_tensor_core_choices_are_unsupported(L):
+    w = LI.Workload("t", B=1, T=64, H=1, m=64, d=64, seed=1)
+    inp = LI.make_inputs(w)
+    for impl in ("tcgen05", "tcgen05_split"):
+        with pytest.raises(L.LatticeError):
+            run_gpu(L, inp, 64, impl=impl, lin=1)
+
+
+@pytest.mark.parametrize("name,pairs", FULL[:1])
+def test_lin1_full_size_sampled(L, name, pairs):
+    w = LI.WORKLOADS[name]
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, w.chunk, lin=1)
+    sub = LI.sample_heads(inp, pairs)
+    yo, So = run_oracle(sub, w.chunk, lin=1)
+    bs = [p[0] for p in pairs]
+    hs = [p[1] for p in pairs]
+    assert y_err(yg[bs, :, hs][:, :, None], yo) <= TOL_TC
+    assert s_err(Sg[bs, hs][:, None], So) <= TOL_TC
