@@ -92,14 +92,16 @@ _MODES = {"sim": 0, "dec": 1}
 
 
 def scan(x, c, q, mu, S0, eta=None, chunk: int = 1, form: str = "token",
-         nthreads: Optional[int] = None, mode: str = "sim", lin: int = 2):
+         nthreads: Optional[int] = None, mode: str = "sim", lin: int = 2, norm: str = "token"):
     """Whole-sequence forward. x[B][T][H][d], c/q[B][T][H][m], mu/eta[B][T][H],
     S0[B][H][m][d]. chunk == 1: exact recurrence; chunk > 1: Eq. 17 chunked
     recurrence, evaluated token by token (form="token") or through the
     chunk-level closed form (form="matrix"). mode "sim": similarity objective
     (h = -x); "dec": reconstruction objective (h = phi(S) c - x). lin selects the
     chunk linearisation of §3.4.1: 2 = Eq. 17 (recurrence_linear2), 1 =
-    recurrence_linear1. Returns (y, S_T, n_degenerate)."""
+    recurrence_linear1. norm "token": the per-token normaliser; "chunk": none inside
+    a chunk, every slot projected onto the unit sphere after each chunk (Appendix C
+    ablation). Returns (y, S_T, n_degenerate)."""
     md = _MODES[mode]
     x, c, q, mu, S0 = map(_f64, (x, c, q, mu, S0))
     eta = None if eta is None else _f64(eta)
@@ -112,12 +114,15 @@ def scan(x, c, q, mu, S0, eta=None, chunk: int = 1, form: str = "token",
     lib = _load()
     nt = _threads(nthreads)
     args = (_p(x), _p(c), _p(q), _p(mu), _p(eta), _p(S0), _p(S), _p(y), nt)
-    if lin not in (1, 2):
-        raise ValueError(lin)
-    if chunk == 1 and form == "token":
+    if lin not in (1, 2) or norm not in ("token", "chunk"):
+        raise ValueError((lin, norm))
+    if norm == "chunk" or lin == 1:
+        code = lin | (4 if norm == "chunk" else 0)
+        if form not in ("token", "matrix"):
+            raise ValueError(form)
+        deg = lib.oracle_chunked_scan_lin(1 if form == "token" else 2, md, code, B, T, H, m, d, chunk, *args)
+    elif chunk == 1 and form == "token":
         deg = lib.oracle_exact_scan_mode(md, B, T, H, m, d, *args)
-    elif lin == 1 and form in ("token", "matrix"):
-        deg = lib.oracle_chunked_scan_lin(1 if form == "token" else 2, md, 1, B, T, H, m, d, chunk, *args)
     elif form == "token":
         deg = lib.oracle_chunked_scan_mode(md, B, T, H, m, d, chunk, *args)
     elif form == "matrix":

@@ -148,21 +148,23 @@ static void exact_token(int m, int d, double *S, const double *x, const double *
 void oracle_chunk_token_gates2(int m, int d, const double *S0, const double *n2,
                                const double *x, const double *c, double mu, double eta,
                                double *g, double *kt, double *dsq_out, long long *degenerate,
-                               double *gs, double *g0);
+                               double *gs, double *g0, int nobeta);
 void oracle_chunk_token_gates(int m, int d, const double *S0, const double *n2,
                               const double *x, const double *c, double mu, double eta,
                               double *g, double *kt, double *dsq_out, long long *degenerate)
 {
-    oracle_chunk_token_gates2(m, d, S0, n2, x, c, mu, eta, g, kt, dsq_out, degenerate, NULL, NULL);
+    oracle_chunk_token_gates2(m, d, S0, n2, x, c, mu, eta, g, kt, dsq_out, degenerate, NULL, NULL, 0);
 }
 
 /* As above, and the two parts of g: gs_i = beta_i mu (what scales the running slot
  * in eq. recurrence_linear1, the G_t of §3.4.1) and g0_i = beta_i eta hhat_i khat_i
- * (what scales the chunk-start slot there); g = gs + g0. */
+ * (what scales the chunk-start slot there); g = gs + g0. nobeta != 0 drops the
+ * per-token normaliser (beta = 1), for normalisation at chunk boundaries only
+ * (Appendix C, "Per-token vs. Per-chunk Normalization"). */
 void oracle_chunk_token_gates2(int m, int d, const double *S0, const double *n2,
                                const double *x, const double *c, double mu, double eta,
                                double *g, double *kt, double *dsq_out, long long *degenerate,
-                               double *gs, double *g0)
+                               double *gs, double *g0, int nobeta)
 {
     double hh = 0.0;
     for (int k = 0; k < d; ++k) hh += x[k] * x[k]; /* |h|^2, h = -x */
@@ -176,6 +178,12 @@ void oracle_chunk_token_gates2(int m, int d, const double *S0, const double *n2,
         double dsq = eta * eta * (t > 0.0 ? t : 0.0);
         double den = mu * mu * n2[i] + dsq;
         if (dsq_out) dsq_out[i] = dsq;
+        if (nobeta) {
+            g[i] = mu + eta * hhat * khat;
+            kt[i] = -eta * khat;
+            if (gs) { gs[i] = mu; g0[i] = eta * hhat * khat; }
+            continue;
+        }
         if (den == 0.0) { /* zero-norm update: keep the slot */
             g[i] = 1.0;
             kt[i] = 0.0;
@@ -198,6 +206,7 @@ typedef struct {
     int B, T, H, m, d, C, form; /* form: 0 exact, 1 chunked token-wise, 2 chunked matrix form */
     int mode;                   /* 0 similarity objective, 1 reconstruction objective */
     int lin;                    /* chunked forms: 2 Eq. 17 (recurrence_linear2), 1 recurrence_linear1 */
+    int cnorm;                  /* chunked forms: 0 per-token normaliser, 1 normalise at chunk ends */
     const double *x, *c, *q, *mu, *eta, *S0;
     double *S_out, *y;
     long long degenerate;
@@ -214,6 +223,18 @@ static void run_exact(job_t *J, int b, int h, double *S, double *w, double *xe, 
         oracle_write_input(J->mode, m, d, S, J->c + tok * m, J->x + tok * d, xe); /* before the update */
         exact_token(m, d, S, xe, J->c + tok * m, J->q + tok * m, J->mu[tok], eta, J->y + tok * d, w,
                     deg);
+    }
+}
+
+/* Projection of every slot onto the unit sphere (§3.2), at a chunk boundary. */
+static void normalise_slots(int m, int d, double *S)
+{
+    for (int i = 0; i < m; ++i) {
+        double *s = S + (size_t)i * d, n2 = 0.0;
+        for (int k = 0; k < d; ++k) n2 += s[k] * s[k];
+        if (n2 == 0.0) continue;
+        double n = sqrt(n2);
+        for (int k = 0; k < d; ++k) s[k] /= n;
     }
 }
 
@@ -236,7 +257,7 @@ static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0,
             const double *x = xe;
             double eta = J->eta ? J->eta[tok] : 1.0;
             oracle_chunk_token_gates2(m, d, S0, n2, x, J->c + tok * m, J->mu[tok], eta, g, kt,
-                                      NULL, deg, gs, g0);
+                                      NULL, deg, gs, g0, J->cnorm);
             if (J->lin == 1) { /* eq. recurrence_linear1: s_i <- gs_i s_i + g0_i s0_i + kt_i h */
                 for (int i = 0; i < m; ++i)
                     for (int k = 0; k < d; ++k)
@@ -253,6 +274,7 @@ static void run_chunked_tokenwise(job_t *J, int b, int h, double *S, double *S0,
             for (int i = 0; i < m; ++i)
                 for (int k = 0; k < d; ++k) y[k] += q[i] * S[(size_t)i * d + k];
         }
+        if (J->cnorm) normalise_slots(m, d, S); /* after the chunk's last read-out */
     }
 }
 
@@ -285,7 +307,7 @@ static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, do
             oracle_write_input(J->mode, m, d, S0, J->c + tok * m, J->x + tok * d, XE + (size_t)tau * d);
             oracle_chunk_token_gates2(m, d, S0, n2, XE + (size_t)tau * d, J->c + tok * m, J->mu[tok],
                                       eta, G + (size_t)tau * m, KT + (size_t)tau * m, NULL, deg,
-                                      GS + (size_t)tau * m, G0 + (size_t)tau * m);
+                                      GS + (size_t)tau * m, G0 + (size_t)tau * m, J->cnorm);
             if (lin1) /* the products run over the running gates */
                 memcpy(G + (size_t)tau * m, GS + (size_t)tau * m, sizeof(double) * (size_t)m);
         }
@@ -336,6 +358,7 @@ static void run_chunked_matrix(job_t *J, int b, int h, double *S, double *S0, do
                 for (int k = 0; k < d; ++k) S[(size_t)i * d + k] += coef * (-xj[k]);
             }
         }
+        if (J->cnorm) normalise_slots(m, d, S);
     }
 }
 
@@ -384,7 +407,9 @@ static long long run_lin(int form, int mode, int lin, int B, int T, int H, int m
 {
     job_t J;
     memset(&J, 0, sizeof(J));
-    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C; J.form = form; J.mode = mode; J.lin = lin;
+    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C; J.form = form; J.mode = mode;
+    J.lin = lin & 3;
+    J.cnorm = (lin >> 2) & 1; /* lin | 4: normalise at chunk boundaries only */
     J.x = x; J.c = c; J.q = q; J.mu = mu; J.eta = eta; J.S0 = S0; J.S_out = S_out; J.y = y;
     pthread_mutex_init(&J.lock, NULL);
     if (nthreads < 1) nthreads = 1;
@@ -410,7 +435,8 @@ static long long run(int form, int mode, int B, int T, int H, int m, int d, int 
 
 /* Chunked recurrence in either linearisation of §3.4.1 (lin 2: Eq. 17,
  * recurrence_linear2; lin 1: recurrence_linear1), token by token (form 1) or through
- * the chunk closed form (form 2). */
+ * the chunk closed form (form 2). lin | 4 drops the per-token normaliser and projects
+ * the slots onto the unit sphere after each chunk instead (Appendix C ablation). */
 long long oracle_chunked_scan_lin(int form, int mode, int lin, int B, int T, int H, int m, int d,
                                   int C, const double *x, const double *c, const double *q,
                                   const double *mu, const double *eta, const double *S0,

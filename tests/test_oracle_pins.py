@@ -532,3 +532,41 @@ def test_lin1_on_the_training_shape_stays_bounded():
     assert np.isfinite(y).all() and deg == 0
     n = np.linalg.norm(S, axis=-1)
     assert 0.05 < n.min() and n.max() < 20.0
+
+
+# --------------------------------- normalisation at chunk boundaries (ablation) ---
+
+@pytest.mark.parametrize("lin", [1, 2])
+def test_chunk_norm_with_chunk_size_one_is_the_exact_recurrence(lin):
+    """Appendix C, "Per-token vs. Per-chunk Normalization": with no normaliser inside
+    a chunk and the unit-sphere projection after each chunk, chunk size 1 writes the
+    unnormalised OSR update and projects it: the exact recurrence (§3.2), for either
+    linearisation."""
+    rng = _rng(41 + lin)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 9, 2, 5, 6, unit=False)
+    ye, Se, _ = oracle.scan(x, c, q, mu, S0, chunk=1)
+    yc, Sc, _ = oracle.scan(x, c, q, mu, S0, chunk=1, lin=lin, norm="chunk")
+    np.testing.assert_allclose(Sc, Se, atol=1e-12)
+    # the read-out of a chunk precedes its boundary projection: y_t = q (|w| s_t)
+    np.testing.assert_allclose(np.linalg.norm(Sc, axis=-1), 1.0, atol=1e-12)
+    assert np.isfinite(yc).all()
+
+
+@pytest.mark.parametrize("lin", [1, 2])
+@pytest.mark.parametrize("C", [4, 16])
+def test_chunk_norm_closed_form_equals_token_form(lin, C):
+    rng = _rng(400 + C + lin)
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 2 * C + 3, 2, 5, 4, unit=True, mu_range=(0.6, 1.0))
+    y1, S1, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="token", lin=lin, norm="chunk")
+    y2, S2, _ = oracle.scan(x, c, q, mu, S0, chunk=C, form="matrix", lin=lin, norm="chunk")
+    np.testing.assert_allclose(y2, y1, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(S2, S1, rtol=1e-10, atol=1e-10)
+
+
+def test_chunk_norm_carried_state_is_on_the_sphere_and_differs_from_per_token():
+    rng = _rng(43)
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 3 * 8, 2, 5, 6, unit=True)
+    yc, Sc, _ = oracle.scan(x, c, q, mu, S0, chunk=8, norm="chunk")
+    yt, St, _ = oracle.scan(x, c, q, mu, S0, chunk=8)
+    np.testing.assert_allclose(np.linalg.norm(Sc, axis=-1), 1.0, atol=1e-12)
+    assert np.abs(yc - yt).max() > 1e-6
