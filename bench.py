@@ -183,13 +183,13 @@ def _dev_inputs(torch, inp, device):
                 mu=torch.from_numpy(inp["mu"]).to(device), S0=torch.from_numpy(inp["S0"]).to(device))
 
 
-def time_scan(torch, L, t, chunk, steps, warmup, flush=None, impl="auto", mode="sim", lin=2):
+def time_scan(torch, L, t, chunk, steps, warmup, flush=None, impl="auto", mode="sim", lin=2, norm="token"):
     """Per-step device time (ms) of lattice_scan_fwd, CUDA events on its stream."""
     stream = torch.cuda.current_stream()
     y = torch.empty(t["x"].shape[:3] + (t["S0"].shape[-1],), dtype=torch.float32, device=t["x"].device)
     S = torch.empty_like(t["S0"])
     run = lambda: L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], chunk=chunk, S_out=S, y=y,
-                             impl=impl, stream=stream, mode=mode, lin=lin)
+                             impl=impl, stream=stream, mode=mode, lin=lin, norm=norm)
     for _ in range(warmup):
         run()
     torch.cuda.synchronize()
@@ -467,6 +467,11 @@ def main():
                                               "kernel": "scan_simt_kernel<chunked, dec>",
                                               "inputs": "c = sigmoid(N(-4,1))"}
             del tdc
+            # the normalisation ablation of Appendix C (CUDA-core kernel)
+            tn = time_scan(torch, L, t, w.chunk, 5, 3, flush=flush, norm="chunk")
+            extra[f"{w.name}_chunk_norm"] = {"ms": statistics.mean(tn),
+                                             "tokens_per_s": w.B * w.T / (statistics.mean(tn) * 1e-3),
+                                             "kernel": "scan_simt_kernel<chunked, norm at chunk ends>"}
             # the other chunk linearisation (recurrence_linear1, CUDA-core kernel)
             tl = time_scan(torch, L, t, w.chunk, 5, 3, flush=flush, lin=1)
             extra[f"{w.name}_lin1_chunked"] = {"ms": statistics.mean(tl),

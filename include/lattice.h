@@ -126,16 +126,27 @@ lattice_status lattice_scan_fwd(const void *x, lattice_dtype x_dtype, const floa
                                 int B, int T, int H, int m, int d, int chunk_size,
                                 lattice_mode mode, void *stream);
 
-/* Chunk linearisation for chunk_size > 1 (§3.4.1):
+/* Chunk form for chunk_size > 1: a linearisation (§3.4.1), optionally OR'ed with
+ * LATTICE_CHUNK_NORM_AT_BOUNDARY.
  *   LATTICE_CHUNK_LIN2  Eq. 17 (recurrence_linear2), the default: within a chunk
  *                       each token's gate g = beta (mu + eta hhat khat) scales the
  *                       running slot.
  *   LATTICE_CHUNK_LIN1  eq. recurrence_linear1: the forget part beta mu scales
  *                       the running slot and the projection part beta eta hhat khat
  *                       the chunk-start slot (its chunk form is eq. chunkwise_OSR).
- * LIN1 runs on the CUDA-core kernel only: tensor-core choices return
- * LATTICE_ERR_UNSUPPORTED, and AUTO takes the CUDA-core kernel. */
-typedef enum { LATTICE_CHUNK_LIN2 = 0, LATTICE_CHUNK_LIN1 = 1 } lattice_chunk_form;
+ *   LATTICE_CHUNK_NORM_AT_BOUNDARY  the normalisation ablation of Appendix C
+ *                       ("Per-token vs. Per-chunk Normalization"): no per-token
+ *                       normaliser inside a chunk (beta = 1); every slot is
+ *                       projected onto the unit sphere after each chunk, once the
+ *                       chunk's read-outs are done. With chunk_size 1 this is the
+ *                       exact recurrence.
+ * LIN1 and NORM_AT_BOUNDARY run on the CUDA-core kernel only: tensor-core choices
+ * return LATTICE_ERR_UNSUPPORTED, and AUTO takes the CUDA-core kernel. */
+typedef enum {
+    LATTICE_CHUNK_LIN2 = 0,
+    LATTICE_CHUNK_LIN1 = 1,
+    LATTICE_CHUNK_NORM_AT_BOUNDARY = 2
+} lattice_chunk_form;
 
 /* As lattice_scan_fwd, with an explicit kernel choice (see lattice_impl). */
 lattice_status lattice_scan_fwd_impl(const void *x, lattice_dtype x_dtype, const float *c,
@@ -144,8 +155,9 @@ lattice_status lattice_scan_fwd_impl(const void *x, lattice_dtype x_dtype, const
                                      int B, int T, int H, int m, int d, int chunk_size,
                                      lattice_mode mode, lattice_impl impl, void *stream);
 
-/* As lattice_scan_fwd_impl, with the chunk linearisation (see lattice_chunk_form;
- * ignored for chunk_size 1). An unknown form is LATTICE_ERR_INVALID_ARG. */
+/* As lattice_scan_fwd_impl, with the chunk form (see lattice_chunk_form; values 0-3;
+ * the linearisation is ignored for chunk_size 1). Any other form is
+ * LATTICE_ERR_INVALID_ARG. */
 lattice_status lattice_scan_fwd_ex(const void *x, lattice_dtype x_dtype, const float *c,
                                    const void *q, lattice_dtype q_dtype, const float *mu,
                                    const float *eta, const float *S0, float *S_out, float *y,

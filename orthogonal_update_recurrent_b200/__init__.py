@@ -114,11 +114,12 @@ def scan_fwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor
              S0: torch.Tensor, eta: Optional[torch.Tensor] = None, chunk: int = 1,
              S_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
              impl: str = "auto", stream=None, mode: str = "sim",
-             lin: int = 2) -> Tuple[torch.Tensor, torch.Tensor]:
+             lin: int = 2, norm: str = "token") -> Tuple[torch.Tensor, torch.Tensor]:
     """Whole-sequence forward (the paper's lattice_compress, Appendix D).
     chunk == 1: exact recurrence; chunk > 1: the chunked form, Eq. 17 (lin=2) or
-    eq. recurrence_linear1 (lin=1). mode "sim": similarity objective; "dec":
-    reconstruction objective.
+    eq. recurrence_linear1 (lin=1); norm "chunk" drops the per-token normaliser and
+    projects the slots onto the unit sphere after each chunk. mode "sim": similarity
+    objective; "dec": reconstruction objective.
     Returns (y [B,T,H,d] float32, S_T [B,H,m,d] float32). S_out may be S0."""
     B, T, H, d = x.shape
     m = c.shape[-1]
@@ -138,7 +139,8 @@ def scan_fwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor
     L = lib()
     code = L.lattice_scan_fwd_ex(_ptr(x), _dt(x), _ptr(c), _ptr(q), _dt(q), _ptr(mu), _ptr(eta),
                                  _ptr(S0), _ptr(S_out), _ptr(y), B, T, H, m, d, int(chunk),
-                                 _MODE[mode], {2: 0, 1: 1}[lin], _IMPL[impl], _stream(stream))
+                                 _MODE[mode], {2: 0, 1: 1}[lin] | {"token": 0, "chunk": 2}[norm],
+                                 _IMPL[impl], _stream(stream))
     _raise(code, "lattice_scan_fwd")
     return y, S_out
 

@@ -174,8 +174,9 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
                                    int B, int T, int H, int m, int d, int chunk_size,
                                    lattice_mode mode, lattice_chunk_form form, lattice_impl impl,
                                    void* stream) {
-    if (form != LATTICE_CHUNK_LIN2 && form != LATTICE_CHUNK_LIN1) return LATTICE_ERR_INVALID_ARG;
-    const bool lin1 = form == LATTICE_CHUNK_LIN1;
+    if ((int)form < 0 || (int)form > 3) return LATTICE_ERR_INVALID_ARG;
+    const bool lin1 = ((int)form & LATTICE_CHUNK_LIN1) != 0;
+    const bool cnorm = ((int)form & LATTICE_CHUNK_NORM_AT_BOUNDARY) != 0;
     if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return LATTICE_ERR_INVALID_ARG;
     if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
     if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05 &&
@@ -214,7 +215,12 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
     ScanArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, S_out, y,
                B, T, H, m, chunk_size};
     const bool tc_choice = impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT;
-    if (chunk_size == 1 || dec || lin1) {  // the tensor-core kernels run Eq. 17, similarity objective
+    a.cnorm = cnorm && chunk_size > 1 ? 1 : 0;
+    if (chunk_size == 1 && cnorm) {  // normalising after every token is the exact recurrence
+        if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
+        return launch_scan_simt<false>(a, d, dec, false, st);
+    }
+    if (chunk_size == 1 || dec || lin1 || cnorm) {  // the tensor-core kernels: Eq. 17, per-token normaliser, similarity objective
         if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
         return chunk_size == 1 ? launch_scan_simt<false>(a, d, dec, false, st)
                                : launch_scan_simt<true>(a, d, dec, lin1, st);

@@ -31,6 +31,7 @@ struct ScanArgs {
     float* S_out;
     float* y;
     int B, T, H, m, chunk;
+    int cnorm;  // chunked CUDA-core path: no per-token normaliser, unit slots after each chunk
 };
 
 // Per-token staged record: x[D] | q[m] | c[m] | mu | eta, padded to a multiple
@@ -238,7 +239,16 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
                 const float qv = valid ? rec[D + slot[r]] : 0.f;
                 if constexpr (CHUNKED && LIN1) {
                     float alpha_s, alpha_0, gamma;
-                    update_coefs_lin1<true>(n0sq[r], p[r], xx, cv, mu, eta, n0[r], alpha_s, alpha_0, gamma);
+                    if (a.cnorm) {  // no per-token normaliser: the bare write (beta = 1)
+                        const bool ok = n0sq[r] > 0.f;
+                        const float ac = ok ? __fdiv_rn(eta * cv, n0[r]) : 0.f;   // eta c / n
+                        const float rr = ok ? __fdiv_rn(p[r], n0sq[r]) : 0.f;     // p / n^2
+                        alpha_s = mu;
+                        alpha_0 = -ac * rr;
+                        gamma = ac;
+                    } else {
+                        update_coefs_lin1<true>(n0sq[r], p[r], xx, cv, mu, eta, n0[r], alpha_s, alpha_0, gamma);
+                    }
                     if (!valid) { alpha_s = 0.f; alpha_0 = 0.f; gamma = 0.f; }
 #pragma unroll
                     for (int k = 0; k < EPL; ++k) {
@@ -247,13 +257,37 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
                     }
                 } else {
                     float alpha, gamma;
-                    update_coefs<CHUNKED || DEC>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
-                                                 CHUNKED ? n0[r] : 1.f, alpha, gamma);
+                    if (CHUNKED && a.cnorm) {  // no per-token normaliser: the bare write (beta = 1)
+                        const bool ok = n0sq[r] > 0.f;
+                        const float ac = ok ? __fdiv_rn(eta * cv, n0[r]) : 0.f;   // eta c / n
+                        const float rr = ok ? __fdiv_rn(p[r], n0sq[r]) : 0.f;     // p / n^2
+                        alpha = ok ? fmaf(-ac, rr, mu) : 1.f;
+                        gamma = ac;
+                    } else {
+                        update_coefs<CHUNKED || DEC>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
+                                                     CHUNKED ? n0[r] : 1.f, alpha, gamma);
+                    }
                     if (!valid) { alpha = 0.f; gamma = 0.f; }
 #pragma unroll
                     for (int k = 0; k < EPL; ++k) {
                         s[r][k] = fmaf(alpha, s[r][k], gamma * xv[k]);
                         yp[k] = fmaf(qv, s[r][k], yp[k]);
+                    }
+                }
+            }
+            if constexpr (CHUNKED) {  // normalisation at chunk boundaries: after the chunk's last read-out
+                if (a.cnorm && ((t + 1) % a.chunk == 0 || t + 1 == T)) {
+#pragma unroll
+                    for (int r = 0; r < RQ; ++r) {
+                        float nn = 0.f;
+#pragma unroll
+                        for (int k = 0; k < EPL; ++k) nn = fmaf(s[r][k], s[r][k], nn);
+                        nn = octet_sum(nn);
+                        if (nn > 0.f) {
+                            const float nr = __fsqrt_rn(nn);
+#pragma unroll
+                            for (int k = 0; k < EPL; ++k) s[r][k] = __fdiv_rn(s[r][k], nr);
+                        }
                     }
                 }
             }

@@ -70,6 +70,8 @@ def test_argument_checks_return_before_launch(lib):
                                                     v(5 << 20), v(6 << 20), v(7 << 20), 1, 4, 1, 64, 64, 64,
                                                     0, form, impl, None)
     assert ex(5, 0) == L.ERR_INVALID_ARG        # unknown chunk form
+    assert ex(4, 0) == L.ERR_INVALID_ARG
+    assert ex(2, 3) == L.ERR_UNSUPPORTED        # normalisation at chunk boundaries: CUDA-core kernel
     assert ex(1, 2) == L.ERR_UNSUPPORTED        # linearisation 1 runs on the CUDA-core kernel
     assert _scan(lib, mode=1, impl=2) == L.ERR_UNSUPPORTED  # DEC runs on the CUDA-core kernels
     assert _scan(lib, mode=1, chunk=64, impl=3) == L.ERR_UNSUPPORTED

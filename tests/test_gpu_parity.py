@@ -33,18 +33,18 @@ def L():
     return L
 
 
-def run_gpu(L, inp, chunk, impl="auto", eta=None, mode="sim", lin=2):
+def run_gpu(L, inp, chunk, impl="auto", eta=None, mode="sim", lin=2, norm="token"):
     t = dev_inputs(inp)
     y, S = L.scan_fwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], eta=t["eta"] if eta is None else eta,
-                      chunk=chunk, impl=impl, mode=mode, lin=lin)
+                      chunk=chunk, impl=impl, mode=mode, lin=lin, norm=norm)
     torch.cuda.synchronize()
     L.device_status()
     return y.cpu().numpy(), S.cpu().numpy()
 
 
-def run_oracle(inp, chunk, mode="sim", lin=2):
+def run_oracle(inp, chunk, mode="sim", lin=2, norm="token"):
     y, S, _ = oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], eta=inp["eta"],
-                          chunk=chunk, mode=mode, lin=lin)
+                          chunk=chunk, mode=mode, lin=lin, norm=norm)
     return y, S
 
 
@@ -515,3 +515,29 @@ def test_lin1_full_size_sampled(L, name, pairs):
     hs = [p[1] for p in pairs]
     assert y_err(yg[bs, :, hs][:, :, None], yo) <= TOL_TC
     assert s_err(Sg[bs, hs][:, None], So) <= TOL_TC
+
+
+# --------------------------------- normalisation at chunk boundaries (ablation)
+
+@pytest.mark.parametrize("lin", [1, 2])
+@pytest.mark.parametrize("m,d,C", [(16, 32, 4), (64, 64, 16), (128, 128, 64), (48, 16, 8)])
+def test_chunk_norm(L, lin, m, d, C):
+    """No per-token normaliser inside a chunk, unit slots after each chunk (Appendix C
+    ablation), either linearisation, vs the oracle; ragged tail included."""
+    w = LI.Workload("t", B=2, T=2 * C + C // 2 + 3, H=2, m=m, d=d, seed=700 + m + d + C + lin)
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, C, lin=lin, norm="chunk")
+    yo, So = run_oracle(inp, C, lin=lin, norm="chunk")
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
+
+
+def test_chunk_norm_chunk_one_is_exact_and_tensor_cores_refuse(L):
+    w = LI.Workload("t", B=1, T=40, H=2, m=64, d=64, seed=710)
+    inp = LI.make_inputs(w)
+    y1, S1 = run_gpu(L, inp, 1, norm="chunk")
+    ye, Se = run_oracle(inp, 1)
+    assert y_err(y1, ye) <= TOL_F32 and s_err(S1, Se) <= TOL_F32
+    for impl in ("tcgen05", "tcgen05_split"):
+        with pytest.raises(L.LatticeError):
+            run_gpu(L, inp, 64, impl=impl, norm="chunk")

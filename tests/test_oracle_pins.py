@@ -570,3 +570,23 @@ def test_chunk_norm_carried_state_is_on_the_sphere_and_differs_from_per_token():
     yt, St, _ = oracle.scan(x, c, q, mu, S0, chunk=8)
     np.testing.assert_allclose(np.linalg.norm(Sc, axis=-1), 1.0, atol=1e-12)
     assert np.abs(yc - yt).max() > 1e-6
+
+
+@pytest.mark.parametrize("lin", [1, 2])
+def test_chunk_norm_zero_write_decays_inside_the_chunk_and_returns_at_the_boundary(lin):
+    """With c = 0 nothing is written: inside a chunk the slots are only scaled by the
+    running product of mu (no normaliser, beta = 1), each read-out sees that decayed
+    state, and the projection after the chunk brings unit slots back to where they
+    started. The read-out of a chunk's last token sees the state before the
+    projection."""
+    rng = _rng(44 + lin)
+    C, B, T, H, m, d = 4, 1, 2 * 4 + 3, 2, 3, 5
+    x, c, q, mu, S0 = _rand_inputs(rng, B, T, H, m, d, unit=True)
+    c[:] = 0.0
+    y, S, _ = oracle.scan(x, c, q, mu, S0, chunk=C, lin=lin, norm="chunk")
+    for t in range(T):
+        t0 = (t // C) * C
+        decay = np.prod(mu[:, t0:t + 1, :], axis=1)                   # [B][H]
+        want = np.einsum("bhi,bhik->bhk", q[:, t], S0) * decay[..., None]
+        np.testing.assert_allclose(y[:, t], want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, S0, atol=1e-12)
