@@ -67,6 +67,8 @@ def _load():
                                                  ctypes.c_double, _D, _D, _D,
                                                  ctypes.POINTER(ll)]
         lib.oracle_chunk_token_gates.restype = None
+        lib.oracle_scan_bwd.argtypes = [i, i, i, i, i, i, i] + [_D] * 14 + [i]
+        lib.oracle_scan_bwd.restype = None
         _lib = lib
     return _lib
 
@@ -130,6 +132,31 @@ def scan(x, c, q, mu, S0, eta=None, chunk: int = 1, form: str = "token",
     else:
         raise ValueError(form)
     return y, S, int(deg)
+
+
+def scan_bwd(x, c, q, mu, S0, dy, dS_T=None, eta=None, chunk: int = 1,
+             nthreads: Optional[int] = None, form: Optional[str] = None):
+    """Gradients of L = sum_t dy_t . y_t + dS_T . S_T through the similarity-objective
+    scan (the exact recurrence for chunk == 1, Eq. 17 with the chunk size otherwise;
+    form="chunked" forces the chunked definition at chunk 1). Returns a dict with
+    dx, dc, dq, dmu, deta (None when eta is None) and dS0, in the inputs' layouts."""
+    x, c, q, mu, S0, dy = map(_f64, (x, c, q, mu, S0, dy))
+    eta = None if eta is None else _f64(eta)
+    dS_T = None if dS_T is None else _f64(dS_T)
+    B, T, H, d = x.shape
+    m = c.shape[-1]
+    assert c.shape == (B, T, H, m) and q.shape == (B, T, H, m) and mu.shape == (B, T, H)
+    assert S0.shape == (B, H, m, d) and dy.shape == (B, T, H, d)
+    if form is None:
+        form = "exact" if chunk == 1 else "chunked"
+    out = {"dx": np.zeros_like(x), "dc": np.zeros_like(c), "dq": np.zeros_like(q),
+           "dmu": np.zeros_like(mu), "deta": None if eta is None else np.zeros_like(eta),
+           "dS0": np.zeros_like(S0)}
+    _load().oracle_scan_bwd({"exact": 0, "chunked": 1}[form], B, T, H, m, d, chunk,
+                            _p(x), _p(c), _p(q), _p(mu), _p(eta), _p(S0), _p(dy), _p(dS_T),
+                            _p(out["dx"]), _p(out["dc"]), _p(out["dq"]), _p(out["dmu"]),
+                            _p(out["deta"]), _p(out["dS0"]), _threads(nthreads))
+    return out
 
 
 def step(S, x, c, q, mu, eta=None, nthreads: Optional[int] = None, mode: str = "sim"):

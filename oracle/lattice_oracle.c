@@ -27,6 +27,9 @@
  *   - Appendix D (Implementation): argument shapes and the read-out y = q S_t
  *     with the updated state.
  *
+ *   - backward pass (oracle_scan_bwd): the paper prints none; the adjoint of the
+ *     similarity-objective forward above, exact and Eq. 17, derived step by step
+ *     and pinned by finite differences of the forward.
  *   - §3.1.1 eq. (decoding_stateNorm_loss) and eq. (decoding_recurrence): the
  *     reconstruction objective writes the part of the reconstruction error
  *     e = phi(S) c - x orthogonal to each slot (h_t = e_t in eq. OSR).
@@ -512,4 +515,281 @@ void oracle_readout(int B, int H, int m, int d, const double *S, const double *q
         for (int i = 0; i < m; ++i)
             for (int k = 0; k < d; ++k) yb[k] += qb[i] * Sb[(size_t)i * d + k];
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass: the adjoint of the forward definitions above.              */
+/* ------------------------------------------------------------------------ */
+/* The paper prints no backward formulas (its training differentiates the JAX
+ * forward automatically, Appendix D). These are the reverse-mode derivatives of
+ * the similarity-objective forward above, taken step by step in the order the
+ * forward computes its intermediates, for the scalar loss
+ *     L = sum_t dy_t . y_t + dS_T . S_T.
+ * Every function below is pinned by central finite differences of the forward
+ * drivers above (tests/test_oracle_pins.py). */
+
+/* Adjoint of one exact slot update (§3.1.1 eq. OSR, §3.2, §3.3, Eq. 14):
+ *   n2 = s.s, p = s.x, n = sqrt(n2), r = p/n2, a = eta c/n,
+ *   x_perp = x - r s, w = mu s + a x_perp, s' = w/|w|.
+ * gb = dL/ds' in, sb = dL/ds out; dL/dx, dL/dmu, dL/deta are added to xb, *mub,
+ * *etab and dL/dc is stored in *cb. A degenerate update (n2 = 0 or w = 0) kept the
+ * slot, so it passes gb through. tmp holds 3d doubles. */
+static void exact_slot_bwd(int d, const double *s, const double *x, double c, double mu,
+                           double eta, const double *gb, double *sb, double *xb, double *cb,
+                           double *mub, double *etab, double *tmp)
+{
+    double *w = tmp, *xp = tmp + d, *wb = tmp + 2 * d;
+    double n2 = 0.0, p = 0.0;
+    for (int k = 0; k < d; ++k) { n2 += s[k] * s[k]; p += s[k] * x[k]; }
+    *cb = 0.0;
+    if (n2 == 0.0) { for (int k = 0; k < d; ++k) sb[k] = gb[k]; return; }
+    double n = sqrt(n2), r = p / n2, a = eta * c / n, nw2 = 0.0;
+    for (int k = 0; k < d; ++k) {
+        xp[k] = x[k] - r * s[k];
+        w[k] = mu * s[k] + a * xp[k];
+        nw2 += w[k] * w[k];
+    }
+    if (nw2 == 0.0) { for (int k = 0; k < d; ++k) sb[k] = gb[k]; return; }
+    double nw = sqrt(nw2);
+    /* s' = w/|w|:  wb = (gb - s'(s'.gb)) / |w| */
+    double sg = 0.0;
+    for (int k = 0; k < d; ++k) sg += (w[k] / nw) * gb[k];
+    for (int k = 0; k < d; ++k) wb[k] = (gb[k] - (w[k] / nw) * sg) / nw;
+    /* w = mu s + a x_perp */
+    double ab = 0.0, rb = 0.0;
+    for (int k = 0; k < d; ++k) {
+        *mub += s[k] * wb[k];
+        ab += xp[k] * wb[k];
+        sb[k] = mu * wb[k];
+    }
+    /* x_perp = x - r s, with xpb = a wb */
+    for (int k = 0; k < d; ++k) {
+        double xpb = a * wb[k];
+        xb[k] += xpb;
+        sb[k] += -r * xpb;
+        rb += -s[k] * xpb;
+    }
+    /* r = p/n2, a = eta c/n, n = sqrt(n2) */
+    double pb = rb / n2;
+    double n2b = -rb * p / (n2 * n2);
+    if (etab) *etab += ab * c / n;
+    *cb = ab * eta / n;
+    double nb = -ab * eta * c / n2;
+    n2b += nb / (2.0 * n);
+    /* p = s.x, n2 = s.s */
+    for (int k = 0; k < d; ++k) {
+        sb[k] += pb * x[k] + 2.0 * n2b * s[k];
+        xb[k] += pb * s[k];
+    }
+}
+
+/* Adjoint of the gates of one slot against its chunk-start state (Eq. 17, eq.
+ * beta_chunk; the definitions of oracle_chunk_token_gates2 with nobeta = 0):
+ *   h = -x, hh = |h|^2, hdot = h.s0, hhat = hdot/n2, khat = c/sqrt(n2),
+ *   tt = khat^2 hh - n2 hhat^2 khat^2, dsq = eta^2 max(tt, 0),
+ *   den = mu^2 n2 + dsq, beta = sqrt(n2)/sqrt(den),
+ *   g = beta (mu + eta hhat khat), kt = -beta eta khat.
+ * gateb = dL/dg and ktb = dL/dkt in; dL/dx and dL/ds0 are added to xb and s0b,
+ * dL/dmu and dL/deta to *mub and *etab, dL/dc is stored in *cb. A degenerate token
+ * (den = 0) had constant gates. */
+static void chunk_gate_slot_bwd(int d, const double *s0, const double *x, double c, double mu,
+                                double eta, double gateb, double ktb, double *xb, double *s0b,
+                                double *cb, double *mub, double *etab)
+{
+    double n2 = 0.0, hh = 0.0, hdot = 0.0;
+    for (int k = 0; k < d; ++k) {
+        n2 += s0[k] * s0[k];
+        hh += x[k] * x[k];
+        hdot += (-x[k]) * s0[k];
+    }
+    double hhat = hdot / n2, khat = c / sqrt(n2);
+    double tt = khat * khat * hh - n2 * hhat * hhat * khat * khat;
+    double dsq = eta * eta * (tt > 0.0 ? tt : 0.0);
+    double den = mu * mu * n2 + dsq;
+    *cb = 0.0;
+    if (den == 0.0) return;
+    double beta = sqrt(n2) / sqrt(den);
+    /* g = beta (mu + eta hhat khat), kt = -beta eta khat */
+    double betab = gateb * (mu + eta * hhat * khat) + ktb * (-eta * khat);
+    double mub_ = gateb * beta;
+    double etab_ = gateb * beta * hhat * khat + ktb * (-beta * khat);
+    double hhatb = gateb * beta * eta * khat;
+    double khatb = gateb * beta * eta * hhat + ktb * (-beta * eta);
+    /* beta = sqrt(n2) den^(-1/2) */
+    double n2b = betab * beta / (2.0 * n2);
+    double denb = -0.5 * betab * beta / den;
+    /* den = mu^2 n2 + dsq */
+    mub_ += denb * 2.0 * mu * n2;
+    n2b += denb * mu * mu;
+    double dsqb = denb;
+    /* dsq = eta^2 max(tt, 0) */
+    etab_ += dsqb * 2.0 * eta * (tt > 0.0 ? tt : 0.0);
+    double ttb = tt > 0.0 ? dsqb * eta * eta : 0.0;
+    /* tt = khat^2 hh - n2 hhat^2 khat^2 */
+    khatb += ttb * (2.0 * khat * hh - 2.0 * n2 * hhat * hhat * khat);
+    double hhb = ttb * khat * khat;
+    n2b += -ttb * hhat * hhat * khat * khat;
+    hhatb += -ttb * 2.0 * n2 * hhat * khat * khat;
+    /* khat = c n2^(-1/2), hhat = hdot/n2 */
+    *cb = khatb / sqrt(n2);
+    n2b += -khatb * 0.5 * c / (n2 * sqrt(n2));
+    double hdotb = hhatb / n2;
+    n2b += -hhatb * hdot / (n2 * n2);
+    /* hdot = -x.s0, hh = x.x, n2 = s0.s0 */
+    for (int k = 0; k < d; ++k) {
+        xb[k] += -hdotb * s0[k] + 2.0 * hhb * x[k];
+        s0b[k] += -hdotb * x[k] + 2.0 * n2b * s0[k];
+    }
+    *mub += mub_;
+    if (etab) *etab += etab_;
+}
+
+typedef struct {
+    int B, T, H, m, d, C, form; /* form 0: exact; 1: chunked (Eq. 17), chunk C */
+    const double *x, *c, *q, *mu, *eta, *S0, *dy, *dST;
+    double *dx, *dc, *dq, *dmu, *deta, *dS0;
+    int next;
+    pthread_mutex_t lock;
+} bwd_job_t;
+
+/* One (b,h) sequence: the forward keeps every state S_t (t = -1 .. T-1), then
+ * the adjoint runs backwards through the tokens. */
+static void bwd_sequence(bwd_job_t *J, int b, int h, double *St, double *gb, double *s0b,
+                         double *sb, double *g, double *kt, double *tmp)
+{
+    const int T = J->T, H = J->H, m = J->m, d = J->d, C = J->C;
+    const size_t md = (size_t)m * d;
+    const size_t so = ((size_t)b * H + h) * md;
+    long long deg = 0;
+    double *n2 = tmp + 3 * d; /* m doubles */
+    memcpy(St, J->S0 + so, sizeof(double) * md);
+    for (int t = 0; t < T; ++t) { /* forward, keeping the states */
+        size_t tok = IDX_TOK(b, t, h, T, H);
+        double eta = J->eta ? J->eta[tok] : 1.0;
+        double *S = St + (size_t)(t + 1) * md;
+        memcpy(S, St + (size_t)t * md, sizeof(double) * md);
+        if (J->form == 0) {
+            exact_token(m, d, S, J->x + tok * d, J->c + tok * m, J->q + tok * m, J->mu[tok], eta,
+                        NULL, tmp, &deg);
+        } else {
+            const double *S0c = St + (size_t)((t / C) * C) * md; /* chunk-start state */
+            for (int i = 0; i < m; ++i) {
+                double a = 0.0;
+                for (int k = 0; k < d; ++k) a += S0c[(size_t)i * d + k] * S0c[(size_t)i * d + k];
+                n2[i] = a;
+            }
+            oracle_chunk_token_gates2(m, d, S0c, n2, J->x + tok * d, J->c + tok * m, J->mu[tok], eta,
+                                      g, kt, NULL, &deg, NULL, NULL, 0);
+            for (int i = 0; i < m; ++i)
+                for (int k = 0; k < d; ++k)
+                    S[(size_t)i * d + k] = g[i] * S[(size_t)i * d + k] + kt[i] * (-J->x[tok * d + k]);
+        }
+    }
+    /* adjoint; gb = dL/dS_t */
+    for (size_t e = 0; e < md; ++e) gb[e] = J->dST ? J->dST[so + e] : 0.0;
+    memset(s0b, 0, sizeof(double) * md);
+    for (int t = T - 1; t >= 0; --t) {
+        size_t tok = IDX_TOK(b, t, h, T, H);
+        const double *x = J->x + tok * d, *c = J->c + tok * m, *q = J->q + tok * m;
+        const double *dy = J->dy + tok * d;
+        const double mu = J->mu[tok], eta = J->eta ? J->eta[tok] : 1.0;
+        const double *Sprev = St + (size_t)t * md, *Scur = St + (size_t)(t + 1) * md;
+        double *xb = J->dx + tok * d, *cb = J->dc + tok * m, *qb = J->dq + tok * m;
+        double mub = 0.0, etab = 0.0;
+        for (int k = 0; k < d; ++k) xb[k] = 0.0;
+        /* read-out y_t = sum_i q_i s_t,i (Appendix D) */
+        for (int i = 0; i < m; ++i) {
+            double v = 0.0;
+            for (int k = 0; k < d; ++k) {
+                v += dy[k] * Scur[(size_t)i * d + k];
+                gb[(size_t)i * d + k] += q[i] * dy[k];
+            }
+            qb[i] = v;
+        }
+        if (J->form == 0) {
+            for (int i = 0; i < m; ++i) {
+                exact_slot_bwd(d, Sprev + (size_t)i * d, x, c[i], mu, eta, gb + (size_t)i * d, sb,
+                               xb, cb + i, &mub, J->eta ? &etab : NULL, tmp);
+                memcpy(gb + (size_t)i * d, sb, sizeof(double) * d);
+            }
+        } else {
+            const int t0 = (t / C) * C;
+            const double *S0c = St + (size_t)t0 * md;
+            for (int i = 0; i < m; ++i) {
+                double a = 0.0;
+                for (int k = 0; k < d; ++k) a += S0c[(size_t)i * d + k] * S0c[(size_t)i * d + k];
+                n2[i] = a;
+            }
+            oracle_chunk_token_gates2(m, d, S0c, n2, x, c, mu, eta, g, kt, NULL, &deg, NULL, NULL, 0);
+            for (int i = 0; i < m; ++i) {
+                /* s_t = g s_{t-1} + kt h, h = -x */
+                double *gbi = gb + (size_t)i * d;
+                const double *sp = Sprev + (size_t)i * d;
+                double gateb = 0.0, ktb = 0.0;
+                for (int k = 0; k < d; ++k) {
+                    gateb += sp[k] * gbi[k];
+                    ktb += (-x[k]) * gbi[k];
+                    xb[k] += -kt[i] * gbi[k];
+                    gbi[k] *= g[i];
+                }
+                chunk_gate_slot_bwd(d, S0c + (size_t)i * d, x, c[i], mu, eta, gateb, ktb, xb,
+                                    s0b + (size_t)i * d, cb + i, &mub, J->eta ? &etab : NULL);
+            }
+            if (t == t0) { /* the chunk-start state is also the running state S_{t0-1} */
+                for (size_t e = 0; e < md; ++e) { gb[e] += s0b[e]; s0b[e] = 0.0; }
+            }
+        }
+        J->dmu[tok] = mub;
+        if (J->deta) J->deta[tok] = etab;
+    }
+    memcpy(J->dS0 + so, gb, sizeof(double) * md);
+}
+
+static void *bwd_worker(void *arg)
+{
+    bwd_job_t *J = (bwd_job_t *)arg;
+    const size_t md = (size_t)J->m * J->d;
+    double *St = malloc(sizeof(double) * md * (size_t)(J->T + 1));
+    double *gb = malloc(sizeof(double) * md), *s0b = malloc(sizeof(double) * md);
+    double *sb = malloc(sizeof(double) * (size_t)J->d);
+    double *g = malloc(sizeof(double) * (size_t)J->m), *kt = malloc(sizeof(double) * (size_t)J->m);
+    double *tmp = malloc(sizeof(double) * (size_t)(3 * J->d + J->m));
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int item = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (item >= J->B * J->H) break;
+        bwd_sequence(J, item / J->H, item % J->H, St, gb, s0b, sb, g, kt, tmp);
+    }
+    free(St); free(gb); free(s0b); free(sb); free(g); free(kt); free(tmp);
+    return NULL;
+}
+
+/* Gradients of L = sum_t dy_t . y_t + dST . S_T (dST may be NULL: zero) with
+ * respect to every input of the similarity-objective scan: form 0, the exact
+ * recurrence; form 1, the chunked recurrence of Eq. 17 with chunk size C.
+ * Outputs have the layouts of the inputs; deta may be NULL (and is not written
+ * when eta is NULL, i.e. eta = 1). */
+void oracle_scan_bwd(int form, int B, int T, int H, int m, int d, int C, const double *x,
+                     const double *c, const double *q, const double *mu, const double *eta,
+                     const double *S0, const double *dy, const double *dST, double *dx,
+                     double *dc, double *dq, double *dmu, double *deta, double *dS0, int nthreads)
+{
+    bwd_job_t J;
+    memset(&J, 0, sizeof(J));
+    J.B = B; J.T = T; J.H = H; J.m = m; J.d = d; J.C = C > 0 ? C : 1; J.form = form;
+    J.x = x; J.c = c; J.q = q; J.mu = mu; J.eta = eta; J.S0 = S0; J.dy = dy; J.dST = dST;
+    J.dx = dx; J.dc = dc; J.dq = dq; J.dmu = dmu; J.deta = eta ? deta : NULL; J.dS0 = dS0;
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > B * H) nthreads = B * H;
+    if (nthreads <= 1) {
+        bwd_worker(&J);
+    } else {
+        pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+        for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, bwd_worker, &J);
+        for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+        free(th);
+    }
+    pthread_mutex_destroy(&J.lock);
 }

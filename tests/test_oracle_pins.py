@@ -590,3 +590,74 @@ def test_chunk_norm_zero_write_decays_inside_the_chunk_and_returns_at_the_bounda
         want = np.einsum("bhi,bhik->bhk", q[:, t], S0) * decay[..., None]
         np.testing.assert_allclose(y[:, t], want, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(S, S0, atol=1e-12)
+
+
+# --------------------------------------------------------------- backward pass ---
+
+def _loss_and_grads(args, dy, dST, chunk):
+    def loss(**kw):
+        y, S, _ = oracle.scan(kw["x"], kw["c"], kw["q"], kw["mu"], kw["S0"], eta=kw["eta"], chunk=chunk)
+        return (dy * y).sum() + (0.0 if dST is None else (dST * S).sum())
+    g = oracle.scan_bwd(args["x"], args["c"], args["q"], args["mu"], args["S0"], dy, dST,
+                        eta=args["eta"], chunk=chunk)
+    return loss, g
+
+
+@pytest.mark.parametrize("chunk", [1, 4])
+@pytest.mark.parametrize("with_eta,with_dST", [(True, True), (False, False)])
+def test_backward_equals_central_differences(chunk, with_eta, with_dST):
+    """The paper prints no backward pass; its adjoint is fixed by the forward. Every
+    gradient entry of L = sum dy.y + dS_T.S_T equals the central difference of the
+    (separately pinned) forward, for the exact recurrence and for Eq. 17 with a
+    ragged last chunk (T = 9, C = 4)."""
+    rng = _rng(50 + chunk + 2 * with_eta)
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 9, 1, 3, 5, unit=False)
+    eta = rng.uniform(0.5, 1.5, mu.shape) if with_eta else None
+    dy = rng.standard_normal(x.shape)
+    dST = rng.standard_normal(S0.shape) if with_dST else None
+    args = dict(x=x, c=c, q=q, mu=mu, eta=eta, S0=S0)
+    loss, g = _loss_and_grads(args, dy, dST, chunk)
+    assert (g["deta"] is None) == (eta is None)
+    h = 1e-6
+    for name, a in args.items():
+        if a is None:
+            continue
+        num = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            ap, am = a.copy(), a.copy()
+            ap[idx] += h
+            am[idx] -= h
+            num[idx] = (loss(**{**args, name: ap}) - loss(**{**args, name: am})) / (2 * h)
+        np.testing.assert_allclose(g["d" + name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_backward_chunk_one_matches_exact_except_the_radial_state_gradient():
+    """At chunk size 1 with unit slots the two forwards agree (§3.4.1), so every
+    gradient agrees too, except the component of dS0 along each slot: the exact
+    recurrence projects onto the unit sphere, Eq. 17 keeps the chunk-start norm."""
+    rng = _rng(52)
+    x, c, q, mu, S0 = _rand_inputs(rng, 2, 7, 2, 3, 5, unit=True)
+    dy = rng.standard_normal(x.shape)
+    dST = rng.standard_normal(S0.shape)
+    a = oracle.scan_bwd(x, c, q, mu, S0, dy, dST, chunk=1)
+    b = oracle.scan_bwd(x, c, q, mu, S0, dy, dST, chunk=1, form="chunked")
+    for k in ("dx", "dc", "dq", "dmu"):
+        np.testing.assert_allclose(a[k], b[k], atol=1e-12, err_msg=k)
+    r = a["dS0"] - b["dS0"]
+    tangential = r - (r * S0).sum(-1, keepdims=True) * S0
+    np.testing.assert_allclose(tangential, 0.0, atol=1e-12)
+    assert np.abs((r * S0).sum(-1)).max() > 1e-3
+
+
+def test_backward_of_a_single_token_readout():
+    """T = 1: dL/dq_i = dy . s_1,i with s_1 the returned final state (Appendix D
+    read-out), and with dy = 0 only dS_T drives the gradients."""
+    rng = _rng(53)
+    x, c, q, mu, S0 = _rand_inputs(rng, 1, 1, 2, 4, 6, unit=True)
+    dy = rng.standard_normal(x.shape)
+    y, S, _ = oracle.scan(x, c, q, mu, S0, chunk=1)
+    g = oracle.scan_bwd(x, c, q, mu, S0, dy, None, chunk=1)
+    np.testing.assert_allclose(g["dq"][:, 0], np.einsum("bhd,bhid->bhi", dy[:, 0], S), atol=1e-13)
+    g0 = oracle.scan_bwd(x, c, q, mu, S0, np.zeros_like(dy), None, chunk=1)
+    for k in ("dx", "dc", "dq", "dmu", "dS0"):
+        assert not np.any(g0[k])
