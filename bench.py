@@ -206,6 +206,33 @@ def time_scan(torch, L, t, chunk, steps, warmup, flush=None, impl="auto", mode="
     return [e0.elapsed_time(e1) for e0, e1 in ev]
 
 
+def time_bwd(torch, L, t, chunk, steps, warmup, flush=None):
+    """Per-step device time (ms) of lattice_scan_bwd (unit cotangents), CUDA events
+    on its stream; the workspace is allocated once, outside the timed region."""
+    stream = torch.cuda.current_stream()
+    B, T, H, d = t["x"].shape
+    m = t["c"].shape[-1]
+    dy = torch.ones((B, T, H, d), dtype=torch.float32, device=t["x"].device)
+    ws = torch.empty(max(L.scan_bwd_workspace_bytes(B, T, H, m, d, chunk), 16), dtype=torch.uint8,
+                     device=t["x"].device)
+    run = lambda: L.scan_bwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], dy, chunk=chunk,
+                             workspace=ws, stream=stream)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for e0, e1 in ev:
+        if flush is not None:
+            flush.add_(1)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    L.device_status()
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+
 def time_scan_e2e(torch, L, inp, chunk, steps, warmup, device):
     """End to end through the public call with host buffers, as a streaming user runs
     it: each step copies its inputs in from pinned host memory, runs the scan and
@@ -477,6 +504,13 @@ def main():
             extra[f"{w.name}_lin1_chunked"] = {"ms": statistics.mean(tl),
                                                "tokens_per_s": w.B * w.T / (statistics.mean(tl) * 1e-3),
                                                "kernel": "scan_simt_kernel<chunked, recurrence_linear1>"}
+            # backward pass (CUDA-core kernel), chunked and exact
+            for cb, tag in ((w.chunk, "chunked"), (1, "exact")):
+                tb = time_bwd(torch, L, t, cb, 3, 2, flush=flush)
+                extra[f"{w.name}_bwd_{tag}"] = {"ms": statistics.mean(tb),
+                                                "tokens_per_s": w.B * w.T / (statistics.mean(tb) * 1e-3),
+                                                "kernel": f"scan_bwd_kernel<{tag}>",
+                                                "allocations": "outputs per call; workspace once"}
             del t
             for name in [n for n in ("mid_layer", "long_ctx") if n != w.name]:
                 wn = LI.WORKLOADS[name]

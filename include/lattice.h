@@ -165,6 +165,39 @@ lattice_status lattice_scan_fwd_ex(const void *x, lattice_dtype x_dtype, const f
                                    lattice_mode mode, lattice_chunk_form form, lattice_impl impl,
                                    void *stream);
 
+/* Backward pass of the similarity-objective scan (exact recurrence for
+ * chunk_size 1, Eq. 17 otherwise). The paper prints no backward formulas; this is
+ * the reverse-mode derivative of the forward of lattice_scan_fwd with
+ * LATTICE_SIM and LATTICE_CHUNK_LIN2, for the scalar loss
+ *     L = sum_t dy_t . y_t + dS_T . S_T.
+ * Inputs as for lattice_scan_fwd (same layouts and dtypes), plus
+ *   dy [B][T][H][d] fp32 (required when T > 0) and dS_T [B][H][m][d] fp32 or NULL (0).
+ * Outputs (fp32, device, the inputs' layouts, written in full): dx, dc, dq, dmu,
+ *   deta (may be NULL; not written when eta is NULL, i.e. eta = 1) and dS0.
+ * States are rebuilt by recomputation from checkpoints every seg_tokens tokens
+ * (0 selects the default: the smallest multiple of chunk_size that is >= 64; any
+ * other value must be a positive multiple of chunk_size, else
+ * LATTICE_ERR_INVALID_ARG). workspace is caller-owned device memory of at least
+ * lattice_scan_bwd_workspace_bytes(...) bytes, 16-byte aligned; the call
+ * overwrites it and keeps no pointer after it returns (the kernel runs on
+ * `stream`). Outputs must not overlap inputs, each other or the workspace
+ * (LATTICE_ERR_INVALID_ARG). CUDA-core kernel only; m <= 128 (larger m:
+ * LATTICE_ERR_UNSUPPORTED). */
+lattice_status lattice_scan_bwd(const void *x, lattice_dtype x_dtype, const float *c,
+                                const void *q, lattice_dtype q_dtype, const float *mu,
+                                const float *eta, const float *S0, const float *dy,
+                                const float *dS_T, float *dx, float *dc, float *dq, float *dmu,
+                                float *deta, float *dS0, void *workspace, size_t workspace_bytes,
+                                int B, int T, int H, int m, int d, int chunk_size, int seg_tokens,
+                                void *stream);
+
+/* Workspace bytes lattice_scan_bwd needs for this shape: B*H*(n_seg - 1 +
+ * seg_tokens)*m*d*4 with n_seg = ceil(T/seg_tokens) (seg_tokens as resolved by
+ * lattice_scan_bwd). Returns 0 for arguments lattice_scan_bwd would reject. Host
+ * function; launches nothing. */
+size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int chunk_size,
+                                        int seg_tokens);
+
 /* One decode step: the exact recurrence for one new token per (b,h), state
  * updated in place (constant work per token, §1-§2 of the paper).
  *   S [B][H][m][d] in/out, x [B][H][d], c [B][H][m], q [B][H][m],

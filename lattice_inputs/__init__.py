@@ -30,7 +30,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "bf16_round_bits", "bf16_bits_to_f32", "make_inputs",
-    "make_decode_state", "make_decode_steps", "sample_heads",
+    "make_decode_state", "make_decode_steps", "sample_heads", "make_cotangents",
 ]
 
 
@@ -187,3 +187,13 @@ def sample_heads(inp: dict, pairs) -> dict:
         inp["eta"][bs, :, hs][:, :, None])
     out.update(B=len(pairs), T=inp["T"], H=1, m=inp["m"], d=inp["d"])
     return out
+
+
+def make_cotangents(inp: dict, seed: int = 0, with_dS_T: bool = True) -> dict:
+    """Upstream gradients for a backward pass over make_inputs(...) = inp:
+    dy [B][T][H][d] ~ N(0, 1) and dS_T [B][H][m][d] ~ N(0, 1) (or None), fp32."""
+    B, T, H, m, d = inp["B"], inp["T"], inp["H"], inp["m"], inp["d"]
+    rng = np.random.default_rng([seed, 3])
+    dy = rng.standard_normal((B, T, H, d), dtype=np.float32)
+    dS_T = rng.standard_normal((B, H, m, d), dtype=np.float32) if with_dS_T else None
+    return dict(dy=dy, dS_T=dS_T)

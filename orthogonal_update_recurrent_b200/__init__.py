@@ -22,8 +22,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["LatticeError", "lib", "scan_fwd", "step", "readout", "chunk_impl", "device_status",
-           "LIB_PATH"]
+__all__ = ["LatticeError", "lib", "scan_fwd", "scan_bwd", "scan_bwd_workspace_bytes", "step",
+           "readout", "chunk_impl", "device_status", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblattice.so")
 
@@ -58,6 +58,10 @@ def lib() -> ctypes.CDLL:
                                             i, i, i, vp]
         L.lattice_scan_fwd_ex.argtypes = [vp, i, fp, vp, i, fp, fp, fp, fp, fp, i, i, i, i, i,
                                           i, i, i, i, vp]
+        L.lattice_scan_bwd.argtypes = [vp, i, fp, vp, i, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp,
+                                       fp, vp, ctypes.c_size_t, i, i, i, i, i, i, i, vp]
+        L.lattice_scan_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.lattice_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.lattice_step.argtypes = [fp, vp, i, fp, vp, i, fp, fp, fp, i, i, i, i, i, vp]
         L.lattice_readout.argtypes = [fp, vp, i, fp, i, i, i, i, vp]
         L.lattice_get_device_status.argtypes = [vp]
@@ -67,7 +71,8 @@ def lib() -> ctypes.CDLL:
         L.lattice_chunk_impl.argtypes = [i, i, i, i, i, i, i]
         L.lattice_last_cuda_error.argtypes = []
         L.lattice_last_cuda_error.restype = ctypes.c_char_p
-        for f in ("lattice_scan_fwd", "lattice_scan_fwd_impl", "lattice_scan_fwd_ex", "lattice_step", "lattice_readout",
+        for f in ("lattice_scan_fwd", "lattice_scan_fwd_impl", "lattice_scan_fwd_ex", "lattice_scan_bwd",
+                  "lattice_step", "lattice_readout",
                   "lattice_get_device_status", "lattice_version", "lattice_chunk_impl"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -143,6 +148,53 @@ def scan_fwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor
                                  _IMPL[impl], _stream(stream))
     _raise(code, "lattice_scan_fwd")
     return y, S_out
+
+
+def scan_bwd_workspace_bytes(B: int, T: int, H: int, m: int, d: int, chunk: int = 1,
+                             seg: int = 0) -> int:
+    """Device workspace bytes scan_bwd needs (0: the shape is not supported)."""
+    return int(lib().lattice_scan_bwd_workspace_bytes(B, T, H, m, d, int(chunk), int(seg)))
+
+
+def scan_bwd(x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor,
+             S0: torch.Tensor, dy: torch.Tensor, dS_T: Optional[torch.Tensor] = None,
+             eta: Optional[torch.Tensor] = None, chunk: int = 1, seg: int = 0,
+             workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Backward pass of scan_fwd (similarity objective; exact for chunk 1, Eq. 17
+    otherwise): gradients of L = sum_t dy_t . y_t + dS_T . S_T. Returns a dict with
+    dx, dc, dq, dmu, deta (None when eta is None) and dS0, all float32. seg: tokens
+    between state checkpoints (0: default). workspace: optional uint8 device tensor of
+    at least scan_bwd_workspace_bytes(...) bytes; allocated when None."""
+    B, T, H, d = x.shape
+    m = c.shape[-1]
+    _chk(x, "x", (B, T, H, d), _XQ)
+    _chk(c, "c", (B, T, H, m))
+    _chk(q, "q", (B, T, H, m), _XQ)
+    _chk(mu, "mu", (B, T, H))
+    _chk(S0, "S0", (B, H, m, d))
+    _chk(dy, "dy", (B, T, H, d))
+    if dS_T is not None:
+        _chk(dS_T, "dS_T", (B, H, m, d))
+    if eta is not None:
+        _chk(eta, "eta", (B, T, H))
+    L = lib()
+    need = L.lattice_scan_bwd_workspace_bytes(B, T, H, m, d, int(chunk), int(seg))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous CUDA tensor")
+    f32 = dict(dtype=torch.float32, device=x.device)
+    out = {"dx": torch.empty((B, T, H, d), **f32), "dc": torch.empty((B, T, H, m), **f32),
+           "dq": torch.empty((B, T, H, m), **f32), "dmu": torch.empty((B, T, H), **f32),
+           "deta": None if eta is None else torch.empty((B, T, H), **f32),
+           "dS0": torch.empty((B, H, m, d), **f32)}
+    code = L.lattice_scan_bwd(_ptr(x), _dt(x), _ptr(c), _ptr(q), _dt(q), _ptr(mu), _ptr(eta),
+                              _ptr(S0), _ptr(dy), _ptr(dS_T), _ptr(out["dx"]), _ptr(out["dc"]),
+                              _ptr(out["dq"]), _ptr(out["dmu"]), _ptr(out["deta"]), _ptr(out["dS0"]),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              B, T, H, m, d, int(chunk), int(seg), _stream(stream))
+    _raise(code, "lattice_scan_bwd")
+    return out
 
 
 def step(S: torch.Tensor, x: torch.Tensor, c: torch.Tensor, q: torch.Tensor, mu: torch.Tensor,

@@ -10,6 +10,7 @@
 #include "step.cuh"
 #include "chunk_tc.cuh"
 #include "chunk_split.cuh"
+#include "scan_bwd.cuh"
 
 using namespace lattice;
 
@@ -131,6 +132,42 @@ lattice_status launch_readout_d(const ReadoutArgs& a, cudaStream_t st) {
         default: readout_kernel<D, 4><<<grid, block, 0, st>>>(a); break;
     }
     return launch_status();
+}
+
+// ---- backward
+constexpr int kBwdMaxM = 128;
+
+int bwd_seg(int chunk, int seg) {
+    if (seg == 0) return chunk >= 64 ? chunk : chunk * ((64 + chunk - 1) / chunk);
+    return (seg > 0 && seg % chunk == 0) ? seg : -1;
+}
+
+template <int D, int RQ, bool CH>
+lattice_status launch_bwd_t(const BwdArgs& a, int nw, cudaStream_t st) {
+    const size_t smem = bwd_smem_bytes(D, a.m, nw);
+    auto k = scan_bwd_kernel<D, RQ, CH>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    k<<<a.B * a.H, nw * 32, smem, st>>>(a);
+    return launch_status();
+}
+
+template <int D, bool CH>
+lattice_status launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
+    const int quads = (a.m + 3) / 4;
+    if (quads <= 16) return launch_bwd_t<D, 1, CH>(a, quads < 4 ? 4 : quads, st);
+    return launch_bwd_t<D, 2, CH>(a, 16, st);
+}
+
+template <bool CH>
+lattice_status launch_bwd(const BwdArgs& a, int d, cudaStream_t st) {
+    switch (d) {
+        case 16: return launch_bwd_d<16, CH>(a, st);
+        case 32: return launch_bwd_d<32, CH>(a, st);
+        case 64: return launch_bwd_d<64, CH>(a, st);
+        case 128: return launch_bwd_d<128, CH>(a, st);
+    }
+    return LATTICE_ERR_UNSUPPORTED;
 }
 
 lattice_status check_dims(int B, int H, int m, int d) {
@@ -307,6 +344,62 @@ lattice_status lattice_readout(const float* S, const void* q, lattice_dtype q_dt
         case 64: return launch_readout_d<64>(a, st);
         default: return launch_readout_d<128>(a, st);
     }
+}
+
+size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int chunk_size,
+                                        int seg_tokens) {
+    if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return 0;
+    if (check_dims(B, H, m, d) != LATTICE_OK || m > kBwdMaxM) return 0;
+    const int seg = bwd_seg(chunk_size, seg_tokens);
+    if (seg < 1) return 0;
+    return (size_t)B * H * bwd_ws_floats_per_seq(T, m, d, seg) * sizeof(float);
+}
+
+lattice_status lattice_scan_bwd(const void* x, lattice_dtype x_dtype, const float* c,
+                                const void* q, lattice_dtype q_dtype, const float* mu,
+                                const float* eta, const float* S0, const float* dy,
+                                const float* dS_T, float* dx, float* dc, float* dq, float* dmu,
+                                float* deta, float* dS0, void* workspace, size_t workspace_bytes,
+                                int B, int T, int H, int m, int d, int chunk_size, int seg_tokens,
+                                void* stream) {
+    if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return LATTICE_ERR_INVALID_ARG;
+    if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
+    lattice_status ds = check_dims(B, H, m, d);
+    if (ds != LATTICE_OK) return ds;
+    if (m > kBwdMaxM) return LATTICE_ERR_UNSUPPORTED;
+    const int seg = bwd_seg(chunk_size, seg_tokens);
+    if (seg < 1) return LATTICE_ERR_INVALID_ARG;
+    const size_t need = lattice_scan_bwd_workspace_bytes(B, T, H, m, d, chunk_size, seg_tokens);
+    if (!S0 || !dS0 || !workspace || workspace_bytes < need) return LATTICE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !c || !q || !mu || !dy || !dx || !dc || !dq || !dmu))
+        return LATTICE_ERR_INVALID_ARG;
+    if (!aligned(S0, 16) || !aligned(dS0, 16) || !aligned(workspace, 16) || (dS_T && !aligned(dS_T, 16)))
+        return LATTICE_ERR_INVALID_ARG;
+    const size_t ntok = (size_t)B * T * H, nS = (size_t)B * H * m * d * 4;
+    if (T > 0 && (!aligned(x, dsize(x_dtype)) || !aligned(c, 4) || !aligned(mu, 4) || !aligned(q, dsize(q_dtype)) ||
+                  !aligned(dy, 4) || !aligned(dx, 4) || !aligned(dc, 4) || !aligned(dq, 4) ||
+                  !aligned(dmu, 4) || (eta && !aligned(eta, 4)) || (deta && !aligned(deta, 4))))
+        return LATTICE_ERR_INVALID_ARG;
+    float* deta_w = eta ? deta : nullptr;
+    const size_t tb = T > 0 ? 1 : 0;  // token-indexed buffers are empty when T == 0
+    const Span ins[] = {span(x, tb * ntok * d * dsize(x_dtype)), span(c, tb * ntok * m * 4),
+                        span(q, tb * ntok * m * dsize(q_dtype)), span(mu, tb * ntok * 4),
+                        span(eta, eta ? tb * ntok * 4 : 0), span(S0, nS),
+                        span(dy, tb * ntok * d * 4), span(dS_T, dS_T ? nS : 0)};
+    const Span outs[] = {span(dx, tb * ntok * d * 4), span(dc, tb * ntok * m * 4),
+                         span(dq, tb * ntok * m * 4), span(dmu, tb * ntok * 4),
+                         span(deta_w, deta_w ? tb * ntok * 4 : 0), span(dS0, nS),
+                         span(workspace, need)};
+    for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+        for (const Span& s : ins)
+            if (overlap(outs[i], s)) return LATTICE_ERR_INVALID_ARG;
+        for (size_t k = i + 1; k < sizeof(outs) / sizeof(outs[0]); ++k)
+            if (overlap(outs[i], outs[k])) return LATTICE_ERR_INVALID_ARG;
+    }
+    BwdArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, dy, dS_T,
+              dx, dc, dq, dmu, deta_w, dS0, static_cast<float*>(workspace), B, T, H, m, chunk_size, seg};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return chunk_size == 1 ? launch_bwd<false>(a, d, st) : launch_bwd<true>(a, d, st);
 }
 
 lattice_status lattice_get_device_status(void* stream) {

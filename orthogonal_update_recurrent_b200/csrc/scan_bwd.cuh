@@ -1,0 +1,445 @@
+// scan_bwd.cuh -- CUDA-core backward pass of the Lattice scan (similarity
+// objective), exact recurrence or chunked form (Eq. 17).
+//
+// "Lattice: Learning to Efficiently Compress the Memory" prints no backward
+// formulas; this kernel evaluates the reverse-mode derivative of the forward that
+// scan_simt.cuh computes, for L = sum_t dy_t . y_t + dS_T . S_T:
+//   per slot and token  n2 = |z|^2, p = z.x, xx = |x|^2 (z = the running slot for
+//   the exact recurrence, the chunk-start slot for Eq. 17), a = eta c/n,
+//   r = p/n2, u = mu - a r, w2 = mu^2 n2 + a^2 (xx - p r), iw = target/sqrt(w2)
+//   (target 1, or n for Eq. 17's normaliser), s_t = (u iw) s_{t-1} + (a iw) x,
+//   y_t = sum_i q_i s_t,i.
+// The adjoint walks the tokens backwards, carrying dL/ds_t in registers.
+//
+// One CTA per (b, h) sequence, slots in registers in the octet layout
+// (common.cuh). States are rebuilt by recomputation, so memory stays O(T/L):
+//   1. a forward sweep stores the state at the start of every segment of L
+//      tokens (L a multiple of the chunk size) in the workspace;
+//   2. for each segment, last to first: recompute its states from the
+//      checkpoint into the segment tape (workspace, L2-resident), then run the
+//      adjoint over the segment's tokens in reverse, reading the tape.
+// Per-token gradients that sum over slots (dx, dmu, deta) are reduced within
+// the warp by shuffles and across warps through shared memory in a fixed order,
+// so results are bit-reproducible.
+#pragma once
+#include "common.cuh"
+
+namespace lattice {
+
+constexpr int kBwdTB = 8;  // tokens per staged block
+
+struct BwdArgs {
+    const void* x; bool x_bf16;
+    const float* c;
+    const void* q; bool q_bf16;
+    const float* mu;
+    const float* eta;  // may be null (=> 1)
+    const float* S0;
+    const float* dy;
+    const float* dST;  // may be null (=> 0)
+    float* dx; float* dc; float* dq; float* dmu;
+    float* deta;       // may be null
+    float* dS0;
+    float* ws;         // workspace: per (b,h) (nseg - 1) checkpoints then the L-token tape
+    int B, T, H, m, chunk, seg;
+};
+
+// Staged record per token: x[D] | dy[D] | q[m] | c[m] | mu | eta, padded so that
+// every record (and its dy) starts 16-byte aligned.
+__host__ __device__ inline int bwd_record_floats(int D, int m) { return (2 * D + 2 * m + 2 + 3) & ~3; }
+
+__host__ __device__ inline size_t bwd_smem_bytes(int D, int m, int nw) {
+    return sizeof(float) * ((size_t)kBwdTB * bwd_record_floats(D, m) + (size_t)kBwdTB * nw * D +
+                            (size_t)kBwdTB * nw * 2);
+}
+
+// Floats of workspace per (b,h) sequence.
+__host__ __device__ inline size_t bwd_ws_floats_per_seq(int T, int m, int D, int seg) {
+    const int nseg = T > 0 ? (T + seg - 1) / seg : 1;
+    return (size_t)(nseg - 1 + seg) * m * D;
+}
+
+// Forward coefficients of one slot and token, with the intermediates the adjoint needs.
+struct SlotFwd {
+    bool ok;
+    float n2, inv_n, r, a, praw, perp2, w2, iw, u, alpha, gamma;
+};
+
+__device__ __forceinline__ SlotFwd slot_fwd(float n2, float p, float xx, float c, float mu, float eta,
+                                            bool chunked) {
+    SlotFwd f;
+    f.ok = n2 > 0.f;
+    f.n2 = f.ok ? n2 : 1.f;
+    f.inv_n = __frsqrt_rn(f.n2);
+    f.r = __fdiv_rn(p, f.n2);
+    f.a = eta * c * f.inv_n;
+    f.praw = fmaf(-p, f.r, xx);
+    f.perp2 = fmaxf(f.praw, 0.f);
+    f.w2 = fmaf(f.a * f.a, f.perp2, mu * mu * f.n2);
+    f.ok = f.ok && f.w2 > 0.f;
+    const float target = chunked ? f.n2 * f.inv_n : 1.f;
+    f.iw = __frsqrt_rn(f.ok ? f.w2 : 1.f) * target;
+    f.u = fmaf(-f.a, f.r, mu);
+    f.alpha = f.ok ? f.u * f.iw : 1.f;
+    f.gamma = f.ok ? f.a * f.iw : 0.f;
+    return f;
+}
+
+// Adjoint of slot_fwd: from dL/dalpha and dL/dgamma to dL/dp, dL/dn2, dL/dxx,
+// dL/dmu, dL/deta, dL/dc. A degenerate slot (ok false) had constant coefficients.
+struct SlotBwd {
+    float pb, n2b, xxb, mub, etab, cb;
+};
+
+__device__ __forceinline__ SlotBwd slot_bwd(const SlotFwd& f, float p, float c, float mu, float eta,
+                                            float alphab, float gammab, bool chunked) {
+    SlotBwd g{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (!f.ok) return g;
+    const float ub = alphab * f.iw;                       // alpha = u iw
+    const float iwb = fmaf(alphab, f.u, gammab * f.a);    // gamma = a iw
+    float ab = fmaf(gammab, f.iw, -ub * f.r);
+    float rb = -ub * f.a;                                 // u = mu - a r
+    g.mub = ub;
+    const float w2b = -0.5f * iwb * __fdiv_rn(f.iw, f.w2);  // iw = target w2^(-1/2)
+    g.mub = fmaf(w2b, 2.f * mu * f.n2, g.mub);            // w2 = mu^2 n2 + a^2 perp2
+    g.n2b = w2b * mu * mu;
+    ab = fmaf(w2b, 2.f * f.a * f.perp2, ab);
+    const float perp2b = f.praw > 0.f ? w2b * f.a * f.a : 0.f;
+    g.xxb = perp2b;                                       // perp2 = xx - p r
+    g.pb = -perp2b * f.r;
+    rb = fmaf(-perp2b, p, rb);
+    const float inv_n2 = f.inv_n * f.inv_n;
+    g.pb = fmaf(rb, inv_n2, g.pb);                        // r = p / n2
+    g.n2b = fmaf(-rb * f.r, inv_n2, g.n2b);
+    g.etab = ab * c * f.inv_n;                            // a = eta c / n
+    g.cb = ab * eta * f.inv_n;
+    float nb = -ab * f.a * f.inv_n;
+    if (chunked) nb = fmaf(iwb * f.iw, f.inv_n, nb);      // target = n
+    g.n2b = fmaf(nb, 0.5f * f.inv_n, g.n2b);              // n = sqrt(n2)
+    return g;
+}
+
+// Sum a per-lane D-vector partial over the 4 octets of the warp and store the
+// warp's total to dst[D] (each lane stores EPL/4 of its octet positions).
+template <int D>
+__device__ __forceinline__ void warp_octets_sum_store(const float* v, float* dst, int lane) {
+    using O = Octet<D>;
+    constexpr int EPL = O::EPL;
+    const int j = lane & 7;
+    const int hi = (lane >> 4) & 1, mid = (lane >> 3) & 1;
+    if constexpr (EPL >= 4) {
+        float v1[EPL / 2];
+#pragma unroll
+        for (int k = 0; k < EPL / 2; ++k) {
+            const float send = hi ? v[k] : v[k + EPL / 2];
+            const float keep = hi ? v[k + EPL / 2] : v[k];
+            v1[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        }
+        float v2[EPL / 4];
+#pragma unroll
+        for (int k = 0; k < EPL / 4; ++k) {
+            const float send = mid ? v1[k] : v1[k + EPL / 4];
+            const float keep = mid ? v1[k + EPL / 4] : v1[k];
+            v2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+        const int kbase = hi * (EPL / 2) + mid * (EPL / 4);
+#pragma unroll
+        for (int k = 0; k < EPL / 4; ++k) dst[O::pos(j, kbase + k)] = v2[k];
+    } else {  // EPL == 2
+        const float send = hi ? v[0] : v[1];
+        const float keep = hi ? v[1] : v[0];
+        float t = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        t += __shfl_xor_sync(0xffffffffu, t, 8);
+        if (!mid) dst[O::pos(j, hi)] = t;
+    }
+}
+
+template <int D, int RQ, bool CHUNKED>
+__global__ void __launch_bounds__(512) scan_bwd_kernel(BwdArgs a) {
+    using O = Octet<D>;
+    constexpr int EPL = O::EPL;
+    extern __shared__ __align__(16) float smem[];
+    const int NW = blockDim.x >> 5, NT = blockDim.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int j = lane & 7, oct = lane >> 3;
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+    const int m = a.m, T = a.T, H = a.H, L = a.seg;
+    const int R = bwd_record_floats(D, m);
+    float* rec_buf = smem;                            // [TB][R]
+    float* dx_buf = smem + kBwdTB * R;                // [TB][NW][D]
+    float* sc_buf = dx_buf + (size_t)kBwdTB * NW * D;  // [TB][NW][2]: dmu, deta partials
+    const int nseg = T > 0 ? (T + L - 1) / L : 1;
+    float* ckpt = a.ws + bh * bwd_ws_floats_per_seq(T, m, D, L);  // [nseg-1][m][D]
+    float* tape = ckpt + (size_t)(nseg - 1) * m * D;                // [L][m][D]
+
+    int slot[RQ];
+    bool valid[RQ];
+#pragma unroll
+    for (int r = 0; r < RQ; ++r) {
+        slot[r] = 4 * (warp + NW * r) + oct;
+        valid[r] = slot[r] < m;
+    }
+    auto load_state = [&](const float* base, float (*v)[EPL]) {
+#pragma unroll
+        for (int r = 0; r < RQ; ++r) {
+            if (valid[r]) load_row_f32<D>(base + (size_t)slot[r] * D, j, v[r]);
+            else {
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) v[r][k] = 0.f;
+            }
+        }
+    };
+    auto store_state = [&](float* base, const float (*v)[EPL]) {
+#pragma unroll
+        for (int r = 0; r < RQ; ++r)
+            if (valid[r]) store_row_f32<D, false>(base + (size_t)slot[r] * D, j, v[r]);
+    };
+    // Stage tokens [t0, t0 + n) into rec_buf (synchronous; callers barrier around it).
+    auto stage = [&](int t0, int n, bool need_qdy) {
+        for (int idx = tid; idx < n * R; idx += NT) {
+            const int tok = idx / R, e = idx - tok * R;
+            const size_t bth = ((size_t)b * T + t0 + tok) * H + h;
+            float v = 0.f;
+            if (e < D) v = load_elem(a.x, a.x_bf16, bth * D + e);
+            else if (e < 2 * D) { if (need_qdy) v = a.dy[bth * D + (e - D)]; }
+            else if (e < 2 * D + m) { if (need_qdy) v = load_elem(a.q, a.q_bf16, bth * m + (e - 2 * D)); }
+            else if (e < 2 * D + 2 * m) v = a.c[bth * m + (e - 2 * D - m)];
+            else if (e == 2 * D + 2 * m) v = a.mu[bth];
+            else if (e == 2 * D + 2 * m + 1) v = a.eta ? a.eta[bth] : 1.f;
+            rec_buf[idx] = v;
+        }
+    };
+
+    float s[RQ][EPL], s0[CHUNKED ? RQ : 1][EPL];
+    float n0sq[RQ];
+    // Forward over tokens [t_begin, t_end) from the state in s. tape_base != null:
+    // store the state before each token at tape_base[t - t_begin]. ckpts: store the
+    // state before each segment start t (t % L == 0, 0 < t < t_end) as a checkpoint.
+    auto forward = [&](int t_begin, int t_end, float* tape_base, bool ckpts) {
+        for (int t0 = t_begin; t0 < t_end; t0 += kBwdTB) {
+            const int n = min(kBwdTB, t_end - t0);
+            __syncthreads();
+            stage(t0, n, false);
+            __syncthreads();
+            for (int tok = 0; tok < n; ++tok) {
+                const int t = t0 + tok;
+                const float* rec = rec_buf + tok * R;
+                if (ckpts && t > 0 && t % L == 0) store_state(ckpt + (size_t)(t / L - 1) * m * D, s);
+                if (tape_base) store_state(tape_base + (size_t)(t - t_begin) * m * D, s);
+                if constexpr (CHUNKED) {
+                    if (t % a.chunk == 0) {
+#pragma unroll
+                        for (int r = 0; r < RQ; ++r) {
+                            float nn = 0.f;
+#pragma unroll
+                            for (int k = 0; k < EPL; ++k) { s0[r][k] = s[r][k]; nn = fmaf(s[r][k], s[r][k], nn); }
+                            n0sq[r] = octet_sum(nn);
+                        }
+                    }
+                }
+                float xv[EPL];
+                load_row_f32<D>(rec, j, xv);
+                const float mu = rec[2 * D + 2 * m], eta = rec[2 * D + 2 * m + 1];
+                float xx = 0.f, p[RQ], n2[RQ];
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) xx = fmaf(xv[k], xv[k], xx);
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    float pp = 0.f, nn = 0.f;
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) {
+                        if constexpr (CHUNKED) pp = fmaf(s0[r][k], xv[k], pp);
+                        else { pp = fmaf(s[r][k], xv[k], pp); nn = fmaf(s[r][k], s[r][k], nn); }
+                    }
+                    p[r] = pp;
+                    n2[r] = nn;
+                }
+                xx = octet_sum(xx);
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    p[r] = octet_sum(p[r]);
+                    if constexpr (!CHUNKED) n2[r] = octet_sum(n2[r]);
+                }
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    const float cv = valid[r] ? rec[2 * D + m + slot[r]] : 0.f;
+                    SlotFwd f = slot_fwd(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta, CHUNKED);
+                    const float al = valid[r] ? f.alpha : 0.f, ga = valid[r] ? f.gamma : 0.f;
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) s[r][k] = fmaf(al, s[r][k], ga * xv[k]);
+                }
+            }
+        }
+    };
+
+    // ---- 1. checkpoints at every segment start (the last segment needs none beyond)
+    load_state(a.S0 + (size_t)bh * m * D, s);
+    if (nseg > 1) {
+        forward(0, (nseg - 1) * L, nullptr, true);
+        store_state(ckpt + (size_t)(nseg - 2) * m * D, s);  // the last segment's start
+    }
+
+    // ---- 2. segments, last to first
+    float gb[RQ][EPL];  // dL/ds_t
+    if (a.dST) load_state(a.dST + (size_t)bh * m * D, gb);
+    else {
+#pragma unroll
+        for (int r = 0; r < RQ; ++r)
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) gb[r][k] = 0.f;
+    }
+    float acc[CHUNKED ? RQ : 1][EPL];  // chunked: sum over the chunk's tokens of dL/dp x
+    float n2acc[RQ];                   // chunked: sum of dL/dn2
+#pragma unroll
+    for (int r = 0; r < RQ; ++r) {
+        n2acc[r] = 0.f;
+        if constexpr (CHUNKED) {
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) acc[r][k] = 0.f;
+        }
+    }
+    for (int seg = nseg - 1; seg >= 0; --seg) {
+        const int ts = seg * L, te = min(T, ts + L);
+        // 2a. rebuild the segment's states into the tape
+        __syncthreads();
+        if (seg == 0) load_state(a.S0 + (size_t)bh * m * D, s);
+        else load_state(ckpt + (size_t)(seg - 1) * m * D, s);
+        forward(ts, te, tape, false);
+        // 2b. adjoint over the segment's tokens, last to first
+        for (int tb_end = te; tb_end > ts; tb_end -= kBwdTB) {
+            const int t0 = max(ts, tb_end - kBwdTB), n = tb_end - t0;
+            __syncthreads();
+            stage(t0, n, true);
+            __syncthreads();
+            for (int tok = n - 1; tok >= 0; --tok) {
+                const int t = t0 + tok;
+                const float* rec = rec_buf + tok * R;
+                const size_t bth = ((size_t)b * T + t) * H + h;
+                float sp[RQ][EPL];
+                load_state(tape + (size_t)(t - ts) * m * D, sp);  // s_{t-1}
+                if constexpr (CHUNKED) {
+                    if (t == te - 1 || (t + 1) % a.chunk == 0) {  // entering a chunk from its end
+                        const int tc = (t / a.chunk) * a.chunk;
+                        load_state(tape + (size_t)(tc - ts) * m * D, s0);
+#pragma unroll
+                        for (int r = 0; r < RQ; ++r) {
+                            float nn = 0.f;
+#pragma unroll
+                            for (int k = 0; k < EPL; ++k) nn = fmaf(s0[r][k], s0[r][k], nn);
+                            n0sq[r] = octet_sum(nn);
+                        }
+                    }
+                }
+                float xv[EPL], yb[EPL];
+                load_row_f32<D>(rec, j, xv);
+                load_row_f32<D>(rec + D, j, yb);
+                const float mu = rec[2 * D + 2 * m], eta = rec[2 * D + 2 * m + 1];
+                // lane-local dot products, then one batch of octet reductions
+                float xx = 0.f, xy = 0.f;
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) { xx = fmaf(xv[k], xv[k], xx); xy = fmaf(xv[k], yb[k], xy); }
+                float p[RQ], n2[RQ], spy[RQ], spg[RQ], xg[RQ];
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    float pp = 0.f, nn = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) {
+                        if constexpr (CHUNKED) pp = fmaf(s0[r][k], xv[k], pp);
+                        else { pp = fmaf(sp[r][k], xv[k], pp); nn = fmaf(sp[r][k], sp[r][k], nn); }
+                        a1 = fmaf(sp[r][k], yb[k], a1);
+                        a2 = fmaf(sp[r][k], gb[r][k], a2);
+                        a3 = fmaf(xv[k], gb[r][k], a3);
+                    }
+                    p[r] = pp; n2[r] = nn; spy[r] = a1; spg[r] = a2; xg[r] = a3;
+                }
+                xx = octet_sum(xx);
+                xy = octet_sum(xy);
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    p[r] = octet_sum(p[r]);
+                    if constexpr (!CHUNKED) n2[r] = octet_sum(n2[r]);
+                    spy[r] = octet_sum(spy[r]);
+                    spg[r] = octet_sum(spg[r]);
+                    xg[r] = octet_sum(xg[r]);
+                }
+                float dxp[EPL];
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) dxp[k] = 0.f;
+                float mub = 0.f, etab = 0.f;
+#pragma unroll
+                for (int r = 0; r < RQ; ++r) {
+                    const float cv = valid[r] ? rec[2 * D + m + slot[r]] : 0.f;
+                    const float qv = valid[r] ? rec[2 * D + slot[r]] : 0.f;
+                    const SlotFwd f = slot_fwd(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta, CHUNKED);
+                    // read-out y_t = sum_i q_i s_t,i, s_t = alpha s_{t-1} + gamma x
+                    const float qb = fmaf(f.alpha, spy[r], f.gamma * xy);
+                    // dL/ds_t including the read-out: g = gb + q dy
+                    const float alphab = fmaf(qv, spy[r], spg[r]);  // s_{t-1} . g
+                    const float gammab = fmaf(qv, xy, xg[r]);       // x . g
+                    SlotBwd d = slot_bwd(f, p[r], cv, mu, eta, alphab, gammab, CHUNKED);
+                    if (!valid[r]) d = SlotBwd{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const float al = valid[r] ? f.alpha : 0.f, ga = valid[r] ? f.gamma : 0.f;
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) {
+                        const float g = fmaf(qv, yb[k], gb[r][k]);
+                        const float z = CHUNKED ? s0[r][k] : sp[r][k];
+                        dxp[k] = fmaf(ga, g, fmaf(d.pb, z, fmaf(2.f * d.xxb, xv[k], dxp[k])));
+                        float ng = al * g;
+                        if constexpr (!CHUNKED) ng = fmaf(d.pb, xv[k], fmaf(2.f * d.n2b, sp[r][k], ng));
+                        else acc[r][k] = fmaf(d.pb, xv[k], acc[r][k]);
+                        gb[r][k] = ng;
+                    }
+                    if constexpr (CHUNKED) n2acc[r] += d.n2b;
+                    mub += d.mub;
+                    etab += d.etab;
+                    if (valid[r] && j == 0) {
+                        a.dq[bth * m + slot[r]] = qb;
+                        a.dc[bth * m + slot[r]] = d.cb;
+                    }
+                }
+                if constexpr (CHUNKED) {
+                    if (t % a.chunk == 0) {  // the chunk-start slot is also s_{t-1}
+#pragma unroll
+                        for (int r = 0; r < RQ; ++r) {
+#pragma unroll
+                            for (int k = 0; k < EPL; ++k) {
+                                gb[r][k] += fmaf(2.f * n2acc[r], s0[r][k], acc[r][k]);
+                                acc[r][k] = 0.f;
+                            }
+                            n2acc[r] = 0.f;
+                        }
+                    }
+                }
+                // per-warp partials of the slot sums
+                warp_octets_sum_store<D>(dxp, dx_buf + ((size_t)tok * NW + warp) * D, lane);
+                mub += __shfl_xor_sync(0xffffffffu, mub, 8);
+                mub += __shfl_xor_sync(0xffffffffu, mub, 16);
+                etab += __shfl_xor_sync(0xffffffffu, etab, 8);
+                etab += __shfl_xor_sync(0xffffffffu, etab, 16);
+                if (lane == 0) {
+                    sc_buf[((size_t)tok * NW + warp) * 2] = mub;
+                    sc_buf[((size_t)tok * NW + warp) * 2 + 1] = etab;
+                }
+            }
+            __syncthreads();
+            // fixed-order sums over the warps
+            for (int idx = tid; idx < n * D; idx += NT) {
+                const int tok = idx / D, k = idx - tok * D;
+                float v = 0.f;
+                for (int w = 0; w < NW; ++w) v += dx_buf[((size_t)tok * NW + w) * D + k];
+                a.dx[(((size_t)b * T + t0 + tok) * H + h) * D + k] = v;
+            }
+            for (int idx = tid; idx < n * 2; idx += NT) {
+                const int tok = idx >> 1, which = idx & 1;
+                float v = 0.f;
+                for (int w = 0; w < NW; ++w) v += sc_buf[((size_t)tok * NW + w) * 2 + which];
+                const size_t bth = ((size_t)b * T + t0 + tok) * H + h;
+                if (which == 0) a.dmu[bth] = v;
+                else if (a.deta) a.deta[bth] = v;
+            }
+        }
+    }
+    store_state(a.dS0 + (size_t)bh * m * D, gb);
+}
+
+}  // namespace lattice

@@ -28,7 +28,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("lattice_scan_fwd", "lattice_step", "lattice_readout", "lattice_get_device_status",
-              "lattice_status_string", "lattice_scan_fwd_impl", "lattice_version"):
+              "lattice_status_string", "lattice_scan_fwd_impl", "lattice_version", "lattice_scan_bwd",
+              "lattice_scan_bwd_workspace_bytes"):
         assert n in names
 
 
@@ -86,6 +87,43 @@ def test_argument_checks_return_before_launch(lib):
                             v(5 << 20), 1, 1, 4, 16, 0, None) == L.ERR_INVALID_ARG
     assert lib.lattice_readout(v(1 << 20), v(2 << 20), 0, v(3 << 20), 1, 1, 4, 24,
                                None) == L.ERR_UNSUPPORTED
+
+
+def _bwd(lib, **kw):
+    a = dict(x=1 << 20, xdt=0, c=2 << 20, q=3 << 20, qdt=0, mu=4 << 20, eta=None, S0=5 << 20,
+             dy=6 << 20, dST=None, dx=7 << 20, dc=8 << 20, dq=9 << 20, dmu=10 << 20, deta=None,
+             dS0=11 << 20, ws=12 << 20, wsb=1 << 20, B=1, T=4, H=1, m=4, d=16, chunk=1, seg=0)
+    a.update(kw)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return lib.lattice_scan_bwd(v(a["x"]), a["xdt"], v(a["c"]), v(a["q"]), a["qdt"], v(a["mu"]),
+                                v(a["eta"]), v(a["S0"]), v(a["dy"]), v(a["dST"]), v(a["dx"]),
+                                v(a["dc"]), v(a["dq"]), v(a["dmu"]), v(a["deta"]), v(a["dS0"]),
+                                v(a["ws"]), a["wsb"], a["B"], a["T"], a["H"], a["m"], a["d"],
+                                a["chunk"], a["seg"], None)
+
+
+def test_backward_workspace_and_argument_checks(lib):
+    # workspace: B*H*(n_seg - 1 + seg)*m*d*4 bytes; the default segment is the
+    # smallest multiple of the chunk size that is >= 64 tokens
+    ws = lib.lattice_scan_bwd_workspace_bytes
+    assert ws(1, 4, 1, 4, 16, 1, 0) == 64 * 4 * 16 * 4
+    assert ws(2, 200, 3, 4, 16, 1, 0) == 2 * 3 * (3 + 64) * 4 * 16 * 4
+    assert ws(1, 200, 1, 4, 16, 24, 0) == (2 + 72) * 4 * 16 * 4
+    assert ws(1, 200, 1, 4, 16, 128, 0) == (1 + 128) * 4 * 16 * 4
+    assert ws(1, 200, 1, 4, 16, 4, 10) == 0      # segment not a multiple of the chunk
+    assert ws(1, 200, 1, 129, 16, 1, 0) == 0     # m > 128
+    # every case below fails validation before any CUDA call
+    assert _bwd(lib, wsb=64 * 4 * 16 * 4 - 4) == L.ERR_INVALID_ARG   # workspace too small
+    assert _bwd(lib, ws=None) == L.ERR_INVALID_ARG
+    assert _bwd(lib, chunk=4, seg=10) == L.ERR_INVALID_ARG
+    assert _bwd(lib, m=129) == L.ERR_UNSUPPORTED
+    assert _bwd(lib, d=48) == L.ERR_UNSUPPORTED
+    assert _bwd(lib, dy=None) == L.ERR_INVALID_ARG
+    assert _bwd(lib, dS0=None) == L.ERR_INVALID_ARG
+    assert _bwd(lib, dx=(1 << 20) + 16) == L.ERR_INVALID_ARG    # dx overlaps x
+    assert _bwd(lib, dc=(7 << 20) + 4) == L.ERR_INVALID_ARG     # dc overlaps dx
+    assert _bwd(lib, ws=(11 << 20) + 64) == L.ERR_INVALID_ARG   # workspace overlaps dS0
+    assert _bwd(lib, ws=(12 << 20) + 8) == L.ERR_INVALID_ARG    # misaligned workspace
 
 
 def test_binding_rejects_host_tensors():

@@ -1,0 +1,173 @@
+"""Parity of the CUDA backward pass (through the C ABI) with the fp64 oracle's
+adjoint (oracle.scan_bwd, itself pinned by finite differences of the forward).
+
+The loss is L = sum_t dy_t . y_t + dS_T . S_T with seeded cotangents from
+lattice_inputs.make_cotangents. Every gradient (dx, dc, dq, dmu, deta, dS0) is
+compared element by element with the per-(b,h)-slice relative error of the
+forward tests. Tolerance: 1e-4 (fp32 arithmetic, exactly representable inputs)
+on sequences of up to a few hundred tokens; the full small training shape uses
+the chunked form's 2e-2 for the bf16-input chunked scan and 1e-3 for the exact
+recurrence, whose adjoint accumulates fp32 rounding over 2048 tokens.
+"""
+import numpy as np
+import pytest
+
+import lattice_inputs as LI
+import oracle
+from helpers import dev_inputs, rel_err_per_slice
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL_BWD = 1e-4
+SLICES = {"dx": (0, 2), "dc": (0, 2), "dq": (0, 2), "dmu": (0, 2), "deta": (0, 2), "dS0": (0, 1)}
+
+
+@pytest.fixture(scope="module")
+def L():
+    import orthogonal_update_recurrent_b200 as L
+    from orthogonal_update_recurrent_b200 import build
+    build.build()
+    return L
+
+
+def with_eta(inp, seed):
+    rng = np.random.default_rng([seed, 9])
+    out = dict(inp)
+    out["eta"] = rng.uniform(0.5, 1.5, inp["mu"].shape).astype(np.float32)
+    return out
+
+
+def run_gpu_bwd(L, inp, cot, chunk, seg=0):
+    t = dev_inputs(inp)
+    dy = torch.from_numpy(cot["dy"]).cuda()
+    dST = None if cot["dS_T"] is None else torch.from_numpy(cot["dS_T"]).cuda()
+    g = L.scan_bwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], dy, dST, eta=t["eta"], chunk=chunk, seg=seg)
+    torch.cuda.synchronize()
+    L.device_status()
+    return {k: (None if v is None else v.cpu().numpy()) for k, v in g.items()}
+
+
+def run_oracle_bwd(inp, cot, chunk):
+    return oracle.scan_bwd(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], cot["dy"],
+                           cot["dS_T"], eta=inp["eta"], chunk=chunk)
+
+
+def errors(gg, go):
+    out = {}
+    for k, ax in SLICES.items():
+        if go[k] is None:
+            assert gg[k] is None
+            continue
+        out[k] = rel_err_per_slice(gg[k], go[k], ax)
+    return out
+
+
+def check(gg, go, tol):
+    e = errors(gg, go)
+    bad = {k: v for k, v in e.items() if not v <= tol}
+    assert not bad, f"gradient errors above {tol}: {bad} (all: {e})"
+
+
+@pytest.mark.parametrize("m,d", [(16, 32), (5, 32), (64, 64), (128, 128), (64, 128), (48, 16)])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_bwd_exact_shapes(L, m, d, dt):
+    """Exact recurrence, three segments of 64 tokens (the last one ragged), eta given."""
+    w = LI.Workload("t", B=2, T=150, H=2, m=m, d=d, x_dtype=dt, q_dtype=dt, chunk=1, seed=800 + m + d)
+    inp = with_eta(LI.make_inputs(w), 800)
+    cot = LI.make_cotangents(inp, seed=800 + m)
+    check(run_gpu_bwd(L, inp, cot, 1), run_oracle_bwd(inp, cot, 1), TOL_BWD)
+
+
+@pytest.mark.parametrize("m,d,C", [(16, 32, 4), (64, 64, 16), (64, 64, 64), (128, 128, 64),
+                                   (48, 16, 8), (64, 128, 32)])
+def test_bwd_chunked_shapes(L, m, d, C):
+    """Eq. 17: several chunks and segments, a ragged last chunk, bf16 x/q."""
+    T = max(2 * C + C // 2 + 3, 150)
+    w = LI.Workload("t", B=2, T=T, H=2, m=m, d=d, seed=820 + m + d + C)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=820 + C)
+    check(run_gpu_bwd(L, inp, cot, C), run_oracle_bwd(inp, cot, C), TOL_BWD)
+
+
+def test_bwd_without_eta_and_final_state_gradient(L):
+    w = LI.Workload("t", B=1, T=70, H=3, m=32, d=64, seed=840)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=840, with_dS_T=False)
+    for C in (1, 16):
+        gg = run_gpu_bwd(L, inp, cot, C)
+        assert gg["deta"] is None
+        check(gg, run_oracle_bwd(inp, cot, C), TOL_BWD)
+
+
+@pytest.mark.parametrize("C", [1, 8])
+def test_bwd_segment_length_does_not_change_the_result(L, C):
+    """States are recomputed from checkpoints with the same arithmetic, so the
+    gradients are bit-identical for any segment length (one chunk per segment, the
+    default, and one segment holding the whole sequence)."""
+    w = LI.Workload("t", B=2, T=100, H=2, m=16, d=32, seed=850 + C)
+    inp = with_eta(LI.make_inputs(w), 850)
+    cot = LI.make_cotangents(inp, seed=850)
+    ref = run_gpu_bwd(L, inp, cot, C)
+    for seg in (C, 8 * C, 104 if C == 8 else 100):
+        g = run_gpu_bwd(L, inp, cot, C, seg=seg)
+        for k in ref:
+            assert (ref[k] is None) == (g[k] is None)
+            if ref[k] is not None:
+                assert np.array_equal(ref[k], g[k]), (seg, k)
+
+
+def test_bwd_is_deterministic(L):
+    w = LI.Workload("t", B=2, T=90, H=2, m=64, d=64, seed=860)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=860)
+    a = run_gpu_bwd(L, inp, cot, 16)
+    b = run_gpu_bwd(L, inp, cot, 16)
+    for k in a:
+        if a[k] is not None:
+            assert np.array_equal(a[k], b[k]), k
+
+
+def test_bwd_empty_sequence_passes_the_state_gradient_through(L):
+    w = LI.Workload("t", B=2, T=0, H=2, m=8, d=16, seed=870)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=870)
+    for C in (1, 4):
+        g = run_gpu_bwd(L, inp, cot, C)
+        assert np.array_equal(g["dS0"], cot["dS_T"])
+
+
+def test_bwd_rejects_unsupported_shapes(L):
+    w = LI.Workload("t", B=1, T=8, H=1, m=130, d=32, seed=880)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=880)
+    with pytest.raises(L.LatticeError):
+        run_gpu_bwd(L, inp, cot, 1)
+    w = LI.Workload("t", B=1, T=8, H=1, m=16, d=32, seed=881)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=881)
+    with pytest.raises(L.LatticeError):
+        run_gpu_bwd(L, inp, cot, 4, seg=6)  # segment not a multiple of the chunk
+
+
+@pytest.mark.parametrize("chunk,tol", [(64, 2e-2), (1, 1e-3)])
+def test_bwd_small_train_full_size_sampled(L, chunk, tol):
+    """The small training shape at full size (B=4, H=8, T=2048, m=d=64, bf16 x/q)
+    on the GPU; four sampled (b,h) sequences are checked against the oracle
+    (sequences are independent, so the sample is exact for them)."""
+    w = LI.WORKLOADS["small_train"]
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=890)
+    gg = run_gpu_bwd(L, inp, cot, chunk)
+    pairs = [(0, 0), (1, 5), (2, 3), (3, 7)]
+    sub = LI.sample_heads(inp, pairs)
+    bs, hs = [p[0] for p in pairs], [p[1] for p in pairs]
+    sub_cot = dict(dy=np.ascontiguousarray(cot["dy"][bs, :, hs][:, :, None, :]),
+                   dS_T=np.ascontiguousarray(cot["dS_T"][bs, hs][:, None]))
+    go = run_oracle_bwd(sub, sub_cot, chunk)
+    gsub = {"dx": gg["dx"][bs, :, hs][:, :, None, :], "dc": gg["dc"][bs, :, hs][:, :, None, :],
+            "dq": gg["dq"][bs, :, hs][:, :, None, :], "dmu": gg["dmu"][bs, :, hs][:, :, None],
+            "deta": None, "dS0": gg["dS0"][bs, hs][:, None]}
+    check(gsub, go, tol)
+    for k in ("dx", "dc", "dq", "dmu", "dS0"):
+        assert np.isfinite(gg[k]).all()
