@@ -198,6 +198,35 @@ lattice_status lattice_scan_bwd(const void *x, lattice_dtype x_dtype, const floa
 size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int chunk_size,
                                         int seg_tokens);
 
+/* Backward pass that allocates nothing, for callers that cannot call cudaMalloc:
+ * for example a plug-in running inside a host application that hands out every
+ * byte of device memory through its own pool, or a process that reserved the
+ * device's memory up front and may not ask the driver for more. The paper has no
+ * counterpart; this is a packaging of lattice_scan_bwd.
+ *
+ * Arguments, layouts, results and errors are those of lattice_scan_bwd without the
+ * workspace: the scratch it needs lives in one static device array of
+ * LATTICE_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits. A shape whose workspace
+ * (lattice_scan_bwd_workspace_bytes) exceeds that size returns
+ * LATTICE_ERR_UNSUPPORTED before any device work. The caller still allocates the
+ * inputs and outputs; the call itself makes no allocation.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * Every call shares the one array: calls that overlap on the GPU (on different
+ * streams, or from different host threads without ordering) race and corrupt each
+ * other's results, so order them. Nothing needs clearing between calls: the kernel
+ * writes every scratch word before it reads it. */
+#define LATTICE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+lattice_status lattice_scan_bwd_noalloc(const void *x, lattice_dtype x_dtype, const float *c,
+                                        const void *q, lattice_dtype q_dtype, const float *mu,
+                                        const float *eta, const float *S0, const float *dy,
+                                        const float *dS_T, float *dx, float *dc, float *dq,
+                                        float *dmu, float *deta, float *dS0, int B, int T, int H,
+                                        int m, int d, int chunk_size, int seg_tokens, void *stream);
+
 /* One decode step: the exact recurrence for one new token per (b,h), state
  * updated in place (constant work per token, §1-§2 of the paper).
  *   S [B][H][m][d] in/out, x [B][H][d], c [B][H][m], q [B][H][m],

@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "../../include/lattice.h"
 #include "common.cuh"
 #include "scan_simt.cuh"
@@ -417,3 +419,52 @@ lattice_status lattice_get_device_status(void* stream) {
 const char* lattice_last_cuda_error(void) { return g_last_error; }
 
 }  // extern "C"
+
+// ---- backward pass without allocation: scratch in a static device array
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = LATTICE_NOALLOC_SCRATCH_BYTES;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device. In host code the array's name is only a host-side stand-in.
+lattice_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return LATTICE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return LATTICE_OK;
+}
+
+}  // namespace
+
+extern "C" lattice_status lattice_scan_bwd_noalloc(
+    const void* x, lattice_dtype x_dtype, const float* c, const void* q, lattice_dtype q_dtype,
+    const float* mu, const float* eta, const float* S0, const float* dy, const float* dS_T,
+    float* dx, float* dc, float* dq, float* dmu, float* deta, float* dS0, int B, int T, int H,
+    int m, int d, int chunk_size, int seg_tokens, void* stream) {
+    const size_t need = lattice_scan_bwd_workspace_bytes(B, T, H, m, d, chunk_size, seg_tokens);
+    if (need == 0)  // a rejected shape: lattice_scan_bwd names the error before using the workspace
+        return lattice_scan_bwd(x, x_dtype, c, q, q_dtype, mu, eta, S0, dy, dS_T, dx, dc, dq, dmu,
+                                deta, dS0, nullptr, 0, B, T, H, m, d, chunk_size, seg_tokens, stream);
+    if (need > kNoAllocScratchBytes) return LATTICE_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    lattice_status s = noalloc_scratch(&scratch);
+    if (s != LATTICE_OK) return s;
+    return lattice_scan_bwd(x, x_dtype, c, q, q_dtype, mu, eta, S0, dy, dS_T, dx, dc, dq, dmu, deta,
+                            dS0, scratch, kNoAllocScratchBytes, B, T, H, m, d, chunk_size, seg_tokens,
+                            stream);
+}
