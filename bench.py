@@ -64,6 +64,15 @@ def scan_alg_bytes(w: LI.Workload, B=None, T=None, H=None) -> int:
     return B * T * H * per_tok + 2 * 4 * B * H * w.m * w.d
 
 
+def bwd_alg_bytes(w: LI.Workload) -> int:
+    """Algorithmic HBM bytes of one backward pass: the forward's inputs, dy and S0/dS_T
+    read once, dx, dc, dq, dmu and dS0 written once (the workspace is scratch)."""
+    xb = 2 if w.x_dtype == "bf16" else 4
+    qb = 2 if w.q_dtype == "bf16" else 4
+    per_tok = (w.d * xb + w.m * qb + 4 * w.m + 4 + 4 * w.d) + (4 * w.d + 8 * w.m + 4)
+    return w.B * w.T * w.H * per_tok + 3 * 4 * w.B * w.H * w.m * w.d
+
+
 def chunk_mma_flops(w: LI.Workload, C: int, B=None, T=None, H=None) -> int:
     """Tensor-core flops of the chunked form per token and head: 6md + C(m+d)
     (projection, inter-chunk read-out and state update: 2md each; causal score
@@ -353,6 +362,44 @@ def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 12.0, max_r
 
 # ---------------------------------------------------------------------- main
 
+def bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush, pk, pk_src):
+    """--pass bwd: one step is one lattice_scan_bwd of the workload (gradients of every
+    input for unit dy), workspace allocated once outside the timed region."""
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        times = time_bwd(torch, L, t, w.chunk, args.steps, args.warmup, flush=flush)
+    torch.cuda.synchronize()
+    total_ms = max_over_ranks(torch, dist, sum(times), device)
+    if dist is not None:
+        dist.barrier()
+    if rank != 0:
+        return 0
+    ms = total_ms / args.steps
+    alg_b = bwd_alg_bytes(w)
+    kern_ms = statistics.mean(times)
+    achieved = alg_b / (kern_ms * 1e-3) / 1e9
+    kname = "scan_bwd_kernel<chunked>" if w.chunk > 1 else "scan_bwd_kernel<exact>"
+    line = {"metric": "Lattice layer bwd tokens/s (1 B200)", "value": job_tokens_per_s(world, w, ms),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "pass": "bwd", "B": w.B, "H": w.H, "T": w.T, "m": w.m,
+                       "d": w.d, "chunk": w.chunk, "x_q_dtype": "bf16",
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "parallelism": f"independent batches per GPU x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": kname,
+                         "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"},
+            "gpu_launches": args.steps}
+    cs = clk.summary()
+    if cs is not None:
+        line["clocks"] = cs
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -364,6 +411,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--workload", default=HEADLINE, choices=["small_train", "mid_layer", "long_ctx"],
                     help="chunked workload of the timed step (default: the small training shape)")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time the backward pass (lattice_scan_bwd) of the workload instead")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -419,6 +468,9 @@ def main():
     inp = LI.make_inputs(w)
     t = _dev_inputs(torch, inp, device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    if args.which == "bwd":
+        return bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush, pk, pk_src)
 
     if dist is not None:
         dist.barrier()
