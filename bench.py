@@ -115,8 +115,7 @@ def job_tokens_per_s(world: int, w: LI.Workload, ms_per_step: float) -> float:
 # DRAM bytes (read + write) per launch, from one `ncu --set full` capture of each kernel on
 # each workload (the profile summaries keep the commands). None where no capture exists.
 CAPTURED_TRAFFIC = {
-    ("chunk_split_kernel", "small_train"): 34.41e6 + 0.19e6,
-    ("chunk_split_kernel", "long_ctx"): 676.22e6 + 500.96e6,
+    ("chunk_split_kernel", "small_train"): 34.56e6,  # dram__bytes.sum.per_second x duration
     ("chunk_tc_kernel", "mid_layer"): 550.62e6 + 240.43e6,
 }
 

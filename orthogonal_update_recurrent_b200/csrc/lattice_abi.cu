@@ -144,21 +144,52 @@ int bwd_seg(int chunk, int seg) {
     return (seg > 0 && seg % chunk == 0) ? seg : -1;
 }
 
-template <int D, int RQ, bool CH>
-lattice_status launch_bwd_t(const BwdArgs& a, int nw, cudaStream_t st) {
-    const size_t smem = bwd_smem_bytes(D, a.m, nw);
-    auto k = scan_bwd_kernel<D, RQ, CH>;
+// CTAs per sequence for the backward: enough clusters to cover the device's SMs when
+// the batch has fewer sequences than SMs (at most 8, the portable cluster size, and
+// at least 4 and at most 32 slots per CTA).
+int bwd_split(int B, int H, int m) {
+    const long long seqs = (long long)B * H;
+    long long G = sm_count() / seqs;
+    if (G > 8) G = 8;
+    if (G > (m + 3) / 4) G = (m + 3) / 4;
+    if (G < 2 || (m + G - 1) / G > 32) return 1;
+    return (int)G;
+}
+
+template <int D, int RQ, bool CH, bool SPLIT>
+lattice_status launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
+    constexpr int nt = bwd_threads(SPLIT);
+    const size_t smem = bwd_smem_bytes(D, a.spc, nt / 32);
+    auto k = scan_bwd_kernel<D, RQ, CH, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e);
-    k<<<a.B * a.H, nw * 32, smem, st>>>(a);
+    if (a.G == 1) {
+        k<<<a.B * a.H, nt, smem, st>>>(a);
+        return launch_status();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.B * a.H * a.G));
+    cfg.blockDim = dim3((unsigned)nt);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)a.G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k, a);
+    if (e != cudaSuccess) return cuda_fail(e);
     return launch_status();
 }
 
+// One CTA per sequence: 16 warps, one slot (m <= 64) or two (m <= 128) per octet.
+// Clusters: 8 warps per CTA, one slot per octet (bwd_split keeps <= 32 slots per CTA).
 template <int D, bool CH>
 lattice_status launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
-    const int quads = (a.m + 3) / 4;
-    if (quads <= 16) return launch_bwd_t<D, 1, CH>(a, quads < 4 ? 4 : quads, st);
-    return launch_bwd_t<D, 2, CH>(a, 16, st);
+    if (a.G == 1) return a.m <= 64 ? launch_bwd_t<D, 1, CH, false>(a, st) : launch_bwd_t<D, 2, CH, false>(a, st);
+    return launch_bwd_t<D, 1, CH, true>(a, st);
 }
 
 template <bool CH>
@@ -354,7 +385,8 @@ size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int c
     if (check_dims(B, H, m, d) != LATTICE_OK || m > kBwdMaxM) return 0;
     const int seg = bwd_seg(chunk_size, seg_tokens);
     if (seg < 1) return 0;
-    return (size_t)B * H * bwd_ws_floats_per_seq(T, m, d, seg) * sizeof(float);
+    const int G = bwd_split(B, H, m), spc = (m + G - 1) / G;
+    return (size_t)B * H * G * bwd_ws_floats_per_seq(T, spc, d, seg) * sizeof(float);
 }
 
 lattice_status lattice_scan_bwd(const void* x, lattice_dtype x_dtype, const float* c,
@@ -398,8 +430,10 @@ lattice_status lattice_scan_bwd(const void* x, lattice_dtype x_dtype, const floa
         for (size_t k = i + 1; k < sizeof(outs) / sizeof(outs[0]); ++k)
             if (overlap(outs[i], outs[k])) return LATTICE_ERR_INVALID_ARG;
     }
+    const int G = bwd_split(B, H, m);
     BwdArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, dy, dS_T,
-              dx, dc, dq, dmu, deta_w, dS0, static_cast<float*>(workspace), B, T, H, m, chunk_size, seg};
+              dx, dc, dq, dmu, deta_w, dS0, static_cast<float*>(workspace), B, T, H, m, chunk_size, seg,
+              G, (m + G - 1) / G};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return chunk_size == 1 ? launch_bwd<false>(a, d, st) : launch_bwd<true>(a, d, st);
 }

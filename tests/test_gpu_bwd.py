@@ -90,6 +90,16 @@ def test_bwd_chunked_shapes(L, m, d, C):
     check(run_gpu_bwd(L, inp, cot, C), run_oracle_bwd(inp, cot, C), TOL_BWD)
 
 
+@pytest.mark.parametrize("m,d,C", [(64, 64, 1), (64, 64, 16), (128, 64, 1), (128, 32, 8)])
+def test_bwd_batch_filling_the_device(L, m, d, C):
+    """80 sequences (more than half the SMs): one CTA per sequence instead of a
+    cluster, including the two-slots-per-octet layout at m = 128."""
+    w = LI.Workload("t", B=10, T=40, H=8, m=m, d=d, seed=830 + m + d + C)
+    inp = with_eta(LI.make_inputs(w), 830)
+    cot = LI.make_cotangents(inp, seed=830 + C)
+    check(run_gpu_bwd(L, inp, cot, C), run_oracle_bwd(inp, cot, C), TOL_BWD)
+
+
 def test_bwd_without_eta_and_final_state_gradient(L):
     w = LI.Workload("t", B=1, T=70, H=3, m=32, d=64, seed=840)
     inp = LI.make_inputs(w)
