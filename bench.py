@@ -116,7 +116,11 @@ def job_tokens_per_s(world: int, w: LI.Workload, ms_per_step: float) -> float:
 # each workload (the profile summaries keep the commands). None where no capture exists.
 CAPTURED_TRAFFIC = {
     ("chunk_split_kernel", "small_train"): 34.56e6,  # dram__bytes.sum.per_second x duration
+    ("chunk_split_kernel", "long_ctx"): 676.05e6 + 498.46e6,
     ("chunk_tc_kernel", "mid_layer"): 550.62e6 + 240.43e6,
+    ("scan_simt_kernel<exact>", "small_train"): 34.48e6 + 0.12e6,
+    ("scan_bwd_kernel<chunked>", "small_train"): 70.75e6 + 57.51e6,
+    ("step_kernel", "decode"): 545.32e6 + 482.93e6,
 }
 
 
@@ -361,6 +365,42 @@ def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 12.0, max_r
 
 # ---------------------------------------------------------------------- main
 
+def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
+    """--pass step: one step is one decode token for every (b,h) of the decode workload
+    (lattice_step, state updated in place), steps replayed from a CUDA graph."""
+    wd = rank_workload(LI.WORKLOADS["decode"], rank)
+    ring = 40
+    n = max(ring, (args.steps // ring) * ring)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms, n = time_decode(torch, L, wd, n, ring, device)
+    torch.cuda.synchronize()
+    step_ms = max_over_ranks(torch, dist, step_ms, device)
+    if rank != 0:
+        return 0
+    sb = step_alg_bytes(wd)
+    gbps = sb / (step_ms * 1e-3) / 1e9
+    line = {"metric": "Lattice decode step GB/s (1 B200)", "value": gbps * world, "unit": "GB/s",
+            "n_gpus": world, "steps": n, "warmup": 3, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wd.name, "pass": "step", "B": wd.B, "H": wd.H, "m": wd.m, "d": wd.d,
+                       "x_q_dtype": "bf16", "state_dtype": "f32",
+                       "l2": "state (512 MiB) and input ring exceed L2",
+                       "parallelism": f"independent batches per GPU x{world}"},
+            "roofline": {"bound": "hbm", "achieved": gbps, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbps / pk["hbm_gbs"], "traffic": CAPTURED_TRAFFIC.get(("step_kernel", "decode")),
+                         "kernel": "step_kernel",
+                         "alg_bytes_per_launch": sb, "peak_source": f"{pk_src} (burst copy)"},
+            "gpu_launches": n}
+    cs = clk.summary()
+    if cs is not None:
+        line["clocks"] = cs
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush, pk, pk_src):
     """--pass bwd: one step is one lattice_scan_bwd of the workload (gradients of every
     input for unit dy), workspace allocated once outside the timed region."""
@@ -389,7 +429,8 @@ def bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush,
                        "l2": "flushed between timed steps (256 MiB write)",
                        "parallelism": f"independent batches per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": kname,
+                         "frac": achieved / pk["hbm_gbs"], "traffic": CAPTURED_TRAFFIC.get((kname, w0.name)),
+                         "kernel": kname,
                          "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"},
             "gpu_launches": args.steps}
     cs = clk.summary()
@@ -410,8 +451,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--workload", default=HEADLINE, choices=["small_train", "mid_layer", "long_ctx"],
                     help="chunked workload of the timed step (default: the small training shape)")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
-                    help="bwd: time the backward pass (lattice_scan_bwd) of the workload instead")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "step"],
+                    help="bwd: time the backward pass (lattice_scan_bwd) of the workload instead; "
+                         "step: time the decode step (lattice_step) on the decode workload")
+    ap.add_argument("--chunk", type=int, default=None,
+                    help="override the workload's chunk size (1: the exact recurrence)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -419,6 +463,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w0 = LI.WORKLOADS[args.workload]
+    if args.chunk is not None:
+        w0 = w0.with_(chunk=args.chunk)
     w = rank_workload(w0, rank)
 
     if args.impl == "reference":
@@ -470,6 +516,8 @@ def main():
 
     if args.which == "bwd":
         return bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush, pk, pk_src)
+    if args.which == "step":
+        return bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src)
 
     if dist is not None:
         dist.barrier()
@@ -489,7 +537,8 @@ def main():
     alg_b = scan_alg_bytes(w)
     kern_ms = statistics.mean(times)
     achieved = alg_b / (kern_ms * 1e-3) / 1e9
-    kname = {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(kimpl, "scan_simt_kernel<chunked>")
+    kname = {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(
+        kimpl, "scan_simt_kernel<chunked>" if w.chunk > 1 else "scan_simt_kernel<exact>")
     roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / pk["hbm_gbs"], "traffic": CAPTURED_TRAFFIC.get((kname, w0.name)),
             "kernel": kname,
