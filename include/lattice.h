@@ -194,7 +194,7 @@ lattice_status lattice_scan_bwd(const void *x, lattice_dtype x_dtype, const floa
 /* Workspace bytes lattice_scan_bwd needs for this shape on the current device:
  * B*H*G*(n_seg - 1 + seg_tokens)*ceil(m/G)*d*4 with n_seg = ceil(T/seg_tokens)
  * (seg_tokens as resolved by lattice_scan_bwd) and G the CTAs per sequence the call
- * uses (G = 1 when the batch fills the device's SMs; up to 8 otherwise, so about
+ * uses (G = 1 when the batch fills the device's SMs; up to 4 otherwise, so about
  * B*H*(n_seg - 1 + seg_tokens)*m*d*4). Returns 0 for arguments lattice_scan_bwd
  * would reject. Host function; launches nothing. */
 size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int chunk_size,

@@ -54,6 +54,38 @@ lattice_status launch_status() {
     return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
 }
 
+// CTAs per sequence for the CUDA-core scans: when the batch has fewer sequences than
+// SMs, a cluster of G CTAs per sequence covers more of the device (G at most 4, at
+// least 4 and at most 32 slots per CTA); otherwise 1. Measured on B200: 8-CTA clusters
+// (8 slots per CTA) ran the long-context backward at half the speed of 4-CTA ones.
+int cluster_split(int B, int H, int m) {
+    const long long seqs = (long long)B * H;
+    long long G = sm_count() / seqs;
+    if (G > 4) G = 4;
+    if (G > (m + 3) / 4) G = (m + 3) / 4;
+    if (G < 2 || (m + G - 1) / G > 32) return 1;
+    return (int)G;
+}
+
+lattice_status launch_clusters(const void* kernel, int grid, int block, size_t smem, int G,
+                               cudaStream_t st, void** args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, args);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return launch_status();
+}
+
 // ---- exact / chunked CUDA-core scan
 template <int D, int RQ, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
@@ -65,8 +97,29 @@ lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
     return launch_status();
 }
 
+// one cluster of a.G CTAs (8 warps each) per sequence; similarity objective
+template <int D, bool CH, bool LIN1>
+lattice_status launch_scan_simt_split(const ScanArgs& a, cudaStream_t st) {
+    const size_t smem = scan_smem_bytes<D>(a.m, 8, false, true);
+    auto k = scan_simt_kernel<D, 1, CH, false, LIN1, true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ScanArgs arg = a;
+    void* args[] = {&arg};
+    return launch_clusters(reinterpret_cast<const void*>(k), a.B * a.H * a.G, 256, smem, a.G, st, args);
+}
+
 template <int D, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
+    if constexpr (!DEC) {  // the reconstruction objective couples every slot on every token
+        const int G = cluster_split(a.B, a.H, a.m);
+        if (G > 1) {
+            ScanArgs s = a;
+            s.G = G;
+            s.spc = (a.m + G - 1) / G;
+            return launch_scan_simt_split<D, CH, LIN1>(s, st);
+        }
+    }
     const int quads = (a.m + 3) / 4;
     if (quads <= 16) return launch_scan_simt_t<D, 1, CH, DEC, LIN1>(a, quads < 4 ? 4 : quads, st);
     if (quads <= 32) return launch_scan_simt_t<D, 2, CH, DEC, LIN1>(a, 16, st);
@@ -144,17 +197,8 @@ int bwd_seg(int chunk, int seg) {
     return (seg > 0 && seg % chunk == 0) ? seg : -1;
 }
 
-// CTAs per sequence for the backward: enough clusters to cover the device's SMs when
-// the batch has fewer sequences than SMs (at most 8, the portable cluster size, and
-// at least 4 and at most 32 slots per CTA).
-int bwd_split(int B, int H, int m) {
-    const long long seqs = (long long)B * H;
-    long long G = sm_count() / seqs;
-    if (G > 8) G = 8;
-    if (G > (m + 3) / 4) G = (m + 3) / 4;
-    if (G < 2 || (m + G - 1) / G > 32) return 1;
-    return (int)G;
-}
+// CTAs per sequence of the backward kernel (see cluster_split).
+int bwd_split(int B, int H, int m) { return cluster_split(B, H, m); }
 
 template <int D, int RQ, bool CH, bool SPLIT>
 lattice_status launch_bwd_t(const BwdArgs& a, cudaStream_t st) {

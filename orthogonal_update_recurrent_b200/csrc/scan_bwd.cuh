@@ -11,7 +11,7 @@
 //   y_t = sum_i q_i s_t,i.
 // The adjoint walks the tokens backwards, carrying dL/ds_t in registers.
 //
-// Each (b, h) sequence runs on a cluster of G CTAs (G = 1: a single CTA); CTA g
+// Each (b, h) sequence runs on a cluster of G <= 4 CTAs (G = 1: a single CTA); CTA g
 // owns slots [g*spc, (g+1)*spc) in registers in the octet layout (common.cuh).
 // Slots evolve independently under the similarity objective, so the CTAs share
 // nothing but the per-token sums over slots (dx, dmu, deta): each CTA reduces its
@@ -556,8 +556,12 @@ __global__ void __launch_bounds__(bwd_threads(SPLIT)) scan_bwd_kernel(BwdArgs a)
                 // peers may still read this one; the next cluster barrier orders the reuse.
                 for (int idx = crank * NT + tid; idx < n * (D + 2); idx += G * NT) {
                     const int tok = idx / (D + 2), k = idx - tok * (D + 2);
+                    float pv[8];  // every peer's load in flight before the fixed-order sum
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) pv[r] = r < G ? bwd_ld_peer(part + idx, (uint32_t)r) : 0.f;
                     float v = 0.f;
-                    for (int r = 0; r < G; ++r) v += bwd_ld_peer(part + idx, (uint32_t)r);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) if (r < G) v += pv[r];
                     const size_t bth = ((size_t)b * T + t0 + tok) * H + h;
                     if (k < D) a.dx[bth * D + k] = v;
                     else if (k == D) a.dmu[bth] = v;

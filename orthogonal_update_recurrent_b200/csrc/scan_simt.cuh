@@ -32,6 +32,8 @@ struct ScanArgs {
     float* y;
     int B, T, H, m, chunk;
     int cnorm;  // chunked CUDA-core path: no per-token normaliser, unit slots after each chunk
+    int G;      // SPLIT kernels: CTAs per sequence (a cluster), each owning spc slots
+    int spc;
 };
 
 // Per-token staged record: x[D] | q[m] | c[m] | mu | eta, padded to a multiple
@@ -39,11 +41,25 @@ struct ScanArgs {
 __host__ __device__ inline int scan_record_floats(int D, int m) { return (D + 2 * m + 2 + 3) & ~3; }
 
 // Shared memory: in[2][TB][record] floats, ybuf[2][TB][NW][D] floats and, for the
-// reconstruction objective, rbuf[2][NW][D] floats (per-warp partial reconstructions).
+// reconstruction objective, rbuf[2][NW][D] floats (per-warp partial reconstructions);
+// split kernels add ypart[2][TB][D] (the CTA's read-out partials for the cluster sum).
 template <int D>
-__host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec) {
+__host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec, bool split = false) {
     return sizeof(float) * (2ull * kScanTB * scan_record_floats(D, m) + 2ull * kScanTB * nw * D +
-                            (dec ? 2ull * nw * D : 0ull));
+                            (dec ? 2ull * nw * D : 0ull) + (split ? 2ull * kScanTB * D : 0ull));
+}
+
+// Cluster barrier and a load from a peer CTA's shared memory (split kernels).
+__device__ __forceinline__ void scan_cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float scan_ld_peer(const float* local_ptr, uint32_t rank) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local_ptr));
+    uint32_t r;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r) : "memory");
+    return v;
 }
 
 // DEC selects the reconstruction objective (§3.1.1 eq. decoding_recurrence): each
@@ -53,8 +69,14 @@ __host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec) {
 // LIN1 (chunked only) selects the chunk linearisation of eq. recurrence_linear1
 // (§3.4.1): the projection part of each token's update scales the chunk-start slot
 // instead of the running one.
-template <int D, int RQ, bool CHUNKED, bool DEC, bool LIN1 = false>
-__global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
+// SPLIT (similarity objective only): each sequence runs on a cluster of a.G CTAs of
+// 8 warps; CTA g owns slots [g*spc, (g+1)*spc), spc <= 32. The slots evolve
+// independently, so the CTAs share only the read-out: each block's per-CTA partial
+// y is added over the cluster through distributed shared memory, ranks in a fixed
+// order (one cluster barrier per block of tokens).
+template <int D, int RQ, bool CHUNKED, bool DEC, bool LIN1 = false, bool SPLIT = false>
+__global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a) {
+    static_assert(!(SPLIT && (DEC || RQ != 1)), "split kernels: similarity objective, one slot per octet");
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
     extern __shared__ __align__(16) float smem[];
@@ -62,13 +84,15 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
     const int NT = blockDim.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j = lane & 7, oct = lane >> 3;
-    const int bh = blockIdx.x;
+    const int G = SPLIT ? a.G : 1, crank = SPLIT ? (int)(blockIdx.x % G) : 0;
+    const int bh = blockIdx.x / G;
     const int b = bh / a.H, h = bh % a.H;
     const int m = a.m, T = a.T, H = a.H;
     const int per_tok = scan_record_floats(D, m);  // x | q | c | mu | eta | pad
     float* in_buf = smem;
     float* ybuf = smem + 2 * kScanTB * per_tok;
     float* rbuf = ybuf + 2 * kScanTB * NW * D;  // DEC only
+    float* ypart = rbuf + (DEC ? 2 * NW * D : 0);  // SPLIT only: [2][TB][D]
 
     // ---- load the initial state into registers
     float s[RQ][EPL];
@@ -79,6 +103,7 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
 #pragma unroll
     for (int r = 0; r < RQ; ++r) {
         slot[r] = 4 * (warp + NW * r) + oct;
+        if constexpr (SPLIT) slot[r] = slot[r] < a.spc ? crank * a.spc + slot[r] : m;  // m: no slot
         if (slot[r] < m) {
             load_row_f32<D>(S0bh + (size_t)slot[r] * D, j, s[r]);
         } else {
@@ -92,8 +117,9 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
     // ---- staging helpers
     const int n_blocks = (T + kScanTB - 1) / kScanTB;
     const int stage_total = kScanTB * per_tok;
-    // per-thread staging registers: the host launches NW >= 4 warps when RQ == 1, NW = 16 otherwise
-    constexpr int kMinThreads = RQ == 1 ? 128 : 512;
+    // per-thread staging registers: the host launches NW >= 4 warps when RQ == 1, NW = 16
+    // otherwise, and 8 warps for split kernels
+    constexpr int kMinThreads = SPLIT ? 256 : (RQ == 1 ? 128 : 512);
     constexpr int kStg = (kScanTB * (D + 2 * kMaxM + 4) + kMinThreads - 1) / kMinThreads;
     float stg[kStg];
     auto stage_load = [&](int blk) {
@@ -126,6 +152,42 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
         }
     };
 
+    // Read-out of block fb: fixed-order sum over the warps (and, for split kernels,
+    // over the cluster's CTAs, each CTA writing a share of the block's entries).
+    auto flush_y = [&](int fb) {
+        const int pt0 = fb * kScanTB, ntok = min(kScanTB, T - pt0);
+        const float* yb = ybuf + (size_t)(fb & 1) * kScanTB * NW * D;
+        if constexpr (!SPLIT) {
+            for (int idx = tid; idx < ntok * D; idx += NT) {
+                int tok = idx / D, k = idx - tok * D;
+                float acc = 0.f;
+                for (int w = 0; w < NW; ++w) acc += yb[((size_t)tok * NW + w) * D + k];
+                a.y[(((size_t)b * T + pt0 + tok) * H + h) * D + k] = acc;
+            }
+        } else {
+            // the partial buffers alternate by block; the next flush's cluster barrier
+            // orders their reuse after every peer has read them
+            float* part = ypart + (size_t)(fb & 1) * kScanTB * D;
+            for (int idx = tid; idx < ntok * D; idx += NT) {
+                int tok = idx / D, k = idx - tok * D;
+                float acc = 0.f;
+                for (int w = 0; w < NW; ++w) acc += yb[((size_t)tok * NW + w) * D + k];
+                part[idx] = acc;
+            }
+            scan_cluster_sync();
+            for (int idx = crank * NT + tid; idx < ntok * D; idx += G * NT) {
+                int tok = idx / D, k = idx - tok * D;
+                float v[8];  // every peer's load in flight before the fixed-order sum
+#pragma unroll
+                for (int r = 0; r < 8; ++r) v[r] = r < G ? scan_ld_peer(part + idx, (uint32_t)r) : 0.f;
+                float acc = 0.f;
+#pragma unroll
+                for (int r = 0; r < 8; ++r) if (r < G) acc += v[r];
+                a.y[(((size_t)b * T + pt0 + tok) * H + h) * D + k] = acc;
+            }
+        }
+    };
+
     if (n_blocks > 0) {
         stage_load(0);
         stage_store(0);
@@ -135,17 +197,8 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
     for (int blk = 0; blk < n_blocks; ++blk) {
         const int buf = blk & 1;
         const int t0 = blk * kScanTB;
-        // flush the previous block's read-out (fixed-order sum over warps)
-        if (blk > 0) {
-            const int pt0 = t0 - kScanTB;
-            const float* yb = ybuf + (size_t)(buf ^ 1) * kScanTB * NW * D;
-            for (int idx = tid; idx < kScanTB * D; idx += NT) {
-                int tok = idx / D, k = idx - tok * D;
-                float acc = 0.f;
-                for (int w = 0; w < NW; ++w) acc += yb[((size_t)tok * NW + w) * D + k];
-                a.y[(((size_t)b * T + pt0 + tok) * H + h) * D + k] = acc;
-            }
-        }
+        // flush the previous block's read-out
+        if (blk > 0) flush_y(blk - 1);
         if (blk + 1 < n_blocks) stage_load(blk + 1);
 
         const float* inb = in_buf + buf * stage_total;
@@ -325,18 +378,8 @@ __global__ void __launch_bounds__(512) scan_simt_kernel(ScanArgs a) {
         __syncthreads();
     }
     // flush the last block
-    if (n_blocks > 0) {
-        const int lb = n_blocks - 1;
-        const int pt0 = lb * kScanTB;
-        const int ntok = min(kScanTB, T - pt0);
-        const float* yb = ybuf + (size_t)(lb & 1) * kScanTB * NW * D;
-        for (int idx = tid; idx < ntok * D; idx += NT) {
-            int tok = idx / D, k = idx - tok * D;
-            float acc = 0.f;
-            for (int w = 0; w < NW; ++w) acc += yb[((size_t)tok * NW + w) * D + k];
-            a.y[(((size_t)b * T + pt0 + tok) * H + h) * D + k] = acc;
-        }
-    }
+    if (n_blocks > 0) flush_y(n_blocks - 1);
+    if constexpr (SPLIT) scan_cluster_sync();  // no CTA leaves while a peer may still read its partials
     // final state
     float* Sbh = a.S_out + (size_t)bh * m * D;
 #pragma unroll

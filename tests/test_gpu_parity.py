@@ -541,3 +541,20 @@ def test_chunk_norm_chunk_one_is_exact_and_tensor_cores_refuse(L):
     for impl in ("tcgen05", "tcgen05_split"):
         with pytest.raises(L.LatticeError):
             run_gpu(L, inp, 64, impl=impl, norm="chunk")
+
+
+# ------------------------------------------- batches that fill the device
+
+@pytest.mark.parametrize("m,d,C,lin,norm", [(64, 64, 1, 2, "token"), (64, 32, 16, 2, "token"),
+                                            (128, 64, 1, 2, "token"), (48, 64, 8, 1, "token"),
+                                            (64, 64, 16, 2, "chunk")])
+def test_cuda_core_scan_batch_filling_the_device(L, m, d, C, lin, norm):
+    """80 sequences (more than half the SMs): one CTA per sequence instead of a
+    cluster per sequence, for the exact recurrence and the CUDA-core chunked forms."""
+    w = LI.Workload("t", B=10, T=37, H=8, m=m, d=d, x_dtype="f32", q_dtype="f32",
+                    seed=950 + m + d + C + lin)
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, C, impl="simt" if C > 1 else "auto", lin=lin, norm=norm)
+    yo, So = run_oracle(inp, C, lin=lin, norm=norm)
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
