@@ -363,6 +363,34 @@ def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 12.0, max_r
     return tok / el, cores, sample
 
 
+def oracle_legs(w: LI.Workload, seconds: float = 3.0) -> dict:
+    """Further oracle timings on the host: the exact recurrence on all cores, the
+    chunked form on one thread, and decode steps of the decode workload (3 steps of
+    the full 512 MiB state, per step)."""
+    import oracle
+    inp = LI.make_inputs(w)
+    cores = len(os.sched_getaffinity(0))
+
+    def rate(chunk, threads):
+        t0, reps = time.perf_counter(), 0
+        while True:
+            oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=chunk, nthreads=threads)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                return w.B * w.T * reps / el
+    out = {"exact_tokens_per_s": rate(1, cores), "chunked_tokens_per_s_1_thread": rate(w.chunk, 1)}
+    wd = LI.WORKLOADS["decode"]
+    S = LI.make_decode_state(wd).astype(np.float64)
+    st = LI.make_decode_steps(wd, 3)
+    t0 = time.perf_counter()
+    for k in range(3):
+        _, S, _ = oracle.step(S, st["x"][k], st["c"][k], st["q"][k], st["mu"][k], nthreads=cores)
+    out["decode_us_per_step"] = 1e6 * (time.perf_counter() - t0) / 3
+    out["decode_sample"] = f"3 steps of B={wd.B} H={wd.H} m={wd.m} d={wd.d}, fp64 oracle, {cores} threads"
+    return out
+
+
 # ---------------------------------------------------------------------- main
 
 def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
@@ -651,7 +679,7 @@ def main():
         if not args.no_cpu:
             v, cores, sample = oracle_baseline(w, w.chunk)
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                    "sample": sample}
+                                    "sample": sample, "legs": oracle_legs(w)}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

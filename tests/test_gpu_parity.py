@@ -558,3 +558,41 @@ def test_cuda_core_scan_batch_filling_the_device(L, m, d, C, lin, norm):
     yo, So = run_oracle(inp, C, lin=lin, norm=norm)
     assert y_err(yg, yo) <= TOL_F32
     assert s_err(Sg, So) <= TOL_F32
+
+
+def test_decode_workload_full_size_1000_steps(L):
+    """The decode workload at full size (B=256, H=32, m=d=128, fp32 state of 512 MiB),
+    1000 consecutive steps in place, inputs cycling through a ring of 40 pre-drawn
+    steps: every head against the oracle for the first 3 steps, then 64 sampled heads
+    at every step and their final state."""
+    w = LI.WORKLOADS["decode"]
+    ring = 40
+    S0 = LI.make_decode_state(w)
+    st = LI.make_decode_steps(w, ring)
+    S = torch.from_numpy(S0).cuda()
+    dev = {k: dev_inputs({"x": st["x"][k], "q": st["q"][k], "c": st["c"][k], "mu": st["mu"][k],
+                          "x_bits": st["x_bits"][k], "q_bits": st["q_bits"][k], "eta": None})
+           for k in range(ring)}
+    rng = np.random.default_rng(5)
+    flat = rng.choice(w.B * w.H, size=64, replace=False)
+    bs, hs = flat // w.H, flat % w.H
+    So = S0.astype(np.float64)
+    for k in range(1000):
+        r = k % ring
+        t = dev[r]
+        y = L.step(S, t["x"], t["c"], t["q"], t["mu"])
+        if k < 3:  # every head
+            yo, So, _ = oracle.step(So, st["x"][r], st["c"][r], st["q"][r], st["mu"][r])
+            torch.cuda.synchronize()
+            assert y_err(y.cpu().numpy()[:, None], yo[:, None]) <= TOL_F32, k
+            if k == 2:
+                So = np.ascontiguousarray(So[bs, hs][:, None])  # keep the sampled heads
+        else:
+            sub = lambda a: np.ascontiguousarray(a[bs, hs][:, None])
+            yo, So, _ = oracle.step(So, sub(st["x"][r]), sub(st["c"][r]), sub(st["q"][r]), sub(st["mu"][r]))
+            yg = y[torch.from_numpy(bs).cuda(), torch.from_numpy(hs).cuda()].cpu().numpy()
+            assert y_err(yg[:, None, None], yo[:, None]) <= TOL_F32, k
+    L.device_status()
+    Sg = S[torch.from_numpy(bs).cuda(), torch.from_numpy(hs).cuda()].cpu().numpy()[:, None]
+    assert s_err(Sg, So) <= TOL_F32
+    np.testing.assert_allclose(np.linalg.norm(Sg, axis=-1), 1.0, atol=1e-5)
