@@ -175,6 +175,57 @@ __device__ __forceinline__ void update_coefs(float n2, float p, float xx, float 
     gamma = ok ? a * iw : 0.f;
 }
 
+// As update_coefs, with |x_perp|^2 = |x - (p/n2) s_ref|^2 given, summed directly over
+// the elements instead of as xx - p^2/n2. The reconstruction objective's write
+// direction can be long and nearly parallel to a slot (|x|^2 ~ 1e4 against
+// |x_perp|^2 ~ 4), where that difference cancels away most of fp32's digits.
+template <bool PRECISE>
+__device__ __forceinline__ void update_coefs_perp(float n2, float p, float perp2, float c, float mu,
+                                                  float eta, float target, float& alpha,
+                                                  float& gamma) {
+    bool ok = n2 > 0.f;
+    float n2s = ok ? n2 : 1.f;
+    float inv_n = PRECISE ? __frsqrt_rn(n2s) : rsqrtf(n2s);
+    float r = PRECISE ? __fdiv_rn(p, n2s) : __fdividef(p, n2s);
+    float a = eta * c * inv_n;
+    float w2 = fmaf(a * a, perp2, mu * mu * n2s);
+    ok = ok && (w2 > 0.f);
+    float iw = (PRECISE ? __frsqrt_rn(ok ? w2 : 1.f) : rsqrtf(ok ? w2 : 1.f)) * target;
+    alpha = ok ? fmaf(-a, r, mu) * iw : 1.f;
+    gamma = ok ? a * iw : 0.f;
+}
+
+// The lane's share of |x - (p/n2) s|^2 (octet-summed by the caller).
+template <int EPL>
+__device__ __forceinline__ float perp2_partial(const float* x, const float* s, float p, float n2) {
+    const float r = n2 > 0.f ? __fdiv_rn(p, n2) : 0.f;
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < EPL; ++k) {
+        const float u = fmaf(-r, s[k], x[k]);
+        acc = fmaf(u, u, acc);
+    }
+    return acc;
+}
+
+// As update_coefs_lin1, with |x_perp|^2 given (see update_coefs_perp).
+template <bool PRECISE>
+__device__ __forceinline__ void update_coefs_lin1_perp(float n2, float p, float perp2, float c, float mu,
+                                                       float eta, float target, float& alpha_s,
+                                                       float& alpha_0, float& gamma) {
+    bool ok = n2 > 0.f;
+    float n2s = ok ? n2 : 1.f;
+    float inv_n = PRECISE ? __frsqrt_rn(n2s) : rsqrtf(n2s);
+    float r = PRECISE ? __fdiv_rn(p, n2s) : __fdividef(p, n2s);
+    float a = eta * c * inv_n;
+    float w2 = fmaf(a * a, perp2, mu * mu * n2s);
+    ok = ok && (w2 > 0.f);
+    float iw = (PRECISE ? __frsqrt_rn(ok ? w2 : 1.f) : rsqrtf(ok ? w2 : 1.f)) * target;
+    alpha_s = ok ? mu * iw : 1.f;
+    alpha_0 = ok ? -a * r * iw : 0.f;
+    gamma = ok ? a * iw : 0.f;
+}
+
 // As update_coefs, split for the chunk linearisation of eq. recurrence_linear1
 // (§3.4.1): the new slot is alpha_s*s + alpha_0*s0 + gamma*x, where the forget part
 // mu scales the running slot s and the projection part (-a p/n^2) the chunk-start

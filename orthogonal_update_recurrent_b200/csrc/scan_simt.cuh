@@ -299,6 +299,9 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
                         alpha_s = mu;
                         alpha_0 = -ac * rr;
                         gamma = ac;
+                    } else if constexpr (DEC) {  // |x_perp|^2 summed directly (see update_coefs_perp)
+                        const float pp2 = octet_sum(perp2_partial<EPL>(xv, s0[r], p[r], n0sq[r]));
+                        update_coefs_lin1_perp<true>(n0sq[r], p[r], pp2, cv, mu, eta, n0[r], alpha_s, alpha_0, gamma);
                     } else {
                         update_coefs_lin1<true>(n0sq[r], p[r], xx, cv, mu, eta, n0[r], alpha_s, alpha_0, gamma);
                     }
@@ -316,9 +319,13 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
                         const float rr = ok ? __fdiv_rn(p[r], n0sq[r]) : 0.f;     // p / n^2
                         alpha = ok ? fmaf(-ac, rr, mu) : 1.f;
                         gamma = ac;
+                    } else if constexpr (DEC) {  // |x_perp|^2 summed directly (see update_coefs_perp)
+                        const float nr2 = CHUNKED ? n0sq[r] : n2[r];
+                        const float pp2 = octet_sum(perp2_partial<EPL>(xv, CHUNKED ? s0[r] : s[r], p[r], nr2));
+                        update_coefs_perp<true>(nr2, p[r], pp2, cv, mu, eta, CHUNKED ? n0[r] : 1.f, alpha, gamma);
                     } else {
-                        update_coefs<CHUNKED || DEC>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
-                                                     CHUNKED ? n0[r] : 1.f, alpha, gamma);
+                        update_coefs<CHUNKED>(CHUNKED ? n0sq[r] : n2[r], p[r], xx, cv, mu, eta,
+                                              CHUNKED ? n0[r] : 1.f, alpha, gamma);
                     }
                     if (!valid) { alpha = 0.f; gamma = 0.f; }
 #pragma unroll

@@ -115,7 +115,12 @@ __global__ void __launch_bounds__(512) step_kernel(StepArgs a) {
 #pragma unroll
     for (int r = 0; r < RQ; ++r) {
         float alpha, gamma;
-        update_coefs<DEC>(n2[r], p[r], xx, cv[r], mu, eta, 1.f, alpha, gamma);
+        if constexpr (DEC) {  // |x_perp|^2 summed directly: the residual can be near a slot
+            const float pp2 = octet_sum(perp2_partial<EPL>(xv, s[r], p[r], n2[r]));
+            update_coefs_perp<true>(n2[r], p[r], pp2, cv[r], mu, eta, 1.f, alpha, gamma);
+        } else {
+            update_coefs<false>(n2[r], p[r], xx, cv[r], mu, eta, 1.f, alpha, gamma);
+        }
 #pragma unroll
         for (int k = 0; k < EPL; ++k) {
             s[r][k] = fmaf(alpha, s[r][k], gamma * xv[k]);

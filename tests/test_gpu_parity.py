@@ -596,3 +596,31 @@ def test_decode_workload_full_size_1000_steps(L):
     Sg = S[torch.from_numpy(bs).cuda(), torch.from_numpy(hs).cuda()].cpu().numpy()[:, None]
     assert s_err(Sg, So) <= TOL_F32
     np.testing.assert_allclose(np.linalg.norm(Sg, axis=-1), 1.0, atol=1e-5)
+
+
+@pytest.mark.parametrize("mode", ["sim", "dec"])
+@pytest.mark.parametrize("m,d", [(128, 128), (64, 64), (16, 32), (7, 16), (256, 64)])
+def test_step_many_heads(L, m, d, mode):
+    """320 heads, several waves of CTAs, for either objective; each step starts from
+    the oracle's state rounded to fp32. At m = 256 the reconstruction objective's
+    write direction becomes long and nearly parallel to some slots (|x|^2 ~ 1.5e4,
+    |x_perp|^2 ~ 4), which needs |x_perp|^2 summed directly rather than by
+    Pythagoras."""
+    w = LI.WORKLOADS["decode"].with_(m=m, d=d)
+    B, H, n = 40, 8, 3
+    So = LI.make_decode_state(w, B=B, H=H).astype(np.float64)
+    st = LI.make_decode_steps(w, n, B=B, H=H)
+    for k in range(n):
+        one = {key: st[key][k] for key in ("x", "q", "c", "mu")}
+        one["x_bits"] = st["x_bits"][k]
+        one["q_bits"] = st["q_bits"][k]
+        one["eta"] = None
+        t = dev_inputs(one)
+        S32 = So.astype(np.float32)
+        S = torch.from_numpy(S32.copy()).cuda()
+        y = L.step(S, t["x"], t["c"], t["q"], t["mu"], mode=mode)
+        yo, So, _ = oracle.step(S32, one["x"], one["c"], one["q"], one["mu"], mode=mode)
+        torch.cuda.synchronize()
+        L.device_status()
+        assert y_err(y.cpu().numpy()[:, None], yo[:, None]) <= TOL_F32
+        assert s_err(S.cpu().numpy(), So) <= TOL_F32
