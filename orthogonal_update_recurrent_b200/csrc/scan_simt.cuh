@@ -1,7 +1,8 @@
 // scan_simt.cuh -- CUDA-core scan of the Lattice recurrence, exact or chunked.
 //
-// One CTA per (b, h) sequence; the m slots live in registers (octet layout,
-// common.cuh), RQ slot quads per warp. Tokens are processed in order; inputs
+// One CTA per (b, h) sequence, or (SPLIT) a cluster of up to 4 CTAs per sequence
+// when the batch has fewer sequences than half the SMs; the slots live in registers
+// (octet layout, common.cuh), RQ slot quads per warp. Tokens are processed in order; inputs
 // are staged through shared memory TB tokens at a time (loaded into registers
 // one block ahead, stored after the current block's compute), and the
 // read-out partial sums of the warps are reduced across warps through shared
