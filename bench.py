@@ -118,8 +118,6 @@ CAPTURED_TRAFFIC = {
     ("chunk_split_kernel", "small_train"): 34.56e6,  # dram__bytes.sum.per_second x duration
     ("chunk_split_kernel", "long_ctx"): 676.05e6 + 498.46e6,
     ("chunk_tc_kernel", "mid_layer"): 550.62e6 + 240.43e6,
-    ("scan_simt_kernel<exact>", "small_train"): 34.48e6 + 0.12e6,
-    ("scan_bwd_kernel<chunked>", "small_train"): 70.75e6 + 57.51e6,
     ("step_kernel", "decode"): 545.32e6 + 482.93e6,
 }
 

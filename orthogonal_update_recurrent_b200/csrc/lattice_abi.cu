@@ -203,7 +203,7 @@ int bwd_split(int B, int H, int m) { return cluster_split(B, H, m); }
 template <int D, int RQ, bool CH, bool SPLIT>
 lattice_status launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
     constexpr int nt = bwd_threads(SPLIT);
-    const size_t smem = bwd_smem_bytes(D, a.spc, nt / 32);
+    const size_t smem = bwd_smem_bytes(D, a.spc, nt / 32, SPLIT);
     auto k = scan_bwd_kernel<D, RQ, CH, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e);

@@ -32,7 +32,8 @@
 
 namespace lattice {
 
-constexpr int kBwdTB = 8;  // tokens per staged block
+constexpr int kBwdTB = 8;        // tokens per staged block
+constexpr int kBwdTBSplit = 16;  // cluster kernels: longer blocks, half the cluster barriers
 
 struct BwdArgs {
     const void* x; bool x_bf16;
@@ -61,9 +62,10 @@ __host__ __device__ inline int bwd_record_floats(int D, int spc) { return (2 * D
 // Threads per CTA: 512 for one CTA per sequence, 256 in a cluster (<= 32 slots per CTA).
 __host__ __device__ constexpr int bwd_threads(bool split) { return split ? 256 : 512; }
 
-__host__ __device__ inline size_t bwd_smem_bytes(int D, int spc, int nw) {
-    return sizeof(float) * (2ull * kBwdTB * bwd_record_floats(D, spc) + (size_t)kBwdTB * nw * D +
-                            (size_t)kBwdTB * nw * 2 + 2ull * kBwdTB * (D + 2));
+__host__ __device__ inline size_t bwd_smem_bytes(int D, int spc, int nw, bool split) {
+    const size_t tb = split ? kBwdTBSplit : kBwdTB;
+    return sizeof(float) * (2ull * tb * bwd_record_floats(D, spc) + tb * nw * D + tb * nw * 2 +
+                            2ull * tb * (D + 2));
 }
 
 // 1/sqrt(x) for x > 0: the hardware approximation and one Newton step.
@@ -195,9 +197,10 @@ __global__ void __launch_bounds__(bwd_threads(SPLIT)) scan_bwd_kernel(BwdArgs a)
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
     constexpr int NT = bwd_threads(SPLIT), NW = NT / 32;
+    constexpr int TB = SPLIT ? kBwdTBSplit : kBwdTB;  // tokens per staged block
     // staging registers per thread: one block of the largest record this instantiation takes
     constexpr int kMaxSpc = SPLIT ? 32 : 64 * RQ;
-    constexpr int KS = (kBwdTB * ((2 * D + 2 * kMaxSpc + 2 + 3) & ~3) + NT - 1) / NT;
+    constexpr int KS = (TB * ((2 * D + 2 * kMaxSpc + 2 + 3) & ~3) + NT - 1) / NT;
     // a cluster CTA has one warp per scheduler, so the next tape entry is loaded one
     // token ahead; with 16 warps the others hide that latency and the registers are short
     constexpr bool kPrefetchTape = SPLIT;
@@ -209,9 +212,9 @@ __global__ void __launch_bounds__(bwd_threads(SPLIT)) scan_bwd_kernel(BwdArgs a)
     const int m = a.m, T = a.T, H = a.H, L = a.seg, SPC = a.spc;
     const int R = bwd_record_floats(D, SPC);
     float* rec_buf = smem;                                   // [2][TB][R]
-    float* dx_buf = smem + 2 * kBwdTB * R;                   // [TB][NW][D]
-    float* sc_buf = dx_buf + (size_t)kBwdTB * NW * D;        // [TB][NW][2]: dmu, deta partials
-    float* cta_part = sc_buf + (size_t)kBwdTB * NW * 2;      // [2][TB][D + 2]: this CTA's sums (G > 1)
+    float* dx_buf = smem + 2 * TB * R;                   // [TB][NW][D]
+    float* sc_buf = dx_buf + (size_t)TB * NW * D;        // [TB][NW][2]: dmu, deta partials
+    float* cta_part = sc_buf + (size_t)TB * NW * 2;      // [2][TB][D + 2]: this CTA's sums (G > 1)
     const int nseg = T > 0 ? (T + L - 1) / L : 1;
     float* ckpt = a.ws + ((size_t)bh * G + crank) * bwd_ws_floats_per_seq(T, SPC, D, L);  // [nseg-1][SPC][D]
     float* tape = ckpt + (size_t)(nseg - 1) * SPC * D;                                     // [L][SPC][D]
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(bwd_threads(SPLIT)) scan_bwd_kernel(BwdArgs a)
         }
     };
     auto put = [&](int buf, int n) {
-        float* dst = rec_buf + (size_t)buf * kBwdTB * R;
+        float* dst = rec_buf + (size_t)buf * TB * R;
 #pragma unroll
         for (int u = 0; u < KS; ++u) {
             const int idx = tid + u * NT;
@@ -332,17 +335,17 @@ __global__ void __launch_bounds__(bwd_threads(SPLIT)) scan_bwd_kernel(BwdArgs a)
     // store the state before each token at tape_base[t - t_begin]. ckpts: store the
     // state before each segment start t (t % L == 0, 0 < t < t_end) as a checkpoint.
     auto forward = [&](int t_begin, int t_end, float* tape_base, bool ckpts) {
-        const int nblk = (t_end - t_begin + kBwdTB - 1) / kBwdTB;
+        const int nblk = (t_end - t_begin + TB - 1) / TB;
         if (nblk == 0) return;
         __syncthreads();  // the record buffers are free
-        fetch(t_begin, min(kBwdTB, t_end - t_begin), false);
-        put(0, min(kBwdTB, t_end - t_begin));
+        fetch(t_begin, min(TB, t_end - t_begin), false);
+        put(0, min(TB, t_end - t_begin));
         __syncthreads();
         for (int k = 0; k < nblk; ++k) {
-            const int t0 = t_begin + k * kBwdTB, n = min(kBwdTB, t_end - t0);
-            const int t1 = t0 + kBwdTB, n1 = k + 1 < nblk ? min(kBwdTB, t_end - t1) : 0;
+            const int t0 = t_begin + k * TB, n = min(TB, t_end - t0);
+            const int t1 = t0 + TB, n1 = k + 1 < nblk ? min(TB, t_end - t1) : 0;
             if (n1 > 0) fetch(t1, n1, false);
-            const float* rb = rec_buf + (size_t)(k & 1) * kBwdTB * R;
+            const float* rb = rec_buf + (size_t)(k & 1) * TB * R;
             for (int tok = 0; tok < n; ++tok) {
                 const int t = t0 + tok;
                 if (ckpts && t > 0 && t % L == 0) store_scratch(ckpt + (size_t)(t / L - 1) * st_sz, s);
@@ -392,20 +395,20 @@ __global__ void __launch_bounds__(bwd_threads(SPLIT)) scan_bwd_kernel(BwdArgs a)
             if (te > ts) load_scratch(tape + (size_t)(te - 1 - ts) * st_sz, spn);
         }
         // 2b. adjoint over the segment's tokens, last to first (blocks from the end)
-        const int nblk = (te - ts + kBwdTB - 1) / kBwdTB;
+        const int nblk = (te - ts + TB - 1) / TB;
         if (nblk > 0) {
             __syncthreads();  // the record buffers are free
-            const int f0 = max(ts, te - kBwdTB);
+            const int f0 = max(ts, te - TB);
             fetch(f0, te - f0, true);
             put(0, te - f0);
             __syncthreads();
         }
         for (int kb = 0; kb < nblk; ++kb) {
-            const int tb_end = te - kb * kBwdTB;
-            const int t0 = max(ts, tb_end - kBwdTB), n = tb_end - t0;
-            const int t0n = max(ts, t0 - kBwdTB), n1 = kb + 1 < nblk ? t0 - t0n : 0;
+            const int tb_end = te - kb * TB;
+            const int t0 = max(ts, tb_end - TB), n = tb_end - t0;
+            const int t0n = max(ts, t0 - TB), n1 = kb + 1 < nblk ? t0 - t0n : 0;
             if (n1 > 0) fetch(t0n, n1, true);
-            const float* rbuf = rec_buf + (size_t)(kb & 1) * kBwdTB * R;
+            const float* rbuf = rec_buf + (size_t)(kb & 1) * TB * R;
             for (int tok = n - 1; tok >= 0; --tok) {
                 const int t = t0 + tok;
                 const float* rec = rbuf + tok * R;
@@ -542,7 +545,7 @@ __global__ void __launch_bounds__(bwd_threads(SPLIT)) scan_bwd_kernel(BwdArgs a)
                 }
             } else {
                 // this CTA's sums over its warps (fixed order) ...
-                float* part = cta_part + (size_t)(pbuf & 1) * kBwdTB * (D + 2);
+                float* part = cta_part + (size_t)(pbuf & 1) * TB * (D + 2);
                 for (int idx = tid; idx < n * (D + 2); idx += NT) {
                     const int tok = idx / (D + 2), k = idx - tok * (D + 2);
                     float v = 0.f;

@@ -19,7 +19,8 @@
 
 namespace lattice {
 
-constexpr int kScanTB = 8;      // tokens per staged block
+constexpr int kScanTB = 8;       // tokens per staged block
+constexpr int kScanTBSplit = 16;  // split kernels: longer blocks, half the cluster barriers
 constexpr int kMaxM = 256;
 
 struct ScanArgs {
@@ -46,8 +47,9 @@ __host__ __device__ inline int scan_record_floats(int D, int m) { return (D + 2 
 // split kernels add ypart[2][TB][D] (the CTA's read-out partials for the cluster sum).
 template <int D>
 __host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec, bool split = false) {
-    return sizeof(float) * (2ull * kScanTB * scan_record_floats(D, m) + 2ull * kScanTB * nw * D +
-                            (dec ? 2ull * nw * D : 0ull) + (split ? 2ull * kScanTB * D : 0ull));
+    const size_t tb = split ? kScanTBSplit : kScanTB;
+    return sizeof(float) * (2ull * tb * scan_record_floats(D, m) + 2ull * tb * nw * D +
+                            (dec ? 2ull * nw * D : 0ull) + (split ? 2ull * tb * D : 0ull));
 }
 
 // Cluster barrier and a load from a peer CTA's shared memory (split kernels).
@@ -78,6 +80,7 @@ __device__ __forceinline__ float scan_ld_peer(const float* local_ptr, uint32_t r
 template <int D, int RQ, bool CHUNKED, bool DEC, bool LIN1 = false, bool SPLIT = false>
 __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a) {
     static_assert(!(SPLIT && (DEC || RQ != 1)), "split kernels: similarity objective, one slot per octet");
+    constexpr int TB = SPLIT ? kScanTBSplit : kScanTB;  // tokens per staged block
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
     extern __shared__ __align__(16) float smem[];
@@ -91,8 +94,8 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
     const int m = a.m, T = a.T, H = a.H;
     const int per_tok = scan_record_floats(D, m);  // x | q | c | mu | eta | pad
     float* in_buf = smem;
-    float* ybuf = smem + 2 * kScanTB * per_tok;
-    float* rbuf = ybuf + 2 * kScanTB * NW * D;  // DEC only
+    float* ybuf = smem + 2 * TB * per_tok;
+    float* rbuf = ybuf + 2 * TB * NW * D;  // DEC only
     float* ypart = rbuf + (DEC ? 2 * NW * D : 0);  // SPLIT only: [2][TB][D]
 
     // ---- load the initial state into registers
@@ -116,15 +119,16 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
     }
 
     // ---- staging helpers
-    const int n_blocks = (T + kScanTB - 1) / kScanTB;
-    const int stage_total = kScanTB * per_tok;
+    const int n_blocks = (T + TB - 1) / TB;
+    const int stage_total = TB * per_tok;
     // per-thread staging registers: the host launches NW >= 4 warps when RQ == 1, NW = 16
     // otherwise, and 8 warps for split kernels
     constexpr int kMinThreads = SPLIT ? 256 : (RQ == 1 ? 128 : 512);
-    constexpr int kStg = (kScanTB * (D + 2 * kMaxM + 4) + kMinThreads - 1) / kMinThreads;
+    constexpr int kStgM = SPLIT ? 128 : kMaxM;  // split kernels: m <= 4 CTAs x 32 slots
+    constexpr int kStg = (TB * (D + 2 * kStgM + 4) + kMinThreads - 1) / kMinThreads;
     float stg[kStg];
     auto stage_load = [&](int blk) {
-        const int t0 = blk * kScanTB;
+        const int t0 = blk * TB;
 #pragma unroll
         for (int u = 0; u < kStg; ++u) {
             int idx = tid + u * NT;
@@ -156,8 +160,8 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
     // Read-out of block fb: fixed-order sum over the warps (and, for split kernels,
     // over the cluster's CTAs, each CTA writing a share of the block's entries).
     auto flush_y = [&](int fb) {
-        const int pt0 = fb * kScanTB, ntok = min(kScanTB, T - pt0);
-        const float* yb = ybuf + (size_t)(fb & 1) * kScanTB * NW * D;
+        const int pt0 = fb * TB, ntok = min(TB, T - pt0);
+        const float* yb = ybuf + (size_t)(fb & 1) * TB * NW * D;
         if constexpr (!SPLIT) {
             for (int idx = tid; idx < ntok * D; idx += NT) {
                 int tok = idx / D, k = idx - tok * D;
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
         } else {
             // the partial buffers alternate by block; the next flush's cluster barrier
             // orders their reuse after every peer has read them
-            float* part = ypart + (size_t)(fb & 1) * kScanTB * D;
+            float* part = ypart + (size_t)(fb & 1) * TB * D;
             for (int idx = tid; idx < ntok * D; idx += NT) {
                 int tok = idx / D, k = idx - tok * D;
                 float acc = 0.f;
@@ -197,14 +201,14 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
 
     for (int blk = 0; blk < n_blocks; ++blk) {
         const int buf = blk & 1;
-        const int t0 = blk * kScanTB;
+        const int t0 = blk * TB;
         // flush the previous block's read-out
         if (blk > 0) flush_y(blk - 1);
         if (blk + 1 < n_blocks) stage_load(blk + 1);
 
         const float* inb = in_buf + buf * stage_total;
-        float* yb = ybuf + (size_t)buf * kScanTB * NW * D;
-        const int ntok = min(kScanTB, T - t0);
+        float* yb = ybuf + (size_t)buf * TB * NW * D;
+        const int ntok = min(TB, T - t0);
         for (int tok = 0; tok < ntok; ++tok) {
             const int t = t0 + tok;
             const float* rec = inb + tok * per_tok;
