@@ -118,6 +118,8 @@ CAPTURED_TRAFFIC = {
     ("chunk_split_kernel", "small_train"): 34.56e6,  # dram__bytes.sum.per_second x duration
     ("chunk_split_kernel", "long_ctx"): 676.05e6 + 498.46e6,
     ("chunk_tc_kernel", "mid_layer"): 550.62e6 + 240.43e6,
+    ("scan_simt_kernel<exact>", "small_train"): 34.43e6 + 0.02e6,
+    ("scan_bwd_kernel<chunked>", "small_train"): 71.00e6 + 57.72e6,
     ("step_kernel", "decode"): 545.32e6 + 482.93e6,
 }
 
