@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(512) step_kernel(StepArgs a) {
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
     __shared__ __align__(16) float ysm[16][D];
+    __shared__ __align__(16) float esm[DEC ? D : 1];  // DEC: the token's write direction
     const int NW = blockDim.x >> 5;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j = lane & 7, oct = lane >> 3;
@@ -76,13 +77,15 @@ __global__ void __launch_bounds__(512) step_kernel(StepArgs a) {
             for (int k = 0; k < EPL; ++k) ysm[warp][O::pos(j, k)] = rp[k];
         }
         __syncthreads();
-#pragma unroll
-        for (int k = 0; k < EPL; ++k) {
+        // one thread per element sums the warps (fixed order) and forms x - sum ...
+        for (int e = tid; e < D; e += blockDim.x) {
             float acc = 0.f;
-            for (int w = 0; w < NW; ++w) acc += ysm[w][O::pos(j, k)];
-            xv[k] -= acc;
+            for (int w = 0; w < NW; ++w) acc += ysm[w][e];
+            esm[e] = acc;
         }
-        __syncthreads();  // ysm is reused for the read-out
+        __syncthreads();  // ... which every lane then reads (ysm is free for the read-out)
+#pragma unroll
+        for (int k = 0; k < EPL; ++k) xv[k] -= esm[O::pos(j, k)];
     }
     float xx = 0.f;
 #pragma unroll
