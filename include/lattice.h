@@ -41,7 +41,8 @@
  *
  * Ownership and execution: every pointer is caller-owned DEVICE memory. The
  * library allocates nothing and keeps no state besides one device status
- * word. Every call is asynchronous on `stream` (a cudaStream_t passed as
+ * word (and the static scratch array of lattice_scan_bwd_noalloc, described
+ * there). Every call is asynchronous on `stream` (a cudaStream_t passed as
  * void*, NULL = the legacy default stream) and returns after the launch.
  *
  * Errors: arguments are checked on the host before anything is launched; a
@@ -50,7 +51,8 @@
  * Device-side waits are bounded: a kernel that gives up sets the status word
  * and returns; lattice_get_device_status() reports it as LATTICE_ERR_TIMEOUT.
  *
- * Supported sizes: d in {16, 32, 64, 128}; 1 <= m <= 256; B, H >= 1; T >= 0.
+ * Supported sizes: d in {16, 32, 64, 128}; 1 <= m <= 256 (m <= 128 for the
+ * backward pass); B, H >= 1; T >= 0.
  * The tensor-core chunked kernel serves C = 64, m in {64, 128},
  * d in {64, 128} with bf16 x and q; other chunked shapes run a CUDA-core
  * kernel of the same definition.

@@ -111,6 +111,10 @@ def test_backward_workspace_and_argument_checks(lib):
     assert ws(1, 200, 1, 4, 16, 24, 0) == (2 + 72) * 4 * 16 * 4
     assert ws(1, 200, 1, 4, 16, 128, 0) == (1 + 128) * 4 * 16 * 4
     assert ws(1, 200, 1, 4, 16, 4, 10) == 0      # segment not a multiple of the chunk
+    # one sequence on a 148-SM device: a cluster of G CTAs, each with ceil(m/G) scratch rows
+    assert ws(1, 200, 1, 64, 16, 1, 0) == 4 * (3 + 64) * 16 * 16 * 4     # G = 4, 16 rows each
+    assert ws(1, 200, 1, 5, 16, 1, 0) == 2 * (3 + 64) * 3 * 16 * 4       # G = 2, 3 rows each (one unused)
+    assert ws(100, 200, 1, 64, 16, 1, 0) == 100 * (3 + 64) * 64 * 16 * 4  # batch fills the SMs: G = 1
     assert ws(1, 200, 1, 129, 16, 1, 0) == 0     # m > 128
     # every case below fails validation before any CUDA call
     assert _bwd(lib, wsb=64 * 4 * 16 * 4 - 4) == L.ERR_INVALID_ARG   # workspace too small
