@@ -1,16 +1,19 @@
 #!/usr/bin/env python
 """Benchmark of the Lattice compression-layer state recurrence on B200.
 
-A step is one lattice_scan_fwd over one batch of the small training shape
-(B=4, H=8, T=2048, m=d=64, chunk 64, bf16 x/q, fp32 state): the whole hot path
-(projection, orthogonal write, forget gate, unit-sphere projection, read-out,
-chunk state carry). Inputs are resident in HBM before the timed region; the L2
-is flushed (a 256 MiB write) between timed steps because this workload's
-inputs fit in L2. Each step is timed with CUDA events on the launching stream.
+A step is one lattice_scan_fwd over one batch of the long-context workload
+(B=1, H=16, T=65536, m=64, d=128, chunk 64, bf16 x/q, fp32 state carried over
+1024 chunks): the whole hot path (projection, orthogonal write, forget gate,
+unit-sphere projection, read-out, chunk state carry). It is the largest of the
+single-GPU workloads (1.05 M token-heads, 1.2 GB of algorithmic traffic).
+Inputs are resident in HBM before the timed region; they exceed the L2, which is
+also flushed (a 256 MiB write) between timed steps. Each step is timed with CUDA
+events on the launching stream.
 
-The same JSON line also reports, as context, the mid-size and long-context
-scans, the exact recurrence, and the decode step (1000 consecutive steps of
-B=256, H=32, m=d=128), each with its roofline fraction.
+The same JSON line also reports, under "extra", the small training shape and the
+mid-size layer (each with its own roofline record), the exact recurrence, the
+chunk-form variants, the backward pass and the decode step (1000 consecutive
+steps of B=256, H=32, m=d=128).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -37,7 +40,7 @@ import numpy as np
 import lattice_inputs as LI
 
 METRIC = "Lattice layer fwd tokens/s (1 B200) + % of roofline; decode step GB/s"
-HEADLINE = "small_train"
+HEADLINE = "long_ctx"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
@@ -112,16 +115,55 @@ def job_tokens_per_s(world: int, w: LI.Workload, ms_per_step: float) -> float:
     return world * w.B * w.T / (ms_per_step * 1e-3)
 
 
-# DRAM bytes (read + write) per launch, from one `ncu --set full` capture of each kernel on
-# each workload (the profile summaries keep the commands). None where no capture exists.
+def scan_config(w: LI.Workload, world: int) -> dict:
+    """The `config` record of a scan line (both arms print the same one)."""
+    big = scan_alg_bytes(w) > 2 * (126 << 20)
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "m": w.m, "d": w.d, "chunk": w.chunk,
+            "x_q_dtype": w.x_dtype, "state_dtype": "f32",
+            "l2": ("inputs exceed the L2; also flushed between timed steps (256 MiB write)" if big
+                   else "flushed between timed steps (256 MiB write)"),
+            "parallelism": f"independent batches per GPU x{world}"}
+
+
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel on each
+# workload. Each entry names the profile summary that holds the capture's command and
+# figures, and the SHA-256 (first 12 hex digits) of the kernel's source file at the
+# time of the capture: traffic_for() reports None once that file has changed, since
+# the counters then describe a kernel that no longer exists.
 CAPTURED_TRAFFIC = {
-    ("chunk_split_kernel", "small_train"): 34.56e6,  # dram__bytes.sum.per_second x duration
-    ("chunk_split_kernel", "long_ctx"): 676.05e6 + 498.46e6,
-    ("chunk_tc_kernel", "mid_layer"): 550.62e6 + 240.43e6,
-    ("scan_simt_kernel<exact>", "small_train"): 34.43e6 + 0.02e6,
-    ("scan_bwd_kernel<chunked>", "small_train"): 71.00e6 + 57.72e6,
-    ("step_kernel", "decode"): 545.32e6 + 482.93e6,
+    ("chunk_split_kernel", "small_train"): dict(bytes=34.56e6, profile="profiles/chunk_split_kernel_full.md",
+                                                source="csrc/chunk_split.cuh", sha="047d8e41962f"),
+    ("chunk_split_kernel", "long_ctx"): dict(bytes=676.05e6 + 498.46e6, profile="profiles/chunk_split_kernel_full.md",
+                                             source="csrc/chunk_split.cuh", sha="047d8e41962f"),
+    # (chunk_tc.cuh since changed only by moving its wait helpers, verbatim, into waits.cuh)
+    ("chunk_tc_kernel", "mid_layer"): dict(bytes=550.62e6 + 240.43e6, profile="profiles/chunk_tc_kernel_full.md",
+                                           source="csrc/chunk_tc.cuh", sha="9b76f603cace"),
+    ("scan_simt_kernel<exact>", "small_train"): dict(bytes=34.43e6 + 0.02e6,
+                                                     profile="profiles/scan_simt_kernel_exact_small_train.md",
+                                                     source="csrc/scan_simt.cuh", sha="b1b556e2f5cf"),
+    ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.00e6 + 57.72e6,
+                                                      profile="profiles/scan_bwd_kernel_small_train.md",
+                                                      source="csrc/scan_bwd.cuh", sha="c2830cd3eeeb"),
+    # captured before the last change of step.cuh: reported as None until re-captured
+    ("step_kernel", "decode"): dict(bytes=545.32e6 + 482.93e6, profile="profiles/step_kernel_decode.md",
+                                    source="csrc/step.cuh", sha=None),
 }
+
+
+def source_sha(rel: str) -> str:
+    import hashlib
+    p = os.path.join(ROOT, "orthogonal_update_recurrent_b200", rel)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:12]
+
+
+def traffic_for(kernel: str, workload: str):
+    """Captured DRAM bytes per launch of `kernel` on `workload`, or None when there is
+    no capture or the kernel's source changed since it was taken."""
+    e = CAPTURED_TRAFFIC.get((kernel, workload))
+    if e is None or e["sha"] is None or source_sha(e["source"]) != e["sha"]:
+        return None
+    return e["bytes"]
 
 
 # -------------------------------------------------------------------- clocks
@@ -343,11 +385,21 @@ def time_decode(torch, L, w, n_steps, ring, device, mode="sim"):
 
 # ---------------------------------------------------------------- CPU oracle
 
+def oracle_sample_tokens(w: LI.Workload) -> int:
+    """Tokens per sequence of one bounded oracle sample: the whole sequence for the
+    shorter workloads, the first 8192 tokens (128 chunks) of every head for longer
+    ones. The oracle's cost per token is the same all along a sequence, so tokens/s
+    over the sample is the workload's rate."""
+    return min(w.T, 8192)
+
+
 def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 12.0, max_reps: int = 10000):
-    """The fp64 oracle, as it stands, on the host cores: whole workload passes
-    repeated until about min_seconds of CPU work. Returns (tokens/s, cores, sample)."""
+    """The fp64 oracle, as it stands, on the host cores: passes over a bounded sample of
+    the workload (every sequence, oracle_sample_tokens tokens each) repeated until about
+    min_seconds of CPU work. Returns (tokens/s, cores, sample)."""
     import oracle
-    inp = LI.make_inputs(w)
+    Ts = oracle_sample_tokens(w)
+    inp = LI.make_inputs(w, T=Ts)
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
     reps = 0
@@ -357,29 +409,33 @@ def oracle_baseline(w: LI.Workload, chunk: int, min_seconds: float = 12.0, max_r
         el = time.perf_counter() - t0
         if el >= min_seconds or reps >= max_reps:
             break
-    tok = w.B * w.T * reps
-    sample = (f"{reps} full pass(es) of {w.name} (B={w.B},H={w.H},T={w.T},m={w.m},d={w.d}), "
+    tok = w.B * Ts * reps
+    what = "full pass(es)" if Ts == w.T else f"pass(es) over the first {Ts} of {w.T} tokens"
+    sample = (f"{reps} {what} of {w.name} (B={w.B},H={w.H},T={w.T},m={w.m},d={w.d}), "
               f"{'exact' if chunk == 1 else f'chunked C={chunk}'}, fp64 oracle, {el:.1f} s")
     return tok / el, cores, sample
 
 
 def oracle_legs(w: LI.Workload, seconds: float = 3.0) -> dict:
-    """Further oracle timings on the host: the exact recurrence on all cores, the
-    chunked form on one thread, and decode steps of the decode workload (3 steps of
-    the full 512 MiB state, per step)."""
+    """Further oracle timings on the host: the exact recurrence on all cores and the
+    chunked form on one thread (each over the bounded sample, the one-thread leg over
+    its first 1024 tokens), and decode steps of the decode workload (3 steps of the full
+    512 MiB state, per step)."""
     import oracle
-    inp = LI.make_inputs(w)
     cores = len(os.sched_getaffinity(0))
 
-    def rate(chunk, threads):
+    def rate(chunk, threads, T):
+        inp = LI.make_inputs(w, T=T)
         t0, reps = time.perf_counter(), 0
         while True:
             oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=chunk, nthreads=threads)
             reps += 1
             el = time.perf_counter() - t0
             if el >= seconds:
-                return w.B * w.T * reps / el
-    out = {"exact_tokens_per_s": rate(1, cores), "chunked_tokens_per_s_1_thread": rate(w.chunk, 1)}
+                return w.B * T * reps / el
+    Ts = oracle_sample_tokens(w)
+    out = {"exact_tokens_per_s": rate(1, cores, Ts),
+           "chunked_tokens_per_s_1_thread": rate(w.chunk, 1, min(Ts, 1024))}
     wd = LI.WORKLOADS["decode"]
     S = LI.make_decode_state(wd).astype(np.float64)
     st = LI.make_decode_steps(wd, 3)
@@ -392,6 +448,36 @@ def oracle_legs(w: LI.Workload, seconds: float = 3.0) -> dict:
 
 
 # ---------------------------------------------------------------------- main
+
+def kernel_name(L, w: LI.Workload, chunk: int) -> str:
+    """The kernel lattice_scan_fwd's automatic choice runs for this workload."""
+    kimpl = L.chunk_impl(w.B, w.H, w.m, w.d, chunk)
+    return {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(
+        kimpl, "scan_simt_kernel<chunked>" if chunk > 1 else "scan_simt_kernel<exact>")
+
+
+def scan_roofline(L, w: LI.Workload, traffic_key: str, kern_ms: float, pk: dict, pk_src: str) -> dict:
+    """Roofline record of one scan launch of `w` that took kern_ms (CUDA events):
+    algorithmic HBM bytes / time against the measured copy bandwidth, and for the
+    tensor-core kernels the algorithmic MMA flops / time against the bf16 peak."""
+    kname = kernel_name(L, w, w.chunk)
+    alg_b = scan_alg_bytes(w)
+    achieved = alg_b / (kern_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(kname, traffic_key),
+            "kernel": kname, "ms_per_launch": kern_ms,
+            "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"}
+    t_roof_ms = 1e3 * alg_b / (pk["hbm_gbs"] * 1e9)
+    if kname.startswith("chunk_"):
+        fl = chunk_mma_flops(w, w.chunk)
+        roof["tensor"] = {"achieved_tflops": fl / (kern_ms * 1e-3) / 1e12,
+                          "peak_tflops": pk["bf16_tflops"],
+                          "frac": fl / (kern_ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                          "flops_per_launch": fl}
+        t_roof_ms = max(t_roof_ms, 1e3 * fl / (pk["bf16_tflops"] * 1e12))
+    roof["frac_of_binding_roofline"] = t_roof_ms / kern_ms
+    return roof
+
 
 def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
     """--pass step: one step is one decode token for every (b,h) of the decode workload
@@ -418,7 +504,7 @@ def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
                        "l2": "state (512 MiB) and input ring exceed L2",
                        "parallelism": f"independent batches per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": gbps, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbps / pk["hbm_gbs"], "traffic": CAPTURED_TRAFFIC.get(("step_kernel", "decode")),
+                         "frac": gbps / pk["hbm_gbs"], "traffic": traffic_for("step_kernel", "decode"),
                          "kernel": "step_kernel",
                          "alg_bytes_per_launch": sb, "peak_source": f"{pk_src} (burst copy)"},
             "gpu_launches": n}
@@ -457,7 +543,7 @@ def bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush,
                        "l2": "flushed between timed steps (256 MiB write)",
                        "parallelism": f"independent batches per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": CAPTURED_TRAFFIC.get((kname, w0.name)),
+                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(kname, w0.name),
                          "kernel": kname,
                          "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"},
             "gpu_launches": args.steps}
@@ -478,7 +564,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--workload", default=HEADLINE, choices=["small_train", "mid_layer", "long_ctx"],
-                    help="chunked workload of the timed step (default: the small training shape)")
+                    help="chunked workload of the timed step (default: the long-context workload)")
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "step"],
                     help="bwd: time the backward pass (lattice_scan_bwd) of the workload instead; "
                          "step: time the decode step (lattice_step) on the decode workload")
@@ -500,7 +586,8 @@ def main():
             return 0
         steps = max(1, args.steps)
         import oracle
-        inp = LI.make_inputs(w)
+        Ts = oracle_sample_tokens(w)
+        inp = LI.make_inputs(w, T=Ts)
         cores = len(os.sched_getaffinity(0))
         for _ in range(args.warmup):  # untimed passes
             oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=w.chunk, nthreads=cores)
@@ -508,15 +595,15 @@ def main():
         for _ in range(steps):
             oracle.scan(inp["x"], inp["c"], inp["q"], inp["mu"], inp["S0"], chunk=w.chunk, nthreads=cores)
         el = time.perf_counter() - t0
-        v = w.B * w.T * steps / el
+        v = w.B * Ts * steps / el
+        what = "one full pass" if Ts == w.T else f"one pass over the first {Ts} of {w.T} tokens of every sequence"
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
                 "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic",
-                "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "m": w.m, "d": w.d,
-                           "chunk": w.chunk},
+                "data": "synthetic", "config": scan_config(w, args.gpus),
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                 "sample": f"one full pass of {w.name} per step, chunked C={w.chunk}, "
+                                 "sample": f"{what} of {w.name} per step, "
+                                           f"{'exact' if w.chunk == 1 else f'chunked C={w.chunk}'}, "
                                            f"fp64 C oracle on {cores} threads"},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -560,35 +647,13 @@ def main():
     value = job_tokens_per_s(world, w, ms)
 
     # roofline of the (single) kernel of the step
-    kimpl = L.chunk_impl(w.B, w.H, w.m, w.d, w.chunk)
-    tc = kimpl.startswith("tcgen05")
-    alg_b = scan_alg_bytes(w)
-    kern_ms = statistics.mean(times)
-    achieved = alg_b / (kern_ms * 1e-3) / 1e9
-    kname = {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(
-        kimpl, "scan_simt_kernel<chunked>" if w.chunk > 1 else "scan_simt_kernel<exact>")
-    roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / pk["hbm_gbs"], "traffic": CAPTURED_TRAFFIC.get((kname, w0.name)),
-            "kernel": kname,
-            "alg_bytes_per_launch": alg_b, "peak_source": f"{pk_src} (burst copy)"}
-    if tc:
-        fl = chunk_mma_flops(w, w.chunk)
-        roof["tensor"] = {"achieved_tflops": fl / (kern_ms * 1e-3) / 1e12,
-                          "peak_tflops": pk["bf16_tflops"],
-                          "frac": fl / (kern_ms * 1e-3) / 1e12 / pk["bf16_tflops"],
-                          "flops_per_launch": fl}
-    t_roof_ms = 1e3 * max(alg_b / (pk["hbm_gbs"] * 1e9),
-                          (chunk_mma_flops(w, w.chunk) / (pk["bf16_tflops"] * 1e12)) if tc else 0.0)
-    roof["frac_of_binding_roofline"] = t_roof_ms / kern_ms
+    roof = scan_roofline(L, w, w0.name, statistics.mean(times), pk, pk_src)
+    tc = "tensor" in roof
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if tc else "f32", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "m": w.m, "d": w.d,
-                       "chunk": w.chunk, "x_q_dtype": "bf16", "state_dtype": "f32",
-                       "l2": "flushed between timed steps (256 MiB write)",
-                       "parallelism": f"independent batches per GPU x{world}"},
-            "roofline": roof, "gpu_launches": args.steps}
+            "config": scan_config(w, world), "roofline": roof, "gpu_launches": args.steps}
     cs = clk.summary()
     if cs is not None:
         line["clocks"] = cs
@@ -604,77 +669,71 @@ def main():
                            "pipelined": "copy-in / scan / copy-out on three streams, two buffer sets"}
         extra = {}
         if not args.no_extra:
-            # exact recurrence on the timed workload
-            te = time_scan(torch, L, t, 1, 5, 3, flush=flush)
-            extra[f"{w.name}_exact"] = {"ms": statistics.mean(te),
+            # the exact recurrence on the timed workload
+            te = time_scan(torch, L, t, 1, 3, 3, flush=flush)
+            extra[f"{w.name}_exact"] = {"ms": statistics.mean(te), "kernel": kernel_name(L, w, 1),
                                         "tokens_per_s": w.B * w.T / (statistics.mean(te) * 1e-3)}
-            # the reconstruction objective (CUDA-core kernels), exact and chunked; the
-            # chunked form takes intensities sigmoid(N(-4,1)), with which it stays bounded
-            td = time_scan(torch, L, t, 1, 5, 3, flush=flush, mode="dec")
-            extra[f"{w.name}_dec_exact"] = {"ms": statistics.mean(td),
-                                            "tokens_per_s": w.B * w.T / (statistics.mean(td) * 1e-3),
-                                            "kernel": "scan_simt_kernel<exact, dec>"}
-            wdc = w.with_(c_loc=-4.0)
-            tdc = _dev_inputs(torch, LI.make_inputs(wdc), device)
-            td = time_scan(torch, L, tdc, w.chunk, 5, 3, flush=flush, mode="dec")
-            extra[f"{w.name}_dec_chunked"] = {"ms": statistics.mean(td),
-                                              "tokens_per_s": w.B * w.T / (statistics.mean(td) * 1e-3),
-                                              "kernel": "scan_simt_kernel<chunked, dec>",
-                                              "inputs": "c = sigmoid(N(-4,1))"}
-            del tdc
-            # the normalisation ablation of Appendix C (CUDA-core kernel)
-            tn = time_scan(torch, L, t, w.chunk, 5, 3, flush=flush, norm="chunk")
-            extra[f"{w.name}_chunk_norm"] = {"ms": statistics.mean(tn),
-                                             "tokens_per_s": w.B * w.T / (statistics.mean(tn) * 1e-3),
-                                             "kernel": "scan_simt_kernel<chunked, norm at chunk ends>"}
-            # the other chunk linearisation (recurrence_linear1, CUDA-core kernel)
-            tl = time_scan(torch, L, t, w.chunk, 5, 3, flush=flush, lin=1)
-            extra[f"{w.name}_lin1_chunked"] = {"ms": statistics.mean(tl),
-                                               "tokens_per_s": w.B * w.T / (statistics.mean(tl) * 1e-3),
-                                               "kernel": "scan_simt_kernel<chunked, recurrence_linear1>"}
-            # backward pass (CUDA-core kernel), chunked and exact
-            for cb, tag in ((w.chunk, "chunked"), (1, "exact")):
-                tb = time_bwd(torch, L, t, cb, 3, 2, flush=flush)
-                extra[f"{w.name}_bwd_{tag}"] = {"ms": statistics.mean(tb),
-                                                "tokens_per_s": w.B * w.T / (statistics.mean(tb) * 1e-3),
-                                                "kernel": f"scan_bwd_kernel<{tag}>",
-                                                "allocations": "outputs per call; workspace once"}
             del t
-            for name in [n for n in ("mid_layer", "long_ctx") if n != w.name]:
+            torch.cuda.empty_cache()
+            # the other chunked workloads, each with its own roofline record
+            for name in [n for n in ("small_train", "mid_layer", "long_ctx") if n != w.name]:
                 wn = LI.WORKLOADS[name]
                 inn = LI.make_inputs(wn)
                 tn = _dev_inputs(torch, inn, device)
                 del inn
-                tch = time_scan(torch, L, tn, wn.chunk, 5, 3)
-                ab = scan_alg_bytes(wn)
+                tch = time_scan(torch, L, tn, wn.chunk, 10, 3, flush=flush)
                 kms = statistics.mean(tch)
-                ent = {"chunk_ms": kms, "tokens_per_s": wn.B * wn.T / (kms * 1e-3),
-                       "hbm_gbs": ab / (kms * 1e-3) / 1e9, "hbm_frac": ab / (kms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                       "alg_bytes": ab}
-                fl = chunk_mma_flops(wn, wn.chunk)
-                kn = {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(
-                    L.chunk_impl(wn.B, wn.H, wn.m, wn.d, wn.chunk), "scan_simt_kernel<chunked>")
-                ent["kernel"] = kn
-                ent["traffic"] = CAPTURED_TRAFFIC.get((kn, name))
-                ent["tensor_tflops"] = fl / (kms * 1e-3) / 1e12
-                ent["frac_of_binding_roofline"] = 1e3 * max(ab / (pk["hbm_gbs"] * 1e9),
-                                                            fl / (pk["bf16_tflops"] * 1e12)) / kms
-                tex = time_scan(torch, L, tn, 1, 3, 3)
+                ent = {"ms": kms, "tokens_per_s": wn.B * wn.T / (kms * 1e-3),
+                       "roofline": scan_roofline(L, wn, name, kms, pk, pk_src)}
+                tex = time_scan(torch, L, tn, 1, 3, 3, flush=flush)
                 ent["exact_ms"] = statistics.mean(tex)
                 ent["exact_tokens_per_s"] = wn.B * wn.T / (ent["exact_ms"] * 1e-3)
                 extra[name] = ent
                 del tn
                 torch.cuda.empty_cache()
+            # chunk-form variants and the backward pass on the small training shape
+            ws = LI.WORKLOADS["small_train"]
+            ts = _dev_inputs(torch, LI.make_inputs(ws), device)
+            tok = lambda ms: ws.B * ws.T / (ms * 1e-3)
+            # the reconstruction objective (CUDA-core kernels), exact and chunked; the
+            # chunked form takes intensities sigmoid(N(-4,1)), with which it stays bounded
+            td = statistics.mean(time_scan(torch, L, ts, 1, 5, 3, flush=flush, mode="dec"))
+            extra["small_train_dec_exact"] = {"ms": td, "tokens_per_s": tok(td),
+                                              "kernel": "scan_simt_kernel<exact, dec>"}
+            tdc = _dev_inputs(torch, LI.make_inputs(ws.with_(c_loc=-4.0)), device)
+            td = statistics.mean(time_scan(torch, L, tdc, ws.chunk, 5, 3, flush=flush, mode="dec"))
+            extra["small_train_dec_chunked"] = {"ms": td, "tokens_per_s": tok(td),
+                                                "kernel": "scan_simt_kernel<chunked, dec>",
+                                                "inputs": "c = sigmoid(N(-4,1))"}
+            del tdc
+            # the normalisation ablation of Appendix C (CUDA-core kernel)
+            tn = statistics.mean(time_scan(torch, L, ts, ws.chunk, 5, 3, flush=flush, norm="chunk"))
+            extra["small_train_chunk_norm"] = {"ms": tn, "tokens_per_s": tok(tn),
+                                               "kernel": "scan_simt_kernel<chunked, norm at chunk ends>"}
+            # the other chunk linearisation (recurrence_linear1, CUDA-core kernel)
+            tl = statistics.mean(time_scan(torch, L, ts, ws.chunk, 5, 3, flush=flush, lin=1))
+            extra["small_train_lin1_chunked"] = {"ms": tl, "tokens_per_s": tok(tl),
+                                                 "kernel": "scan_simt_kernel<chunked, recurrence_linear1>"}
+            # backward pass (CUDA-core kernel), chunked and exact
+            for cb, tag in ((ws.chunk, "chunked"), (1, "exact")):
+                tb = statistics.mean(time_bwd(torch, L, ts, cb, 3, 2, flush=flush))
+                extra[f"small_train_bwd_{tag}"] = {"ms": tb, "tokens_per_s": tok(tb),
+                                                   "kernel": f"scan_bwd_kernel<{tag}>",
+                                                   "allocations": "outputs per call; workspace once"}
+            del ts
+            torch.cuda.empty_cache()
             wd = LI.WORKLOADS["decode"]
             us_ms, n = time_decode(torch, L, wd, 1000, 40, device)
             sb = step_alg_bytes(wd)
             extra["decode"] = {"us_per_step": us_ms * 1e3, "steps": n, "gbps": sb / (us_ms * 1e-3) / 1e9,
                                "hbm_frac": sb / (us_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                               "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb}
+                               "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb,
+                               "kernel": "step_kernel"}
             us_ms, n = time_decode(torch, L, wd, 1000, 40, device, mode="dec")
             extra["decode_dec"] = {"us_per_step": us_ms * 1e3, "steps": n, "gbps": sb / (us_ms * 1e-3) / 1e9,
                                    "hbm_frac": sb / (us_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                                   "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb}
+                                   "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb,
+                                   "kernel": "step_kernel<dec>"}
         line["extra"] = extra
         if not args.no_cpu:
             v, cores, sample = oracle_baseline(w, w.chunk)

@@ -216,11 +216,12 @@ size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int c
  * LATTICE_ERR_UNSUPPORTED before any device work. The caller still allocates the
  * inputs and outputs; the call itself makes no allocation.
  *
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream capture.
- * Every call shares the one array: calls that overlap on the GPU (on different
- * streams, or from different host threads without ordering) race and corrupt each
- * other's results, so order them. Nothing needs clearing between calls: the kernel
+ * The first call in each CUDA context (the device's primary context, or a context
+ * the caller created and made current) looks up the array's device address in that
+ * context with cudaGetSymbolAddress and caches it under the context's unique id; make
+ * that first call before any stream capture. Every call shares the one array:
+ * calls that overlap on the GPU (on different streams, or from different host
+ * threads without ordering) race and corrupt each other's results, so order them. Nothing needs clearing between calls: the kernel
  * writes every scratch word before it reads it. */
 #define LATTICE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
@@ -250,6 +251,15 @@ lattice_status lattice_readout(const float *S, const void *q, lattice_dtype q_dt
  * last call gave up a bounded wait (and clears the flag), LATTICE_ERR_CUDA if
  * the stream reports an error, else LATTICE_OK. */
 lattice_status lattice_get_device_status(void *stream);
+
+/* Failure-detection self-test (the paper has no counterpart): launches one warp
+ * that waits, with the same bounded device-side wait the tensor-core kernels use,
+ * on an mbarrier that nothing ever completes. After limit_ns nanoseconds (1 ns to
+ * 1 s; else LATTICE_ERR_INVALID_ARG, nothing launched) the wait gives up, sets the
+ * device status word and the kernel returns, so the next
+ * lattice_get_device_status(stream) returns LATTICE_ERR_TIMEOUT (and clears the
+ * word) while the CUDA context stays usable. Asynchronous on `stream`. */
+lattice_status lattice_selftest_bounded_wait(unsigned long long limit_ns, void *stream);
 
 /* Name and description of the last CUDA error the library saw on this host
  * thread when a call returned LATTICE_ERR_CUDA ("" if none). The text is

@@ -23,7 +23,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["LatticeError", "lib", "scan_fwd", "scan_bwd", "scan_bwd_workspace_bytes", "step",
-           "readout", "chunk_impl", "device_status", "LIB_PATH"]
+           "readout", "chunk_impl", "device_status", "selftest_bounded_wait", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblattice.so")
 
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.lattice_step.argtypes = [fp, vp, i, fp, vp, i, fp, fp, fp, i, i, i, i, i, vp]
         L.lattice_readout.argtypes = [fp, vp, i, fp, i, i, i, i, vp]
         L.lattice_get_device_status.argtypes = [vp]
+        L.lattice_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, vp]
         L.lattice_status_string.argtypes = [i]
         L.lattice_status_string.restype = ctypes.c_char_p
         L.lattice_version.argtypes = []
@@ -72,7 +73,7 @@ def lib() -> ctypes.CDLL:
         L.lattice_last_cuda_error.argtypes = []
         L.lattice_last_cuda_error.restype = ctypes.c_char_p
         for f in ("lattice_scan_fwd", "lattice_scan_fwd_impl", "lattice_scan_fwd_ex", "lattice_scan_bwd",
-                  "lattice_step", "lattice_readout",
+                  "lattice_step", "lattice_readout", "lattice_selftest_bounded_wait",
                   "lattice_get_device_status", "lattice_version", "lattice_chunk_impl"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -247,3 +248,11 @@ def device_status(stream=None) -> int:
     code = lib().lattice_get_device_status(_stream(stream))
     _raise(code, "lattice_get_device_status")
     return code
+
+
+def selftest_bounded_wait(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Launch the library's bounded-wait self-test: one warp waits on a barrier that
+    nothing completes and gives up after limit_ns. The next device_status() on the
+    same stream then raises LatticeError with code ERR_TIMEOUT."""
+    _raise(lib().lattice_selftest_bounded_wait(int(limit_ns), _stream(stream)),
+           "lattice_selftest_bounded_wait")

@@ -18,7 +18,7 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
     "-shared", "-Xcompiler", "-fPIC,-O2", "-cudart", "static",
-    "-Xptxas", "-warn-spills",
+    "-Xptxas", "-warn-spills", "-split-compile=0",
 ]
 
 

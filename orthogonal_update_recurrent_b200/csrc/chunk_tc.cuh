@@ -51,6 +51,7 @@
 #include "common.cuh"
 #include "scan_simt.cuh"
 #include "tc_ptx.cuh"
+#include "waits.cuh"
 
 namespace lattice {
 
@@ -58,7 +59,6 @@ constexpr int kTcC = 64;            // chunk size of the tensor-core path
 constexpr int kTcSub = 16;          // sub-chunk: the longest product ever divided by
 constexpr int kTcWorkers = 512;     // 16 worker warps: 4 lane quadrants x 4 sub-chunks
 constexpr int kTcThreads = kTcWorkers + 128;  // + control warpgroup (MMA warp, TMA warp, 2 idle)
-constexpr uint64_t kTcWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
 inline bool chunk_tc_supported(int m, int d, int chunk, bool x_bf16, bool q_bf16) {
     return chunk == kTcC && x_bf16 && q_bf16 && (m == 64 || m == 128) && (d == 64 || d == 128);
@@ -106,47 +106,6 @@ struct TcLayout {
 struct TcMaps {
     CUtensorMap x, q, c;
 };
-
-// Bounded wait: true when the phase completed; false (and the abort flag set)
-// when the bound elapsed or another thread already aborted.
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
-    if (*abort) return false;
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = ptx::globaltimer();
-    for (;;) {
-        if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;  // sleep <= 20 us per try
-        if (*abort) return false;
-        if (ptx::globaltimer() - t0 > kTcWaitNs) {
-            *abort = 1u;
-            flag_timeout();
-            return false;
-        }
-    }
-}
-
-// Warp-uniform form for the MMA warp: every lane waits, the warp agrees on the
-// outcome (and is converged for the elect.sync issue that follows).
-__device__ __forceinline__ bool tc_wait_warp(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
-    const bool ok = tc_wait(bar, parity, abort);
-    return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ bool tc_live(volatile uint32_t* abort) {
-    return __all_sync(0xffffffffu, *abort == 0u);
-}
-
-// Bounded wait that ignores the abort flag: used at exit so that no TMA write
-// into shared memory is still in flight when the CTA retires.
-__device__ __forceinline__ void tc_drain(uint32_t bar, uint32_t parity) {
-    const uint64_t t0 = ptx::globaltimer();
-    for (;;) {
-        if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return;
-        if (ptx::globaltimer() - t0 > kTcWaitNs) {
-            flag_timeout();
-            return;
-        }
-    }
-}
 
 __device__ __forceinline__ uint4 pack8(const float* v) {
     uint4 u;

@@ -247,6 +247,23 @@ lattice_status launch_bwd(const BwdArgs& a, int d, cudaStream_t st) {
     return LATTICE_ERR_UNSUPPORTED;
 }
 
+// One warp waits, with the library's bounded wait, on an mbarrier that nothing ever
+// arrives on: after limit_ns the wait gives up, sets the device status word and the
+// kernel returns. Used to check, on a live GPU, that a wait that runs out is reported
+// on the host and leaves the context usable.
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    const uint32_t b = ptx::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(b, 1);
+        abort_flag = 0u;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    tc_wait(b, 0, &abort_flag, limit_ns);
+}
+
 lattice_status check_dims(int B, int H, int m, int d) {
     if (B < 1 || H < 1 || m < 1 || d < 1) return LATTICE_ERR_INVALID_ARG;
     if ((long long)B * H > 0x7fffffffLL) return LATTICE_ERR_UNSUPPORTED;
@@ -482,6 +499,12 @@ lattice_status lattice_scan_bwd(const void* x, lattice_dtype x_dtype, const floa
     return chunk_size == 1 ? launch_bwd<false>(a, d, st) : launch_bwd<true>(a, d, st);
 }
 
+lattice_status lattice_selftest_bounded_wait(unsigned long long limit_ns, void* stream) {
+    if (limit_ns < 1 || limit_ns > 1000000000ull) return LATTICE_ERR_INVALID_ARG;
+    bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return launch_status();
+}
+
 lattice_status lattice_get_device_status(void* stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);
@@ -502,28 +525,73 @@ const char* lattice_last_cuda_error(void) { return g_last_error; }
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = LATTICE_NOALLOC_SCRATCH_BYTES;
-constexpr int kNoAllocMaxDevices = 64;
+constexpr int kNoAllocCacheEntries = 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
+// The array's device address differs from context to context (each context loads its
+// own copy of the module), so the looked-up address is cached per context, keyed by
+// the driver's unique context id. A caller running inside its own driver-API context,
+// or a process that reset the device and so got a new primary context, gets a fresh
+// lookup instead of an address that belongs to another context.
+struct NoAllocEntry {
+    unsigned long long ctx_id;
+    void* addr;
+};
 std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+NoAllocEntry g_noalloc_cache[kNoAllocCacheEntries] = {};
+int g_noalloc_next = 0;
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device. In host code the array's name is only a host-side stand-in.
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext*);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long*);
+
+// Unique id of the context current on this thread (false if none is current).
+bool current_ctx_id(unsigned long long* id) {
+    static PfnCtxGetCurrent get_current = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PfnCtxGetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PfnCtxGetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_noalloc_scratch in the current context, looked up once per
+// context with cudaGetSymbolAddress (a host-side query, no stream work). In host
+// code the array's name is only a host-side stand-in, never a device address.
 lattice_status noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return LATTICE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e);
-        g_noalloc_addr[dev] = p;
+    unsigned long long id = 0;
+    bool have_id = current_ctx_id(&id);
+    if (have_id) {
+        for (const NoAllocEntry& en : g_noalloc_cache)
+            if (en.addr && en.ctx_id == id) {
+                *out = en.addr;
+                return LATTICE_OK;
+            }
     }
-    *out = g_noalloc_addr[dev];
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the device's primary context current if none is
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!have_id) have_id = current_ctx_id(&id);
+    if (have_id) {
+        g_noalloc_cache[g_noalloc_next] = NoAllocEntry{id, p};
+        g_noalloc_next = (g_noalloc_next + 1) % kNoAllocCacheEntries;
+    }
+    *out = p;
     return LATTICE_OK;
 }
 

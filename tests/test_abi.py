@@ -136,3 +136,31 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(TypeError):
         L.scan_fwd(x, torch.zeros(1, 2, 1, 4), torch.zeros(1, 2, 1, 4), torch.zeros(1, 2, 1),
                    torch.zeros(1, 1, 4, 16))
+
+
+def test_noalloc_backward_rejects_shapes_beyond_its_scratch(lib):
+    """lattice_scan_bwd_noalloc: the small training shape's backward workspace (about
+    50 MB) fits the library's static 64 MiB scratch array; a shape that needs more is
+    refused on the host, before any device work (no CUDA call is made here)."""
+    lib.lattice_scan_bwd_noalloc.restype = ctypes.c_int
+    assert 0 < lib.lattice_scan_bwd_workspace_bytes(4, 2048, 8, 64, 64, 64, 0) <= 64 << 20
+    big = lib.lattice_scan_bwd_workspace_bytes(8, 4096, 16, 128, 128, 64, 0)
+    assert big > 64 << 20
+    v = ctypes.c_void_p
+    code = lib.lattice_scan_bwd_noalloc(v(1 << 20), 0, v(2 << 20), v(3 << 20), 0, v(4 << 20), None,
+                                        v(5 << 20), v(6 << 20), None, v(7 << 20), v(8 << 20),
+                                        v(9 << 20), v(10 << 20), None, v(11 << 20), 8, 4096, 16, 128,
+                                        128, 64, 0, None)
+    assert code == L.ERR_UNSUPPORTED
+    # rejected arguments are named by the same checks as lattice_scan_bwd's
+    code = lib.lattice_scan_bwd_noalloc(v(1 << 20), 0, v(2 << 20), v(3 << 20), 0, v(4 << 20), None,
+                                        v(5 << 20), v(6 << 20), None, v(7 << 20), v(8 << 20),
+                                        v(9 << 20), v(10 << 20), None, v(11 << 20), 1, 4, 1, 4,
+                                        48, 1, 0, None)
+    assert code == L.ERR_UNSUPPORTED  # d = 48
+
+
+def test_bounded_wait_selftest_checks_its_limit(lib):
+    # out-of-range limits are refused before any launch (no CUDA call is made here)
+    assert lib.lattice_selftest_bounded_wait(0, None) == L.ERR_INVALID_ARG
+    assert lib.lattice_selftest_bounded_wait(2_000_000_000, None) == L.ERR_INVALID_ARG

@@ -68,7 +68,7 @@ def test_reference_arm_prints_one_contract_line(monkeypatch):
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "tokens/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
-    assert line["config"]["workload"] == "small_train"
+    assert line["config"]["workload"] == "long_ctx"
 
 
 def test_bench_rejects_too_few_warmup_steps(monkeypatch):

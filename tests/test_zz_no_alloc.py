@@ -4,11 +4,15 @@ through its own pool, or a process that reserved the device's memory up front).
 It runs the same backward kernel with its scratch in a static array inside the
 library; the caller passes only inputs and outputs.
 
-This file is collected last on purpose. The test calls the new entry point
-through the C ABI twice in a row, on different shapes and data, and checks each
-result against lattice_scan_bwd (the entry point that takes a caller-allocated
-workspace) within the backward tests' tolerance. The second call would expose
-scratch contents left over from the first.
+The test calls the entry point through the C ABI twice in a row, on different
+shapes and data, and checks each result against lattice_scan_bwd (the entry point
+that takes a caller-allocated workspace) within the backward tests' tolerance. The
+second call would expose scratch contents left over from the first.
+
+The file sorts last so that pytest collects it after every other test: the entry
+point's static array stays resident on the device once used, and a run that stops
+at the first failure has then already run the rest of the suite. The test passes
+both alone in a fresh process and after the other tests.
 """
 import ctypes
 
@@ -83,18 +87,3 @@ def test_noalloc_backward_matches_the_workspace_entry_point_on_two_calls_in_a_ro
                 continue
             err = rel_err_per_slice(got[k].cpu().numpy(), ref[k].cpu().numpy(), ax)
             assert err <= TOL_BWD, (w.name, k, err)
-
-
-def test_noalloc_backward_rejects_shapes_beyond_its_scratch(L):
-    """The small training shape needs about 50 MB of scratch and fits; a shape that
-    needs more than the library's static array is refused before any device work."""
-    lib = L.lib()
-    assert 0 < lib.lattice_scan_bwd_workspace_bytes(4, 2048, 8, 64, 64, 64, 0) <= 64 << 20
-    big = lib.lattice_scan_bwd_workspace_bytes(8, 4096, 16, 128, 128, 64, 0)
-    assert big > 64 << 20
-    v = lambda a: ctypes.c_void_p(a)
-    code = lib.lattice_scan_bwd_noalloc(v(1 << 20), 0, v(2 << 20), v(3 << 20), 0, v(4 << 20), None,
-                                        v(5 << 20), v(6 << 20), None, v(7 << 20), v(8 << 20),
-                                        v(9 << 20), v(10 << 20), None, v(11 << 20), 8, 4096, 16, 128,
-                                        128, 64, 0, None)
-    assert code == L.ERR_UNSUPPORTED
