@@ -98,6 +98,11 @@ typedef enum { LATTICE_SIM = 0, LATTICE_DEC = 1 } lattice_mode;
  *   TCGEN05_SPLIT   the tensor-core kernel with each sequence's 64 slots split
  *                   over a cluster of 4 CTAs (chunk 64, bf16 x and q, m = 64,
  *                   d in {64, 128}); for batches with fewer sequences than SMs.
+ *   SPLIT_REG       the same split and read-out, with each CTA's share of the
+ *                   state held in registers and advanced chunk to chunk by
+ *                   warp-synchronous tensor-core MMAs (mma.sync), which keeps the
+ *                   per-chunk dependency chain off every asynchronous round trip
+ *                   (chunk 64, bf16 x and q, m = 64, d in {64, 128}).
  * An explicit choice that cannot run the shape returns LATTICE_ERR_UNSUPPORTED.
  * All tensor-core choices compute the same chunked form; they differ only in
  * fp32 summation order. */
@@ -105,7 +110,8 @@ typedef enum {
     LATTICE_IMPL_AUTO = 0,
     LATTICE_IMPL_SIMT = 1,
     LATTICE_IMPL_TCGEN05 = 2,
-    LATTICE_IMPL_TCGEN05_SPLIT = 3
+    LATTICE_IMPL_TCGEN05_SPLIT = 3,
+    LATTICE_IMPL_SPLIT_REG = 4
 } lattice_impl;
 
 /* Which kernel LATTICE_IMPL_AUTO runs for a chunked scan of B x H sequences of

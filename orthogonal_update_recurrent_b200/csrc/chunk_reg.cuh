@@ -1,0 +1,750 @@
+// chunk_reg.cuh -- chunked scan with each sequence's 64 slots split over a 4-CTA
+// cluster, the state chain held in registers and advanced with warp-synchronous
+// tensor-core MMAs, the read-out on tcgen05 tensor cores.
+//
+// Computes the chunked form, Eq. 17 of "Lattice: Learning to Efficiently Compress the
+// Memory" (§3.4.1 and Appendix B.1), chunk size 64, as chunk_tc.cuh and
+// chunk_split.cuh do. Each chunk of a sequence depends on the state the previous
+// chunk left, through the projections p = x . s0 and the normaliser of
+// eq. beta_chunk, so a sequence is a chain of T/64 dependent steps and its time is
+// the chain's latency times the number of chunks. This kernel keeps that chain off
+// every asynchronous round trip. Per CTA (16 slots) four chain warps, one per SM
+// sub-partition, hold the fp32 state in registers and, per chunk:
+//   projection  D[t][i] = x_t . s0_i            warp w: tokens 16w..16w+15, all slots
+//   gates       g, kappa of Eq. 17 per (token, slot), in the MMA's output registers
+//   scans       running products R (prefix) and Suf (suffix) of the gates over the
+//               warp's 16-token sub-chunk: shuffles over the fragment's rows
+//   update      S <- diag(A_C) S + sum_b f_b . (X_b^T KS_b)   warp w: state columns
+//               w*d/4..(w+1)*d/4; KS_j = kappa_j Suf(j) per sub-chunk b, scaled after
+//               the MMA by f_b = prod_{c>b} G_c (G_c: sub-chunk products), so no
+//               product of gates is ever divided in the state chain
+// with mma.sync m16n8k16 (bf16 operands, fp32 accumulation in registers; the state
+// operand is a hi+lo bf16 pair, so the carried state keeps close to fp32 accuracy)
+// and two 128-thread named barriers per chunk: one after the gates (sub-chunk
+// products and KS exchanged through shared memory), one after the update (the next
+// chunk's state operand and slot norms). An asynchronous tcgen05 MMA would put a
+// commit, an mbarrier wake-up and a tensor-memory load on the chain twice per chunk.
+//
+// The read-out y_t = sum_i q_ti s_i(t) is off the chain and uses the chunk-parallel
+// form of chunk_split.cuh: the chain warps write QR_b(t) = q_t prod_{l=16b..t} g_l
+// (times the sub-chunk products in between) and KD(j) = kappa_j / prod_{l=16b..j} g_l
+// (a division inside one 16-token sub-chunk only) and the chunk-start state hi part;
+// one MMA warp issues, on tcgen05 with fp32 accumulators in tensor memory,
+//   G4: Y_r  [C x d]  = QR_0 . S0hi                 inter-chunk read-out (K = 16)
+//   G5: P_r  [C x 16] = QR_b . KD_b^T, b = 0..3     scores per key sub-chunk
+//   G6: Y_r  [C x d] += P_r . X                     intra-chunk read-out (K = C)
+// and four read-out warps mask the scores, reduce-scatter the four CTAs' partial
+// Y_r through distributed shared memory (asynchronous remote stores that count
+// their bytes on the receiver's mbarrier; each CTA sums its quarter of the columns
+// in a fixed order) and store y. One TMA warp streams x, q and c through a 4-stage
+// ring (no multicast). Every mbarrier wait is bounded (waits.cuh).
+#pragma once
+#include "chunk_split.cuh"
+
+namespace lattice {
+
+constexpr int kRgSlots = 16;                    // slots per CTA
+constexpr int kRgNC = 4;                        // CTAs per sequence (64 slots)
+constexpr int kRgChain = 128;                   // 4 chain warps
+constexpr int kRgReadout = 128;                 // 4 read-out warps
+constexpr int kRgThreads = kRgChain + kRgReadout + 64;  // + MMA warp + TMA warp
+constexpr int kRgStages = 4;                    // x/q/c ring depth (chunks)
+
+inline bool chunk_reg_supported(int m, int d, int chunk, bool x_bf16, bool q_bf16) {
+    return chunk == kTcC && x_bf16 && q_bf16 && m == kRgSlots * kRgNC && (d == 64 || d == 128);
+}
+
+template <int DS>
+struct RgLayout {
+    static constexpr int DSL = DS / kRgNC;                 // y columns reduced by each CTA
+    static constexpr uint32_t X_STAGE = DS * 128;          // [C][d] bf16 in d/64 SW128 blocks
+    static constexpr uint32_t Q_STAGE = kTcC * kRgSlots * 2;  // [C][16] bf16
+    static constexpr uint32_t C_STAGE = kTcC * kRgSlots * 4;  // [C][16] fp32
+    static constexpr uint32_t X_OFF = 0;
+    static constexpr uint32_t Q_OFF = X_OFF + kRgStages * X_STAGE;
+    static constexpr uint32_t C_OFF = Q_OFF + kRgStages * Q_STAGE;
+    // chunk-start state, double-buffered by chunk parity: [d rows = state column e][128 B],
+    // slots 0-15 hi at columns 0-15, lo at columns 16-31 (SW128)
+    static constexpr uint32_t S0_BUF = DS * 128;
+    static constexpr uint32_t S0_OFF = C_OFF + kRgStages * C_STAGE;
+    static constexpr uint32_t QR_OFF = S0_OFF + 2 * S0_BUF;     // [C][128 B]: QR_b at columns 16b..16b+15
+    static constexpr uint32_t KT_OFF = QR_OFF + kTcC * 128;     // [C][128 B]: KD 0-15, KS hi 16-31, KS lo 32-47
+    static constexpr uint32_t P_OFF = KT_OFF + kTcC * 128;      // [C][C] bf16 masked scores
+    static constexpr uint32_t RECV_OFF = P_OFF + kTcC * 128;    // [2][NC][C][d/NC] fp32
+    static constexpr uint32_t RECV_BYTES = 2 * kRgNC * kTcC * DSL * 4;
+    static constexpr uint32_t AUX_OFF = RECV_OFF + RECV_BYTES;  // [2][C] float4: mu, eta, |x|^2, mu^2
+    static constexpr uint32_t GSUB_OFF = AUX_OFF + 2 * kTcC * 16;   // [4 sub-chunks][16 slots]
+    static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * kRgSlots * 4;  // [4 warps][16 slots]
+    static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * kRgSlots * 4;
+    static constexpr int NBAR = 2 * kRgStages + 8;
+    static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr uint32_t BYTES = MISC_OFF + 64;
+    static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;
+    // TMEM columns: P | Y double-buffered
+    static constexpr uint32_t P_COL = 0;
+    static constexpr uint32_t Y_COL = kTcC;
+    static constexpr uint32_t TMEM_COLS = (Y_COL + 2 * DS <= 256) ? 256 : 512;
+    static constexpr uint32_t STAGE_TX = X_STAGE + Q_STAGE + C_STAGE;
+    static_assert(S0_OFF % 1024 == 0 && QR_OFF % 1024 == 0 && KT_OFF % 1024 == 0 && P_OFF % 1024 == 0,
+                  "SW128 tiles are 1024-byte aligned");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+template <int DS>
+__global__ void __launch_bounds__(kRgThreads, 1)
+    chunk_reg_kernel(const __grid_constant__ TcMaps maps, ScanArgs a) {
+    using Lay = RgLayout<DS>;
+    constexpr int DSL = Lay::DSL;
+    constexpr int NST = kRgStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rank = (int)ptx::cluster_ctarank();
+    const int bh = blockIdx.x / kRgNC, b = bh / a.H, h = bh % a.H;
+    const int T = a.T, H = a.H;
+    const int nch = (T + kTcC - 1) / kTcC;
+    constexpr int RO_WARP0 = kRgChain / 32, MMA_WARP = RO_WARP0 + 4, TMA_WARP = MMA_WARP + 1;
+
+    // mbarriers: ring stage full [NST] (TMA bytes) and empty [NST] (4 chain warps + the
+    // MMA warp's commit after G6), scores ready (G4, G5), read-out done (G6), peers'
+    // partial y in [2], per-token inputs ready [2], read-out buffer drained [2]
+    const uint32_t bar_full0 = sbase + Lay::BAR_OFF;
+    const uint32_t bar_empty0 = bar_full0 + 8 * NST;
+    const uint32_t bar_p5 = bar_empty0 + 8 * NST;
+    const uint32_t bar_y = bar_p5 + 8;
+    const uint32_t bar_recv0 = bar_y + 8;
+    const uint32_t bar_aux0 = bar_recv0 + 16;
+    const uint32_t bar_yfree0 = bar_aux0 + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+    volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 4);
+    volatile uint32_t* zmu = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 8);
+    float4* aux = reinterpret_cast<float4*>(smem + Lay::AUX_OFF);
+    float* gsub = reinterpret_cast<float*>(smem + Lay::GSUB_OFF);
+    float* tsq = reinterpret_cast<float*>(smem + Lay::TSQ_OFF);
+
+    // named barriers: chain warps alone (C1 after the gates, C2 after the update), chain
+    // warps (arrive) + MMA warp (A: read-out operands written), read-out warps (arrive)
+    // + MMA warp (P: masked scores written)
+    constexpr uint32_t BAR_C1 = 1, BAR_C2 = 2, BAR_A = 3, BAR_P = 4;
+    constexpr uint32_t N_CM = kRgChain + 32, N_RM = kRgReadout + 32;
+
+    if (warp == MMA_WARP) {
+        if (lane == 0) {
+            for (int s = 0; s < NST; ++s) {
+                ptx::mbar_init(bar_full0 + 8 * s, 1);
+                ptx::mbar_init(bar_empty0 + 8 * s, kRgChain / 32 + 1);
+            }
+            ptx::mbar_init(bar_p5, 1);
+            ptx::mbar_init(bar_y, 1);
+            ptx::mbar_init(bar_recv0, 1);
+            ptx::mbar_init(bar_recv0 + 8, 1);
+            ptx::mbar_init(bar_aux0, kRgReadout);
+            ptx::mbar_init(bar_aux0 + 8, kRgReadout);
+            ptx::mbar_init(bar_yfree0, kRgReadout);
+            ptx::mbar_init(bar_yfree0 + 8, kRgReadout);
+            *abort = 0u;
+            zmu[0] = 0u;
+            zmu[1] = 0u;
+            ptx::fence_mbar_init();
+        }
+        __syncwarp();
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), Lay::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();  // every CTA's barriers exist before any peer arrives on them
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == MMA_WARP) {
+        // ------------------------------------------------------------ MMA issue (tcgen05)
+        constexpr uint32_t idesc_g4 = ptx::idesc_bf16(kTcC, DS, 0, 0);
+        constexpr uint32_t idesc_g5 = ptx::idesc_bf16(kTcC, kRgSlots, 0, 0);
+        constexpr uint32_t idesc_g6 = ptx::idesc_bf16(kTcC, DS, 0, 1);
+        auto off = [](uint32_t bytes) { return uint64_t(bytes >> 4); };
+        const uint64_t dK_qr = ptx::sdesc_sw128(sbase + Lay::QR_OFF, 16, 1024);
+        const uint64_t dK_kd = ptx::sdesc_sw128(sbase + Lay::KT_OFF, 16, 1024);
+        const uint64_t dK_s0 = ptx::sdesc_sw128(sbase + Lay::S0_OFF, 16, 1024);
+        const uint64_t dK_p = ptx::sdesc_sw128(sbase + Lay::P_OFF, 16, 1024);
+        const uint64_t dM_x = ptx::sdesc_sw128(sbase + Lay::X_OFF, 64 * 128, 1024);
+        for (int k = 0; k < nch; ++k) {
+            const int s = k % NST, p = k & 1;
+            const uint32_t ycol = Lay::Y_COL + p * DS;
+            ptx::named_bar(BAR_A, N_CM);  // QR, KD of chunk k and its start state written
+            ptx::tc_fence_after();
+            // the read-out of chunk k-2 (same accumulator buffer) has been drained
+            const bool yfree = k < 2 || tc_wait_warp(bar_yfree0 + 8 * p, ((k - 2) >> 1) & 1, abort);
+            ptx::tc_fence_after();
+            if (yfree && tc_live(abort)) {
+                // G4: Y_r = QR_0 . S0hi  (M = C, N = d, K = 16); both K-major
+                ptx::mma_bf16_elect(tmem + ycol, dK_qr, dK_s0 + off(p * Lay::S0_BUF), idesc_g4, 0);
+                // G5: P[:, 16b..16b+15] = QR_b . KD_b^T  (M = C, N = 16, K = 16)
+#pragma unroll
+                for (int sb = 0; sb < 4; ++sb)
+                    ptx::mma_bf16_elect(tmem + Lay::P_COL + sb * 16, dK_qr + off(32 * sb),
+                                        dK_kd + off(sb * 16 * 128), idesc_g5, 0);
+            }
+            ptx::mma_commit_elect(bar_p5);
+            ptx::named_bar(BAR_P, N_RM);  // masked scores written by the read-out warps
+            ptx::tc_fence_after();
+            const bool xok = tc_wait_warp(bar_full0 + 8 * s, (k / NST) & 1, abort);
+            if (xok && tc_live(abort)) {
+                // G6: Y_r += P . X  (M = C, N = d, K = C); A K-major, B MN-major
+#pragma unroll
+                for (int kk = 0; kk < kTcC / 16; ++kk)
+                    ptx::mma_bf16_elect(tmem + ycol, dK_p + off(kk * 32),
+                                        dM_x + off(s * Lay::X_STAGE + kk * 2048), idesc_g6, 1);
+            }
+            ptx::mma_commit_elect(bar_y);
+            ptx::mma_commit_elect(bar_empty0 + 8 * s);  // the MMAs are done with stage s
+        }
+        if (nch > 0) tc_drain(bar_y, (nch - 1) & 1);
+    } else if (warp == TMA_WARP) {
+        // ------------------------------------------------------------ TMA issue (lane 0)
+        if (lane == 0 && nch > 0) {
+            const int s_lo = rank * kRgSlots;  // this CTA's slots in the q and c rows
+            int last[NST];
+#pragma unroll
+            for (int s = 0; s < NST; ++s) last[s] = -1;
+            auto prefetch_l2 = [&](int k) {
+#pragma unroll
+                for (int kb = 0; kb < DS / 64; ++kb) ptx::tma_prefetch_l2_4d(&maps.x, kb * 64, h, k * kTcC, b);
+                ptx::tma_prefetch_l2_4d(&maps.q, s_lo, h, k * kTcC, b);
+                ptx::tma_prefetch_l2_4d(&maps.c, s_lo, h, k * kTcC, b);
+            };
+            ptx::prefetch_tensormap(&maps.x);
+            ptx::prefetch_tensormap(&maps.q);
+            ptx::prefetch_tensormap(&maps.c);
+            for (int k = NST; k < NST + 4 && k < nch; ++k) prefetch_l2(k);
+            for (int k = 0; k < nch; ++k) {
+                const int s = k % NST;
+                if (k >= NST && !tc_wait(bar_empty0 + 8 * s, ((k / NST) - 1) & 1, abort)) break;
+                const uint32_t full = bar_full0 + 8 * s;
+                ptx::mbar_arrive_expect_tx(full, Lay::STAGE_TX);
+#pragma unroll
+                for (int kb = 0; kb < DS / 64; ++kb)
+                    ptx::tma_load_4d(sbase + Lay::X_OFF + s * Lay::X_STAGE + kb * (64 * 128), &maps.x, full,
+                                     kb * 64, h, k * kTcC, b);
+                ptx::tma_load_4d(sbase + Lay::Q_OFF + s * Lay::Q_STAGE, &maps.q, full, s_lo, h, k * kTcC, b);
+                ptx::tma_load_4d(sbase + Lay::C_OFF + s * Lay::C_STAGE, &maps.c, full, s_lo, h, k * kTcC, b);
+                last[s] = k;
+                if (k + NST + 4 < nch) prefetch_l2(k + NST + 4);
+            }
+#pragma unroll
+            for (int s = 0; s < NST; ++s)  // no TMA write may be in flight when the CTA retires
+                if (last[s] >= 0) tc_drain(bar_full0 + 8 * s, (last[s] / NST) & 1);
+        }
+        __syncwarp();
+    } else if (warp >= RO_WARP0) {
+        // ------------------------------------------------------------ read-out warps
+        const int q = warp & 3;
+        const int rt = tid - kRgChain;     // 0..127
+        const uint32_t lane_base = uint32_t(32 * q) << 16;
+        const bool row_ok = lane < 16;     // M = 64 accumulators: lanes 0-15 of each quadrant
+        const int trow = 16 * q + lane;    // accumulator row (token) of this lane
+        // per-token mu, eta, |x|^2, mu^2 of chunk k: 2 threads per token, each half of x
+        auto aux_chunk = [&](int k) {
+            const int s = k % NST, p = k & 1;
+            const int tk = rt >> 1, half = rt & 1;
+            const int t = k * kTcC + tk;
+            float mu = 0.f, eta = 1.f;
+            if (half == 0 && t < T) {
+                const size_t bth = ((size_t)b * T + t) * H + h;
+                mu = __ldg(a.mu + bth);
+                if (a.eta) eta = __ldg(a.eta + bth);
+            }
+            const bool ok = tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
+            const uint8_t* xs = smem + Lay::X_OFF + s * Lay::X_STAGE;
+            float2 acc = ptx::f2(0.f);
+            if (ok) {
+#pragma unroll
+                for (int u = 0; u < DS / 16; ++u) {  // DS/16 chunks of 16 B per thread
+                    const int ch = half * (DS / 16) + u;  // block ch/8, chunk ch%8 (any order sums the row)
+                    uint4 v = *reinterpret_cast<const uint4*>(xs + (ch >> 3) * (64 * 128) + tk * 128 + (ch & 7) * 16);
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float2 xv = make_float2(__uint_as_float(w4[c] << 16), __uint_as_float(w4[c] & 0xffff0000u));
+                        acc = ptx::f2fma(xv, xv, acc);
+                    }
+                }
+            }
+            float xx = acc.x + acc.y;
+            xx += __shfl_xor_sync(0xffffffffu, xx, 1);
+            if (half == 0) {
+                const float mu2 = mu * mu;
+                aux[p * kTcC + tk] = make_float4(mu, eta, xx, mu2);
+                if (!(mu2 >= 8.6736174e-19f)) zmu[p] = 1u;  // mu^2 < 2^-60 (or zero)
+            }
+            ptx::mbar_arrive(bar_aux0 + 8 * p);
+        };
+        // the four partials of this CTA's columns of chunk kc -> y. Summing chunk k-1
+        // before sending chunk k keeps two receive buffers enough: a peer's chunk k+1
+        // follows its sum of chunk k, which needs this CTA's chunk k, sent after this sum.
+        constexpr uint32_t RECV_TX = kRgNC * kTcC * DSL * 4;  // bytes of one chunk's partials
+        auto recv_y = [&](int kc) {
+            const int par = kc & 1;
+            tc_wait_cluster(bar_recv0 + 8 * par, (kc >> 1) & 1, abort);
+            if (rt == 0 && kc + 2 < nch) ptx::mbar_arrive_expect_tx(bar_recv0 + 8 * par, RECV_TX);  // chunk kc+2
+            if (*abort) return;
+            const int tk = rt >> 1;
+            const int t = kc * kTcC + tk;
+            constexpr int PER = DSL / 2;  // floats per thread: 8 (d = 64) or 16 (d = 128)
+            const int c0 = (rt & 1) * PER;
+            float acc[PER];
+#pragma unroll
+            for (int c = 0; c < PER; ++c) acc[c] = 0.f;
+#pragma unroll
+            for (int src = 0; src < kRgNC; ++src) {
+                const float* rb = reinterpret_cast<const float*>(
+                                      smem + Lay::RECV_OFF + ((par * kRgNC + src) * kTcC + tk) * (DSL * 4)) + c0;
+#pragma unroll
+                for (int c = 0; c < PER; c += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(rb + c);
+                    acc[c] += v.x; acc[c + 1] += v.y; acc[c + 2] += v.z; acc[c + 3] += v.w;
+                }
+            }
+            if (t < T) {
+                float* yp = a.y + (((size_t)b * T + t) * H + h) * DS + rank * DSL + c0;
+#pragma unroll
+                for (int c = 0; c < PER; c += 4)
+                    *reinterpret_cast<float4*>(yp + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+            }
+        };
+        if (rt == 0) {  // arm the receive barriers of chunks 0 and 1
+            if (nch > 0) ptx::mbar_arrive_expect_tx(bar_recv0, RECV_TX);
+            if (nch > 1) ptx::mbar_arrive_expect_tx(bar_recv0 + 8, RECV_TX);
+        }
+        if (nch > 0) aux_chunk(0);
+        for (int k = 0; k < nch; ++k) {
+            const int par = k & 1;
+            if (k + 1 < nch) aux_chunk(k + 1);
+            // causal mask of this chunk's scores: row trow, all 64 keys
+            tc_wait(bar_p5, k & 1, abort);
+            __syncwarp();
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tmem + lane_base + Lay::P_COL + 32 * half, r);
+                ptx::tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        float v[8];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int key = 32 * half + 8 * c8 + c;
+                            v[c] = (key <= trow) ? __uint_as_float(r[8 * c8 + c]) : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(smem + Lay::P_OFF + ptx::sw128_chunk(trow, 4 * half + c8)) = pack8(v);
+                    }
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::named_bar_arrive(BAR_P, N_RM);
+            if (k > 0) recv_y(k - 1);
+            // partial read-out of this chunk: every peer's quarter of the columns
+            tc_wait(bar_y, k & 1, abort);
+            __syncwarp();
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int pp = 0; pp < kRgNC; ++pp) {
+                __syncwarp();  // tcgen05.ld is warp-collective
+                uint32_t yv[DSL];
+                ptx::tmem_ld<DSL>(tmem + lane_base + Lay::Y_COL + par * DS + pp * DSL, yv);
+                ptx::tmem_wait_ld();
+                if (row_ok && !*abort) {
+                    const uint32_t dst = Lay::RECV_OFF + ((par * kRgNC + rank) * kTcC + trow) * (DSL * 4);
+                    const uint32_t cdst = ptx::mapa(sbase + dst, (uint32_t)pp);
+                    const uint32_t cbar = ptx::mapa(bar_recv0 + 8 * par, (uint32_t)pp);
+#pragma unroll
+                    for (int c = 0; c < DSL; c += 4)
+                        ptx::st_async_v4(cdst + c * 4, make_float4(__uint_as_float(yv[c]), __uint_as_float(yv[c + 1]),
+                                                                   __uint_as_float(yv[c + 2]), __uint_as_float(yv[c + 3])),
+                                         cbar);
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_yfree0 + 8 * par);  // this buffer may take chunk k+2
+        }
+        if (nch > 0) recv_y(nch - 1);
+    } else {
+        // ================================================================ chain warps
+        // Warp w: the projections and gates of tokens 16w..16w+15 (sub-chunk w), and the
+        // state columns w*d/4..(w+1)*d/4 in the update. Fragment coordinates: g = lane/4
+        // (a row: a token, or a state column), cq = lane%4 (a pair of slots 2cq, 2cq+1 of
+        // each 8-slot n-tile nt); index i of a 4-register fragment is (row g + 8(i/2),
+        // slot 8nt + 2cq + i%2).
+        const int w = warp;
+        const int g = lane >> 2, cq = lane & 3;
+        const int tok0 = 16 * w + g;                  // rows g and g+8 of the warp's tile
+        constexpr int MT = DS / 64;                   // 16-column m-tiles of the update per warp
+        const int e_base = w * (DS / 4);
+        const int lj = lane >> 3, lr = lane & 7;      // ldmatrix: matrix lj, row lr
+        uint8_t* qr = smem + Lay::QR_OFF;
+        uint8_t* kt = smem + Lay::KT_OFF;
+
+        // fp32 state: st[mt][nt][i] = s_{slot}[e], e = e_base + 16mt + g + 8(i/2)
+        float st[MT][2][4];
+        {
+            const float* S0g = a.S0 + ((size_t)bh * (kRgSlots * kRgNC) + rank * kRgSlots) * DS;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int e = e_base + 16 * mt + g + 8 * (i >> 1);
+                        const int sl = 8 * nt + 2 * cq + (i & 1);
+                        st[mt][nt][i] = S0g[(size_t)sl * DS + e];
+                    }
+        }
+        // the state as the next chunk's operand: hi/lo bf16 into S0 buffer p, and each
+        // slot's partial |s|^2 over this warp's columns into tsq[w]
+        auto write_state = [&](int p) {
+            uint8_t* dst = smem + Lay::S0_OFF + p * Lay::S0_BUF;
+            float ns[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int e = e_base + 16 * mt + g + 8 * hf;
+                        const float2 v = make_float2(st[mt][nt][2 * hf], st[mt][nt][2 * hf + 1]);
+                        uint32_t hi, lo;
+                        split2(v, hi, lo);
+                        const int col = 8 * nt + 2 * cq;
+                        *reinterpret_cast<uint32_t*>(dst + ptx::sw128_off(e, col)) = hi;
+                        *reinterpret_cast<uint32_t*>(dst + ptx::sw128_off(e, 16 + col)) = lo;
+                        ns[nt][0] = fmaf(v.x, v.x, ns[nt][0]);
+                        ns[nt][1] = fmaf(v.y, v.y, ns[nt][1]);
+                    }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float v = ns[nt][j];
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 8);
+                    v += __shfl_xor_sync(0xffffffffu, v, 16);
+                    if (g == 0) tsq[w * kRgSlots + 8 * nt + 2 * cq + j] = v;
+                }
+        };
+        // n = |s0|, 1/n, 1/n^2 of this thread's slots (index 2nt + j: slot 8nt + 2cq + j)
+        float nrm[4], inv_n[4], inv_n2[4];
+        auto load_norms = [&]() {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
+                const float nsq = ((tsq[sl] + tsq[kRgSlots + sl]) + tsq[2 * kRgSlots + sl]) + tsq[3 * kRgSlots + sl];
+                inv_n[u] = ptx::rsqrt_nr(nsq);
+                nrm[u] = nsq * inv_n[u];
+                inv_n2[u] = inv_n[u] * inv_n[u];
+            }
+        };
+
+        // ---- prologue: query tiles zeroed (blocks of later sub-chunks stay zero), state operand
+        for (int o = tid; o < int(kTcC * 128 / 16); o += kRgChain)
+            reinterpret_cast<uint4*>(qr)[o] = make_uint4(0u, 0u, 0u, 0u);
+        write_state(0);
+        ptx::named_bar(BAR_C2, kRgChain);
+        load_norms();
+
+        for (int k = 0; k < nch; ++k) {
+            const int s = k % NST, p = k & 1;
+            tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
+            const uint32_t xs_a = sbase + Lay::X_OFF + s * Lay::X_STAGE;
+            const uint32_t s0_a = sbase + Lay::S0_OFF + p * Lay::S0_BUF;
+            // ---- projection D[t][i] = x_t . (s0hi_i + s0lo_i), tokens 16w..16w+15
+            float acc[2][2][2][4];  // [k-step parity][hi, lo][nt][i]
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int v = 0; v < 2; ++v)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[u][v][nt][i] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < DS / 16; ++ks) {
+                uint32_t af[4], bhi[4], blo[4];
+                {   // A: x rows 16w + 8(lj&1) + lr, columns 16ks + 8(lj>>1)
+                    const int row = 16 * w + 8 * (lj & 1) + lr;
+                    const int col = 16 * ks + 8 * (lj >> 1);
+                    ptx::ldsm_x4(xs_a + (col >> 6) * (64 * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4), af);
+                }
+                {   // B: state rows e = 16ks + 8(lj&1) + lr; slots 8(lj>>1).. (hi), +16 (lo)
+                    const int e = 16 * ks + 8 * (lj & 1) + lr;
+                    ptx::ldsm_x4_t(s0_a + e * 128 + (((lj >> 1) ^ (e & 7)) << 4), bhi);
+                    ptx::ldsm_x4_t(s0_a + e * 128 + (((2 + (lj >> 1)) ^ (e & 7)) << 4), blo);
+                }
+                ptx::mma16816(acc[ks & 1][0][0], af, bhi);
+                ptx::mma16816(acc[ks & 1][0][1], af, bhi + 2);
+                ptx::mma16816(acc[ks & 1][1][0], af, blo);
+                ptx::mma16816(acc[ks & 1][1][1], af, blo + 2);
+            }
+            float pr[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    pr[nt][i] = (acc[0][0][nt][i] + acc[1][0][nt][i]) + (acc[0][1][nt][i] + acc[1][1][nt][i]);
+
+            // ---- gates of Eq. 17 (eq. beta_chunk with the chunk-start norm n):
+            //   e2 = eta c / n^2, pn = p / n, den = mu^2 + e2^2 max(|x|^2 - pn^2, 0),
+            //   g = (mu - e2 pn) / sqrt(den), kappa / n = e2 / sqrt(den); den = 0 keeps the slot
+            tc_wait(bar_aux0 + 8 * p, (k >> 1) & 1, abort);  // per-token inputs of chunk k
+            const bool zero_mu = zmu[p] != 0u;
+            const float* cs = reinterpret_cast<const float*>(smem + Lay::C_OFF + s * Lay::C_STAGE);
+            const uint16_t* qs = reinterpret_cast<const uint16_t*>(smem + Lay::Q_OFF + s * Lay::Q_STAGE);
+            float gt[2][4], kap[2][4], qv[2][4];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int tk = tok0 + 8 * hf;
+                const float4 z = aux[p * kTcC + tk];  // mu, eta, |x|^2, mu^2
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int u0 = 2 * nt;  // norm index of slot 8nt + 2cq
+                    const float2 cc = *reinterpret_cast<const float2*>(cs + tk * kRgSlots + 8 * nt + 2 * cq);
+                    const uint32_t q2 = *reinterpret_cast<const uint32_t*>(qs + tk * kRgSlots + 8 * nt + 2 * cq);
+                    const float2 pp = make_float2(pr[nt][2 * hf], pr[nt][2 * hf + 1]);
+                    const float2 e2 = ptx::f2mul(cc, ptx::f2mul(ptx::f2(z.y), make_float2(inv_n2[u0], inv_n2[u0 + 1])));
+                    const float2 pn = ptx::f2mul(pp, make_float2(inv_n[u0], inv_n[u0 + 1]));
+                    float2 perp = ptx::f2fma(ptx::f2neg(pn), pn, ptx::f2(z.z));
+                    perp.x = fmaxf(perp.x, 0.f);
+                    perp.y = fmaxf(perp.y, 0.f);
+                    const float2 den = ptx::f2fma(ptx::f2mul(e2, e2), perp, ptx::f2(z.w));
+                    float2 bn = ptx::rsqrt2_nr(den);
+                    if (zero_mu)
+                        bn = make_float2(den.x > 0.f ? ptx::rsqrt_nr(den.x) : 0.f, den.y > 0.f ? ptx::rsqrt_nr(den.y) : 0.f);
+                    float2 gg = ptx::f2mul(bn, ptx::f2fma(ptx::f2neg(e2), pn, ptx::f2(z.x)));
+                    float2 kk = ptx::f2mul(ptx::f2mul(bn, e2), make_float2(nrm[u0], nrm[u0 + 1]));  // kappa
+                    if (zero_mu) {
+                        if (!(den.x > 0.f)) { gg.x = 1.f; kk.x = 0.f; }
+                        if (!(den.y > 0.f)) { gg.y = 1.f; kk.y = 0.f; }
+                    }
+                    gt[nt][2 * hf] = gg.x;
+                    gt[nt][2 * hf + 1] = gg.y;
+                    kap[nt][2 * hf] = kk.x;
+                    kap[nt][2 * hf + 1] = kk.y;
+                    qv[nt][2 * hf] = __uint_as_float(q2 << 16);
+                    qv[nt][2 * hf + 1] = __uint_as_float(q2 & 0xffff0000u);
+                }
+            }
+            // ---- running products over the sub-chunk's 16 tokens (rows g and g+8 of
+            // each column): R = inclusive prefix, suf = exclusive suffix, Gs = the total
+            float R[2][4], suf[2][4], Gs[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float rl = gt[nt][j], rh = gt[nt][2 + j];
+                    float ul = rl, uh = rh;
+#pragma unroll
+                    for (int o = 1; o < 8; o <<= 1) {
+                        const float tl = __shfl_up_sync(0xffffffffu, rl, 4 * o);
+                        const float th = __shfl_up_sync(0xffffffffu, rh, 4 * o);
+                        const float dl = __shfl_down_sync(0xffffffffu, ul, 4 * o);
+                        const float dh = __shfl_down_sync(0xffffffffu, uh, 4 * o);
+                        if (g >= o) { rl *= tl; rh *= th; }
+                        if (g + o <= 7) { ul *= dl; uh *= dh; }
+                    }
+                    rh *= __shfl_sync(0xffffffffu, rl, 28 + cq);        // times prod of rows 0..7
+                    const float U = __shfl_sync(0xffffffffu, uh, cq);   // prod of rows 8..15
+                    ul *= U;                                            // prod of rows g..15
+                    const float nl = __shfl_down_sync(0xffffffffu, ul, 4);
+                    const float nh = __shfl_down_sync(0xffffffffu, uh, 4);
+                    R[nt][j] = rl;
+                    R[nt][2 + j] = rh;
+                    suf[nt][j] = g < 7 ? nl : U;       // prod of rows g+1..15
+                    suf[nt][2 + j] = g < 7 ? nh : 1.f;  // prod of rows g+9..15
+                    Gs[nt][j] = __shfl_sync(0xffffffffu, rh, 28 + cq);
+                }
+            // ---- read-out and state-update operands of this sub-chunk
+            if (k > 0) tc_wait(bar_p5, (k - 1) & 1, abort);  // G4/G5 of chunk k-1 are done with QR, KD
+            float qrw[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int tk = tok0 + 8 * hf, col = 8 * nt + 2 * cq;
+                    float kd[2], ks[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int i = 2 * hf + j;
+                        const float r = R[nt][i];
+                        kd[j] = kap[nt][i] * ptx::rcp_nr(copysignf(fmaxf(fabsf(r), 1e-37f), r));
+                        ks[j] = kap[nt][i] * suf[nt][i];
+                        qrw[nt][i] = qv[nt][i] * r;
+                    }
+                    uint32_t khi, klo;
+                    split2(make_float2(ks[0], ks[1]), khi, klo);
+                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(tk, col)) = ptx::pack_bf16x2(kd[0], kd[1]);
+                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(tk, 16 + col)) = khi;
+                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(tk, 32 + col)) = klo;
+                    *reinterpret_cast<uint32_t*>(qr + ptx::sw128_off(tk, 16 * w + col)) =
+                        ptx::pack_bf16x2(qrw[nt][2 * hf], qrw[nt][2 * hf + 1]);
+                }
+            if (g == 0) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    *reinterpret_cast<float2*>(gsub + w * kRgSlots + 8 * nt + 2 * cq) = make_float2(Gs[nt][0], Gs[nt][1]);
+            }
+            ptx::named_bar(BAR_C1, kRgChain);  // every sub-chunk's products and KS written
+            if (tid == 0) zmu[p] = 0u;         // every chain thread read it before the barrier
+            // per slot: the chunk decay A_C and f_b = prod_{c>b} G_c of each sub-chunk b
+            float AC[4], fb[3][4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
+                const float G0 = gsub[sl], G1 = gsub[kRgSlots + sl], G2 = gsub[2 * kRgSlots + sl],
+                            G3 = gsub[3 * kRgSlots + sl];
+                fb[2][u] = G3;
+                fb[1][u] = G2 * G3;
+                fb[0][u] = G1 * fb[1][u];
+                AC[u] = G0 * fb[0][u];
+            }
+            // query operands of the earlier key blocks bb < w for this warp's tokens:
+            // QR_bb(t) = QR_w(t) prod_{c=bb..w-1} G_c
+#pragma unroll
+            for (int bb = 0; bb < 3; ++bb) {
+                if (bb >= w) break;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float v[2];
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int sl = 8 * nt + 2 * cq + j;
+                            float cgb = 1.f;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                if (c >= bb && c < w) cgb *= gsub[c * kRgSlots + sl];
+                            v[j] = qrw[nt][2 * hf + j] * cgb;
+                        }
+                        const int tk = tok0 + 8 * hf, col = 8 * nt + 2 * cq;
+                        *reinterpret_cast<uint32_t*>(qr + ptx::sw128_off(tk, 16 * bb + col)) = ptx::pack_bf16x2(v[0], v[1]);
+                    }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_bar_arrive(BAR_A, N_CM);  // QR, KD and the chunk-start state are ready for G4/G5
+
+            // ---- state update: per key sub-chunk bb, U_bb[e][i] = sum_{j in bb} x_j[e] KS_j[i]
+            float ua[4][MT][2][4];
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) ua[bb][mt][nt][i] = 0.f;
+            const uint32_t kt_a = sbase + Lay::KT_OFF;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                uint32_t khi[4], klo[4];
+                {   // B: KS rows (tokens) 16bb + 8(lj&1) + lr, slots 8(lj>>1).. at columns 16.. (hi), 32.. (lo)
+                    const int row = 16 * bb + 8 * (lj & 1) + lr;
+                    ptx::ldsm_x4_t(kt_a + row * 128 + (((2 + (lj >> 1)) ^ (row & 7)) << 4), khi);
+                    ptx::ldsm_x4_t(kt_a + row * 128 + (((4 + (lj >> 1)) ^ (row & 7)) << 4), klo);
+                }
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t af[4];
+                    {   // A = X^T: x rows (tokens) 16bb + 8(lj>>1) + lr, columns e = e_base + 16mt + 8(lj&1)
+                        const int row = 16 * bb + 8 * (lj >> 1) + lr;
+                        const int e = e_base + 16 * mt + 8 * (lj & 1);
+                        ptx::ldsm_x4_t(xs_a + (e >> 6) * (64 * 128) + row * 128 + ((((e & 63) >> 3) ^ (row & 7)) << 4), af);
+                    }
+                    ptx::mma16816(ua[bb][mt][0], af, khi);
+                    ptx::mma16816(ua[bb][mt][1], af, khi + 2);
+                    ptx::mma16816(ua[bb][mt][0], af, klo);
+                    ptx::mma16816(ua[bb][mt][1], af, klo + 2);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_empty0 + 8 * s);  // done with x, q, c of stage s
+            // S <- A_C S + f_0 U_0 + f_1 U_1 + f_2 U_2 + U_3
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int u = 2 * nt + (i & 1);
+                        float v = ua[3][mt][nt][i];
+                        v = fmaf(fb[2][u], ua[2][mt][nt][i], v);
+                        v = fmaf(fb[1][u], ua[1][mt][nt][i], v);
+                        v = fmaf(fb[0][u], ua[0][mt][nt][i], v);
+                        st[mt][nt][i] = fmaf(AC[u], st[mt][nt][i], v);
+                    }
+            if (k + 1 < nch) {
+                write_state((k + 1) & 1);  // G4 of chunk k-1 (the buffer's last reader) is done
+                ptx::named_bar(BAR_C2, kRgChain);
+                load_norms();
+            }
+        }
+        // final state
+        float* So = a.S_out + ((size_t)bh * (kRgSlots * kRgNC) + rank * kRgSlots) * DS;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int e = e_base + 16 * mt + g + 8 * (i >> 1);
+                    const int sl = 8 * nt + 2 * cq + (i & 1);
+                    So[(size_t)sl * DS + e] = st[mt][nt][i];
+                }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();  // no peer still writes into this CTA's shared memory
+    ptx::tc_fence_after();
+    if (warp == MMA_WARP) ptx::tmem_dealloc(tmem, Lay::TMEM_COLS);
+}
+
+template <int DS>
+cudaError_t launch_chunk_reg_t(const ScanArgs& a, cudaStream_t st) {
+    using Lay = RgLayout<DS>;
+    TcMaps maps;
+    const int m = kRgSlots * kRgNC;
+    if (!make_map_4d(&maps.x, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DS, a.H, a.T, a.B, 64, true) ||
+        !make_map_4d(&maps.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, m, a.H, a.T, a.B, kRgSlots, false) ||
+        !make_map_4d(&maps.c, a.c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, m, a.H, a.T, a.B, kRgSlots, false))
+        return cudaErrorInvalidValue;
+    auto k = chunk_reg_kernel<DS>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * a.H * kRgNC);
+    cfg.blockDim = dim3(kRgThreads);
+    cfg.dynamicSmemBytes = Lay::SMEM_ALLOC;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kRgNC;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k, maps, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_chunk_reg(const ScanArgs& a, int d, cudaStream_t st) {
+    if (a.m != kRgSlots * kRgNC) return cudaErrorNotSupported;
+    if (d == 128) return launch_chunk_reg_t<128>(a, st);
+    if (d == 64) return launch_chunk_reg_t<64>(a, st);
+    return cudaErrorNotSupported;
+}
+
+}  // namespace lattice

@@ -12,6 +12,7 @@
 #include "step.cuh"
 #include "chunk_tc.cuh"
 #include "chunk_split.cuh"
+#include "chunk_reg.cuh"
 #include "scan_bwd.cuh"
 
 using namespace lattice;
@@ -311,7 +312,7 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
     if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return LATTICE_ERR_INVALID_ARG;
     if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
     if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05 &&
-        impl != LATTICE_IMPL_TCGEN05_SPLIT)
+        impl != LATTICE_IMPL_TCGEN05_SPLIT && impl != LATTICE_IMPL_SPLIT_REG)
         return LATTICE_ERR_INVALID_ARG;
     if (mode != LATTICE_SIM && mode != LATTICE_DEC) return LATTICE_ERR_INVALID_ARG;
     const bool dec = mode == LATTICE_DEC;
@@ -345,7 +346,8 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
 
     ScanArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, S_out, y,
                B, T, H, m, chunk_size};
-    const bool tc_choice = impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT;
+    const bool tc_choice = impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT ||
+                           impl == LATTICE_IMPL_SPLIT_REG;
     a.cnorm = cnorm && chunk_size > 1 ? 1 : 0;
     if (chunk_size == 1 && cnorm) {  // normalising after every token is the exact recurrence
         if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
@@ -357,6 +359,11 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
                                : launch_scan_simt<true>(a, d, dec, lin1, st);
     }
     if (impl == LATTICE_IMPL_AUTO) impl = lattice_chunk_impl(B, H, m, d, chunk_size, x_dtype, q_dtype);
+    if (impl == LATTICE_IMPL_SPLIT_REG) {
+        if (!chunk_reg_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
+        cudaError_t e = launch_chunk_reg(a, d, st);
+        return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
+    }
     if (impl == LATTICE_IMPL_TCGEN05_SPLIT) {
         if (!chunk_split_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
         cudaError_t e = launch_chunk_split(a, d, st);

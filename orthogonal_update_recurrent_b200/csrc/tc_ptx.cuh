@@ -342,6 +342,37 @@ __device__ __forceinline__ float rcp_nr(float x) {
     return fmaf(y, e, y);
 }
 
+// ---------------------------------------------------------------- warp-level MMA
+// Synchronous warp-wide MMA, m16n8k16, bf16 operands from registers, fp32 accumulate
+// in registers. Fragments (g = lane / 4, c = lane % 4; the lower half of each 32-bit
+// register holds the lower-indexed element):
+//   A 16x16: a[0] = (row g, cols 2c..2c+1), a[1] = (row g+8, cols 2c..), a[2] = (row g,
+//            cols 2c+8..), a[3] = (row g+8, cols 2c+8..)
+//   B 16x8:  b[0] = (rows 2c..2c+1, col g), b[1] = (rows 2c+8.., col g)
+//   C 16x8:  d[0..1] = (row g, cols 2c, 2c+1), d[2..3] = (row g+8, cols 2c, 2c+1)
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// Four 8x8 b16 matrices from shared memory: lanes 8j..8j+7 give the row addresses of
+// matrix j (16 contiguous bytes each); lane t receives (row t/4, cols 2(t%4)..+1) of
+// matrix j in r[j]. The .trans form delivers the transpose: (rows 2(t%4)..+1, col t/4).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -120,7 +120,7 @@ def test_empty_sequence_copies_state(L):
 
 
 @pytest.mark.parametrize("chunk,T1,impl", [(1, 13, "simt"), (64, 128, "simt"), (64, 128, "tcgen05"),
-                                           (64, 128, "tcgen05_split")])
+                                           (64, 128, "tcgen05_split"), (64, 128, "split_reg")])
 def test_resume(L, chunk, T1, impl):
     """scan(T1) then scan(T2) from the carried state equals scan(T1 + T2):
     bitwise on CUDA cores; within the bf16 tolerance on tensor cores, which
@@ -145,7 +145,8 @@ def test_resume(L, chunk, T1, impl):
         assert s_err(Sb.cpu().numpy(), S.cpu().numpy()) <= TOL_TC
 
 
-@pytest.mark.parametrize("m,chunk,impl", [(128, 1, "auto"), (128, 64, "tcgen05"), (64, 64, "tcgen05_split")])
+@pytest.mark.parametrize("m,chunk,impl", [(128, 1, "auto"), (128, 64, "tcgen05"), (64, 64, "tcgen05_split"),
+                                          (64, 64, "split_reg")])
 def test_deterministic(L, m, chunk, impl):
     """Repeated calls give bitwise-equal results (every reduction has a fixed order,
     the cluster read-out reduction included)."""
@@ -185,7 +186,7 @@ def test_chunked_tcgen05(L, m, d, T):
     assert s_err(Sg, So) <= TOL_TC
 
 
-@pytest.mark.parametrize("m,impl", [(128, "tcgen05"), (64, "tcgen05_split")])
+@pytest.mark.parametrize("m,impl", [(128, "tcgen05"), (64, "tcgen05_split"), (64, "split_reg")])
 def test_chunked_tcgen05_eta_and_gate_edges(L, m, impl):
     """eta given, mu = 1 and mu = 0 tokens, a token with mu = 0 and no write (a
     zero-norm update keeps every slot), zero intensities, duplicates."""
@@ -206,25 +207,27 @@ def test_chunked_tcgen05_eta_and_gate_edges(L, m, impl):
 
 # ------------------------------- chunked (Eq. 17), slots split over a cluster
 
+@pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg"])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("T", [64, 2 * 64 + 37, 5 * 64])
-def test_chunked_tcgen05_split(L, d, T):
-    """Cluster kernel (16 slots per CTA, read-out reduced across the 4 CTAs) vs the
-    oracle's Eq. 17 chunked form: several chunks and a ragged tail."""
+@pytest.mark.parametrize("T", [1, 64, 2 * 64 + 37, 5 * 64])
+def test_chunked_tcgen05_split(L, d, T, impl):
+    """Cluster kernels (16 slots per CTA, read-out reduced across the 4 CTAs) vs the
+    oracle's Eq. 17 chunked form: one token, several chunks and a ragged tail."""
     w = LI.Workload("t", B=2, T=T, H=3, m=64, d=d, seed=2000 + d + T)
     inp = LI.make_inputs(w)
-    yg, Sg = run_gpu(L, inp, 64, impl="tcgen05_split")
+    yg, Sg = run_gpu(L, inp, 64, impl=impl)
     yo, So = run_oracle(inp, 64)
     assert y_err(yg, yo) <= TOL_TC
     assert s_err(Sg, So) <= TOL_TC
 
 
-def test_chunked_split_and_wide_agree(L):
-    """The two tensor-core kernels compute the same chunked form."""
+@pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg"])
+def test_chunked_split_and_wide_agree(L, impl):
+    """The tensor-core kernels compute the same chunked form."""
     w = LI.Workload("t", B=3, T=700, H=2, m=64, d=128, seed=12)
     inp = LI.make_inputs(w)
     y1, S1 = run_gpu(L, inp, 64, impl="tcgen05")
-    y2, S2 = run_gpu(L, inp, 64, impl="tcgen05_split")
+    y2, S2 = run_gpu(L, inp, 64, impl=impl)
     assert y_err(y2, y1) <= 1e-2
     assert s_err(S2, S1) <= 1e-3
 
@@ -275,43 +278,54 @@ def test_readout(L):
         assert y_err(y.cpu().numpy()[:, None], yo[:, None]) <= TOL_F32
 
 
-# ------------------------------------- full-size workloads, sampled sequences
+# ---------------------------------------------- full-size workloads, every head
+#
+# The launches the benchmark times, compared head by head with the oracle over every
+# (b, h) sequence of the workload (the oracle runs each sequence on a host thread).
 
-FULL = [("small_train", [(0, 0), (3, 7), (2, 4)]),
-        ("mid_layer", [(0, 0), (7, 15), (4, 9)]),
-        ("long_ctx", [(0, 0), (0, 11)])]
+FULL = ["small_train", "mid_layer", "long_ctx"]
+# a few sequences of each workload, for the paths that are checked on samples
+FULL_PAIRS = {"small_train": [(0, 0), (3, 7), (2, 4)], "mid_layer": [(0, 0), (7, 15), (4, 9)],
+              "long_ctx": [(0, 0), (0, 11)]}
 
 
-@pytest.mark.parametrize("name,pairs", FULL)
-def test_full_size_exact_sampled(L, name, pairs):
-    """Full-size workload on the GPU (the launch the benchmark times), sampled
-    (b,h) sequences recomputed by the oracle over the whole sequence."""
+def every_head(w):
+    return [(b, h) for b in range(w.B) for h in range(w.H)]
+
+
+def oracle_every_head(inp, w, chunk, **kw):
+    """The oracle over every sequence of a full workload, as [B, T, H, d] / [B, H, m, d]."""
+    pairs = every_head(w)
+    yo, So = run_oracle(LI.sample_heads(inp, pairs), chunk, **kw)
+    yo = yo[:, :, 0].reshape(w.B, w.H, w.T, w.d).transpose(0, 2, 1, 3)
+    So = So[:, 0].reshape(w.B, w.H, w.m, w.d)
+    return yo, So
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_exact_every_head(L, name):
+    """Full-size workload, exact recurrence, every sequence against the oracle."""
     w = LI.WORKLOADS[name]
     inp = LI.make_inputs(w)
     yg, Sg = run_gpu(L, inp, 1)
-    sub = LI.sample_heads(inp, pairs)
-    yo, So = run_oracle(sub, 1)
-    bs = [p[0] for p in pairs]
-    hs = [p[1] for p in pairs]
-    assert y_err(yg[bs, :, hs][:, :, None], yo) <= TOL_F32
-    assert s_err(Sg[bs, hs][:, None], So) <= TOL_F32
+    yo, So = oracle_every_head(inp, w, 1)
+    assert y_err(yg, yo) <= TOL_F32
+    assert s_err(Sg, So) <= TOL_F32
 
 
-@pytest.mark.parametrize("name,pairs", FULL)
-@pytest.mark.parametrize("impl", ["simt", "tcgen05", "tcgen05_split"])
-def test_full_size_chunked_sampled(L, name, pairs, impl):
-    """Full-size workload, chunk 64, against the oracle's Eq. 17 chunked form."""
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_chunked_every_head(L, name):
+    """Full-size workload, chunk 64, every sequence against the oracle's Eq. 17 chunked
+    form, for every kernel that runs the shape (the automatic choice included)."""
     w = LI.WORKLOADS[name]
-    if impl == "tcgen05_split" and w.m != 64:
-        pytest.skip("the cluster kernel splits 64 slots")
     inp = LI.make_inputs(w)
-    yg, Sg = run_gpu(L, inp, w.chunk, impl=impl)
-    sub = LI.sample_heads(inp, pairs)
-    yo, So = run_oracle(sub, w.chunk)
-    bs = [p[0] for p in pairs]
-    hs = [p[1] for p in pairs]
-    assert y_err(yg[bs, :, hs][:, :, None], yo) <= TOL_TC
-    assert s_err(Sg[bs, hs][:, None], So) <= TOL_TC
+    yo, So = oracle_every_head(inp, w, w.chunk)
+    impls = ["auto", "simt", "tcgen05"] + (["tcgen05_split", "split_reg"] if w.m == 64 else [])
+    for impl in impls:
+        yg, Sg = run_gpu(L, inp, w.chunk, impl=impl)
+        assert y_err(yg, yo) <= TOL_TC, impl
+        assert s_err(Sg, So) <= TOL_TC, impl
+        del yg, Sg
 
 
 # ------------------------------------------- reconstruction objective (DEC)
@@ -435,7 +449,7 @@ def test_dec_step_resynchronised(L, m, d):
 def test_dec_tensor_core_choices_are_unsupported(L):
     w = LI.Workload("t", B=1, T=4, H=1, m=64, d=64, seed=1)
     inp = LI.make_inputs(w)
-    for impl in ("tcgen05", "tcgen05_split"):
+    for impl in ("tcgen05", "tcgen05_split", "split_reg"):
         with pytest.raises(L.LatticeError):
             run_gpu(L, inp, 64, impl=impl, mode="dec")
     yg, _ = run_gpu(L, inp, 64, mode="dec")  # AUTO takes the CUDA-core kernel
@@ -443,9 +457,9 @@ def test_dec_tensor_core_choices_are_unsupported(L):
     assert y_err(yg, yo) <= TOL_F32
 
 
-@pytest.mark.parametrize("name,pairs", FULL[:2])
+@pytest.mark.parametrize("name", FULL[:2])
 @pytest.mark.parametrize("chunk", [1, 64])
-def test_dec_full_size(L, name, pairs, chunk):
+def test_dec_full_size(L, name, chunk):
     """Full-size workload under the reconstruction objective (the launch bench.py
     times): finite everywhere, unit slots after the exact recurrence, and the
     sampled sequences' first 4 tokens equal to the oracle's."""
@@ -458,6 +472,7 @@ def test_dec_full_size(L, name, pairs, chunk):
     if chunk == 1:
         # each step renormalises in fp32: the norm error random-walks (1.3e-5 seen after 4096)
         np.testing.assert_allclose(np.linalg.norm(Sg, axis=-1), 1.0, atol=TOL_F32)
+    pairs = FULL_PAIRS[name]
     sub = LI.sample_heads(inp, pairs)
     sub = {k: (v[:, :4] if isinstance(v, np.ndarray) and v.ndim >= 3 and k != "S0" else v)
            for k, v in sub.items()}
@@ -499,14 +514,15 @@ def test_lin1_dec_resynchronised(L):
 def test_lin1_tensor_core_choices_are_unsupported(L):
     w = LI.Workload("t", B=1, T=64, H=1, m=64, d=64, seed=1)
     inp = LI.make_inputs(w)
-    for impl in ("tcgen05", "tcgen05_split"):
+    for impl in ("tcgen05", "tcgen05_split", "split_reg"):
         with pytest.raises(L.LatticeError):
             run_gpu(L, inp, 64, impl=impl, lin=1)
 
 
-@pytest.mark.parametrize("name,pairs", FULL[:1])
-def test_lin1_full_size_sampled(L, name, pairs):
+@pytest.mark.parametrize("name", FULL[:1])
+def test_lin1_full_size_sampled(L, name):
     w = LI.WORKLOADS[name]
+    pairs = FULL_PAIRS[name]
     inp = LI.make_inputs(w)
     yg, Sg = run_gpu(L, inp, w.chunk, lin=1)
     sub = LI.sample_heads(inp, pairs)
@@ -538,7 +554,7 @@ def test_chunk_norm_chunk_one_is_exact_and_tensor_cores_refuse(L):
     y1, S1 = run_gpu(L, inp, 1, norm="chunk")
     ye, Se = run_oracle(inp, 1)
     assert y_err(y1, ye) <= TOL_F32 and s_err(S1, Se) <= TOL_F32
-    for impl in ("tcgen05", "tcgen05_split"):
+    for impl in ("tcgen05", "tcgen05_split", "split_reg"):
         with pytest.raises(L.LatticeError):
             run_gpu(L, inp, 64, impl=impl, norm="chunk")
 
