@@ -449,18 +449,20 @@ def oracle_legs(w: LI.Workload, seconds: float = 3.0) -> dict:
 
 # ---------------------------------------------------------------------- main
 
-def kernel_name(L, w: LI.Workload, chunk: int) -> str:
-    """The kernel lattice_scan_fwd's automatic choice runs for this workload."""
-    kimpl = L.chunk_impl(w.B, w.H, w.m, w.d, chunk)
-    return {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel"}.get(
+def kernel_name(L, w: LI.Workload, chunk: int, impl: str = "auto") -> str:
+    """The kernel lattice_scan_fwd runs for this workload (the automatic choice by default)."""
+    kimpl = L.chunk_impl(w.B, w.H, w.m, w.d, chunk) if impl == "auto" else impl
+    return {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel",
+            "split_reg": "chunk_reg_kernel"}.get(
         kimpl, "scan_simt_kernel<chunked>" if chunk > 1 else "scan_simt_kernel<exact>")
 
 
-def scan_roofline(L, w: LI.Workload, traffic_key: str, kern_ms: float, pk: dict, pk_src: str) -> dict:
+def scan_roofline(L, w: LI.Workload, traffic_key: str, kern_ms: float, pk: dict, pk_src: str,
+                  impl: str = "auto") -> dict:
     """Roofline record of one scan launch of `w` that took kern_ms (CUDA events):
     algorithmic HBM bytes / time against the measured copy bandwidth, and for the
     tensor-core kernels the algorithmic MMA flops / time against the bf16 peak."""
-    kname = kernel_name(L, w, w.chunk)
+    kname = kernel_name(L, w, w.chunk, impl)
     alg_b = scan_alg_bytes(w)
     achieved = alg_b / (kern_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -568,6 +570,8 @@ def main():
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "step"],
                     help="bwd: time the backward pass (lattice_scan_bwd) of the workload instead; "
                          "step: time the decode step (lattice_step) on the decode workload")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05", "tcgen05_split", "split_reg"],
+                    help="kernel choice of the timed scan (default: the library's automatic choice)")
     ap.add_argument("--chunk", type=int, default=None,
                     help="override the workload's chunk size (1: the exact recurrence)")
     args = ap.parse_args()
@@ -638,7 +642,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        times = time_scan(torch, L, t, w.chunk, args.steps, args.warmup, flush=flush)
+        times = time_scan(torch, L, t, w.chunk, args.steps, args.warmup, flush=flush, impl=args.kernel)
     torch.cuda.synchronize()
     total_ms = max_over_ranks(torch, dist, sum(times), device)
     if dist is not None:
@@ -647,7 +651,7 @@ def main():
     value = job_tokens_per_s(world, w, ms)
 
     # roofline of the (single) kernel of the step
-    roof = scan_roofline(L, w, w0.name, statistics.mean(times), pk, pk_src)
+    roof = scan_roofline(L, w, w0.name, statistics.mean(times), pk, pk_src, impl=args.kernel)
     tc = "tensor" in roof
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -673,6 +677,9 @@ def main():
             te = time_scan(torch, L, t, 1, 3, 3, flush=flush)
             extra[f"{w.name}_exact"] = {"ms": statistics.mean(te), "kernel": kernel_name(L, w, 1),
                                         "tokens_per_s": w.B * w.T / (statistics.mean(te) * 1e-3)}
+            if w.m == 64 and w.chunk == 64:  # the earlier cluster kernel, for comparison
+                extra[f"{w.name}_tcgen05_split_ms"] = statistics.mean(
+                    time_scan(torch, L, t, w.chunk, 5, 3, flush=flush, impl="tcgen05_split"))
             del t
             torch.cuda.empty_cache()
             # the other chunked workloads, each with its own roofline record
@@ -685,6 +692,9 @@ def main():
                 kms = statistics.mean(tch)
                 ent = {"ms": kms, "tokens_per_s": wn.B * wn.T / (kms * 1e-3),
                        "roofline": scan_roofline(L, wn, name, kms, pk, pk_src)}
+                if wn.m == 64:  # the earlier cluster kernel, for comparison
+                    ent["tcgen05_split_ms"] = statistics.mean(
+                        time_scan(torch, L, tn, wn.chunk, 5, 3, flush=flush, impl="tcgen05_split"))
                 tex = time_scan(torch, L, tn, 1, 3, 3, flush=flush)
                 ent["exact_ms"] = statistics.mean(tex)
                 ent["exact_tokens_per_s"] = wn.B * wn.T / (ent["exact_ms"] * 1e-3)

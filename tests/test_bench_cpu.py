@@ -75,3 +75,16 @@ def test_bench_rejects_too_few_warmup_steps(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--warmup", "2"])
     with pytest.raises(AssertionError):
         bench.main()
+
+
+def test_captured_traffic_is_dropped_once_the_kernel_changes(monkeypatch):
+    """A DRAM-traffic figure is reported only while the kernel's source file still has
+    the hash recorded with its capture; each entry names its profile summary."""
+    for (kern, wl), e in bench.CAPTURED_TRAFFIC.items():
+        assert os.path.exists(os.path.join(ROOT, e["profile"])), e["profile"]
+        expect = e["bytes"] if e["sha"] is not None and bench.source_sha(e["source"]) == e["sha"] else None
+        assert bench.traffic_for(kern, wl) == expect
+    key = next(iter(bench.CAPTURED_TRAFFIC))
+    monkeypatch.setitem(bench.CAPTURED_TRAFFIC, key, dict(bench.CAPTURED_TRAFFIC[key], sha="000000000000"))
+    assert bench.traffic_for(*key) is None
+    assert bench.traffic_for("no_such_kernel", "small_train") is None
