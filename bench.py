@@ -453,7 +453,7 @@ def kernel_name(L, w: LI.Workload, chunk: int, impl: str = "auto") -> str:
     """The kernel lattice_scan_fwd runs for this workload (the automatic choice by default)."""
     kimpl = L.chunk_impl(w.B, w.H, w.m, w.d, chunk) if impl == "auto" else impl
     return {"tcgen05": "chunk_tc_kernel", "tcgen05_split": "chunk_split_kernel",
-            "split_reg": "chunk_reg_kernel"}.get(
+            "split_reg": "chunk_reg_kernel<16 slots>", "split_reg8": "chunk_reg_kernel<8 slots>"}.get(
         kimpl, "scan_simt_kernel<chunked>" if chunk > 1 else "scan_simt_kernel<exact>")
 
 
@@ -570,7 +570,7 @@ def main():
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "step"],
                     help="bwd: time the backward pass (lattice_scan_bwd) of the workload instead; "
                          "step: time the decode step (lattice_step) on the decode workload")
-    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05", "tcgen05_split", "split_reg"],
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05", "tcgen05_split", "split_reg", "split_reg8"],
                     help="kernel choice of the timed scan (default: the library's automatic choice)")
     ap.add_argument("--chunk", type=int, default=None,
                     help="override the workload's chunk size (1: the exact recurrence)")

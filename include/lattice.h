@@ -103,6 +103,9 @@ typedef enum { LATTICE_SIM = 0, LATTICE_DEC = 1 } lattice_mode;
  *                   warp-synchronous tensor-core MMAs (mma.sync), which keeps the
  *                   per-chunk dependency chain off every asynchronous round trip
  *                   (chunk 64, bf16 x and q, m = 64, d in {64, 128}).
+ *   SPLIT_REG8      as SPLIT_REG with 8 slots per CTA over a cluster of 8 CTAs:
+ *                   half the tensor work on each CTA's chain; needs B*H clusters
+ *                   of 8 SMs within one GPC each.
  * An explicit choice that cannot run the shape returns LATTICE_ERR_UNSUPPORTED.
  * All tensor-core choices compute the same chunked form; they differ only in
  * fp32 summation order. */
@@ -111,7 +114,8 @@ typedef enum {
     LATTICE_IMPL_SIMT = 1,
     LATTICE_IMPL_TCGEN05 = 2,
     LATTICE_IMPL_TCGEN05_SPLIT = 3,
-    LATTICE_IMPL_SPLIT_REG = 4
+    LATTICE_IMPL_SPLIT_REG = 4,
+    LATTICE_IMPL_SPLIT_REG8 = 5
 } lattice_impl;
 
 /* Which kernel LATTICE_IMPL_AUTO runs for a chunked scan of B x H sequences of

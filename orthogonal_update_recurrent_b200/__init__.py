@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblattice.
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
 _F32, _BF16 = 0, 1
-_IMPL = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3, "split_reg": 4}
+_IMPL = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3, "split_reg": 4, "split_reg8": 5}
 _MODE = {"sim": 0, "dec": 1}
 _lib = None
 
@@ -240,7 +240,7 @@ def chunk_impl(B: int, H: int, m: int, d: int, chunk: int, x_dtype=torch.bfloat1
     "split_reg", "tcgen05_split", "tcgen05" or "simt"."""
     dt = lambda t: _BF16 if t == torch.bfloat16 else _F32
     code = lib().lattice_chunk_impl(B, H, m, d, chunk, dt(x_dtype), dt(q_dtype))
-    return {1: "simt", 2: "tcgen05", 3: "tcgen05_split", 4: "split_reg"}[code]
+    return {1: "simt", 2: "tcgen05", 3: "tcgen05_split", 4: "split_reg", 5: "split_reg8"}[code]
 
 
 def device_status(stream=None) -> int:

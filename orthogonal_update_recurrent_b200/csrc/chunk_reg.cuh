@@ -43,39 +43,42 @@
 
 namespace lattice {
 
-constexpr int kRgSlots = 16;                    // slots per CTA
-constexpr int kRgNC = 4;                        // CTAs per sequence (64 slots)
+constexpr int kRgM = 64;                        // slots per sequence
 constexpr int kRgChain = 128;                   // 4 chain warps
 constexpr int kRgReadout = 128;                 // 4 read-out warps
 constexpr int kRgThreads = kRgChain + kRgReadout + 64;  // + MMA warp + TMA warp
 constexpr int kRgStages = 4;                    // x/q/c ring depth (chunks)
 
 inline bool chunk_reg_supported(int m, int d, int chunk, bool x_bf16, bool q_bf16) {
-    return chunk == kTcC && x_bf16 && q_bf16 && m == kRgSlots * kRgNC && (d == 64 || d == 128);
+    return chunk == kTcC && x_bf16 && q_bf16 && m == kRgM && (d == 64 || d == 128);
 }
 
-template <int DS>
+// SPC slots per CTA (16: clusters of 4 CTAs; 8: clusters of 8), state width DS.
+template <int DS, int SPC>
 struct RgLayout {
-    static constexpr int DSL = DS / kRgNC;                 // y columns reduced by each CTA
+    static_assert(SPC == 8 || SPC == 16, "8 or 16 slots per CTA");
+    static constexpr int NC = kRgM / SPC;                  // CTAs per sequence (cluster size)
+    static constexpr int DSL = DS / NC;                    // y columns reduced by each CTA
     static constexpr uint32_t X_STAGE = DS * 128;          // [C][d] bf16 in d/64 SW128 blocks
-    static constexpr uint32_t Q_STAGE = kTcC * kRgSlots * 2;  // [C][16] bf16
-    static constexpr uint32_t C_STAGE = kTcC * kRgSlots * 4;  // [C][16] fp32
+    static constexpr uint32_t Q_STAGE = kTcC * SPC * 2;    // [C][SPC] bf16
+    static constexpr uint32_t C_STAGE = kTcC * SPC * 4;    // [C][SPC] fp32
     static constexpr uint32_t X_OFF = 0;
     static constexpr uint32_t Q_OFF = X_OFF + kRgStages * X_STAGE;
     static constexpr uint32_t C_OFF = Q_OFF + kRgStages * Q_STAGE;
     // chunk-start state, double-buffered by chunk parity: [d rows = state column e][128 B],
-    // slots 0-15 hi at columns 0-15, lo at columns 16-31 (SW128)
+    // the slots' hi parts at columns 0..SPC-1, lo parts at 16..16+SPC-1 (SW128); the
+    // columns up to 16 stay zero (the read-out GEMM takes K = 16)
     static constexpr uint32_t S0_BUF = DS * 128;
     static constexpr uint32_t S0_OFF = C_OFF + kRgStages * C_STAGE;
-    static constexpr uint32_t QR_OFF = S0_OFF + 2 * S0_BUF;     // [C][128 B]: QR_b at columns 16b..16b+15
-    static constexpr uint32_t KT_OFF = QR_OFF + kTcC * 128;     // [C][128 B]: KD 0-15, KS hi 16-31, KS lo 32-47
+    static constexpr uint32_t QR_OFF = S0_OFF + 2 * S0_BUF;     // [C][128 B]: QR_b at columns 16b..
+    static constexpr uint32_t KT_OFF = QR_OFF + kTcC * 128;     // [C][128 B]: KD at 0.., KS hi at 16.., lo at 32..
     static constexpr uint32_t P_OFF = KT_OFF + kTcC * 128;      // [C][C] bf16 masked scores
     static constexpr uint32_t RECV_OFF = P_OFF + kTcC * 128;    // [2][NC][C][d/NC] fp32
-    static constexpr uint32_t RECV_BYTES = 2 * kRgNC * kTcC * DSL * 4;
+    static constexpr uint32_t RECV_BYTES = 2 * NC * kTcC * DSL * 4;
     static constexpr uint32_t AUX_OFF = RECV_OFF + RECV_BYTES;  // [2][C] float4: mu, eta, |x|^2, mu^2
-    static constexpr uint32_t GSUB_OFF = AUX_OFF + 2 * kTcC * 16;   // [4 sub-chunks][16 slots]
-    static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * kRgSlots * 4;  // [4 warps][16 slots]
-    static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * kRgSlots * 4;
+    static constexpr uint32_t GSUB_OFF = AUX_OFF + 2 * kTcC * 16;   // [4 sub-chunks][16] (SPC used)
+    static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * 16 * 4;        // [4 warps][16] (SPC used)
+    static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * 16 * 4;
     static constexpr int NBAR = 2 * kRgStages + 8;
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr uint32_t BYTES = MISC_OFF + 64;
@@ -90,11 +93,13 @@ struct RgLayout {
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-template <int DS>
+template <int DS, int SPC>
 __global__ void __launch_bounds__(kRgThreads, 1)
     chunk_reg_kernel(const __grid_constant__ TcMaps maps, ScanArgs a) {
-    using Lay = RgLayout<DS>;
+    using Lay = RgLayout<DS, SPC>;
     constexpr int DSL = Lay::DSL;
+    constexpr int NC = Lay::NC;
+    constexpr int NT = SPC / 8;  // 8-slot n-tiles per CTA
     constexpr int NST = kRgStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -102,7 +107,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     const uint32_t sbase = ptx::smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = (int)ptx::cluster_ctarank();
-    const int bh = blockIdx.x / kRgNC, b = bh / a.H, h = bh % a.H;
+    const int bh = blockIdx.x / NC, b = bh / a.H, h = bh % a.H;
     const int T = a.T, H = a.H;
     const int nch = (T + kTcC - 1) / kTcC;
     constexpr int RO_WARP0 = kRgChain / 32, MMA_WARP = RO_WARP0 + 4, TMA_WARP = MMA_WARP + 1;
@@ -162,7 +167,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issue (tcgen05)
         constexpr uint32_t idesc_g4 = ptx::idesc_bf16(kTcC, DS, 0, 0);
-        constexpr uint32_t idesc_g5 = ptx::idesc_bf16(kTcC, kRgSlots, 0, 0);
+        constexpr uint32_t idesc_g5 = ptx::idesc_bf16(kTcC, kTcSub, 0, 0);
         constexpr uint32_t idesc_g6 = ptx::idesc_bf16(kTcC, DS, 0, 1);
         auto off = [](uint32_t bytes) { return uint64_t(bytes >> 4); };
         const uint64_t dK_qr = ptx::sdesc_sw128(sbase + Lay::QR_OFF, 16, 1024);
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     } else if (warp == TMA_WARP) {
         // ------------------------------------------------------------ TMA issue (lane 0)
         if (lane == 0 && nch > 0) {
-            const int s_lo = rank * kRgSlots;  // this CTA's slots in the q and c rows
+            const int s_lo = rank * SPC;  // this CTA's slots in the q and c rows
             int last[NST];
 #pragma unroll
             for (int s = 0; s < NST; ++s) last[s] = -1;
@@ -284,7 +289,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         // the four partials of this CTA's columns of chunk kc -> y. Summing chunk k-1
         // before sending chunk k keeps two receive buffers enough: a peer's chunk k+1
         // follows its sum of chunk k, which needs this CTA's chunk k, sent after this sum.
-        constexpr uint32_t RECV_TX = kRgNC * kTcC * DSL * 4;  // bytes of one chunk's partials
+        constexpr uint32_t RECV_TX = NC * kTcC * DSL * 4;  // bytes of one chunk's partials
         auto recv_y = [&](int kc) {
             const int par = kc & 1;
             tc_wait_cluster(bar_recv0 + 8 * par, (kc >> 1) & 1, abort);
@@ -292,15 +297,15 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             if (*abort) return;
             const int tk = rt >> 1;
             const int t = kc * kTcC + tk;
-            constexpr int PER = DSL / 2;  // floats per thread: 8 (d = 64) or 16 (d = 128)
+            constexpr int PER = DSL / 2;  // floats per thread: 4 to 16
             const int c0 = (rt & 1) * PER;
             float acc[PER];
 #pragma unroll
             for (int c = 0; c < PER; ++c) acc[c] = 0.f;
 #pragma unroll
-            for (int src = 0; src < kRgNC; ++src) {
+            for (int src = 0; src < NC; ++src) {
                 const float* rb = reinterpret_cast<const float*>(
-                                      smem + Lay::RECV_OFF + ((par * kRgNC + src) * kTcC + tk) * (DSL * 4)) + c0;
+                                      smem + Lay::RECV_OFF + ((par * NC + src) * kTcC + tk) * (DSL * 4)) + c0;
 #pragma unroll
                 for (int c = 0; c < PER; c += 4) {
                     const float4 v = *reinterpret_cast<const float4*>(rb + c);
@@ -353,13 +358,13 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             __syncwarp();
             ptx::tc_fence_after();
 #pragma unroll
-            for (int pp = 0; pp < kRgNC; ++pp) {
+            for (int pp = 0; pp < NC; ++pp) {
                 __syncwarp();  // tcgen05.ld is warp-collective
                 uint32_t yv[DSL];
                 ptx::tmem_ld<DSL>(tmem + lane_base + Lay::Y_COL + par * DS + pp * DSL, yv);
                 ptx::tmem_wait_ld();
                 if (row_ok && !*abort) {
-                    const uint32_t dst = Lay::RECV_OFF + ((par * kRgNC + rank) * kTcC + trow) * (DSL * 4);
+                    const uint32_t dst = Lay::RECV_OFF + ((par * NC + rank) * kTcC + trow) * (DSL * 4);
                     const uint32_t cdst = ptx::mapa(sbase + dst, (uint32_t)pp);
                     const uint32_t cbar = ptx::mapa(bar_recv0 + 8 * par, (uint32_t)pp);
 #pragma unroll
@@ -390,13 +395,13 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         uint8_t* kt = smem + Lay::KT_OFF;
 
         // fp32 state: st[mt][nt][i] = s_{slot}[e], e = e_base + 16mt + g + 8(i/2)
-        float st[MT][2][4];
+        float st[MT][NT][4];
         {
-            const float* S0g = a.S0 + ((size_t)bh * (kRgSlots * kRgNC) + rank * kRgSlots) * DS;
+            const float* S0g = a.S0 + ((size_t)bh * kRgM + rank * SPC) * DS;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int e = e_base + 16 * mt + g + 8 * (i >> 1);
@@ -408,11 +413,13 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         // slot's partial |s|^2 over this warp's columns into tsq[w]
         auto write_state = [&](int p) {
             uint8_t* dst = smem + Lay::S0_OFF + p * Lay::S0_BUF;
-            float ns[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            float ns[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) ns[nt][0] = ns[nt][1] = 0.f;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
                         const int e = e_base + 16 * mt + g + 8 * hf;
@@ -426,32 +433,56 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         ns[nt][1] = fmaf(v.y, v.y, ns[nt][1]);
                     }
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     float v = ns[nt][j];
                     v += __shfl_xor_sync(0xffffffffu, v, 4);
                     v += __shfl_xor_sync(0xffffffffu, v, 8);
                     v += __shfl_xor_sync(0xffffffffu, v, 16);
-                    if (g == 0) tsq[w * kRgSlots + 8 * nt + 2 * cq + j] = v;
+                    if (g == 0) tsq[w * 16 + 8 * nt + 2 * cq + j] = v;
                 }
         };
         // n = |s0|, 1/n, 1/n^2 of this thread's slots (index 2nt + j: slot 8nt + 2cq + j)
-        float nrm[4], inv_n[4], inv_n2[4];
+        float nrm[2 * NT], inv_n[2 * NT], inv_n2[2 * NT];
         auto load_norms = [&]() {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 2 * NT; ++u) {
                 const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
-                const float nsq = ((tsq[sl] + tsq[kRgSlots + sl]) + tsq[2 * kRgSlots + sl]) + tsq[3 * kRgSlots + sl];
+                const float nsq = ((tsq[sl] + tsq[16 + sl]) + tsq[32 + sl]) + tsq[48 + sl];
                 inv_n[u] = ptx::rsqrt_nr(nsq);
                 nrm[u] = nsq * inv_n[u];
                 inv_n2[u] = inv_n[u] * inv_n[u];
             }
         };
 
-        // ---- prologue: query tiles zeroed (blocks of later sub-chunks stay zero), state operand
-        for (int o = tid; o < int(kTcC * 128 / 16); o += kRgChain)
+        // B fragments (k = 16 rows from row0, n = 8 slots per n-tile) of a hi/lo operand pair
+        // stored row-major in an SW128 tile: hi slots at columns col0 + 8nt, lo at col0 + 16 + 8nt.
+        // ldmatrix.trans turns the stored [k][n] rows into the fragment layout.
+        auto load_b_pairs = [&](uint32_t tile, int row0, int col0, uint32_t (&bfr)[2][NT][2]) {
+            const int row = row0 + 8 * (lj & 1) + lr;
+            const uint32_t ra = tile + row * 128;
+            uint32_t r4[4];
+            if constexpr (NT == 2) {
+                ptx::ldsm_x4_t(ra + ((((col0 >> 3) + (lj >> 1)) ^ (row & 7)) << 4), r4);
+                bfr[0][0][0] = r4[0]; bfr[0][0][1] = r4[1]; bfr[0][1][0] = r4[2]; bfr[0][1][1] = r4[3];
+                ptx::ldsm_x4_t(ra + ((((col0 >> 3) + 2 + (lj >> 1)) ^ (row & 7)) << 4), r4);
+                bfr[1][0][0] = r4[0]; bfr[1][0][1] = r4[1]; bfr[1][1][0] = r4[2]; bfr[1][1][1] = r4[3];
+            } else {
+                ptx::ldsm_x4_t(ra + ((((col0 >> 3) + 2 * (lj >> 1)) ^ (row & 7)) << 4), r4);
+                bfr[0][0][0] = r4[0]; bfr[0][0][1] = r4[1]; bfr[1][0][0] = r4[2]; bfr[1][0][1] = r4[3];
+            }
+        };
+
+        // ---- prologue: operand tiles zeroed (the blocks of later sub-chunks in the query
+        // tile, and with 8 slots per CTA the K padding up to 16, are never written)
+        for (int o = tid; o < int(kTcC * 128 / 16); o += kRgChain) {
             reinterpret_cast<uint4*>(qr)[o] = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4*>(kt)[o] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (int o = tid; o < int(2 * Lay::S0_BUF / 16); o += kRgChain)
+            reinterpret_cast<uint4*>(smem + Lay::S0_OFF)[o] = make_uint4(0u, 0u, 0u, 0u);
+        ptx::named_bar(BAR_C2, kRgChain);
         write_state(0);
         ptx::named_bar(BAR_C2, kRgChain);
         load_norms();
@@ -462,36 +493,33 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             const uint32_t xs_a = sbase + Lay::X_OFF + s * Lay::X_STAGE;
             const uint32_t s0_a = sbase + Lay::S0_OFF + p * Lay::S0_BUF;
             // ---- projection D[t][i] = x_t . (s0hi_i + s0lo_i), tokens 16w..16w+15
-            float acc[2][2][2][4];  // [k-step parity][hi, lo][nt][i]
+            float acc[2][2][NT][4];  // [k-step parity][hi, lo][nt][i]
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int v = 0; v < 2; ++v)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) acc[u][v][nt][i] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < DS / 16; ++ks) {
-                uint32_t af[4], bhi[4], blo[4];
+                uint32_t af[4], bf[2][NT][2];  // B fragments [hi, lo][nt]
                 {   // A: x rows 16w + 8(lj&1) + lr, columns 16ks + 8(lj>>1)
                     const int row = 16 * w + 8 * (lj & 1) + lr;
                     const int col = 16 * ks + 8 * (lj >> 1);
                     ptx::ldsm_x4(xs_a + (col >> 6) * (64 * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4), af);
                 }
-                {   // B: state rows e = 16ks + 8(lj&1) + lr; slots 8(lj>>1).. (hi), +16 (lo)
-                    const int e = 16 * ks + 8 * (lj & 1) + lr;
-                    ptx::ldsm_x4_t(s0_a + e * 128 + (((lj >> 1) ^ (e & 7)) << 4), bhi);
-                    ptx::ldsm_x4_t(s0_a + e * 128 + (((2 + (lj >> 1)) ^ (e & 7)) << 4), blo);
-                }
-                ptx::mma16816(acc[ks & 1][0][0], af, bhi);
-                ptx::mma16816(acc[ks & 1][0][1], af, bhi + 2);
-                ptx::mma16816(acc[ks & 1][1][0], af, blo);
-                ptx::mma16816(acc[ks & 1][1][1], af, blo + 2);
-            }
-            float pr[2][4];
+                // B: state rows e = 16ks + 8(lj&1) + lr, slots 8nt.. (hi at column 0, lo at 16)
+                load_b_pairs(s0_a, 16 * ks, 0, bf);
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+                for (int v = 0; v < 2; ++v)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) ptx::mma16816(acc[ks & 1][v][nt], af, bf[v][nt]);
+            }
+            float pr[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     pr[nt][i] = (acc[0][0][nt][i] + acc[1][0][nt][i]) + (acc[0][1][nt][i] + acc[1][1][nt][i]);
@@ -503,16 +531,16 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             const bool zero_mu = zmu[p] != 0u;
             const float* cs = reinterpret_cast<const float*>(smem + Lay::C_OFF + s * Lay::C_STAGE);
             const uint16_t* qs = reinterpret_cast<const uint16_t*>(smem + Lay::Q_OFF + s * Lay::Q_STAGE);
-            float gt[2][4], kap[2][4], qv[2][4];
+            float gt[NT][4], kap[NT][4], qv[NT][4];
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int tk = tok0 + 8 * hf;
                 const float4 z = aux[p * kTcC + tk];  // mu, eta, |x|^2, mu^2
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
+                for (int nt = 0; nt < NT; ++nt) {
                     const int u0 = 2 * nt;  // norm index of slot 8nt + 2cq
-                    const float2 cc = *reinterpret_cast<const float2*>(cs + tk * kRgSlots + 8 * nt + 2 * cq);
-                    const uint32_t q2 = *reinterpret_cast<const uint32_t*>(qs + tk * kRgSlots + 8 * nt + 2 * cq);
+                    const float2 cc = *reinterpret_cast<const float2*>(cs + tk * SPC + 8 * nt + 2 * cq);
+                    const uint32_t q2 = *reinterpret_cast<const uint32_t*>(qs + tk * SPC + 8 * nt + 2 * cq);
                     const float2 pp = make_float2(pr[nt][2 * hf], pr[nt][2 * hf + 1]);
                     const float2 e2 = ptx::f2mul(cc, ptx::f2mul(ptx::f2(z.y), make_float2(inv_n2[u0], inv_n2[u0 + 1])));
                     const float2 pn = ptx::f2mul(pp, make_float2(inv_n[u0], inv_n[u0 + 1]));
@@ -539,9 +567,9 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             }
             // ---- running products over the sub-chunk's 16 tokens (rows g and g+8 of
             // each column): R = inclusive prefix, suf = exclusive suffix, Gs = the total
-            float R[2][4], suf[2][4], Gs[2][2];
+            float R[NT][4], suf[NT][4], Gs[NT][2];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     float rl = gt[nt][j], rh = gt[nt][2 + j];
@@ -568,9 +596,9 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                 }
             // ---- read-out and state-update operands of this sub-chunk
             if (k > 0) tc_wait(bar_p5, (k - 1) & 1, abort);  // G4/G5 of chunk k-1 are done with QR, KD
-            float qrw[2][4];
+            float qrw[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int tk = tok0 + 8 * hf, col = 8 * nt + 2 * cq;
@@ -593,18 +621,17 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                 }
             if (g == 0) {
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    *reinterpret_cast<float2*>(gsub + w * kRgSlots + 8 * nt + 2 * cq) = make_float2(Gs[nt][0], Gs[nt][1]);
+                for (int nt = 0; nt < NT; ++nt)
+                    *reinterpret_cast<float2*>(gsub + w * 16 + 8 * nt + 2 * cq) = make_float2(Gs[nt][0], Gs[nt][1]);
             }
             ptx::named_bar(BAR_C1, kRgChain);  // every sub-chunk's products and KS written
             if (tid == 0) zmu[p] = 0u;         // every chain thread read it before the barrier
             // per slot: the chunk decay A_C and f_b = prod_{c>b} G_c of each sub-chunk b
-            float AC[4], fb[3][4];
+            float AC[2 * NT], fb[3][2 * NT];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 2 * NT; ++u) {
                 const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
-                const float G0 = gsub[sl], G1 = gsub[kRgSlots + sl], G2 = gsub[2 * kRgSlots + sl],
-                            G3 = gsub[3 * kRgSlots + sl];
+                const float G0 = gsub[sl], G1 = gsub[16 + sl], G2 = gsub[32 + sl], G3 = gsub[48 + sl];
                 fb[2][u] = G3;
                 fb[1][u] = G2 * G3;
                 fb[0][u] = G1 * fb[1][u];
@@ -616,7 +643,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             for (int bb = 0; bb < 3; ++bb) {
                 if (bb >= w) break;
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
                         float v[2];
@@ -626,7 +653,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                             float cgb = 1.f;
 #pragma unroll
                             for (int c = 0; c < 4; ++c)
-                                if (c >= bb && c < w) cgb *= gsub[c * kRgSlots + sl];
+                                if (c >= bb && c < w) cgb *= gsub[c * 16 + sl];
                             v[j] = qrw[nt][2 * hf + j] * cgb;
                         }
                         const int tk = tok0 + 8 * hf, col = 8 * nt + 2 * cq;
@@ -637,24 +664,20 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             ptx::named_bar_arrive(BAR_A, N_CM);  // QR, KD and the chunk-start state are ready for G4/G5
 
             // ---- state update: per key sub-chunk bb, U_bb[e][i] = sum_{j in bb} x_j[e] KS_j[i]
-            float ua[4][MT][2][4];
+            float ua[4][MT][NT][4];
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb)
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) ua[bb][mt][nt][i] = 0.f;
             const uint32_t kt_a = sbase + Lay::KT_OFF;
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
-                uint32_t khi[4], klo[4];
-                {   // B: KS rows (tokens) 16bb + 8(lj&1) + lr, slots 8(lj>>1).. at columns 16.. (hi), 32.. (lo)
-                    const int row = 16 * bb + 8 * (lj & 1) + lr;
-                    ptx::ldsm_x4_t(kt_a + row * 128 + (((2 + (lj >> 1)) ^ (row & 7)) << 4), khi);
-                    ptx::ldsm_x4_t(kt_a + row * 128 + (((4 + (lj >> 1)) ^ (row & 7)) << 4), klo);
-                }
+                uint32_t kf[2][NT][2];  // B: KS rows (tokens) 16bb.., hi at columns 16.., lo at 32..
+                load_b_pairs(kt_a, 16 * bb, 16, kf);
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     uint32_t af[4];
@@ -663,10 +686,10 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         const int e = e_base + 16 * mt + 8 * (lj & 1);
                         ptx::ldsm_x4_t(xs_a + (e >> 6) * (64 * 128) + row * 128 + ((((e & 63) >> 3) ^ (row & 7)) << 4), af);
                     }
-                    ptx::mma16816(ua[bb][mt][0], af, khi);
-                    ptx::mma16816(ua[bb][mt][1], af, khi + 2);
-                    ptx::mma16816(ua[bb][mt][0], af, klo);
-                    ptx::mma16816(ua[bb][mt][1], af, klo + 2);
+#pragma unroll
+                    for (int v = 0; v < 2; ++v)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) ptx::mma16816(ua[bb][mt][nt], af, kf[v][nt]);
                 }
             }
             __syncwarp();
@@ -675,7 +698,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int u = 2 * nt + (i & 1);
@@ -692,11 +715,11 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             }
         }
         // final state
-        float* So = a.S_out + ((size_t)bh * (kRgSlots * kRgNC) + rank * kRgSlots) * DS;
+        float* So = a.S_out + ((size_t)bh * kRgM + rank * SPC) * DS;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int e = e_base + 16 * mt + g + 8 * (i >> 1);
@@ -711,26 +734,25 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     if (warp == MMA_WARP) ptx::tmem_dealloc(tmem, Lay::TMEM_COLS);
 }
 
-template <int DS>
+template <int DS, int SPC>
 cudaError_t launch_chunk_reg_t(const ScanArgs& a, cudaStream_t st) {
-    using Lay = RgLayout<DS>;
+    using Lay = RgLayout<DS, SPC>;
     TcMaps maps;
-    const int m = kRgSlots * kRgNC;
     if (!make_map_4d(&maps.x, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DS, a.H, a.T, a.B, 64, true) ||
-        !make_map_4d(&maps.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, m, a.H, a.T, a.B, kRgSlots, false) ||
-        !make_map_4d(&maps.c, a.c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, m, a.H, a.T, a.B, kRgSlots, false))
+        !make_map_4d(&maps.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kRgM, a.H, a.T, a.B, SPC, false) ||
+        !make_map_4d(&maps.c, a.c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kRgM, a.H, a.T, a.B, SPC, false))
         return cudaErrorInvalidValue;
-    auto k = chunk_reg_kernel<DS>;
+    auto k = chunk_reg_kernel<DS, SPC>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.B * a.H * kRgNC);
+    cfg.gridDim = dim3(a.B * a.H * Lay::NC);
     cfg.blockDim = dim3(kRgThreads);
     cfg.dynamicSmemBytes = Lay::SMEM_ALLOC;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kRgNC;
+    attr[0].val.clusterDim.x = Lay::NC;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -740,10 +762,45 @@ cudaError_t launch_chunk_reg_t(const ScanArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-inline cudaError_t launch_chunk_reg(const ScanArgs& a, int d, cudaStream_t st) {
-    if (a.m != kRgSlots * kRgNC) return cudaErrorNotSupported;
-    if (d == 128) return launch_chunk_reg_t<128>(a, st);
-    if (d == 64) return launch_chunk_reg_t<64>(a, st);
+// Clusters of the kernel with `spc` slots per CTA (8 or 16) that the current device can
+// hold at once (each cluster takes 64/spc SMs of one GPC); 0 if the query fails.
+template <int DS, int SPC>
+int chunk_reg_max_clusters_t() {
+    using Lay = RgLayout<DS, SPC>;
+    auto k = chunk_reg_kernel<DS, SPC>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM_ALLOC) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(Lay::NC * 64);
+    cfg.blockDim = dim3(kRgThreads);
+    cfg.dynamicSmemBytes = Lay::SMEM_ALLOC;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = Lay::NC;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+inline int chunk_reg_max_clusters(int d, int spc) {
+    if (d == 128) return spc == 8 ? chunk_reg_max_clusters_t<128, 8>() : chunk_reg_max_clusters_t<128, 16>();
+    if (d == 64) return spc == 8 ? chunk_reg_max_clusters_t<64, 8>() : chunk_reg_max_clusters_t<64, 16>();
+    return 0;
+}
+
+inline cudaError_t launch_chunk_reg(const ScanArgs& a, int d, int spc, cudaStream_t st) {
+    if (a.m != kRgM || (spc != 8 && spc != 16)) return cudaErrorNotSupported;
+    if (d == 128) return spc == 8 ? launch_chunk_reg_t<128, 8>(a, st) : launch_chunk_reg_t<128, 16>(a, st);
+    if (d == 64) return spc == 8 ? launch_chunk_reg_t<64, 8>(a, st) : launch_chunk_reg_t<64, 16>(a, st);
     return cudaErrorNotSupported;
 }
 

@@ -312,7 +312,8 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
     if (B < 1 || H < 1 || m < 1 || d < 1 || T < 0 || chunk_size < 1) return LATTICE_ERR_INVALID_ARG;
     if (!dtype_ok(x_dtype) || !dtype_ok(q_dtype)) return LATTICE_ERR_INVALID_ARG;
     if (impl != LATTICE_IMPL_AUTO && impl != LATTICE_IMPL_SIMT && impl != LATTICE_IMPL_TCGEN05 &&
-        impl != LATTICE_IMPL_TCGEN05_SPLIT && impl != LATTICE_IMPL_SPLIT_REG)
+        impl != LATTICE_IMPL_TCGEN05_SPLIT && impl != LATTICE_IMPL_SPLIT_REG &&
+        impl != LATTICE_IMPL_SPLIT_REG8)
         return LATTICE_ERR_INVALID_ARG;
     if (mode != LATTICE_SIM && mode != LATTICE_DEC) return LATTICE_ERR_INVALID_ARG;
     const bool dec = mode == LATTICE_DEC;
@@ -347,7 +348,7 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
     ScanArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, S_out, y,
                B, T, H, m, chunk_size};
     const bool tc_choice = impl == LATTICE_IMPL_TCGEN05 || impl == LATTICE_IMPL_TCGEN05_SPLIT ||
-                           impl == LATTICE_IMPL_SPLIT_REG;
+                           impl == LATTICE_IMPL_SPLIT_REG || impl == LATTICE_IMPL_SPLIT_REG8;
     a.cnorm = cnorm && chunk_size > 1 ? 1 : 0;
     if (chunk_size == 1 && cnorm) {  // normalising after every token is the exact recurrence
         if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
@@ -359,9 +360,9 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
                                : launch_scan_simt<true>(a, d, dec, lin1, st);
     }
     if (impl == LATTICE_IMPL_AUTO) impl = lattice_chunk_impl(B, H, m, d, chunk_size, x_dtype, q_dtype);
-    if (impl == LATTICE_IMPL_SPLIT_REG) {
+    if (impl == LATTICE_IMPL_SPLIT_REG || impl == LATTICE_IMPL_SPLIT_REG8) {
         if (!chunk_reg_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
-        cudaError_t e = launch_chunk_reg(a, d, st);
+        cudaError_t e = launch_chunk_reg(a, d, impl == LATTICE_IMPL_SPLIT_REG8 ? 8 : 16, st);
         return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
     }
     if (impl == LATTICE_IMPL_TCGEN05_SPLIT) {

@@ -120,7 +120,8 @@ def test_empty_sequence_copies_state(L):
 
 
 @pytest.mark.parametrize("chunk,T1,impl", [(1, 13, "simt"), (64, 128, "simt"), (64, 128, "tcgen05"),
-                                           (64, 128, "tcgen05_split"), (64, 128, "split_reg")])
+                                           (64, 128, "tcgen05_split"), (64, 128, "split_reg"),
+                                           (64, 128, "split_reg8")])
 def test_resume(L, chunk, T1, impl):
     """scan(T1) then scan(T2) from the carried state equals scan(T1 + T2):
     bitwise on CUDA cores; within the bf16 tolerance on tensor cores, which
@@ -146,7 +147,7 @@ def test_resume(L, chunk, T1, impl):
 
 
 @pytest.mark.parametrize("m,chunk,impl", [(128, 1, "auto"), (128, 64, "tcgen05"), (64, 64, "tcgen05_split"),
-                                          (64, 64, "split_reg")])
+                                          (64, 64, "split_reg"), (64, 64, "split_reg8")])
 def test_deterministic(L, m, chunk, impl):
     """Repeated calls give bitwise-equal results (every reduction has a fixed order,
     the cluster read-out reduction included)."""
@@ -186,7 +187,8 @@ def test_chunked_tcgen05(L, m, d, T):
     assert s_err(Sg, So) <= TOL_TC
 
 
-@pytest.mark.parametrize("m,impl", [(128, "tcgen05"), (64, "tcgen05_split"), (64, "split_reg")])
+@pytest.mark.parametrize("m,impl", [(128, "tcgen05"), (64, "tcgen05_split"), (64, "split_reg"),
+                                    (64, "split_reg8")])
 def test_chunked_tcgen05_eta_and_gate_edges(L, m, impl):
     """eta given, mu = 1 and mu = 0 tokens, a token with mu = 0 and no write (a
     zero-norm update keeps every slot), zero intensities, duplicates."""
@@ -207,7 +209,7 @@ def test_chunked_tcgen05_eta_and_gate_edges(L, m, impl):
 
 # ------------------------------- chunked (Eq. 17), slots split over a cluster
 
-@pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg"])
+@pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg", "split_reg8"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("T", [1, 64, 2 * 64 + 37, 5 * 64])
 def test_chunked_tcgen05_split(L, d, T, impl):
@@ -221,7 +223,7 @@ def test_chunked_tcgen05_split(L, d, T, impl):
     assert s_err(Sg, So) <= TOL_TC
 
 
-@pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg"])
+@pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg", "split_reg8"])
 def test_chunked_split_and_wide_agree(L, impl):
     """The tensor-core kernels compute the same chunked form."""
     w = LI.Workload("t", B=3, T=700, H=2, m=64, d=128, seed=12)
@@ -320,7 +322,7 @@ def test_full_size_chunked_every_head(L, name):
     w = LI.WORKLOADS[name]
     inp = LI.make_inputs(w)
     yo, So = oracle_every_head(inp, w, w.chunk)
-    impls = ["auto", "simt", "tcgen05"] + (["tcgen05_split", "split_reg"] if w.m == 64 else [])
+    impls = ["auto", "simt", "tcgen05"] + (["tcgen05_split", "split_reg", "split_reg8"] if w.m == 64 else [])
     for impl in impls:
         yg, Sg = run_gpu(L, inp, w.chunk, impl=impl)
         assert y_err(yg, yo) <= TOL_TC, impl
@@ -449,7 +451,7 @@ def test_dec_step_resynchronised(L, m, d):
 def test_dec_tensor_core_choices_are_unsupported(L):
     w = LI.Workload("t", B=1, T=4, H=1, m=64, d=64, seed=1)
     inp = LI.make_inputs(w)
-    for impl in ("tcgen05", "tcgen05_split", "split_reg"):
+    for impl in ("tcgen05", "tcgen05_split", "split_reg", "split_reg8"):
         with pytest.raises(L.LatticeError):
             run_gpu(L, inp, 64, impl=impl, mode="dec")
     yg, _ = run_gpu(L, inp, 64, mode="dec")  # AUTO takes the CUDA-core kernel
@@ -514,7 +516,7 @@ def test_lin1_dec_resynchronised(L):
 def test_lin1_tensor_core_choices_are_unsupported(L):
     w = LI.Workload("t", B=1, T=64, H=1, m=64, d=64, seed=1)
     inp = LI.make_inputs(w)
-    for impl in ("tcgen05", "tcgen05_split", "split_reg"):
+    for impl in ("tcgen05", "tcgen05_split", "split_reg", "split_reg8"):
         with pytest.raises(L.LatticeError):
             run_gpu(L, inp, 64, impl=impl, lin=1)
 
@@ -554,7 +556,7 @@ def test_chunk_norm_chunk_one_is_exact_and_tensor_cores_refuse(L):
     y1, S1 = run_gpu(L, inp, 1, norm="chunk")
     ye, Se = run_oracle(inp, 1)
     assert y_err(y1, ye) <= TOL_F32 and s_err(S1, Se) <= TOL_F32
-    for impl in ("tcgen05", "tcgen05_split", "split_reg"):
+    for impl in ("tcgen05", "tcgen05_split", "split_reg", "split_reg8"):
         with pytest.raises(L.LatticeError):
             run_gpu(L, inp, 64, impl=impl, norm="chunk")
 
