@@ -102,7 +102,7 @@ typedef enum { LATTICE_SIM = 0, LATTICE_DEC = 1 } lattice_mode;
  *                   state held in registers and advanced chunk to chunk by
  *                   warp-synchronous tensor-core MMAs (mma.sync), which keeps the
  *                   per-chunk dependency chain off every asynchronous round trip
- *                   (chunk 64, bf16 x and q, m = 64, d in {64, 128}).
+ *                   (chunk 64 or 16, bf16 x and q, m = 64, d in {64, 128}).
  *   SPLIT_REG8      as SPLIT_REG with 8 slots per CTA over a cluster of 8 CTAs:
  *                   half the tensor work on each CTA's chain; needs B*H clusters
  *                   of 8 SMs within one GPC each.

@@ -47,39 +47,45 @@ constexpr int kRgM = 64;                        // slots per sequence
 constexpr int kRgChain = 128;                   // 4 chain warps
 constexpr int kRgReadout = 128;                 // 4 read-out warps
 constexpr int kRgThreads = kRgChain + kRgReadout + 64;  // + MMA warp + TMA warp
-constexpr int kRgStages = 4;                    // x/q/c ring depth (chunks)
 
 inline bool chunk_reg_supported(int m, int d, int chunk, bool x_bf16, bool q_bf16) {
-    return chunk == kTcC && x_bf16 && q_bf16 && m == kRgM && (d == 64 || d == 128);
+    return (chunk == kTcC || chunk == 16) && x_bf16 && q_bf16 && m == kRgM && (d == 64 || d == 128);
 }
 
-// SPC slots per CTA (16: clusters of 4 CTAs; 8: clusters of 8), state width DS.
-template <int DS, int SPC>
+// SPC slots per CTA (16: clusters of 4 CTAs; 8: clusters of 8), state width DS, chunk
+// size CH (64, or 16: four chunks per 64-token ring stage and read-out round).
+template <int DS, int SPC, int CH>
 struct RgLayout {
     static_assert(SPC == 8 || SPC == 16, "8 or 16 slots per CTA");
+    static_assert(CH == 64 || CH == 16, "chunk size 64 or 16");
+    static constexpr int NST = (CH == 16 && DS == 128) ? 3 : 4;  // x/q/c ring depth (stages of 64 tokens)
     static constexpr int NC = kRgM / SPC;                  // CTAs per sequence (cluster size)
     static constexpr int DSL = DS / NC;                    // y columns reduced by each CTA
     static constexpr uint32_t X_STAGE = DS * 128;          // [C][d] bf16 in d/64 SW128 blocks
     static constexpr uint32_t Q_STAGE = kTcC * SPC * 2;    // [C][SPC] bf16
     static constexpr uint32_t C_STAGE = kTcC * SPC * 4;    // [C][SPC] fp32
     static constexpr uint32_t X_OFF = 0;
-    static constexpr uint32_t Q_OFF = X_OFF + kRgStages * X_STAGE;
-    static constexpr uint32_t C_OFF = Q_OFF + kRgStages * Q_STAGE;
+    static constexpr uint32_t Q_OFF = X_OFF + NST * X_STAGE;
+    static constexpr uint32_t C_OFF = Q_OFF + NST * Q_STAGE;
     // chunk-start state, double-buffered by chunk parity: [d rows = state column e][128 B],
     // the slots' hi parts at columns 0..SPC-1, lo parts at 16..16+SPC-1 (SW128); the
     // columns up to 16 stay zero (the read-out GEMM takes K = 16)
     static constexpr uint32_t S0_BUF = DS * 128;
-    static constexpr uint32_t S0_OFF = C_OFF + kRgStages * C_STAGE;
-    static constexpr uint32_t QR_OFF = S0_OFF + 2 * S0_BUF;     // [C][128 B]: QR_b at columns 16b..
+    static constexpr uint32_t S0_OFF = C_OFF + NST * C_STAGE;
+    // C = 16: the read-out's stacked chunk-start states of a stage, double-buffered by
+    // stage parity: [d rows][128 B], chunk c's hi part at columns 16c..16c+SPC-1
+    static constexpr uint32_t S0ST_OFF = S0_OFF + 2 * S0_BUF;
+    static constexpr int S0_TILES = CH == 16 ? 4 : 2;
+    static constexpr uint32_t QR_OFF = S0_OFF + S0_TILES * S0_BUF;  // [C][128 B]: QR_b at columns 16b..
     static constexpr uint32_t KT_OFF = QR_OFF + kTcC * 128;     // [C][128 B]: KD at 0.., KS hi at 16.., lo at 32..
     static constexpr uint32_t P_OFF = KT_OFF + kTcC * 128;      // [C][C] bf16 masked scores
     static constexpr uint32_t RECV_OFF = P_OFF + kTcC * 128;    // [2][NC][C][d/NC] fp32
     static constexpr uint32_t RECV_BYTES = 2 * NC * kTcC * DSL * 4;
     static constexpr uint32_t AUX_OFF = RECV_OFF + RECV_BYTES;  // [2][C] float4: mu, eta, |x|^2, mu^2
     static constexpr uint32_t GSUB_OFF = AUX_OFF + 2 * kTcC * 16;   // [4 sub-chunks][16] (SPC used)
-    static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * 16 * 4;        // [4 warps][16] (SPC used)
-    static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * 16 * 4;
-    static constexpr int NBAR = 2 * kRgStages + 8;
+    static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * 16 * 4;        // [2][4 warps][16] (SPC used)
+    static constexpr uint32_t BAR_OFF = TSQ_OFF + 2 * 4 * 16 * 4;
+    static constexpr int NBAR = 2 * NST + 8;
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr uint32_t BYTES = MISC_OFF + 64;
     static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;
@@ -93,14 +99,14 @@ struct RgLayout {
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-template <int DS, int SPC>
+template <int DS, int SPC, int CH>
 __global__ void __launch_bounds__(kRgThreads, 1)
     chunk_reg_kernel(const __grid_constant__ TcMaps maps, ScanArgs a) {
-    using Lay = RgLayout<DS, SPC>;
+    using Lay = RgLayout<DS, SPC, CH>;
     constexpr int DSL = Lay::DSL;
     constexpr int NC = Lay::NC;
     constexpr int NT = SPC / 8;  // 8-slot n-tiles per CTA
-    constexpr int NST = kRgStages;
+    constexpr int NST = Lay::NST;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -109,7 +115,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     const int rank = (int)ptx::cluster_ctarank();
     const int bh = blockIdx.x / NC, b = bh / a.H, h = bh % a.H;
     const int T = a.T, H = a.H;
-    const int nch = (T + kTcC - 1) / kTcC;
+    const int nch = (T + kTcC - 1) / kTcC;  // ring stages of 64 tokens (chunks when C = 64)
     constexpr int RO_WARP0 = kRgChain / 32, MMA_WARP = RO_WARP0 + 4, TMA_WARP = MMA_WARP + 1;
 
     // mbarriers: ring stage full [NST] (TMA bytes) and empty [NST] (4 chain warps + the
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         auto off = [](uint32_t bytes) { return uint64_t(bytes >> 4); };
         const uint64_t dK_qr = ptx::sdesc_sw128(sbase + Lay::QR_OFF, 16, 1024);
         const uint64_t dK_kd = ptx::sdesc_sw128(sbase + Lay::KT_OFF, 16, 1024);
-        const uint64_t dK_s0 = ptx::sdesc_sw128(sbase + Lay::S0_OFF, 16, 1024);
+        const uint64_t dK_s0 = ptx::sdesc_sw128(sbase + (CH == 64 ? Lay::S0_OFF : Lay::S0ST_OFF), 16, 1024);
         const uint64_t dK_p = ptx::sdesc_sw128(sbase + Lay::P_OFF, 16, 1024);
         const uint64_t dM_x = ptx::sdesc_sw128(sbase + Lay::X_OFF, 64 * 128, 1024);
         for (int k = 0; k < nch; ++k) {
@@ -184,8 +190,16 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             const bool yfree = k < 2 || tc_wait_warp(bar_yfree0 + 8 * p, ((k - 2) >> 1) & 1, abort);
             ptx::tc_fence_after();
             if (yfree && tc_live(abort)) {
-                // G4: Y_r = QR_0 . S0hi  (M = C, N = d, K = 16); both K-major
-                ptx::mma_bf16_elect(tmem + ycol, dK_qr, dK_s0 + off(p * Lay::S0_BUF), idesc_g4, 0);
+                if constexpr (CH == 64) {
+                    // G4: Y_r = QR_0 . S0hi  (M = C, N = d, K = 16); both K-major
+                    ptx::mma_bf16_elect(tmem + ycol, dK_qr, dK_s0 + off(p * Lay::S0_BUF), idesc_g4, 0);
+                } else {
+                    // G4: Y_r = QR_bd . S0stack  (K = 64: chunk c's rows of QR meet chunk c's start state)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        ptx::mma_bf16_elect(tmem + ycol, dK_qr + off(32 * kk), dK_s0 + off(p * Lay::S0_BUF + 32 * kk),
+                                            idesc_g4, kk > 0);
+                }
                 // G5: P[:, 16b..16b+15] = QR_b . KD_b^T  (M = C, N = 16, K = 16)
 #pragma unroll
                 for (int sb = 0; sb < 4; ++sb)
@@ -380,19 +394,19 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         if (nch > 0) recv_y(nch - 1);
     } else {
         // ================================================================ chain warps
-        // Warp w: the projections and gates of tokens 16w..16w+15 (sub-chunk w), and the
-        // state columns w*d/4..(w+1)*d/4 in the update. Fragment coordinates: g = lane/4
-        // (a row: a token, or a state column), cq = lane%4 (a pair of slots 2cq, 2cq+1 of
-        // each 8-slot n-tile nt); index i of a 4-register fragment is (row g + 8(i/2),
-        // slot 8nt + 2cq + i%2).
+        // Fragment coordinates: g = lane/4 (a row: a token, or a state column), cq = lane%4
+        // (a pair of slots 2cq, 2cq+1 of each 8-slot n-tile nt); index i of a 4-register
+        // fragment is (row g + 8(i/2), slot 8nt + 2cq + i%2). Warp w owns the state columns
+        // w*d/4..(w+1)*d/4 in the update; with C = 64 it also owns the projections and gates
+        // of sub-chunk w (tokens 16w..16w+15).
         const int w = warp;
         const int g = lane >> 2, cq = lane & 3;
-        const int tok0 = 16 * w + g;                  // rows g and g+8 of the warp's tile
         constexpr int MT = DS / 64;                   // 16-column m-tiles of the update per warp
         const int e_base = w * (DS / 4);
         const int lj = lane >> 3, lr = lane & 7;      // ldmatrix: matrix lj, row lr
         uint8_t* qr = smem + Lay::QR_OFF;
         uint8_t* kt = smem + Lay::KT_OFF;
+        const uint32_t kt_a = sbase + Lay::KT_OFF;
 
         // fp32 state: st[mt][nt][i] = s_{slot}[e], e = e_base + 16mt + g + 8(i/2)
         float st[MT][NT][4];
@@ -409,10 +423,12 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         st[mt][nt][i] = S0g[(size_t)sl * DS + e];
                     }
         }
-        // the state as the next chunk's operand: hi/lo bf16 into S0 buffer p, and each
-        // slot's partial |s|^2 over this warp's columns into tsq[w]
-        auto write_state = [&](int p) {
-            uint8_t* dst = smem + Lay::S0_OFF + p * Lay::S0_BUF;
+        // the state as the next chunk's operand: hi/lo bf16 into S0 buffer pb (and, with
+        // C = 16, its hi part into the read-out's stacked-state tile sto at column scol),
+        // and each slot's partial |s|^2 over this warp's columns into tsq[pb][w] (double
+        // buffered: a warp may start the next chunk before the others have read them)
+        auto write_state = [&](int pb, uint8_t* sto, int scol) {
+            uint8_t* dst = smem + Lay::S0_OFF + pb * Lay::S0_BUF;
             float ns[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) ns[nt][0] = ns[nt][1] = 0.f;
@@ -429,6 +445,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         const int col = 8 * nt + 2 * cq;
                         *reinterpret_cast<uint32_t*>(dst + ptx::sw128_off(e, col)) = hi;
                         *reinterpret_cast<uint32_t*>(dst + ptx::sw128_off(e, 16 + col)) = lo;
+                        if (CH == 16) *reinterpret_cast<uint32_t*>(sto + ptx::sw128_off(e, scol + col)) = hi;
                         ns[nt][0] = fmaf(v.x, v.x, ns[nt][0]);
                         ns[nt][1] = fmaf(v.y, v.y, ns[nt][1]);
                     }
@@ -440,22 +457,21 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                     v += __shfl_xor_sync(0xffffffffu, v, 4);
                     v += __shfl_xor_sync(0xffffffffu, v, 8);
                     v += __shfl_xor_sync(0xffffffffu, v, 16);
-                    if (g == 0) tsq[w * 16 + 8 * nt + 2 * cq + j] = v;
+                    if (g == 0) tsq[pb * 64 + w * 16 + 8 * nt + 2 * cq + j] = v;
                 }
         };
         // n = |s0|, 1/n, 1/n^2 of this thread's slots (index 2nt + j: slot 8nt + 2cq + j)
         float nrm[2 * NT], inv_n[2 * NT], inv_n2[2 * NT];
-        auto load_norms = [&]() {
+        auto load_norms = [&](int pb) {
 #pragma unroll
             for (int u = 0; u < 2 * NT; ++u) {
-                const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
-                const float nsq = ((tsq[sl] + tsq[16 + sl]) + tsq[32 + sl]) + tsq[48 + sl];
+                const float* t4 = tsq + pb * 64 + 8 * (u >> 1) + 2 * cq + (u & 1);
+                const float nsq = ((t4[0] + t4[16]) + t4[32]) + t4[48];
                 inv_n[u] = ptx::rsqrt_nr(nsq);
                 nrm[u] = nsq * inv_n[u];
                 inv_n2[u] = inv_n[u] * inv_n[u];
             }
         };
-
         // B fragments (k = 16 rows from row0, n = 8 slots per n-tile) of a hi/lo operand pair
         // stored row-major in an SW128 tile: hi slots at columns col0 + 8nt, lo at col0 + 16 + 8nt.
         // ldmatrix.trans turns the stored [k][n] rows into the fragment layout.
@@ -473,26 +489,9 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                 bfr[0][0][0] = r4[0]; bfr[0][0][1] = r4[1]; bfr[1][0][0] = r4[2]; bfr[1][0][1] = r4[3];
             }
         };
-
-        // ---- prologue: operand tiles zeroed (the blocks of later sub-chunks in the query
-        // tile, and with 8 slots per CTA the K padding up to 16, are never written)
-        for (int o = tid; o < int(kTcC * 128 / 16); o += kRgChain) {
-            reinterpret_cast<uint4*>(qr)[o] = make_uint4(0u, 0u, 0u, 0u);
-            reinterpret_cast<uint4*>(kt)[o] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        for (int o = tid; o < int(2 * Lay::S0_BUF / 16); o += kRgChain)
-            reinterpret_cast<uint4*>(smem + Lay::S0_OFF)[o] = make_uint4(0u, 0u, 0u, 0u);
-        ptx::named_bar(BAR_C2, kRgChain);
-        write_state(0);
-        ptx::named_bar(BAR_C2, kRgChain);
-        load_norms();
-
-        for (int k = 0; k < nch; ++k) {
-            const int s = k % NST, p = k & 1;
-            tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
-            const uint32_t xs_a = sbase + Lay::X_OFF + s * Lay::X_STAGE;
-            const uint32_t s0_a = sbase + Lay::S0_OFF + p * Lay::S0_BUF;
-            // ---- projection D[t][i] = x_t . (s0hi_i + s0lo_i), tokens 16w..16w+15
+        // projections D[t][i] = x_t . (s0hi_i + s0lo_i) of the 16 tokens at stage rows
+        // row0..row0+15, all the CTA's slots; pr[nt][i] in the fragment layout
+        auto project = [&](uint32_t xs_a, uint32_t s0_a, int row0, float (&pr)[NT][4]) {
             float acc[2][2][NT][4];  // [k-step parity][hi, lo][nt][i]
 #pragma unroll
             for (int u = 0; u < 2; ++u)
@@ -504,37 +503,35 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         for (int i = 0; i < 4; ++i) acc[u][v][nt][i] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < DS / 16; ++ks) {
-                uint32_t af[4], bf[2][NT][2];  // B fragments [hi, lo][nt]
-                {   // A: x rows 16w + 8(lj&1) + lr, columns 16ks + 8(lj>>1)
-                    const int row = 16 * w + 8 * (lj & 1) + lr;
+                uint32_t af[4], bf[2][NT][2];
+                {   // A: x rows row0 + 8(lj&1) + lr, columns 16ks + 8(lj>>1)
+                    const int row = row0 + 8 * (lj & 1) + lr;
                     const int col = 16 * ks + 8 * (lj >> 1);
                     ptx::ldsm_x4(xs_a + (col >> 6) * (64 * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4), af);
                 }
-                // B: state rows e = 16ks + 8(lj&1) + lr, slots 8nt.. (hi at column 0, lo at 16)
-                load_b_pairs(s0_a, 16 * ks, 0, bf);
+                load_b_pairs(s0_a, 16 * ks, 0, bf);  // the state rows e = 16ks..16ks+15
 #pragma unroll
                 for (int v = 0; v < 2; ++v)
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) ptx::mma16816(acc[ks & 1][v][nt], af, bf[v][nt]);
             }
-            float pr[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     pr[nt][i] = (acc[0][0][nt][i] + acc[1][0][nt][i]) + (acc[0][1][nt][i] + acc[1][1][nt][i]);
-
-            // ---- gates of Eq. 17 (eq. beta_chunk with the chunk-start norm n):
-            //   e2 = eta c / n^2, pn = p / n, den = mu^2 + e2^2 max(|x|^2 - pn^2, 0),
-            //   g = (mu - e2 pn) / sqrt(den), kappa / n = e2 / sqrt(den); den = 0 keeps the slot
-            tc_wait(bar_aux0 + 8 * p, (k >> 1) & 1, abort);  // per-token inputs of chunk k
-            const bool zero_mu = zmu[p] != 0u;
+        };
+        // gates of Eq. 17 (eq. beta_chunk with the chunk-start norm n) of the 16 tokens at
+        // rows row0.. of ring stage s (per-token inputs in aux buffer p):
+        //   e2 = eta c / n^2, pn = p / n, den = mu^2 + e2^2 max(|x|^2 - pn^2, 0),
+        //   g = (mu - e2 pn) / sqrt(den), kappa = n e2 / sqrt(den); den = 0 keeps the slot
+        auto gates = [&](const float (&pr)[NT][4], int s, int p, int row0, bool zero_mu, float (&gt)[NT][4],
+                         float (&kap)[NT][4], float (&qv)[NT][4]) {
             const float* cs = reinterpret_cast<const float*>(smem + Lay::C_OFF + s * Lay::C_STAGE);
             const uint16_t* qs = reinterpret_cast<const uint16_t*>(smem + Lay::Q_OFF + s * Lay::Q_STAGE);
-            float gt[NT][4], kap[NT][4], qv[NT][4];
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const int tk = tok0 + 8 * hf;
+                const int tk = row0 + g + 8 * hf;
                 const float4 z = aux[p * kTcC + tk];  // mu, eta, |x|^2, mu^2
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -565,9 +562,10 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                     qv[nt][2 * hf + 1] = __uint_as_float(q2 & 0xffff0000u);
                 }
             }
-            // ---- running products over the sub-chunk's 16 tokens (rows g and g+8 of
-            // each column): R = inclusive prefix, suf = exclusive suffix, Gs = the total
-            float R[NT][4], suf[NT][4], Gs[NT][2];
+        };
+        // running products over 16 tokens (rows g and g+8 of each column): R = inclusive
+        // prefix, suf = exclusive suffix, Gs = the total
+        auto scans = [&](const float (&gt)[NT][4], float (&R)[NT][4], float (&suf)[NT][4], float (&Gs)[NT][2]) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -594,14 +592,18 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                     suf[nt][2 + j] = g < 7 ? nh : 1.f;  // prod of rows g+9..15
                     Gs[nt][j] = __shfl_sync(0xffffffffu, rh, 28 + cq);
                 }
-            // ---- read-out and state-update operands of this sub-chunk
-            if (k > 0) tc_wait(bar_p5, (k - 1) & 1, abort);  // G4/G5 of chunk k-1 are done with QR, KD
-            float qrw[NT][4];
+        };
+        // KD = kappa / R (R clamped away from zero, sign kept) and KS = kappa suf (hi + lo)
+        // of the fragment's rows into the KT tile, rows kd_row0.. and ks_row0..; the
+        // query operand q R into the QR tile at rows qr_row0.., columns qcol.. (unless null)
+        auto write_operands = [&](const float (&kap)[NT][4], const float (&R)[NT][4], const float (&suf)[NT][4],
+                                  const float (&qv)[NT][4], int kd_row0, int ks_row0, int qcol, float (&qrw)[NT][4],
+                                  bool write_kd_qr) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    const int tk = tok0 + 8 * hf, col = 8 * nt + 2 * cq;
+                    const int col = 8 * nt + 2 * cq;
                     float kd[2], ks[2];
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
@@ -613,105 +615,198 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                     }
                     uint32_t khi, klo;
                     split2(make_float2(ks[0], ks[1]), khi, klo);
-                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(tk, col)) = ptx::pack_bf16x2(kd[0], kd[1]);
-                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(tk, 16 + col)) = khi;
-                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(tk, 32 + col)) = klo;
-                    *reinterpret_cast<uint32_t*>(qr + ptx::sw128_off(tk, 16 * w + col)) =
-                        ptx::pack_bf16x2(qrw[nt][2 * hf], qrw[nt][2 * hf + 1]);
-                }
-            if (g == 0) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    *reinterpret_cast<float2*>(gsub + w * 16 + 8 * nt + 2 * cq) = make_float2(Gs[nt][0], Gs[nt][1]);
-            }
-            ptx::named_bar(BAR_C1, kRgChain);  // every sub-chunk's products and KS written
-            if (tid == 0) zmu[p] = 0u;         // every chain thread read it before the barrier
-            // per slot: the chunk decay A_C and f_b = prod_{c>b} G_c of each sub-chunk b
-            float AC[2 * NT], fb[3][2 * NT];
-#pragma unroll
-            for (int u = 0; u < 2 * NT; ++u) {
-                const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
-                const float G0 = gsub[sl], G1 = gsub[16 + sl], G2 = gsub[32 + sl], G3 = gsub[48 + sl];
-                fb[2][u] = G3;
-                fb[1][u] = G2 * G3;
-                fb[0][u] = G1 * fb[1][u];
-                AC[u] = G0 * fb[0][u];
-            }
-            // query operands of the earlier key blocks bb < w for this warp's tokens:
-            // QR_bb(t) = QR_w(t) prod_{c=bb..w-1} G_c
-#pragma unroll
-            for (int bb = 0; bb < 3; ++bb) {
-                if (bb >= w) break;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        float v[2];
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const int sl = 8 * nt + 2 * cq + j;
-                            float cgb = 1.f;
-#pragma unroll
-                            for (int c = 0; c < 4; ++c)
-                                if (c >= bb && c < w) cgb *= gsub[c * 16 + sl];
-                            v[j] = qrw[nt][2 * hf + j] * cgb;
-                        }
-                        const int tk = tok0 + 8 * hf, col = 8 * nt + 2 * cq;
-                        *reinterpret_cast<uint32_t*>(qr + ptx::sw128_off(tk, 16 * bb + col)) = ptx::pack_bf16x2(v[0], v[1]);
+                    const int rs = ks_row0 + g + 8 * hf;
+                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(rs, 16 + col)) = khi;
+                    *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(rs, 32 + col)) = klo;
+                    if (write_kd_qr) {
+                        const int rk = kd_row0 + g + 8 * hf;
+                        *reinterpret_cast<uint32_t*>(kt + ptx::sw128_off(rk, col)) = ptx::pack_bf16x2(kd[0], kd[1]);
+                        *reinterpret_cast<uint32_t*>(qr + ptx::sw128_off(rk, qcol + col)) =
+                            ptx::pack_bf16x2(qrw[nt][2 * hf], qrw[nt][2 * hf + 1]);
                     }
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_arrive(BAR_A, N_CM);  // QR, KD and the chunk-start state are ready for G4/G5
-
-            // ---- state update: per key sub-chunk bb, U_bb[e][i] = sum_{j in bb} x_j[e] KS_j[i]
-            float ua[4][MT][NT][4];
+                }
+        };
+        // U[e][i] += sum_{tokens j of stage rows row0..row0+15} x_j[e] KS_j[i] for this warp's
+        // columns, KS from the KT tile rows ks_row0.. (B), x^T from the stage (A)
+        auto update_mma = [&](uint32_t xs_a, int row0, int ks_row0, float (&u)[MT][NT][4]) {
+            uint32_t kf[2][NT][2];
+            load_b_pairs(kt_a, ks_row0, 16, kf);
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb)
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t af[4];
+                {   // A = X^T: x rows row0 + 8(lj>>1) + lr, columns e = e_base + 16mt + 8(lj&1)
+                    const int row = row0 + 8 * (lj >> 1) + lr;
+                    const int e = e_base + 16 * mt + 8 * (lj & 1);
+                    ptx::ldsm_x4_t(xs_a + (e >> 6) * (64 * 128) + row * 128 + ((((e & 63) >> 3) ^ (row & 7)) << 4), af);
+                }
+#pragma unroll
+                for (int v = 0; v < 2; ++v)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) ptx::mma16816(u[mt][nt], af, kf[v][nt]);
+            }
+        };
+
+        // ---- prologue: operand tiles zeroed (blocks of the query tile that are never
+        // written, and with 8 slots per CTA the K padding up to 16)
+        for (int o = tid; o < int(kTcC * 128 / 16); o += kRgChain) {
+            reinterpret_cast<uint4*>(qr)[o] = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4*>(kt)[o] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (int o = tid; o < int(Lay::S0_TILES * Lay::S0_BUF / 16); o += kRgChain)
+            reinterpret_cast<uint4*>(smem + Lay::S0_OFF)[o] = make_uint4(0u, 0u, 0u, 0u);
+        ptx::named_bar(BAR_C2, kRgChain);
+        write_state(0, smem + Lay::S0ST_OFF, 0);
+        ptx::named_bar(BAR_C2, kRgChain);
+        load_norms(0);
+
+        if constexpr (CH == 64) {
+            const int tok0 = 16 * w;  // this warp's sub-chunk
+            for (int k = 0; k < nch; ++k) {
+                const int s = k % NST, p = k & 1;
+                tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
+                const uint32_t xs_a = sbase + Lay::X_OFF + s * Lay::X_STAGE;
+                float pr[NT][4];
+                project(xs_a, sbase + Lay::S0_OFF + p * Lay::S0_BUF, tok0, pr);
+                tc_wait(bar_aux0 + 8 * p, (k >> 1) & 1, abort);  // per-token inputs of chunk k
+                float gt[NT][4], kap[NT][4], qv[NT][4], R[NT][4], suf[NT][4], Gs[NT][2], qrw[NT][4];
+                gates(pr, s, p, tok0, zmu[p] != 0u, gt, kap, qv);
+                scans(gt, R, suf, Gs);
+                if (k > 0) tc_wait(bar_p5, (k - 1) & 1, abort);  // G4/G5 of chunk k-1 are done with QR, KD
+                write_operands(kap, R, suf, qv, tok0, tok0, 16 * w, qrw, true);
+                if (g == 0) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        *reinterpret_cast<float2*>(gsub + w * 16 + 8 * nt + 2 * cq) = make_float2(Gs[nt][0], Gs[nt][1]);
+                }
+                ptx::named_bar(BAR_C1, kRgChain);  // every sub-chunk's products and KS written
+                if (tid == 0) zmu[p] = 0u;         // every chain thread read it before the barrier
+                // per slot: the chunk decay A_C and f_b = prod_{c>b} G_c of each sub-chunk b
+                float AC[2 * NT], fb[3][2 * NT];
+#pragma unroll
+                for (int u = 0; u < 2 * NT; ++u) {
+                    const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
+                    const float G0 = gsub[sl], G1 = gsub[16 + sl], G2 = gsub[32 + sl], G3 = gsub[48 + sl];
+                    fb[2][u] = G3;
+                    fb[1][u] = G2 * G3;
+                    fb[0][u] = G1 * fb[1][u];
+                    AC[u] = G0 * fb[0][u];
+                }
+                // query operands of the earlier key blocks bb < w for this warp's tokens:
+                // QR_bb(t) = QR_w(t) prod_{c=bb..w-1} G_c
+#pragma unroll
+                for (int bb = 0; bb < 3; ++bb) {
+                    if (bb >= w) break;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            float v[2];
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const int sl = 8 * nt + 2 * cq + j;
+                                float cgb = 1.f;
+#pragma unroll
+                                for (int c = 0; c < 4; ++c)
+                                    if (c >= bb && c < w) cgb *= gsub[c * 16 + sl];
+                                v[j] = qrw[nt][2 * hf + j] * cgb;
+                            }
+                            const int tk = tok0 + g + 8 * hf, col = 8 * nt + 2 * cq;
+                            *reinterpret_cast<uint32_t*>(qr + ptx::sw128_off(tk, 16 * bb + col)) =
+                                ptx::pack_bf16x2(v[0], v[1]);
+                        }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_arrive(BAR_A, N_CM);  // QR, KD and the chunk-start state are ready for G4/G5
+
+                // ---- state update: per key sub-chunk bb, U_bb[e][i] = sum_{j in bb} x_j[e] KS_j[i]
+                float ua[4][MT][NT][4];
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) ua[bb][mt][nt][i] = 0.f;
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) update_mma(xs_a, 16 * bb, 16 * bb, ua[bb]);
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar_empty0 + 8 * s);  // done with x, q, c of stage s
+                // S <- A_C S + f_0 U_0 + f_1 U_1 + f_2 U_2 + U_3
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) ua[bb][mt][nt][i] = 0.f;
-            const uint32_t kt_a = sbase + Lay::KT_OFF;
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                uint32_t kf[2][NT][2];  // B: KS rows (tokens) 16bb.., hi at columns 16.., lo at 32..
-                load_b_pairs(kt_a, 16 * bb, 16, kf);
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    uint32_t af[4];
-                    {   // A = X^T: x rows (tokens) 16bb + 8(lj>>1) + lr, columns e = e_base + 16mt + 8(lj&1)
-                        const int row = 16 * bb + 8 * (lj >> 1) + lr;
-                        const int e = e_base + 16 * mt + 8 * (lj & 1);
-                        ptx::ldsm_x4_t(xs_a + (e >> 6) * (64 * 128) + row * 128 + ((((e & 63) >> 3) ^ (row & 7)) << 4), af);
-                    }
-#pragma unroll
-                    for (int v = 0; v < 2; ++v)
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) ptx::mma16816(ua[bb][mt][nt], af, kf[v][nt]);
+                        for (int i = 0; i < 4; ++i) {
+                            const int u = 2 * nt + (i & 1);
+                            float v = ua[3][mt][nt][i];
+                            v = fmaf(fb[2][u], ua[2][mt][nt][i], v);
+                            v = fmaf(fb[1][u], ua[1][mt][nt][i], v);
+                            v = fmaf(fb[0][u], ua[0][mt][nt][i], v);
+                            st[mt][nt][i] = fmaf(AC[u], st[mt][nt][i], v);
+                        }
+                if (k + 1 < nch) {
+                    write_state((k + 1) & 1, nullptr, 0);  // G4 of chunk k-1 (the buffer's last reader) is done
+                    ptx::named_bar(BAR_C2, kRgChain);
+                    load_norms((k + 1) & 1);
                 }
             }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar_empty0 + 8 * s);  // done with x, q, c of stage s
-            // S <- A_C S + f_0 U_0 + f_1 U_1 + f_2 U_2 + U_3
+        } else {
+            // C = 16: each ring stage (64 tokens) holds four consecutive chunks, run one after
+            // the other by all four chain warps together. Every warp forms the projections,
+            // gates and products of the whole chunk (16 tokens x the CTA's slots); warp 0 writes
+            // the chunk's read-out operands (QR in the block-diagonal position of chunk c, KD,
+            // the chunk-start state in column block c of the stacked-state tile), and each warp
+            // writes KS into its own rows of the KT tile for its update, so one barrier per
+            // chunk (the new state) remains on the chain.
+            int step = 0;
+            for (int k = 0; k < nch; ++k) {
+                const int s = k % NST, p = k & 1;
+                tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
+                tc_wait(bar_aux0 + 8 * p, (k >> 1) & 1, abort);  // per-token inputs of stage k
+                const bool zero_mu = zmu[p] != 0u;
+                if (k > 0) tc_wait(bar_p5, (k - 1) & 1, abort);  // G4/G5 of stage k-1 are done with QR, KD
+                const uint32_t xs_a = sbase + Lay::X_OFF + s * Lay::X_STAGE;
+                for (int c = 0; c < 4; ++c, ++step) {
+                    float pr[NT][4];
+                    project(xs_a, sbase + Lay::S0_OFF + (step & 1) * Lay::S0_BUF, 16 * c, pr);
+                    float gt[NT][4], kap[NT][4], qv[NT][4], R[NT][4], suf[NT][4], Gs[NT][2], qrw[NT][4];
+                    gates(pr, s, p, 16 * c, zero_mu, gt, kap, qv);
+                    scans(gt, R, suf, Gs);
+                    write_operands(kap, R, suf, qv, 16 * c, 16 * w, 16 * c, qrw, w == 0);
+                    __syncwarp();
+                    float ua[MT][NT][4];
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
+                    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int u = 2 * nt + (i & 1);
-                        float v = ua[3][mt][nt][i];
-                        v = fmaf(fb[2][u], ua[2][mt][nt][i], v);
-                        v = fmaf(fb[1][u], ua[1][mt][nt][i], v);
-                        v = fmaf(fb[0][u], ua[0][mt][nt][i], v);
-                        st[mt][nt][i] = fmaf(AC[u], st[mt][nt][i], v);
+                            for (int i = 0; i < 4; ++i) ua[mt][nt][i] = 0.f;
+                    update_mma(xs_a, 16 * c, 16 * w, ua);
+                    // S <- G S + U, G the chunk's product of gates
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                st[mt][nt][i] = fmaf(Gs[nt][i & 1], st[mt][nt][i], ua[mt][nt][i]);
+                    if (k + 1 < nch || c < 3) {
+                        // the next chunk's state operand; its hi part also goes to the read-out's
+                        // stacked-state tile of this stage (block c+1) or of the next one (block 0)
+                        uint8_t* sto = smem + Lay::S0ST_OFF + (c < 3 ? p : p ^ 1) * Lay::S0_BUF;
+                        write_state((step + 1) & 1, sto, c < 3 ? 16 * (c + 1) : 0);
+                        ptx::named_bar(BAR_C2, kRgChain);
+                        load_norms((step + 1) & 1);
                     }
-            if (k + 1 < nch) {
-                write_state((k + 1) & 1);  // G4 of chunk k-1 (the buffer's last reader) is done
-                ptx::named_bar(BAR_C2, kRgChain);
-                load_norms();
+                    __syncwarp();
+                }
+                if (tid == 0) zmu[p] = 0u;  // every chain thread read it before the chunks' barriers
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_arrive(BAR_A, N_CM);  // QR, KD and the stage's chunk-start states are ready
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar_empty0 + 8 * s);  // done with x, q, c of stage s
             }
         }
         // final state
@@ -734,15 +829,15 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     if (warp == MMA_WARP) ptx::tmem_dealloc(tmem, Lay::TMEM_COLS);
 }
 
-template <int DS, int SPC>
+template <int DS, int SPC, int CH>
 cudaError_t launch_chunk_reg_t(const ScanArgs& a, cudaStream_t st) {
-    using Lay = RgLayout<DS, SPC>;
+    using Lay = RgLayout<DS, SPC, CH>;
     TcMaps maps;
     if (!make_map_4d(&maps.x, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DS, a.H, a.T, a.B, 64, true) ||
         !make_map_4d(&maps.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kRgM, a.H, a.T, a.B, SPC, false) ||
         !make_map_4d(&maps.c, a.c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kRgM, a.H, a.T, a.B, SPC, false))
         return cudaErrorInvalidValue;
-    auto k = chunk_reg_kernel<DS, SPC>;
+    auto k = chunk_reg_kernel<DS, SPC, CH>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -766,8 +861,8 @@ cudaError_t launch_chunk_reg_t(const ScanArgs& a, cudaStream_t st) {
 // hold at once (each cluster takes 64/spc SMs of one GPC); 0 if the query fails.
 template <int DS, int SPC>
 int chunk_reg_max_clusters_t() {
-    using Lay = RgLayout<DS, SPC>;
-    auto k = chunk_reg_kernel<DS, SPC>;
+    using Lay = RgLayout<DS, SPC, 64>;
+    auto k = chunk_reg_kernel<DS, SPC, 64>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM_ALLOC) != cudaSuccess) {
         cudaGetLastError();
         return 0;
@@ -797,10 +892,17 @@ inline int chunk_reg_max_clusters(int d, int spc) {
     return 0;
 }
 
+template <int CH>
+cudaError_t launch_chunk_reg_c(const ScanArgs& a, int d, int spc, cudaStream_t st) {
+    if (d == 128) return spc == 8 ? launch_chunk_reg_t<128, 8, CH>(a, st) : launch_chunk_reg_t<128, 16, CH>(a, st);
+    if (d == 64) return spc == 8 ? launch_chunk_reg_t<64, 8, CH>(a, st) : launch_chunk_reg_t<64, 16, CH>(a, st);
+    return cudaErrorNotSupported;
+}
+
 inline cudaError_t launch_chunk_reg(const ScanArgs& a, int d, int spc, cudaStream_t st) {
     if (a.m != kRgM || (spc != 8 && spc != 16)) return cudaErrorNotSupported;
-    if (d == 128) return spc == 8 ? launch_chunk_reg_t<128, 8>(a, st) : launch_chunk_reg_t<128, 16>(a, st);
-    if (d == 64) return spc == 8 ? launch_chunk_reg_t<64, 8>(a, st) : launch_chunk_reg_t<64, 16>(a, st);
+    if (a.chunk == 64) return launch_chunk_reg_c<64>(a, d, spc, st);
+    if (a.chunk == 16) return launch_chunk_reg_c<16>(a, d, spc, st);
     return cudaErrorNotSupported;
 }
 

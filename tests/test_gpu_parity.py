@@ -223,6 +223,20 @@ def test_chunked_tcgen05_split(L, d, T, impl):
     assert s_err(Sg, So) <= TOL_TC
 
 
+@pytest.mark.parametrize("impl", ["split_reg", "split_reg8"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 16, 37, 64 + 16 + 5, 5 * 64 + 9])
+def test_chunked_reg_chunk16(L, d, T, impl):
+    """Chunk size 16 on the register-chain kernels (four chunks per 64-token read-out
+    round) vs the oracle's Eq. 17 chunked form with C = 16: partial chunks and stages."""
+    w = LI.Workload("t", B=2, T=T, H=3, m=64, d=d, seed=2100 + d + T)
+    inp = LI.make_inputs(w)
+    yg, Sg = run_gpu(L, inp, 16, impl=impl)
+    yo, So = run_oracle(inp, 16)
+    assert y_err(yg, yo) <= TOL_TC
+    assert s_err(Sg, So) <= TOL_TC
+
+
 @pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg", "split_reg8"])
 def test_chunked_split_and_wide_agree(L, impl):
     """The tensor-core kernels compute the same chunked form."""
