@@ -44,9 +44,7 @@
 namespace lattice {
 
 constexpr int kRgM = 64;                        // slots per sequence
-constexpr int kRgChain = 128;                   // 4 chain warps
 constexpr int kRgReadout = 128;                 // 4 read-out warps
-constexpr int kRgThreads = kRgChain + kRgReadout + 64;  // + MMA warp + TMA warp
 
 inline bool chunk_reg_supported(int m, int d, int chunk, bool x_bf16, bool q_bf16) {
     return (chunk == kTcC || chunk == 16) && x_bf16 && q_bf16 && m == kRgM && (d == 64 || d == 128);
@@ -58,6 +56,9 @@ template <int DS, int SPC, int CH>
 struct RgLayout {
     static_assert(SPC == 8 || SPC == 16, "8 or 16 slots per CTA");
     static_assert(CH == 64 || CH == 16, "chunk size 64 or 16");
+    static constexpr int HALVES = SPC / 8;                 // 8-slot halves, each with its own 4 chain warps
+    static constexpr int CHAIN = 128 * HALVES;             // chain threads
+    static constexpr int THREADS = CHAIN + kRgReadout + 64;  // + 4 read-out warps, MMA warp, TMA warp
     static constexpr int NST = (CH == 16 && DS == 128) ? 3 : 4;  // x/q/c ring depth (stages of 64 tokens)
     static constexpr int NC = kRgM / SPC;                  // CTAs per sequence (cluster size)
     static constexpr int DSL = DS / NC;                    // y columns reduced by each CTA
@@ -100,12 +101,13 @@ struct RgLayout {
 };
 
 template <int DS, int SPC, int CH>
-__global__ void __launch_bounds__(kRgThreads, 1)
+__global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
     chunk_reg_kernel(const __grid_constant__ TcMaps maps, ScanArgs a) {
     using Lay = RgLayout<DS, SPC, CH>;
     constexpr int DSL = Lay::DSL;
     constexpr int NC = Lay::NC;
-    constexpr int NT = SPC / 8;  // 8-slot n-tiles per CTA
+    constexpr int CHAIN = Lay::CHAIN;
+    constexpr int NT = 1;  // 8-slot n-tiles per chain warp
     constexpr int NST = Lay::NST;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -116,9 +118,9 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     const int bh = blockIdx.x / NC, b = bh / a.H, h = bh % a.H;
     const int T = a.T, H = a.H;
     const int nch = (T + kTcC - 1) / kTcC;  // ring stages of 64 tokens (chunks when C = 64)
-    constexpr int RO_WARP0 = kRgChain / 32, MMA_WARP = RO_WARP0 + 4, TMA_WARP = MMA_WARP + 1;
+    constexpr int RO_WARP0 = CHAIN / 32, MMA_WARP = RO_WARP0 + 4, TMA_WARP = MMA_WARP + 1;
 
-    // mbarriers: ring stage full [NST] (TMA bytes) and empty [NST] (4 chain warps + the
+    // mbarriers: ring stage full [NST] (TMA bytes) and empty [NST] (the chain warps + the
     // MMA warp's commit after G6), scores ready (G4, G5), read-out done (G6), peers'
     // partial y in [2], per-token inputs ready [2], read-out buffer drained [2]
     const uint32_t bar_full0 = sbase + Lay::BAR_OFF;
@@ -135,17 +137,18 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     float* gsub = reinterpret_cast<float*>(smem + Lay::GSUB_OFF);
     float* tsq = reinterpret_cast<float*>(smem + Lay::TSQ_OFF);
 
-    // named barriers: chain warps alone (C1 after the gates, C2 after the update), chain
-    // warps (arrive) + MMA warp (A: read-out operands written), read-out warps (arrive)
-    // + MMA warp (P: masked scores written)
-    constexpr uint32_t BAR_C1 = 1, BAR_C2 = 2, BAR_A = 3, BAR_P = 4;
-    constexpr uint32_t N_CM = kRgChain + 32, N_RM = kRgReadout + 32;
+    // named barriers: each half's 4 chain warps alone (C1 after the gates, C2 after the
+    // update: ids 1, 2 for half 0 and 5, 6 for half 1), every chain warp (INIT, at the
+    // start), chain warps (arrive) + MMA warp (A: read-out operands written), read-out
+    // warps (arrive) + MMA warp (P: masked scores written)
+    constexpr uint32_t BAR_A = 3, BAR_P = 4, BAR_INIT = 7;
+    constexpr uint32_t N_CM = CHAIN + 32, N_RM = kRgReadout + 32;
 
     if (warp == MMA_WARP) {
         if (lane == 0) {
             for (int s = 0; s < NST; ++s) {
                 ptx::mbar_init(bar_full0 + 8 * s, 1);
-                ptx::mbar_init(bar_empty0 + 8 * s, kRgChain / 32 + 1);
+                ptx::mbar_init(bar_empty0 + 8 * s, CHAIN / 32 + 1);
             }
             ptx::mbar_init(bar_p5, 1);
             ptx::mbar_init(bar_y, 1);
@@ -185,6 +188,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             const int s = k % NST, p = k & 1;
             const uint32_t ycol = Lay::Y_COL + p * DS;
             ptx::named_bar(BAR_A, N_CM);  // QR, KD of chunk k and its start state written
+            if (lane == 0) zmu[p] = 0u;   // every chain thread read it before arriving
             ptx::tc_fence_after();
             // the read-out of chunk k-2 (same accumulator buffer) has been drained
             const bool yfree = k < 2 || tc_wait_warp(bar_yfree0 + 8 * p, ((k - 2) >> 1) & 1, abort);
@@ -260,7 +264,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
     } else if (warp >= RO_WARP0) {
         // ------------------------------------------------------------ read-out warps
         const int q = warp & 3;
-        const int rt = tid - kRgChain;     // 0..127
+        const int rt = tid - CHAIN;        // 0..127
         const uint32_t lane_base = uint32_t(32 * q) << 16;
         const bool row_ok = lane < 16;     // M = 64 accumulators: lanes 0-15 of each quadrant
         const int trow = 16 * q + lane;    // accumulator row (token) of this lane
@@ -394,12 +398,16 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         if (nch > 0) recv_y(nch - 1);
     } else {
         // ================================================================ chain warps
-        // Fragment coordinates: g = lane/4 (a row: a token, or a state column), cq = lane%4
-        // (a pair of slots 2cq, 2cq+1 of each 8-slot n-tile nt); index i of a 4-register
-        // fragment is (row g + 8(i/2), slot 8nt + 2cq + i%2). Warp w owns the state columns
-        // w*d/4..(w+1)*d/4 in the update; with C = 64 it also owns the projections and gates
-        // of sub-chunk w (tokens 16w..16w+15).
-        const int w = warp;
+        // Chain warp w + 4hv runs half hv of the CTA's slots (8 slots, sh = 8hv..8hv+7); the
+        // two halves never exchange anything, so each runs its own chain with its own named
+        // barriers and the warp scheduler overlaps one half's gate arithmetic with the other
+        // half's MMAs. Fragment coordinates: g = lane/4 (a row: a token, or a state column),
+        // cq = lane%4 (a pair of slots sh + 2cq, sh + 2cq + 1); index i of a 4-register
+        // fragment is (row g + 8(i/2), slot sh + 2cq + i%2). Warp w owns the state columns
+        // w*d/4..(w+1)*d/4 of its half in the update; with C = 64 it also owns the
+        // projections and gates of sub-chunk w (tokens 16w..16w+15).
+        const int w = warp & 3, hv = warp >> 2, sh = 8 * hv;
+        const uint32_t BAR_C1 = hv ? 5 : 1, BAR_C2 = hv ? 6 : 2;
         const int g = lane >> 2, cq = lane & 3;
         constexpr int MT = DS / 64;                   // 16-column m-tiles of the update per warp
         const int e_base = w * (DS / 4);
@@ -419,7 +427,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int e = e_base + 16 * mt + g + 8 * (i >> 1);
-                        const int sl = 8 * nt + 2 * cq + (i & 1);
+                        const int sl = sh + 8 * nt + 2 * cq + (i & 1);
                         st[mt][nt][i] = S0g[(size_t)sl * DS + e];
                     }
         }
@@ -442,7 +450,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         const float2 v = make_float2(st[mt][nt][2 * hf], st[mt][nt][2 * hf + 1]);
                         uint32_t hi, lo;
                         split2(v, hi, lo);
-                        const int col = 8 * nt + 2 * cq;
+                        const int col = sh + 8 * nt + 2 * cq;
                         *reinterpret_cast<uint32_t*>(dst + ptx::sw128_off(e, col)) = hi;
                         *reinterpret_cast<uint32_t*>(dst + ptx::sw128_off(e, 16 + col)) = lo;
                         if (CH == 16) *reinterpret_cast<uint32_t*>(sto + ptx::sw128_off(e, scol + col)) = hi;
@@ -457,7 +465,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                     v += __shfl_xor_sync(0xffffffffu, v, 4);
                     v += __shfl_xor_sync(0xffffffffu, v, 8);
                     v += __shfl_xor_sync(0xffffffffu, v, 16);
-                    if (g == 0) tsq[pb * 64 + w * 16 + 8 * nt + 2 * cq + j] = v;
+                    if (g == 0) tsq[pb * 64 + w * 16 + sh + 8 * nt + 2 * cq + j] = v;
                 }
         };
         // n = |s0|, 1/n, 1/n^2 of this thread's slots (index 2nt + j: slot 8nt + 2cq + j)
@@ -465,7 +473,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         auto load_norms = [&](int pb) {
 #pragma unroll
             for (int u = 0; u < 2 * NT; ++u) {
-                const float* t4 = tsq + pb * 64 + 8 * (u >> 1) + 2 * cq + (u & 1);
+                const float* t4 = tsq + pb * 64 + sh + 8 * (u >> 1) + 2 * cq + (u & 1);
                 const float nsq = ((t4[0] + t4[16]) + t4[32]) + t4[48];
                 inv_n[u] = ptx::rsqrt_nr(nsq);
                 nrm[u] = nsq * inv_n[u];
@@ -509,7 +517,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                     const int col = 16 * ks + 8 * (lj >> 1);
                     ptx::ldsm_x4(xs_a + (col >> 6) * (64 * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4), af);
                 }
-                load_b_pairs(s0_a, 16 * ks, 0, bf);  // the state rows e = 16ks..16ks+15
+                load_b_pairs(s0_a, 16 * ks, sh, bf);  // the state rows e = 16ks..16ks+15
 #pragma unroll
                 for (int v = 0; v < 2; ++v)
 #pragma unroll
@@ -536,8 +544,8 @@ __global__ void __launch_bounds__(kRgThreads, 1)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int u0 = 2 * nt;  // norm index of slot 8nt + 2cq
-                    const float2 cc = *reinterpret_cast<const float2*>(cs + tk * SPC + 8 * nt + 2 * cq);
-                    const uint32_t q2 = *reinterpret_cast<const uint32_t*>(qs + tk * SPC + 8 * nt + 2 * cq);
+                    const float2 cc = *reinterpret_cast<const float2*>(cs + tk * SPC + sh + 8 * nt + 2 * cq);
+                    const uint32_t q2 = *reinterpret_cast<const uint32_t*>(qs + tk * SPC + sh + 8 * nt + 2 * cq);
                     const float2 pp = make_float2(pr[nt][2 * hf], pr[nt][2 * hf + 1]);
                     const float2 e2 = ptx::f2mul(cc, ptx::f2mul(ptx::f2(z.y), make_float2(inv_n2[u0], inv_n2[u0 + 1])));
                     const float2 pn = ptx::f2mul(pp, make_float2(inv_n[u0], inv_n[u0 + 1]));
@@ -603,7 +611,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    const int col = 8 * nt + 2 * cq;
+                    const int col = sh + 8 * nt + 2 * cq;
                     float kd[2], ks[2];
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
@@ -630,7 +638,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
         // columns, KS from the KT tile rows ks_row0.. (B), x^T from the stage (A)
         auto update_mma = [&](uint32_t xs_a, int row0, int ks_row0, float (&u)[MT][NT][4]) {
             uint32_t kf[2][NT][2];
-            load_b_pairs(kt_a, ks_row0, 16, kf);
+            load_b_pairs(kt_a, ks_row0, 16 + sh, kf);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 uint32_t af[4];
@@ -648,15 +656,15 @@ __global__ void __launch_bounds__(kRgThreads, 1)
 
         // ---- prologue: operand tiles zeroed (blocks of the query tile that are never
         // written, and with 8 slots per CTA the K padding up to 16)
-        for (int o = tid; o < int(kTcC * 128 / 16); o += kRgChain) {
+        for (int o = tid; o < int(kTcC * 128 / 16); o += CHAIN) {
             reinterpret_cast<uint4*>(qr)[o] = make_uint4(0u, 0u, 0u, 0u);
             reinterpret_cast<uint4*>(kt)[o] = make_uint4(0u, 0u, 0u, 0u);
         }
-        for (int o = tid; o < int(Lay::S0_TILES * Lay::S0_BUF / 16); o += kRgChain)
+        for (int o = tid; o < int(Lay::S0_TILES * Lay::S0_BUF / 16); o += CHAIN)
             reinterpret_cast<uint4*>(smem + Lay::S0_OFF)[o] = make_uint4(0u, 0u, 0u, 0u);
-        ptx::named_bar(BAR_C2, kRgChain);
+        ptx::named_bar(BAR_INIT, CHAIN);  // every chain thread's zeros before any state is written
         write_state(0, smem + Lay::S0ST_OFF, 0);
-        ptx::named_bar(BAR_C2, kRgChain);
+        ptx::named_bar(BAR_C2, 128);
         load_norms(0);
 
         if constexpr (CH == 64) {
@@ -676,15 +684,14 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                 if (g == 0) {
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
-                        *reinterpret_cast<float2*>(gsub + w * 16 + 8 * nt + 2 * cq) = make_float2(Gs[nt][0], Gs[nt][1]);
+                        *reinterpret_cast<float2*>(gsub + w * 16 + sh + 8 * nt + 2 * cq) = make_float2(Gs[nt][0], Gs[nt][1]);
                 }
-                ptx::named_bar(BAR_C1, kRgChain);  // every sub-chunk's products and KS written
-                if (tid == 0) zmu[p] = 0u;         // every chain thread read it before the barrier
+                ptx::named_bar(BAR_C1, 128);  // every sub-chunk's products and KS of this half written
                 // per slot: the chunk decay A_C and f_b = prod_{c>b} G_c of each sub-chunk b
                 float AC[2 * NT], fb[3][2 * NT];
 #pragma unroll
                 for (int u = 0; u < 2 * NT; ++u) {
-                    const int sl = 8 * (u >> 1) + 2 * cq + (u & 1);
+                    const int sl = sh + 8 * (u >> 1) + 2 * cq + (u & 1);
                     const float G0 = gsub[sl], G1 = gsub[16 + sl], G2 = gsub[32 + sl], G3 = gsub[48 + sl];
                     fb[2][u] = G3;
                     fb[1][u] = G2 * G3;
@@ -703,14 +710,14 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                             float v[2];
 #pragma unroll
                             for (int j = 0; j < 2; ++j) {
-                                const int sl = 8 * nt + 2 * cq + j;
+                                const int sl = sh + 8 * nt + 2 * cq + j;
                                 float cgb = 1.f;
 #pragma unroll
                                 for (int c = 0; c < 4; ++c)
                                     if (c >= bb && c < w) cgb *= gsub[c * 16 + sl];
                                 v[j] = qrw[nt][2 * hf + j] * cgb;
                             }
-                            const int tk = tok0 + g + 8 * hf, col = 8 * nt + 2 * cq;
+                            const int tk = tok0 + g + 8 * hf, col = sh + 8 * nt + 2 * cq;
                             *reinterpret_cast<uint32_t*>(qr + ptx::sw128_off(tk, 16 * bb + col)) =
                                 ptx::pack_bf16x2(v[0], v[1]);
                         }
@@ -748,7 +755,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         }
                 if (k + 1 < nch) {
                     write_state((k + 1) & 1, nullptr, 0);  // G4 of chunk k-1 (the buffer's last reader) is done
-                    ptx::named_bar(BAR_C2, kRgChain);
+                    ptx::named_bar(BAR_C2, 128);
                     load_norms((k + 1) & 1);
                 }
             }
@@ -797,12 +804,11 @@ __global__ void __launch_bounds__(kRgThreads, 1)
                         // stacked-state tile of this stage (block c+1) or of the next one (block 0)
                         uint8_t* sto = smem + Lay::S0ST_OFF + (c < 3 ? p : p ^ 1) * Lay::S0_BUF;
                         write_state((step + 1) & 1, sto, c < 3 ? 16 * (c + 1) : 0);
-                        ptx::named_bar(BAR_C2, kRgChain);
+                        ptx::named_bar(BAR_C2, 128);
                         load_norms((step + 1) & 1);
                     }
                     __syncwarp();
                 }
-                if (tid == 0) zmu[p] = 0u;  // every chain thread read it before the chunks' barriers
                 ptx::fence_proxy_async_smem();
                 ptx::named_bar_arrive(BAR_A, N_CM);  // QR, KD and the stage's chunk-start states are ready
                 __syncwarp();
@@ -818,7 +824,7 @@ __global__ void __launch_bounds__(kRgThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int e = e_base + 16 * mt + g + 8 * (i >> 1);
-                    const int sl = 8 * nt + 2 * cq + (i & 1);
+                    const int sl = sh + 8 * nt + 2 * cq + (i & 1);
                     So[(size_t)sl * DS + e] = st[mt][nt][i];
                 }
     }
@@ -842,7 +848,7 @@ cudaError_t launch_chunk_reg_t(const ScanArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.H * Lay::NC);
-    cfg.blockDim = dim3(kRgThreads);
+    cfg.blockDim = dim3(Lay::THREADS);
     cfg.dynamicSmemBytes = Lay::SMEM_ALLOC;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -869,7 +875,7 @@ int chunk_reg_max_clusters_t() {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(Lay::NC * 64);
-    cfg.blockDim = dim3(kRgThreads);
+    cfg.blockDim = dim3(Lay::THREADS);
     cfg.dynamicSmemBytes = Lay::SMEM_ALLOC;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
