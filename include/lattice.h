@@ -119,10 +119,10 @@ typedef enum {
 } lattice_impl;
 
 /* Which kernel LATTICE_IMPL_AUTO runs for a chunked scan of B x H sequences of
- * this shape: TCGEN05_SPLIT when it applies and B*H*4 CTAs fit on the current
- * device's SMs at once, else TCGEN05 when it applies, else SIMT (chunk_size 1
- * is always SIMT). Host function; launches nothing (without a device it
- * assumes 148 SMs). */
+ * this shape: SPLIT_REG when it applies (chunk 64 or 16, m = 64) and the current
+ * device holds B*H of its 4-CTA clusters at once, else TCGEN05 when it applies,
+ * else SIMT (chunk_size 1 is always SIMT). Host function; launches nothing
+ * (without a device it assumes the 37 clusters of a 148-SM part). */
 lattice_impl lattice_chunk_impl(int B, int H, int m, int d, int chunk_size, lattice_dtype x_dtype,
                                 lattice_dtype q_dtype);
 

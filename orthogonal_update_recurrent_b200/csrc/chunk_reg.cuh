@@ -59,7 +59,7 @@ struct RgLayout {
     static constexpr int HALVES = SPC / 8;                 // 8-slot halves, each with its own 4 chain warps
     static constexpr int CHAIN = 128 * HALVES;             // chain threads
     static constexpr int THREADS = CHAIN + kRgReadout + 64;  // + 4 read-out warps, MMA warp, TMA warp
-    static constexpr int NST = (CH == 16 && DS == 128) ? 3 : 4;  // x/q/c ring depth (stages of 64 tokens)
+    static constexpr int NST = DS == 128 ? (CH == 16 ? 2 : 3) : 4;  // x/q/c ring depth (stages of 64 tokens)
     static constexpr int NC = kRgM / SPC;                  // CTAs per sequence (cluster size)
     static constexpr int DSL = DS / NC;                    // y columns reduced by each CTA
     static constexpr uint32_t X_STAGE = DS * 128;          // [C][d] bf16 in d/64 SW128 blocks
@@ -82,7 +82,11 @@ struct RgLayout {
     static constexpr uint32_t P_OFF = KT_OFF + kTcC * 128;      // [C][C] bf16 masked scores
     static constexpr uint32_t RECV_OFF = P_OFF + kTcC * 128;    // [2][NC][C][d/NC] fp32
     static constexpr uint32_t RECV_BYTES = 2 * NC * kTcC * DSL * 4;
-    static constexpr uint32_t AUX_OFF = RECV_OFF + RECV_BYTES;  // [2][C] float4: mu, eta, |x|^2, mu^2
+    // outgoing partials, one [C][d/NC] fp32 block per peer (this CTA's own block goes
+    // straight into its receive buffer), moved by one bulk copy per peer
+    static constexpr uint32_t PEER_BLOCK = kTcC * DSL * 4;
+    static constexpr uint32_t STG_OFF = RECV_OFF + RECV_BYTES;
+    static constexpr uint32_t AUX_OFF = STG_OFF + (NC - 1) * PEER_BLOCK;  // [2][C] float4: mu, eta, |x|^2, mu^2
     static constexpr uint32_t GSUB_OFF = AUX_OFF + 2 * kTcC * 16;   // [4 sub-chunks][16] (SPC used)
     static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * 16 * 4;        // [2][4 warps][16] (SPC used)
     static constexpr uint32_t BAR_OFF = TSQ_OFF + 2 * 4 * 16 * 4;
@@ -128,12 +132,9 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
     const uint32_t bar_p5 = bar_empty0 + 8 * NST;
     const uint32_t bar_y = bar_p5 + 8;
     const uint32_t bar_recv0 = bar_y + 8;
-    const uint32_t bar_aux0 = bar_recv0 + 16;
-    const uint32_t bar_yfree0 = bar_aux0 + 16;
+    const uint32_t bar_yfree0 = bar_recv0 + 16;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
     volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 4);
-    volatile uint32_t* zmu = reinterpret_cast<volatile uint32_t*>(smem + Lay::MISC_OFF + 8);
-    float4* aux = reinterpret_cast<float4*>(smem + Lay::AUX_OFF);
     float* gsub = reinterpret_cast<float*>(smem + Lay::GSUB_OFF);
     float* tsq = reinterpret_cast<float*>(smem + Lay::TSQ_OFF);
 
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
     // update: ids 1, 2 for half 0 and 5, 6 for half 1), every chain warp (INIT, at the
     // start), chain warps (arrive) + MMA warp (A: read-out operands written), read-out
     // warps (arrive) + MMA warp (P: masked scores written)
-    constexpr uint32_t BAR_A = 3, BAR_P = 4, BAR_INIT = 7;
+    constexpr uint32_t BAR_A = 3, BAR_P = 4, BAR_INIT = 7, BAR_RO = 8;
     constexpr uint32_t N_CM = CHAIN + 32, N_RM = kRgReadout + 32;
 
     if (warp == MMA_WARP) {
@@ -154,13 +155,9 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
             ptx::mbar_init(bar_y, 1);
             ptx::mbar_init(bar_recv0, 1);
             ptx::mbar_init(bar_recv0 + 8, 1);
-            ptx::mbar_init(bar_aux0, kRgReadout);
-            ptx::mbar_init(bar_aux0 + 8, kRgReadout);
             ptx::mbar_init(bar_yfree0, kRgReadout);
             ptx::mbar_init(bar_yfree0 + 8, kRgReadout);
             *abort = 0u;
-            zmu[0] = 0u;
-            zmu[1] = 0u;
             ptx::fence_mbar_init();
         }
         __syncwarp();
@@ -188,7 +185,6 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
             const int s = k % NST, p = k & 1;
             const uint32_t ycol = Lay::Y_COL + p * DS;
             ptx::named_bar(BAR_A, N_CM);  // QR, KD of chunk k and its start state written
-            if (lane == 0) zmu[p] = 0u;   // every chain thread read it before arriving
             ptx::tc_fence_after();
             // the read-out of chunk k-2 (same accumulator buffer) has been drained
             const bool yfree = k < 2 || tc_wait_warp(bar_yfree0 + 8 * p, ((k - 2) >> 1) & 1, abort);
@@ -268,83 +264,42 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
         const uint32_t lane_base = uint32_t(32 * q) << 16;
         const bool row_ok = lane < 16;     // M = 64 accumulators: lanes 0-15 of each quadrant
         const int trow = 16 * q + lane;    // accumulator row (token) of this lane
-        // per-token mu, eta, |x|^2, mu^2 of chunk k: 2 threads per token, each half of x
-        auto aux_chunk = [&](int k) {
-            const int s = k % NST, p = k & 1;
-            const int tk = rt >> 1, half = rt & 1;
-            const int t = k * kTcC + tk;
-            float mu = 0.f, eta = 1.f;
-            if (half == 0 && t < T) {
-                const size_t bth = ((size_t)b * T + t) * H + h;
-                mu = __ldg(a.mu + bth);
-                if (a.eta) eta = __ldg(a.eta + bth);
-            }
-            const bool ok = tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
-            const uint8_t* xs = smem + Lay::X_OFF + s * Lay::X_STAGE;
-            float2 acc = ptx::f2(0.f);
-            if (ok) {
-#pragma unroll
-                for (int u = 0; u < DS / 16; ++u) {  // DS/16 chunks of 16 B per thread
-                    const int ch = half * (DS / 16) + u;  // block ch/8, chunk ch%8 (any order sums the row)
-                    uint4 v = *reinterpret_cast<const uint4*>(xs + (ch >> 3) * (64 * 128) + tk * 128 + (ch & 7) * 16);
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float2 xv = make_float2(__uint_as_float(w4[c] << 16), __uint_as_float(w4[c] & 0xffff0000u));
-                        acc = ptx::f2fma(xv, xv, acc);
-                    }
-                }
-            }
-            float xx = acc.x + acc.y;
-            xx += __shfl_xor_sync(0xffffffffu, xx, 1);
-            if (half == 0) {
-                const float mu2 = mu * mu;
-                aux[p * kTcC + tk] = make_float4(mu, eta, xx, mu2);
-                if (!(mu2 >= 8.6736174e-19f)) zmu[p] = 1u;  // mu^2 < 2^-60 (or zero)
-            }
-            ptx::mbar_arrive(bar_aux0 + 8 * p);
-        };
-        // the four partials of this CTA's columns of chunk kc -> y. Summing chunk k-1
-        // before sending chunk k keeps two receive buffers enough: a peer's chunk k+1
-        // follows its sum of chunk k, which needs this CTA's chunk k, sent after this sum.
-        constexpr uint32_t RECV_TX = NC * kTcC * DSL * 4;  // bytes of one chunk's partials
+        // the NC partials of this CTA's columns of chunk kc -> y. Summing chunk k-1 before
+        // sending chunk k keeps two receive buffers enough: a peer's chunk k+1 follows its
+        // sum of chunk k, which needs this CTA's chunk k, sent after this sum. A partial
+        // block is [C rows][d/NC fp32 columns] with the 16-byte chunk j of row r stored at
+        // position j ^ (r mod G) (G chunks per row), so that neither the writers (one row
+        // per lane) nor the readers (one chunk per lane) meet bank conflicts.
+        constexpr int G = DSL / 4;          // 16-byte chunks per row of a partial block
+        constexpr uint32_t RECV_TX = (NC - 1) * Lay::PEER_BLOCK;  // bytes of one chunk's partials from the peers
         auto recv_y = [&](int kc) {
             const int par = kc & 1;
             tc_wait_cluster(bar_recv0 + 8 * par, (kc >> 1) & 1, abort);
             if (rt == 0 && kc + 2 < nch) ptx::mbar_arrive_expect_tx(bar_recv0 + 8 * par, RECV_TX);  // chunk kc+2
             if (*abort) return;
-            const int tk = rt >> 1;
-            const int t = kc * kTcC + tk;
-            constexpr int PER = DSL / 2;  // floats per thread: 4 to 16
-            const int c0 = (rt & 1) * PER;
-            float acc[PER];
+            constexpr int TPR = kRgReadout / G;  // tokens per round
+            const int gg = rt % G;
 #pragma unroll
-            for (int c = 0; c < PER; ++c) acc[c] = 0.f;
+            for (int r = 0; r < kTcC / TPR; ++r) {
+                const int tk = r * TPR + rt / G;
+                const uint32_t o = tk * (DSL * 4) + ((gg ^ (tk & (G - 1))) << 4);
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int src = 0; src < NC; ++src) {
-                const float* rb = reinterpret_cast<const float*>(
-                                      smem + Lay::RECV_OFF + ((par * NC + src) * kTcC + tk) * (DSL * 4)) + c0;
-#pragma unroll
-                for (int c = 0; c < PER; c += 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(rb + c);
-                    acc[c] += v.x; acc[c + 1] += v.y; acc[c + 2] += v.z; acc[c + 3] += v.w;
+                for (int src = 0; src < NC; ++src) {
+                    const float4 v = *reinterpret_cast<const float4*>(smem + Lay::RECV_OFF + (par * NC + src) * Lay::PEER_BLOCK + o);
+                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
                 }
-            }
-            if (t < T) {
-                float* yp = a.y + (((size_t)b * T + t) * H + h) * DS + rank * DSL + c0;
-#pragma unroll
-                for (int c = 0; c < PER; c += 4)
-                    *reinterpret_cast<float4*>(yp + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                const int t = kc * kTcC + tk;
+                if (t < T)
+                    *reinterpret_cast<float4*>(a.y + (((size_t)b * T + t) * H + h) * DS + rank * DSL + 4 * gg) = acc;
             }
         };
         if (rt == 0) {  // arm the receive barriers of chunks 0 and 1
             if (nch > 0) ptx::mbar_arrive_expect_tx(bar_recv0, RECV_TX);
             if (nch > 1) ptx::mbar_arrive_expect_tx(bar_recv0 + 8, RECV_TX);
         }
-        if (nch > 0) aux_chunk(0);
         for (int k = 0; k < nch; ++k) {
             const int par = k & 1;
-            if (k + 1 < nch) aux_chunk(k + 1);
             // causal mask of this chunk's scores: row trow, all 64 keys
             tc_wait(bar_p5, k & 1, abort);
             __syncwarp();
@@ -371,9 +326,12 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
             ptx::tc_fence_before();
             ptx::named_bar_arrive(BAR_P, N_RM);
             if (k > 0) recv_y(k - 1);
-            // partial read-out of this chunk: every peer's quarter of the columns
+            // partial read-out of this chunk: every peer's block of columns, staged in shared
+            // memory and sent with one bulk copy per peer (this CTA's own block goes straight
+            // into its receive buffer)
             tc_wait(bar_y, k & 1, abort);
-            __syncwarp();
+            if (rt == 0) ptx::bulk_wait_read_all();  // the previous chunk's copies have read the staging
+            ptx::named_bar(BAR_RO, kRgReadout);
             ptx::tc_fence_after();
 #pragma unroll
             for (int pp = 0; pp < NC; ++pp) {
@@ -381,21 +339,35 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
                 uint32_t yv[DSL];
                 ptx::tmem_ld<DSL>(tmem + lane_base + Lay::Y_COL + par * DS + pp * DSL, yv);
                 ptx::tmem_wait_ld();
-                if (row_ok && !*abort) {
-                    const uint32_t dst = Lay::RECV_OFF + ((par * NC + rank) * kTcC + trow) * (DSL * 4);
-                    const uint32_t cdst = ptx::mapa(sbase + dst, (uint32_t)pp);
-                    const uint32_t cbar = ptx::mapa(bar_recv0 + 8 * par, (uint32_t)pp);
+                if (row_ok) {
+                    const uint32_t off = pp == rank ? Lay::RECV_OFF + (par * NC + rank) * Lay::PEER_BLOCK
+                                                    : Lay::STG_OFF + (pp - (pp > rank)) * Lay::PEER_BLOCK;
+                    uint8_t* dst = smem + off + trow * (DSL * 4);
 #pragma unroll
                     for (int c = 0; c < DSL; c += 4)
-                        ptx::st_async_v4(cdst + c * 4, make_float4(__uint_as_float(yv[c]), __uint_as_float(yv[c + 1]),
-                                                                   __uint_as_float(yv[c + 2]), __uint_as_float(yv[c + 3])),
-                                         cbar);
+                        *reinterpret_cast<float4*>(dst + (((c / 4) ^ (trow & (G - 1))) << 4)) =
+                            make_float4(__uint_as_float(yv[c]), __uint_as_float(yv[c + 1]),
+                                        __uint_as_float(yv[c + 2]), __uint_as_float(yv[c + 3]));
                 }
+            }
+            ptx::fence_proxy_async_smem();  // the staged blocks are read by the copy engine
+            ptx::named_bar(BAR_RO, kRgReadout);
+            if (rt == 0 && !*abort) {
+#pragma unroll
+                for (int pp = 0; pp < NC; ++pp) {
+                    if (pp == rank) continue;
+                    const uint32_t dst = sbase + Lay::RECV_OFF + (par * NC + rank) * Lay::PEER_BLOCK;
+                    ptx::bulk_copy_s2cluster(ptx::mapa(dst, (uint32_t)pp),
+                                             sbase + Lay::STG_OFF + (pp - (pp > rank)) * Lay::PEER_BLOCK,
+                                             Lay::PEER_BLOCK, ptx::mapa(bar_recv0 + 8 * par, (uint32_t)pp));
+                }
+                ptx::bulk_commit();
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar_yfree0 + 8 * par);  // this buffer may take chunk k+2
         }
         if (nch > 0) recv_y(nch - 1);
+        if (rt == 0) ptx::bulk_wait_all();  // no copy still reads this CTA's shared memory
     } else {
         // ================================================================ chain warps
         // Chain warp w + 4hv runs half hv of the CTA's slots (8 slots, sh = 8hv..8hv+7); the
@@ -499,7 +471,8 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
         };
         // projections D[t][i] = x_t . (s0hi_i + s0lo_i) of the 16 tokens at stage rows
         // row0..row0+15, all the CTA's slots; pr[nt][i] in the fragment layout
-        auto project = [&](uint32_t xs_a, uint32_t s0_a, int row0, float (&pr)[NT][4]) {
+        auto project = [&](uint32_t xs_a, uint32_t s0_a, int row0, float (&pr)[NT][4], float (&xx)[2]) {
+            float2 xa = ptx::f2(0.f), xb = ptx::f2(0.f);  // |x|^2 partials of rows g and g+8
             float acc[2][2][NT][4];  // [k-step parity][hi, lo][nt][i]
 #pragma unroll
             for (int u = 0; u < 2; ++u)
@@ -517,6 +490,13 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
                     const int col = 16 * ks + 8 * (lj >> 1);
                     ptx::ldsm_x4(xs_a + (col >> 6) * (64 * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4), af);
                 }
+#pragma unroll
+                for (int j = 0; j < 4; j += 2) {  // af[0], af[2]: row g; af[1], af[3]: row g+8
+                    const float2 u = make_float2(__uint_as_float(af[j] << 16), __uint_as_float(af[j] & 0xffff0000u));
+                    const float2 v = make_float2(__uint_as_float(af[j + 1] << 16), __uint_as_float(af[j + 1] & 0xffff0000u));
+                    xa = ptx::f2fma(u, u, xa);
+                    xb = ptx::f2fma(v, v, xb);
+                }
                 load_b_pairs(s0_a, 16 * ks, sh, bf);  // the state rows e = 16ks..16ks+15
 #pragma unroll
                 for (int v = 0; v < 2; ++v)
@@ -528,19 +508,40 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     pr[nt][i] = (acc[0][0][nt][i] + acc[1][0][nt][i]) + (acc[0][1][nt][i] + acc[1][1][nt][i]);
+            xx[0] = xa.x + xa.y;
+            xx[1] = xb.x + xb.y;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // the quad's four lanes hold the rest of each row
+                xx[j] += __shfl_xor_sync(0xffffffffu, xx[j], 1);
+                xx[j] += __shfl_xor_sync(0xffffffffu, xx[j], 2);
+            }
+        };
+        // mu and eta of the tokens at rows row0 + g and row0 + g + 8 of chunk (or stage) k
+        auto load_mueta = [&](int k, int row0, float (&mu)[2], float (&eta)[2]) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int t = k * kTcC + row0 + g + 8 * j;
+                mu[j] = 0.f;
+                eta[j] = 1.f;
+                if (k < nch && t < T) {
+                    const size_t bth = ((size_t)b * T + t) * H + h;
+                    mu[j] = __ldg(a.mu + bth);
+                    if (a.eta) eta[j] = __ldg(a.eta + bth);
+                }
+            }
         };
         // gates of Eq. 17 (eq. beta_chunk with the chunk-start norm n) of the 16 tokens at
-        // rows row0.. of ring stage s (per-token inputs in aux buffer p):
+        // rows row0.. of ring stage s; z[hf] = (mu, eta, |x|^2, mu^2) of row g + 8hf:
         //   e2 = eta c / n^2, pn = p / n, den = mu^2 + e2^2 max(|x|^2 - pn^2, 0),
         //   g = (mu - e2 pn) / sqrt(den), kappa = n e2 / sqrt(den); den = 0 keeps the slot
-        auto gates = [&](const float (&pr)[NT][4], int s, int p, int row0, bool zero_mu, float (&gt)[NT][4],
-                         float (&kap)[NT][4], float (&qv)[NT][4]) {
+        auto gates = [&](const float (&pr)[NT][4], int s, const float4 (&zr)[2], int row0, bool zero_mu,
+                         float (&gt)[NT][4], float (&kap)[NT][4], float (&qv)[NT][4]) {
             const float* cs = reinterpret_cast<const float*>(smem + Lay::C_OFF + s * Lay::C_STAGE);
             const uint16_t* qs = reinterpret_cast<const uint16_t*>(smem + Lay::Q_OFF + s * Lay::Q_STAGE);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int tk = row0 + g + 8 * hf;
-                const float4 z = aux[p * kTcC + tk];  // mu, eta, |x|^2, mu^2
+                const float4 z = zr[hf];  // mu, eta, |x|^2, mu^2
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int u0 = 2 * nt;  // norm index of slot 8nt + 2cq
@@ -665,19 +666,27 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
         ptx::named_bar(BAR_INIT, CHAIN);  // every chain thread's zeros before any state is written
         write_state(0, smem + Lay::S0ST_OFF, 0);
         ptx::named_bar(BAR_C2, 128);
-        load_norms(0);
+        if (CH == 16) load_norms(0);
 
         if constexpr (CH == 64) {
             const int tok0 = 16 * w;  // this warp's sub-chunk
+            float mu_n[2], eta_n[2];
+            load_mueta(0, tok0, mu_n, eta_n);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % NST, p = k & 1;
                 tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
                 const uint32_t xs_a = sbase + Lay::X_OFF + s * Lay::X_STAGE;
-                float pr[NT][4];
-                project(xs_a, sbase + Lay::S0_OFF + p * Lay::S0_BUF, tok0, pr);
-                tc_wait(bar_aux0 + 8 * p, (k >> 1) & 1, abort);  // per-token inputs of chunk k
+                float pr[NT][4], xx[2];
+                project(xs_a, sbase + Lay::S0_OFF + p * Lay::S0_BUF, tok0, pr, xx);
+                load_norms(p);  // this chunk's slot norms (written with its start state), while the MMAs run
+                float4 zr[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) zr[j] = make_float4(mu_n[j], eta_n[j], xx[j], mu_n[j] * mu_n[j]);
+                // mu^2 < 2^-60 (or zero): the normaliser's argument may be denormal or zero
+                const bool zero_mu = __any_sync(0xffffffffu, !(zr[0].w >= 8.6736174e-19f) || !(zr[1].w >= 8.6736174e-19f));
+                load_mueta(k + 1, tok0, mu_n, eta_n);  // the next chunk's, in flight meanwhile
                 float gt[NT][4], kap[NT][4], qv[NT][4], R[NT][4], suf[NT][4], Gs[NT][2], qrw[NT][4];
-                gates(pr, s, p, tok0, zmu[p] != 0u, gt, kap, qv);
+                gates(pr, s, zr, tok0, zero_mu, gt, kap, qv);
                 scans(gt, R, suf, Gs);
                 if (k > 0) tc_wait(bar_p5, (k - 1) & 1, abort);  // G4/G5 of chunk k-1 are done with QR, KD
                 write_operands(kap, R, suf, qv, tok0, tok0, 16 * w, qrw, true);
@@ -756,7 +765,6 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
                 if (k + 1 < nch) {
                     write_state((k + 1) & 1, nullptr, 0);  // G4 of chunk k-1 (the buffer's last reader) is done
                     ptx::named_bar(BAR_C2, 128);
-                    load_norms((k + 1) & 1);
                 }
             }
         } else {
@@ -768,18 +776,36 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
             // writes KS into its own rows of the KT tile for its update, so one barrier per
             // chunk (the new state) remains on the chain.
             int step = 0;
+            float mu_s[4][2], eta_s[4][2];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) load_mueta(0, 16 * c, mu_s[c], eta_s[c]);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % NST, p = k & 1;
                 tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
-                tc_wait(bar_aux0 + 8 * p, (k >> 1) & 1, abort);  // per-token inputs of stage k
-                const bool zero_mu = zmu[p] != 0u;
+                float mu_c[4][2], eta_c[4][2];  // this stage's four chunks (loaded one stage ahead)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) { mu_c[c][j] = mu_s[c][j]; eta_c[c][j] = eta_s[c][j]; }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) load_mueta(k + 1, 16 * c, mu_s[c], eta_s[c]);
+                bool zero_mu = false;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) zero_mu = zero_mu || !(mu_c[c][j] * mu_c[c][j] >= 8.6736174e-19f);
+                zero_mu = __any_sync(0xffffffffu, zero_mu);  // mu^2 < 2^-60 somewhere in the stage
                 if (k > 0) tc_wait(bar_p5, (k - 1) & 1, abort);  // G4/G5 of stage k-1 are done with QR, KD
                 const uint32_t xs_a = sbase + Lay::X_OFF + s * Lay::X_STAGE;
                 for (int c = 0; c < 4; ++c, ++step) {
-                    float pr[NT][4];
-                    project(xs_a, sbase + Lay::S0_OFF + (step & 1) * Lay::S0_BUF, 16 * c, pr);
+                    float pr[NT][4], xx[2];
+                    project(xs_a, sbase + Lay::S0_OFF + (step & 1) * Lay::S0_BUF, 16 * c, pr, xx);
+                    float4 zr[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+                        zr[j] = make_float4(mu_c[c][j], eta_c[c][j], xx[j], mu_c[c][j] * mu_c[c][j]);
                     float gt[NT][4], kap[NT][4], qv[NT][4], R[NT][4], suf[NT][4], Gs[NT][2], qrw[NT][4];
-                    gates(pr, s, p, 16 * c, zero_mu, gt, kap, qv);
+                    gates(pr, s, zr, 16 * c, zero_mu, gt, kap, qv);
                     scans(gt, R, suf, Gs);
                     write_operands(kap, R, suf, qv, 16 * c, 16 * w, 16 * c, qrw, w == 0);
                     __syncwarp();

@@ -289,13 +289,30 @@ const char* lattice_status_string(lattice_status s) {
     return "unknown status";
 }
 
+// Clusters of 4 CTAs of the register-chain kernel the current device holds at once
+// (queried once per device; without a device, the SMs / 4 of a 148-SM B200).
+int reg_cluster_capacity(int d) {
+    static int cache[64][2] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return sm_count() / 4;
+    }
+    int& c = cache[dev][d == 128 ? 1 : 0];
+    if (c == 0) {
+        c = chunk_reg_max_clusters(d, 16);
+        if (c <= 0) c = -1;
+    }
+    return c > 0 ? c : sm_count() / 4;
+}
+
 lattice_impl lattice_chunk_impl(int B, int H, int m, int d, int chunk_size, lattice_dtype x_dtype,
                                 lattice_dtype q_dtype) {
     if (chunk_size <= 1) return LATTICE_IMPL_SIMT;
     const bool xb = x_dtype == LATTICE_BF16, qb = q_dtype == LATTICE_BF16;
-    if (chunk_split_supported(m, d, chunk_size, xb, qb) && B >= 1 && H >= 1 &&
-        (long long)B * H * kSpNC <= sm_count())
-        return LATTICE_IMPL_TCGEN05_SPLIT;
+    if (chunk_reg_supported(m, d, chunk_size, xb, qb) && B >= 1 && H >= 1 &&
+        (long long)B * H <= reg_cluster_capacity(d))
+        return LATTICE_IMPL_SPLIT_REG;
     if (chunk_tc_supported(m, d, chunk_size, xb, qb)) return LATTICE_IMPL_TCGEN05;
     return LATTICE_IMPL_SIMT;
 }

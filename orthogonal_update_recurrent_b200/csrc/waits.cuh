@@ -26,8 +26,8 @@ constexpr uint64_t kTcDrainNs = 4000000000ull;  // 4 s bound on each exit drain
 // when the bound elapsed or another thread already aborted.
 __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
                                         uint64_t limit_ns = kTcWaitNs) {
+    if (ptx::mbar_try_wait(bar, parity)) return *abort == 0u;  // the common case: already complete
     if (*abort) return false;
-    if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer();
     for (;;) {
         if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;  // sleep <= 20 us per try

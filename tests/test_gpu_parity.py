@@ -250,9 +250,11 @@ def test_chunked_split_and_wide_agree(L, impl):
 
 def test_chunked_automatic_choice(L):
     import torch as _t
-    assert L.chunk_impl(4, 8, 64, 64, 64) == "tcgen05_split"      # 32 sequences: 128 CTAs
-    assert L.chunk_impl(1, 16, 64, 128, 64) == "tcgen05_split"
+    assert L.chunk_impl(4, 8, 64, 64, 64) == "split_reg"          # 32 sequences: 32 clusters of 4 CTAs
+    assert L.chunk_impl(1, 16, 64, 128, 64) == "split_reg"
+    assert L.chunk_impl(4, 8, 64, 64, 16) == "split_reg"          # chunk 16 on tensor cores too
     assert L.chunk_impl(8, 16, 64, 64, 64) == "tcgen05"           # 128 sequences fill the SMs
+    assert L.chunk_impl(8, 16, 64, 64, 16) == "simt"
     assert L.chunk_impl(8, 16, 128, 128, 64) == "tcgen05"
     assert L.chunk_impl(1, 1, 128, 128, 64) == "tcgen05"          # the split kernel is for m = 64
     assert L.chunk_impl(4, 8, 128, 128, 32) == "simt"
