@@ -572,6 +572,8 @@ def main():
                          "step: time the decode step (lattice_step) on the decode workload")
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05", "tcgen05_split", "split_reg", "split_reg8"],
                     help="kernel choice of the timed scan (default: the library's automatic choice)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's sequence length T (for profiling a smaller case)")
     ap.add_argument("--chunk", type=int, default=None,
                     help="override the workload's chunk size (1: the exact recurrence)")
     args = ap.parse_args()
@@ -583,6 +585,8 @@ def main():
     w0 = LI.WORKLOADS[args.workload]
     if args.chunk is not None:
         w0 = w0.with_(chunk=args.chunk)
+    if args.tokens is not None:
+        w0 = w0.with_(T=args.tokens)
     w = rank_workload(w0, rank)
 
     if args.impl == "reference":
