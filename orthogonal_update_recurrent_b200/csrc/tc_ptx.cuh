@@ -375,6 +375,18 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
+// m16n8k8 variant (bf16): A 16x8 in two registers (a[0] = row g, cols 2c..2c+1;
+// a[1] = row g+8), B 8x8 in one (rows 2c..2c+1, col g); C as for m16n8k16.
+__device__ __forceinline__ void mma1688(float* d, const uint32_t* a, uint32_t b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(b));
+}
+// Two 8x8 b16 matrices (lanes 0-7 and 8-15 give the row addresses).
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr) : "memory");
+}
 // Four 8x8 b16 matrices from shared memory: lanes 8j..8j+7 give the row addresses of
 // matrix j (16 contiguous bytes each); lane t receives (row t/4, cols 2(t%4)..+1) of
 // matrix j in r[j]. The .trans form delivers the transpose: (rows 2(t%4)..+1, col t/4).
