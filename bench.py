@@ -144,6 +144,10 @@ CAPTURED_TRAFFIC = {
     ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.00e6 + 57.72e6,
                                                       profile="profiles/scan_bwd_kernel_small_train.md",
                                                       source="csrc/scan_bwd.cuh", sha="c2830cd3eeeb"),
+    # full-size launch, dram counters alone (one pass)
+    ("chunk_reg_kernel<16 slots>", "long_ctx"): dict(bytes=675.95e6 + 501.79e6,
+                                                    profile="profiles/chunk_reg_kernel_long_ctx.md",
+                                                    source="csrc/chunk_reg.cuh", sha="7de313fee29e"),
     # captured before the last change of step.cuh: reported as None until re-captured
     ("step_kernel", "decode"): dict(bytes=545.32e6 + 482.93e6, profile="profiles/step_kernel_decode.md",
                                     source="csrc/step.cuh", sha=None),
@@ -491,7 +495,7 @@ def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        step_ms, n = time_decode(torch, L, wd, n, ring, device)
+        step_ms, n = time_decode(torch, L, wd, n, ring, device, mode=args.mode)
     torch.cuda.synchronize()
     step_ms = max_over_ranks(torch, dist, step_ms, device)
     if rank != 0:
@@ -502,12 +506,13 @@ def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
             "n_gpus": world, "steps": n, "warmup": 3, "ms_per_step": step_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wd.name, "pass": "step", "B": wd.B, "H": wd.H, "m": wd.m, "d": wd.d,
-                       "x_q_dtype": "bf16", "state_dtype": "f32",
+                       "objective": args.mode, "x_q_dtype": "bf16", "state_dtype": "f32",
                        "l2": "state (512 MiB) and input ring exceed L2",
                        "parallelism": f"independent batches per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": gbps, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbps / pk["hbm_gbs"], "traffic": traffic_for("step_kernel", "decode"),
-                         "kernel": "step_kernel",
+                         "frac": gbps / pk["hbm_gbs"],
+                         "traffic": traffic_for("step_kernel", "decode") if args.mode == "sim" else None,
+                         "kernel": "step_kernel" if args.mode == "sim" else "step_kernel<dec>",
                          "alg_bytes_per_launch": sb, "peak_source": f"{pk_src} (burst copy)"},
             "gpu_launches": n}
     cs = clk.summary()
@@ -574,6 +579,8 @@ def main():
                     help="kernel choice of the timed scan (default: the library's automatic choice)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's sequence length T (for profiling a smaller case)")
+    ap.add_argument("--mode", default="sim", choices=["sim", "dec"],
+                    help="objective of the --pass step timing: similarity (default) or reconstruction")
     ap.add_argument("--chunk", type=int, default=None,
                     help="override the workload's chunk size (1: the exact recurrence)")
     args = ap.parse_args()
