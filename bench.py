@@ -148,10 +148,18 @@ CAPTURED_TRAFFIC = {
     ("chunk_reg_kernel<16 slots>", "long_ctx"): dict(bytes=675.95e6 + 501.79e6,
                                                     profile="profiles/chunk_reg_kernel_long_ctx.md",
                                                     source="csrc/chunk_reg.cuh", sha="7de313fee29e"),
-    # captured before the last change of step.cuh: reported as None until re-captured
-    ("step_kernel", "decode"): dict(bytes=545.32e6 + 482.93e6, profile="profiles/step_kernel_decode.md",
-                                    source="csrc/step.cuh", sha=None),
+    # the persistent decode step, dram counters alone (one pass), both objectives
+    ("step_pf_kernel", "decode"): dict(bytes=545.33e6 + 480.71e6, profile="profiles/step_kernel_decode.md",
+                                       source="csrc/step.cuh", sha="39ad7e5e1973"),
+    ("step_pf_kernel<dec>", "decode"): dict(bytes=545.36e6 + 480.70e6, profile="profiles/step_kernel_decode.md",
+                                            source="csrc/step.cuh", sha="39ad7e5e1973"),
 }
+
+
+def step_kernel_name(mode: str) -> str:
+    """The decode-step kernel the library launches on the decode workload (8192 heads,
+    more than the SMs: the persistent kernel, for either objective)."""
+    return "step_pf_kernel" if mode == "sim" else "step_pf_kernel<dec>"
 
 
 def source_sha(rel: str) -> str:
@@ -511,8 +519,8 @@ def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
                        "parallelism": f"independent batches per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": gbps, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbps / pk["hbm_gbs"],
-                         "traffic": traffic_for("step_kernel", "decode") if args.mode == "sim" else None,
-                         "kernel": "step_kernel" if args.mode == "sim" else "step_kernel<dec>",
+                         "traffic": traffic_for(step_kernel_name(args.mode), "decode"),
+                         "kernel": step_kernel_name(args.mode),
                          "alg_bytes_per_launch": sb, "peak_source": f"{pk_src} (burst copy)"},
             "gpu_launches": n}
     cs = clk.summary()
@@ -749,12 +757,14 @@ def main():
             extra["decode"] = {"us_per_step": us_ms * 1e3, "steps": n, "gbps": sb / (us_ms * 1e-3) / 1e9,
                                "hbm_frac": sb / (us_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                                "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb,
-                               "kernel": "step_kernel"}
+                               "kernel": step_kernel_name("sim"),
+                               "traffic": traffic_for(step_kernel_name("sim"), "decode")}
             us_ms, n = time_decode(torch, L, wd, 1000, 40, device, mode="dec")
             extra["decode_dec"] = {"us_per_step": us_ms * 1e3, "steps": n, "gbps": sb / (us_ms * 1e-3) / 1e9,
                                    "hbm_frac": sb / (us_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                                    "tokens_per_s": wd.B / (us_ms * 1e-3), "alg_bytes_per_step": sb,
-                                   "kernel": "step_kernel<dec>"}
+                                   "kernel": step_kernel_name("dec"),
+                                   "traffic": traffic_for(step_kernel_name("dec"), "decode")}
         line["extra"] = extra
         if not args.no_cpu:
             v, cores, sample = oracle_baseline(w, w.chunk)

@@ -633,6 +633,33 @@ def test_decode_workload_full_size_1000_steps(L):
 
 
 @pytest.mark.parametrize("mode", ["sim", "dec"])
+@pytest.mark.parametrize("m,d,xq_f32", [(128, 128, False), (64, 64, True), (7, 16, False), (256, 64, True)])
+def test_step_persistent_many_heads_per_cta(L, m, d, xq_f32, mode):
+    """4096 heads: the persistent decode kernel takes several heads per CTA, each
+    head's state (and x, c, mu, eta) copied in while the CTA computes the one before.
+    With eta, fp32 or bf16 x and q, two consecutive steps on the same state."""
+    w = LI.WORKLOADS["decode"].with_(m=m, d=d)
+    B, H, n = 64, 64, 2
+    So = LI.make_decode_state(w, B=B, H=H).astype(np.float64)
+    st = LI.make_decode_steps(w, n, B=B, H=H)
+    rng = np.random.default_rng([m, d, 17])
+    S = torch.from_numpy(So.astype(np.float32)).cuda()
+    for k in range(n):
+        one = {key: st[key][k] for key in ("x", "q", "c", "mu")}
+        one["x_bits"] = None if xq_f32 else st["x_bits"][k]
+        one["q_bits"] = None if xq_f32 else st["q_bits"][k]
+        one["eta"] = rng.uniform(0.5, 1.5, size=(B, H)).astype(np.float32)
+        t = dev_inputs(one)
+        S32 = S.cpu().numpy()
+        y = L.step(S, t["x"], t["c"], t["q"], t["mu"], eta=t["eta"], mode=mode)
+        yo, So, _ = oracle.step(S32, one["x"], one["c"], one["q"], one["mu"], eta=one["eta"], mode=mode)
+        torch.cuda.synchronize()
+        L.device_status()
+        assert y_err(y.cpu().numpy()[:, None], yo[:, None]) <= TOL_F32
+        assert s_err(S.cpu().numpy(), So) <= TOL_F32
+
+
+@pytest.mark.parametrize("mode", ["sim", "dec"])
 @pytest.mark.parametrize("m,d", [(128, 128), (64, 64), (16, 32), (7, 16), (256, 64)])
 def test_step_many_heads(L, m, d, mode):
     """320 heads, several waves of CTAs, for either objective; each step starts from
