@@ -14,12 +14,15 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblattice.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-NVCC_FLAGS = [
-    "-gencode", "arch=compute_100a,code=sm_100a",
-    "-O3", "-lineinfo", "-std=c++17",
-    "-shared", "-Xcompiler", "-fPIC,-O2", "-cudart", "static",
-    "-Xptxas", "-warn-spills", "-split-compile=0",
-]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# Each translation unit is compiled whole (no split compilation: nvcc's split mode
+# gave different register allocations, and spills, from one build to the next) and
+# the units are compiled in parallel.
+COMPILE_FLAGS = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-Xptxas", "-warn-spills"]
+LINK_FLAGS = [*ARCH, "-shared", "-cudart", "static"]
+# the C ABI and one unit per kernel family (csrc/launch.h joins them)
+UNITS = ["lattice_abi.cu", "tu_simt_exact.cu", "tu_simt_chunked.cu", "tu_step.cu", "tu_bwd.cu", "tu_tc.cu"]
+OBJDIR = os.path.join(HERE, "_build")
 
 
 def _nvcc() -> str:
@@ -30,7 +33,7 @@ def _nvcc() -> str:
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + glob.glob(os.path.join(INCLUDE, "*.h")))
+                  + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def stale() -> bool:
@@ -43,13 +46,30 @@ def stale() -> bool:
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", tmp,
-           os.path.join(CSRC, "lattice_abi.cu")]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    os.makedirs(OBJDIR, exist_ok=True)
+    tag = f"{os.getpid()}"
+    jobs = []
+    for unit in UNITS:
+        obj = os.path.join(OBJDIR, unit[:-3] + f".{tag}.o")
+        cmd = [_nvcc(), *COMPILE_FLAGS, *extra, "-I", INCLUDE, "-c", "-o", obj, os.path.join(CSRC, unit)]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        jobs.append((subprocess.Popen(cmd), obj, cmd))
+    failed = [cmd for p, _, cmd in jobs if p.wait() != 0]
+    objs = [obj for _, obj, _ in jobs]
+    try:
+        if failed:
+            raise subprocess.CalledProcessError(1, failed[0])
+        tmp = LIB + f".tmp{tag}"
+        cmd = [_nvcc(), *LINK_FLAGS, "-o", tmp, *objs]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        subprocess.check_call(cmd)
+        os.replace(tmp, LIB)
+    finally:
+        for obj in objs:
+            if os.path.exists(obj):
+                os.remove(obj)
     return LIB
 
 

@@ -20,6 +20,17 @@ constexpr unsigned int kStatusTimeout = 1u;
 
 __device__ __forceinline__ void flag_timeout() { atomicOr(&g_device_status, kStatusTimeout); }
 
+// Reads, and zeroes when set, this translation unit's copy of the status word: every
+// translation unit of the library is a module of its own with its own copy, so the C
+// ABI asks each unit in turn.
+static inline cudaError_t read_clear_module_status(unsigned int* v) {
+    unsigned int zero = 0;
+    *v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(v, g_device_status, sizeof(*v));
+    if (e == cudaSuccess && *v) e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+    return e;
+}
+
 template <int D>
 struct Octet {
     static_assert(D == 16 || D == 32 || D == 64 || D == 128, "D must be 16, 32, 64 or 128");

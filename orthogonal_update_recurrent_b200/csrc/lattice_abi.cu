@@ -1,19 +1,15 @@
 // lattice_abi.cu -- extern "C" entry points of liblattice (declared in
-// include/lattice.h): argument checks, kernel choice and launches.
+// include/lattice.h): argument checks and kernel choice. The launches live in one
+// translation unit per kernel family (tu_*.cu, through launch.h).
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
 
 #include <mutex>
 
-#include "../../include/lattice.h"
-#include "common.cuh"
-#include "scan_simt.cuh"
-#include "step.cuh"
-#include "chunk_tc.cuh"
-#include "chunk_split.cuh"
-#include "chunk_reg.cuh"
-#include "scan_bwd.cuh"
+#include "launch.h"
+#include "waits.cuh"
 
 using namespace lattice;
 
@@ -34,6 +30,10 @@ size_t dsize(lattice_dtype t) { return t == LATTICE_BF16 ? 2 : 4; }
 bool d_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
 thread_local char g_last_error[256] = "";
+
+}  // namespace
+
+namespace lattice {
 
 // SMs of the current device (148 on B200; also the answer without a device).
 int sm_count() {
@@ -68,180 +68,12 @@ int cluster_split(int B, int H, int m) {
     return (int)G;
 }
 
-lattice_status launch_clusters(const void* kernel, int grid, int block, size_t smem, int G,
-                               cudaStream_t st, void** args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3((unsigned)block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)G;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, args);
-    if (e != cudaSuccess) return cuda_fail(e);
-    return launch_status();
-}
+}  // namespace lattice
 
-// ---- exact / chunked CUDA-core scan
-template <int D, int RQ, bool CH, bool DEC, bool LIN1>
-lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
-    size_t smem = scan_smem_bytes<D>(a.m, nw, DEC);
-    auto k = scan_simt_kernel<D, RQ, CH, DEC, LIN1>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    k<<<a.B * a.H, nw * 32, smem, st>>>(a);
-    return launch_status();
-}
-
-// one cluster of a.G CTAs (8 warps each) per sequence; similarity objective
-template <int D, bool CH, bool LIN1>
-lattice_status launch_scan_simt_split(const ScanArgs& a, cudaStream_t st) {
-    const size_t smem = scan_smem_bytes<D>(a.m, 8, false, true);
-    auto k = scan_simt_kernel<D, 1, CH, false, LIN1, true>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    ScanArgs arg = a;
-    void* args[] = {&arg};
-    return launch_clusters(reinterpret_cast<const void*>(k), a.B * a.H * a.G, 256, smem, a.G, st, args);
-}
-
-template <int D, bool CH, bool DEC, bool LIN1>
-lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
-    if constexpr (!DEC) {  // the reconstruction objective couples every slot on every token
-        const int G = cluster_split(a.B, a.H, a.m);
-        if (G > 1) {
-            ScanArgs s = a;
-            s.G = G;
-            s.spc = (a.m + G - 1) / G;
-            return launch_scan_simt_split<D, CH, LIN1>(s, st);
-        }
-    }
-    const int quads = (a.m + 3) / 4;
-    if (quads <= 16) return launch_scan_simt_t<D, 1, CH, DEC, LIN1>(a, quads < 4 ? 4 : quads, st);
-    if (quads <= 32) return launch_scan_simt_t<D, 2, CH, DEC, LIN1>(a, 16, st);
-    return launch_scan_simt_t<D, 4, CH, DEC, LIN1>(a, 16, st);
-}
-
-template <bool CH, bool DEC, bool LIN1>
-lattice_status launch_scan_simt_m(const ScanArgs& a, int d, cudaStream_t st) {
-    switch (d) {
-        case 16: return launch_scan_simt_d<16, CH, DEC, LIN1>(a, st);
-        case 32: return launch_scan_simt_d<32, CH, DEC, LIN1>(a, st);
-        case 64: return launch_scan_simt_d<64, CH, DEC, LIN1>(a, st);
-        case 128: return launch_scan_simt_d<128, CH, DEC, LIN1>(a, st);
-    }
-    return LATTICE_ERR_UNSUPPORTED;
-}
-
-// exact: CH = false (LIN1 does not apply); chunked: either linearisation
-template <bool CH>
-lattice_status launch_scan_simt(const ScanArgs& a, int d, bool dec, bool lin1, cudaStream_t st) {
-    if constexpr (!CH) {
-        return dec ? launch_scan_simt_m<false, true, false>(a, d, st) : launch_scan_simt_m<false, false, false>(a, d, st);
-    } else {
-        if (lin1)
-            return dec ? launch_scan_simt_m<true, true, true>(a, d, st) : launch_scan_simt_m<true, false, true>(a, d, st);
-        return dec ? launch_scan_simt_m<true, true, false>(a, d, st) : launch_scan_simt_m<true, false, false>(a, d, st);
-    }
-}
-
-// ---- decode step / read-out: NW warps x RQ quads per warp
-void step_shape(int m, int& nw, int& rq) {
-    const int quads = (m + 3) / 4;
-    if (quads <= 8) { nw = quads; rq = 1; }
-    else if (quads <= 16) { nw = 8; rq = 2; }
-    else if (quads <= 32) { nw = 8; rq = 4; }
-    else { nw = 16; rq = 4; }
-}
-
-// The persistent decode step (step_pf_kernel): as many CTAs as fit on the device at
-// once (cached per device, m and x dtype), each taking every G-th head.
-constexpr int kStepMaxDevices = 16;
-
-template <int D, int RQ, bool DEC>
-lattice_status launch_step_pf(const StepArgs& a, int nw, int nheads, cudaStream_t st) {
-    const StepPfLayout L(a.m, D, a.x_bf16);
-    auto k = step_pf_kernel<D, RQ, DEC>;
-    static int cache[kStepMaxDevices][2][kMaxM + 1];  // CTAs resident on the device; 0 = unknown
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e);
-    int* slot = dev < kStepMaxDevices ? &cache[dev][a.x_bf16 ? 1 : 0][a.m] : nullptr;
-    int resident = slot ? *slot : 0;
-    if (resident == 0) {
-        // the largest buffer this instantiation can take (every m it serves, fp32 x), so
-        // that a later launch with a larger m never meets a smaller limit
-        const int m_max = 64 * RQ < kMaxM ? 64 * RQ : kMaxM;
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)StepPfLayout(m_max, D, false).bytes);
-        if (e != cudaSuccess) return cuda_fail(e);
-        int per_sm = 0, sms = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, nw * 32, L.bytes);
-        if (e != cudaSuccess) return cuda_fail(e);
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return cuda_fail(e);
-        if (per_sm < 1) return LATTICE_ERR_UNSUPPORTED;
-        resident = per_sm * sms;
-        if (slot) *slot = resident;
-    }
-    k<<<dim3(nheads < resident ? nheads : resident), dim3(nw * 32), L.bytes, st>>>(a);
-    return launch_status();
-}
-
-// Decode step. Under the reconstruction objective, with at least as many heads as SMs,
-// the persistent kernel streams the next head's state in while computing the current
-// one (measured at the decode shape, m = d = 128, 8192 heads: 234 us per step against
-// 277 us). Otherwise every head has its own CTA, which loads its state straight into
-// registers: the similarity objective's short arithmetic hides behind the other
-// resident CTA's loads (186 us per step there, 193 us persistent).
-template <int D, bool DEC>
-lattice_status launch_step_dm(const StepArgs& a, cudaStream_t st) {
-    int nw, rq;
-    step_shape(a.m, nw, rq);
-    const int nheads = a.B * a.H;
-    int sms = 0, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && nheads >= sms) {
-        switch (rq) {
-            case 1: return launch_step_pf<D, 1, DEC>(a, nw, nheads, st);
-            case 2: return launch_step_pf<D, 2, DEC>(a, nw, nheads, st);
-            default: return launch_step_pf<D, 4, DEC>(a, nw, nheads, st);
-        }
-    }
-    dim3 grid(nheads), block(nw * 32);
-    switch (rq) {
-        case 1: step_kernel<D, 1, DEC><<<grid, block, 0, st>>>(a); break;
-        case 2: step_kernel<D, 2, DEC><<<grid, block, 0, st>>>(a); break;
-        default: step_kernel<D, 4, DEC><<<grid, block, 0, st>>>(a); break;
-    }
-    return launch_status();
-}
-
-template <int D>
-lattice_status launch_step_d(const StepArgs& a, bool dec, cudaStream_t st) {
-    return dec ? launch_step_dm<D, true>(a, st) : launch_step_dm<D, false>(a, st);
-}
-
-template <int D>
-lattice_status launch_readout_d(const ReadoutArgs& a, cudaStream_t st) {
-    int nw, rq;
-    step_shape(a.m, nw, rq);
-    dim3 grid(a.B * a.H), block(nw * 32);
-    switch (rq) {
-        case 1: readout_kernel<D, 1><<<grid, block, 0, st>>>(a); break;
-        case 2: readout_kernel<D, 2><<<grid, block, 0, st>>>(a); break;
-        default: readout_kernel<D, 4><<<grid, block, 0, st>>>(a); break;
-    }
-    return launch_status();
-}
+namespace {
 
 // ---- backward
-constexpr int kBwdMaxM = 128;
+constexpr int kBwdMaxM = 128;  // slots per head of the backward kernels
 
 int bwd_seg(int chunk, int seg) {
     if (seg == 0) return chunk >= 64 ? chunk : chunk * ((64 + chunk - 1) / chunk);
@@ -250,53 +82,6 @@ int bwd_seg(int chunk, int seg) {
 
 // CTAs per sequence of the backward kernel (see cluster_split).
 int bwd_split(int B, int H, int m) { return cluster_split(B, H, m); }
-
-template <int D, int RQ, bool CH, bool SPLIT>
-lattice_status launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
-    constexpr int nt = bwd_threads(SPLIT);
-    const size_t smem = bwd_smem_bytes(D, a.spc, nt / 32, SPLIT);
-    auto k = scan_bwd_kernel<D, RQ, CH, SPLIT>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    if (a.G == 1) {
-        k<<<a.B * a.H, nt, smem, st>>>(a);
-        return launch_status();
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.B * a.H * a.G));
-    cfg.blockDim = dim3((unsigned)nt);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)a.G;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k, a);
-    if (e != cudaSuccess) return cuda_fail(e);
-    return launch_status();
-}
-
-// One CTA per sequence: 16 warps, one slot (m <= 64) or two (m <= 128) per octet.
-// Clusters: 8 warps per CTA, one slot per octet (bwd_split keeps <= 32 slots per CTA).
-template <int D, bool CH>
-lattice_status launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
-    if (a.G == 1) return a.m <= 64 ? launch_bwd_t<D, 1, CH, false>(a, st) : launch_bwd_t<D, 2, CH, false>(a, st);
-    return launch_bwd_t<D, 1, CH, true>(a, st);
-}
-
-template <bool CH>
-lattice_status launch_bwd(const BwdArgs& a, int d, cudaStream_t st) {
-    switch (d) {
-        case 16: return launch_bwd_d<16, CH>(a, st);
-        case 32: return launch_bwd_d<32, CH>(a, st);
-        case 64: return launch_bwd_d<64, CH>(a, st);
-        case 128: return launch_bwd_d<128, CH>(a, st);
-    }
-    return LATTICE_ERR_UNSUPPORTED;
-}
 
 // One warp waits, with the library's bounded wait, on an mbarrier that nothing ever
 // arrives on: after limit_ns the wait gives up, sets the device status word and the
@@ -339,31 +124,14 @@ const char* lattice_status_string(lattice_status s) {
     return "unknown status";
 }
 
-// Clusters of 4 CTAs of the register-chain kernel the current device holds at once
-// (queried once per device; without a device, the SMs / 4 of a 148-SM B200).
-int reg_cluster_capacity(int d) {
-    static int cache[64][2] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-        cudaGetLastError();
-        return sm_count() / 4;
-    }
-    int& c = cache[dev][d == 128 ? 1 : 0];
-    if (c == 0) {
-        c = chunk_reg_max_clusters(d, 16);
-        if (c <= 0) c = -1;
-    }
-    return c > 0 ? c : sm_count() / 4;
-}
-
 lattice_impl lattice_chunk_impl(int B, int H, int m, int d, int chunk_size, lattice_dtype x_dtype,
                                 lattice_dtype q_dtype) {
     if (chunk_size <= 1) return LATTICE_IMPL_SIMT;
     const bool xb = x_dtype == LATTICE_BF16, qb = q_dtype == LATTICE_BF16;
-    if (chunk_reg_supported(m, d, chunk_size, xb, qb) && B >= 1 && H >= 1 &&
+    if (tc_supported(LATTICE_IMPL_SPLIT_REG, m, d, chunk_size, xb, qb) && B >= 1 && H >= 1 &&
         (long long)B * H <= reg_cluster_capacity(d))
         return LATTICE_IMPL_SPLIT_REG;
-    if (chunk_tc_supported(m, d, chunk_size, xb, qb)) return LATTICE_IMPL_TCGEN05;
+    if (tc_supported(LATTICE_IMPL_TCGEN05, m, d, chunk_size, xb, qb)) return LATTICE_IMPL_TCGEN05;
     return LATTICE_IMPL_SIMT;
 }
 
@@ -419,30 +187,18 @@ lattice_status lattice_scan_fwd_ex(const void* x, lattice_dtype x_dtype, const f
     a.cnorm = cnorm && chunk_size > 1 ? 1 : 0;
     if (chunk_size == 1 && cnorm) {  // normalising after every token is the exact recurrence
         if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
-        return launch_scan_simt<false>(a, d, dec, false, st);
+        return launch_scan_simt(a, d, false, dec, false, st);
     }
     if (chunk_size == 1 || dec || lin1 || cnorm) {  // the tensor-core kernels: Eq. 17, per-token normaliser, similarity objective
         if (tc_choice) return LATTICE_ERR_UNSUPPORTED;
-        return chunk_size == 1 ? launch_scan_simt<false>(a, d, dec, false, st)
-                               : launch_scan_simt<true>(a, d, dec, lin1, st);
+        return launch_scan_simt(a, d, chunk_size > 1, dec, lin1, st);
     }
     if (impl == LATTICE_IMPL_AUTO) impl = lattice_chunk_impl(B, H, m, d, chunk_size, x_dtype, q_dtype);
-    if (impl == LATTICE_IMPL_SPLIT_REG || impl == LATTICE_IMPL_SPLIT_REG8) {
-        if (!chunk_reg_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
-        cudaError_t e = launch_chunk_reg(a, d, impl == LATTICE_IMPL_SPLIT_REG8 ? 8 : 16, st);
-        return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
+    if (impl != LATTICE_IMPL_SIMT) {
+        if (!tc_supported(impl, m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
+        return launch_tc(impl, a, d, st);
     }
-    if (impl == LATTICE_IMPL_TCGEN05_SPLIT) {
-        if (!chunk_split_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
-        cudaError_t e = launch_chunk_split(a, d, st);
-        return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
-    }
-    if (impl == LATTICE_IMPL_TCGEN05) {
-        if (!chunk_tc_supported(m, d, chunk_size, a.x_bf16, a.q_bf16)) return LATTICE_ERR_UNSUPPORTED;
-        cudaError_t e = launch_chunk_tc(a, d, st);
-        return e == cudaSuccess ? LATTICE_OK : cuda_fail(e);
-    }
-    return launch_scan_simt<true>(a, d, false, false, st);
+    return launch_scan_simt(a, d, true, false, false, st);
 }
 
 lattice_status lattice_scan_fwd_impl(const void* x, lattice_dtype x_dtype, const float* c,
@@ -485,13 +241,7 @@ lattice_status lattice_step(float* S, const void* x, lattice_dtype x_dtype, cons
         if (overlap(s, sS) || overlap(s, sy)) return LATTICE_ERR_INVALID_ARG;
     if (overlap(sS, sy)) return LATTICE_ERR_INVALID_ARG;
     StepArgs a{S, x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, y, B, H, m};
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (d) {
-        case 16: return launch_step_d<16>(a, dec, st);
-        case 32: return launch_step_d<32>(a, dec, st);
-        case 64: return launch_step_d<64>(a, dec, st);
-        default: return launch_step_d<128>(a, dec, st);
-    }
+    return launch_step(a, d, dec, static_cast<cudaStream_t>(stream));
 }
 
 lattice_status lattice_readout(const float* S, const void* q, lattice_dtype q_dtype, float* y,
@@ -506,13 +256,7 @@ lattice_status lattice_readout(const float* S, const void* q, lattice_dtype q_dt
     if (overlap(sy, span(S, nbh * m * d * 4)) || overlap(sy, span(q, nbh * m * dsize(q_dtype))))
         return LATTICE_ERR_INVALID_ARG;
     ReadoutArgs a{S, q, q_dtype == LATTICE_BF16, y, B, H, m};
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (d) {
-        case 16: return launch_readout_d<16>(a, st);
-        case 32: return launch_readout_d<32>(a, st);
-        case 64: return launch_readout_d<64>(a, st);
-        default: return launch_readout_d<128>(a, st);
-    }
+    return launch_readout(a, d, static_cast<cudaStream_t>(stream));
 }
 
 size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int chunk_size,
@@ -570,8 +314,7 @@ lattice_status lattice_scan_bwd(const void* x, lattice_dtype x_dtype, const floa
     BwdArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, dy, dS_T,
               dx, dc, dq, dmu, deta_w, dS0, static_cast<float*>(workspace), B, T, H, m, chunk_size, seg,
               G, (m + G - 1) / G};
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return chunk_size == 1 ? launch_bwd<false>(a, d, st) : launch_bwd<true>(a, d, st);
+    return launch_bwd(a, d, static_cast<cudaStream_t>(stream));
 }
 
 lattice_status lattice_selftest_bounded_wait(unsigned long long limit_ns, void* stream) {
@@ -584,12 +327,17 @@ lattice_status lattice_get_device_status(void* stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e);
-    unsigned int v = 0, zero = 0;
-    e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
-    if (e != cudaSuccess) return cuda_fail(e);
-    if (v && (e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero))) != cudaSuccess)
-        return cuda_fail(e);
-    return v ? LATTICE_ERR_TIMEOUT : LATTICE_OK;
+    // every translation unit's copy of the status word (each unit is a module of its own)
+    cudaError_t (*const units[])(unsigned int*) = {read_clear_module_status, status_simt_exact,
+                                                   status_simt_chunked, status_step, status_bwd, status_tc};
+    unsigned int any = 0;
+    for (auto unit : units) {
+        unsigned int v = 0;
+        e = unit(&v);
+        if (e != cudaSuccess) return cuda_fail(e);
+        any |= v;
+    }
+    return any ? LATTICE_ERR_TIMEOUT : LATTICE_OK;
 }
 
 const char* lattice_last_cuda_error(void) { return g_last_error; }

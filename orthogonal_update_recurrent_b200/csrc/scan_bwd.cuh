@@ -28,6 +28,7 @@
 // the warp by shuffles and across warps through shared memory in a fixed order,
 // so results are bit-reproducible.
 #pragma once
+#include "args.h"
 #include "common.cuh"
 
 namespace lattice {
@@ -35,23 +36,6 @@ namespace lattice {
 constexpr int kBwdTB = 8;        // tokens per staged block
 constexpr int kBwdTBSplit = 16;  // cluster kernels: longer blocks, half the cluster barriers
 
-struct BwdArgs {
-    const void* x; bool x_bf16;
-    const float* c;
-    const void* q; bool q_bf16;
-    const float* mu;
-    const float* eta;  // may be null (=> 1)
-    const float* S0;
-    const float* dy;
-    const float* dST;  // may be null (=> 0)
-    float* dx; float* dc; float* dq; float* dmu;
-    float* deta;       // may be null
-    float* dS0;
-    float* ws;         // workspace: per (b,h) and CTA, (nseg - 1) checkpoints then the L-token tape
-    int B, T, H, m, chunk, seg;
-    int G;             // CTAs per sequence (a cluster when > 1)
-    int spc;           // slots per CTA
-};
 
 // Staged record per token: x[D] | dy[D] | q[spc] | c[spc] | mu | eta (q and c of
 // this CTA's slots only), padded so that every record (and its dy) starts 16-byte
@@ -87,11 +71,6 @@ __device__ __forceinline__ float bwd_ld_peer(const float* local_ptr, uint32_t ra
     return v;
 }
 
-// Floats of workspace per (b,h) sequence.
-__host__ __device__ inline size_t bwd_ws_floats_per_seq(int T, int m, int D, int seg) {
-    const int nseg = T > 0 ? (T + seg - 1) / seg : 1;
-    return (size_t)(nseg - 1 + seg) * m * D;
-}
 
 // Forward coefficients of one slot and token, with the intermediates the adjoint needs.
 struct SlotFwd {

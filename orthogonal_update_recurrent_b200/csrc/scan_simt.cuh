@@ -15,28 +15,13 @@
 // normaliser n/sqrt(mu^2 n^2 + |Delta|^2) keeps the chunk-start norm n (the
 // paper's Appendix D listing scales its rsqrt by the slot norm).
 #pragma once
+#include "args.h"
 #include "common.cuh"
 
 namespace lattice {
 
 constexpr int kScanTB = 8;       // tokens per staged block
 constexpr int kScanTBSplit = 16;  // split kernels: longer blocks, half the cluster barriers
-constexpr int kMaxM = 256;
-
-struct ScanArgs {
-    const void* x; bool x_bf16;
-    const float* c;
-    const void* q; bool q_bf16;
-    const float* mu;
-    const float* eta;            // may be null (=> 1)
-    const float* S0;
-    float* S_out;
-    float* y;
-    int B, T, H, m, chunk;
-    int cnorm;  // chunked CUDA-core path: no per-token normaliser, unit slots after each chunk
-    int G;      // SPLIT kernels: CTAs per sequence (a cluster), each owning spc slots
-    int spc;
-};
 
 // Per-token staged record: x[D] | q[m] | c[m] | mu | eta, padded to a multiple
 // of 4 floats so that every record starts 16-byte aligned.

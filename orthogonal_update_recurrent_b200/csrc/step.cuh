@@ -7,22 +7,13 @@
 // bytes of traffic per head) dominates, so each lane issues all of its
 // streaming 16-byte loads before any arithmetic.
 #pragma once
+#include "args.h"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "waits.cuh"
 
 namespace lattice {
 
-struct StepArgs {
-    float* S;
-    const void* x; bool x_bf16;
-    const float* c;
-    const void* q; bool q_bf16;
-    const float* mu;
-    const float* eta;  // may be null
-    float* y;
-    int B, H, m;
-};
 
 // The step of one head, after its state rows (s), input (xv), mu and eta are in
 // registers; cv(r) and qv(r) give the intensity and query of the lane's slot r (from
@@ -351,12 +342,6 @@ __global__ void __launch_bounds__(512) step_pf_kernel(StepArgs a) {
     if (pending && tid == 0) tc_drain(bar, it & 1);
 }
 
-struct ReadoutArgs {
-    const float* S;
-    const void* q; bool q_bf16;
-    float* y;
-    int B, H, m;
-};
 
 // y[b][h][:] = sum_i q_i s_i (§2 eq. LA read-out; Appendix D y = q @ S).
 template <int D, int RQ>
