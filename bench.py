@@ -135,24 +135,26 @@ CAPTURED_TRAFFIC = {
                                                 source="csrc/chunk_split.cuh", sha="047d8e41962f"),
     ("chunk_split_kernel", "long_ctx"): dict(bytes=676.05e6 + 498.46e6, profile="profiles/chunk_split_kernel_full.md",
                                              source="csrc/chunk_split.cuh", sha="047d8e41962f"),
-    # (chunk_tc.cuh since changed only by moving its wait helpers, verbatim, into waits.cuh)
-    ("chunk_tc_kernel", "mid_layer"): dict(bytes=550.62e6 + 240.43e6, profile="profiles/chunk_tc_kernel_full.md",
+    ("chunk_tc_kernel", "mid_layer"): dict(bytes=551.09e6 + 236.40e6, profile="profiles/chunk_tc_kernel_full.md",
                                            source="csrc/chunk_tc.cuh", sha="9b76f603cace"),
-    ("scan_simt_kernel<exact>", "small_train"): dict(bytes=34.43e6 + 0.02e6,
+    ("scan_simt_kernel<exact>", "small_train"): dict(bytes=34.43e6 + 0.04e6,
                                                      profile="profiles/scan_simt_kernel_exact_small_train.md",
-                                                     source="csrc/scan_simt.cuh", sha="b1b556e2f5cf"),
-    ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.00e6 + 57.72e6,
+                                                     source="csrc/scan_simt.cuh", sha="327f91817ab8"),
+    ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.41e6 + 54.81e6,
                                                       profile="profiles/scan_bwd_kernel_small_train.md",
-                                                      source="csrc/scan_bwd.cuh", sha="c2830cd3eeeb"),
-    # full-size launch, dram counters alone (one pass)
+                                                      source="csrc/scan_bwd.cuh", sha="3fa6eb987d11"),
+    # full-size launches, dram counters alone (one pass)
     ("chunk_reg_kernel<16 slots>", "long_ctx"): dict(bytes=675.95e6 + 501.79e6,
                                                     profile="profiles/chunk_reg_kernel_long_ctx.md",
                                                     source="csrc/chunk_reg.cuh", sha="7de313fee29e"),
-    # the persistent decode step, dram counters alone (one pass), both objectives
-    ("step_pf_kernel", "decode"): dict(bytes=545.33e6 + 480.71e6, profile="profiles/step_kernel_decode.md",
-                                       source="csrc/step.cuh", sha="39ad7e5e1973"),
-    ("step_pf_kernel<dec>", "decode"): dict(bytes=545.36e6 + 480.70e6, profile="profiles/step_kernel_decode.md",
-                                            source="csrc/step.cuh", sha="39ad7e5e1973"),
+    ("chunk_reg_kernel<16 slots>", "small_train"): dict(bytes=34.40e6 + 0.05e6,
+                                                       profile="profiles/chunk_reg_kernel_small_train.md",
+                                                       source="csrc/chunk_reg.cuh", sha="7de313fee29e"),
+    # the persistent decode step, both objectives
+    ("step_pf_kernel", "decode"): dict(bytes=545.33e6 + 480.69e6, profile="profiles/step_kernel_decode.md",
+                                       source="csrc/step.cuh", sha="71553fca01a5"),
+    ("step_pf_kernel<dec>", "decode"): dict(bytes=545.34e6 + 480.52e6, profile="profiles/step_kernel_decode.md",
+                                            source="csrc/step.cuh", sha="71553fca01a5"),
 }
 
 
