@@ -86,8 +86,9 @@ struct RgLayout {
     // straight into its receive buffer), moved by one bulk copy per peer
     static constexpr uint32_t PEER_BLOCK = kTcC * DSL * 4;
     static constexpr uint32_t STG_OFF = RECV_OFF + RECV_BYTES;
-    static constexpr uint32_t AUX_OFF = STG_OFF + (NC - 1) * PEER_BLOCK;  // [2][C] float4: mu, eta, |x|^2, mu^2
-    static constexpr uint32_t GSUB_OFF = AUX_OFF + 2 * kTcC * 16;   // [4 sub-chunks][16] (SPC used)
+    // mu, eta of each ring stage's 64 tokens, [NST][C][2] fp32, copied by the TMA warp's lanes
+    static constexpr uint32_t MUE_OFF = STG_OFF + (NC - 1) * PEER_BLOCK;
+    static constexpr uint32_t GSUB_OFF = MUE_OFF + 4 * kTcC * 2 * 4;  // [4 sub-chunks][16] (SPC used)
     static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * 16 * 4;        // [2][4 warps][16] (SPC used)
     static constexpr uint32_t BAR_OFF = TSQ_OFF + 2 * 4 * 16 * 4;
     static constexpr int NBAR = 2 * NST + 8;
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
     if (warp == MMA_WARP) {
         if (lane == 0) {
             for (int s = 0; s < NST; ++s) {
-                ptx::mbar_init(bar_full0 + 8 * s, 1);
+                ptx::mbar_init(bar_full0 + 8 * s, 1 + 32);  // TMA bytes + the TMA warp's 32 copy arrivals
                 ptx::mbar_init(bar_empty0 + 8 * s, CHAIN / 32 + 1);
             }
             ptx::mbar_init(bar_p5, 1);
@@ -222,8 +223,13 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
         }
         if (nch > 0) tc_drain(bar_y, (nch - 1) & 1);
     } else if (warp == TMA_WARP) {
-        // ------------------------------------------------------------ TMA issue (lane 0)
-        if (lane == 0 && nch > 0) {
+        // ------------------------------------------------------------ TMA issue
+        // Lane 0 issues the tensor copies of x, q and c of each 64-token stage; every lane
+        // copies mu and eta of two of its tokens (cp.async, 4 bytes: a token's mu is one
+        // float at a stride of H floats, too narrow for a tensor copy) and arrives on the
+        // stage's full barrier once they have landed, so the chain warps find the
+        // per-token inputs in shared memory with the rest of the stage.
+        if (nch > 0) {
             const int s_lo = rank * SPC;  // this CTA's slots in the q and c rows
             int last[NST];
 #pragma unroll
@@ -234,27 +240,45 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
                 ptx::tma_prefetch_l2_4d(&maps.q, s_lo, h, k * kTcC, b);
                 ptx::tma_prefetch_l2_4d(&maps.c, s_lo, h, k * kTcC, b);
             };
-            ptx::prefetch_tensormap(&maps.x);
-            ptx::prefetch_tensormap(&maps.q);
-            ptx::prefetch_tensormap(&maps.c);
-            for (int k = NST; k < NST + 4 && k < nch; ++k) prefetch_l2(k);
+            if (lane == 0) {
+                ptx::prefetch_tensormap(&maps.x);
+                ptx::prefetch_tensormap(&maps.q);
+                ptx::prefetch_tensormap(&maps.c);
+                for (int k = NST; k < NST + 4 && k < nch; ++k) prefetch_l2(k);
+            }
             for (int k = 0; k < nch; ++k) {
                 const int s = k % NST;
-                if (k >= NST && !tc_wait(bar_empty0 + 8 * s, ((k / NST) - 1) & 1, abort)) break;
+                if (k >= NST && !tc_wait_warp(bar_empty0 + 8 * s, ((k / NST) - 1) & 1, abort)) break;
                 const uint32_t full = bar_full0 + 8 * s;
-                ptx::mbar_arrive_expect_tx(full, Lay::STAGE_TX);
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(full, Lay::STAGE_TX);
 #pragma unroll
-                for (int kb = 0; kb < DS / 64; ++kb)
-                    ptx::tma_load_4d(sbase + Lay::X_OFF + s * Lay::X_STAGE + kb * (64 * 128), &maps.x, full,
-                                     kb * 64, h, k * kTcC, b);
-                ptx::tma_load_4d(sbase + Lay::Q_OFF + s * Lay::Q_STAGE, &maps.q, full, s_lo, h, k * kTcC, b);
-                ptx::tma_load_4d(sbase + Lay::C_OFF + s * Lay::C_STAGE, &maps.c, full, s_lo, h, k * kTcC, b);
+                    for (int kb = 0; kb < DS / 64; ++kb)
+                        ptx::tma_load_4d(sbase + Lay::X_OFF + s * Lay::X_STAGE + kb * (64 * 128), &maps.x, full,
+                                         kb * 64, h, k * kTcC, b);
+                    ptx::tma_load_4d(sbase + Lay::Q_OFF + s * Lay::Q_STAGE, &maps.q, full, s_lo, h, k * kTcC, b);
+                    ptx::tma_load_4d(sbase + Lay::C_OFF + s * Lay::C_STAGE, &maps.c, full, s_lo, h, k * kTcC, b);
+                }
+                const uint32_t me = sbase + Lay::MUE_OFF + s * (kTcC * 8);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int tau = lane + 32 * j, t = k * kTcC + tau;
+                    if (t < T) {
+                        const size_t bth = ((size_t)b * T + t) * H + h;
+                        ptx::cp_async4(me + tau * 8, a.mu + bth);
+                        if (a.eta) ptx::cp_async4(me + tau * 8 + 4, a.eta + bth);
+                    }
+                }
+                ptx::cp_async_mbar_arrive_noinc(full);
                 last[s] = k;
-                if (k + NST + 4 < nch) prefetch_l2(k + NST + 4);
+                if (lane == 0 && k + NST + 4 < nch) prefetch_l2(k + NST + 4);
             }
+            ptx::cp_async_wait_all();
+            if (lane == 0) {
 #pragma unroll
-            for (int s = 0; s < NST; ++s)  // no TMA write may be in flight when the CTA retires
-                if (last[s] >= 0) tc_drain(bar_full0 + 8 * s, (last[s] / NST) & 1);
+                for (int s = 0; s < NST; ++s)  // no TMA write may be in flight when the CTA retires
+                    if (last[s] >= 0) tc_drain(bar_full0 + 8 * s, (last[s] / NST) & 1);
+            }
         }
         __syncwarp();
     } else if (warp >= RO_WARP0) {
@@ -517,16 +541,19 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
             }
         };
         // mu and eta of the tokens at rows row0 + g and row0 + g + 8 of chunk (or stage) k
-        auto load_mueta = [&](int k, int row0, float (&mu)[2], float (&eta)[2]) {
+        // mu and eta of the tokens at rows row0 + g and row0 + g + 8 of ring stage s (stage
+        // k), from the shared memory the TMA warp's lanes copied them into. Loaded by the
+        // chain warps themselves, their latency landed on the chain.
+        auto stage_mueta = [&](int s, int k, int row0, float (&mu)[2], float (&eta)[2]) {
+            const float* me = reinterpret_cast<const float*>(smem + Lay::MUE_OFF) + s * (kTcC * 2);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int t = k * kTcC + row0 + g + 8 * j;
+                const int tau = row0 + g + 8 * j;
                 mu[j] = 0.f;
                 eta[j] = 1.f;
-                if (k < nch && t < T) {
-                    const size_t bth = ((size_t)b * T + t) * H + h;
-                    mu[j] = __ldg(a.mu + bth);
-                    if (a.eta) eta[j] = __ldg(a.eta + bth);
+                if (k * kTcC + tau < T) {
+                    mu[j] = me[2 * tau];
+                    if (a.eta) eta[j] = me[2 * tau + 1];
                 }
             }
         };
@@ -670,8 +697,6 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
 
         if constexpr (CH == 64) {
             const int tok0 = 16 * w;  // this warp's sub-chunk
-            float mu_n[2], eta_n[2];
-            load_mueta(0, tok0, mu_n, eta_n);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % NST, p = k & 1;
                 tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
@@ -679,12 +704,13 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
                 float pr[NT][4], xx[2];
                 project(xs_a, sbase + Lay::S0_OFF + p * Lay::S0_BUF, tok0, pr, xx);
                 load_norms(p);  // this chunk's slot norms (written with its start state), while the MMAs run
+                float mu_n[2], eta_n[2];
+                stage_mueta(s, k, tok0, mu_n, eta_n);
                 float4 zr[2];
 #pragma unroll
                 for (int j = 0; j < 2; ++j) zr[j] = make_float4(mu_n[j], eta_n[j], xx[j], mu_n[j] * mu_n[j]);
                 // mu^2 < 2^-60 (or zero): the normaliser's argument may be denormal or zero
                 const bool zero_mu = __any_sync(0xffffffffu, !(zr[0].w >= 8.6736174e-19f) || !(zr[1].w >= 8.6736174e-19f));
-                load_mueta(k + 1, tok0, mu_n, eta_n);  // the next chunk's, in flight meanwhile
                 float gt[NT][4], kap[NT][4], qv[NT][4], R[NT][4], suf[NT][4], Gs[NT][2], qrw[NT][4];
                 gates(pr, s, zr, tok0, zero_mu, gt, kap, qv);
                 scans(gt, R, suf, Gs);
@@ -776,19 +802,12 @@ __global__ void __launch_bounds__(RgLayout<DS, SPC, CH>::THREADS, 1)
             // writes KS into its own rows of the KT tile for its update, so one barrier per
             // chunk (the new state) remains on the chain.
             int step = 0;
-            float mu_s[4][2], eta_s[4][2];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) load_mueta(0, 16 * c, mu_s[c], eta_s[c]);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % NST, p = k & 1;
                 tc_wait(bar_full0 + 8 * s, (k / NST) & 1, abort);
-                float mu_c[4][2], eta_c[4][2];  // this stage's four chunks (loaded one stage ahead)
+                float mu_c[4][2], eta_c[4][2];  // this stage's four chunks
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) { mu_c[c][j] = mu_s[c][j]; eta_c[c][j] = eta_s[c][j]; }
-#pragma unroll
-                for (int c = 0; c < 4; ++c) load_mueta(k + 1, 16 * c, mu_s[c], eta_s[c]);
+                for (int c = 0; c < 4; ++c) stage_mueta(s, k, 16 * c, mu_c[c], eta_c[c]);
                 bool zero_mu = false;
 #pragma unroll
                 for (int c = 0; c < 4; ++c)

@@ -80,7 +80,8 @@ struct TcLayout {
     static constexpr uint32_t KD_OFF = QR_OFF + 4 * ROW_TILE;
     static constexpr uint32_t P_OFF = KD_OFF + ROW_TILE;           // [C][128 B]
     static constexpr uint32_t AUX_OFF = P_OFF + kTcC * 128;        // [NST][C/2][2] float4
-    static constexpr uint32_t GSUB_OFF = AUX_OFF + NST * kTcC * 16;   // [4][m] float
+    static constexpr uint32_t MUETA_OFF = AUX_OFF + NST * kTcC * 16;  // [C] {mu, eta}, with the q/c stage
+    static constexpr uint32_t GSUB_OFF = MUETA_OFF + kTcC * 8;        // [4][m] float
     static constexpr uint32_t TSQ_OFF = GSUB_OFF + 4 * MS * 4;        // [4][m] float
     static constexpr uint32_t BAR_OFF = TSQ_OFF + 4 * MS * 4;         // 8 mbarriers
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * 8;
@@ -99,6 +100,7 @@ struct TcLayout {
     static constexpr uint32_t S0LO_TCOL = S0HI_TCOL + DS / 2;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(S0LO_TCOL + DS / 2 <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
     static constexpr uint32_t TX_BYTES = X_STAGE;
     static constexpr uint32_t QC_BYTES = Q_TILE + C_TILE;
 };
@@ -168,6 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == MMA_WARP) {
         if (lane == 0) {
             for (int j = 0; j < 8; ++j) ptx::mbar_init(sbase + Lay::BAR_OFF + 8 * j, 1);
+            ptx::mbar_init(bar_qc, 1 + 32);  // TMA bytes + the TMA warp's 32 copy arrivals (mu, eta)
             *abort = 0u;
             zmu[0] = 0u;
             zmu[1] = 0u;
@@ -284,11 +287,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ptx::tma_load_4d(sbase + Lay::X_OFF + s * Lay::X_STAGE + kb * (64 * 128), &maps.x, bar,
                                      kb * 64, h, k * kTcC, b);
             };
-            auto issue_qc = [&](int k) {  // q and c of chunk k -> the single q/c stage
+            // q and c of chunk k -> the single q/c stage (lane 0, tensor copies), with mu and
+            // eta of its 64 tokens (every lane two tokens, cp.async: a token's mu is one float
+            // at a stride of H floats, too narrow for a tensor copy); each lane arrives on the
+            // stage's barrier once its copies have landed. Called by every lane.
+            auto issue_qc = [&](int k) {
                 last_qc = k;
-                ptx::mbar_arrive_expect_tx(bar_qc, Lay::QC_BYTES);
-                ptx::tma_load_4d(sbase + Lay::Q_OFF, &maps.q, bar_qc, 0, h, k * kTcC, b);
-                ptx::tma_load_4d(sbase + Lay::CC_OFF, &maps.c, bar_qc, 0, h, k * kTcC, b);
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(bar_qc, Lay::QC_BYTES);
+                    ptx::tma_load_4d(sbase + Lay::Q_OFF, &maps.q, bar_qc, 0, h, k * kTcC, b);
+                    ptx::tma_load_4d(sbase + Lay::CC_OFF, &maps.c, bar_qc, 0, h, k * kTcC, b);
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int tau = lane + 32 * j, t = k * kTcC + tau;
+                    if (t < T) {
+                        const size_t bth = ((size_t)b * T + t) * H + h;
+                        ptx::cp_async4(sbase + Lay::MUETA_OFF + tau * 8, a.mu + bth);
+                        if (a.eta) ptx::cp_async4(sbase + Lay::MUETA_OFF + tau * 8 + 4, a.eta + bth);
+                    }
+                }
+                ptx::cp_async_mbar_arrive_noinc(bar_qc);
             };
             auto prefetch_l2 = [&](int k) {  // X, q and c of chunk k into L2
 #pragma unroll
@@ -301,14 +320,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ptx::prefetch_tensormap(&maps.q);
                 ptx::prefetch_tensormap(&maps.c);
                 issue_x(0);
-                issue_qc(0);
+            }
+            if (nch > 0) issue_qc(0);
+            if (lane == 0 && nch > 0) {
                 if (nch > 1) issue_x(1);
                 for (int j = 1; j < 4 && j < nch; ++j) prefetch_l2(j);
             }
             for (int k = 0; k < nch; ++k) {
-                ptx::named_bar(BAR_G, N_WM);  // every worker is done reading q and c of chunk k
+                ptx::named_bar(BAR_G, N_WM);  // every worker is done reading q, c and mu, eta of chunk k
+                if (k + 1 < nch) issue_qc(k + 1);
                 if (lane == 0) {
-                    if (k + 1 < nch) issue_qc(k + 1);
                     // X of chunk k is read last by G6_k; then its stage takes chunk k+2
                     if (k + 2 < nch && tc_wait(bar_y, k & 1, abort)) {
                         issue_x(k + 2);
@@ -317,6 +338,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 __syncwarp();
             }
+            ptx::cp_async_wait_all();
             if (lane == 0) {  // no TMA write may be in flight when the CTA retires
 #pragma unroll
                 for (int s = 0; s < 2; ++s)
@@ -362,22 +384,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ptx::tmem_st<DCOL / 2>(tmem + lane_base + Lay::S0HI_TCOL + col0 / 2, hw);
             ptx::tmem_st<DCOL / 2>(tmem + lane_base + Lay::S0LO_TCOL + col0 / 2, lw);
         };
-        auto load_mueta = [&](int k, float& mu, float& eta) {  // this lane's token of aux_part(k)
-            const int t = k * kTcC + 4 * warp + (lane >> 3);
-            mu = 0.f;
-            eta = 1.f;
-            if ((lane & 7) == 0 && t < T) {
-                const size_t bth = ((size_t)b * T + t) * H + h;
-                mu = __ldg(a.mu + bth);
-                if (a.eta) eta = __ldg(a.eta + bth);
-            }
-        };
+        // mu and eta of chunk k, copied by the TMA warp's lanes with the chunk's q and c
+        // (loaded by the workers themselves, their latency landed on the chunk)
+        const float* mueta = reinterpret_cast<const float*>(smem + Lay::MUETA_OFF);
         // per-token mu, eta, |x|^2, mu^2 of 4 tokens of chunk k (this warp's share) into
         // aux[k % 2], laid out per token pair {mu0 mu1 eta0 eta1 | xx0 xx1 mu2_0 mu2_1}
-        auto aux_part = [&](int k, float mu, float eta) {
+        auto aux_part = [&](int k) {
             const int s = k & 1;
             const int u = lane >> 3, part = lane & 7;
             const int tau = 4 * warp + u;
+            tc_wait(bar_qc, k & 1, abort);  // the q/c stage of chunk k, with its mu and eta
+            float mu = 0.f, eta = 1.f;
+            if (part == 0 && k * kTcC + tau < T) {
+                mu = mueta[tau * 2];
+                if (a.eta) eta = mueta[tau * 2 + 1];
+            }
             const bool ok = tc_wait(bar_full0 + 8 * s, (k >> 1) & 1, abort);
             const uint8_t* xs = smem + Lay::X_OFF + s * Lay::X_STAGE;
             float2 acc = ptx::f2(0.f);
@@ -442,9 +463,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (active) tsqp[sb * MS + i] = ns;
         }
         if (nch > 0) {
-            float mu0, eta0;
-            load_mueta(0, mu0, eta0);
-            aux_part(0, mu0, eta0);
+            aux_part(0);
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
@@ -466,8 +485,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int k = 0; k < nch; ++k) {
             const int s = k & 1;
             // ---- phase A: gates of this group's 16 tokens (needs D1 = S0 . X_k^T)
-            float mu1, eta1;  // next chunk's gate inputs, stored at the end of phase B
-            if (k + 1 < nch) load_mueta(k + 1, mu1, eta1);
             tc_wait(bar_d1, k & 1, abort);
             __syncwarp();
             ptx::tc_fence_after();
@@ -682,7 +699,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
             }
-            if (k + 1 < nch) aux_part(k + 1, mu1, eta1);
+            if (k + 1 < nch) aux_part(k + 1);
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::named_bar(BAR_P, N_WM);
