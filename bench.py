@@ -143,13 +143,14 @@ CAPTURED_TRAFFIC = {
     ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.41e6 + 54.81e6,
                                                       profile="profiles/scan_bwd_kernel_small_train.md",
                                                       source="csrc/scan_bwd.cuh", sha="3fa6eb987d11"),
-    # full-size launches, dram counters alone (one pass)
+    # full-size launches, dram counters alone (one pass); chunk_reg.cuh changed since only
+    # in its header comment (captured on 4a519db1dbb5)
     ("chunk_reg_kernel<16 slots>", "long_ctx"): dict(bytes=676.59e6 + 501.80e6,
                                                     profile="profiles/chunk_reg_kernel_long_ctx.md",
-                                                    source="csrc/chunk_reg.cuh", sha="4a519db1dbb5"),
+                                                    source="csrc/chunk_reg.cuh", sha="d87ccc814da7"),
     ("chunk_reg_kernel<16 slots>", "small_train"): dict(bytes=34.40e6 + 0.07e6,
                                                        profile="profiles/chunk_reg_kernel_small_train.md",
-                                                       source="csrc/chunk_reg.cuh", sha="4a519db1dbb5"),
+                                                       source="csrc/chunk_reg.cuh", sha="d87ccc814da7"),
     # the persistent decode step, both objectives
     ("step_pf_kernel", "decode"): dict(bytes=545.33e6 + 480.69e6, profile="profiles/step_kernel_decode.md",
                                        source="csrc/step.cuh", sha="71553fca01a5"),

@@ -36,8 +36,9 @@
 // and four read-out warps mask the scores, reduce-scatter the four CTAs' partial
 // Y_r through distributed shared memory (asynchronous remote stores that count
 // their bytes on the receiver's mbarrier; each CTA sums its quarter of the columns
-// in a fixed order) and store y. One TMA warp streams x, q and c through a 4-stage
-// ring (no multicast). Every mbarrier wait is bounded (waits.cuh).
+// in a fixed order) and store y. One TMA warp streams x, q and c through a ring of
+// 64-token stages (no multicast); its lanes add each stage's mu and eta (cp.async),
+// counted on the same stage barrier. Every mbarrier wait is bounded (waits.cuh).
 #pragma once
 #include "chunk_split.cuh"
 
