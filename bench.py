@@ -738,6 +738,13 @@ def main():
                                                 "kernel": "scan_simt_kernel<chunked, dec>",
                                                 "inputs": "c = sigmoid(N(-4,1))"}
             del tdc
+            # chunk 16, the throughput figure's other chunk size: the register-chain kernel
+            # (four chunks per 64-token stage) and the CUDA-core kernel
+            t16 = statistics.mean(time_scan(torch, L, ts, 16, 5, 3, flush=flush))
+            t16s = statistics.mean(time_scan(torch, L, ts, 16, 5, 3, flush=flush, impl="simt"))
+            extra["small_train_chunk16"] = {"ms": t16, "tokens_per_s": tok(t16),
+                                            "kernel": kernel_name(L, ws, 16),
+                                            "simt_ms": t16s, "simt_tokens_per_s": tok(t16s)}
             # the normalisation ablation of Appendix C (CUDA-core kernel)
             tn = statistics.mean(time_scan(torch, L, ts, ws.chunk, 5, 3, flush=flush, norm="chunk"))
             extra["small_train_chunk_norm"] = {"ms": tn, "tokens_per_s": tok(tn),
