@@ -207,6 +207,27 @@ def test_chunked_tcgen05_eta_and_gate_edges(L, m, impl):
     assert s_err(Sg, So) <= TOL_TC
 
 
+@pytest.mark.parametrize("impl", ["split_reg", "split_reg8"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_chunked_reg_chunk16_eta_and_gate_edges(L, d, impl):
+    """Chunk 16 on the register-chain kernels with eta given (per-token inputs staged with
+    each 64-token stage), mu = 1 and mu = 0 tokens, a zero-norm update, zero
+    intensities, duplicates and a ragged last stage."""
+    w = LI.Workload("t", B=2, T=150, H=2, m=64, d=d, dup_frac=0.1, seed=78 + d)
+    inp = LI.make_inputs(w)
+    rng = np.random.default_rng(2)
+    inp["eta"] = rng.uniform(0.3, 1.5, inp["mu"].shape).astype(np.float32)
+    inp["mu"][:, 10] = 1.0
+    inp["mu"][:, 70] = 0.0
+    inp["c"][:, 20] = 0.0
+    inp["mu"][:, 100] = 0.0
+    inp["c"][:, 100] = 0.0
+    yg, Sg = run_gpu(L, inp, 16, impl=impl)
+    yo, So = run_oracle(inp, 16)
+    assert y_err(yg, yo) <= TOL_TC
+    assert s_err(Sg, So) <= TOL_TC
+
+
 # ------------------------------- chunked (Eq. 17), slots split over a cluster
 
 @pytest.mark.parametrize("impl", ["tcgen05_split", "split_reg", "split_reg8"])
