@@ -28,20 +28,22 @@
 //   G1: D1  [m x C]  = (S0hi + S0lo) . X^T       projections x_t . s0_i (A in TMEM)
 //   G7: T   [m x d] += (KShi + KSlo)^T . X       state update (A in TMEM)
 //   G4: Y^T [d x C]  = S0hi^T . QR_0^T           inter-chunk read-out (smem operands)
-//   G5: P   [C x 16] = QR_b . KD_b^T, b = 0..3    scores, one 16-column block each
 //   G6: Y^T [d x C] += X^T . P_causal^T          intra-chunk read-out
+// and the causal scores P = QR_b . KD_b^T (16 x 16 blocks, keys of sub-chunk b) with
+// warp-synchronous MMAs (mma.sync) on two warps of their own.
 //
 // Warp roles (640 threads, 5 warpgroups). Warps 0-15 are workers: warp 4*sb + q
 // owns TMEM lane quadrant q (slots 32q..32q+31) and sub-chunk sb. It computes
 // the gates of tokens 16sb..16sb+15 for its 32 slots (the 64-token gate
 // recurrence runs as four independent 16-token pieces, tied together by four
 // sub-chunk products per slot exchanged through shared memory), converts state
-// columns sb*d/4..(sb+1)*d/4, masks score columns 16sb..16sb+15, stores y for
+// columns sb*d/4..(sb+1)*d/4, stores y for
 // tokens 16sb..16sb+15 and prepares |x|^2, mu, eta of four tokens of the next
 // chunk. Warp 16 issues every MMA, warp 17 every TMA copy (an MMA issue blocks
-// its warp while the MMA runs, so neither sits on a worker). The state chain
-// (G1 -> gates -> G7 -> state conversion -> next G1) is signalled separately
-// from the read-out path (G5, P mask, G6), which overlaps the next chunk.
+// its warp while the MMA runs, so neither sits on a worker), warps 18 and 19 form
+// the masked scores. The state chain (G1 -> gates -> G7 -> state conversion -> next
+// G1) is signalled separately from the read-out path (scores, G6), which overlaps
+// the next chunk.
 // Every mbarrier wait is bounded by %globaltimer: on timeout the kernel sets the
 // device status word, skips the remaining work and still meets every named barrier.
 #pragma once
@@ -89,12 +91,11 @@ struct TcLayout {
     static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;          // room to align the base
     // TMEM columns: fp32 state T | D1 (projections; its columns also hold the bf16
     // hi/lo pairs of the state-update operand KS, whose lifetime never overlaps
-    // D1's) | P | Y^T, double-buffered | S0 hi/lo bf16 pairs (two per column, d/2 each)
+    // D1's) | (unused) | Y^T, double-buffered | S0 hi/lo bf16 pairs (two per column, d/2 each)
     static constexpr uint32_t T_COL = 0;
     static constexpr uint32_t D1_COL = DS;
     static constexpr uint32_t KSHI_TCOL = D1_COL;
     static constexpr uint32_t KSLO_TCOL = D1_COL + kTcC / 2;
-    static constexpr uint32_t P_COL = DS + kTcC;
     static constexpr uint32_t Y_COL = DS + 2 * kTcC;               // + (chunk & 1) * C
     static constexpr uint32_t S0HI_TCOL = DS + 4 * kTcC;
     static constexpr uint32_t S0LO_TCOL = S0HI_TCOL + DS / 2;
@@ -145,13 +146,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nch = (T + kTcC - 1) / kTcC;
     constexpr int MMA_WARP = 16, TMA_WARP = 17;
 
-    // mbarriers: X stage landed [2], q/c landed, D1 ready, T updated (G7), S0 operand
-    // read (G4), scores ready (G5), read-out complete (G6)
+    // mbarriers: X stage landed [2], q/c landed, D1 ready, T updated (G7), (unused),
+    // read-out complete (G6), S0 operand read (G4)
     const uint32_t bar_full0 = sbase + Lay::BAR_OFF;
     const uint32_t bar_qc = sbase + Lay::BAR_OFF + 16;
     const uint32_t bar_d1 = sbase + Lay::BAR_OFF + 24;
     const uint32_t bar_t = sbase + Lay::BAR_OFF + 32;
-    const uint32_t bar_p5 = sbase + Lay::BAR_OFF + 40;
     const uint32_t bar_y = sbase + Lay::BAR_OFF + 48;
     const uint32_t bar_g4 = sbase + Lay::BAR_OFF + 56;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // named barriers (ids, participants): workers + MMA warp, or workers + TMA warp
     constexpr uint32_t BAR_INIT = 1, BAR_G = 2, BAR_A = 3, BAR_S0 = 4, BAR_P = 5;
     constexpr uint32_t N_WM = kTcWorkers + 32;
+    constexpr uint32_t N_WMS = kTcWorkers + 32 + 64;  // + the two score warps (BAR_A, BAR_P)
+    constexpr int SCORE_WARP0 = 18;                    // warps 18, 19: the causal scores
 
     if (warp == MMA_WARP) {
         if (lane == 0) {
@@ -192,7 +194,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // one elected lane issues; descriptors get per-MMA start-address offsets)
             constexpr uint32_t idesc_g1 = ptx::idesc_bf16(MS, kTcC, 0, 0);
             constexpr uint32_t idesc_g7 = ptx::idesc_bf16(MS, DS, 0, 1);
-            constexpr uint32_t idesc_g5 = ptx::idesc_bf16(kTcC, kTcSub, 1, 1);
             constexpr uint32_t idesc_g4 = ptx::idesc_bf16(DS, kTcC, 1, 1);
             constexpr uint32_t idesc_g6 = ptx::idesc_bf16(DS, kTcC, 1, 0);
             auto off = [](uint32_t bytes) { return uint64_t(bytes >> 4); };
@@ -218,13 +219,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             const uint64_t dM_x = ptx::sdesc_sw128(sbase + Lay::X_OFF, 64 * 128, 1024);
             const uint64_t dM_qr = ptx::sdesc_sw128(sbase + Lay::QR_OFF, MS * 128, 1024);
-            const uint64_t dM_kd = ptx::sdesc_sw128(sbase + Lay::KD_OFF, MS * 128, 1024);
             const uint64_t dM_s0hi = ptx::sdesc_sw128(sbase + Lay::S0HI_OFF, MS * 128, 1024);
             const uint64_t dK_p = ptx::sdesc_sw128(sbase + Lay::P_OFF, 16, 1024);
             for (int k = 0; k < nch; ++k) {
                 const uint32_t xo = (k & 1) * Lay::X_STAGE;
                 const uint32_t ycol = Lay::Y_COL + (k & 1) * kTcC;
-                ptx::named_bar(BAR_A, N_WM);  // KS in TMEM, QR/KD written, T prescaled
+                ptx::named_bar(BAR_A, N_WMS);  // KS in TMEM, QR/KD written, T prescaled
                 ptx::tc_fence_after();
                 if (tc_live(abort)) {
                     // G7: T += (KShi + KSlo)^T . X  (M = m, N = d, K = C); A in TMEM, B MN-major
@@ -245,24 +245,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                             idesc_g4, kk > 0);
                 }
                 ptx::mma_commit_elect(bar_g4);
-                if (tc_live(abort)) {
-                    // G5: P[:, 16b..16b+15] = QR_b . KD_b^T  (M = C, N = 16, K = m); both MN-major
-#pragma unroll
-                    for (int kk = 0; kk < MS / 16; ++kk)
-#pragma unroll
-                        for (int sb = 0; sb < NSUB; ++sb)
-                            ptx::mma_bf16_elect(tmem + Lay::P_COL + sb * kTcSub,
-                                                dM_qr + off(sb * Lay::ROW_TILE + kk * 2048),
-                                                dM_kd + off(sb * (kTcSub * 2) + kk * 2048), idesc_g5, kk > 0);
-                }
-                ptx::mma_commit_elect(bar_p5);
                 ptx::named_bar(BAR_S0, N_WM);  // S0 operand of chunk k+1 written
                 ptx::tc_fence_after();
                 if (k + 1 < nch) {
                     if (tc_wait_warp(bar_full0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1, abort)) g1(k + 1);
                     ptx::mma_commit_elect(bar_d1);
                 }
-                ptx::named_bar(BAR_P, N_WM);  // masked scores written
+                ptx::named_bar(BAR_P, N_WMS);  // masked scores written
                 ptx::tc_fence_after();
                 if (tc_live(abort)) {
                     // G6: Y^T += X^T . P^T  (M = d, N = C, K = C); A MN-major, B K-major
@@ -346,6 +335,66 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (last_qc >= 0) tc_drain(bar_qc, last_qc & 1);
             }
             __syncwarp();
+        } else if (warp == SCORE_WARP0 || warp == SCORE_WARP0 + 1) {
+            // -------------------------------------------------- score warps
+            // The causal scores P_tj = sum_i QR_b(t)_i KD(j)_i (K = m), one 16 x 16 block
+            // (tokens 16wt.., keys 16b.., b <= wt) at a time, with warp-synchronous MMAs
+            // (m16n8k16, bf16 operands by ldmatrix.trans from the slot-major QR and KD tiles,
+            // fp32 in registers), masked to j <= t in the diagonal block and written in bf16
+            // to the score tile for G6. Warp 18 takes token blocks 0 and 3, warp 19 blocks 1
+            // and 2 (five blocks each). On tcgen05 these 16-column blocks cost the tensor
+            // pipe about a hundred cycles per K = 16 step, 32 steps a chunk, queued ahead of
+            // the next chunk's projection.
+            const int lj = lane >> 3, lr = lane & 7, gq = lane >> 2, cq = lane & 3;
+            uint8_t* ps = smem + Lay::P_OFF;
+            const uint32_t kd_a = sbase + Lay::KD_OFF;
+            auto block = [&](int wt, int bk) {
+                const uint32_t qr_a = sbase + Lay::QR_OFF + bk * Lay::ROW_TILE;
+                float acc[2][4];
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < MS / 16; ++ks) {
+                    uint32_t af[4], bf[4];
+                    {   // A = QR^T block: stored rows are slots (K), columns tokens (M)
+                        const int row = 16 * ks + 8 * (lj >> 1) + lr;
+                        const int col = 16 * wt + 8 * (lj & 1);
+                        ptx::ldsm_x4_t(qr_a + row * 128 + (((col >> 3) ^ (row & 7)) << 4), af);
+                    }
+                    {   // B = KD^T block: stored rows are slots (K), columns keys (N)
+                        const int row = 16 * ks + 8 * (lj & 1) + lr;
+                        const int col = 16 * bk + 8 * (lj >> 1);
+                        ptx::ldsm_x4_t(kd_a + row * 128 + (((col >> 3) ^ (row & 7)) << 4), bf);
+                    }
+                    ptx::mma16816(acc[0], af, bf);      // keys 16bk .. 16bk+7
+                    ptx::mma16816(acc[1], af, bf + 2);  // keys 16bk+8 .. 16bk+15
+                }
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int t = 16 * wt + gq + 8 * hf, j = 16 * bk + 8 * n + 2 * cq;
+                        const float v0 = (j > t) ? 0.f : acc[n][2 * hf];
+                        const float v1 = (j + 1 > t) ? 0.f : acc[n][2 * hf + 1];
+                        *reinterpret_cast<uint32_t*>(ps + ptx::sw128_off(t, j)) = ptx::pack_bf16x2(v0, v1);
+                    }
+            };
+            const int wa = warp == SCORE_WARP0 ? 0 : 1, wb = warp == SCORE_WARP0 ? 3 : 2;
+            for (int k = 0; k < nch; ++k) {
+                ptx::named_bar(BAR_A, N_WMS);  // QR and KD of chunk k written
+                // G6 of the previous chunk has read the old scores
+                if (k > 0) tc_wait(bar_y, (k - 1) & 1, abort);
+                __syncwarp();
+                ptx::tc_fence_after();
+                if (!*abort) {
+                    for (int bk = 0; bk <= wa; ++bk) block(wa, bk);
+                    for (int bk = 0; bk <= wb; ++bk) block(wb, bk);
+                }
+                ptx::fence_proxy_async_smem();  // G6 reads the scores through the async proxy
+                ptx::named_bar(BAR_P, N_WMS);
+            }
         }
     } else {
         // ================================================================ workers
@@ -357,8 +406,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // y column in the Y^T accumulator (M = d) and P row (M = 64: lanes 0-15 per quadrant)
         const bool ycol_ok = (DS == 128) || (lane < 16);
         const int kcol = (DS == 128) ? (32 * q4 + lane) : (16 * q4 + lane);
-        const bool prow_ok = lane < 16;
-        const int tau_row = 16 * q4 + lane;
         uint8_t* s0hi = smem + Lay::S0HI_OFF;
         uint8_t* qr = smem + Lay::QR_OFF;
         uint8_t* kd = smem + Lay::KD_OFF;
@@ -462,6 +509,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ptx::tmem_wait_st();
             if (active) tsqp[sb * MS + i] = ns;
         }
+        for (int o = tid; o < int(kTcC * 128 / 16); o += kTcWorkers)  // score blocks above the diagonal
+            reinterpret_cast<uint4*>(ps)[o] = make_uint4(0u, 0u, 0u, 0u);
         if (nch > 0) {
             aux_part(0);
         }
@@ -621,7 +670,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             sigma = pre ? 1.f : sig_c;
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::named_bar(BAR_A, N_WM);
+            ptx::named_bar(BAR_A, N_WMS);
 
             // ---- phase B: y of the previous chunk (first half), while G7 and G4 run
             if (k > 0) {
@@ -679,30 +728,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (k > 0) store_y(k - 1, 1);  // second half of the previous chunk's y
 
             // ---- masked scores, next chunk's per-token inputs
-            tc_wait(bar_p5, k & 1, abort);  // G5 complete
-            __syncwarp();
-            ptx::tc_fence_after();
-            {   // causal mask of P: this group's 16 score columns of row tau_row
-                uint32_t r[kTcSub];
-                ptx::tmem_ld16(tmem + lane_base + Lay::P_COL + sb * kTcSub, r);
-                ptx::tmem_wait_ld();
-                if (prow_ok) {
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float v[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int j = sb * kTcSub + 8 * hh + e;
-                            v[e] = (j <= tau_row) ? __uint_as_float(r[8 * hh + e]) : 0.f;
-                        }
-                        *reinterpret_cast<uint4*>(ps + ptx::sw128_chunk(tau_row, 2 * sb + hh)) = pack8(v);
-                    }
-                }
-            }
+
             if (k + 1 < nch) aux_part(k + 1);
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::named_bar(BAR_P, N_WM);
+            ptx::named_bar(BAR_P, N_WMS);
         }
         if (nch > 0) {  // read-out of the last chunk
             tc_wait(bar_y, (nch - 1) & 1, abort);
