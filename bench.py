@@ -135,8 +135,8 @@ CAPTURED_TRAFFIC = {
                                                 source="csrc/chunk_split.cuh", sha="047d8e41962f"),
     ("chunk_split_kernel", "long_ctx"): dict(bytes=676.05e6 + 498.46e6, profile="profiles/chunk_split_kernel_full.md",
                                              source="csrc/chunk_split.cuh", sha="047d8e41962f"),
-    ("chunk_tc_kernel", "mid_layer"): dict(bytes=551.19e6 + 237.23e6, profile="profiles/chunk_tc_kernel_full.md",
-                                           source="csrc/chunk_tc.cuh", sha="aa446c46e88a"),
+    ("chunk_tc_kernel", "mid_layer"): dict(bytes=550.70e6 + 237.14e6, profile="profiles/chunk_tc_kernel_full.md",
+                                           source="csrc/chunk_tc.cuh", sha="488f569268b7"),
     ("scan_simt_kernel<exact>", "small_train"): dict(bytes=34.43e6 + 0.04e6,
                                                      profile="profiles/scan_simt_kernel_exact_small_train.md",
                                                      source="csrc/scan_simt.cuh", sha="327f91817ab8"),
