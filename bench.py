@@ -533,6 +533,14 @@ def bench_step(args, torch, L, dist, world, rank, local, device, pk, pk_src):
     return 0
 
 
+def bwd_kernel_name(chunk: int, d: int) -> str:
+    """The kernel lattice_scan_bwd runs (16-byte-aligned buffers): the chunk-parallel
+    kernel for chunks of 2..64 tokens at d >= 32, else the token-by-token kernel."""
+    if 2 <= chunk <= 64 and d in (32, 64, 128):
+        return "chunk_bwd_kernel"
+    return "scan_bwd_kernel<chunked>" if chunk > 1 else "scan_bwd_kernel<exact>"
+
+
 def bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush, pk, pk_src):
     """--pass bwd: one step is one lattice_scan_bwd of the workload (gradients of every
     input for unit dy), workspace allocated once outside the timed region."""
@@ -551,7 +559,7 @@ def bench_bwd(args, torch, L, dist, t, w, w0, world, rank, local, device, flush,
     alg_b = bwd_alg_bytes(w)
     kern_ms = statistics.mean(times)
     achieved = alg_b / (kern_ms * 1e-3) / 1e9
-    kname = "scan_bwd_kernel<chunked>" if w.chunk > 1 else "scan_bwd_kernel<exact>"
+    kname = bwd_kernel_name(w.chunk, w.d)
     line = {"metric": "Lattice layer bwd tokens/s (1 B200)", "value": job_tokens_per_s(world, w, ms),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -753,11 +761,11 @@ def main():
             tl = statistics.mean(time_scan(torch, L, ts, ws.chunk, 5, 3, flush=flush, lin=1))
             extra["small_train_lin1_chunked"] = {"ms": tl, "tokens_per_s": tok(tl),
                                                  "kernel": "scan_simt_kernel<chunked, recurrence_linear1>"}
-            # backward pass (CUDA-core kernel), chunked and exact
+            # backward pass, chunked (chunk-parallel kernel) and exact (token kernel)
             for cb, tag in ((ws.chunk, "chunked"), (1, "exact")):
                 tb = statistics.mean(time_bwd(torch, L, ts, cb, 3, 2, flush=flush))
                 extra[f"small_train_bwd_{tag}"] = {"ms": tb, "tokens_per_s": tok(tb),
-                                                   "kernel": f"scan_bwd_kernel<{tag}>",
+                                                   "kernel": bwd_kernel_name(cb, ws.d),
                                                    "allocations": "outputs per call; workspace once"}
             del ts
             torch.cuda.empty_cache()

@@ -75,4 +75,22 @@ LATTICE_HD inline size_t bwd_ws_floats_per_seq(int T, int m, int D, int seg) {
     return (size_t)(nseg - 1 + seg) * m * D;
 }
 
+// Chunk-parallel backward (chunk_bwd.cuh): 16 slots per CTA, 512 threads, chunks of
+// 2..64 tokens, a sequence's slots on a cluster of ceil(m/16) <= 8 CTAs.
+constexpr int kCbSlots = 16;
+constexpr int kCbThreads = 512;
+constexpr int kCbMaxL = 64;
+constexpr int kCbMaxG = 8;
+
+inline bool chunk_bwd_supported(int m, int d, int chunk) {
+    return chunk >= 2 && chunk <= kCbMaxL && (d == 32 || d == 64 || d == 128) && m >= 1 &&
+           m <= kCbMaxG * kCbSlots;
+}
+inline int chunk_bwd_ctas(int m) { return (m + kCbSlots - 1) / kCbSlots; }
+// Workspace floats of the chunk-parallel backward: each CTA's slots of every chunk-start state.
+inline size_t chunk_bwd_ws_floats(int B, int T, int H, int m, int D, int chunk) {
+    const size_t nc = T > 0 ? (size_t)((T + chunk - 1) / chunk) : 0;
+    return (size_t)B * H * chunk_bwd_ctas(m) * nc * kCbSlots * D;
+}
+
 }  // namespace lattice

@@ -266,7 +266,12 @@ size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int c
     const int seg = bwd_seg(chunk_size, seg_tokens);
     if (seg < 1) return 0;
     const int G = bwd_split(B, H, m), spc = (m + G - 1) / G;
-    return (size_t)B * H * G * bwd_ws_floats_per_seq(T, spc, d, seg) * sizeof(float);
+    const size_t tok = (size_t)B * H * G * bwd_ws_floats_per_seq(T, spc, d, seg) * sizeof(float);
+    if (!chunk_bwd_supported(m, d, chunk_size)) return tok;
+    // the chunk-parallel kernel serves the shape; the token kernel stays the fallback
+    // for buffers it cannot read with vector loads, so the workspace covers both
+    const size_t cb = chunk_bwd_ws_floats(B, T, H, m, d, chunk_size) * sizeof(float);
+    return cb > tok ? cb : tok;
 }
 
 lattice_status lattice_scan_bwd(const void* x, lattice_dtype x_dtype, const float* c,
@@ -309,6 +314,16 @@ lattice_status lattice_scan_bwd(const void* x, lattice_dtype x_dtype, const floa
             if (overlap(outs[i], s)) return LATTICE_ERR_INVALID_ARG;
         for (size_t k = i + 1; k < sizeof(outs) / sizeof(outs[0]); ++k)
             if (overlap(outs[i], outs[k])) return LATTICE_ERR_INVALID_ARG;
+    }
+    // Chunks of 2..64 tokens: the chunk-parallel kernel, when x, dy and dx take 16-byte
+    // vector accesses; otherwise (and for the exact recurrence) the token kernel.
+    if (chunk_bwd_supported(m, d, chunk_size) &&
+        (T == 0 || (aligned(x, 16) && aligned(dy, 16) && aligned(dx, 16)))) {
+        const int G = chunk_bwd_ctas(m);
+        BwdArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, dy, dS_T,
+                  dx, dc, dq, dmu, deta_w, dS0, static_cast<float*>(workspace), B, T, H, m, chunk_size,
+                  seg, G, kCbSlots};
+        return launch_chunk_bwd(a, d, static_cast<cudaStream_t>(stream));
     }
     const int G = bwd_split(B, H, m);
     BwdArgs a{x, x_dtype == LATTICE_BF16, c, q, q_dtype == LATTICE_BF16, mu, eta, S0, dy, dS_T,

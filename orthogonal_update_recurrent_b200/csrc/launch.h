@@ -30,6 +30,7 @@ lattice_status launch_readout(const ReadoutArgs& a, int d, cudaStream_t st);
 
 // tu_bwd.cu: backward pass (a.G, a.spc set by the caller)
 lattice_status launch_bwd(const BwdArgs& a, int d, cudaStream_t st);
+lattice_status launch_chunk_bwd(const BwdArgs& a, int d, cudaStream_t st);
 
 // tu_tc.cu: tensor-core chunked scans
 bool tc_supported(lattice_impl impl, int m, int d, int chunk, bool x_bf16, bool q_bf16);

@@ -68,6 +68,19 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t caddr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(caddr)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t caddr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
+    return v;
+}
 __device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float4 v) {
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(v.x), "f"(v.y),
                  "f"(v.z), "f"(v.w)
@@ -416,6 +429,22 @@ __device__ __forceinline__ void mma1688(float* d, const uint32_t* a, uint32_t b)
         "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(b));
+}
+// m16n8k8 with tf32 operands and fp32 accumulation. Lane l, g = l/4, c = l%4:
+// A 16x8 row-major: a[0] (g, c), a[1] (g+8, c), a[2] (g, c+4), a[3] (g+8, c+4);
+// B 8x8 col: b[0] (k = c, n = g), b[1] (k = c+4, n = g); D as for m16n8k16.
+__device__ __forceinline__ void mma_tf32(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// fp32 -> tf32 (round to nearest, ties away), as a 32-bit pattern with the low 13 bits zero.
+__device__ __forceinline__ uint32_t cvt_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
 // Two 8x8 b16 matrices (lanes 0-7 and 8-15 give the row addresses).
 __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t* r) {

@@ -1,4 +1,5 @@
-// tu_bwd.cu -- launches of the backward-pass kernels (scan_bwd.cuh).
+// tu_bwd.cu -- launches of the backward-pass kernels (scan_bwd.cuh, chunk_bwd.cuh).
+#include "chunk_bwd.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "scan_bwd.cuh"
@@ -53,7 +54,40 @@ lattice_status launch_bwd_c(const BwdArgs& a, int d, cudaStream_t st) {
     return LATTICE_ERR_UNSUPPORTED;
 }
 
+template <int D>
+lattice_status launch_chunk_bwd_t(const BwdArgs& a, cudaStream_t st) {
+    const size_t smem = CbLayout<D>::BYTES;
+    auto k = chunk_bwd_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.B * a.H * a.G));
+    cfg.blockDim = dim3((unsigned)kCbThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)a.G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.G > 1 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, k, a);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return launch_status();
+}
+
 }  // namespace
+
+// The chunk-parallel backward (chunk_bwd.cuh); a.G must be chunk_bwd_ctas(m).
+lattice_status launch_chunk_bwd(const BwdArgs& a, int d, cudaStream_t st) {
+    switch (d) {
+        case 32: return launch_chunk_bwd_t<32>(a, st);
+        case 64: return launch_chunk_bwd_t<64>(a, st);
+        case 128: return launch_chunk_bwd_t<128>(a, st);
+    }
+    return LATTICE_ERR_UNSUPPORTED;
+}
 
 lattice_status launch_bwd(const BwdArgs& a, int d, cudaStream_t st) {
     return a.chunk == 1 ? launch_bwd_c<false>(a, d, st) : launch_bwd_c<true>(a, d, st);

@@ -147,6 +147,71 @@ def test_bwd_empty_sequence_passes_the_state_gradient_through(L):
         assert np.array_equal(g["dS0"], cot["dS_T"])
 
 
+@pytest.mark.parametrize("m,d,C,T", [(5, 32, 8, 70), (40, 64, 12, 100), (128, 64, 2, 37),
+                                     (16, 128, 64, 50), (100, 128, 24, 130)])
+def test_bwd_chunk_parallel_edges(L, m, d, C, T):
+    """The chunk-parallel kernel (chunks of 2..64, d >= 32): slot counts that leave the
+    last CTA of a sequence partly empty (m = 5, 40, 100), chunk sizes that are not a
+    multiple of 8 (12, 24, 2), a single ragged chunk shorter than C (T = 50 < 64),
+    clusters of 1 to 8 CTAs, eta given."""
+    w = LI.Workload("t", B=2, T=T, H=2, m=m, d=d, seed=900 + m + d + C)
+    inp = with_eta(LI.make_inputs(w), 900 + C)
+    cot = LI.make_cotangents(inp, seed=900 + T)
+    check(run_gpu_bwd(L, inp, cot, C), run_oracle_bwd(inp, cot, C), TOL_BWD)
+
+
+def test_bwd_chunk_parallel_empty_sequence(L):
+    w = LI.Workload("t", B=2, T=0, H=3, m=40, d=64, seed=910)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=910)
+    g = run_gpu_bwd(L, inp, cot, 16)
+    assert np.array_equal(g["dS0"], cot["dS_T"])
+
+
+def test_bwd_unaligned_x_falls_back_to_the_token_kernel(L):
+    """x that does not start on a 16-byte boundary cannot take the chunk-parallel
+    kernel's vector loads; the call runs the token-by-token kernel instead, on the same
+    definition, and agrees with the oracle (and, within rounding, with the aligned call)."""
+    w = LI.Workload("t", B=1, T=90, H=2, m=32, d=64, seed=920)
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=920)
+    t = dev_inputs(inp)
+    flat = torch.empty(t["x"].numel() + 1, dtype=t["x"].dtype, device="cuda")
+    xs = flat[1:].view(t["x"].shape)
+    xs.copy_(t["x"])
+    assert xs.data_ptr() % 16 != 0
+    dy = torch.from_numpy(cot["dy"]).cuda()
+    dST = torch.from_numpy(cot["dS_T"]).cuda()
+    gu = L.scan_bwd(xs, t["c"], t["q"], t["mu"], t["S0"], dy, dST, chunk=16)
+    ga = L.scan_bwd(t["x"], t["c"], t["q"], t["mu"], t["S0"], dy, dST, chunk=16)
+    torch.cuda.synchronize()
+    L.device_status()
+    go = run_oracle_bwd(inp, cot, 16)
+    for g in (gu, ga):
+        check({k: (None if v is None else v.cpu().numpy()) for k, v in g.items()}, go, TOL_BWD)
+
+
+def test_bwd_mid_layer_full_size_sampled(L):
+    """The mid-size layer at full size (B=8, H=16, T=4096, m=d=128, 10% duplicate
+    tokens): clusters of 8 CTAs, 64 chunks; two sampled sequences against the oracle."""
+    w = LI.WORKLOADS["mid_layer"]
+    inp = LI.make_inputs(w)
+    cot = LI.make_cotangents(inp, seed=930)
+    gg = run_gpu_bwd(L, inp, cot, w.chunk)
+    pairs = [(0, 0), (7, 15)]
+    sub = LI.sample_heads(inp, pairs)
+    bs, hs = [p[0] for p in pairs], [p[1] for p in pairs]
+    sub_cot = dict(dy=np.ascontiguousarray(cot["dy"][bs, :, hs][:, :, None, :]),
+                   dS_T=np.ascontiguousarray(cot["dS_T"][bs, hs][:, None]))
+    go = run_oracle_bwd(sub, sub_cot, w.chunk)
+    gsub = {"dx": gg["dx"][bs, :, hs][:, :, None, :], "dc": gg["dc"][bs, :, hs][:, :, None, :],
+            "dq": gg["dq"][bs, :, hs][:, :, None, :], "dmu": gg["dmu"][bs, :, hs][:, :, None],
+            "deta": None, "dS0": gg["dS0"][bs, hs][:, None]}
+    check(gsub, go, 2e-2)
+    for k in ("dx", "dc", "dq", "dmu", "dS0"):
+        assert np.isfinite(gg[k]).all()
+
+
 def test_bwd_rejects_unsupported_shapes(L):
     w = LI.Workload("t", B=1, T=8, H=1, m=130, d=32, seed=880)
     inp = LI.make_inputs(w)
