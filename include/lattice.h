@@ -193,8 +193,15 @@ lattice_status lattice_scan_fwd_ex(const void *x, lattice_dtype x_dtype, const f
  * lattice_scan_bwd_workspace_bytes(...) bytes, 16-byte aligned; the call
  * overwrites it and keeps no pointer after it returns (the kernel runs on
  * `stream`). Outputs must not overlap inputs, each other or the workspace
- * (LATTICE_ERR_INVALID_ARG). CUDA-core kernel only; m <= 128 (larger m:
- * LATTICE_ERR_UNSUPPORTED). */
+ * (LATTICE_ERR_INVALID_ARG). m <= 128 (larger m: LATTICE_ERR_UNSUPPORTED).
+ * Kernels: chunk sizes 2..64 with d in {32, 64, 128}, and x, dy, dx on 16-byte
+ * boundaries, run a chunk-parallel kernel: a forward sweep stores every chunk-start
+ * state in the workspace, then each chunk, last to first, is differentiated as a whole
+ * (matrix products on the tensor cores in tf32 with a hi/lo split of each operand,
+ * about fp32 accuracy), and only the state adjoint passes from chunk to chunk;
+ * seg_tokens is checked but not used. Other shapes (the exact recurrence included)
+ * run token by token on CUDA cores with the segment checkpoints described above.
+ * Both are deterministic: sums across CTAs are taken in a fixed order. */
 lattice_status lattice_scan_bwd(const void *x, lattice_dtype x_dtype, const float *c,
                                 const void *q, lattice_dtype q_dtype, const float *mu,
                                 const float *eta, const float *S0, const float *dy,
@@ -203,12 +210,14 @@ lattice_status lattice_scan_bwd(const void *x, lattice_dtype x_dtype, const floa
                                 int B, int T, int H, int m, int d, int chunk_size, int seg_tokens,
                                 void *stream);
 
-/* Workspace bytes lattice_scan_bwd needs for this shape on the current device:
- * B*H*G*(n_seg - 1 + seg_tokens)*ceil(m/G)*d*4 with n_seg = ceil(T/seg_tokens)
- * (seg_tokens as resolved by lattice_scan_bwd) and G the CTAs per sequence the call
- * uses (G = 1 when the batch fills the device's SMs; up to 4 otherwise, so about
- * B*H*(n_seg - 1 + seg_tokens)*m*d*4). Returns 0 for arguments lattice_scan_bwd
- * would reject. Host function; launches nothing. */
+/* Workspace bytes lattice_scan_bwd needs for this shape on the current device: the
+ * token kernel's B*H*G*(n_seg - 1 + seg_tokens)*ceil(m/G)*d*4 with
+ * n_seg = ceil(T/seg_tokens) (seg_tokens as resolved by lattice_scan_bwd) and G the
+ * CTAs per sequence it uses (G = 1 when the batch fills the device's SMs; up to 4
+ * otherwise), and, where the chunk-parallel kernel serves the shape, the larger of
+ * that and its B*H*ceil(m/16)*ceil(T/chunk)*16*d*4 (every chunk-start state), so that
+ * either kernel can run. Returns 0 for arguments lattice_scan_bwd would reject. Host
+ * function; launches nothing. */
 size_t lattice_scan_bwd_workspace_bytes(int B, int T, int H, int m, int d, int chunk_size,
                                         int seg_tokens);
 

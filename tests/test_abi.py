@@ -116,6 +116,13 @@ def test_backward_workspace_and_argument_checks(lib):
     assert ws(1, 200, 1, 5, 16, 1, 0) == 2 * (3 + 64) * 3 * 16 * 4       # G = 2, 3 rows each (one unused)
     assert ws(100, 200, 1, 64, 16, 1, 0) == 100 * (3 + 64) * 64 * 16 * 4  # batch fills the SMs: G = 1
     assert ws(1, 200, 1, 129, 16, 1, 0) == 0     # m > 128
+    # chunks of 2..64 at d >= 32 may run the chunk-parallel kernel: the workspace covers
+    # both kernels, its own term being ceil(m/16) CTAs x ceil(T/C) chunk-start states
+    tok = 4 * (3 + 64) * 10 * 64 * 4                        # G = 4, 10 rows each, seg 64
+    assert ws(1, 200, 1, 40, 64, 16, 0) == max(tok, 3 * 13 * 16 * 64 * 4) == tok
+    tok = 4 * (102 + 640) * 16 * 128 * 4                    # seg 640: 103 segments
+    cb = 4 * 1024 * 16 * 128 * 4                            # 1024 chunks of 64
+    assert ws(1, 65536, 1, 64, 128, 64, 640) == max(tok, cb) == cb
     # every case below fails validation before any CUDA call
     assert _bwd(lib, wsb=64 * 4 * 16 * 4 - 4) == L.ERR_INVALID_ARG   # workspace too small
     assert _bwd(lib, ws=None) == L.ERR_INVALID_ARG
