@@ -67,7 +67,10 @@ struct CbLayout {
     static constexpr int MU = DKT + TSA, ETA = MU + kCbMaxL, HH = ETA + kCbMaxL,
                          HHB = HH + kCbMaxL, MUB = HHB + kCbMaxL, ETAB = MUB + kCbMaxL;
     static constexpr int N2 = ETAB + kCbMaxL, E0 = N2 + kCbSlots, AL = E0 + kCbSlots;
-    static constexpr int FLOATS = AL + kCbSlots;
+    // 16-token blocks: q times the in-block prefix of g, kappa times the in-block suffix,
+    // and the products of the whole blocks between two blocks (pairs b1 < b2)
+    static constexpr int QA = AL + kCbSlots, KU = QA + TSA, W = KU + TSA;
+    static constexpr int FLOATS = W + 6 * kCbSlots;
     static constexpr size_t BYTES = (size_t)FLOATS * 4;
     static_assert(BYTES <= 232448, "shared memory per CTA");
     static_assert(X % 4 == 0 && DY % 4 == 0 && DX % 4 == 0 && SA % 4 == 0 && SB % 4 == 0 &&
@@ -212,6 +215,45 @@ __device__ __forceinline__ void cb_mma(float (&acc)[NT][4], const float* A, int 
         }
     }
 }
+// cb_mma with a per-slot scale: SIDE 1 scales A's element (r, k) by scale[k], SIDE 2
+// scales B's element (k, n) by scale[8nt + n].
+template <int NT, int SIDE>
+__device__ __forceinline__ void cb_mma_s(float (&acc)[NT][4], const float* A, int am, int ak,
+                                         const float* B, int bk, int bn, int k0, int k1, int lane,
+                                         const float* scale) {
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll 2
+    for (int k = k0; k < k1; k += 8) {
+        float av[4] = {A[g * am + (k + c) * ak], A[(g + 8) * am + (k + c) * ak],
+                       A[g * am + (k + c + 4) * ak], A[(g + 8) * am + (k + c + 4) * ak]};
+        if (SIDE == 1) {
+            const float s0 = scale[k + c], s1 = scale[k + c + 4];
+            av[0] *= s0; av[1] *= s0; av[2] *= s1; av[3] *= s1;
+        }
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            ah[r] = ptx::cvt_tf32(av[r]);
+            al[r] = ptx::cvt_tf32(av[r] - __uint_as_float(ah[r]));
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float b0 = B[(k + c) * bk + (8 * nt + g) * bn];
+            float b1 = B[(k + c + 4) * bk + (8 * nt + g) * bn];
+            if (SIDE == 2) {
+                const float sn = scale[8 * nt + g];
+                b0 *= sn; b1 *= sn;
+            }
+            const uint32_t bh[2] = {ptx::cvt_tf32(b0), ptx::cvt_tf32(b1)};
+            const uint32_t bl[2] = {ptx::cvt_tf32(b0 - __uint_as_float(bh[0])),
+                                    ptx::cvt_tf32(b1 - __uint_as_float(bh[1]))};
+            ptx::mma_tf32(acc[nt], al, bh);
+            ptx::mma_tf32(acc[nt], ah, bl);
+            ptx::mma_tf32(acc[nt], ah, bh);
+        }
+    }
+}
+
 template <int NT>
 __device__ __forceinline__ void cb_zero(float (&acc)[NT][4]) {
 #pragma unroll
@@ -253,6 +295,9 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
     float* sN2 = sm + Lo::N2;
     float* sE0 = sm + Lo::E0;
     float* sAL = sm + Lo::AL;
+    float* sQA = sm + Lo::QA;
+    float* sKU = sm + Lo::KU;
+    float* sW = sm + Lo::W;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = a.G, crank = G > 1 ? (int)ptx::cluster_ctarank() : 0;
@@ -407,6 +452,32 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
             sU[t1 * TS + wi] = U1;
             const float q0 = sQ[t0 * TS + wi], q1 = sQ[t1 * TS + wi];
             *reinterpret_cast<float2*>(sAQT + wi * PS + t0) = make_float2(A0 * q0, A1 * q1);
+            // the same products inside 16-token blocks (8 lanes each), and the block totals
+            float pb = a1, sb = a1;
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                const float up = __shfl_up_sync(0xffffffffu, pb, o);
+                const float dn = __shfl_down_sync(0xffffffffu, sb, o);
+                if ((lane & 7) >= o) pb *= up;
+                if ((lane & 7) + o < 8) sb *= dn;
+            }
+            float exb = __shfl_up_sync(0xffffffffu, pb, 1);
+            float rtb = __shfl_down_sync(0xffffffffu, sb, 1);
+            if ((lane & 7) == 0) exb = 1.f;
+            if ((lane & 7) == 7) rtb = 1.f;
+            sQA[t0 * TS + wi] = q0 * exb * g0;
+            sQA[t1 * TS + wi] = q1 * pb;
+            sKU[t0 * TS + wi] = k0 * g1 * rtb;
+            sKU[t1 * TS + wi] = k1 * rtb;
+            const float G1 = __shfl_sync(0xffffffffu, pb, 15), G2 = __shfl_sync(0xffffffffu, pb, 23);
+            if (lane == 0) {   // pairs (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+                sW[0 * kCbSlots + wi] = 1.f;
+                sW[1 * kCbSlots + wi] = G1;
+                sW[2 * kCbSlots + wi] = G1 * G2;
+                sW[3 * kCbSlots + wi] = 1.f;
+                sW[4 * kCbSlots + wi] = G2;
+                sW[5 * kCbSlots + wi] = 1.f;
+            }
         }
     };
 
@@ -505,63 +576,114 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
         slot_scans(true);
         __syncthreads();
 
-        // dq_t,i = A_t,i dy_t.s0_i + sum_{j<=t} D_i[t][j] kappa_j,i dy_t.h_j (pairs, on
-        // tokens pt0 and 63 - pt0, so that every thread walks 65 steps)
-#pragma unroll 1
+        // The decayed sums over token pairs, split by 16-token blocks. For k in block bk
+        // and t in an earlier block bt, D_i[k][t] = KU-suffix(t) * W_i(bt, bk) * QA-prefix(k)
+        // (the in-block suffix after t, the whole blocks between, the in-block prefix up to
+        // k), so each pair of blocks is a 16x16 matrix product with a per-slot scale:
+        //   P[k][t]   += sum_i QA_k,i W_i KU_t,i                  (bt < bk)
+        //   dq_t,i    += Ahat_t,i sum_{bj<bt} W_i (M2[t][bj] . KU_bj)_i
+        //   dkappa_t,i += Uhat_t,i sum_{bk>bt} W_i (M2[bk][t]^T . QA_bk)_i
+        // (Ahat, Uhat: the in-block prefix and suffix; the in-block loops that follow form
+        // them as they walk the block, and apply them to the block sums stored here).
+        {
+            const int g = lane >> 2, c = lane & 3;
+            auto pidx = [](int b1, int b2) { return b1 == 0 ? b2 - 1 : (b1 == 1 ? b2 + 1 : 5); };
+            for (int task = warp; task < 14; task += kCbThreads / 32) {
+                float acc[2][4];
+                cb_zero(acc);
+                if (task < 6) {   // scores of block pair (bt, bk), bt < bk
+                    const int bt = task < 3 ? 0 : (task < 5 ? 1 : 2);
+                    const int bk = task < 3 ? task + 1 : (task < 5 ? task - 1 : 3);
+                    cb_mma_s<2, 1>(acc, sQA + 16 * bk * TS, TS, 1, sKU + 16 * bt * TS, 1, TS, 0, kCbSlots, lane,
+                                   sW + pidx(bt, bk) * kCbSlots);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        float* o = sP + (16 * bk + g) * PS + 16 * bt + 8 * nt + 2 * c;
+                        o[0] = acc[nt][0];
+                        o[1] = acc[nt][1];
+                        o[8 * PS] = acc[nt][2];
+                        o[8 * PS + 1] = acc[nt][3];
+                    }
+                } else if (task < 10) {   // dq of block bt from the earlier blocks
+                    const int bt = task - 6;
+                    for (int bj = 0; bj < bt; ++bj)
+                        cb_mma_s<2, 2>(acc, sM2 + 16 * bt * PS + 16 * bj, PS, 1, sKU + 16 * bj * TS, TS, 1, 0, 16,
+                                       lane, sW + pidx(bj, bt) * kCbSlots);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int t = 16 * bt + g + 8 * (r >> 1), i = 8 * nt + 2 * c + (r & 1);
+                            sDQ[t * TS + i] = bt > 0 ? acc[nt][r] : 0.f;
+                        }
+                } else {   // dkappa of block bt from the later blocks
+                    const int bt = task - 10;
+                    for (int bk = bt + 1; bk < 4; ++bk)
+                        cb_mma_s<2, 2>(acc, sM2 + 16 * bk * PS + 16 * bt, 1, PS, sQA + 16 * bk * TS, TS, 1, 0, 16,
+                                       lane, sW + pidx(bt, bk) * kCbSlots);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int t = 16 * bt + g + 8 * (r >> 1), i = 8 * nt + 2 * c + (r & 1);
+                            sDKT[t * TS + i] = bt < 3 ? acc[nt][r] : 0.f;
+                        }
+                }
+            }
+        }
+        __syncthreads();
+
+        // in-block parts: dq over j <= t in t's block (pairs), the scores and dkappa over
+        // k >= t in t's block (half-warps: lanes = slots; tokens hw and 63 - hw)
+#pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-            const int t = h2 == 0 ? pt0 : kCbMaxL - 1 - pt0;
+            const int t = pt0 + 32 * h2;
             float dq = 0.f;
             if (t < L) {
                 dq = sA[t * TS + pi] * sM1[t * TS + pi];
                 float Dp = 1.f;
-                for (int j = t; j >= 0; --j) {
+                for (int j = t; j >= (t & ~15); --j) {
                     dq += Dp * sKT[j * TS + pi] * sM2[t * PS + j];
                     Dp *= sG[j * TS + pi];
                 }
+                dq += Dp * sDQ[t * TS + pi];   // Dp is now Ahat_t
             }
             sDQ[t * TS + pi] = dq;
         }
-        // causal scores P[k][t] and dkappa_t,i (half-warps: lanes = slots; tokens hw and
-        // 63 - hw), walking k >= t with D = D_i[k][t] and w = q_k,i D:
-        //   P[k][t] = sum over the lanes of kappa_t,i w,   dkappa_t,i += w dy_k.h_t,
-        // on top of U_t,i h_t.dS_i. Score rows below the 16-token block of the warp's lower
-        // token are never read, and are skipped.
         {
             const int hw = tid >> 4;
 #pragma unroll 1
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int t = h2 == 0 ? hw : kCbMaxL - 1 - hw;
-                const int tmin = h2 == 0 ? (hw & ~1) : kCbMaxL - 2 - (hw & ~1);  // warp-uniform
+                const int bb = (h2 == 0 ? (hw & ~1) : kCbMaxL - 2 - (hw & ~1)) & ~15;  // warp-uniform block
                 const float ktv = sKT[t * TS + pi];
                 float Dp = 1.f, dk = 0.f;
-#pragma unroll 1
-                for (int bb = tmin & ~15; bb < kCbMaxL; bb += 16) {
-                    float v[16];
+                float v[16];
 #pragma unroll
-                    for (int n = 0; n < 16; ++n) {
-                        const int kk = bb + n;
-                        v[n] = 0.f;
-                        if (kk >= t) {
-                            const float w = sQ[kk * TS + pi] * Dp;
-                            v[n] = ktv * w;
-                            dk += w * sM2[kk * PS + t];
-                            if (kk + 1 < kCbMaxL) Dp *= sG[(kk + 1) * TS + pi];
-                        }
+                for (int n = 0; n < 16; ++n) {
+                    const int kk = bb + n;
+                    v[n] = 0.f;
+                    if (kk >= t) {
+                        const float w = sQ[kk * TS + pi] * Dp;
+                        v[n] = ktv * w;
+                        dk += w * sM2[kk * PS + t];
+                        if (n < 15) Dp *= sG[(kk + 1) * TS + pi];   // stays inside the block
                     }
-                    // reduce the 16 values over the half-warp's 16 lanes: lane n keeps entry n
-#pragma unroll
-                    for (int s = 8; s >= 1; s >>= 1) {
-                        const bool up = (pi & s) != 0;
-#pragma unroll
-                        for (int n = 0; n < s; ++n) {
-                            const float send = up ? v[n] : v[n + s];
-                            const float keep = up ? v[n + s] : v[n];
-                            v[n] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-                        }
-                    }
-                    sP[(bb + pi) * PS + t] = v[0];
                 }
-                sDKT[t * TS + pi] = t < L ? sU[t * TS + pi] * sM3[t * TS + pi] + dk : 0.f;
+                // reduce the 16 values over the half-warp's 16 lanes: lane n keeps entry n
+#pragma unroll
+                for (int s = 8; s >= 1; s >>= 1) {
+                    const bool up = (pi & s) != 0;
+#pragma unroll
+                    for (int n = 0; n < s; ++n) {
+                        const float send = up ? v[n] : v[n + s];
+                        const float keep = up ? v[n + s] : v[n];
+                        v[n] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+                    }
+                }
+                sP[(bb + pi) * PS + t] = v[0];
+                // Dp is now Uhat_t, the product of g over the block after t
+                sDKT[t * TS + pi] = t < L ? Dp * sDKT[t * TS + pi] + sU[t * TS + pi] * sM3[t * TS + pi] + dk : 0.f;
             }
         }
         __syncthreads();
