@@ -322,47 +322,80 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
     const bool wvalid = wi < nvalid;
     const int wc = lane * CPT;
 
-    // ---- stage one chunk's token inputs (x, and with dy: dy, q); |x_t|^2 per token
-    auto stage = [&](int t0, int L, bool bwd) {
-        for (int e = tid; e < kCbMaxL * DV; e += kCbThreads) {
-            const int t = e / DV, c4 = e % DV;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f), dy = v;
+    // ---- stage one chunk's token inputs (x, and with dy: dy, q); |x_t|^2 per token. The
+    // loads go to registers first (stage_load, issued a phase ahead where possible) and
+    // are converted and stored to shared memory by stage_store.
+    constexpr int NI = kCbMaxL * DV / kCbThreads;   // row pieces per thread (D >= 32: >= 1)
+    struct Pre {
+        float4 x[NI], dy[NI];   // x raw: fp32, or bf16 pairs in the .x/.y bit patterns
+        uint32_t c[2], q[2];    // q raw (fp32 bits, or the bf16 bits)
+        float mu, eta;
+    };
+    auto stage_load = [&](Pre& pr, int t0, int L, bool bwd) {
+#pragma unroll
+        for (int it = 0; it < NI; ++it) {
+            const int e = tid + it * kCbThreads, t = e / DV, c4 = e % DV;
+            pr.x[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+            pr.dy[it] = pr.x[it];
             if (t < L) {
                 const size_t ro = tok(t0 + t) * D + 4 * c4;
                 if (a.x_bf16) {
                     const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.x) + ro);
-                    v.x = __uint_as_float(u.x << 16);
-                    v.y = __uint_as_float(u.x & 0xffff0000u);
-                    v.z = __uint_as_float(u.y << 16);
-                    v.w = __uint_as_float(u.y & 0xffff0000u);
+                    pr.x[it].x = __uint_as_float(u.x);
+                    pr.x[it].y = __uint_as_float(u.y);
                 } else {
-                    v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + ro);
+                    pr.x[it] = *reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + ro);
                 }
-                if (bwd) dy = *reinterpret_cast<const float4*>(a.dy + ro);
+                if (bwd) pr.dy[it] = *reinterpret_cast<const float4*>(a.dy + ro);
+            }
+        }
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const int e = tid + it * kCbThreads, t = e >> 4, i = e & 15;
+            pr.c[it] = 0u;
+            pr.q[it] = 0u;
+            if (t < L && i < nvalid) {
+                const size_t ro = tok(t0 + t) * m + slot0 + i;
+                pr.c[it] = __float_as_uint(a.c[ro]);
+                if (bwd)
+                    pr.q[it] = a.q_bf16 ? (uint32_t)(static_cast<const unsigned short*>(a.q)[ro])
+                                        : __float_as_uint(static_cast<const float*>(a.q)[ro]);
+            }
+        }
+        pr.mu = 0.f;
+        pr.eta = 1.f;
+        if (tid < L) {
+            pr.mu = a.mu[tok(t0 + tid)];
+            if (has_eta) pr.eta = a.eta[tok(t0 + tid)];
+        }
+    };
+    auto stage_store = [&](const Pre& pr, bool bwd) {
+#pragma unroll
+        for (int it = 0; it < NI; ++it) {
+            const int e = tid + it * kCbThreads, t = e / DV, c4 = e % DV;
+            float4 v = pr.x[it];
+            if (a.x_bf16) {
+                const uint32_t u0 = __float_as_uint(v.x), u1 = __float_as_uint(v.y);
+                v = make_float4(__uint_as_float(u0 << 16), __uint_as_float(u0 & 0xffff0000u),
+                                __uint_as_float(u1 << 16), __uint_as_float(u1 & 0xffff0000u));
             }
             *reinterpret_cast<float4*>(sX + t * XS + 4 * c4) = v;
-            if (bwd) *reinterpret_cast<float4*>(sDY + t * XS + 4 * c4) = dy;
+            if (bwd) *reinterpret_cast<float4*>(sDY + t * XS + 4 * c4) = pr.dy[it];
             // |x_t|^2: the DV threads of a row are consecutive lanes (DV divides 32 or is 32)
             float s = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
 #pragma unroll
             for (int o = DV / 2; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
             if (c4 == 0) sHH[t] = s;
         }
-        for (int e = tid; e < kCbMaxL * kCbSlots; e += kCbThreads) {
-            const int t = e >> 4, i = e & 15;
-            float cv = 0.f, qv = 0.f;
-            if (t < L && i < nvalid) {
-                const size_t ro = tok(t0 + t) * m + slot0 + i;
-                cv = a.c[ro];
-                if (bwd) qv = load_elem(a.q, a.q_bf16, ro);
-            }
-            sC[t * TS + i] = cv;
-            sQ[t * TS + i] = qv;
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const int e = tid + it * kCbThreads, t = e >> 4, i = e & 15;
+            sC[t * TS + i] = __uint_as_float(pr.c[it]);
+            sQ[t * TS + i] = a.q_bf16 ? __uint_as_float(pr.q[it] << 16) : __uint_as_float(pr.q[it]);
         }
         if (tid < kCbMaxL) {
-            const bool in = tid < L;
-            sMU[tid] = in ? a.mu[tok(t0 + tid)] : 0.f;
-            sETA[tid] = in && has_eta ? a.eta[tok(t0 + tid)] : 1.f;
+            sMU[tid] = pr.mu;
+            sETA[tid] = pr.eta;
         }
     };
 
@@ -504,6 +537,8 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
     // ================= forward sweep: the start state of every chunk into the workspace
     const int g4 = lane >> 2, c4 = lane & 3;   // MMA fragment coordinates
     load_state(Scur, a.S0 + sbase + (size_t)slot0 * D, D, wvalid);
+    Pre pre;
+    if (nc > 0) stage_load(pre, 0, min(C, T), false);
     for (int k = 0; k < nc; ++k) {
         const int t0 = k * C, L = min(C, T - t0), kend = (L + 7) & ~7;
         {   // checkpoint, and |s_i|^2 of this chunk's start state
@@ -516,7 +551,7 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
             s = cb_warp_sum(s);
             if (lane == 0) sN2[wi] = s;
         }
-        stage(t0, L, false);
+        stage_store(pre, false);
         __syncthreads();
         projections(Scur, false);
         __syncthreads();
@@ -524,6 +559,7 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
         __syncthreads();
         slot_scans(false);
         __syncthreads();
+        if (k + 1 < nc) stage_load(pre, t0 + C, min(C, T - t0 - C), false);   // next chunk's inputs
         // S_next,i = A_L,i S_i - sum_t kappa_t,i U_t,i x_t   (h = -x): [16 slots] x [8 columns] per warp
         for (int task = warp; task < D / 8; task += kCbThreads / 32) {
             float acc[1][4];
@@ -562,10 +598,22 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
     }
     float* SL = Scur;   // end state of the chunk being differentiated
     float* S0 = Soth;   // its start state (from the workspace)
+    float pck[CPT];     // the start state's row piece of this lane, loaded a phase ahead
+    if (nc > 0) {
+        stage_load(pre, (nc - 1) * C, T - (nc - 1) * C, true);
+        cb_ld<CPT>(ws + ((size_t)(nc - 1) * kCbSlots + wi) * D + wc, pck);
+    }
     for (int k = nc - 1; k >= 0; --k) {
         const int t0 = k * C, L = min(C, T - t0), kend = (L + 7) & ~7;
-        load_state(S0, ws + (size_t)k * kCbSlots * D, D, true);
-        stage(t0, L, true);
+        {   // start state (and |s_i|^2) and token inputs into shared memory
+            cb_st<CPT>(S0 + wi * XS + wc, pck);
+            float s = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) s += pck[c] * pck[c];
+            s = cb_warp_sum(s);
+            if (lane == 0) sN2[wi] = s;
+        }
+        stage_store(pre, true);
         __syncthreads();
         projections(S0, true);
         __syncthreads();
@@ -770,6 +818,10 @@ __global__ void __launch_bounds__(kCbThreads, 1) chunk_bwd_kernel(const BwdArgs 
             }
         }
         cta_sync();   // every CTA's dx share, dmu and deta sums are in place
+        if (k > 0) {   // the previous chunk's inputs and start state, while this one finishes
+            stage_load(pre, t0 - C, C, true);
+            cb_ld<CPT>(ws + ((size_t)(k - 1) * kCbSlots + wi) * D + wc, pck);
+        }
 
         // the adjoint carried into the previous chunk (slot warps), in place; e0 for it
         {
