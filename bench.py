@@ -144,12 +144,12 @@ CAPTURED_TRAFFIC = {
                                                       profile="profiles/scan_bwd_kernel_small_train.md",
                                                       source="csrc/scan_bwd.cuh", sha="3fa6eb987d11"),
     # the chunk-parallel backward, full-size launches, dram counters alone (one pass)
-    ("chunk_bwd_kernel", "small_train"): dict(bytes=61.09e6 + 26.74e6,
+    ("chunk_bwd_kernel", "small_train"): dict(bytes=62.00e6 + 26.59e6,
                                               profile="profiles/chunk_bwd_kernel_small_train.md",
-                                              source="csrc/chunk_bwd.cuh", sha="acb133729b91"),
+                                              source="csrc/chunk_bwd.cuh", sha="3fb59cd3d40e"),
     ("chunk_bwd_kernel", "mid_layer"): dict(bytes=1.41e9 + 1.32e9,
                                             profile="profiles/chunk_bwd_kernel_small_train.md",
-                                            source="csrc/chunk_bwd.cuh", sha="acb133729b91"),
+                                            source="csrc/chunk_bwd.cuh", sha="3fb59cd3d40e"),
     # full-size launches, dram counters alone (one pass); chunk_reg.cuh changed since only
     # in its header comment (captured on 4a519db1dbb5)
     ("chunk_reg_kernel<16 slots>", "long_ctx"): dict(bytes=676.59e6 + 501.80e6,
