@@ -212,6 +212,26 @@ def test_bwd_mid_layer_full_size_sampled(L):
         assert np.isfinite(gg[k]).all()
 
 
+def test_bwd_long_context_slice_sampled(L):
+    """The long-context shape's first 8192 tokens (B=1, H=16, m=64, d=128, chunk 64,
+    mu = sigmoid(N(4, 0.5))): 128 chunks on 4-CTA clusters; two sampled heads against the
+    oracle (the whole 65536 tokens would need 4 GB of oracle states per head)."""
+    w = LI.WORKLOADS["long_ctx"]
+    inp = LI.make_inputs(w, T=8192)
+    cot = LI.make_cotangents(inp, seed=940)
+    gg = run_gpu_bwd(L, inp, cot, w.chunk)
+    pairs = [(0, 3), (0, 12)]
+    sub = LI.sample_heads(inp, pairs)
+    bs, hs = [p[0] for p in pairs], [p[1] for p in pairs]
+    sub_cot = dict(dy=np.ascontiguousarray(cot["dy"][bs, :, hs][:, :, None, :]),
+                   dS_T=np.ascontiguousarray(cot["dS_T"][bs, hs][:, None]))
+    go = run_oracle_bwd(sub, sub_cot, w.chunk)
+    gsub = {"dx": gg["dx"][bs, :, hs][:, :, None, :], "dc": gg["dc"][bs, :, hs][:, :, None, :],
+            "dq": gg["dq"][bs, :, hs][:, :, None, :], "dmu": gg["dmu"][bs, :, hs][:, :, None],
+            "deta": None, "dS0": gg["dS0"][bs, hs][:, None]}
+    check(gsub, go, 2e-2)
+
+
 def test_bwd_rejects_unsupported_shapes(L):
     w = LI.Workload("t", B=1, T=8, H=1, m=130, d=32, seed=880)
     inp = LI.make_inputs(w)
