@@ -143,13 +143,14 @@ CAPTURED_TRAFFIC = {
     ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.41e6 + 54.81e6,
                                                       profile="profiles/scan_bwd_kernel_small_train.md",
                                                       source="csrc/scan_bwd.cuh", sha="3fa6eb987d11"),
-    # the chunk-parallel backward, full-size launches, dram counters alone (one pass)
+    # the chunk-parallel backward, full-size launches, dram counters alone (one pass);
+    # chunk_bwd.cuh changed since only in its header comment (captured on 3fb59cd3d40e)
     ("chunk_bwd_kernel", "small_train"): dict(bytes=62.00e6 + 26.59e6,
                                               profile="profiles/chunk_bwd_kernel_small_train.md",
-                                              source="csrc/chunk_bwd.cuh", sha="3fb59cd3d40e"),
+                                              source="csrc/chunk_bwd.cuh", sha="d2425c5dc1fa"),
     ("chunk_bwd_kernel", "mid_layer"): dict(bytes=1.41e9 + 1.32e9,
                                             profile="profiles/chunk_bwd_kernel_small_train.md",
-                                            source="csrc/chunk_bwd.cuh", sha="3fb59cd3d40e"),
+                                            source="csrc/chunk_bwd.cuh", sha="d2425c5dc1fa"),
     # full-size launches, dram counters alone (one pass); chunk_reg.cuh changed since only
     # in its header comment (captured on 4a519db1dbb5)
     ("chunk_reg_kernel<16 slots>", "long_ctx"): dict(bytes=676.59e6 + 501.80e6,

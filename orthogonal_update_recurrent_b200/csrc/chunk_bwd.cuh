@@ -1,5 +1,6 @@
 // chunk_bwd.cuh -- backward pass of the chunked recurrence (Eq. 17) in chunk-parallel
-// form: fp32 on CUDA cores, one cluster of CTAs per sequence.
+// form, one cluster of CTAs per sequence: the matrix products on the tensor cores
+// (tf32 with a hi/lo split of each operand), the rest in fp32 on CUDA cores.
 //
 // Reverse-mode derivative of the forward of "Lattice: Learning to Efficiently
 // Compress the Memory" §3.4.1 Eq. 17 with the chunk normaliser of eq. beta_chunk
@@ -31,7 +32,8 @@
 // token-indexed sums over slots (dx, dmu, deta) cross CTAs, added through distributed
 // shared memory in rank order (bit-reproducible). A forward sweep first stores each
 // chunk's start state in the workspace; the backward sweep then walks the chunks in
-// reverse. Thread roles inside a phase:
+// reverse, loading each chunk's inputs and start state into registers while the chunk
+// after it finishes. Thread roles inside a phase:
 //   pairs      thread -> (token tid/16 and tid/16 + 32, slot tid%16)
 //   slot warps warp w -> slot w; lane -> tokens 2l, 2l+1 (scans) or D/32 state columns
 //   MMA tiles  warp w -> 16x16 / 16xD/4 / 16x8 output tiles of the matrix products, on
