@@ -718,6 +718,10 @@ def main():
             if w.m == 64 and w.chunk == 64:  # the earlier cluster kernel, for comparison
                 extra[f"{w.name}_tcgen05_split_ms"] = statistics.mean(
                     time_scan(torch, L, t, w.chunk, 5, 3, flush=flush, impl="tcgen05_split"))
+            # the backward pass on the timed workload
+            tbw = statistics.mean(time_bwd(torch, L, t, w.chunk, 3, 2, flush=flush))
+            extra[f"{w.name}_bwd"] = {"ms": tbw, "tokens_per_s": w.B * w.T / (tbw * 1e-3),
+                                      "kernel": bwd_kernel_name(w.chunk, w.d)}
             del t
             torch.cuda.empty_cache()
             # the other chunked workloads, each with its own roofline record
@@ -736,6 +740,9 @@ def main():
                 tex = time_scan(torch, L, tn, 1, 3, 3, flush=flush)
                 ent["exact_ms"] = statistics.mean(tex)
                 ent["exact_tokens_per_s"] = wn.B * wn.T / (ent["exact_ms"] * 1e-3)
+                if name == "mid_layer":   # the backward pass (small_train's is timed below)
+                    ent["bwd_ms"] = statistics.mean(time_bwd(torch, L, tn, wn.chunk, 3, 2, flush=flush))
+                    ent["bwd_kernel"] = bwd_kernel_name(wn.chunk, wn.d)
                 extra[name] = ent
                 del tn
                 torch.cuda.empty_cache()
