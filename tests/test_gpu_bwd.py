@@ -160,6 +160,18 @@ def test_bwd_chunk_parallel_edges(L, m, d, C, T):
     check(run_gpu_bwd(L, inp, cot, C), run_oracle_bwd(inp, cot, C), TOL_BWD)
 
 
+@pytest.mark.parametrize("m,d,C,T,xd,qd", [(64, 64, 64, 150, "f32", "f32"), (40, 128, 16, 90, "f32", "f32"),
+                                           (16, 32, 8, 61, "f32", "f32"), (64, 64, 32, 100, "bf16", "f32"),
+                                           (48, 128, 64, 70, "f32", "bf16")])
+def test_bwd_chunk_parallel_input_dtypes(L, m, d, C, T, xd, qd):
+    """The chunk-parallel kernel with fp32 x and/or q (16-byte vector loads of fp32 x,
+    fp32 q), eta given, a ragged last chunk."""
+    w = LI.Workload("t", B=2, T=T, H=2, m=m, d=d, x_dtype=xd, q_dtype=qd, seed=950 + m + d + C)
+    inp = with_eta(LI.make_inputs(w), 950 + C)
+    cot = LI.make_cotangents(inp, seed=950 + T)
+    check(run_gpu_bwd(L, inp, cot, C), run_oracle_bwd(inp, cot, C), TOL_BWD)
+
+
 def test_bwd_chunk_parallel_empty_sequence(L):
     w = LI.Workload("t", B=2, T=0, H=3, m=40, d=64, seed=910)
     inp = LI.make_inputs(w)
