@@ -127,12 +127,14 @@ def test_bwd_segment_length_does_not_change_the_result(L, C):
                 assert np.array_equal(ref[k], g[k]), (seg, k)
 
 
-def test_bwd_is_deterministic(L):
-    w = LI.Workload("t", B=2, T=90, H=2, m=64, d=64, seed=860)
-    inp = LI.make_inputs(w)
+@pytest.mark.parametrize("m,d,C", [(64, 64, 16), (128, 64, 32), (100, 128, 64)])
+def test_bwd_is_deterministic(L, m, d, C):
+    """Run to run bit-identity, including the sums over a cluster's CTAs (4, 8 and 7 CTAs)."""
+    w = LI.Workload("t", B=2, T=90, H=2, m=m, d=d, seed=860)
+    inp = with_eta(LI.make_inputs(w), 860)
     cot = LI.make_cotangents(inp, seed=860)
-    a = run_gpu_bwd(L, inp, cot, 16)
-    b = run_gpu_bwd(L, inp, cot, 16)
+    a = run_gpu_bwd(L, inp, cot, C)
+    b = run_gpu_bwd(L, inp, cot, C)
     for k in a:
         if a[k] is not None:
             assert np.array_equal(a[k], b[k]), k
