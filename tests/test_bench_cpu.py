@@ -88,3 +88,18 @@ def test_captured_traffic_is_dropped_once_the_kernel_changes(monkeypatch):
     monkeypatch.setitem(bench.CAPTURED_TRAFFIC, key, dict(bench.CAPTURED_TRAFFIC[key], sha="000000000000"))
     assert bench.traffic_for(*key) is None
     assert bench.traffic_for("no_such_kernel", "small_train") is None
+
+
+def test_backward_kernel_label_follows_the_dispatch_rule():
+    # the library runs the chunk-parallel backward for chunks of 2..64 at d in {32, 64, 128}
+    # (16-byte-aligned buffers), and the token-by-token kernel otherwise
+    assert bench.bwd_kernel_name(64, 64) == "chunk_bwd_kernel"
+    assert bench.bwd_kernel_name(2, 128) == "chunk_bwd_kernel"
+    assert bench.bwd_kernel_name(16, 32) == "chunk_bwd_kernel"
+    assert bench.bwd_kernel_name(1, 64) == "scan_bwd_kernel<exact>"
+    assert bench.bwd_kernel_name(128, 64) == "scan_bwd_kernel<chunked>"
+    assert bench.bwd_kernel_name(16, 16) == "scan_bwd_kernel<chunked>"
+    # and every workload's backward names a kernel with a captured-traffic entry or none
+    for w in ("small_train", "mid_layer"):
+        name = bench.bwd_kernel_name(LI.WORKLOADS[w].chunk, LI.WORKLOADS[w].d)
+        assert (name, w) in bench.CAPTURED_TRAFFIC
