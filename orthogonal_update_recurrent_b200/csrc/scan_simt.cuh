@@ -29,12 +29,15 @@ __host__ __device__ inline int scan_record_floats(int D, int m) { return (D + 2 
 
 // Shared memory: in[2][TB][record] floats, ybuf[2][TB][NW][D] floats and, for the
 // reconstruction objective, rbuf[2][NW][D] floats (per-warp partial reconstructions);
-// split kernels add ypart[2][TB][D] (the CTA's read-out partials for the cluster sum).
+// split kernels add ypart[2][TB][D] (the CTA's read-out partials for the cluster sum),
+// and with the reconstruction objective rwarp[TB][NW][D], rpart[2][TB][D] and
+// rsum[TB][D] (a block's reconstructions: per warp, per CTA, over the cluster).
 template <int D>
 __host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec, bool split = false) {
     const size_t tb = split ? kScanTBSplit : kScanTB;
     return sizeof(float) * (2ull * tb * scan_record_floats(D, m) + 2ull * tb * nw * D +
-                            (dec ? 2ull * nw * D : 0ull) + (split ? 2ull * tb * D : 0ull));
+                            (dec ? 2ull * nw * D : 0ull) + (split ? 2ull * tb * D : 0ull) +
+                            (split && dec ? tb * nw * D + 3ull * tb * D : 0ull));
 }
 
 // Cluster barrier and a load from a peer CTA's shared memory (split kernels).
@@ -57,14 +60,19 @@ __device__ __forceinline__ float scan_ld_peer(const float* local_ptr, uint32_t r
 // LIN1 (chunked only) selects the chunk linearisation of eq. recurrence_linear1
 // (§3.4.1): the projection part of each token's update scales the chunk-start slot
 // instead of the running one.
-// SPLIT (similarity objective only): each sequence runs on a cluster of a.G CTAs of
-// 8 warps; CTA g owns slots [g*spc, (g+1)*spc), spc <= 32. The slots evolve
+// SPLIT: each sequence runs on a cluster of a.G CTAs of 8 warps; CTA g owns slots
+// [g*spc, (g+1)*spc), spc <= 32. Under the similarity objective the slots evolve
 // independently, so the CTAs share only the read-out: each block's per-CTA partial
 // y is added over the cluster through distributed shared memory, ranks in a fixed
-// order (one cluster barrier per block of tokens).
+// order (one cluster barrier per block of tokens). With the reconstruction objective
+// (chunked only, chunks made of whole blocks) the residual of every token uses the
+// chunk-start state, so each block's reconstructions sum_i (c_i/|s0_i|) s0_i are formed
+// before its tokens: per CTA over its slots, then over the cluster the same way (a
+// second cluster barrier per block).
 template <int D, int RQ, bool CHUNKED, bool DEC, bool LIN1 = false, bool SPLIT = false>
 __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a) {
-    static_assert(!(SPLIT && (DEC || RQ != 1)), "split kernels: similarity objective, one slot per octet");
+    static_assert(!(SPLIT && ((DEC && !CHUNKED) || RQ != 1)),
+                  "split kernels: one slot per octet; the reconstruction objective chunked only");
     constexpr int TB = SPLIT ? kScanTBSplit : kScanTB;  // tokens per staged block
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
@@ -82,6 +90,9 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
     float* ybuf = smem + 2 * TB * per_tok;
     float* rbuf = ybuf + 2 * TB * NW * D;  // DEC only
     float* ypart = rbuf + (DEC ? 2 * NW * D : 0);  // SPLIT only: [2][TB][D]
+    float* rwarp = ypart + (SPLIT ? 2 * TB * D : 0);  // SPLIT and DEC: [TB][NW][D]
+    float* rpart = rwarp + TB * NW * D;               // [2][TB][D], read by the cluster
+    float* rsum = rpart + 2 * TB * D;                 // [TB][D]
 
     // ---- load the initial state into registers
     float s[RQ][EPL];
@@ -194,6 +205,47 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
         const float* inb = in_buf + buf * stage_total;
         float* yb = ybuf + (size_t)buf * TB * NW * D;
         const int ntok = min(TB, T - t0);
+        if constexpr (SPLIT && DEC) {
+            // chunk-start snapshot (chunks start on block boundaries), then the block's
+            // reconstructions: per warp, per CTA, and over the cluster in rank order
+            if (t0 % a.chunk == 0) {
+                float n2 = 0.f;
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) { s0[0][k] = s[0][k]; n2 = fmaf(s[0][k], s[0][k], n2); }
+                n0sq[0] = octet_sum(n2);
+                n0[0] = __fsqrt_rn(n0sq[0]);
+            }
+            for (int tok = 0; tok < ntok; ++tok) {
+                const float* rec = inb + tok * per_tok;
+                const float cv = slot[0] < m ? rec[D + m + slot[0]] : 0.f;
+                float f[1], rp[EPL];
+                f[0] = n0sq[0] > 0.f ? __fdiv_rn(cv, __fsqrt_rn(n0sq[0])) : 0.f;
+                recon_warp_partial<D, 1>(s0, f, rp);
+                if (oct == 0) {
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) rwarp[((size_t)tok * NW + warp) * D + O::pos(j, k)] = rp[k];
+                }
+            }
+            __syncthreads();
+            float* part = rpart + (size_t)(blk & 1) * TB * D;  // the next cluster barrier orders its reuse
+            for (int idx = tid; idx < ntok * D; idx += NT) {
+                const int tok = idx / D, k = idx - tok * D;
+                float acc = 0.f;
+                for (int w = 0; w < NW; ++w) acc += rwarp[((size_t)tok * NW + w) * D + k];
+                part[idx] = acc;
+            }
+            scan_cluster_sync();
+            for (int idx = tid; idx < ntok * D; idx += NT) {
+                float v[8];  // every peer's load in flight before the fixed-order sum
+#pragma unroll
+                for (int r = 0; r < 8; ++r) v[r] = r < G ? scan_ld_peer(part + idx, (uint32_t)r) : 0.f;
+                float acc = 0.f;
+#pragma unroll
+                for (int r = 0; r < 8; ++r) if (r < G) acc += v[r];
+                rsum[idx] = acc;
+            }
+            __syncthreads();
+        }
         for (int tok = 0; tok < ntok; ++tok) {
             const int t = t0 + tok;
             const float* rec = inb + tok * per_tok;
@@ -201,7 +253,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
             load_row_f32<D>(rec, j, xv);
             const float mu = rec[D + 2 * m], eta = rec[D + 2 * m + 1];
 
-            if constexpr (CHUNKED) {
+            if constexpr (CHUNKED && !(SPLIT && DEC)) {
                 if (t % a.chunk == 0) {  // chunk start: snapshot the state and its norms
 #pragma unroll
                     for (int r = 0; r < RQ; ++r) {
@@ -213,7 +265,10 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
                     }
                 }
             }
-            if constexpr (DEC) {  // x <- x - sum_i (c_i/|s_i|) s_i over every slot of the CTA
+            if constexpr (SPLIT && DEC) {  // the block's reconstructions, formed above
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) xv[k] -= rsum[(size_t)tok * D + O::pos(j, k)];
+            } else if constexpr (DEC) {  // x <- x - sum_i (c_i/|s_i|) s_i over every slot of the CTA
                 float f[RQ], rp[EPL];
 #pragma unroll
                 for (int r = 0; r < RQ; ++r) {

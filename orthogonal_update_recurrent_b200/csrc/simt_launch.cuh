@@ -39,11 +39,11 @@ lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
     return launch_status();
 }
 
-// one cluster of a.G CTAs (8 warps each) per sequence; similarity objective
-template <int D, bool CH, bool LIN1>
+// one cluster of a.G CTAs (8 warps each) per sequence
+template <int D, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_split(const ScanArgs& a, cudaStream_t st) {
-    const size_t smem = scan_smem_bytes<D>(a.m, 8, false, true);
-    auto k = scan_simt_kernel<D, 1, CH, false, LIN1, true>;
+    const size_t smem = scan_smem_bytes<D>(a.m, 8, DEC, true);
+    auto k = scan_simt_kernel<D, 1, CH, DEC, LIN1, true>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e);
     ScanArgs arg = a;
@@ -53,13 +53,16 @@ lattice_status launch_scan_simt_split(const ScanArgs& a, cudaStream_t st) {
 
 template <int D, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
-    if constexpr (!DEC) {  // the reconstruction objective couples every slot on every token
+    // The exact reconstruction objective couples every slot on every token, so it runs on
+    // one CTA per sequence; chunked, it splits when its chunks are whole 16-token blocks
+    // (d <= 64: the block's reconstruction buffers then fit in shared memory).
+    if constexpr (!DEC || (CH && D <= 64)) {
         const int G = cluster_split(a.B, a.H, a.m);
-        if (G > 1) {
+        if (G > 1 && (!DEC || a.chunk % kScanTBSplit == 0)) {
             ScanArgs s = a;
             s.G = G;
             s.spc = (a.m + G - 1) / G;
-            return launch_scan_simt_split<D, CH, LIN1>(s, st);
+            return launch_scan_simt_split<D, CH, DEC, LIN1>(s, st);
         }
     }
     const int quads = (a.m + 3) / 4;

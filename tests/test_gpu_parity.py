@@ -446,6 +446,19 @@ def test_dec_chunked_resynchronised(L, m, d, C):
     assert wy <= TOL_F32 and ws <= TOL_F32
 
 
+@pytest.mark.parametrize("m,d,C", [(64, 64, 16), (48, 32, 32), (64, 64, 64)])
+def test_dec_chunked_split_several_chunks_per_call(L, m, d, C):
+    """The chunked reconstruction objective on the cluster kernel (few sequences, chunks
+    of whole 16-token blocks, d <= 64): three chunks per call, so the chunk-start state
+    is taken again inside a call, with the block's reconstructions summed over the
+    cluster; resynchronised with the oracle every three chunks, eta given."""
+    w = LI.Workload("t", B=2, T=7 * C + 5, H=2, m=m, d=d, seed=470 + m + d + C, c_loc=DEC_CHUNK_C_LOC)
+    inp = LI.make_inputs(w)
+    inp["eta"] = np.random.default_rng(7).uniform(0.5, 1.5, inp["mu"].shape).astype(np.float32)
+    wy, ws = _dec_segments(L, inp, C, 3 * C)
+    assert wy <= TOL_F32 and ws <= TOL_F32
+
+
 def test_dec_with_eta_and_gate_edges(L):
     w = LI.Workload("t", B=2, T=40, H=2, m=32, d=64, seed=500)
     inp = LI.make_inputs(w)
