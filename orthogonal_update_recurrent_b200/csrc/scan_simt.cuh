@@ -64,15 +64,15 @@ __device__ __forceinline__ float scan_ld_peer(const float* local_ptr, uint32_t r
 // [g*spc, (g+1)*spc), spc <= 32. Under the similarity objective the slots evolve
 // independently, so the CTAs share only the read-out: each block's per-CTA partial
 // y is added over the cluster through distributed shared memory, ranks in a fixed
-// order (one cluster barrier per block of tokens). With the reconstruction objective
-// (chunked only, chunks made of whole blocks) the residual of every token uses the
+// order (one cluster barrier per block of tokens). With the reconstruction objective,
+// chunked (chunks made of whole blocks), the residual of every token uses the
 // chunk-start state, so each block's reconstructions sum_i (c_i/|s0_i|) s0_i are formed
 // before its tokens: per CTA over its slots, then over the cluster the same way (a
-// second cluster barrier per block).
+// second cluster barrier per block). Exact, every token's reconstruction is summed over
+// the cluster before the token's update (a cluster barrier per token).
 template <int D, int RQ, bool CHUNKED, bool DEC, bool LIN1 = false, bool SPLIT = false>
 __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a) {
-    static_assert(!(SPLIT && ((DEC && !CHUNKED) || RQ != 1)),
-                  "split kernels: one slot per octet; the reconstruction objective chunked only");
+    static_assert(!(SPLIT && RQ != 1), "split kernels: one slot per octet");
     constexpr int TB = SPLIT ? kScanTBSplit : kScanTB;  // tokens per staged block
     using O = Octet<D>;
     constexpr int EPL = O::EPL;
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
         const float* inb = in_buf + buf * stage_total;
         float* yb = ybuf + (size_t)buf * TB * NW * D;
         const int ntok = min(TB, T - t0);
-        if constexpr (SPLIT && DEC) {
+        if constexpr (SPLIT && DEC && CHUNKED) {
             // chunk-start snapshot (chunks start on block boundaries), then the block's
             // reconstructions: per warp, per CTA, and over the cluster in rank order
             if (t0 % a.chunk == 0) {
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
             load_row_f32<D>(rec, j, xv);
             const float mu = rec[D + 2 * m], eta = rec[D + 2 * m + 1];
 
-            if constexpr (CHUNKED && !(SPLIT && DEC)) {
+            if constexpr (CHUNKED && !(SPLIT && DEC)) {  // (split DEC: taken per block above)
                 if (t % a.chunk == 0) {  // chunk start: snapshot the state and its norms
 #pragma unroll
                     for (int r = 0; r < RQ; ++r) {
@@ -265,9 +265,44 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
                     }
                 }
             }
-            if constexpr (SPLIT && DEC) {  // the block's reconstructions, formed above
+            if constexpr (SPLIT && DEC && CHUNKED) {  // the block's reconstructions, formed above
 #pragma unroll
                 for (int k = 0; k < EPL; ++k) xv[k] -= rsum[(size_t)tok * D + O::pos(j, k)];
+            } else if constexpr (SPLIT && DEC) {
+                // exact: this token's reconstruction from the current slots, per warp, per
+                // CTA (part, double-buffered by token), then over the cluster in rank order
+                float nn = 0.f;
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) nn = fmaf(s[0][k], s[0][k], nn);
+                const float nsq = octet_sum(nn);
+                const float cv = slot[0] < m ? rec[D + m + slot[0]] : 0.f;
+                float f[1], rp[EPL];
+                f[0] = nsq > 0.f ? __fdiv_rn(cv, __fsqrt_rn(nsq)) : 0.f;
+                recon_warp_partial<D, 1>(s, f, rp);
+                if (oct == 0) {
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) rwarp[warp * D + O::pos(j, k)] = rp[k];
+                }
+                __syncthreads();
+                float* part = rpart + (size_t)(t & 1) * D;  // the next cluster barrier orders its reuse
+                for (int idx = tid; idx < D; idx += NT) {
+                    float acc = 0.f;
+                    for (int w = 0; w < NW; ++w) acc += rwarp[w * D + idx];
+                    part[idx] = acc;
+                }
+                scan_cluster_sync();
+                for (int idx = tid; idx < D; idx += NT) {
+                    float v[8];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) v[r] = r < G ? scan_ld_peer(part + idx, (uint32_t)r) : 0.f;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) if (r < G) acc += v[r];
+                    rsum[idx] = acc;
+                }
+                __syncthreads();
+#pragma unroll
+                for (int k = 0; k < EPL; ++k) xv[k] -= rsum[O::pos(j, k)];
             } else if constexpr (DEC) {  // x <- x - sum_i (c_i/|s_i|) s_i over every slot of the CTA
                 float f[RQ], rp[EPL];
 #pragma unroll

@@ -53,12 +53,13 @@ lattice_status launch_scan_simt_split(const ScanArgs& a, cudaStream_t st) {
 
 template <int D, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
-    // The exact reconstruction objective couples every slot on every token, so it runs on
-    // one CTA per sequence; chunked, it splits when its chunks are whole 16-token blocks
-    // (d <= 64: the block's reconstruction buffers then fit in shared memory).
-    if constexpr (!DEC || (CH && D <= 64)) {
+    // The reconstruction objective couples every slot on every token: split, its
+    // reconstructions are summed over the cluster once per token (exact) or once per
+    // 16-token block (chunked, chunks made of whole blocks); d <= 64, where the
+    // reconstruction buffers fit in shared memory.
+    if constexpr (!DEC || D <= 64) {
         const int G = cluster_split(a.B, a.H, a.m);
-        if (G > 1 && (!DEC || a.chunk % kScanTBSplit == 0)) {
+        if (G > 1 && (!DEC || !CH || a.chunk % kScanTBSplit == 0)) {
             ScanArgs s = a;
             s.G = G;
             s.spc = (a.m + G - 1) / G;
