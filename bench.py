@@ -139,7 +139,7 @@ CAPTURED_TRAFFIC = {
                                            source="csrc/chunk_tc.cuh", sha="488f569268b7"),
     ("scan_simt_kernel<exact>", "small_train"): dict(bytes=34.43e6 + 0.05e6,
                                                      profile="profiles/scan_simt_kernel_exact_small_train.md",
-                                                     source="csrc/scan_simt.cuh", sha="8754281be921"),
+                                                     source="csrc/scan_simt.cuh", sha="028bc6c080c6"),
     ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.41e6 + 54.81e6,
                                                       profile="profiles/scan_bwd_kernel_small_train.md",
                                                       source="csrc/scan_bwd.cuh", sha="3fa6eb987d11"),

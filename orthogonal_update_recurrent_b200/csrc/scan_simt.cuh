@@ -56,7 +56,8 @@ __device__ __forceinline__ float scan_ld_peer(const float* local_ptr, uint32_t r
 // DEC selects the reconstruction objective (§3.1.1 eq. decoding_recurrence): each
 // token's write direction is x - sum_i (c_i/|s_i|) s_i, with the slots of the state
 // the token's projection uses (the current state; the chunk-start state when
-// CHUNKED). It costs one cross-warp reduction and one barrier per token.
+// CHUNKED). On one CTA per sequence it costs one cross-warp reduction and one barrier
+// per token; on a cluster (SPLIT, below) the sums also cross the CTAs.
 // LIN1 (chunked only) selects the chunk linearisation of eq. recurrence_linear1
 // (§3.4.1): the projection part of each token's update scales the chunk-start slot
 // instead of the running one.
