@@ -30,14 +30,17 @@ __host__ __device__ inline int scan_record_floats(int D, int m) { return (D + 2 
 // Shared memory: in[2][TB][record] floats, ybuf[2][TB][NW][D] floats and, for the
 // reconstruction objective, rbuf[2][NW][D] floats (per-warp partial reconstructions);
 // split kernels add ypart[2][TB][D] (the CTA's read-out partials for the cluster sum),
-// and with the reconstruction objective rwarp[TB][NW][D], rpart[2][TB][D] and
-// rsum[TB][D] (a block's reconstructions: per warp, per CTA, over the cluster).
+// and with the reconstruction objective rwarp[R][NW][D], rpart[2][R][D] and rsum[R][D]
+// (reconstructions per warp, per CTA, over the cluster) for R = TB tokens when chunked
+// (a block at a time) and R = 1 when exact (a token at a time).
 template <int D>
-__host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec, bool split = false) {
+__host__ __device__ inline size_t scan_smem_bytes(int m, int nw, bool dec, bool split = false,
+                                                  bool chunked = true) {
     const size_t tb = split ? kScanTBSplit : kScanTB;
+    const size_t rr = chunked ? tb : 1;
     return sizeof(float) * (2ull * tb * scan_record_floats(D, m) + 2ull * tb * nw * D +
                             (dec ? 2ull * nw * D : 0ull) + (split ? 2ull * tb * D : 0ull) +
-                            (split && dec ? tb * nw * D + 3ull * tb * D : 0ull));
+                            (split && dec ? rr * nw * D + 3ull * rr * D : 0ull));
 }
 
 // Cluster barrier and a load from a peer CTA's shared memory (split kernels).
@@ -91,9 +94,10 @@ __global__ void __launch_bounds__(SPLIT ? 256 : 512) scan_simt_kernel(ScanArgs a
     float* ybuf = smem + 2 * TB * per_tok;
     float* rbuf = ybuf + 2 * TB * NW * D;  // DEC only
     float* ypart = rbuf + (DEC ? 2 * NW * D : 0);  // SPLIT only: [2][TB][D]
-    float* rwarp = ypart + (SPLIT ? 2 * TB * D : 0);  // SPLIT and DEC: [TB][NW][D]
-    float* rpart = rwarp + TB * NW * D;               // [2][TB][D], read by the cluster
-    float* rsum = rpart + 2 * TB * D;                 // [TB][D]
+    constexpr int RR = CHUNKED ? TB : 1;              // reconstructions formed at a time
+    float* rwarp = ypart + (SPLIT ? 2 * TB * D : 0);  // SPLIT and DEC: [RR][NW][D]
+    float* rpart = rwarp + RR * NW * D;               // [2][RR][D], read by the cluster
+    float* rsum = rpart + 2 * RR * D;                 // [RR][D]
 
     // ---- load the initial state into registers
     float s[RQ][EPL];

@@ -42,7 +42,7 @@ lattice_status launch_scan_simt_t(const ScanArgs& a, int nw, cudaStream_t st) {
 // one cluster of a.G CTAs (8 warps each) per sequence
 template <int D, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_split(const ScanArgs& a, cudaStream_t st) {
-    const size_t smem = scan_smem_bytes<D>(a.m, 8, DEC, true);
+    const size_t smem = scan_smem_bytes<D>(a.m, 8, DEC, true, CH);
     auto k = scan_simt_kernel<D, 1, CH, DEC, LIN1, true>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -55,9 +55,9 @@ template <int D, bool CH, bool DEC, bool LIN1>
 lattice_status launch_scan_simt_d(const ScanArgs& a, cudaStream_t st) {
     // The reconstruction objective couples every slot on every token: split, its
     // reconstructions are summed over the cluster once per token (exact) or once per
-    // 16-token block (chunked, chunks made of whole blocks); d <= 64, where the
-    // reconstruction buffers fit in shared memory.
-    if constexpr (!DEC || D <= 64) {
+    // 16-token block (chunked, chunks made of whole blocks, d <= 64, where a block's
+    // reconstruction buffers fit in shared memory).
+    if constexpr (!DEC || !CH || D <= 64) {
         const int G = cluster_split(a.B, a.H, a.m);
         if (G > 1 && (!DEC || !CH || a.chunk % kScanTBSplit == 0)) {
             ScanArgs s = a;
