@@ -137,9 +137,9 @@ CAPTURED_TRAFFIC = {
                                              source="csrc/chunk_split.cuh", sha="047d8e41962f"),
     ("chunk_tc_kernel", "mid_layer"): dict(bytes=550.70e6 + 237.14e6, profile="profiles/chunk_tc_kernel_full.md",
                                            source="csrc/chunk_tc.cuh", sha="488f569268b7"),
-    ("scan_simt_kernel<exact>", "small_train"): dict(bytes=34.43e6 + 0.05e6,
+    ("scan_simt_kernel<exact>", "small_train"): dict(bytes=34.43e6 + 0.00e6,
                                                      profile="profiles/scan_simt_kernel_exact_small_train.md",
-                                                     source="csrc/scan_simt.cuh", sha="028bc6c080c6"),
+                                                     source="csrc/scan_simt.cuh", sha="9b2b98fd3aeb"),
     ("scan_bwd_kernel<chunked>", "small_train"): dict(bytes=71.41e6 + 54.81e6,
                                                       profile="profiles/scan_bwd_kernel_small_train.md",
                                                       source="csrc/scan_bwd.cuh", sha="3fa6eb987d11"),
